@@ -1,0 +1,70 @@
+"""Oracle: linear fast weight with KV binding (test infrastructure only).
+
+Source: "Test-Time Training with KV Binding Is Secretly Linear Attention"
+(gist.science summary, section "B. Reformulación Teórica"; podcast transcript
+at 7:50-9:39).  A fast weight W (dv x dk) takes, for every token, one gradient
+step on the binding loss  l_t(W) = -<W k_t, v_t>  with the token's learning
+rate eta_t.  The gradient is -v_t k_t^T, independent of W, so the step is
+    W_t = W_{t-1} + eta_t v_t k_t^T,
+and the read is o_t = W q_t.  Unrolled, o_t = W_0 q_t + sum_{s<=t} eta_s
+(q_t . k_s) v_s: causal linear attention, which is the pages' central claim.
+
+Conventions (readings of the pages, all stated once here):
+  * the state handed across calls is S = W^T with shape [dk, dv];
+  * ``include_diag=True`` (default): token t reads W after its own update
+    (o_t = W_t q_t, inclusive causal mask); ``False`` reads before it.
+All arithmetic is float64.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _f64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def ttt_linear_recurrent(q, k, v, lr, S0=None, include_diag=True):
+    """Token-by-token TTT recurrence (the definition).
+
+    q, k: [B,H,N,dk]; v: [B,H,N,dv]; lr: [B,H,N]; S0: [B,H,dk,dv] or None.
+    Returns (out [B,H,N,dv] float64, S_end [B,H,dk,dv] float64).
+    """
+    q, k, v, lr = _f64(q), _f64(k), _f64(v), _f64(lr)
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    # W = S^T  (dv x dk) per (b, h)
+    W = np.zeros((B, H, dv, dk)) if S0 is None else np.swapaxes(_f64(S0), -1, -2).copy()
+    out = np.empty((B, H, N, dv))
+    for t in range(N):
+        # gradient of -<W k_t, v_t> w.r.t. W is -v_t k_t^T; one GD step of size eta_t
+        step = lr[:, :, t, None, None] * (v[:, :, t, :, None] * k[:, :, t, None, :])
+        if include_diag:
+            W += step
+            out[:, :, t] = np.einsum("bhij,bhj->bhi", W, q[:, :, t])
+        else:
+            out[:, :, t] = np.einsum("bhij,bhj->bhi", W, q[:, :, t])
+            W += step
+    return out, np.swapaxes(W, -1, -2).copy()
+
+
+def ttt_linear_attention_sum(q, k, v, lr, S0=None, include_diag=True, t_index=None):
+    """The same outputs written as the causal linear-attention sum
+        o_t = S0^T q_t + sum_{s <= t (or s < t)} eta_s (q_t . k_s) v_s
+    evaluated directly for the token positions in ``t_index`` (all if None).
+    Cost O(|t_index| * N * d); used for sampled checks at full sizes.
+    Returns [B,H,len(t_index),dv] float64.
+    """
+    q, k, v, lr = _f64(q), _f64(k), _f64(v), _f64(lr)
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    idx = np.arange(N) if t_index is None else np.asarray(t_index)
+    out = np.zeros((B, H, len(idx), dv))
+    for j, t in enumerate(idx):
+        last = t + 1 if include_diag else t
+        if last > 0:
+            scores = np.einsum("bhd,bhsd->bhs", q[:, :, t], k[:, :, :last]) * lr[:, :, :last]
+            out[:, :, j] = np.einsum("bhs,bhsd->bhd", scores, v[:, :, :last])
+        if S0 is not None:
+            out[:, :, j] += np.einsum("bhij,bhi->bhj", _f64(S0), q[:, :, t])
+    return out
