@@ -1,0 +1,212 @@
+/*
+ * ttt.h -- C ABI of the B200 (sm_100a) TTT-KV fast-weight layer library
+ *          (libttt_b200.so).
+ *
+ * The layer: fast weights trained at test time by one gradient step per token
+ * (linear case) or per chunk (LaCT case) on the key->value binding loss
+ * l_t(W) = -<f_W(k_t), v_t>, read by the queries.
+ *
+ *   * "Test-Time Training with KV Binding Is Secretly Linear Attention"
+ *     (summary page, "B. Reformulación Teórica"): with a linear fast weight
+ *     the recurrence W_t = W_{t-1} + eta_t v_t k_t^T, o_t = W_t q_t is causal
+ *     linear attention and admits a chunked / prefix-scan form
+ *     ("Formulación Paralela").
+ *   * "Test-Time Training Done Right" (LaCT review): a SwiGLU memory with
+ *     three matrices, chunk gradients summed with per-token learning rates,
+ *     GD / momentum / Muon (Newton-Schulz) updates followed by L2
+ *     normalisation ("Memoria no lineal y atención local"); causal chunks read
+ *     the memory of earlier chunks before updating it, posed-image sets are
+ *     written first and queried afterwards ("El orden de lectura evita
+ *     información futura").
+ *
+ * General conventions for every entry point
+ *   * Every tensor pointer is a DEVICE pointer owned by the caller.  The
+ *     library never allocates device memory and keeps no global state apart
+ *     from a per-process cache of kernel attributes.
+ *   * Token tensors are [B, H, T, D], contiguous, D innermost.  Learning
+ *     rates are float32 [B, H, T].  Pointers must be 16-byte aligned and
+ *     D * sizeof(element) a multiple of 16 bytes (TMA rule).
+ *   * Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream) and runs asynchronously.  Arguments are
+ *     validated on the host before anything is enqueued; a negative
+ *     ttt_status is returned and nothing runs when validation fails.
+ *   * Kernels never trap.  Every wait inside a kernel is bounded; when a
+ *     bound is exceeded the kernel writes a code into the status word at the
+ *     start of the workspace and returns.  ttt_check_device_status() reads it.
+ *   * Functions are thread-safe for distinct buffers.
+ */
+#ifndef TTT_B200_H
+#define TTT_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_ARG = -1,          /* null pointer / bad enum / non-positive size     */
+  TTT_ERR_SHAPE = -2,        /* inconsistent or out-of-range shapes            */
+  TTT_ERR_ALIGN = -3,        /* pointer or row pitch not 16-byte aligned        */
+  TTT_ERR_DTYPE = -4,        /* unsupported dtype combination                  */
+  TTT_ERR_UNSUPPORTED = -5,  /* head dims outside the compiled tile set        */
+  TTT_ERR_WORKSPACE = -6,    /* workspace too small                            */
+  TTT_ERR_CUDA = -7,         /* a CUDA runtime/driver call failed               */
+  TTT_ERR_TIMEOUT = -8       /* a bounded in-kernel wait ran out               */
+} ttt_status;
+
+typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
+typedef enum { TTT_CAUSAL = 0, TTT_BIDIRECTIONAL = 1 } ttt_order;
+typedef enum { TTT_OPT_GD = 0, TTT_OPT_MOMENTUM = 1, TTT_OPT_MUON = 2 } ttt_opt;
+
+/* Bytes of the device status word block at the start of every workspace. */
+#define TTT_STATUS_BYTES 256
+
+/* ------------------------------------------------------------------------
+ * Case (a): linear fast weight == causal linear attention.
+ * "Test-Time Training with KV Binding Is Secretly Linear Attention",
+ * summary "B. Reformulación Teórica" and "Formulación Paralela".
+ *
+ *   state S = W^T, float32 [B, H, dk, dv]
+ *   for t in 0..N-1:  S += lr_t k_t v_t^T ;  out_t = S^T q_t
+ *   (include_diag = 0: out_t is read before token t's own update)
+ *
+ * `chunk` is the blocking of the chunked form.  Because the gradient of the
+ * binding loss does not depend on W, the result is the same for every chunk
+ * size up to rounding; the tensor-core kernel processes 128-token tiles.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int B, H, N;          /* batch, heads, tokens (N >= 0)                     */
+  int dk, dv;           /* key/query dim, value dim                          */
+  int chunk;            /* > 0                                               */
+  int include_diag;     /* 1: token reads after its own update (default)    */
+  ttt_dtype in_dtype;   /* q, k, v element type (TTT_F32 or TTT_BF16)        */
+  ttt_dtype out_dtype;  /* out element type                                  */
+} ttt_linear_desc;
+
+/* Workspace bytes needed by ttt_linear_fwd (status word only). */
+int ttt_linear_workspace_bytes(const ttt_linear_desc* desc, size_t* bytes);
+
+/* S <- S0 (device float32 [B,H,dk,dv]); S0 == NULL zero-fills S. */
+int ttt_linear_state_init(const ttt_linear_desc* desc, const float* S0, float* S, void* stream);
+
+/* dst <- S; dst may be a device pointer or pinned/registered host memory. */
+int ttt_linear_state_readout(const ttt_linear_desc* desc, const float* S, float* dst, void* stream);
+
+/* One call over N tokens.  q, k: [B,H,N,dk]; v: [B,H,N,dv]; lr: [B,H,N];
+ * S: in = state before the first token, out = state after the last token;
+ * out: [B,H,N,dv].  Supported: in_dtype F32 (any dk, dv <= 128) and BF16
+ * (dk = dv = 64 on tensor cores; other dims <= 128 on CUDA cores). */
+int ttt_linear_fwd(const ttt_linear_desc* desc, const void* q, const void* k, const void* v,
+                   const float* lr, float* S, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Case (b): LaCT, SwiGLU fast-weight memory with large chunks.
+ * "Test-Time Training Done Right" review, "Memoria no lineal y atención
+ * local" and "El orden de lectura evita información futura".
+ *
+ * Per (b,h): W1, W3 in R^{dh x d}, W2 in R^{d x dh};
+ *   f_W(x) = W2 (silu(W1 x) * (W3 x)),  l_t = -<f_W(k_t), v_t>.
+ * For each chunk of `chunk` input tokens (the last may be shorter):
+ *   causal:        out = f_W(q) for the chunk's tokens with the weights left
+ *                  by earlier chunks, then update;
+ *   bidirectional: update only; after the last chunk the N_q queries read.
+ * Update: G = sum_t lr_t grad_W l_t (all at the chunk-start W), then
+ *   GD:       W -= G
+ *   MOMENTUM: M = beta M + G;  W -= M
+ *   MUON:     M = beta M + G;  W -= NS(M)  (ns_steps quintic Newton-Schulz
+ *             steps with ns_coef on M/(||M||_F + ns_eps), wide orientation)
+ * then, if normalize_rows, every row of each updated matrix is rescaled to
+ * unit L2 norm: W[i,:] /= max(||W[i,:]||, norm_eps).
+ * update_mask selects the updated matrices: bit0 W1, bit1 W3, bit2 W2.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int B, H;
+  int N_in;             /* input (key/value) tokens                          */
+  int N_q;              /* query tokens; must equal N_in when causal         */
+  int d, dh;            /* head dim (multiple of 64), hidden dim (mult. 64)  */
+  int chunk;            /* > 0                                               */
+  ttt_order order;
+  ttt_opt opt;
+  float beta;           /* momentum (MOMENTUM, MUON)                         */
+  int ns_steps;         /* Newton-Schulz steps (MUON), >= 0                  */
+  float ns_coef[3];     /* (a, b, c) of a*X + (b*A + c*A^2) X                */
+  float ns_eps;
+  int normalize_rows;
+  float norm_eps;
+  int update_mask;      /* 1..7                                              */
+  ttt_dtype in_dtype;   /* q, k, v: TTT_BF16                                 */
+  ttt_dtype out_dtype;  /* out: TTT_F32 or TTT_BF16                          */
+} lact_desc;
+
+/* Bytes of the state: W1, W3, W2 float32 per (b,h) (+ M1, M3, M2 for
+ * MOMENTUM and MUON).  Layout: [W1 | W3 | W2 | M1 | M3 | M2], each block
+ * [B*H, rows, cols] row-major. */
+int lact_state_bytes(const lact_desc* desc, size_t* bytes);
+
+/* Workspace bytes for lact_chunk_fwd (status word, bf16 operand copies of
+ * the weights, per-chunk intermediates, split-K partial sums, NS buffers). */
+int lact_workspace_bytes(const lact_desc* desc, size_t* bytes);
+
+/* Initialise the state from float32 device weights.  w_per_batch = 0: W1,
+ * W3 are [H,dh,d] and W2 [H,d,dh], shared by every batch entry; 1: they are
+ * [B,H,...].  Momentum buffers are zeroed. */
+int lact_state_init(const lact_desc* desc, const float* W1, const float* W3, const float* W2,
+                    int w_per_batch, void* state, void* stream);
+
+/* Copy the state out: W1, W3 [B,H,dh,d], W2 [B,H,d,dh]; M (nullable) gets
+ * [M1 | M3 | M2] when the optimizer keeps momentum.  Destinations may be
+ * device pointers or pinned host memory. */
+int lact_state_readout(const lact_desc* desc, const void* state, float* W1, float* W3, float* W2,
+                       float* M, void* stream);
+
+/* One call of the layer.  q: causal [B,H,N_in,d], bidirectional [B,H,N_q,d];
+ * k, v: [B,H,N_in,d]; lr: [B,H,N_in]; state in/out; out: [B,H,N_in,d]
+ * (causal) or [B,H,N_q,d] (bidirectional).  A causal call may be followed by
+ * another call on the continuation of the sequence with the same state;
+ * chunk boundaries restart at every call. */
+int lact_chunk_fwd(const lact_desc* desc, const void* q, const void* k, const void* v,
+                   const float* lr, void* state, void* out, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/* ------------------------------------------------------------------------
+ * Status and diagnostics
+ * ---------------------------------------------------------------------- */
+
+/* Synchronises `stream`, then reads and clears the status word of `ws`.
+ * Returns TTT_OK, TTT_ERR_TIMEOUT (a bounded wait ran out) or TTT_ERR_CUDA. */
+int ttt_check_device_status(void* ws, void* stream);
+
+/* Launch a one-CTA kernel that waits, with a bound of `timeout_us`
+ * microseconds, on an mbarrier that nothing ever completes; it must record
+ * TTT_ERR_TIMEOUT in the status word of `ws` and return.  Exercises the
+ * failure path of every bounded wait without faulting the GPU. */
+int ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, int timeout_us, void* stream);
+
+/* Optional per-kernel timing.  Between ttt_profile_begin() and
+ * ttt_profile_end() every kernel launch of this library is bracketed by two
+ * CUDA events recorded on its launch stream.  ttt_profile_end() waits for
+ * them and returns, per kernel kind, the number of launches and the summed
+ * event time; `entries` (nullable) receives up to `max_entries` of them and
+ * `*n_entries` the number of kinds seen.  Process-wide; not for concurrent
+ * use from several threads. */
+typedef struct {
+  char name[32];
+  int launches;
+  double total_ms;
+} ttt_prof_entry;
+int ttt_profile_begin(void);
+int ttt_profile_end(ttt_prof_entry* entries, int max_entries, int* n_entries);
+
+/* Human-readable name of a ttt_status value. */
+const char* ttt_status_string(int status);
+
+/* Library build string (compiler, arch). */
+const char* ttt_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_B200_H */

@@ -1,0 +1,75 @@
+// kernels.h -- internal interface between the C ABI (api.cu) and the kernel
+// launchers.  Not part of the public ABI.
+#pragma once
+
+#include <stdio.h>
+
+#include "common.cuh"
+
+namespace ttt {
+
+// ----------------------------------------------------------------- tensor maps
+// 3-D bf16 tensor map {inner, rows, batch} with 128-byte swizzle; strides in
+// bytes; box {box_inner, box_rows, 1}.  Out-of-range elements read as zero.
+// Returns 0 on success.
+int make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                      uint64_t batch, uint64_t row_stride, uint64_t batch_stride,
+                      uint32_t box_inner, uint32_t box_rows);
+
+// ----------------------------------------------------------------- TTT-linear
+struct LinearLaunch {
+  int B, H, N, dk, dv, chunk, include_diag;
+  int in_bf16, out_bf16;
+  const void *q, *k, *v;
+  const float* lr;
+  float* S;
+  void* out;
+  DevStatus st;
+};
+int launch_ttt_linear_simt(const LinearLaunch& L, cudaStream_t stream);
+int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream);
+size_t ttt_linear_simt_smem(int dk, int dv);
+
+// ----------------------------------------------------------------- LaCT
+struct LactLaunch {
+  int B, H, N_in, N_q, d, dh, chunk;
+  int causal;
+  int opt;                 // 0 GD, 1 momentum, 2 Muon
+  float beta;
+  int ns_steps;
+  float ns_a, ns_b, ns_c, ns_eps;
+  int normalize_rows;
+  float norm_eps;
+  int update_mask;
+  int out_bf16;
+  const void *q, *k, *v;
+  const float* lr;
+  float* state;            // [W1 | W3 | W2 | M1 | M3 | M2] fp32
+  void* out;
+  uint8_t* ws;             // workspace (status block first)
+  size_t ws_bytes;
+  DevStatus st;
+};
+// Workspace layout (byte offsets) for a given problem.
+struct LactWorkspace {
+  size_t status, w1b, w3b, w2b, dh1, dh3, gm, aq, part, rowss, nsx32, nsxb, nsa32, nsab, nsbb,
+      total;
+  int cmax;                // rows of the per-chunk intermediates
+  int splits;              // split-K factor of the gradient GEMMs
+};
+LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
+                                    int causal, int opt);
+int launch_lact(const LactLaunch& L, cudaStream_t stream);
+
+// ----------------------------------------------------------------- profiling
+enum KernelKind {
+  K_LIN_SIMT, K_LIN_UMMA, K_LACT_CAST, K_KEYPASS, K_GEMM_READ, K_GEMM_GRAD, K_UPDATE,
+  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_NUM
+};
+void prof_before(int kind, cudaStream_t s);
+void prof_after(int kind, cudaStream_t s);
+
+// ----------------------------------------------------------------- self test
+int launch_wait_timeout_probe(DevStatus st, cudaStream_t stream);
+
+}  // namespace ttt

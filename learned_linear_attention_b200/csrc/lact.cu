@@ -1,0 +1,766 @@
+// lact.cu -- LaCT fast-weight layer: SwiGLU memory with large chunks
+// ("Test-Time Training Done Right" review: "Memoria no lineal y atención
+// local", "El orden de lectura evita información futura").
+//
+// Per chunk c of C input tokens (all heads at once, every step on the GPU):
+//   1. key pass   (tcgen05):  [H1|H3] = K_c [W1;W3]^T, dGr = V_c W2 and, for
+//      the causal order, [Hq1|Hq3] = Q_c [W1;W3]^T.  The epilogue forms
+//        dH3 = dG*silu(H1), dH1 = dG*H3*silu'(H1), Gm' = -eta*silu(H1)*H3
+//      with dG = -eta*dGr (token rows), and Aq = silu(Hq1)*Hq3; all bf16.
+//   2. read       (tcgen05):  out_c = Aq W2^T             (causal order)
+//   3. gradients  (tcgen05, split-K over tokens):
+//        G1 = dH1^T K_c,  G3 = dH3^T K_c,  G2 = V_c^T Gm'
+//   4. update: GD / momentum in one row kernel with the row L2
+//      normalisation; Muon: momentum, Newton-Schulz on tensor cores, apply +
+//      normalisation.  Each writes the fp32 state and the bf16 operand copy
+//      used by the next chunk.
+// Bidirectional order: steps 1 (keys only), 3, 4 for every chunk, then the
+// queries run step 1 (queries only) and step 2 with the final weights.
+#include <algorithm>
+
+#include "gemm.cuh"
+#include "kernels.h"
+
+namespace ttt {
+
+// =====================================================================
+// key pass
+// =====================================================================
+namespace kp {
+constexpr int BM = 128, HB = 64;          // token rows, hidden units per tile
+constexpr uint32_t X_BYTES = BM * 64 * 2;            // 16 KB (K or Q tile)
+constexpr uint32_t V_BYTES = BM * 64 * 2;            // 16 KB
+constexpr uint32_t W13_BYTES = 2 * HB * 64 * 2;      // 16 KB (W1 rows | W3 rows)
+constexpr uint32_t W2_BYTES = 64 * HB * 2;           // 8 KB  (W2 block, MN-major)
+constexpr uint32_t STAGE = X_BYTES + V_BYTES + W13_BYTES + W2_BYTES;
+constexpr int STAGES = 3;
+constexpr uint32_t BAR_OFF = STAGES * STAGE;
+constexpr uint32_t SMEM = BAR_OFF + 256 + 1024;
+constexpr uint32_t ACC_COLS = 256;                   // [H1 64 | H3 64 | dG 64 | pad]
+}  // namespace kp
+
+struct KeyPassArgs {
+  int C;            // rows of this pass (chunk length or N_q)
+  int t0;           // first token row in the token tensors
+  int n_key_tiles, n_q_tiles;
+  int n_hb;         // dh / 64
+  int BH;
+  int d_steps;      // d / 64
+  int dh;
+  int lr_len;       // row length of lr ([BH][lr_len])
+  const float* lr;
+  __nv_bfloat16 *dH1, *dH3, *Gm, *Aq;   // [BH][cmax][dh]
+  long long inter_bs;
+  DevStatus st;
+};
+
+struct KeyPassMaps {
+  CUtensorMap k, v, q, w1, w3, w2;
+};
+
+TTT_DEVICE_INLINE float sigmoidf_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+
+__global__ void __launch_bounds__(192, 1)
+    lact_keypass_kernel(const __grid_constant__ KeyPassMaps maps, const KeyPassArgs a) {
+  using namespace kp;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint64_t* empty = full + STAGES;
+  uint64_t* afull = empty + STAGES;
+  uint64_t* aempty = afull + 2;
+  uint64_t* fin = aempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_per_bh = (a.n_key_tiles + a.n_q_tiles) * a.n_hb;
+  const int n_tiles = tiles_per_bh * a.BH;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&afull[s], 1);
+      mbar_init(&aempty[s], 128);
+    }
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * ACC_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.k);
+    tma_prefetch_desc(&maps.v);
+    tma_prefetch_desc(&maps.q);
+    tma_prefetch_desc(&maps.w1);
+    tma_prefetch_desc(&maps.w3);
+    tma_prefetch_desc(&maps.w2);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  Waiter W{abort_flag, a.st, 200};
+
+  // tile id -> (bh, token tile, hidden block); hidden block fastest so the
+  // CTAs sharing a token tile run together and its K/V rows hit in L2.
+  auto decode = [&](int t, int& bh, int& tt, int& hb) {
+    hb = t % a.n_hb;
+    tt = (t / a.n_hb) % (a.n_key_tiles + a.n_q_tiles);
+    bh = t / tiles_per_bh;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        int bh, tt, hb;
+        decode(t, bh, tt, hb);
+        const bool is_key = tt < a.n_key_tiles;
+        const int row = a.t0 + (is_key ? tt : tt - a.n_key_tiles) * BM;
+        const int j0 = hb * HB;
+        for (int ks = 0; ks < a.d_steps; ++ks, ++it) {
+          const uint32_t s = it % STAGES;
+          if (it >= (uint32_t)STAGES && !W.wait(&empty[s], ((it / STAGES) - 1) & 1, 1)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * STAGE;
+          mbar_arrive_expect_tx(&full[s], is_key ? STAGE : X_BYTES + W13_BYTES);
+          tma_load_3d(st, is_key ? &maps.k : &maps.q, &full[s], ks * 64, row, bh);
+          tma_load_3d(st + X_BYTES + V_BYTES, &maps.w1, &full[s], ks * 64, j0, bh);
+          tma_load_3d(st + X_BYTES + V_BYTES + W13_BYTES / 2, &maps.w3, &full[s], ks * 64, j0, bh);
+          if (is_key) {
+            tma_load_3d(st + X_BYTES, &maps.v, &full[s], ks * 64, row, bh);
+            tma_load_3d(st + X_BYTES + V_BYTES + W13_BYTES, &maps.w2, &full[s], j0, ks * 64, bh);
+          }
+        }
+      }
+      if (W.aborted()) {
+        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+        for (uint32_t i = first; i < it; ++i) W.drain(&full[i % STAGES], (i / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_h = make_idesc(128, 128, false, false);
+      const uint32_t id_g = make_idesc(128, 64, false, true);
+      uint32_t it = 0, lt = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++lt) {
+        int bh, tt, hb;
+        decode(t, bh, tt, hb);
+        const bool is_key = tt < a.n_key_tiles;
+        const uint32_t ab = lt & 1;
+        if (lt >= 2 && !W.wait(&aempty[ab], ((lt >> 1) - 1) & 1, 2)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + ab * ACC_COLS;
+        for (int ks = 0; ks < a.d_steps; ++ks, ++it) {
+          const uint32_t s = it % STAGES;
+          if (!W.wait(&full[s], (it / STAGES) & 1, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sx = smem_u32(smem + s * STAGE);
+          const uint32_t sv = sx + X_BYTES;
+          const uint32_t sw13 = sv + V_BYTES;
+          const uint32_t sw2 = sw13 + W13_BYTES;
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            mma_bf16(d, make_sdesc(sx + k4 * 32, 16, 1024), make_sdesc(sw13 + k4 * 32, 16, 1024),
+                     id_h, (ks | k4) != 0);
+            if (is_key)
+              mma_bf16(d + 128, make_sdesc(sv + k4 * 32, 16, 1024),
+                       make_sdesc(sw2 + k4 * 2048, 8192, 1024), id_g, (ks | k4) != 0);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&afull[ab]);
+      }
+      mma_commit(fin);
+      W.drain(fin, 0);
+    }
+  } else {
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    uint32_t lt = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
+      int bh, tt, hb;
+      decode(t, bh, tt, hb);
+      const bool is_key = tt < a.n_key_tiles;
+      const int tc = (is_key ? tt : tt - a.n_key_tiles) * BM + r;   // row within the pass
+      const bool valid = tc < a.C;
+      const uint32_t ab = lt & 1;
+      if (!W.wait(&afull[ab], (lt >> 1) & 1, 4)) break;
+      tc_fence_after();
+      const uint32_t base = tmem + lane_base + ab * ACC_COLS;
+      const size_t obase = (size_t)bh * a.inter_bs + (size_t)tc * a.dh + hb * HB;
+      const float eta = (is_key && valid) ? a.lr[(size_t)bh * a.lr_len + a.t0 + tc] : 0.f;
+#pragma unroll 1
+      for (int jc = 0; jc < HB; jc += 32) {
+        float h1[32], h3[32];
+        tmem_ld32(base + jc, h1);
+        tmem_ld32(base + 64 + jc, h3);
+        if (is_key) {
+          float g[32];
+          tmem_ld32(base + 128 + jc, g);
+          if (valid) {
+            uint32_t o1[16], o3[16], om[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float r1[2], r3[2], rm[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const float x = h1[j + u], y = h3[j + u];
+                const float sg = sigmoidf_fast(x);
+                const float act = x * sg;
+                const float dg = -eta * g[j + u];
+                r3[u] = dg * act;
+                r1[u] = dg * y * (sg * (1.f + x * (1.f - sg)));
+                rm[u] = -eta * act * y;
+              }
+              o1[j >> 1] = pack_bf16x2(r1[0], r1[1]);
+              o3[j >> 1] = pack_bf16x2(r3[0], r3[1]);
+              om[j >> 1] = pack_bf16x2(rm[0], rm[1]);
+            }
+            uint4* d1 = reinterpret_cast<uint4*>(a.dH1 + obase + jc);
+            uint4* d3 = reinterpret_cast<uint4*>(a.dH3 + obase + jc);
+            uint4* dm = reinterpret_cast<uint4*>(a.Gm + obase + jc);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              d1[j] = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
+              d3[j] = make_uint4(o3[4 * j], o3[4 * j + 1], o3[4 * j + 2], o3[4 * j + 3]);
+              dm[j] = make_uint4(om[4 * j], om[4 * j + 1], om[4 * j + 2], om[4 * j + 3]);
+            }
+          }
+        } else if (valid) {
+          uint32_t oq[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float a0 = h1[j] * sigmoidf_fast(h1[j]) * h3[j];
+            const float a1 = h1[j + 1] * sigmoidf_fast(h1[j + 1]) * h3[j + 1];
+            oq[j >> 1] = pack_bf16x2(a0, a1);
+          }
+          uint4* dq = reinterpret_cast<uint4*>(a.Aq + obase + jc);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dq[j] = make_uint4(oq[4 * j], oq[4 * j + 1], oq[4 * j + 2], oq[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&aempty[ab]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * ACC_COLS);
+  }
+}
+
+// =====================================================================
+// row kernels: bf16 copies, GD / momentum update, Muon pieces
+// =====================================================================
+struct RowArgs {
+  int BH, d, dh, splits, opt, normalize, mask;
+  float beta, norm_eps, ns_eps;
+  float* W[3];              // fp32 state per matrix [BH][rows][cols]
+  float* M[3];              // momentum (nullable)
+  __nv_bfloat16* Wb[3];     // bf16 copies
+  const float* part[3];     // split-K partial gradients [splits][BH][rows][cols]
+  float* rowss;             // [3][BH][rows] row sums of squares (Muon)
+  const float* X32;         // NS result [3][BH][r][c] (Muon apply)
+};
+
+constexpr int ROW_MAXV = 32;  // columns per lane (cols <= 1024)
+
+TTT_DEVICE_INLINE void row_decode(const RowArgs& a, int gw, int& mat, int& bh, int& row, int& rows,
+                                  int& cols) {
+  const int per_bh = 2 * a.dh + a.d;
+  bh = gw / per_bh;
+  int rr = gw % per_bh;
+  if (rr < a.dh) {
+    mat = 0; row = rr; rows = a.dh; cols = a.d;
+  } else if (rr < 2 * a.dh) {
+    mat = 1; row = rr - a.dh; rows = a.dh; cols = a.d;
+  } else {
+    mat = 2; row = rr - 2 * a.dh; rows = a.d; cols = a.dh;
+  }
+}
+
+TTT_DEVICE_INLINE float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// bf16 operand copies of all three matrices.
+__global__ void lact_cast_kernel(RowArgs a) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= a.BH * (2 * a.dh + a.d)) return;
+  int mat, bh, row, rows, cols;
+  row_decode(a, gw, mat, bh, row, rows, cols);
+  const size_t off = ((size_t)bh * rows + row) * cols;
+  for (int c = lane; c < cols; c += 32) a.Wb[mat][off + c] = __float2bfloat16_rn(a.W[mat][off + c]);
+}
+
+// GD / momentum: sum the split-K partials, update, normalise the row.
+__global__ void lact_update_kernel(RowArgs a) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= a.BH * (2 * a.dh + a.d)) return;
+  int mat, bh, row, rows, cols;
+  row_decode(a, gw, mat, bh, row, rows, cols);
+  if (!(a.mask & (1 << mat))) return;
+  const size_t off = ((size_t)bh * rows + row) * cols;
+  const size_t split_stride = (size_t)a.BH * rows * cols;
+  float w[ROW_MAXV];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < ROW_MAXV; ++i) {
+    const int c = lane + 32 * i;
+    w[i] = 0.f;
+    if (c < cols) {
+      float g = 0.f;
+      for (int s = 0; s < a.splits; ++s) g += a.part[mat][s * split_stride + off + c];
+      float u = g;
+      if (a.opt == 1) {
+        u = a.beta * a.M[mat][off + c] + g;
+        a.M[mat][off + c] = u;
+      }
+      w[i] = a.W[mat][off + c] - u;
+      ss += w[i] * w[i];
+    }
+  }
+  float scale = 1.f;
+  if (a.normalize) scale = 1.f / fmaxf(sqrtf(warp_sum(ss)), a.norm_eps);
+#pragma unroll
+  for (int i = 0; i < ROW_MAXV; ++i) {
+    const int c = lane + 32 * i;
+    if (c < cols) {
+      const float x = w[i] * scale;
+      a.W[mat][off + c] = x;
+      a.Wb[mat][off + c] = __float2bfloat16_rn(x);
+    }
+  }
+}
+
+// Muon step 1: M = beta M + G, and the row sums of squares of M.
+__global__ void muon_momentum_kernel(RowArgs a) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= a.BH * (2 * a.dh + a.d)) return;
+  int mat, bh, row, rows, cols;
+  row_decode(a, gw, mat, bh, row, rows, cols);
+  if (!(a.mask & (1 << mat))) return;
+  const size_t off = ((size_t)bh * rows + row) * cols;
+  const size_t split_stride = (size_t)a.BH * rows * cols;
+  float ss = 0.f;
+  for (int c = lane; c < cols; c += 32) {
+    float g = 0.f;
+    for (int s = 0; s < a.splits; ++s) g += a.part[mat][s * split_stride + off + c];
+    const float m = a.beta * a.M[mat][off + c] + g;
+    a.M[mat][off + c] = m;
+    ss += m * m;
+  }
+  ss = warp_sum(ss);
+  if (lane == 0) a.rowss[(size_t)mat * a.BH * a.dh + (size_t)bh * rows + row] = ss;
+}
+
+// Muon step 2: X = M / (||M||_F + eps) in the wide orientation (r x c with
+// r = min(d, dh)), fp32 and bf16.  One CTA row-block per (mat, bh, x-row).
+struct NsPrepArgs {
+  int BH, d, dh, r, c;
+  float eps;
+  const float* M[3];
+  const float* rowss;
+  float* X32;              // [3*BH][r][c]
+  __nv_bfloat16* Xb;       // [3*BH][r][c]
+};
+__global__ void ns_prep_kernel(NsPrepArgs a) {
+  const int mb = blockIdx.y;                 // mat * BH + bh
+  const int mat = mb / a.BH, bh = mb % a.BH;
+  const int rows = mat < 2 ? a.dh : a.d, cols = mat < 2 ? a.d : a.dh;
+  __shared__ float s_scale;
+  if (threadIdx.x < 32) {
+    float ss = 0.f;
+    const float* rs = a.rowss + (size_t)mat * a.BH * a.dh + (size_t)bh * rows;
+    for (int i = threadIdx.x; i < rows; i += 32) ss += rs[i];
+    ss = warp_sum(ss);
+    if (threadIdx.x == 0) s_scale = 1.f / (sqrtf(ss) + a.eps);
+  }
+  __syncthreads();
+  const float scale = s_scale;
+  const bool tall = rows > cols;
+  const float* Mm = a.M[mat] + (size_t)bh * rows * cols;
+  float* x32 = a.X32 + (size_t)mb * a.r * a.c;
+  __nv_bfloat16* xb = a.Xb + (size_t)mb * a.r * a.c;
+  const int xr = blockIdx.x;  // row of X
+  for (int xc = threadIdx.x; xc < a.c; xc += blockDim.x) {
+    const float v = (tall ? Mm[(size_t)xc * cols + xr] : Mm[(size_t)xr * cols + xc]) * scale;
+    x32[(size_t)xr * a.c + xc] = v;
+    xb[(size_t)xr * a.c + xc] = __float2bfloat16_rn(v);
+  }
+}
+
+// Muon step 4: W -= NS(M) (orientation restored), normalise the row.
+__global__ void muon_apply_kernel(RowArgs a, int r, int c) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= a.BH * (2 * a.dh + a.d)) return;
+  int mat, bh, row, rows, cols;
+  row_decode(a, gw, mat, bh, row, rows, cols);
+  if (!(a.mask & (1 << mat))) return;
+  const bool tall = rows > cols;
+  const float* X = a.X32 + (size_t)(mat * a.BH + bh) * r * c;
+  const size_t off = ((size_t)bh * rows + row) * cols;
+  float w[ROW_MAXV];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < ROW_MAXV; ++i) {
+    const int cc = lane + 32 * i;
+    w[i] = 0.f;
+    if (cc < cols) {
+      const float u = tall ? X[(size_t)cc * c + row] : X[(size_t)row * c + cc];
+      w[i] = a.W[mat][off + cc] - u;
+      ss += w[i] * w[i];
+    }
+  }
+  float scale = 1.f;
+  if (a.normalize) scale = 1.f / fmaxf(sqrtf(warp_sum(ss)), a.norm_eps);
+#pragma unroll
+  for (int i = 0; i < ROW_MAXV; ++i) {
+    const int cc = lane + 32 * i;
+    if (cc < cols) {
+      const float x = w[i] * scale;
+      a.W[mat][off + cc] = x;
+      a.Wb[mat][off + cc] = __float2bfloat16_rn(x);
+    }
+  }
+}
+
+// =====================================================================
+// host side
+// =====================================================================
+static int g_num_sms = 0;
+static int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static int grad_splits(int BH, int d, int dh, int cmax) {
+  const int tiles = BH * 3 * (dh / 128) * (d / 128);
+  const int ksteps = (cmax + 63) / 64;
+  int s = (2 * num_sms() + tiles - 1) / tiles;
+  s = std::max(1, std::min(s, std::max(1, ksteps / 8)));
+  return s;
+}
+
+LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
+                                    int causal, int opt) {
+  LactWorkspace w{};
+  const size_t BH = (size_t)B * H;
+  const int cin = std::min(chunk, std::max(N_in, 1));
+  int cmax = std::max(cin, causal ? 0 : N_q);
+  cmax = (cmax + 127) / 128 * 128;
+  w.cmax = cmax;
+  w.splits = grad_splits((int)BH, d, dh, cin);
+  size_t o = 0;
+  w.status = o; o = align256(o + 256);
+  w.w1b = o; o = align256(o + BH * dh * d * 2);
+  w.w3b = o; o = align256(o + BH * dh * d * 2);
+  w.w2b = o; o = align256(o + BH * d * dh * 2);
+  w.dh1 = o; o = align256(o + BH * cmax * dh * 2);
+  w.dh3 = o; o = align256(o + BH * cmax * dh * 2);
+  w.gm = o; o = align256(o + BH * cmax * dh * 2);
+  w.aq = o; o = align256(o + BH * cmax * dh * 2);
+  w.part = o; o = align256(o + (size_t)w.splits * BH * 3 * d * dh * 4);
+  w.rowss = w.nsx32 = w.nsxb = w.nsa32 = w.nsab = w.nsbb = o;
+  if (opt == 2) {
+    const size_t r = std::min(d, dh), c = std::max(d, dh);
+    w.rowss = o; o = align256(o + 3 * BH * std::max(d, dh) * 4);
+    w.nsx32 = o; o = align256(o + 3 * BH * r * c * 4);
+    w.nsxb = o; o = align256(o + 2 * 3 * BH * r * c * 2);
+    w.nsa32 = o; o = align256(o + 3 * BH * r * r * 4);
+    w.nsab = o; o = align256(o + 3 * BH * r * r * 2);
+    w.nsbb = o; o = align256(o + 3 * BH * r * r * 2);
+  }
+  w.total = o;
+  return w;
+}
+
+template <int BN, bool A_MN, bool B_MN, int STAGES>
+static int run_gemm(const GemmMaps& maps, const GemmArgs& g, cudaStream_t stream, int kind) {
+  auto kfn = gemm_bf16_kernel<BN, A_MN, B_MN, STAGES>;
+  const int smem = (int)GemmSmem<BN, STAGES>::BYTES;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return -1;
+    attr_done = true;
+  }
+  const int tiles = ((g.M + 127) / 128) * (g.N / BN) * g.splits * g.batch;
+  if (tiles <= 0) return 0;
+  const int grid = std::min(tiles, num_sms());
+  prof_before(kind, stream);
+  kfn<<<grid, 192, smem, stream>>>(maps, g);
+  prof_after(kind, stream);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+static GemmArgs gemm_defaults(const DevStatus& st) {
+  GemmArgs g{};
+  g.splits = 1;
+  g.npairs = 1;
+  g.alpha = 1.f;
+  g.st = st;
+  return g;
+}
+
+#define TTT_TRY(...)                      \
+  do {                                    \
+    if ((__VA_ARGS__) != 0) return -1;    \
+  } while (0)
+
+int launch_lact(const LactLaunch& L, cudaStream_t stream) {
+  const int BH = L.B * L.H, d = L.d, dh = L.dh;
+  const LactWorkspace w =
+      lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt);
+  uint8_t* ws = L.ws;
+  __nv_bfloat16* w1b = reinterpret_cast<__nv_bfloat16*>(ws + w.w1b);
+  __nv_bfloat16* w3b = reinterpret_cast<__nv_bfloat16*>(ws + w.w3b);
+  __nv_bfloat16* w2b = reinterpret_cast<__nv_bfloat16*>(ws + w.w2b);
+  __nv_bfloat16* dH1 = reinterpret_cast<__nv_bfloat16*>(ws + w.dh1);
+  __nv_bfloat16* dH3 = reinterpret_cast<__nv_bfloat16*>(ws + w.dh3);
+  __nv_bfloat16* Gm = reinterpret_cast<__nv_bfloat16*>(ws + w.gm);
+  __nv_bfloat16* Aq = reinterpret_cast<__nv_bfloat16*>(ws + w.aq);
+  float* part = reinterpret_cast<float*>(ws + w.part);
+  const size_t mat_elems = (size_t)BH * d * dh;
+  float* W1 = L.state;
+  float* W3 = W1 + mat_elems;
+  float* W2 = W3 + mat_elems;
+  float* M1 = L.opt != 0 ? W2 + mat_elems : nullptr;
+  float* M3 = M1 ? M1 + mat_elems : nullptr;
+  float* M2 = M3 ? M3 + mat_elems : nullptr;
+
+  RowArgs ra{};
+  ra.BH = BH; ra.d = d; ra.dh = dh; ra.splits = w.splits; ra.opt = L.opt;
+  ra.normalize = L.normalize_rows; ra.mask = L.update_mask; ra.beta = L.beta;
+  ra.norm_eps = L.norm_eps; ra.ns_eps = L.ns_eps;
+  ra.W[0] = W1; ra.W[1] = W3; ra.W[2] = W2;
+  ra.M[0] = M1; ra.M[1] = M3; ra.M[2] = M2;
+  ra.Wb[0] = w1b; ra.Wb[1] = w3b; ra.Wb[2] = w2b;
+  ra.part[0] = part;
+  ra.part[1] = part + (size_t)w.splits * mat_elems;
+  ra.part[2] = part + 2 * (size_t)w.splits * mat_elems;
+  ra.rowss = reinterpret_cast<float*>(ws + w.rowss);
+  ra.X32 = reinterpret_cast<float*>(ws + w.nsx32);
+  const int row_warps = BH * (2 * dh + d);
+  const int row_blocks = (row_warps * 32 + 255) / 256;
+
+  prof_before(K_LACT_CAST, stream);
+  lact_cast_kernel<<<row_blocks, 256, 0, stream>>>(ra);
+  prof_after(K_LACT_CAST, stream);
+  TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+
+  // token tensors: {d, rows, BH}
+  KeyPassMaps km{};
+  const uint64_t tok_row = (uint64_t)d * 2;
+  const int q_rows = L.causal ? L.N_in : L.N_q;
+  if (L.N_in > 0) {
+    TTT_TRY(make_tmap_bf16_3d(&km.k, L.k, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 128));
+    TTT_TRY(make_tmap_bf16_3d(&km.v, L.v, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 128));
+  }
+  if (q_rows > 0)
+    TTT_TRY(make_tmap_bf16_3d(&km.q, L.q, d, q_rows, BH, tok_row, tok_row * q_rows, 64, 128));
+  else
+    km.q = km.k;
+  if (L.N_in == 0) { km.k = km.q; km.v = km.q; }
+  // weights (bf16 copies): W1, W3 [BH][dh][d] (K-major boxes of 64 rows),
+  // W2 [BH][d][dh] as an MN-major operand (box {64 hidden, 64 d-rows}).
+  TTT_TRY(make_tmap_bf16_3d(&km.w1, w1b, d, dh, BH, (uint64_t)d * 2, (uint64_t)d * dh * 2, 64, 64));
+  TTT_TRY(make_tmap_bf16_3d(&km.w3, w3b, d, dh, BH, (uint64_t)d * 2, (uint64_t)d * dh * 2, 64, 64));
+  TTT_TRY(make_tmap_bf16_3d(&km.w2, w2b, dh, d, BH, (uint64_t)dh * 2, (uint64_t)d * dh * 2, 64, 64));
+  // read GEMM operand: W2 as K-major B (N = d rows, K = dh)
+  GemmMaps rm{};
+  TTT_TRY(make_tmap_bf16_3d(&rm.b[0], w2b, dh, d, BH, (uint64_t)dh * 2, (uint64_t)d * dh * 2, 64, 128));
+
+  static bool kp_attr = false;
+  if (!kp_attr) {
+    if (cudaFuncSetAttribute(lact_keypass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kp::SMEM) != cudaSuccess)
+      return -1;
+    kp_attr = true;
+  }
+
+  auto key_pass = [&](int t0, int C, int nkt, int nqt) -> int {
+    KeyPassArgs a{};
+    a.C = C; a.t0 = t0; a.n_key_tiles = nkt; a.n_q_tiles = nqt; a.n_hb = dh / 64; a.BH = BH;
+    a.d_steps = d / 64; a.dh = dh; a.lr_len = L.N_in; a.lr = L.lr;
+    a.dH1 = dH1; a.dH3 = dH3; a.Gm = Gm; a.Aq = Aq;
+    a.inter_bs = (long long)w.cmax * dh; a.st = L.st;
+    const int tiles = (nkt + nqt) * a.n_hb * BH;
+    if (tiles <= 0) return 0;
+    prof_before(K_KEYPASS, stream);
+    lact_keypass_kernel<<<std::min(tiles, num_sms()), 192, kp::SMEM, stream>>>(km, a);
+    prof_after(K_KEYPASS, stream);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  };
+  auto read_out = [&](int t0, int C) -> int {
+    GemmArgs g = gemm_defaults(L.st);
+    g.M = C; g.N = d; g.batch = BH; g.k_steps = dh / 64;
+    g.a_m_off[0] = 0; g.a_k_off[0] = 0; g.b_n_off[0] = 0; g.b_k_off[0] = 0;
+    g.out_row_off = t0;
+    const int orows = L.causal ? L.N_in : L.N_q;
+    if (L.out_bf16) {
+      g.o16 = reinterpret_cast<__nv_bfloat16*>(L.out);
+      g.o16_bs = (long long)orows * d;
+      g.ld16 = d;
+    } else {
+      g.o32 = reinterpret_cast<float*>(L.out);
+      g.o32_bs = (long long)orows * d;
+      g.ld32 = d;
+    }
+    GemmMaps m = rm;
+    if (make_tmap_bf16_3d(&m.a[0], Aq, dh, C, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64,
+                          128))
+      return -1;
+    return run_gemm<128, false, false, 4>(m, g, stream, K_GEMM_READ);
+  };
+  auto gradients = [&](int t0, int C) -> int {
+    // intermediates [BH][cmax][dh] limited to C rows: rows >= C read as zero
+    CUtensorMap mdh1, mdh3, mgm;
+    if (make_tmap_bf16_3d(&mdh1, dH1, dh, C, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64, 64) ||
+        make_tmap_bf16_3d(&mdh3, dH3, dh, C, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64, 64) ||
+        make_tmap_bf16_3d(&mgm, Gm, dh, C, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64, 64))
+      return -1;
+    CUtensorMap mk, mv;  // token tensors as MN-major operands, box {64 d, 64 tokens}
+    if (make_tmap_bf16_3d(&mk, L.k, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 64) ||
+        make_tmap_bf16_3d(&mv, L.v, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 64))
+      return -1;
+    const int ksteps_total = (C + 63) / 64;
+    const int splits = std::min(w.splits, ksteps_total);
+    const int kps = (ksteps_total + splits - 1) / splits;
+    GemmArgs g = gemm_defaults(L.st);
+    g.batch = BH; g.splits = splits; g.k_steps = kps;
+    g.o32_ss = (long long)BH * d * dh;
+    g.o32_bs = (long long)d * dh;
+    // G1 = dH1^T K, G3 = dH3^T K: M = dh, N = d, K = tokens
+    g.M = dh; g.N = d; g.ld32 = d;
+    g.a_k_off[0] = 0; g.b_k_off[0] = t0;
+    GemmMaps m{};
+    m.a[0] = mdh1; m.b[0] = mk;
+    g.o32 = part;
+    TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
+    m.a[0] = mdh3;
+    g.o32 = part + (size_t)w.splits * mat_elems;
+    TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
+    // G2 = V^T Gm': M = d, N = dh
+    g.M = d; g.N = dh; g.ld32 = dh;
+    g.a_k_off[0] = t0; g.b_k_off[0] = 0;
+    m.a[0] = mv; m.b[0] = mgm;
+    g.o32 = part + 2 * (size_t)w.splits * mat_elems;
+    TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
+    // the update kernels sum exactly `splits` partials
+    return splits;
+  };
+  auto muon = [&]() -> int {
+    const int r = std::min(d, dh), c = std::max(d, dh);
+    const int nb = 3 * BH;
+    float* X32 = reinterpret_cast<float*>(ws + w.nsx32);
+    __nv_bfloat16* Xb[2] = {reinterpret_cast<__nv_bfloat16*>(ws + w.nsxb),
+                            reinterpret_cast<__nv_bfloat16*>(ws + w.nsxb) + (size_t)nb * r * c};
+    float* A32 = reinterpret_cast<float*>(ws + w.nsa32);
+    __nv_bfloat16* Ab = reinterpret_cast<__nv_bfloat16*>(ws + w.nsab);
+    __nv_bfloat16* Bb = reinterpret_cast<__nv_bfloat16*>(ws + w.nsbb);
+    prof_before(K_MUON_MOM, stream);
+    muon_momentum_kernel<<<row_blocks, 256, 0, stream>>>(ra);
+    prof_after(K_MUON_MOM, stream);
+    NsPrepArgs pa{};
+    pa.BH = BH; pa.d = d; pa.dh = dh; pa.r = r; pa.c = c; pa.eps = L.ns_eps;
+    pa.M[0] = M1; pa.M[1] = M3; pa.M[2] = M2; pa.rowss = ra.rowss; pa.X32 = X32; pa.Xb = Xb[0];
+    prof_before(K_NS_PREP, stream);
+    ns_prep_kernel<<<dim3(r, nb), 256, 0, stream>>>(pa);
+    prof_after(K_NS_PREP, stream);
+    TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    CUtensorMap mab, mbb, mxk[2], mxn[2];
+    TTT_TRY(make_tmap_bf16_3d(&mab, Ab, r, r, nb, (uint64_t)r * 2, (uint64_t)r * r * 2, 64, 128));
+    TTT_TRY(make_tmap_bf16_3d(&mbb, Bb, r, r, nb, (uint64_t)r * 2, (uint64_t)r * r * 2, 64, 128));
+    for (int i = 0; i < 2; ++i) {
+      TTT_TRY(make_tmap_bf16_3d(&mxk[i], Xb[i], c, r, nb, (uint64_t)c * 2, (uint64_t)r * c * 2, 64, 128));
+      TTT_TRY(make_tmap_bf16_3d(&mxn[i], Xb[i], c, r, nb, (uint64_t)c * 2, (uint64_t)r * c * 2, 64, 64));
+    }
+    for (int it = 0; it < L.ns_steps; ++it) {
+      const int cur = it & 1;
+      GemmMaps m{};
+      // A = X X^T  (fp32 + bf16)
+      GemmArgs g = gemm_defaults(L.st);
+      g.M = r; g.N = r; g.batch = nb; g.k_steps = c / 64;
+      g.o32 = A32; g.o32_bs = (long long)r * r; g.ld32 = r;
+      g.o16 = Ab; g.o16_bs = (long long)r * r; g.ld16 = r;
+      m.a[0] = mxk[cur]; m.b[0] = mxk[cur];
+      TTT_TRY(run_gemm<128, false, false, 4>(m, g, stream, K_GEMM_NS));
+      // B = b A + c A A  (bf16)
+      g = gemm_defaults(L.st);
+      g.M = r; g.N = r; g.batch = nb; g.k_steps = r / 64;
+      g.alpha = L.ns_c; g.beta = L.ns_b; g.cin = A32; g.cin_bs = (long long)r * r; g.ldc = r;
+      g.o16 = Bb; g.o16_bs = (long long)r * r; g.ld16 = r;
+      m.a[0] = mab; m.b[0] = mab;
+      TTT_TRY(run_gemm<128, false, false, 4>(m, g, stream, K_GEMM_NS));
+      // X <- a X + B X  (fp32 in place, bf16 into the other buffer)
+      g = gemm_defaults(L.st);
+      g.M = r; g.N = c; g.batch = nb; g.k_steps = r / 64;
+      g.alpha = 1.f; g.beta = L.ns_a; g.cin = X32; g.cin_bs = (long long)r * c; g.ldc = c;
+      g.o32 = X32; g.o32_bs = (long long)r * c; g.ld32 = c;
+      g.o16 = Xb[cur ^ 1]; g.o16_bs = (long long)r * c; g.ld16 = c;
+      m.a[0] = mbb; m.b[0] = mxn[cur];
+      TTT_TRY(run_gemm<128, false, true, 4>(m, g, stream, K_GEMM_NS));
+    }
+    prof_before(K_MUON_APPLY, stream);
+    muon_apply_kernel<<<row_blocks, 256, 0, stream>>>(ra, r, c);
+    prof_after(K_MUON_APPLY, stream);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  };
+
+  // ------------------------------------------------------------ chunk loop
+  for (int t0 = 0; t0 < L.N_in; t0 += L.chunk) {
+    const int C = std::min(L.chunk, L.N_in - t0);
+    const int nt = (C + 127) / 128;
+    TTT_TRY(key_pass(t0, C, nt, L.causal ? nt : 0));
+    if (L.causal) TTT_TRY(read_out(t0, C));
+    const int splits = gradients(t0, C);
+    if (splits < 0) return -1;
+    ra.splits = splits;
+    if (L.opt == 2) {
+      TTT_TRY(muon());
+    } else {
+      prof_before(K_UPDATE, stream);
+      lact_update_kernel<<<row_blocks, 256, 0, stream>>>(ra);
+      prof_after(K_UPDATE, stream);
+      TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    }
+  }
+  if (!L.causal && L.N_q > 0) {
+    TTT_TRY(key_pass(0, L.N_q, 0, (L.N_q + 127) / 128));
+    TTT_TRY(read_out(0, L.N_q));
+  }
+  return 0;
+}
+
+}  // namespace ttt

@@ -1,0 +1,430 @@
+// ttt_linear.cu -- linear fast weight trained on -<W k, v> == causal linear
+// attention ("Test-Time Training with KV Binding Is Secretly Linear
+// Attention", summary "B. Reformulación Teórica", "Formulación Paralela").
+//
+// Chunked form per (b, h), state S = W^T [dk, dv] in fp32:
+//   O_c   = (Q_c K_c^T  o  causal mask) (diag(eta_c) V_c) + Q_c S_{c-1}
+//   S_c   = S_{c-1} + K_c^T diag(eta_c) V_c
+//
+// Two kernels:
+//  * ttt_linear_simt_kernel   -- exact fp32 FFMA on CUDA cores; any dk, dv <=
+//    128, fp32 or bf16 inputs; honours the caller's chunk (capped at 32).
+//  * ttt_linear_umma_kernel   -- bf16, dk = dv = 64, one persistent CTA per
+//    (b, h) chain walking 128-token tiles: TMA loads Q/K/V, tcgen05 MMAs with
+//    fp32 accumulators in TMEM, the fp32 state S resident in TMEM for the
+//    whole sequence, causal mask and per-token lr applied by the epilogue
+//    warps between the MMAs.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ttt {
+
+// =====================================================================
+// CUDA-core kernel
+// =====================================================================
+constexpr int SIMT_THREADS = 256;
+constexpr int SIMT_MAXC = 32;
+
+template <typename Tin>
+TTT_DEVICE_INLINE float load_in(const Tin* p, size_t i);
+template <>
+TTT_DEVICE_INLINE float load_in<float>(const float* p, size_t i) { return p[i]; }
+template <>
+TTT_DEVICE_INLINE float load_in<__nv_bfloat16>(const __nv_bfloat16* p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(SIMT_THREADS)
+    ttt_linear_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                           const Tin* __restrict__ v, const float* __restrict__ lr,
+                           float* __restrict__ S, Tout* __restrict__ out, int N, int dk, int dv,
+                           int C, int include_diag) {
+  extern __shared__ float sm[];
+  float* Ss = sm;                       // [dk][dv]
+  float* Qs = Ss + dk * dv;             // [C][dk]
+  float* Ks = Qs + SIMT_MAXC * dk;      // [C][dk]
+  float* Vs = Ks + SIMT_MAXC * dk;      // [C][dv]  (pre-scaled by eta)
+  float* Ps = Vs + SIMT_MAXC * dv;      // [C][C]
+  const int bh = blockIdx.x;
+  const size_t qk_base = (size_t)bh * N * dk;
+  const size_t v_base = (size_t)bh * N * dv;
+  float* Sg = S + (size_t)bh * dk * dv;
+
+  for (int i = threadIdx.x; i < dk * dv; i += blockDim.x) Ss[i] = Sg[i];
+  __syncthreads();
+
+  for (int t0 = 0; t0 < N; t0 += C) {
+    const int Cc = min(C, N - t0);
+    for (int i = threadIdx.x; i < Cc * dk; i += blockDim.x) {
+      Qs[i] = load_in(q, qk_base + (size_t)t0 * dk + i);
+      Ks[i] = load_in(k, qk_base + (size_t)t0 * dk + i);
+    }
+    for (int i = threadIdx.x; i < Cc * dv; i += blockDim.x) {
+      const int t = i / dv;
+      Vs[i] = lr[(size_t)bh * N + t0 + t] * load_in(v, v_base + (size_t)t0 * dv + i);
+    }
+    __syncthreads();
+    // P[i][j] = q_i . k_j for j <= i (j < i without the diagonal)
+    for (int e = threadIdx.x; e < Cc * Cc; e += blockDim.x) {
+      const int i = e / Cc, j = e % Cc;
+      float acc = 0.f;
+      if (j < i || (include_diag && j == i)) {
+        for (int r = 0; r < dk; ++r) acc = fmaf(Qs[i * dk + r], Ks[j * dk + r], acc);
+      }
+      Ps[i * SIMT_MAXC + j] = acc;
+    }
+    __syncthreads();
+    // out_i = sum_j P[i][j] (eta_j v_j) + S^T q_i
+    for (int e = threadIdx.x; e < Cc * dv; e += blockDim.x) {
+      const int i = e / dv, c = e % dv;
+      float acc = 0.f;
+      for (int r = 0; r < dk; ++r) acc = fmaf(Qs[i * dk + r], Ss[r * dv + c], acc);
+      for (int j = 0; j < Cc; ++j) acc = fmaf(Ps[i * SIMT_MAXC + j], Vs[j * dv + c], acc);
+      out[v_base + (size_t)(t0 + i) * dv + c] = static_cast<Tout>(acc);
+    }
+    __syncthreads();
+    // S += K^T diag(eta) V
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
+      const int r = e / dv, c = e % dv;
+      float acc = Ss[e];
+      for (int j = 0; j < Cc; ++j) acc = fmaf(Ks[j * dk + r], Vs[j * dv + c], acc);
+      Ss[e] = acc;
+    }
+    __syncthreads();
+  }
+  for (int i = threadIdx.x; i < dk * dv; i += blockDim.x) Sg[i] = Ss[i];
+}
+
+size_t ttt_linear_simt_smem(int dk, int dv) {
+  return sizeof(float) *
+         ((size_t)dk * dv + 2 * SIMT_MAXC * dk + SIMT_MAXC * dv + SIMT_MAXC * SIMT_MAXC);
+}
+
+int launch_ttt_linear_simt(const LinearLaunch& L, cudaStream_t stream) {
+  const int C = L.chunk < SIMT_MAXC ? L.chunk : SIMT_MAXC;
+  const size_t smem = ttt_linear_simt_smem(L.dk, L.dv);
+  dim3 grid(L.B * L.H), block(SIMT_THREADS);
+#define TTT_SIMT_LAUNCH(TI, TO)                                                              \
+  do {                                                                                       \
+    auto kfn = ttt_linear_simt_kernel<TI, TO>;                                               \
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != \
+        cudaSuccess)                                                                         \
+      return -1;                                                                             \
+    prof_before(K_LIN_SIMT, stream);                                                         \
+    kfn<<<grid, block, smem, stream>>>((const TI*)L.q, (const TI*)L.k, (const TI*)L.v, L.lr, \
+                                       L.S, (TO*)L.out, L.N, L.dk, L.dv, C, L.include_diag); \
+    prof_after(K_LIN_SIMT, stream);                                                          \
+  } while (0)
+  if (L.in_bf16) {
+    if (L.out_bf16) TTT_SIMT_LAUNCH(__nv_bfloat16, __nv_bfloat16);
+    else TTT_SIMT_LAUNCH(__nv_bfloat16, float);
+  } else {
+    if (L.out_bf16) TTT_SIMT_LAUNCH(float, __nv_bfloat16);
+    else TTT_SIMT_LAUNCH(float, float);
+  }
+#undef TTT_SIMT_LAUNCH
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// =====================================================================
+// tcgen05 kernel, bf16, dk = dv = 64
+// =====================================================================
+namespace lin {
+constexpr int T = 128;          // tokens per tile
+constexpr int D = 64;           // dk = dv
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int THREADS = (2 + NUM_EPI_WARPS) * 32;
+constexpr uint32_t TILE_BYTES = T * D * 2;          // 16 KB (Q, K, V, eta*V tiles)
+constexpr uint32_t STAGE_BYTES = 3 * TILE_BYTES;    // Q, K, V
+constexpr int STAGES = 2;
+constexpr uint32_t OFF_STAGE = 0;
+constexpr uint32_t OFF_PT = OFF_STAGE + STAGES * STAGE_BYTES;      // 2 x 32 KB (masked P, bf16)
+constexpr uint32_t OFF_EV = OFF_PT + 2 * 2 * TILE_BYTES;          // 2 x 16 KB (eta*V, bf16)
+constexpr uint32_t OFF_SB = OFF_EV + 2 * TILE_BYTES;              // 8 KB (S, bf16)
+constexpr uint32_t OFF_BAR = OFF_SB + D * D * 2;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;             // + alignment slack
+// TMEM columns
+constexpr uint32_t TM_P0 = 0, TM_P1 = 128, TM_O = 256, TM_S = 320, TM_COLS = 512;
+}  // namespace lin
+
+struct LinUmmaArgs {
+  const float* lr;
+  float* S;           // [BH][64][64] fp32, in/out
+  void* out;          // [BH][N][64]
+  int N;
+  int include_diag;
+  int out_bf16;
+  DevStatus st;
+};
+
+__global__ void __launch_bounds__(lin::THREADS, 1)
+    ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap mapQ,
+                           const __grid_constant__ CUtensorMap mapK,
+                           const __grid_constant__ CUtensorMap mapV, LinUmmaArgs a) {
+  using namespace lin;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);   // [2]
+  uint64_t* empty = full + 2;                                       // [2]
+  uint64_t* pfull = empty + 2;                                      // [2]
+  uint64_t* ops = pfull + 2;                                        // [1]
+  uint64_t* ofull = ops + 1;                                        // [1]
+  uint64_t* fin = ofull + 1;                                        // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int n_tiles = (a.N + T - 1) / T;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&pfull[s], 1);
+    }
+    mbar_init(ops, NUM_EPI_WARPS * 32);
+    mbar_init(ofull, 1);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapQ);
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  Waiter W{abort_flag, a.st, 0};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i & 1;
+        if (i >= STAGES && !W.wait(&empty[s], ((i >> 1) - 1) & 1, 1)) break;
+        uint8_t* st = smem + OFF_STAGE + s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+        tma_load_3d(st, &mapQ, &full[s], 0, i * T, bh);
+        tma_load_3d(st + TILE_BYTES, &mapK, &full[s], 0, i * T, bh);
+        tma_load_3d(st + 2 * TILE_BYTES, &mapV, &full[s], 0, i * T, bh);
+        issued = i + 1;
+      }
+      if (W.aborted()) {  // drain the copies still in flight into our smem
+        for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; ++i)
+          W.drain(&full[i & 1], (i >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t id_qk = make_idesc(128, 128, false, false);
+      const uint32_t id_o = make_idesc(128, 64, false, true);
+      const uint32_t id_s = make_idesc(64, 64, true, true);
+      const uint32_t pt_base = smem_u32(smem + OFF_PT);
+      const uint32_t ev_base = smem_u32(smem + OFF_EV);
+      const uint32_t sb_base = smem_u32(smem + OFF_SB);
+      bool ok = W.wait(&full[0], 0, 2);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t qs = smem_u32(smem + OFF_STAGE), ks = qs + TILE_BYTES;
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + TM_P0, make_sdesc(qs + kk * 32, 16, 1024),
+                   make_sdesc(ks + kk * 32, 16, 1024), id_qk, kk > 0);
+        mma_commit(&pfull[0]);
+      }
+      for (int i = 0; ok && i < n_tiles; ++i) {
+        const int s = i & 1;
+        if (!W.wait(ops, i & 1, 3)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qs = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES);
+        const uint32_t ks = qs + TILE_BYTES;
+        const uint32_t pt = pt_base + s * 2 * TILE_BYTES;
+        const uint32_t ev = ev_base + s * TILE_BYTES;
+        // O = mask(P) (eta V): K = 128 keys, two 64-key atoms of the P tile
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + TM_O, make_sdesc(pt + (kk >> 2) * TILE_BYTES + (kk & 3) * 32, 16, 1024),
+                   make_sdesc(ev + kk * 2048, 8192, 1024), id_o, kk > 0);
+        // O += Q S_{prev}
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + TM_O, make_sdesc(qs + kk * 32, 16, 1024),
+                   make_sdesc(sb_base + kk * 2048, 8192, 1024), id_o, 1);
+        // S += K^T (eta V)   (M = 64: rows live in lanes 0-15 of each quadrant)
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + TM_S, make_sdesc(ks + kk * 2048, 8192, 1024),
+                   make_sdesc(ev + kk * 2048, 8192, 1024), id_s, 1);
+        mma_commit(ofull);
+        mma_commit(&empty[s]);
+        if (i + 1 < n_tiles) {
+          const int s1 = (i + 1) & 1;
+          if (!W.wait(&full[s1], ((i + 1) >> 1) & 1, 4)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qs1 = smem_u32(smem + OFF_STAGE + s1 * STAGE_BYTES);
+          const uint32_t ks1 = qs1 + TILE_BYTES;
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + (s1 ? TM_P1 : TM_P0), make_sdesc(qs1 + kk * 32, 16, 1024),
+                     make_sdesc(ks1 + kk * 32, 16, 1024), id_qk, kk > 0);
+          mma_commit(&pfull[s1]);
+        }
+      }
+      (void)ok;
+    }
+    if (lane == 0) {  // every MMA issued by this thread completes before teardown
+      mma_commit(fin);
+      W.drain(fin, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp & 3;                  // TMEM lane quadrant
+    const int hf = (warp - 2) >> 2;           // column half
+    const int r = q4 * 32 + lane;             // row of the tile
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    float* Sg = a.S + (size_t)bh * D * D;
+    const float* lrg = a.lr + (size_t)bh * a.N;
+    uint8_t* sb = smem + OFF_SB;
+    // S rows of the M = 64 accumulator: lanes 0-15 of quadrant q4 hold rows 16*q4 + lane
+    const bool s_owner = lane < 16;
+    const int srow = q4 * 16 + lane;
+    {
+      float vals[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) vals[j] = s_owner ? Sg[srow * D + hf * 32 + j] : 0.f;
+      tmem_st16(tmem + lane_base + TM_S + hf * 32, vals);
+      tmem_st16(tmem + lane_base + TM_S + hf * 32 + 16, vals + 16);
+      if (s_owner) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 8)
+          st_shared_v4(smem_u32(sb) + sw128_offset(srow, hf * 32 + j),
+                       pack_bf16x2(vals[j], vals[j + 1]), pack_bf16x2(vals[j + 2], vals[j + 3]),
+                       pack_bf16x2(vals[j + 4], vals[j + 5]), pack_bf16x2(vals[j + 6], vals[j + 7]));
+      }
+    }
+    auto store_out = [&](int tile) {
+      const int t = tile * T + r;
+      float o[32];
+      tmem_ld32(tmem + lane_base + TM_O + hf * 32, o);
+      if (t < a.N) {
+        const size_t base = ((size_t)bh * a.N + t) * D + hf * 32;
+        if (a.out_bf16) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pack_bf16x2(o[8 * j], o[8 * j + 1]), pack_bf16x2(o[8 * j + 2], o[8 * j + 3]),
+                                pack_bf16x2(o[8 * j + 4], o[8 * j + 5]), pack_bf16x2(o[8 * j + 6], o[8 * j + 7]));
+        } else {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+        }
+      }
+    };
+    bool ok = true;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int s = i & 1;
+      if (!W.wait(&pfull[s], (i >> 1) & 1, 5)) { ok = false; break; }
+      tc_fence_after();
+      const int t = i * T + r;
+      const float eta = (t < a.N) ? lrg[t] : 0.f;
+      // eta * V  -> EV[s]  (same swizzled layout as the TMA-loaded V tile)
+      {
+        const uint32_t vsrc = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES + 2 * TILE_BYTES);
+        const uint32_t evdst = smem_u32(smem + OFF_EV + s * TILE_BYTES);
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          const uint32_t off = sw128_offset(r, hf * 32 + j);
+          uint32_t w0, w1, w2, w3;
+          ld_shared_v4(vsrc + off, w0, w1, w2, w3);
+          st_shared_v4(evdst + off, pack_bf16x2(eta * bf16lo(w0), eta * bf16hi(w0)),
+                       pack_bf16x2(eta * bf16lo(w1), eta * bf16hi(w1)),
+                       pack_bf16x2(eta * bf16lo(w2), eta * bf16hi(w2)),
+                       pack_bf16x2(eta * bf16lo(w3), eta * bf16hi(w3)));
+        }
+      }
+      // masked P -> Pt[s] (keys hf*64 .. hf*64+63 form atom hf)
+      {
+        const uint32_t pdst = smem_u32(smem + OFF_PT + s * 2 * TILE_BYTES + hf * TILE_BYTES);
+        const uint32_t pcol = (s ? TM_P1 : TM_P0) + hf * 64;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          float p[32];
+          tmem_ld32(tmem + lane_base + pcol + h2 * 32, p);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int key = hf * 64 + h2 * 32 + j;
+            const bool keep = a.include_diag ? (key <= r) : (key < r);
+            p[j] = keep ? p[j] : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; j += 8)
+            st_shared_v4(pdst + sw128_offset(r, h2 * 32 + j), pack_bf16x2(p[j], p[j + 1]),
+                         pack_bf16x2(p[j + 2], p[j + 3]), pack_bf16x2(p[j + 4], p[j + 5]),
+                         pack_bf16x2(p[j + 6], p[j + 7]));
+        }
+      }
+      if (i > 0) {
+        if (!W.wait(ofull, (i - 1) & 1, 6)) { ok = false; break; }
+        tc_fence_after();
+        store_out(i - 1);
+        // S after tile i-1 -> bf16 operand copy for tile i
+        float sv[32];
+        tmem_ld32(tmem + lane_base + TM_S + hf * 32, sv);
+        if (s_owner) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8)
+            st_shared_v4(smem_u32(sb) + sw128_offset(srow, hf * 32 + j),
+                         pack_bf16x2(sv[j], sv[j + 1]), pack_bf16x2(sv[j + 2], sv[j + 3]),
+                         pack_bf16x2(sv[j + 4], sv[j + 5]), pack_bf16x2(sv[j + 6], sv[j + 7]));
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(ops);
+    }
+    if (ok && n_tiles > 0 && W.wait(ofull, (n_tiles - 1) & 1, 7)) {
+      tc_fence_after();
+      store_out(n_tiles - 1);
+      float sv[32];
+      tmem_ld32(tmem + lane_base + TM_S + hf * 32, sv);
+      if (s_owner) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) Sg[srow * D + hf * 32 + j] = sv[j];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
+int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv;
+  const uint64_t BH = (uint64_t)L.B * L.H;
+  if (make_tmap_bf16_3d(&mq, L.q, 64, L.N, BH, 64 * 2, (uint64_t)L.N * 64 * 2, 64, 128) ||
+      make_tmap_bf16_3d(&mk, L.k, 64, L.N, BH, 64 * 2, (uint64_t)L.N * 64 * 2, 64, 128) ||
+      make_tmap_bf16_3d(&mv, L.v, 64, L.N, BH, 64 * 2, (uint64_t)L.N * 64 * 2, 64, 128))
+    return -1;
+  LinUmmaArgs a{L.lr, L.S, L.out, L.N, L.include_diag, L.out_bf16, L.st};
+  if (cudaFuncSetAttribute(ttt_linear_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)lin::SMEM_BYTES) != cudaSuccess)
+    return -1;
+  prof_before(K_LIN_UMMA, stream);
+  ttt_linear_umma_kernel<<<dim3((unsigned)BH), dim3(lin::THREADS), lin::SMEM_BYTES, stream>>>(
+      mq, mk, mv, a);
+  prof_after(K_LIN_UMMA, stream);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace ttt

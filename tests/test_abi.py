@@ -1,0 +1,139 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/ttt.h declares, the ctypes structs match the C layout, and host-side
+validation rejects bad arguments before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import learned_linear_attention_b200 as T
+from learned_linear_attention_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ttt.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^(?:int|const char\*)\s+(\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from learned_linear_attention_b200 import build
+        build.build()
+    return T.load()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("ttt_linear_fwd", "lact_chunk_fwd", "lact_state_init", "lact_state_readout",
+              "ttt_linear_state_init", "ttt_linear_state_readout", "ttt_check_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(_declared_functions()) <= set(_lib._SIGS)
+
+
+def test_ctypes_structs_match_c_layout(lib):
+    fields = {"ttt_linear_desc": [f[0] for f in T.ttt_linear_desc._fields_],
+              "lact_desc": [f[0] for f in T.lact_desc._fields_]}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', 'int main(void){']
+    for s, fl in fields.items():
+        lines.append(f'printf("{s} %zu\\n", sizeof({s}));')
+        for f in fl:
+            lines.append(f'printf("{s}.{f} %zu\\n", offsetof({s}, {f}));')
+    lines.append("return 0;}")
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "l.c")
+        open(c, "w").write("\n".join(lines))
+        subprocess.run(["gcc", "-o", os.path.join(d, "l"), c], check=True)
+        out = subprocess.run([os.path.join(d, "l")], capture_output=True, text=True,
+                             check=True).stdout.split("\n")
+    got = dict(line.split() for line in out if line)
+    for s, fl in fields.items():
+        cls = getattr(T, s)
+        assert int(got[s]) == ctypes.sizeof(cls), s
+        for f in fl:
+            assert int(got[f"{s}.{f}"]) == getattr(cls, f).offset, f"{s}.{f}"
+
+
+def test_status_strings(lib):
+    assert T.status_string(0) == "TTT_OK"
+    assert T.status_string(-8) == "TTT_ERR_TIMEOUT"
+    assert T.status_string(-99) == "TTT_ERR_UNKNOWN"
+    assert "sm_100a" in T.ttt_build_info()
+
+
+def _call_linear_fwd(desc, q=16, k=16, v=16, lr=16, S=16, out=16, ws=16, ws_bytes=256):
+    return T.load().ttt_linear_fwd(ctypes.byref(desc), q, k, v, lr, S, out, ws, ws_bytes, None)
+
+
+def test_linear_validation_before_launch(lib):
+    good = T.make_linear_desc(1, 2, 8, 64, 64, 16)
+    bad_shape = T.make_linear_desc(0, 2, 8, 64, 64, 16)
+    assert _call_linear_fwd(bad_shape) == T.TTT_ERR_SHAPE
+    assert _call_linear_fwd(T.make_linear_desc(1, 2, 8, 64, 64, 0)) == T.TTT_ERR_ARG
+    assert _call_linear_fwd(T.make_linear_desc(1, 2, 8, 256, 64, 16)) == T.TTT_ERR_UNSUPPORTED
+    d = T.make_linear_desc(1, 2, 8, 64, 64, 16)
+    d.in_dtype = 7
+    assert _call_linear_fwd(d) == T.TTT_ERR_DTYPE
+    assert _call_linear_fwd(good, ws_bytes=8) == T.TTT_ERR_WORKSPACE
+    assert _call_linear_fwd(good, q=0) == T.TTT_ERR_ARG
+    assert _call_linear_fwd(good, k=24) == T.TTT_ERR_ALIGN
+    # N = 0 is a valid empty call and launches nothing
+    assert _call_linear_fwd(T.make_linear_desc(1, 2, 0, 64, 64, 16)) == T.TTT_OK
+    assert T.ttt_linear_workspace_bytes(good) == T.TTT_STATUS_BYTES
+
+
+def _call_lact(desc, ws_bytes=1 << 40, **ptrs):
+    p = dict(q=16, k=16, v=16, lr=16, state=16, out=16, ws=16)
+    p.update(ptrs)
+    return T.load().lact_chunk_fwd(ctypes.byref(desc), p["q"], p["k"], p["v"], p["lr"],
+                                   p["state"], p["out"], p["ws"], ws_bytes, None)
+
+
+def test_lact_validation_before_launch(lib):
+    assert _call_lact(T.make_lact_desc(1, 2, 64, 96, 256, 32)) == T.TTT_ERR_UNSUPPORTED
+    assert _call_lact(T.make_lact_desc(1, 2, 64, 128, 200, 32)) == T.TTT_ERR_UNSUPPORTED
+    assert _call_lact(T.make_lact_desc(1, 2, 64, 128, 256, 0)) == T.TTT_ERR_ARG
+    d = T.make_lact_desc(1, 2, 64, 128, 256, 32)
+    d.N_q = 10                                    # causal needs N_q == N_in
+    assert _call_lact(d) == T.TTT_ERR_SHAPE
+    d = T.make_lact_desc(1, 2, 64, 128, 256, 32, update_mask=0)
+    assert _call_lact(d) == T.TTT_ERR_ARG
+    d = T.make_lact_desc(1, 2, 64, 128, 256, 32)
+    d.in_dtype = T.TTT_F32
+    assert _call_lact(d) == T.TTT_ERR_DTYPE
+    good = T.make_lact_desc(1, 2, 64, 128, 256, 32)
+    assert _call_lact(good, ws_bytes=100) == T.TTT_ERR_WORKSPACE
+    assert _call_lact(good, k=0) == T.TTT_ERR_ARG
+    assert _call_lact(good, v=40) == T.TTT_ERR_ALIGN
+
+
+@pytest.mark.parametrize("opt,mult", [("gd", 3), ("momentum", 6), ("muon", 6)])
+def test_lact_state_bytes(lib, opt, mult):
+    d = T.make_lact_desc(2, 4, 32768, 128, 256, 2048, opt=opt)
+    assert T.lact_state_bytes(d) == mult * 2 * 4 * 128 * 256 * 4
+
+
+def test_lact_workspace_sizes_for_the_workloads(lib):
+    # 32K-token causal layer: bf16 weights + four [BH, 2048, dh] intermediates + partials
+    d3 = T.make_lact_desc(2, 4, 32768, 128, 256, 2048)
+    ws3 = T.lact_workspace_bytes(d3)
+    assert 4 * 8 * 2048 * 256 * 2 < ws3 < 64 << 20
+    # 196K-token view-synthesis set in one chunk: intermediates dominate
+    d4 = T.make_lact_desc(1, 2, 196608, 384, 768, 196608, N_q=4096, order="bidirectional")
+    assert T.lact_workspace_bytes(d4) > 3 * 2 * 196608 * 768 * 2
+    # ~1M tokens in 64K chunks with Muon: Newton-Schulz buffers present
+    d5 = T.make_lact_desc(1, 2, 1029120, 384, 768, 65536, N_q=8040, order="bidirectional",
+                          opt="muon")
+    assert T.lact_workspace_bytes(d5) < 2 << 30

@@ -1,0 +1,119 @@
+"""GPU parity for the LaCT SwiGLU fast-weight layer against the fp64 oracle,
+through the C ABI.  Tolerance: normwise max relative error 2e-2 (bf16
+operands, fp32 accumulation and fp32 state)."""
+import numpy as np
+import pytest
+
+from oracle import lact_forward
+from oracle.lact import lact_init_state
+from ttt_synth import make_lact_inputs, make_workload
+from gpu_util import LaCTRun, rel_err
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+def _oracle(x, opt="gd", **kw):
+    B = x.k.values.shape[0]
+    st = lact_init_state(x.W1, x.W3, x.W2, B, opt)
+    return lact_forward(x.q.values, x.k.values, x.v.values, x.lr, st, chunk=x.chunk,
+                        order=x.order, opt=opt, **kw)
+
+
+def _check(x, opt="gd", out_dtype="f32", tol=TOL, **kw):
+    run = LaCTRun(x, opt=opt, out_dtype=out_dtype, **kw)
+    out = run.run()
+    ref, st = _oracle(x, opt, **kw)
+    assert not np.isnan(out).any()
+    assert rel_err(out, ref) <= tol, rel_err(out, ref)
+    W = run.weights()
+    for g, r in zip(W[:3], (st.W1, st.W3, st.W2)):
+        assert rel_err(g, r) <= tol, rel_err(g, r)
+    return run, out, ref, st
+
+
+@pytest.mark.parametrize("opt", ["gd", "momentum"])
+def test_causal_ragged_chunks(cuda_device, opt):
+    # chunks 256, 256, 128+40: several token tiles and a ragged last chunk
+    x = make_lact_inputs(1, 2, 680, 128, 256, chunk=256, order="causal", cfg=31)
+    _check(x, opt)
+
+
+def test_causal_bf16_output(cuda_device):
+    x = make_lact_inputs(2, 1, 384, 128, 256, chunk=128, order="causal", cfg=32)
+    _check(x, out_dtype="bf16")
+
+
+@pytest.mark.parametrize("opt", ["gd", "momentum", "muon"])
+def test_bidirectional_ragged_queries(cuda_device, opt):
+    x = make_lact_inputs(1, 2, 700, 128, 256, chunk=256, order="bidirectional", Nq=200,
+                         v_norm=True, lr_kind="0.01sig", cfg=33)
+    _check(x, opt)
+
+
+def test_wide_hidden_and_head_dims(cuda_device):
+    x = make_lact_inputs(1, 1, 300, 384, 768, chunk=300, order="bidirectional", Nq=130,
+                         v_norm=True, lr_kind="0.01sig", cfg=34)
+    _check(x)
+
+
+def test_update_mask_without_normalisation(cuda_device):
+    x = make_lact_inputs(1, 2, 512, 128, 256, chunk=128, order="causal", cfg=35)
+    run, *_ = _check(x, update_mask=4, normalize_rows=False)
+    W = run.weights()
+    assert np.array_equal(W[0][0], x.W1) and np.array_equal(W[1][0], x.W3)
+
+
+def test_rows_are_unit_norm_after_update(cuda_device):
+    x = make_lact_inputs(1, 2, 256, 128, 256, chunk=128, order="causal", cfg=36)
+    run = LaCTRun(x)
+    run.run()
+    for W in run.weights():
+        assert np.abs(np.linalg.norm(W.astype(np.float64), axis=-1) - 1).max() < 1e-5
+
+
+def test_causal_outputs_ignore_future_tokens(cuda_device):
+    x = make_lact_inputs(1, 2, 512, 128, 256, chunk=128, order="causal", cfg=37)
+    o1 = LaCTRun(x).run()
+    x2 = make_lact_inputs(1, 2, 512, 128, 256, chunk=128, order="causal", cfg=38)
+    for a, b in ((x2.q, x.q), (x2.k, x.k), (x2.v, x.v)):
+        a.values[:, :, :256], a.bits[:, :, :256] = b.values[:, :, :256], b.bits[:, :, :256]
+    x2.lr[:, :, :256] = x.lr[:, :, :256]
+    x2.W1, x2.W3, x2.W2 = x.W1, x.W3, x.W2
+    o2 = LaCTRun(x2).run()
+    assert np.array_equal(o1[:, :, :256], o2[:, :, :256])
+
+
+def test_streaming_split_equals_single_call(cuda_device):
+    import copy
+    x = make_lact_inputs(1, 2, 512, 128, 256, chunk=128, order="causal", cfg=39)
+    full = LaCTRun(x, opt="momentum")
+    of = full.run()
+    a = copy.deepcopy(x)
+    for tt in (a.q, a.k, a.v):
+        tt.values, tt.bits = tt.values[:, :, :256], tt.bits[:, :, :256]
+    a.lr = a.lr[:, :, :256]
+    b = copy.deepcopy(x)
+    for tt in (b.q, b.k, b.v):
+        tt.values, tt.bits = tt.values[:, :, 256:], tt.bits[:, :, 256:]
+    b.lr = b.lr[:, :, 256:]
+    ra = LaCTRun(a, opt="momentum")
+    oa = ra.run()
+    Wa = ra.weights()
+    rb = LaCTRun(b, opt="momentum")
+    rb.init_state(Wa[0], Wa[1], Wa[2], per_batch=True)
+    rb.set_momentum(*Wa[3:])
+    ob = rb.run()
+    assert rel_err(np.concatenate([oa, ob], 2), of) <= 1e-5
+
+
+@pytest.mark.slow
+def test_causal_n32k_workload(cuda_device):
+    x = make_workload("lact_causal_n32k")
+    _check(x)
+
+
+@pytest.mark.slow
+def test_bidirectional_196k_workload(cuda_device):
+    x = make_workload("lact_bidir_196k")
+    _check(x)

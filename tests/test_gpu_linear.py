@@ -1,0 +1,134 @@
+"""GPU parity for the linear fast weight (TTT-linear == causal linear
+attention) against the fp64 oracle, through the C ABI.
+
+Tolerances (normwise max relative error, max|gpu-ref| / max|ref|): 1e-4 for
+fp32 inputs on the CUDA-core kernel, 2e-2 for bf16 inputs with fp32
+accumulation on the tensor-core kernel."""
+import numpy as np
+import pytest
+import torch
+
+import learned_linear_attention_b200 as T
+from oracle import ttt_linear_attention_sum, ttt_linear_recurrent
+from ttt_synth import make_linear_inputs, make_workload
+from gpu_util import rel_err, run_linear
+
+pytestmark = pytest.mark.gpu
+TOL_F32, TOL_BF16 = 1e-4, 2e-2
+
+
+def _oracle(x, include_diag=True, S0=None):
+    return ttt_linear_recurrent(x.q.values, x.k.values, x.v.values, x.lr, S0, include_diag)
+
+
+def test_f32_n256_workload(cuda_device):
+    x = make_workload("ttt_linear_f32_n256")
+    out, S = run_linear(x)
+    ref, Sref = _oracle(x)
+    assert rel_err(out, ref) <= TOL_F32
+    assert rel_err(S, Sref) <= TOL_F32
+
+
+@pytest.mark.parametrize("include_diag", [True, False])
+def test_f32_ragged_with_initial_state(cuda_device, include_diag):
+    x = make_linear_inputs(2, 3, 77, 24, 40, chunk=9, dtype="f32", lr_kind="0.1sig", cfg=11,
+                           with_S0=True)
+    out, S = run_linear(x, include_diag, S0=x.S0)
+    ref, Sref = _oracle(x, include_diag, x.S0)
+    assert rel_err(out, ref) <= TOL_F32
+    assert rel_err(S, Sref) <= TOL_F32
+
+
+@pytest.mark.parametrize("include_diag", [True, False])
+@pytest.mark.parametrize("N", [1, 128, 300, 1000])
+def test_bf16_tensor_core_kernel(cuda_device, include_diag, N):
+    x = make_linear_inputs(2, 3, N, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=12,
+                           with_S0=True)
+    out, S = run_linear(x, include_diag, S0=x.S0)
+    ref, Sref = _oracle(x, include_diag, x.S0)
+    assert not np.isnan(out).any()
+    assert rel_err(out, ref) <= TOL_BF16
+    assert rel_err(S, Sref) <= TOL_BF16
+
+
+def test_bf16_output_dtype(cuda_device):
+    x = make_linear_inputs(1, 2, 400, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=13)
+    out, _ = run_linear(x, out_dtype="bf16")
+    ref, _ = _oracle(x)
+    assert rel_err(out, ref) <= TOL_BF16
+
+
+def test_bf16_cuda_core_dims(cuda_device):
+    x = make_linear_inputs(1, 2, 150, 32, 48, chunk=16, dtype="bf16", lr_kind="sig-2", cfg=14)
+    out, S = run_linear(x)
+    ref, Sref = _oracle(x)
+    assert rel_err(out, ref) <= TOL_BF16 and rel_err(S, Sref) <= TOL_BF16
+
+
+def test_chunk_size_invariance(cuda_device):
+    x = make_linear_inputs(1, 2, 96, 32, 32, chunk=16, dtype="f32", lr_kind="0.1sig", cfg=15)
+    outs = [run_linear(x, chunk=c)[0] for c in (1, 5, 16, 32, 96)]
+    for o in outs[1:]:
+        assert rel_err(o, outs[0]) <= 1e-5
+
+
+def test_gradient_ascent_negates_output(cuda_device):
+    x = make_linear_inputs(1, 2, 260, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=16)
+    o1, _ = run_linear(x)
+    x.lr = -x.lr
+    o2, _ = run_linear(x)
+    assert np.abs(o1 + o2).max() <= 1e-6 * np.abs(o1).max()
+
+
+def test_streaming_two_calls_equal_one(cuda_device):
+    x = make_linear_inputs(1, 2, 512, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=17)
+    full, Sfull = run_linear(x)
+    import copy
+    a, b = copy.deepcopy(x), copy.deepcopy(x)
+    for tt, src in ((a.q, x.q), (a.k, x.k), (a.v, x.v)):
+        tt.values, tt.bits = src.values[:, :, :256], src.bits[:, :, :256]
+    a.lr = x.lr[:, :, :256]
+    for tt, src in ((b.q, x.q), (b.k, x.k), (b.v, x.v)):
+        tt.values, tt.bits = src.values[:, :, 256:], src.bits[:, :, 256:]
+    b.lr = x.lr[:, :, 256:]
+    oa, Sa = run_linear(a)
+    ob, Sb = run_linear(b, S0=Sa)
+    assert rel_err(np.concatenate([oa, ob], 2), full) <= 1e-2
+    assert rel_err(Sb, Sfull) <= 1e-3
+
+
+def test_empty_sequence_is_a_no_op(cuda_device):
+    desc = T.make_linear_desc(1, 2, 0, 64, 64, 64)
+    S = torch.ones(1, 2, 64, 64, device="cuda")
+    ws = T.alloc_workspace(256)
+    e = torch.empty(0, device="cuda")
+    T.ttt_linear_fwd(desc, e, e, e, e, S, e, ws)
+    assert T.ttt_check_device_status(ws) == T.TTT_OK
+    assert bool((S == 1).all())
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+def test_bf16_n32k_workload_sampled(cuda_device, out_dtype):
+    """Full 4x16x32768 (d = 64) workload: sampled outputs against the
+    linear-attention sum, and the final state against sum eta k v^T."""
+    x = make_workload("ttt_linear_bf16_n32k")
+    out, S = run_linear(x, out_dtype=out_dtype)
+    idx = np.array([0, 1, 127, 128, 4095, 16384, 32766, 32767])
+    ref = ttt_linear_attention_sum(x.q.values, x.k.values, x.v.values, x.lr, t_index=idx)
+    assert rel_err(out[:, :, idx], ref) <= TOL_BF16
+    k64 = x.k.values.astype(np.float64)
+    ev = x.lr[..., None].astype(np.float64) * x.v.values.astype(np.float64)
+    Sref = np.matmul(np.swapaxes(k64, -1, -2), ev)
+    assert rel_err(S, Sref) <= TOL_BF16
+    assert not np.isnan(out).any()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
+    ws = T.alloc_workspace(256)
+    assert T.ttt_selftest_wait_timeout(ws, 2000) == T.TTT_OK
+    assert T.ttt_check_device_status(ws) == T.TTT_ERR_TIMEOUT
+    assert T.ttt_check_device_status(ws) == T.TTT_OK      # cleared
+    x = make_linear_inputs(1, 1, 64, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=18)
+    out, _ = run_linear(x)
+    assert rel_err(out, _oracle(x)[0]) <= TOL_BF16
