@@ -468,7 +468,7 @@ def main():
     tflops = bench.flops_per_step() / (step_ms * 1e-3) / 1e12
 
     secondary = None
-    if args.secondary and args.secondary != args.workload:
+    if args.secondary and args.secondary not in ("none", args.workload):
         sb = make_bench(args.secondary, device, seed=rank)
         for _ in range(args.warmup):
             sb.step(stream)
