@@ -170,6 +170,21 @@ int lact_chunk_fwd(const lact_desc* desc, const void* q, const void* k, const vo
                    const float* lr, void* state, void* out, void* ws, size_t ws_bytes,
                    void* stream);
 
+/* Same computation as lact_chunk_fwd for callers that cannot allocate device
+ * memory (code hosted by a program that owns all device allocations and
+ * hands it only its tensors; paths where cudaMalloc/cudaFree and their
+ * possible device synchronisation are not allowed).  The pages have no
+ * counterpart: this is a deployment variant, not part of the method.
+ * The workspace is a file-scope device array of 64 MiB held by every GPU
+ * that loads the library until exit; problems needing more (see
+ * lact_workspace_bytes) return TTT_ERR_WORKSPACE and nothing runs.  The
+ * first call on a device looks up the array's address with that device
+ * current.  All calls share the array: each call clears its status block on
+ * `stream`; calls whose GPU work overlaps race and must not be issued.  The
+ * status block is not readable through ttt_check_device_status. */
+int lact_chunk_fwd_noalloc(const lact_desc* desc, const void* q, const void* k, const void* v,
+                           const float* lr, void* state, void* out, void* stream);
+
 /* ------------------------------------------------------------------------
  * Status and diagnostics
  * ---------------------------------------------------------------------- */

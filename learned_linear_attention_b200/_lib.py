@@ -61,6 +61,7 @@ _SIGS = {
     "lact_state_init": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _I, _VP, _VP],
     "lact_state_readout": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _VP, _VP, _VP],
     "lact_chunk_fwd": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "lact_chunk_fwd_noalloc": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "ttt_check_device_status": [_VP, _VP],
     "ttt_selftest_wait_timeout": [_VP, _SZ, _I, _VP],
     "ttt_profile_begin": [],
@@ -174,6 +175,13 @@ def lact_chunk_fwd(desc, q, k, v, lr, state, out, ws, ws_bytes=None, stream=None
     st = load().lact_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lr),
                                _ptr(state), _ptr(out), _ptr(ws), nbytes, _stream(stream))
     return _check("lact_chunk_fwd", st) if check else st
+
+
+def lact_chunk_fwd_noalloc(desc, q, k, v, lr, state, out, stream=None, check=True):
+    """lact_chunk_fwd with the library's fixed device scratch as workspace."""
+    st = load().lact_chunk_fwd_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lr),
+                                       _ptr(state), _ptr(out), _stream(stream))
+    return _check("lact_chunk_fwd_noalloc", st) if check else st
 
 
 # ------------------------------------------------------------------ status
