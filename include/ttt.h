@@ -138,6 +138,11 @@ typedef struct {
   int update_mask;      /* 1..7                                              */
   ttt_dtype in_dtype;   /* q, k, v: TTT_BF16                                 */
   ttt_dtype out_dtype;  /* out: TTT_F32 or TTT_BF16                          */
+  int split_operands;   /* 0: bf16 tensor-core operands; 1: every weight,
+                           gradient intermediate and Newton-Schulz operand is
+                           carried as bf16 hi + lo (x = hi + lo), which keeps
+                           ~16 significant bits at 2-3x the MMA work.  Needed
+                           by MUON, whose update amplifies operand rounding */
 } lact_desc;
 
 /* Bytes of the state: W1, W3, W2 float32 per (b,h) (+ M1, M3, M2 for

@@ -31,7 +31,9 @@ def make_linear_desc(B, H, N, dk, dv, chunk, include_diag=True, in_dtype="bf16",
 def make_lact_desc(B, H, N_in, d, dh, chunk, *, N_q=None, order="causal", opt="gd", beta=0.9,
                    ns_steps=5, ns_coef=(3.4445, -4.7750, 2.0315), ns_eps=1e-7,
                    normalize_rows=True, norm_eps=1e-12, update_mask=7,
-                   out_dtype="f32") -> lact_desc:
+                   out_dtype="f32", split_operands=None) -> lact_desc:
+    """Fill a lact_desc.  split_operands defaults to on for Muon (its update
+    amplifies bf16 operand rounding) and off otherwise."""
     nq = N_in if order == "causal" else (N_q if N_q is not None else 0)
     desc = lact_desc()
     desc.B, desc.H, desc.N_in, desc.N_q, desc.d, desc.dh, desc.chunk = B, H, N_in, nq, d, dh, chunk
@@ -40,6 +42,7 @@ def make_lact_desc(B, H, N_in, d, dh, chunk, *, N_q=None, order="causal", opt="g
         desc.ns_coef[i] = ns_coef[i]
     desc.ns_eps, desc.normalize_rows, desc.norm_eps = ns_eps, int(bool(normalize_rows)), norm_eps
     desc.update_mask, desc.in_dtype, desc.out_dtype = update_mask, TTT_BF16, _DT[out_dtype]
+    desc.split_operands = int(opt == "muon") if split_operands is None else int(bool(split_operands))
     return desc
 
 

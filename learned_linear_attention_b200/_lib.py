@@ -41,7 +41,7 @@ class lact_desc(ctypes.Structure):
                 ("ns_coef", ctypes.c_float * 3), ("ns_eps", ctypes.c_float),
                 ("normalize_rows", ctypes.c_int), ("norm_eps", ctypes.c_float),
                 ("update_mask", ctypes.c_int), ("in_dtype", ctypes.c_int),
-                ("out_dtype", ctypes.c_int)]
+                ("out_dtype", ctypes.c_int), ("split_operands", ctypes.c_int)]
 
 
 class ttt_prof_entry(ctypes.Structure):

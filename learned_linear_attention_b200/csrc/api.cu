@@ -71,7 +71,7 @@ int check_lact(const lact_desc* d) {
 
 LactWorkspace layout_of(const lact_desc* d) {
   return lact_workspace_layout(d->B, d->H, d->N_in, d->N_q, d->d, d->dh, d->chunk,
-                               d->order == TTT_CAUSAL, (int)d->opt);
+                               d->order == TTT_CAUSAL, (int)d->opt, d->split_operands ? 1 : 0);
 }
 
 size_t lact_state_elems(const lact_desc* d) {
@@ -240,6 +240,7 @@ int lact_chunk_fwd(const lact_desc* d, const void* q, const void* k, const void*
   L.ns_a = d->ns_coef[0]; L.ns_b = d->ns_coef[1]; L.ns_c = d->ns_coef[2]; L.ns_eps = d->ns_eps;
   L.normalize_rows = d->normalize_rows ? 1 : 0; L.norm_eps = d->norm_eps;
   L.update_mask = d->update_mask; L.out_bf16 = d->out_dtype == TTT_BF16;
+  L.split = d->split_operands ? 1 : 0;
   L.q = q; L.k = k; L.v = v; L.lr = lr;
   L.state = reinterpret_cast<float*>(state);
   L.out = out;

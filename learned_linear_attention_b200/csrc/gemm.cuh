@@ -34,9 +34,21 @@ struct GemmArgs {
   long long o32_bs, o32_ss;
   int ld32;
   __nv_bfloat16* o16;    // (nullable)
+  __nv_bfloat16* o16lo;  // (nullable) residual v - bf16(v), same layout as o16
   long long o16_bs;
   int ld16;
   int out_row_off;       // added to the output row index
+  // ---- fused split-K reduction + optimizer + row normalisation (epi == 1);
+  // requires one N tile per row (N == BN).  W rows are the output rows.
+  int epi;               // 0: store (alpha/beta/cin/o32/o16), 1: update
+  float* W;              // fp32 weights [batch][M][N]
+  float* Mom;            // momentum [batch][M][N] (nullable: plain GD)
+  __nv_bfloat16* Wb;     // bf16 operand copy [batch][M][N]
+  __nv_bfloat16* Wlo;    // residual copy W - bf16(W) (nullable)
+  float* part;           // split-K partials [splits][batch][M][N] (splits > 1)
+  int* counters;         // [batch][tiles_m], zero on entry, left zero on exit
+  float mom_beta, norm_eps;
+  int normalize;
   DevStatus st;
 };
 
@@ -53,6 +65,102 @@ struct GemmSmem {
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
 };
 
+// Named barrier of the four epilogue warps (ids 0 is __syncthreads).
+TTT_DEVICE_INLINE void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Split-K reduction + GD / momentum update + row L2 normalisation of one
+// output tile whose N extent is a whole weight row.  Every split CTA stores
+// its partial; the last one to arrive (per-tile counter) sums them with its
+// own accumulator, applies the optimizer to the fp32 weights, normalises the
+// rows and refreshes the bf16 operand copy.
+template <int BN>
+TTT_DEVICE_INLINE void epilogue_update(const GemmArgs& g, uint32_t tacc, int b, int sp, int tm,
+                                       int m, bool valid, uint32_t* epi_flag) {
+  const size_t row_off = ((size_t)b * g.M + m) * BN;
+  const size_t split_stride = (size_t)g.batch * g.M * BN;
+  if (g.splits > 1) {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(tacc + c, v);
+      if (valid) {
+        float4* dst = reinterpret_cast<float4*>(g.part + sp * split_stride + row_off + c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      }
+    }
+    __threadfence();
+    epi_bar();
+    if (threadIdx.x == 64) {
+      int* cnt = g.counters + (size_t)b * ((g.M + 127) / 128) + tm;
+      const int prev = atomicAdd(cnt, 1);
+      const bool last = prev == g.splits - 1;
+      if (last) *cnt = 0;
+      *epi_flag = last ? 1u : 0u;
+    }
+    epi_bar();
+    if (*epi_flag == 0u) return;
+    __threadfence();
+  }
+  float ss = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    float v[32];
+    tmem_ld32(tacc + c, v);
+    if (!valid) continue;
+    for (int s = 0; s < g.splits; ++s) {
+      if (s == sp) continue;
+      const float4* src = reinterpret_cast<const float4*>(g.part + s * split_stride + row_off + c);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 x = __ldcg(src + j);
+        v[4 * j] += x.x; v[4 * j + 1] += x.y; v[4 * j + 2] += x.z; v[4 * j + 3] += x.w;
+      }
+    }
+    float* wr = g.W + row_off + c;
+    if (g.Mom != nullptr) {
+      float* mr = g.Mom + row_off + c;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float mm = g.mom_beta * mr[j] + v[j];
+        mr[j] = mm;
+        v[j] = mm;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float w = wr[j] - v[j];
+      v[j] = w;
+      ss += w * w;
+    }
+    if (g.normalize) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) wr[j] = v[j];
+    } else {
+      __nv_bfloat16* br = g.Wb + row_off + c;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        wr[j] = v[j];
+        br[j] = __float2bfloat16_rn(v[j]);
+        if (g.Wlo != nullptr) g.Wlo[row_off + c + j] = __float2bfloat16_rn(v[j] - __bfloat162float(br[j]));
+      }
+    }
+  }
+  if (g.normalize && valid) {
+    const float scale = 1.f / fmaxf(sqrtf(ss), g.norm_eps);
+    float* wr = g.W + row_off;
+    __nv_bfloat16* br = g.Wb + row_off;
+#pragma unroll 4
+    for (int c = 0; c < BN; ++c) {
+      const float w = wr[c] * scale;
+      wr[c] = w;
+      const __nv_bfloat16 h = __float2bfloat16_rn(w);
+      br[c] = h;
+      if (g.Wlo != nullptr) g.Wlo[row_off + c] = __float2bfloat16_rn(w - __bfloat162float(h));
+    }
+  }
+}
+
 template <int BN, bool A_MN, bool B_MN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
     gemm_bf16_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs g) {
@@ -67,6 +175,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* fin = aempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   uint32_t* abort_flag = tmem_slot + 1;
+  uint32_t* epi_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (g.M + 127) / 128, tiles_n = g.N / BN;
@@ -196,6 +305,12 @@ __global__ void __launch_bounds__(192, 1)
       const int m = tm * 128 + row;
       const bool valid = m < g.M;
       const int orow = m + g.out_row_off;
+      if (g.epi == 1) {
+        epilogue_update<BN>(g, tmem + lane_base + ab * BN, b, sp, tm, m, valid, epi_flag);
+        tc_fence_before();
+        mbar_arrive(&aempty[ab]);
+        continue;
+      }
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         float v[32];
@@ -225,12 +340,26 @@ __global__ void __launch_bounds__(192, 1)
               dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           }
           if (g.o16 != nullptr) {
-            uint4* dst = reinterpret_cast<uint4*>(g.o16 + b * g.o16_bs + (size_t)orow * g.ld16 + n);
+            const size_t o = b * g.o16_bs + (size_t)orow * g.ld16 + n;
+            uint32_t hv[16];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                                  pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
-                                  pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+            for (int j = 0; j < 16; ++j) hv[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(g.o16 + o);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(hv[4 * j], hv[4 * j + 1], hv[4 * j + 2], hv[4 * j + 3]);
+            if (g.o16lo != nullptr) {
+              uint4* dlo = reinterpret_cast<uint4*>(g.o16lo + o);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                uint32_t l[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const int e = 8 * j + 2 * u;
+                  l[u] = pack_bf16x2(v[e] - bf16lo(hv[e >> 1]), v[e + 1] - bf16hi(hv[e >> 1]));
+                }
+                dlo[j] = make_uint4(l[0], l[1], l[2], l[3]);
+              }
+            }
           }
         }
       }

@@ -42,6 +42,7 @@ struct LactLaunch {
   float norm_eps;
   int update_mask;
   int out_bf16;
+  int split;               // split-bf16 operands (hi + lo)
   const void *q, *k, *v;
   const float* lr;
   float* state;            // [W1 | W3 | W2 | M1 | M3 | M2] fp32
@@ -52,13 +53,15 @@ struct LactLaunch {
 };
 // Workspace layout (byte offsets) for a given problem.
 struct LactWorkspace {
-  size_t status, w1b, w3b, w2b, dh1, dh3, gm, aq, part, rowss, nsx32, nsxb, nsa32, nsab, nsbb,
-      total;
+  size_t status, w1b, w3b, w2b, dh1, dh3, gm, aq, part, cnt, rowss, nsx32, nsxb, nsa32, nsab,
+      nsbb, total;
+  // split operands (hi + lo bf16): residual copies
+  size_t w1lo, w3lo, w2lo, dh1lo, dh3lo, gmlo, aqlo, nsxlo, nsalo, nsblo;
   int cmax;                // rows of the per-chunk intermediates
   int splits;              // split-K factor of the gradient GEMMs
 };
 LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
-                                    int causal, int opt);
+                                    int causal, int opt, int split);
 int launch_lact(const LactLaunch& L, cudaStream_t stream);
 
 // ----------------------------------------------------------------- profiling

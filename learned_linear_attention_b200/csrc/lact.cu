@@ -50,13 +50,22 @@ struct KeyPassArgs {
   int lr_len;       // row length of lr ([BH][lr_len])
   const float* lr;
   __nv_bfloat16 *dH1, *dH3, *Gm, *Aq;   // [BH][cmax][dh]
+  // split operands: W = W_hi + W_lo (the K loop runs twice) and the
+  // intermediates are written as hi and lo bf16 parts
+  int split;
+  __nv_bfloat16 *dH1lo, *dH3lo, *Gmlo, *Aqlo;
   long long inter_bs;
   DevStatus st;
 };
 
 struct KeyPassMaps {
-  CUtensorMap k, v, q, w1, w3, w2;
+  CUtensorMap k, v, q, w1, w3, w2, w1lo, w3lo, w2lo;
 };
+
+// bf16 residual of x given its bf16 rounding h: the "lo" part of x = hi + lo.
+TTT_DEVICE_INLINE __nv_bfloat16 bf16_residual(float x, __nv_bfloat16 h) {
+  return __float2bfloat16_rn(x - __bfloat162float(h));
+}
 
 TTT_DEVICE_INLINE float sigmoidf_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
@@ -127,7 +136,10 @@ __global__ void __launch_bounds__(192, 1)
         const bool is_key = tt < a.n_key_tiles;
         const int row = a.t0 + (is_key ? tt : tt - a.n_key_tiles) * BM;
         const int j0 = hb * HB;
-        for (int ks = 0; ks < a.d_steps; ++ks, ++it) {
+        const int steps = a.d_steps * (a.split ? 2 : 1);
+        for (int kk = 0; kk < steps; ++kk, ++it) {
+          const bool lo = kk >= a.d_steps;
+          const int ks = lo ? kk - a.d_steps : kk;
           const uint32_t s = it % STAGES;
           if (it >= (uint32_t)STAGES && !W.wait(&empty[s], ((it / STAGES) - 1) & 1, 1)) {
             ok = false;
@@ -136,11 +148,13 @@ __global__ void __launch_bounds__(192, 1)
           uint8_t* st = smem + s * STAGE;
           mbar_arrive_expect_tx(&full[s], is_key ? STAGE : X_BYTES + W13_BYTES);
           tma_load_3d(st, is_key ? &maps.k : &maps.q, &full[s], ks * 64, row, bh);
-          tma_load_3d(st + X_BYTES + V_BYTES, &maps.w1, &full[s], ks * 64, j0, bh);
-          tma_load_3d(st + X_BYTES + V_BYTES + W13_BYTES / 2, &maps.w3, &full[s], ks * 64, j0, bh);
+          tma_load_3d(st + X_BYTES + V_BYTES, lo ? &maps.w1lo : &maps.w1, &full[s], ks * 64, j0, bh);
+          tma_load_3d(st + X_BYTES + V_BYTES + W13_BYTES / 2, lo ? &maps.w3lo : &maps.w3, &full[s],
+                      ks * 64, j0, bh);
           if (is_key) {
             tma_load_3d(st + X_BYTES, &maps.v, &full[s], ks * 64, row, bh);
-            tma_load_3d(st + X_BYTES + V_BYTES + W13_BYTES, &maps.w2, &full[s], j0, ks * 64, bh);
+            tma_load_3d(st + X_BYTES + V_BYTES + W13_BYTES, lo ? &maps.w2lo : &maps.w2, &full[s],
+                        j0, ks * 64, bh);
           }
         }
       }
@@ -163,7 +177,8 @@ __global__ void __launch_bounds__(192, 1)
         if (lt >= 2 && !W.wait(&aempty[ab], ((lt >> 1) - 1) & 1, 2)) break;
         tc_fence_after();
         const uint32_t d = tmem + ab * ACC_COLS;
-        for (int ks = 0; ks < a.d_steps; ++ks, ++it) {
+        const int steps = a.d_steps * (a.split ? 2 : 1);
+        for (int ks = 0; ks < steps; ++ks, ++it) {
           const uint32_t s = it % STAGES;
           if (!W.wait(&full[s], (it / STAGES) & 1, 3)) {
             ok = false;
@@ -216,7 +231,7 @@ __global__ void __launch_bounds__(192, 1)
           float g[32];
           tmem_ld32(base + 128 + jc, g);
           if (valid) {
-            uint32_t o1[16], o3[16], om[16];
+            uint32_t o1[16], o3[16], om[16], l1[16], l3[16], lm[16];
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               float r1[2], r3[2], rm[2];
@@ -233,6 +248,11 @@ __global__ void __launch_bounds__(192, 1)
               o1[j >> 1] = pack_bf16x2(r1[0], r1[1]);
               o3[j >> 1] = pack_bf16x2(r3[0], r3[1]);
               om[j >> 1] = pack_bf16x2(rm[0], rm[1]);
+              if (a.split) {
+                l1[j >> 1] = pack_bf16x2(r1[0] - bf16lo(o1[j >> 1]), r1[1] - bf16hi(o1[j >> 1]));
+                l3[j >> 1] = pack_bf16x2(r3[0] - bf16lo(o3[j >> 1]), r3[1] - bf16hi(o3[j >> 1]));
+                lm[j >> 1] = pack_bf16x2(rm[0] - bf16lo(om[j >> 1]), rm[1] - bf16hi(om[j >> 1]));
+              }
             }
             uint4* d1 = reinterpret_cast<uint4*>(a.dH1 + obase + jc);
             uint4* d3 = reinterpret_cast<uint4*>(a.dH3 + obase + jc);
@@ -243,19 +263,37 @@ __global__ void __launch_bounds__(192, 1)
               d3[j] = make_uint4(o3[4 * j], o3[4 * j + 1], o3[4 * j + 2], o3[4 * j + 3]);
               dm[j] = make_uint4(om[4 * j], om[4 * j + 1], om[4 * j + 2], om[4 * j + 3]);
             }
+            if (a.split) {
+              uint4* e1 = reinterpret_cast<uint4*>(a.dH1lo + obase + jc);
+              uint4* e3 = reinterpret_cast<uint4*>(a.dH3lo + obase + jc);
+              uint4* em = reinterpret_cast<uint4*>(a.Gmlo + obase + jc);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                e1[j] = make_uint4(l1[4 * j], l1[4 * j + 1], l1[4 * j + 2], l1[4 * j + 3]);
+                e3[j] = make_uint4(l3[4 * j], l3[4 * j + 1], l3[4 * j + 2], l3[4 * j + 3]);
+                em[j] = make_uint4(lm[4 * j], lm[4 * j + 1], lm[4 * j + 2], lm[4 * j + 3]);
+              }
+            }
           }
         } else if (valid) {
-          uint32_t oq[16];
+          uint32_t oq[16], lq[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
             const float a0 = h1[j] * sigmoidf_fast(h1[j]) * h3[j];
             const float a1 = h1[j + 1] * sigmoidf_fast(h1[j + 1]) * h3[j + 1];
             oq[j >> 1] = pack_bf16x2(a0, a1);
+            if (a.split) lq[j >> 1] = pack_bf16x2(a0 - bf16lo(oq[j >> 1]), a1 - bf16hi(oq[j >> 1]));
           }
           uint4* dq = reinterpret_cast<uint4*>(a.Aq + obase + jc);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             dq[j] = make_uint4(oq[4 * j], oq[4 * j + 1], oq[4 * j + 2], oq[4 * j + 3]);
+          if (a.split) {
+            uint4* eq = reinterpret_cast<uint4*>(a.Aqlo + obase + jc);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              eq[j] = make_uint4(lq[4 * j], lq[4 * j + 1], lq[4 * j + 2], lq[4 * j + 3]);
+          }
         }
       }
       tc_fence_before();
@@ -279,6 +317,7 @@ struct RowArgs {
   float* W[3];              // fp32 state per matrix [BH][rows][cols]
   float* M[3];              // momentum (nullable)
   __nv_bfloat16* Wb[3];     // bf16 copies
+  __nv_bfloat16* Wlo[3];    // bf16 residual copies (split operands; nullable)
   const float* part[3];     // split-K partial gradients [splits][BH][rows][cols]
   float* rowss;             // [3][BH][rows] row sums of squares (Muon)
   const float* X32;         // NS result [3][BH][r][c] (Muon apply)
@@ -313,30 +352,59 @@ __global__ void lact_cast_kernel(RowArgs a) {
   int mat, bh, row, rows, cols;
   row_decode(a, gw, mat, bh, row, rows, cols);
   const size_t off = ((size_t)bh * rows + row) * cols;
-  for (int c = lane; c < cols; c += 32) a.Wb[mat][off + c] = __float2bfloat16_rn(a.W[mat][off + c]);
+  for (int c = lane; c < cols; c += 32) {
+    const float x = a.W[mat][off + c];
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    a.Wb[mat][off + c] = h;
+    if (a.Wlo[mat] != nullptr) a.Wlo[mat][off + c] = bf16_residual(x, h);
+  }
+}
+
+// Row kernels run one 128-thread block per weight row; each thread owns up
+// to ROW_PER_THREAD columns so the split-K partial loads are independent.
+constexpr int ROW_THREADS = 128, ROW_PER_THREAD = 8;   // cols <= 1024
+
+TTT_DEVICE_INLINE float block_sum128(float x, float* red) {
+  x = warp_sum(x);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = x;
+  __syncthreads();
+  const float t = red[0] + red[1] + red[2] + red[3];
+  __syncthreads();
+  return t;
+}
+
+TTT_DEVICE_INLINE void sum_partials(const RowArgs& a, int mat, size_t off, size_t split_stride,
+                                    int cols, float* g) {
+#pragma unroll
+  for (int i = 0; i < ROW_PER_THREAD; ++i) g[i] = 0.f;
+  for (int s = 0; s < a.splits; ++s) {
+    const float* p = a.part[mat] + s * split_stride + off;
+#pragma unroll
+    for (int i = 0; i < ROW_PER_THREAD; ++i) {
+      const int c = threadIdx.x + ROW_THREADS * i;
+      if (c < cols) g[i] += __ldcg(p + c);
+    }
+  }
 }
 
 // GD / momentum: sum the split-K partials, update, normalise the row.
-__global__ void lact_update_kernel(RowArgs a) {
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (gw >= a.BH * (2 * a.dh + a.d)) return;
+__global__ void __launch_bounds__(ROW_THREADS) lact_update_kernel(RowArgs a) {
+  __shared__ float red[4];
   int mat, bh, row, rows, cols;
-  row_decode(a, gw, mat, bh, row, rows, cols);
+  row_decode(a, blockIdx.x, mat, bh, row, rows, cols);
   if (!(a.mask & (1 << mat))) return;
   const size_t off = ((size_t)bh * rows + row) * cols;
   const size_t split_stride = (size_t)a.BH * rows * cols;
-  float w[ROW_MAXV];
+  float w[ROW_PER_THREAD];
+  sum_partials(a, mat, off, split_stride, cols, w);
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < ROW_MAXV; ++i) {
-    const int c = lane + 32 * i;
-    w[i] = 0.f;
+  for (int i = 0; i < ROW_PER_THREAD; ++i) {
+    const int c = threadIdx.x + ROW_THREADS * i;
     if (c < cols) {
-      float g = 0.f;
-      for (int s = 0; s < a.splits; ++s) g += a.part[mat][s * split_stride + off + c];
-      float u = g;
+      float u = w[i];
       if (a.opt == 1) {
-        u = a.beta * a.M[mat][off + c] + g;
+        u = a.beta * a.M[mat][off + c] + u;
         a.M[mat][off + c] = u;
       }
       w[i] = a.W[mat][off + c] - u;
@@ -344,37 +412,42 @@ __global__ void lact_update_kernel(RowArgs a) {
     }
   }
   float scale = 1.f;
-  if (a.normalize) scale = 1.f / fmaxf(sqrtf(warp_sum(ss)), a.norm_eps);
+  if (a.normalize) scale = 1.f / fmaxf(sqrtf(block_sum128(ss, red)), a.norm_eps);
 #pragma unroll
-  for (int i = 0; i < ROW_MAXV; ++i) {
-    const int c = lane + 32 * i;
+  for (int i = 0; i < ROW_PER_THREAD; ++i) {
+    const int c = threadIdx.x + ROW_THREADS * i;
     if (c < cols) {
       const float x = w[i] * scale;
+      const __nv_bfloat16 h = __float2bfloat16_rn(x);
       a.W[mat][off + c] = x;
-      a.Wb[mat][off + c] = __float2bfloat16_rn(x);
+      a.Wb[mat][off + c] = h;
+      if (a.Wlo[mat] != nullptr) a.Wlo[mat][off + c] = bf16_residual(x, h);
     }
   }
 }
 
 // Muon step 1: M = beta M + G, and the row sums of squares of M.
-__global__ void muon_momentum_kernel(RowArgs a) {
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (gw >= a.BH * (2 * a.dh + a.d)) return;
+__global__ void __launch_bounds__(ROW_THREADS) muon_momentum_kernel(RowArgs a) {
+  __shared__ float red[4];
   int mat, bh, row, rows, cols;
-  row_decode(a, gw, mat, bh, row, rows, cols);
+  row_decode(a, blockIdx.x, mat, bh, row, rows, cols);
   if (!(a.mask & (1 << mat))) return;
   const size_t off = ((size_t)bh * rows + row) * cols;
   const size_t split_stride = (size_t)a.BH * rows * cols;
+  float g[ROW_PER_THREAD];
+  sum_partials(a, mat, off, split_stride, cols, g);
   float ss = 0.f;
-  for (int c = lane; c < cols; c += 32) {
-    float g = 0.f;
-    for (int s = 0; s < a.splits; ++s) g += a.part[mat][s * split_stride + off + c];
-    const float m = a.beta * a.M[mat][off + c] + g;
-    a.M[mat][off + c] = m;
-    ss += m * m;
+#pragma unroll
+  for (int i = 0; i < ROW_PER_THREAD; ++i) {
+    const int c = threadIdx.x + ROW_THREADS * i;
+    if (c < cols) {
+      const float m = a.beta * a.M[mat][off + c] + g[i];
+      a.M[mat][off + c] = m;
+      ss += m * m;
+    }
   }
-  ss = warp_sum(ss);
-  if (lane == 0) a.rowss[(size_t)mat * a.BH * a.dh + (size_t)bh * rows + row] = ss;
+  ss = block_sum128(ss, red);
+  if (threadIdx.x == 0) a.rowss[(size_t)mat * a.BH * a.dh + (size_t)bh * rows + row] = ss;
 }
 
 // Muon step 2: X = M / (||M||_F + eps) in the wide orientation (r x c with
@@ -386,6 +459,7 @@ struct NsPrepArgs {
   const float* rowss;
   float* X32;              // [3*BH][r][c]
   __nv_bfloat16* Xb;       // [3*BH][r][c]
+  __nv_bfloat16* Xlo;      // residual (split operands; nullable)
 };
 __global__ void ns_prep_kernel(NsPrepArgs a) {
   const int mb = blockIdx.y;                 // mat * BH + bh
@@ -409,7 +483,9 @@ __global__ void ns_prep_kernel(NsPrepArgs a) {
   for (int xc = threadIdx.x; xc < a.c; xc += blockDim.x) {
     const float v = (tall ? Mm[(size_t)xc * cols + xr] : Mm[(size_t)xr * cols + xc]) * scale;
     x32[(size_t)xr * a.c + xc] = v;
-    xb[(size_t)xr * a.c + xc] = __float2bfloat16_rn(v);
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    xb[(size_t)xr * a.c + xc] = h;
+    if (a.Xlo != nullptr) a.Xlo[(size_t)mb * a.r * a.c + (size_t)xr * a.c + xc] = bf16_residual(v, h);
   }
 }
 
@@ -442,8 +518,10 @@ __global__ void muon_apply_kernel(RowArgs a, int r, int c) {
     const int cc = lane + 32 * i;
     if (cc < cols) {
       const float x = w[i] * scale;
+      const __nv_bfloat16 h = __float2bfloat16_rn(x);
       a.W[mat][off + cc] = x;
-      a.Wb[mat][off + cc] = __float2bfloat16_rn(x);
+      a.Wb[mat][off + cc] = h;
+      if (a.Wlo[mat] != nullptr) a.Wlo[mat][off + cc] = bf16_residual(x, h);
     }
   }
 }
@@ -473,7 +551,7 @@ static int grad_splits(int BH, int d, int dh, int cmax) {
 }
 
 LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
-                                    int causal, int opt) {
+                                    int causal, int opt, int split) {
   LactWorkspace w{};
   const size_t BH = (size_t)B * H;
   const int cin = std::min(chunk, std::max(N_in, 1));
@@ -491,6 +569,7 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
   w.gm = o; o = align256(o + BH * cmax * dh * 2);
   w.aq = o; o = align256(o + BH * cmax * dh * 2);
   w.part = o; o = align256(o + (size_t)w.splits * BH * 3 * d * dh * 4);
+  w.cnt = o; o = align256(o + BH * 3 * ((std::max(d, dh) + 127) / 128) * sizeof(int));
   w.rowss = w.nsx32 = w.nsxb = w.nsa32 = w.nsab = w.nsbb = o;
   if (opt == 2) {
     const size_t r = std::min(d, dh), c = std::max(d, dh);
@@ -500,6 +579,22 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
     w.nsa32 = o; o = align256(o + 3 * BH * r * r * 4);
     w.nsab = o; o = align256(o + 3 * BH * r * r * 2);
     w.nsbb = o; o = align256(o + 3 * BH * r * r * 2);
+  }
+  w.w1lo = w.w3lo = w.w2lo = w.dh1lo = w.dh3lo = w.gmlo = w.aqlo = w.nsxlo = w.nsalo = w.nsblo = o;
+  if (split) {
+    w.w1lo = o; o = align256(o + BH * dh * d * 2);
+    w.w3lo = o; o = align256(o + BH * dh * d * 2);
+    w.w2lo = o; o = align256(o + BH * d * dh * 2);
+    w.dh1lo = o; o = align256(o + BH * cmax * dh * 2);
+    w.dh3lo = o; o = align256(o + BH * cmax * dh * 2);
+    w.gmlo = o; o = align256(o + BH * cmax * dh * 2);
+    w.aqlo = o; o = align256(o + BH * cmax * dh * 2);
+    if (opt == 2) {
+      const size_t r = std::min(d, dh), c = std::max(d, dh);
+      w.nsxlo = o; o = align256(o + 2 * 3 * BH * r * c * 2);
+      w.nsalo = o; o = align256(o + 3 * BH * r * r * 2);
+      w.nsblo = o; o = align256(o + 3 * BH * r * r * 2);
+    }
   }
   w.total = o;
   return w;
@@ -540,16 +635,17 @@ static GemmArgs gemm_defaults(const DevStatus& st) {
 
 int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   const int BH = L.B * L.H, d = L.d, dh = L.dh;
+  const bool split = L.split != 0;
   const LactWorkspace w =
-      lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt);
+      lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt, L.split);
   uint8_t* ws = L.ws;
-  __nv_bfloat16* w1b = reinterpret_cast<__nv_bfloat16*>(ws + w.w1b);
-  __nv_bfloat16* w3b = reinterpret_cast<__nv_bfloat16*>(ws + w.w3b);
-  __nv_bfloat16* w2b = reinterpret_cast<__nv_bfloat16*>(ws + w.w2b);
-  __nv_bfloat16* dH1 = reinterpret_cast<__nv_bfloat16*>(ws + w.dh1);
-  __nv_bfloat16* dH3 = reinterpret_cast<__nv_bfloat16*>(ws + w.dh3);
-  __nv_bfloat16* Gm = reinterpret_cast<__nv_bfloat16*>(ws + w.gm);
-  __nv_bfloat16* Aq = reinterpret_cast<__nv_bfloat16*>(ws + w.aq);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
+  __nv_bfloat16 *w1b = bf(w.w1b), *w3b = bf(w.w3b), *w2b = bf(w.w2b);
+  __nv_bfloat16 *dH1 = bf(w.dh1), *dH3 = bf(w.dh3), *Gm = bf(w.gm), *Aq = bf(w.aq);
+  __nv_bfloat16 *w1lo = split ? bf(w.w1lo) : nullptr, *w3lo = split ? bf(w.w3lo) : nullptr,
+                *w2lo = split ? bf(w.w2lo) : nullptr;
+  __nv_bfloat16 *dH1lo = split ? bf(w.dh1lo) : nullptr, *dH3lo = split ? bf(w.dh3lo) : nullptr,
+                *Gmlo = split ? bf(w.gmlo) : nullptr, *Aqlo = split ? bf(w.aqlo) : nullptr;
   float* part = reinterpret_cast<float*>(ws + w.part);
   const size_t mat_elems = (size_t)BH * d * dh;
   float* W1 = L.state;
@@ -566,6 +662,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   ra.W[0] = W1; ra.W[1] = W3; ra.W[2] = W2;
   ra.M[0] = M1; ra.M[1] = M3; ra.M[2] = M2;
   ra.Wb[0] = w1b; ra.Wb[1] = w3b; ra.Wb[2] = w2b;
+  ra.Wlo[0] = w1lo; ra.Wlo[1] = w3lo; ra.Wlo[2] = w2lo;
   ra.part[0] = part;
   ra.part[1] = part + (size_t)w.splits * mat_elems;
   ra.part[2] = part + 2 * (size_t)w.splits * mat_elems;
@@ -579,27 +676,53 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   prof_after(K_LACT_CAST, stream);
   TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
 
-  // token tensors: {d, rows, BH}
-  KeyPassMaps km{};
+  // ---- tensor maps.  Token tensors {d, rows, BH}; K-major boxes {64, 128},
+  // MN-major boxes {64, 64}.  Weights (bf16 copies): W1, W3 [BH][dh][d],
+  // W2 [BH][d][dh].
   const uint64_t tok_row = (uint64_t)d * 2;
   const int q_rows = L.causal ? L.N_in : L.N_q;
+  auto tok_map = [&](CUtensorMap* m, const void* p, int rows, uint32_t box_rows) {
+    return make_tmap_bf16_3d(m, p, d, rows, BH, tok_row, tok_row * rows, 64, box_rows);
+  };
+  auto w13_map = [&](CUtensorMap* m, const void* p) {    // K-major, 64 hidden rows per box
+    return make_tmap_bf16_3d(m, p, d, dh, BH, (uint64_t)d * 2, (uint64_t)d * dh * 2, 64, 64);
+  };
+  auto w2_mn_map = [&](CUtensorMap* m, const void* p) {  // MN-major (hidden contiguous)
+    return make_tmap_bf16_3d(m, p, dh, d, BH, (uint64_t)dh * 2, (uint64_t)d * dh * 2, 64, 64);
+  };
+  auto w2_k_map = [&](CUtensorMap* m, const void* p) {   // K-major B for the read (N = d)
+    return make_tmap_bf16_3d(m, p, dh, d, BH, (uint64_t)dh * 2, (uint64_t)d * dh * 2, 64, 128);
+  };
+  auto inter_map = [&](CUtensorMap* m, const void* p, int rows, uint32_t box_rows) {
+    return make_tmap_bf16_3d(m, p, dh, rows, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64,
+                             box_rows);
+  };
+  KeyPassMaps km{};
   if (L.N_in > 0) {
-    TTT_TRY(make_tmap_bf16_3d(&km.k, L.k, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 128));
-    TTT_TRY(make_tmap_bf16_3d(&km.v, L.v, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 128));
+    TTT_TRY(tok_map(&km.k, L.k, L.N_in, 128));
+    TTT_TRY(tok_map(&km.v, L.v, L.N_in, 128));
   }
-  if (q_rows > 0)
-    TTT_TRY(make_tmap_bf16_3d(&km.q, L.q, d, q_rows, BH, tok_row, tok_row * q_rows, 64, 128));
-  else
-    km.q = km.k;
+  if (q_rows > 0) TTT_TRY(tok_map(&km.q, L.q, q_rows, 128));
+  else km.q = km.k;
   if (L.N_in == 0) { km.k = km.q; km.v = km.q; }
-  // weights (bf16 copies): W1, W3 [BH][dh][d] (K-major boxes of 64 rows),
-  // W2 [BH][d][dh] as an MN-major operand (box {64 hidden, 64 d-rows}).
-  TTT_TRY(make_tmap_bf16_3d(&km.w1, w1b, d, dh, BH, (uint64_t)d * 2, (uint64_t)d * dh * 2, 64, 64));
-  TTT_TRY(make_tmap_bf16_3d(&km.w3, w3b, d, dh, BH, (uint64_t)d * 2, (uint64_t)d * dh * 2, 64, 64));
-  TTT_TRY(make_tmap_bf16_3d(&km.w2, w2b, dh, d, BH, (uint64_t)dh * 2, (uint64_t)d * dh * 2, 64, 64));
-  // read GEMM operand: W2 as K-major B (N = d rows, K = dh)
-  GemmMaps rm{};
-  TTT_TRY(make_tmap_bf16_3d(&rm.b[0], w2b, dh, d, BH, (uint64_t)dh * 2, (uint64_t)d * dh * 2, 64, 128));
+  TTT_TRY(w13_map(&km.w1, w1b));
+  TTT_TRY(w13_map(&km.w3, w3b));
+  TTT_TRY(w2_mn_map(&km.w2, w2b));
+  if (split) {
+    TTT_TRY(w13_map(&km.w1lo, w1lo));
+    TTT_TRY(w13_map(&km.w3lo, w3lo));
+    TTT_TRY(w2_mn_map(&km.w2lo, w2lo));
+  } else {
+    km.w1lo = km.w1; km.w3lo = km.w3; km.w2lo = km.w2;
+  }
+  CUtensorMap mw2k, mw2klo;
+  TTT_TRY(w2_k_map(&mw2k, w2b));
+  if (split) TTT_TRY(w2_k_map(&mw2klo, w2lo));
+  CUtensorMap mk_mn{}, mv_mn{};   // token tensors as MN-major operands
+  if (L.N_in > 0) {
+    TTT_TRY(tok_map(&mk_mn, L.k, L.N_in, 64));
+    TTT_TRY(tok_map(&mv_mn, L.v, L.N_in, 64));
+  }
 
   static bool kp_attr = false;
   if (!kp_attr) {
@@ -614,6 +737,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     a.C = C; a.t0 = t0; a.n_key_tiles = nkt; a.n_q_tiles = nqt; a.n_hb = dh / 64; a.BH = BH;
     a.d_steps = d / 64; a.dh = dh; a.lr_len = L.N_in; a.lr = L.lr;
     a.dH1 = dH1; a.dH3 = dH3; a.Gm = Gm; a.Aq = Aq;
+    a.split = split ? 1 : 0; a.dH1lo = dH1lo; a.dH3lo = dH3lo; a.Gmlo = Gmlo; a.Aqlo = Aqlo;
     a.inter_bs = (long long)w.cmax * dh; a.st = L.st;
     const int tiles = (nkt + nqt) * a.n_hb * BH;
     if (tiles <= 0) return 0;
@@ -622,10 +746,10 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     prof_after(K_KEYPASS, stream);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   };
+  // out rows [t0, t0 + C) = Aq W2^T (split: hi*hi + hi*lo + lo*hi)
   auto read_out = [&](int t0, int C) -> int {
     GemmArgs g = gemm_defaults(L.st);
     g.M = C; g.N = d; g.batch = BH; g.k_steps = dh / 64;
-    g.a_m_off[0] = 0; g.a_k_off[0] = 0; g.b_n_off[0] = 0; g.b_k_off[0] = 0;
     g.out_row_off = t0;
     const int orows = L.causal ? L.N_in : L.N_q;
     if (L.out_bf16) {
@@ -637,99 +761,156 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       g.o32_bs = (long long)orows * d;
       g.ld32 = d;
     }
-    GemmMaps m = rm;
-    if (make_tmap_bf16_3d(&m.a[0], Aq, dh, C, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64,
-                          128))
-      return -1;
+    GemmMaps m{};
+    TTT_TRY(inter_map(&m.a[0], Aq, C, 128));
+    m.b[0] = mw2k;
+    if (split) {
+      g.npairs = 3;
+      m.a[1] = m.a[0];
+      m.b[1] = mw2klo;
+      TTT_TRY(inter_map(&m.a[2], Aqlo, C, 128));
+      m.b[2] = mw2k;
+    }
     return run_gemm<128, false, false, 4>(m, g, stream, K_GEMM_READ);
   };
-  auto gradients = [&](int t0, int C) -> int {
-    // intermediates [BH][cmax][dh] limited to C rows: rows >= C read as zero
-    CUtensorMap mdh1, mdh3, mgm;
-    if (make_tmap_bf16_3d(&mdh1, dH1, dh, C, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64, 64) ||
-        make_tmap_bf16_3d(&mdh3, dH3, dh, C, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64, 64) ||
-        make_tmap_bf16_3d(&mgm, Gm, dh, C, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64, 64))
-      return -1;
-    CUtensorMap mk, mv;  // token tensors as MN-major operands, box {64 d, 64 tokens}
-    if (make_tmap_bf16_3d(&mk, L.k, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 64) ||
-        make_tmap_bf16_3d(&mv, L.v, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 64))
-      return -1;
+  // Chunk gradients G1 = dH1^T K, G3 = dH3^T K (rows = hidden units, N = d)
+  // and G2 = V^T Gm' (rows = d, N = dh); split-K over the chunk's tokens.
+  // fused: the epilogue of the last split also applies GD / momentum and the
+  // row normalisation (whole rows fit one N tile); otherwise partial sums
+  // go to the update kernels.
+  const bool fused_update = L.opt != 2 && (d == 128 || d == 256) && (dh == 128 || dh == 256);
+  int* counters = reinterpret_cast<int*>(ws + w.cnt);
+  const int cnt_stride = BH * ((std::max(d, dh) + 127) / 128);
+  if (fused_update && cudaMemsetAsync(counters, 0, 3 * cnt_stride * sizeof(int), stream) != cudaSuccess)
+    return -1;
+  auto gradients = [&](int t0, int C, bool fused) -> int {
+    CUtensorMap mi[3], mil[3];
+    __nv_bfloat16* hi[3] = {dH1, dH3, Gm};
+    __nv_bfloat16* lo[3] = {dH1lo, dH3lo, Gmlo};
+    for (int i = 0; i < 3; ++i) {
+      TTT_TRY(inter_map(&mi[i], hi[i], C, 64));
+      if (split) TTT_TRY(inter_map(&mil[i], lo[i], C, 64));
+    }
     const int ksteps_total = (C + 63) / 64;
     const int splits = std::min(w.splits, ksteps_total);
     const int kps = (ksteps_total + splits - 1) / splits;
     GemmArgs g = gemm_defaults(L.st);
     g.batch = BH; g.splits = splits; g.k_steps = kps;
-    g.o32_ss = (long long)BH * d * dh;
-    g.o32_bs = (long long)d * dh;
-    // G1 = dH1^T K, G3 = dH3^T K: M = dh, N = d, K = tokens
-    g.M = dh; g.N = d; g.ld32 = d;
-    g.a_k_off[0] = 0; g.b_k_off[0] = t0;
-    GemmMaps m{};
-    m.a[0] = mdh1; m.b[0] = mk;
-    g.o32 = part;
-    TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
-    m.a[0] = mdh3;
-    g.o32 = part + (size_t)w.splits * mat_elems;
-    TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
-    // G2 = V^T Gm': M = d, N = dh
-    g.M = d; g.N = dh; g.ld32 = dh;
-    g.a_k_off[0] = t0; g.b_k_off[0] = 0;
-    m.a[0] = mv; m.b[0] = mgm;
-    g.o32 = part + 2 * (size_t)w.splits * mat_elems;
-    TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
-    // the update kernels sum exactly `splits` partials
+    g.npairs = split ? 2 : 1;
+    if (fused) {
+      g.epi = 1;
+      g.mom_beta = L.beta; g.norm_eps = L.norm_eps; g.normalize = L.normalize_rows;
+    } else {
+      g.o32_ss = (long long)BH * d * dh;
+      g.o32_bs = (long long)d * dh;
+    }
+    for (int mat = 0; mat < 3; ++mat) {
+      if (fused && !(L.update_mask & (1 << mat))) continue;
+      GemmMaps m{};
+      if (mat < 2) {
+        g.M = dh; g.N = d; g.ld32 = d;
+        for (int p = 0; p < g.npairs; ++p) {
+          m.a[p] = p == 0 ? mi[mat] : mil[mat];
+          m.b[p] = mk_mn;
+          g.a_k_off[p] = 0; g.b_k_off[p] = t0;
+        }
+      } else {
+        g.M = d; g.N = dh; g.ld32 = dh;
+        for (int p = 0; p < g.npairs; ++p) {
+          m.a[p] = mv_mn;
+          m.b[p] = p == 0 ? mi[2] : mil[2];
+          g.a_k_off[p] = t0; g.b_k_off[p] = 0;
+        }
+      }
+      if (fused) {
+        g.W = ra.W[mat]; g.Mom = ra.M[mat]; g.Wb = ra.Wb[mat]; g.Wlo = ra.Wlo[mat];
+        g.part = const_cast<float*>(ra.part[mat]);
+        g.counters = counters + mat * cnt_stride;
+        if (g.N == 128) TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
+        else TTT_TRY(run_gemm<256, true, true, 3>(m, g, stream, K_GEMM_GRAD));
+      } else {
+        g.o32 = const_cast<float*>(ra.part[mat]);
+        TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
+      }
+    }
     return splits;
   };
+  // Muon: momentum, Newton-Schulz on the wide orientation, apply + norm.
   auto muon = [&]() -> int {
     const int r = std::min(d, dh), c = std::max(d, dh);
     const int nb = 3 * BH;
     float* X32 = reinterpret_cast<float*>(ws + w.nsx32);
-    __nv_bfloat16* Xb[2] = {reinterpret_cast<__nv_bfloat16*>(ws + w.nsxb),
-                            reinterpret_cast<__nv_bfloat16*>(ws + w.nsxb) + (size_t)nb * r * c};
+    __nv_bfloat16* Xb[2] = {bf(w.nsxb), bf(w.nsxb) + (size_t)nb * r * c};
+    __nv_bfloat16* Xl[2] = {split ? bf(w.nsxlo) : nullptr,
+                            split ? bf(w.nsxlo) + (size_t)nb * r * c : nullptr};
     float* A32 = reinterpret_cast<float*>(ws + w.nsa32);
-    __nv_bfloat16* Ab = reinterpret_cast<__nv_bfloat16*>(ws + w.nsab);
-    __nv_bfloat16* Bb = reinterpret_cast<__nv_bfloat16*>(ws + w.nsbb);
+    __nv_bfloat16 *Ab = bf(w.nsab), *Bb = bf(w.nsbb);
+    __nv_bfloat16 *Al = split ? bf(w.nsalo) : nullptr, *Bl = split ? bf(w.nsblo) : nullptr;
     prof_before(K_MUON_MOM, stream);
-    muon_momentum_kernel<<<row_blocks, 256, 0, stream>>>(ra);
+    muon_momentum_kernel<<<row_warps, ROW_THREADS, 0, stream>>>(ra);
     prof_after(K_MUON_MOM, stream);
     NsPrepArgs pa{};
     pa.BH = BH; pa.d = d; pa.dh = dh; pa.r = r; pa.c = c; pa.eps = L.ns_eps;
-    pa.M[0] = M1; pa.M[1] = M3; pa.M[2] = M2; pa.rowss = ra.rowss; pa.X32 = X32; pa.Xb = Xb[0];
+    pa.M[0] = M1; pa.M[1] = M3; pa.M[2] = M2; pa.rowss = ra.rowss; pa.X32 = X32;
+    pa.Xb = Xb[0]; pa.Xlo = Xl[0];
     prof_before(K_NS_PREP, stream);
     ns_prep_kernel<<<dim3(r, nb), 256, 0, stream>>>(pa);
     prof_after(K_NS_PREP, stream);
     TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
-    CUtensorMap mab, mbb, mxk[2], mxn[2];
-    TTT_TRY(make_tmap_bf16_3d(&mab, Ab, r, r, nb, (uint64_t)r * 2, (uint64_t)r * r * 2, 64, 128));
-    TTT_TRY(make_tmap_bf16_3d(&mbb, Bb, r, r, nb, (uint64_t)r * 2, (uint64_t)r * r * 2, 64, 128));
+    auto sq_map = [&](CUtensorMap* m, const void* p) {
+      return make_tmap_bf16_3d(m, p, r, r, nb, (uint64_t)r * 2, (uint64_t)r * r * 2, 64, 128);
+    };
+    CUtensorMap mab, mbb, mal, mbl, mxk[2], mxn[2], mxkl[2], mxnl[2];
+    TTT_TRY(sq_map(&mab, Ab));
+    TTT_TRY(sq_map(&mbb, Bb));
+    if (split) {
+      TTT_TRY(sq_map(&mal, Al));
+      TTT_TRY(sq_map(&mbl, Bl));
+    }
     for (int i = 0; i < 2; ++i) {
       TTT_TRY(make_tmap_bf16_3d(&mxk[i], Xb[i], c, r, nb, (uint64_t)c * 2, (uint64_t)r * c * 2, 64, 128));
       TTT_TRY(make_tmap_bf16_3d(&mxn[i], Xb[i], c, r, nb, (uint64_t)c * 2, (uint64_t)r * c * 2, 64, 64));
+      if (split) {
+        TTT_TRY(make_tmap_bf16_3d(&mxkl[i], Xl[i], c, r, nb, (uint64_t)c * 2, (uint64_t)r * c * 2, 64, 128));
+        TTT_TRY(make_tmap_bf16_3d(&mxnl[i], Xl[i], c, r, nb, (uint64_t)c * 2, (uint64_t)r * c * 2, 64, 64));
+      }
     }
+    // products of split operands: hi*hi + hi*lo + lo*hi
+    auto pairs = [&](GemmMaps& m, GemmArgs& g, const CUtensorMap& ah, const CUtensorMap& al,
+                     const CUtensorMap& bh, const CUtensorMap& bl) {
+      m.a[0] = ah; m.b[0] = bh;
+      if (split) {
+        m.a[1] = ah; m.b[1] = bl;
+        m.a[2] = al; m.b[2] = bh;
+        g.npairs = 3;
+      }
+    };
     for (int it = 0; it < L.ns_steps; ++it) {
       const int cur = it & 1;
       GemmMaps m{};
-      // A = X X^T  (fp32 + bf16)
+      // A = X X^T  (fp32 + bf16 hi/lo)
       GemmArgs g = gemm_defaults(L.st);
       g.M = r; g.N = r; g.batch = nb; g.k_steps = c / 64;
       g.o32 = A32; g.o32_bs = (long long)r * r; g.ld32 = r;
-      g.o16 = Ab; g.o16_bs = (long long)r * r; g.ld16 = r;
-      m.a[0] = mxk[cur]; m.b[0] = mxk[cur];
+      g.o16 = Ab; g.o16lo = Al; g.o16_bs = (long long)r * r; g.ld16 = r;
+      pairs(m, g, mxk[cur], mxkl[cur], mxk[cur], mxkl[cur]);
       TTT_TRY(run_gemm<128, false, false, 4>(m, g, stream, K_GEMM_NS));
-      // B = b A + c A A  (bf16)
+      // B = b A + c A A
+      m = GemmMaps{};
       g = gemm_defaults(L.st);
       g.M = r; g.N = r; g.batch = nb; g.k_steps = r / 64;
       g.alpha = L.ns_c; g.beta = L.ns_b; g.cin = A32; g.cin_bs = (long long)r * r; g.ldc = r;
-      g.o16 = Bb; g.o16_bs = (long long)r * r; g.ld16 = r;
-      m.a[0] = mab; m.b[0] = mab;
+      g.o16 = Bb; g.o16lo = Bl; g.o16_bs = (long long)r * r; g.ld16 = r;
+      pairs(m, g, mab, mal, mab, mal);
       TTT_TRY(run_gemm<128, false, false, 4>(m, g, stream, K_GEMM_NS));
-      // X <- a X + B X  (fp32 in place, bf16 into the other buffer)
+      // X <- a X + B X  (fp32 in place; bf16 hi/lo into the other buffers)
+      m = GemmMaps{};
       g = gemm_defaults(L.st);
       g.M = r; g.N = c; g.batch = nb; g.k_steps = r / 64;
       g.alpha = 1.f; g.beta = L.ns_a; g.cin = X32; g.cin_bs = (long long)r * c; g.ldc = c;
       g.o32 = X32; g.o32_bs = (long long)r * c; g.ld32 = c;
-      g.o16 = Xb[cur ^ 1]; g.o16_bs = (long long)r * c; g.ld16 = c;
-      m.a[0] = mbb; m.b[0] = mxn[cur];
+      g.o16 = Xb[cur ^ 1]; g.o16lo = Xl[cur ^ 1]; g.o16_bs = (long long)r * c; g.ld16 = c;
+      pairs(m, g, mbb, mbl, mxn[cur], mxnl[cur]);
       TTT_TRY(run_gemm<128, false, true, 4>(m, g, stream, K_GEMM_NS));
     }
     prof_before(K_MUON_APPLY, stream);
@@ -744,14 +925,15 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     const int nt = (C + 127) / 128;
     TTT_TRY(key_pass(t0, C, nt, L.causal ? nt : 0));
     if (L.causal) TTT_TRY(read_out(t0, C));
-    const int splits = gradients(t0, C);
+    const int splits = gradients(t0, C, fused_update);
     if (splits < 0) return -1;
+    if (fused_update) continue;
     ra.splits = splits;
     if (L.opt == 2) {
       TTT_TRY(muon());
     } else {
       prof_before(K_UPDATE, stream);
-      lact_update_kernel<<<row_blocks, 256, 0, stream>>>(ra);
+      lact_update_kernel<<<row_warps, ROW_THREADS, 0, stream>>>(ra);
       prof_after(K_UPDATE, stream);
       TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     }

@@ -245,6 +245,19 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       }
       for (int i = 0; ok && i < n_tiles; ++i) {
         const int s = i & 1;
+        // P of the next tile first: the epilogue converts it while this
+        // tile's O and S products run.
+        if (i + 1 < n_tiles) {
+          const int s1 = (i + 1) & 1;
+          if (!W.wait(&full[s1], ((i + 1) >> 1) & 1, 4)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qs1 = smem_u32(smem + OFF_STAGE + s1 * STAGE_BYTES);
+          const uint32_t ks1 = qs1 + TILE_BYTES;
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + (s1 ? TM_P1 : TM_P0), make_sdesc(qs1 + kk * 32, 16, 1024),
+                     make_sdesc(ks1 + kk * 32, 16, 1024), id_qk, kk > 0);
+          mma_commit(&pfull[s1]);
+        }
         if (!W.wait(ops, i & 1, 3)) { ok = false; break; }
         tc_fence_after();
         const uint32_t qs = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES);
@@ -265,17 +278,6 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
                    make_sdesc(ev + kk * 2048, 8192, 1024), id_s, 1);
         mma_commit(ofull);
         mma_commit(&empty[s]);
-        if (i + 1 < n_tiles) {
-          const int s1 = (i + 1) & 1;
-          if (!W.wait(&full[s1], ((i + 1) >> 1) & 1, 4)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t qs1 = smem_u32(smem + OFF_STAGE + s1 * STAGE_BYTES);
-          const uint32_t ks1 = qs1 + TILE_BYTES;
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + (s1 ? TM_P1 : TM_P0), make_sdesc(qs1 + kk * 32, 16, 1024),
-                     make_sdesc(ks1 + kk * 32, 16, 1024), id_qk, kk > 0);
-          mma_commit(&pfull[s1]);
-        }
       }
       (void)ok;
     }

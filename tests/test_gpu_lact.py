@@ -117,3 +117,21 @@ def test_causal_n32k_workload(cuda_device):
 def test_bidirectional_196k_workload(cuda_device):
     x = make_workload("lact_bidir_196k")
     _check(x)
+
+
+def test_split_operands_tighten_gd(cuda_device):
+    """hi+lo bf16 operands (about 16 significant bits) must track the fp64
+    oracle at least 4x closer than plain bf16 operands."""
+    x = make_lact_inputs(1, 2, 640, 128, 256, chunk=256, order="causal", cfg=40)
+    ref, _ = _oracle(x)
+    e_plain = rel_err(LaCTRun(x, split_operands=False).run(), ref)
+    e_split = rel_err(LaCTRun(x, split_operands=True).run(), ref)
+    assert e_split <= TOL and e_split * 4 <= e_plain, (e_split, e_plain)
+
+
+@pytest.mark.slow
+def test_bidirectional_muon_1m_workload(cuda_device):
+    """~1M input tokens in 64K chunks (15 full + one 46080-token chunk) with
+    momentum 0.9 and five Newton-Schulz steps, then 8040 queries."""
+    x = make_workload("lact_bidir_muon_1m")
+    _check(x, "muon", beta=0.9, ns_steps=5)
