@@ -11,8 +11,15 @@
 // * Warp 0: TMA producer; warp 1: MMA issuer + TMEM owner; warps 2-5:
 //   epilogue (TMEM -> registers -> global).  TMEM holds two accumulators so
 //   the epilogue of one tile overlaps the MMAs of the next.
-// * Split-K over blockIdx-independent tile ids: tile = ((b*splits + s) *
-//   tiles_n + tn) * tiles_m + tm; each CTA walks tiles with stride gridDim.x.
+// * Tiles: tile = ((b*splits + s) * tiles_n + tn) * tiles_m + tm; each CTA
+//   walks tiles with stride gridDim.x.  In cluster mode (cluster_n > 1) the
+//   cluster_n CTAs of a cluster take the N tiles of one output row block
+//   (tn fastest) and exchange per-row partial sums over distributed shared
+//   memory; one tile per CTA.
+// * epi == 1: the epilogue is the weight update of a chunk -- optimizer step
+//   on the fp32 weights, row L2 normalisation, bf16 operand copies -- with
+//   the output rows being weight rows (rows >= rows_first go to the second
+//   matrix, so [W1; W3] can be updated by one launch).
 #pragma once
 #include "common.cuh"
 
@@ -38,15 +45,16 @@ struct GemmArgs {
   long long o16_bs;
   int ld16;
   int out_row_off;       // added to the output row index
-  // ---- fused split-K reduction + optimizer + row normalisation (epi == 1);
-  // requires one N tile per row (N == BN).  W rows are the output rows.
-  int epi;               // 0: store (alpha/beta/cin/o32/o16), 1: update
-  float* W;              // fp32 weights [batch][M][N]
-  float* Mom;            // momentum [batch][M][N] (nullable: plain GD)
-  __nv_bfloat16* Wb;     // bf16 operand copy [batch][M][N]
-  __nv_bfloat16* Wlo;    // residual copy W - bf16(W) (nullable)
-  float* part;           // split-K partials [splits][batch][M][N] (splits > 1)
-  int* counters;         // [batch][tiles_m], zero on entry, left zero on exit
+  int cluster_n;         // > 1: N tiles of a row block form one cluster
+  // ---- epi == 1: weight update (splits == 1).  Row m of batch b is row m of
+  // matrix 0 ([batch][rows_first][ldw]) or row m - rows_first of matrix 1.
+  int epi;
+  int rows_first;
+  float* W[2];           // fp32 weights
+  float* Mom[2];         // momentum (nullable: plain GD)
+  __nv_bfloat16* Wb[2];  // bf16 operand copies
+  __nv_bfloat16* Wlo[2]; // bf16 residual copies (nullable)
+  int ldw;               // row length of the weights (= N)
   float mom_beta, norm_eps;
   int normalize;
   DevStatus st;
@@ -62,101 +70,132 @@ struct GemmSmem {
   static constexpr uint32_t B_BYTES = BN * 64 * 2;
   static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
   static constexpr uint32_t BAR_OFF = STAGES * STAGE;
-  static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
+  static constexpr uint32_t RED_OFF = BAR_OFF + 256;          // 128 floats (row sums)
+  static constexpr uint32_t BYTES = RED_OFF + 512 + 1024;
 };
 
-// Named barrier of the four epilogue warps (ids 0 is __syncthreads).
-TTT_DEVICE_INLINE void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+TTT_DEVICE_INLINE void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+TTT_DEVICE_INLINE float ld_dsmem_f32(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
 
-// Split-K reduction + GD / momentum update + row L2 normalisation of one
-// output tile whose N extent is a whole weight row.  Every split CTA stores
-// its partial; the last one to arrive (per-tile counter) sums them with its
-// own accumulator, applies the optimizer to the fp32 weights, normalises the
-// rows and refreshes the bf16 operand copy.
+// Weight update from one accumulator tile (epi == 1).  One thread owns one
+// row (its TMEM lane): pass 1 reads G from TMEM and the fp32 weights (and
+// momentum) from global, forms the unnormalised row, writes it back into
+// TMEM and accumulates its squared norm; in cluster mode the partial norms
+// of the N tiles are added over distributed shared memory; pass 2 scales
+// the row and stores fp32 weights and bf16 copies.
 template <int BN>
-TTT_DEVICE_INLINE void epilogue_update(const GemmArgs& g, uint32_t tacc, int b, int sp, int tm,
-                                       int m, bool valid, uint32_t* epi_flag) {
-  const size_t row_off = ((size_t)b * g.M + m) * BN;
-  const size_t split_stride = (size_t)g.batch * g.M * BN;
-  if (g.splits > 1) {
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      float v[32];
-      tmem_ld32(tacc + c, v);
-      if (valid) {
-        float4* dst = reinterpret_cast<float4*>(g.part + sp * split_stride + row_off + c);
+TTT_DEVICE_INLINE void epilogue_update(const GemmArgs& g, uint32_t tacc, int b, int m, int n0,
+                                       bool valid, float* red) {
+  const int mat = m >= g.rows_first ? 1 : 0;
+  const int mr = m - mat * g.rows_first;
+  const size_t ro = ((size_t)b * g.rows_first + mr) * g.ldw + n0;
+  float* Wr = g.W[mat] + ro;
+  float* Mr = g.Mom[mat] != nullptr ? g.Mom[mat] + ro : nullptr;
+  float ss = 0.f;
+  float4 wn[8];
+  if (valid) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    for (int j = 0; j < 8; ++j) wn[j] = reinterpret_cast<const float4*>(Wr)[j];
+  }
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t r0[16], r1[16];
+    tmem_ld16_issue(tacc + c, r0);
+    tmem_ld16_issue(tacc + c + 16, r1);
+    float4 wc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wc[j] = wn[j];
+    if (valid && c + 32 < BN) {   // prefetch the next 32 weights
+#pragma unroll
+      for (int j = 0; j < 8; ++j) wn[j] = reinterpret_cast<const float4*>(Wr + c + 32)[j];
+    }
+    float4 mc[8];
+    if (valid && Mr != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mc[j] = reinterpret_cast<const float4*>(Mr + c)[j];
+    }
+    tmem_wait_ld();
+    float u[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      u[j] = __uint_as_float(r0[j]);
+      u[16 + j] = __uint_as_float(r1[j]);
+    }
+    if (valid && Mr != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        mc[j].x = g.mom_beta * mc[j].x + u[4 * j];
+        mc[j].y = g.mom_beta * mc[j].y + u[4 * j + 1];
+        mc[j].z = g.mom_beta * mc[j].z + u[4 * j + 2];
+        mc[j].w = g.mom_beta * mc[j].w + u[4 * j + 3];
+        reinterpret_cast<float4*>(Mr + c)[j] = mc[j];
+        u[4 * j] = mc[j].x; u[4 * j + 1] = mc[j].y; u[4 * j + 2] = mc[j].z; u[4 * j + 3] = mc[j].w;
       }
     }
-    __threadfence();
-    epi_bar();
-    if (threadIdx.x == 64) {
-      int* cnt = g.counters + (size_t)b * ((g.M + 127) / 128) + tm;
-      const int prev = atomicAdd(cnt, 1);
-      const bool last = prev == g.splits - 1;
-      if (last) *cnt = 0;
-      *epi_flag = last ? 1u : 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      u[4 * j] = wc[j].x - u[4 * j];
+      u[4 * j + 1] = wc[j].y - u[4 * j + 1];
+      u[4 * j + 2] = wc[j].z - u[4 * j + 2];
+      u[4 * j + 3] = wc[j].w - u[4 * j + 3];
     }
-    epi_bar();
-    if (*epi_flag == 0u) return;
-    __threadfence();
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ss += u[j] * u[j];
+    }
+    tmem_st16(tacc + c, u);
+    tmem_st16(tacc + c + 16, u + 16);
   }
-  float ss = 0.f;
+  if (g.cluster_n > 1) {
+    const int row = threadIdx.x - 64;
+    red[row] = ss;
+    // warps 0-1 join this cluster barrier at the end of their roles
+    cluster_sync_all();
+    float tot = 0.f;
+    for (int r = 0; r < g.cluster_n; ++r) tot += ld_dsmem_f32(&red[row], (uint32_t)r);
+    ss = tot;
+  }
+  // pass 2 (tcgen05.ld is warp-collective: every lane runs it, stores are
+  // guarded by the row's validity)
+  const float scale = g.normalize ? 1.f / fmaxf(sqrtf(ss), g.norm_eps) : 1.f;
+  __nv_bfloat16* Br = g.Wb[mat] + ro;
+  __nv_bfloat16* Lr = g.Wlo[mat] != nullptr ? g.Wlo[mat] + ro : nullptr;
 #pragma unroll 1
   for (int c = 0; c < BN; c += 32) {
     float v[32];
     tmem_ld32(tacc + c, v);
     if (!valid) continue;
-    for (int s = 0; s < g.splits; ++s) {
-      if (s == sp) continue;
-      const float4* src = reinterpret_cast<const float4*>(g.part + s * split_stride + row_off + c);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float4 x = __ldcg(src + j);
-        v[4 * j] += x.x; v[4 * j + 1] += x.y; v[4 * j + 2] += x.z; v[4 * j + 3] += x.w;
+    for (int j = 0; j < 32; ++j) v[j] *= scale;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      reinterpret_cast<float4*>(Wr + c)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    uint32_t h[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) h[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      reinterpret_cast<uint4*>(Br + c)[j] = make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+    if (Lr != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t l[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int e = 8 * j + 2 * q;
+          l[q] = pack_bf16x2(v[e] - bf16lo(h[e >> 1]), v[e + 1] - bf16hi(h[e >> 1]));
+        }
+        reinterpret_cast<uint4*>(Lr + c)[j] = make_uint4(l[0], l[1], l[2], l[3]);
       }
-    }
-    float* wr = g.W + row_off + c;
-    if (g.Mom != nullptr) {
-      float* mr = g.Mom + row_off + c;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float mm = g.mom_beta * mr[j] + v[j];
-        mr[j] = mm;
-        v[j] = mm;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float w = wr[j] - v[j];
-      v[j] = w;
-      ss += w * w;
-    }
-    if (g.normalize) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) wr[j] = v[j];
-    } else {
-      __nv_bfloat16* br = g.Wb + row_off + c;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        wr[j] = v[j];
-        br[j] = __float2bfloat16_rn(v[j]);
-        if (g.Wlo != nullptr) g.Wlo[row_off + c + j] = __float2bfloat16_rn(v[j] - __bfloat162float(br[j]));
-      }
-    }
-  }
-  if (g.normalize && valid) {
-    const float scale = 1.f / fmaxf(sqrtf(ss), g.norm_eps);
-    float* wr = g.W + row_off;
-    __nv_bfloat16* br = g.Wb + row_off;
-#pragma unroll 4
-    for (int c = 0; c < BN; ++c) {
-      const float w = wr[c] * scale;
-      wr[c] = w;
-      const __nv_bfloat16 h = __float2bfloat16_rn(w);
-      br[c] = h;
-      if (g.Wlo != nullptr) g.Wlo[row_off + c] = __float2bfloat16_rn(w - __bfloat162float(h));
     }
   }
 }
@@ -175,12 +214,13 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* fin = aempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   uint32_t* abort_flag = tmem_slot + 1;
-  uint32_t* epi_flag = abort_flag + 1;
+  float* red = reinterpret_cast<float*>(smem + L::RED_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (g.M + 127) / 128, tiles_n = g.N / BN;
   const int n_tiles = tiles_m * tiles_n * g.splits * g.batch;
   const int total_k = g.k_steps * g.npairs;
+  const bool clustered = g.cluster_n > 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -208,18 +248,31 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   Waiter W{abort_flag, g.st, 100};
+
+  auto decode = [&](int t, int& tm, int& tn, int& b, int& sp) {
+    if (clustered) {
+      tn = t % tiles_n;
+      tm = (t / tiles_n) % tiles_m;
+    } else {
+      tm = t % tiles_m;
+      tn = (t / tiles_m) % tiles_n;
+    }
+    const int bs = t / (tiles_m * tiles_n);
+    b = bs / g.splits;
+    sp = bs % g.splits;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-        const int tm = t % tiles_m;
-        const int tn = (t / tiles_m) % tiles_n;
-        const int bs = t / (tiles_m * tiles_n);
-        const int b = bs / g.splits, sp = bs % g.splits;
+        int tm, tn, b, sp;
+        decode(t, tm, tn, b, sp);
         for (int kk = 0; kk < total_k; ++kk, ++it) {
           const int p = kk / g.k_steps;
           const int ks = (kk % g.k_steps) + sp * g.k_steps;
@@ -253,6 +306,7 @@ __global__ void __launch_bounds__(192, 1)
         for (uint32_t i = first; i < it; ++i) W.drain(&full[i % STAGES], (i / STAGES) & 1);
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = make_idesc(128, BN, A_MN, B_MN);
@@ -288,17 +342,17 @@ __global__ void __launch_bounds__(192, 1)
       mma_commit(fin);
       W.drain(fin, 0);
     }
+    __syncwarp();
   } else {
     // epilogue: warps 2..5 -> TMEM lane quadrants 2,3,0,1
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     uint32_t lt = 0;
+    bool synced = false;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
-      const int tm = t % tiles_m;
-      const int tn = (t / tiles_m) % tiles_n;
-      const int bs = t / (tiles_m * tiles_n);
-      const int b = bs / g.splits, sp = bs % g.splits;
+      int tm, tn, b, sp;
+      decode(t, tm, tn, b, sp);
       const uint32_t ab = lt & 1;
       if (!W.wait(&afull[ab], (lt >> 1) & 1, 4)) break;
       tc_fence_after();
@@ -306,7 +360,8 @@ __global__ void __launch_bounds__(192, 1)
       const bool valid = m < g.M;
       const int orow = m + g.out_row_off;
       if (g.epi == 1) {
-        epilogue_update<BN>(g, tmem + lane_base + ab * BN, b, sp, tm, m, valid, epi_flag);
+        epilogue_update<BN>(g, tmem + lane_base + ab * BN, b, m, tn * BN, valid, red);
+        synced = clustered;
         tc_fence_before();
         mbar_arrive(&aempty[ab]);
         continue;
@@ -366,6 +421,15 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(&aempty[ab]);
     }
+    // an epilogue that never reached the update (abort) still joins the
+    // cluster barrier its peers wait on
+    if (clustered && !synced) cluster_sync_all();
+  }
+  // cluster mode: warps 0-1 join the row-sum barrier here; then every
+  // thread waits until the peers have finished reading this CTA's row sums
+  if (clustered) {
+    if (warp < 2) cluster_sync_all();
+    cluster_sync_all();
   }
   tc_fence_before();
   __syncthreads();

@@ -4,9 +4,45 @@
 
 #include <stdio.h>
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace ttt {
+
+// ----------------------------------------------------------------- launches
+// Launch with programmatic stream serialisation (the kernel calls pdl_wait()
+// before reading what earlier work on the stream wrote).
+// cluster_x > 1 additionally groups consecutive CTAs into clusters.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                                      size_t smem, cudaStream_t stream, int cluster_x,
+                                      Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster_x > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  return launch_pdl_cluster(kernel, grid, block, smem, stream, 1, std::forward<Args>(args)...);
+}
 
 // ----------------------------------------------------------------- tensor maps
 // 3-D bf16 tensor map {inner, rows, batch} with 128-byte swizzle; strides in
@@ -53,10 +89,9 @@ struct LactLaunch {
 };
 // Workspace layout (byte offsets) for a given problem.
 struct LactWorkspace {
-  size_t status, w1b, w3b, w2b, dh1, dh3, gm, aq, part, cnt, rowss, nsx32, nsxb, nsa32, nsab,
-      nsbb, total;
+  size_t status, w1b, w3b, w2b, d13, gm, aq, part, rowss, nsx32, nsxb, nsa32, nsab, nsbb, total;
   // split operands (hi + lo bf16): residual copies
-  size_t w1lo, w3lo, w2lo, dh1lo, dh3lo, gmlo, aqlo, nsxlo, nsalo, nsblo;
+  size_t w1lo, w3lo, w2lo, d13lo, gmlo, aqlo, nsxlo, nsalo, nsblo;
   int cmax;                // rows of the per-chunk intermediates
   int splits;              // split-K factor of the gradient GEMMs
 };

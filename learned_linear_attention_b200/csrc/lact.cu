@@ -17,6 +17,7 @@
 // Bidirectional order: steps 1 (keys only), 3, 4 for every chunk, then the
 // queries run step 1 (queries only) and step 2 with the final weights.
 #include <algorithm>
+#include <mutex>
 
 #include "gemm.cuh"
 #include "kernels.h"
@@ -37,6 +38,8 @@ constexpr int STAGES = 3;
 constexpr uint32_t BAR_OFF = STAGES * STAGE;
 constexpr uint32_t SMEM = BAR_OFF + 256 + 1024;
 constexpr uint32_t ACC_COLS = 256;                   // [H1 64 | H3 64 | dG 64 | pad]
+constexpr int EPI_WARPS = 8;                         // two per TMEM lane quadrant
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
 }  // namespace kp
 
 struct KeyPassArgs {
@@ -49,12 +52,13 @@ struct KeyPassArgs {
   int dh;
   int lr_len;       // row length of lr ([BH][lr_len])
   const float* lr;
-  __nv_bfloat16 *dH1, *dH3, *Gm, *Aq;   // [BH][cmax][dh]
+  // dH1 | dH3 side by side in D13 [BH][cmax][2*dh]; Gm', Aq [BH][cmax][dh]
+  __nv_bfloat16 *D13, *Gm, *Aq;
   // split operands: W = W_hi + W_lo (the K loop runs twice) and the
   // intermediates are written as hi and lo bf16 parts
   int split;
-  __nv_bfloat16 *dH1lo, *dH3lo, *Gmlo, *Aqlo;
-  long long inter_bs;
+  __nv_bfloat16 *D13lo, *Gmlo, *Aqlo;
+  long long inter_bs;      // cmax * dh (Gm', Aq); D13 uses twice that
   DevStatus st;
 };
 
@@ -68,8 +72,16 @@ TTT_DEVICE_INLINE __nv_bfloat16 bf16_residual(float x, __nv_bfloat16 h) {
 }
 
 TTT_DEVICE_INLINE float sigmoidf_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// sigma(x) = 1/2 + tanh(x/2)/2 with the hardware tanh approximation (one
+// MUFU op, max relative error about 2^-11): used when the outputs are
+// rounded to bf16 anyway.
+TTT_DEVICE_INLINE float sigmoidf_tanh(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
+}
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kp::THREADS, 1)
     lact_keypass_kernel(const __grid_constant__ KeyPassMaps maps, const KeyPassArgs a) {
   using namespace kp;
   extern __shared__ uint8_t smem_raw[];
@@ -94,7 +106,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&afull[s], 1);
-      mbar_init(&aempty[s], 128);
+      mbar_init(&aempty[s], EPI_WARPS * 32);
     }
     mbar_init(fin, 1);
     *abort_flag = 0;
@@ -115,6 +127,8 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   Waiter W{abort_flag, a.st, 200};
 
@@ -206,7 +220,10 @@ __global__ void __launch_bounds__(192, 1)
       W.drain(fin, 0);
     }
   } else {
+    // epilogue: warps 2..9; quadrant q4 = TMEM lanes, column group cg = 32
+    // of the tile's 64 hidden units, processed as two 16-column halves
     const int q4 = warp & 3;
+    const int cg = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     uint32_t lt = 0;
@@ -217,58 +234,72 @@ __global__ void __launch_bounds__(192, 1)
       const int tc = (is_key ? tt : tt - a.n_key_tiles) * BM + r;   // row within the pass
       const bool valid = tc < a.C;
       const uint32_t ab = lt & 1;
+      // the learning rate is fetched before waiting for the accumulator
+      const float eta = (is_key && valid) ? a.lr[(size_t)bh * a.lr_len + a.t0 + tc] : 0.f;
       if (!W.wait(&afull[ab], (lt >> 1) & 1, 4)) break;
       tc_fence_after();
       const uint32_t base = tmem + lane_base + ab * ACC_COLS;
       const size_t obase = (size_t)bh * a.inter_bs + (size_t)tc * a.dh + hb * HB;
-      const float eta = (is_key && valid) ? a.lr[(size_t)bh * a.lr_len + a.t0 + tc] : 0.f;
+      const size_t dbase = 2 * ((size_t)bh * a.inter_bs + (size_t)tc * a.dh) + hb * HB;
 #pragma unroll 1
-      for (int jc = 0; jc < HB; jc += 32) {
-        float h1[32], h3[32];
-        tmem_ld32(base + jc, h1);
-        tmem_ld32(base + 64 + jc, h3);
+      for (int half = 0; half < 2; ++half) {
+        const int jc = cg * 32 + half * 16;
+        uint32_t rh1[16], rh3[16], rg[16];
+        tmem_ld16_issue(base + jc, rh1);
+        tmem_ld16_issue(base + 64 + jc, rh3);
+        if (is_key) tmem_ld16_issue(base + 128 + jc, rg);
+        tmem_wait_ld();
+        float h1[16], h3[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          h1[j] = __uint_as_float(rh1[j]);
+          h3[j] = __uint_as_float(rh3[j]);
+        }
         if (is_key) {
-          float g[32];
-          tmem_ld32(base + 128 + jc, g);
+          float g[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) g[j] = __uint_as_float(rg[j]);
           if (valid) {
-            uint32_t o1[16], o3[16], om[16], l1[16], l3[16], lm[16];
+            uint32_t o1[8], o3[8], om[8];
+            float r1[16], r3[16], rm[16];
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              float r1[2], r3[2], rm[2];
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const float x = h1[j + u], y = h3[j + u];
-                const float sg = sigmoidf_fast(x);
-                const float act = x * sg;
-                const float dg = -eta * g[j + u];
-                r3[u] = dg * act;
-                r1[u] = dg * y * (sg * (1.f + x * (1.f - sg)));
-                rm[u] = -eta * act * y;
-              }
-              o1[j >> 1] = pack_bf16x2(r1[0], r1[1]);
-              o3[j >> 1] = pack_bf16x2(r3[0], r3[1]);
-              om[j >> 1] = pack_bf16x2(rm[0], rm[1]);
-              if (a.split) {
-                l1[j >> 1] = pack_bf16x2(r1[0] - bf16lo(o1[j >> 1]), r1[1] - bf16hi(o1[j >> 1]));
-                l3[j >> 1] = pack_bf16x2(r3[0] - bf16lo(o3[j >> 1]), r3[1] - bf16hi(o3[j >> 1]));
-                lm[j >> 1] = pack_bf16x2(rm[0] - bf16lo(om[j >> 1]), rm[1] - bf16hi(om[j >> 1]));
-              }
+            for (int j = 0; j < 16; ++j) {
+              const float x = h1[j], y = h3[j];
+              const float sg = a.split ? sigmoidf_fast(x) : sigmoidf_tanh(x);
+              const float act = x * sg;
+              const float dg = -eta * g[j];
+              r3[j] = dg * act;
+              r1[j] = dg * y * (sg * (1.f + x * (1.f - sg)));
+              rm[j] = -eta * act * y;
             }
-            uint4* d1 = reinterpret_cast<uint4*>(a.dH1 + obase + jc);
-            uint4* d3 = reinterpret_cast<uint4*>(a.dH3 + obase + jc);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              o1[j] = pack_bf16x2(r1[2 * j], r1[2 * j + 1]);
+              o3[j] = pack_bf16x2(r3[2 * j], r3[2 * j + 1]);
+              om[j] = pack_bf16x2(rm[2 * j], rm[2 * j + 1]);
+            }
+            uint4* d1 = reinterpret_cast<uint4*>(a.D13 + dbase + jc);
+            uint4* d3 = reinterpret_cast<uint4*>(a.D13 + dbase + a.dh + jc);
             uint4* dm = reinterpret_cast<uint4*>(a.Gm + obase + jc);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
               d1[j] = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
               d3[j] = make_uint4(o3[4 * j], o3[4 * j + 1], o3[4 * j + 2], o3[4 * j + 3]);
               dm[j] = make_uint4(om[4 * j], om[4 * j + 1], om[4 * j + 2], om[4 * j + 3]);
             }
             if (a.split) {
-              uint4* e1 = reinterpret_cast<uint4*>(a.dH1lo + obase + jc);
-              uint4* e3 = reinterpret_cast<uint4*>(a.dH3lo + obase + jc);
+              uint32_t l1[8], l3[8], lm[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                l1[j] = pack_bf16x2(r1[2 * j] - bf16lo(o1[j]), r1[2 * j + 1] - bf16hi(o1[j]));
+                l3[j] = pack_bf16x2(r3[2 * j] - bf16lo(o3[j]), r3[2 * j + 1] - bf16hi(o3[j]));
+                lm[j] = pack_bf16x2(rm[2 * j] - bf16lo(om[j]), rm[2 * j + 1] - bf16hi(om[j]));
+              }
+              uint4* e1 = reinterpret_cast<uint4*>(a.D13lo + dbase + jc);
+              uint4* e3 = reinterpret_cast<uint4*>(a.D13lo + dbase + a.dh + jc);
               uint4* em = reinterpret_cast<uint4*>(a.Gmlo + obase + jc);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
+              for (int j = 0; j < 2; ++j) {
                 e1[j] = make_uint4(l1[4 * j], l1[4 * j + 1], l1[4 * j + 2], l1[4 * j + 3]);
                 e3[j] = make_uint4(l3[4 * j], l3[4 * j + 1], l3[4 * j + 2], l3[4 * j + 3]);
                 em[j] = make_uint4(lm[4 * j], lm[4 * j + 1], lm[4 * j + 2], lm[4 * j + 3]);
@@ -276,22 +307,25 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         } else if (valid) {
-          uint32_t oq[16], lq[16];
+          float aq[16];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float a0 = h1[j] * sigmoidf_fast(h1[j]) * h3[j];
-            const float a1 = h1[j + 1] * sigmoidf_fast(h1[j + 1]) * h3[j + 1];
-            oq[j >> 1] = pack_bf16x2(a0, a1);
-            if (a.split) lq[j >> 1] = pack_bf16x2(a0 - bf16lo(oq[j >> 1]), a1 - bf16hi(oq[j >> 1]));
-          }
+          for (int j = 0; j < 16; ++j)
+            aq[j] = h1[j] * (a.split ? sigmoidf_fast(h1[j]) : sigmoidf_tanh(h1[j])) * h3[j];
+          uint32_t oq[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) oq[j] = pack_bf16x2(aq[2 * j], aq[2 * j + 1]);
           uint4* dq = reinterpret_cast<uint4*>(a.Aq + obase + jc);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < 2; ++j)
             dq[j] = make_uint4(oq[4 * j], oq[4 * j + 1], oq[4 * j + 2], oq[4 * j + 3]);
           if (a.split) {
+            uint32_t lq[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              lq[j] = pack_bf16x2(aq[2 * j] - bf16lo(oq[j]), aq[2 * j + 1] - bf16hi(oq[j]));
             uint4* eq = reinterpret_cast<uint4*>(a.Aqlo + obase + jc);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
               eq[j] = make_uint4(lq[4 * j], lq[4 * j + 1], lq[4 * j + 2], lq[4 * j + 3]);
           }
         }
@@ -347,6 +381,8 @@ TTT_DEVICE_INLINE float warp_sum(float x) {
 
 // bf16 operand copies of all three matrices.
 __global__ void lact_cast_kernel(RowArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (gw >= a.BH * (2 * a.dh + a.d)) return;
   int mat, bh, row, rows, cols;
@@ -389,6 +425,8 @@ TTT_DEVICE_INLINE void sum_partials(const RowArgs& a, int mat, size_t off, size_
 
 // GD / momentum: sum the split-K partials, update, normalise the row.
 __global__ void __launch_bounds__(ROW_THREADS) lact_update_kernel(RowArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float red[4];
   int mat, bh, row, rows, cols;
   row_decode(a, blockIdx.x, mat, bh, row, rows, cols);
@@ -428,6 +466,8 @@ __global__ void __launch_bounds__(ROW_THREADS) lact_update_kernel(RowArgs a) {
 
 // Muon step 1: M = beta M + G, and the row sums of squares of M.
 __global__ void __launch_bounds__(ROW_THREADS) muon_momentum_kernel(RowArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float red[4];
   int mat, bh, row, rows, cols;
   row_decode(a, blockIdx.x, mat, bh, row, rows, cols);
@@ -462,6 +502,8 @@ struct NsPrepArgs {
   __nv_bfloat16* Xlo;      // residual (split operands; nullable)
 };
 __global__ void ns_prep_kernel(NsPrepArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int mb = blockIdx.y;                 // mat * BH + bh
   const int mat = mb / a.BH, bh = mb % a.BH;
   const int rows = mat < 2 ? a.dh : a.d, cols = mat < 2 ? a.d : a.dh;
@@ -491,6 +533,8 @@ __global__ void ns_prep_kernel(NsPrepArgs a) {
 
 // Muon step 4: W -= NS(M) (orientation restored), normalise the row.
 __global__ void muon_apply_kernel(RowArgs a, int r, int c) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (gw >= a.BH * (2 * a.dh + a.d)) return;
   int mat, bh, row, rows, cols;
@@ -542,6 +586,31 @@ static int num_sms() {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Helper streams (per device, created once) on which the independent GEMMs
+// of a chunk run concurrently; fork/join with events keeps every call
+// ordered on the caller's stream.
+struct SideStreams {
+  cudaStream_t s[3] = {nullptr, nullptr, nullptr};
+  cudaEvent_t fork = nullptr, join[3] = {nullptr, nullptr, nullptr};
+  bool ok = false;
+};
+static SideStreams* side_streams() {
+  static SideStreams per_dev[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  SideStreams& x = per_dev[dev];
+  if (!x.ok) {
+    bool good = cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < 3 && good; ++i)
+      good = cudaStreamCreateWithFlags(&x.s[i], cudaStreamNonBlocking) == cudaSuccess &&
+             cudaEventCreateWithFlags(&x.join[i], cudaEventDisableTiming) == cudaSuccess;
+    x.ok = good;
+  }
+  return x.ok ? &x : nullptr;
+}
+
 static int grad_splits(int BH, int d, int dh, int cmax) {
   const int tiles = BH * 3 * (dh / 128) * (d / 128);
   const int ksteps = (cmax + 63) / 64;
@@ -564,12 +633,10 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
   w.w1b = o; o = align256(o + BH * dh * d * 2);
   w.w3b = o; o = align256(o + BH * dh * d * 2);
   w.w2b = o; o = align256(o + BH * d * dh * 2);
-  w.dh1 = o; o = align256(o + BH * cmax * dh * 2);
-  w.dh3 = o; o = align256(o + BH * cmax * dh * 2);
+  w.d13 = o; o = align256(o + BH * cmax * 2 * dh * 2);
   w.gm = o; o = align256(o + BH * cmax * dh * 2);
   w.aq = o; o = align256(o + BH * cmax * dh * 2);
   w.part = o; o = align256(o + (size_t)w.splits * BH * 3 * d * dh * 4);
-  w.cnt = o; o = align256(o + BH * 3 * ((std::max(d, dh) + 127) / 128) * sizeof(int));
   w.rowss = w.nsx32 = w.nsxb = w.nsa32 = w.nsab = w.nsbb = o;
   if (opt == 2) {
     const size_t r = std::min(d, dh), c = std::max(d, dh);
@@ -580,13 +647,12 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
     w.nsab = o; o = align256(o + 3 * BH * r * r * 2);
     w.nsbb = o; o = align256(o + 3 * BH * r * r * 2);
   }
-  w.w1lo = w.w3lo = w.w2lo = w.dh1lo = w.dh3lo = w.gmlo = w.aqlo = w.nsxlo = w.nsalo = w.nsblo = o;
+  w.w1lo = w.w3lo = w.w2lo = w.d13lo = w.gmlo = w.aqlo = w.nsxlo = w.nsalo = w.nsblo = o;
   if (split) {
     w.w1lo = o; o = align256(o + BH * dh * d * 2);
     w.w3lo = o; o = align256(o + BH * dh * d * 2);
     w.w2lo = o; o = align256(o + BH * d * dh * 2);
-    w.dh1lo = o; o = align256(o + BH * cmax * dh * 2);
-    w.dh3lo = o; o = align256(o + BH * cmax * dh * 2);
+    w.d13lo = o; o = align256(o + BH * cmax * 2 * dh * 2);
     w.gmlo = o; o = align256(o + BH * cmax * dh * 2);
     w.aqlo = o; o = align256(o + BH * cmax * dh * 2);
     if (opt == 2) {
@@ -612,9 +678,13 @@ static int run_gemm(const GemmMaps& maps, const GemmArgs& g, cudaStream_t stream
   }
   const int tiles = ((g.M + 127) / 128) * (g.N / BN) * g.splits * g.batch;
   if (tiles <= 0) return 0;
-  const int grid = std::min(tiles, num_sms());
+  // cluster mode: one tile per CTA, N tiles of a row block in one cluster
+  const int cl = g.cluster_n > 1 ? g.cluster_n : 1;
+  if (cl > 1 && (g.N / BN != cl || g.splits != 1)) return -1;
+  const int grid = cl > 1 ? tiles : std::min(tiles, num_sms());
   prof_before(kind, stream);
-  kfn<<<grid, 192, smem, stream>>>(maps, g);
+  if (launch_pdl_cluster(kfn, dim3(grid), dim3(192), smem, stream, cl, maps, g) != cudaSuccess)
+    return -1;
   prof_after(kind, stream);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
@@ -641,11 +711,10 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   uint8_t* ws = L.ws;
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
   __nv_bfloat16 *w1b = bf(w.w1b), *w3b = bf(w.w3b), *w2b = bf(w.w2b);
-  __nv_bfloat16 *dH1 = bf(w.dh1), *dH3 = bf(w.dh3), *Gm = bf(w.gm), *Aq = bf(w.aq);
+  __nv_bfloat16 *D13 = bf(w.d13), *Gm = bf(w.gm), *Aq = bf(w.aq);
   __nv_bfloat16 *w1lo = split ? bf(w.w1lo) : nullptr, *w3lo = split ? bf(w.w3lo) : nullptr,
                 *w2lo = split ? bf(w.w2lo) : nullptr;
-  __nv_bfloat16 *dH1lo = split ? bf(w.dh1lo) : nullptr, *dH3lo = split ? bf(w.dh3lo) : nullptr,
-                *Gmlo = split ? bf(w.gmlo) : nullptr, *Aqlo = split ? bf(w.aqlo) : nullptr;
+  __nv_bfloat16 *D13lo = split ? bf(w.d13lo) : nullptr, *Gmlo = split ? bf(w.gmlo) : nullptr, *Aqlo = split ? bf(w.aqlo) : nullptr;
   float* part = reinterpret_cast<float*>(ws + w.part);
   const size_t mat_elems = (size_t)BH * d * dh;
   float* W1 = L.state;
@@ -672,7 +741,8 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   const int row_blocks = (row_warps * 32 + 255) / 256;
 
   prof_before(K_LACT_CAST, stream);
-  lact_cast_kernel<<<row_blocks, 256, 0, stream>>>(ra);
+  if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
+    return -1;
   prof_after(K_LACT_CAST, stream);
   TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
 
@@ -736,18 +806,20 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     KeyPassArgs a{};
     a.C = C; a.t0 = t0; a.n_key_tiles = nkt; a.n_q_tiles = nqt; a.n_hb = dh / 64; a.BH = BH;
     a.d_steps = d / 64; a.dh = dh; a.lr_len = L.N_in; a.lr = L.lr;
-    a.dH1 = dH1; a.dH3 = dH3; a.Gm = Gm; a.Aq = Aq;
-    a.split = split ? 1 : 0; a.dH1lo = dH1lo; a.dH3lo = dH3lo; a.Gmlo = Gmlo; a.Aqlo = Aqlo;
+    a.D13 = D13; a.Gm = Gm; a.Aq = Aq;
+    a.split = split ? 1 : 0; a.D13lo = D13lo; a.Gmlo = Gmlo; a.Aqlo = Aqlo;
     a.inter_bs = (long long)w.cmax * dh; a.st = L.st;
     const int tiles = (nkt + nqt) * a.n_hb * BH;
     if (tiles <= 0) return 0;
     prof_before(K_KEYPASS, stream);
-    lact_keypass_kernel<<<std::min(tiles, num_sms()), 192, kp::SMEM, stream>>>(km, a);
+    if (launch_pdl(lact_keypass_kernel, dim3(std::min(tiles, num_sms())), dim3(kp::THREADS),
+                   kp::SMEM, stream, km, a) != cudaSuccess)
+      return -1;
     prof_after(K_KEYPASS, stream);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   };
   // out rows [t0, t0 + C) = Aq W2^T (split: hi*hi + hi*lo + lo*hi)
-  auto read_out = [&](int t0, int C) -> int {
+  auto read_out = [&](int t0, int C, cudaStream_t rstream) -> int {
     GemmArgs g = gemm_defaults(L.st);
     g.M = C; g.N = d; g.batch = BH; g.k_steps = dh / 64;
     g.out_row_off = t0;
@@ -771,67 +843,92 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       TTT_TRY(inter_map(&m.a[2], Aqlo, C, 128));
       m.b[2] = mw2k;
     }
-    return run_gemm<128, false, false, 4>(m, g, stream, K_GEMM_READ);
+    return run_gemm<128, false, false, 4>(m, g, rstream, K_GEMM_READ);
   };
   // Chunk gradients G1 = dH1^T K, G3 = dH3^T K (rows = hidden units, N = d)
-  // and G2 = V^T Gm' (rows = d, N = dh); split-K over the chunk's tokens.
-  // fused: the epilogue of the last split also applies GD / momentum and the
-  // row normalisation (whole rows fit one N tile); otherwise partial sums
-  // go to the update kernels.
-  const bool fused_update = L.opt != 2 && (d == 128 || d == 256) && (dh == 128 || dh == 256);
-  int* counters = reinterpret_cast<int*>(ws + w.cnt);
-  const int cnt_stride = BH * ((std::max(d, dh) + 127) / 128);
-  if (fused_update && cudaMemsetAsync(counters, 0, 3 * cnt_stride * sizeof(int), stream) != cudaSuccess)
-    return -1;
-  auto gradients = [&](int t0, int C, bool fused) -> int {
-    CUtensorMap mi[3], mil[3];
-    __nv_bfloat16* hi[3] = {dH1, dH3, Gm};
-    __nv_bfloat16* lo[3] = {dH1lo, dH3lo, Gmlo};
-    for (int i = 0; i < 3; ++i) {
-      TTT_TRY(inter_map(&mi[i], hi[i], C, 64));
-      if (split) TTT_TRY(inter_map(&mil[i], lo[i], C, 64));
+  // and G2 = V^T Gm' (rows = d, N = dh), contracted over the chunk's tokens.
+  // fused (GD / momentum, d in {128, 256}, dh <= 256, chunk <= 8192): one
+  // launch for [G1; G3] (stacked rows of D13^T) and one for G2 (N tiles of
+  // a W2 row block in one cluster), each with the weight update, row
+  // normalisation and bf16 copies in the epilogue.  Otherwise split-K
+  // partial sums go to the row update kernels.
+  const int cmax_chunk = std::min(L.chunk, std::max(L.N_in, 1));
+  const bool fused_update = L.opt != 2 && (d == 128 || d == 256) && (dh == 128 || dh == 256) &&
+                            cmax_chunk <= 8192;
+  auto d13_map = [&](CUtensorMap* m, const void* p, int rows) {
+    return make_tmap_bf16_3d(m, p, 2 * dh, rows, BH, (uint64_t)dh * 4, (uint64_t)w.cmax * dh * 4,
+                             64, 64);
+  };
+  auto gradients = [&](int t0, int C, cudaStream_t* mstream) -> int {
+    CUtensorMap md, mdl, mg, mgl;
+    TTT_TRY(d13_map(&md, D13, C));
+    TTT_TRY(inter_map(&mg, Gm, C, 64));
+    if (split) {
+      TTT_TRY(d13_map(&mdl, D13lo, C));
+      TTT_TRY(inter_map(&mgl, Gmlo, C, 64));
     }
     const int ksteps_total = (C + 63) / 64;
+    const int np = split ? 2 : 1;
+    if (fused_update) {
+      GemmArgs g = gemm_defaults(L.st);
+      g.batch = BH; g.splits = 1; g.k_steps = ksteps_total; g.npairs = np; g.epi = 1;
+      g.mom_beta = L.beta; g.norm_eps = L.norm_eps; g.normalize = L.normalize_rows;
+      GemmMaps m{};
+      // [G1; G3]: rows 0..dh-1 update W1, rows dh..2dh-1 update W3
+      if ((L.update_mask & 3) != 0) {
+        GemmArgs g13 = g;
+        g13.M = 2 * dh; g13.N = d; g13.ldw = d; g13.rows_first = dh;
+        g13.W[0] = W1; g13.W[1] = W3; g13.Mom[0] = M1; g13.Mom[1] = M3;
+        g13.Wb[0] = w1b; g13.Wb[1] = w3b; g13.Wlo[0] = w1lo; g13.Wlo[1] = w3lo;
+        if ((L.update_mask & 3) == 2) { g13.a_m_off[0] = g13.a_m_off[1] = dh; g13.M = dh; g13.rows_first = 0; }
+        if ((L.update_mask & 3) == 1) { g13.M = dh; }
+        for (int p = 0; p < np; ++p) {
+          m.a[p] = p == 0 ? md : mdl;
+          m.b[p] = mk_mn;
+          g13.b_k_off[p] = t0;
+        }
+        if (d == 128) TTT_TRY(run_gemm<128, true, true, 4>(m, g13, mstream[0], K_GEMM_GRAD));
+        else TTT_TRY(run_gemm<256, true, true, 3>(m, g13, mstream[0], K_GEMM_GRAD));
+      }
+      if (L.update_mask & 4) {
+        GemmArgs g2 = g;
+        g2.M = d; g2.N = dh; g2.ldw = dh; g2.rows_first = d; g2.cluster_n = dh / 128;
+        g2.W[0] = W2; g2.Mom[0] = M2; g2.Wb[0] = w2b; g2.Wlo[0] = w2lo;
+        for (int p = 0; p < np; ++p) {
+          m.a[p] = mv_mn;
+          m.b[p] = p == 0 ? mg : mgl;
+          g2.a_k_off[p] = t0;
+          g2.b_k_off[p] = 0;
+        }
+        TTT_TRY(run_gemm<128, true, true, 4>(m, g2, mstream[1], K_GEMM_GRAD));
+      }
+      return 1;
+    }
     const int splits = std::min(w.splits, ksteps_total);
     const int kps = (ksteps_total + splits - 1) / splits;
     GemmArgs g = gemm_defaults(L.st);
-    g.batch = BH; g.splits = splits; g.k_steps = kps;
-    g.npairs = split ? 2 : 1;
-    if (fused) {
-      g.epi = 1;
-      g.mom_beta = L.beta; g.norm_eps = L.norm_eps; g.normalize = L.normalize_rows;
-    } else {
-      g.o32_ss = (long long)BH * d * dh;
-      g.o32_bs = (long long)d * dh;
-    }
+    g.batch = BH; g.splits = splits; g.k_steps = kps; g.npairs = np;
+    g.o32_ss = (long long)BH * d * dh;
+    g.o32_bs = (long long)d * dh;
     for (int mat = 0; mat < 3; ++mat) {
-      if (fused && !(L.update_mask & (1 << mat))) continue;
       GemmMaps m{};
       if (mat < 2) {
         g.M = dh; g.N = d; g.ld32 = d;
-        for (int p = 0; p < g.npairs; ++p) {
-          m.a[p] = p == 0 ? mi[mat] : mil[mat];
+        for (int p = 0; p < np; ++p) {
+          m.a[p] = p == 0 ? md : mdl;
           m.b[p] = mk_mn;
-          g.a_k_off[p] = 0; g.b_k_off[p] = t0;
+          g.a_m_off[p] = mat * dh; g.a_k_off[p] = 0; g.b_k_off[p] = t0;
         }
       } else {
         g.M = d; g.N = dh; g.ld32 = dh;
-        for (int p = 0; p < g.npairs; ++p) {
+        for (int p = 0; p < np; ++p) {
           m.a[p] = mv_mn;
-          m.b[p] = p == 0 ? mi[2] : mil[2];
-          g.a_k_off[p] = t0; g.b_k_off[p] = 0;
+          m.b[p] = p == 0 ? mg : mgl;
+          g.a_m_off[p] = 0; g.a_k_off[p] = t0; g.b_k_off[p] = 0;
         }
       }
-      if (fused) {
-        g.W = ra.W[mat]; g.Mom = ra.M[mat]; g.Wb = ra.Wb[mat]; g.Wlo = ra.Wlo[mat];
-        g.part = const_cast<float*>(ra.part[mat]);
-        g.counters = counters + mat * cnt_stride;
-        if (g.N == 128) TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
-        else TTT_TRY(run_gemm<256, true, true, 3>(m, g, stream, K_GEMM_GRAD));
-      } else {
-        g.o32 = const_cast<float*>(ra.part[mat]);
-        TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
-      }
+      g.o32 = const_cast<float*>(ra.part[mat]);
+      TTT_TRY(run_gemm<128, true, true, 4>(m, g, mstream[mat], K_GEMM_GRAD));
     }
     return splits;
   };
@@ -847,14 +944,17 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     __nv_bfloat16 *Ab = bf(w.nsab), *Bb = bf(w.nsbb);
     __nv_bfloat16 *Al = split ? bf(w.nsalo) : nullptr, *Bl = split ? bf(w.nsblo) : nullptr;
     prof_before(K_MUON_MOM, stream);
-    muon_momentum_kernel<<<row_warps, ROW_THREADS, 0, stream>>>(ra);
+    if (launch_pdl(muon_momentum_kernel, dim3(row_warps), dim3(ROW_THREADS), 0, stream, ra) !=
+        cudaSuccess)
+      return -1;
     prof_after(K_MUON_MOM, stream);
     NsPrepArgs pa{};
     pa.BH = BH; pa.d = d; pa.dh = dh; pa.r = r; pa.c = c; pa.eps = L.ns_eps;
     pa.M[0] = M1; pa.M[1] = M3; pa.M[2] = M2; pa.rowss = ra.rowss; pa.X32 = X32;
     pa.Xb = Xb[0]; pa.Xlo = Xl[0];
     prof_before(K_NS_PREP, stream);
-    ns_prep_kernel<<<dim3(r, nb), 256, 0, stream>>>(pa);
+    if (launch_pdl(ns_prep_kernel, dim3(r, nb), dim3(256), 0, stream, pa) != cudaSuccess)
+      return -1;
     prof_after(K_NS_PREP, stream);
     TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     auto sq_map = [&](CUtensorMap* m, const void* p) {
@@ -914,33 +1014,60 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       TTT_TRY(run_gemm<128, false, true, 4>(m, g, stream, K_GEMM_NS));
     }
     prof_before(K_MUON_APPLY, stream);
-    muon_apply_kernel<<<row_blocks, 256, 0, stream>>>(ra, r, c);
+    if (launch_pdl(muon_apply_kernel, dim3(row_blocks), dim3(256), 0, stream, ra, r, c) !=
+        cudaSuccess)
+      return -1;
     prof_after(K_MUON_APPLY, stream);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   };
 
   // ------------------------------------------------------------ chunk loop
+  // Per chunk: key pass; then the memory read and the three gradient GEMMs,
+  // which are independent, run concurrently on the caller's stream and the
+  // helper streams; then (unfused path) the update.
+  SideStreams* ss = side_streams();
+  cudaStream_t gstream[3] = {stream, ss ? ss->s[0] : stream, ss ? ss->s[1] : stream};
+  cudaStream_t rstream = ss ? ss->s[2] : stream;
+  auto fork = [&]() -> int {
+    if (!ss) return 0;
+    if (cudaEventRecord(ss->fork, stream) != cudaSuccess) return -1;
+    for (int i = 0; i < 3; ++i)
+      if (cudaStreamWaitEvent(ss->s[i], ss->fork, 0) != cudaSuccess) return -1;
+    return 0;
+  };
+  auto join = [&]() -> int {
+    if (!ss) return 0;
+    for (int i = 0; i < 3; ++i)
+      if (cudaEventRecord(ss->join[i], ss->s[i]) != cudaSuccess ||
+          cudaStreamWaitEvent(stream, ss->join[i], 0) != cudaSuccess)
+        return -1;
+    return 0;
+  };
   for (int t0 = 0; t0 < L.N_in; t0 += L.chunk) {
     const int C = std::min(L.chunk, L.N_in - t0);
     const int nt = (C + 127) / 128;
     TTT_TRY(key_pass(t0, C, nt, L.causal ? nt : 0));
-    if (L.causal) TTT_TRY(read_out(t0, C));
-    const int splits = gradients(t0, C, fused_update);
+    TTT_TRY(fork());
+    if (L.causal) TTT_TRY(read_out(t0, C, rstream));
+    const int splits = gradients(t0, C, gstream);
     if (splits < 0) return -1;
+    TTT_TRY(join());
     if (fused_update) continue;
     ra.splits = splits;
     if (L.opt == 2) {
       TTT_TRY(muon());
     } else {
       prof_before(K_UPDATE, stream);
-      lact_update_kernel<<<row_warps, ROW_THREADS, 0, stream>>>(ra);
+      if (launch_pdl(lact_update_kernel, dim3(row_warps), dim3(ROW_THREADS), 0, stream, ra) !=
+          cudaSuccess)
+        return -1;
       prof_after(K_UPDATE, stream);
       TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     }
   }
   if (!L.causal && L.N_q > 0) {
     TTT_TRY(key_pass(0, L.N_q, 0, (L.N_q + 127) / 128));
-    TTT_TRY(read_out(0, L.N_q));
+    TTT_TRY(read_out(0, L.N_q, stream));
   }
   return 0;
 }
