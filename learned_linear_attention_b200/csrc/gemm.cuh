@@ -326,14 +326,16 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * L::STAGE);
           const uint32_t sb = sa + L::A_BYTES;
+          // descriptors of the stage; the four K=16 slices advance the start
+          // address field (16-byte units) by 32 B (K-major) or 2 KB (MN-major)
+          const uint64_t ad0 = A_MN ? make_sdesc(sa, 8192, 1024) : make_sdesc(sa, 16, 1024);
+          const uint64_t bd0 = B_MN ? make_sdesc(sb, 8192, 1024) : make_sdesc(sb, 16, 1024);
+          constexpr uint64_t ASTEP = A_MN ? (2048 >> 4) : (32 >> 4);
+          constexpr uint64_t BSTEP = B_MN ? (2048 >> 4) : (32 >> 4);
+          mma_bf16(d, ad0, bd0, idesc, kk != 0);
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const uint64_t ad = A_MN ? make_sdesc(sa + k4 * 2048, 8192, 1024)
-                                     : make_sdesc(sa + k4 * 32, 16, 1024);
-            const uint64_t bd = B_MN ? make_sdesc(sb + k4 * 2048, 8192, 1024)
-                                     : make_sdesc(sb + k4 * 32, 16, 1024);
-            mma_bf16(d, ad, bd, idesc, (kk | k4) != 0);
-          }
+          for (int k4 = 1; k4 < 4; ++k4)
+            mma_bf16(d, ad0 + k4 * ASTEP, bd0 + k4 * BSTEP, idesc, 1u);
           mma_commit(&empty[s]);
         }
         if (!ok) break;

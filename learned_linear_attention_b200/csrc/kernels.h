@@ -99,10 +99,22 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
                                     int causal, int opt, int split);
 int launch_lact(const LactLaunch& L, cudaStream_t stream);
 
+// Fused key pass + chunk gradient (head dim 128): partial sums per token group.
+struct KeyGradLaunch {
+  int BH, N_in, C, t0, dh, groups;
+  const void *k, *v;
+  const float* lr;
+  const void *w1b, *w3b, *w2b;
+  float* part[3];
+  DevStatus st;
+};
+int keygrad_groups(int BH, int dh, int C, int max_groups);
+int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream);
+
 // ----------------------------------------------------------------- profiling
 enum KernelKind {
   K_LIN_SIMT, K_LIN_UMMA, K_LACT_CAST, K_KEYPASS, K_GEMM_READ, K_GEMM_GRAD, K_UPDATE,
-  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_NUM
+  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_NUM
 };
 void prof_before(int kind, cudaStream_t s);
 void prof_after(int kind, cudaStream_t s);

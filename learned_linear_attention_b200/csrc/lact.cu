@@ -423,43 +423,67 @@ TTT_DEVICE_INLINE void sum_partials(const RowArgs& a, int mat, size_t off, size_
   }
 }
 
-// GD / momentum: sum the split-K partials, update, normalise the row.
-__global__ void __launch_bounds__(ROW_THREADS) lact_update_kernel(RowArgs a) {
+// GD / momentum: sum the split-K partials, update, normalise the row.  One
+// warp per row, lanes own 4 consecutive columns per 128-column chunk (16-byte
+// loads; every partial sum of a chunk is in flight at once).
+constexpr int UPD_ROWS_PER_BLOCK = 8;
+__global__ void __launch_bounds__(UPD_ROWS_PER_BLOCK * 32) lact_update_kernel(RowArgs a) {
   pdl_wait();
   pdl_launch_dependents();
-  __shared__ float red[4];
+  const int gw = blockIdx.x * UPD_ROWS_PER_BLOCK + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (gw >= a.BH * (2 * a.dh + a.d)) return;
   int mat, bh, row, rows, cols;
-  row_decode(a, blockIdx.x, mat, bh, row, rows, cols);
+  row_decode(a, gw, mat, bh, row, rows, cols);
   if (!(a.mask & (1 << mat))) return;
   const size_t off = ((size_t)bh * rows + row) * cols;
   const size_t split_stride = (size_t)a.BH * rows * cols;
-  float w[ROW_PER_THREAD];
-  sum_partials(a, mat, off, split_stride, cols, w);
-  float ss = 0.f;
+  const int nch = cols >> 7;                        // 128-column chunks (cols % 128 == 0)
+  float4 w[8];
 #pragma unroll
-  for (int i = 0; i < ROW_PER_THREAD; ++i) {
-    const int c = threadIdx.x + ROW_THREADS * i;
-    if (c < cols) {
-      float u = w[i];
-      if (a.opt == 1) {
-        u = a.beta * a.M[mat][off + c] + u;
-        a.M[mat][off + c] = u;
+  for (int i = 0; i < 8; ++i) w[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < a.splits; ++s) {
+    const float4* p = reinterpret_cast<const float4*>(a.part[mat] + s * split_stride + off) + lane;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i < nch) {
+        const float4 x = __ldcg(p + 32 * i);
+        w[i].x += x.x; w[i].y += x.y; w[i].z += x.z; w[i].w += x.w;
       }
-      w[i] = a.W[mat][off + c] - u;
-      ss += w[i] * w[i];
+    }
+  }
+  float ss = 0.f;
+  float4* Wr = reinterpret_cast<float4*>(a.W[mat] + off) + lane;
+  float4* Mr = a.opt == 1 ? reinterpret_cast<float4*>(a.M[mat] + off) + lane : nullptr;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i < nch) {
+      float4 u = w[i];
+      if (Mr != nullptr) {
+        float4 m = Mr[32 * i];
+        m.x = a.beta * m.x + u.x; m.y = a.beta * m.y + u.y;
+        m.z = a.beta * m.z + u.z; m.w = a.beta * m.w + u.w;
+        Mr[32 * i] = m;
+        u = m;
+      }
+      const float4 x = Wr[32 * i];
+      w[i] = make_float4(x.x - u.x, x.y - u.y, x.z - u.z, x.w - u.w);
+      ss += w[i].x * w[i].x + w[i].y * w[i].y + w[i].z * w[i].z + w[i].w * w[i].w;
     }
   }
   float scale = 1.f;
-  if (a.normalize) scale = 1.f / fmaxf(sqrtf(block_sum128(ss, red)), a.norm_eps);
+  if (a.normalize) scale = 1.f / fmaxf(sqrtf(warp_sum(ss)), a.norm_eps);
+  uint2* Br = reinterpret_cast<uint2*>(a.Wb[mat] + off) + lane;
+  uint2* Lr = a.Wlo[mat] != nullptr ? reinterpret_cast<uint2*>(a.Wlo[mat] + off) + lane : nullptr;
 #pragma unroll
-  for (int i = 0; i < ROW_PER_THREAD; ++i) {
-    const int c = threadIdx.x + ROW_THREADS * i;
-    if (c < cols) {
-      const float x = w[i] * scale;
-      const __nv_bfloat16 h = __float2bfloat16_rn(x);
-      a.W[mat][off + c] = x;
-      a.Wb[mat][off + c] = h;
-      if (a.Wlo[mat] != nullptr) a.Wlo[mat][off + c] = bf16_residual(x, h);
+  for (int i = 0; i < 8; ++i) {
+    if (i < nch) {
+      const float4 x = make_float4(w[i].x * scale, w[i].y * scale, w[i].z * scale, w[i].w * scale);
+      Wr[32 * i] = x;
+      const uint32_t h0 = pack_bf16x2(x.x, x.y), h1 = pack_bf16x2(x.z, x.w);
+      Br[32 * i] = make_uint2(h0, h1);
+      if (Lr != nullptr)
+        Lr[32 * i] = make_uint2(pack_bf16x2(x.x - bf16lo(h0), x.y - bf16hi(h0)),
+                                pack_bf16x2(x.z - bf16lo(h1), x.w - bf16hi(h1)));
     }
   }
 }
@@ -591,7 +615,7 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // ordered on the caller's stream.
 struct SideStreams {
   cudaStream_t s[3] = {nullptr, nullptr, nullptr};
-  cudaEvent_t fork = nullptr, join[3] = {nullptr, nullptr, nullptr};
+  cudaEvent_t fork = nullptr, join[3] = {nullptr, nullptr, nullptr}, read_done[2] = {nullptr, nullptr};
   bool ok = false;
 };
 static SideStreams* side_streams() {
@@ -602,7 +626,9 @@ static SideStreams* side_streams() {
   std::lock_guard<std::mutex> lk(mu);
   SideStreams& x = per_dev[dev];
   if (!x.ok) {
-    bool good = cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess;
+    bool good = cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess &&
+                cudaEventCreateWithFlags(&x.read_done[0], cudaEventDisableTiming) == cudaSuccess &&
+                cudaEventCreateWithFlags(&x.read_done[1], cudaEventDisableTiming) == cudaSuccess;
     for (int i = 0; i < 3 && good; ++i)
       good = cudaStreamCreateWithFlags(&x.s[i], cudaStreamNonBlocking) == cudaSuccess &&
              cudaEventCreateWithFlags(&x.join[i], cudaEventDisableTiming) == cudaSuccess;
@@ -628,11 +654,14 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
   cmax = (cmax + 127) / 128 * 128;
   w.cmax = cmax;
   w.splits = grad_splits((int)BH, d, dh, cin);
+  if (d == 128 && dh % 64 == 0) w.splits = std::max(w.splits, keygrad_groups((int)BH, dh, cin, 0));
   size_t o = 0;
   w.status = o; o = align256(o + 256);
-  w.w1b = o; o = align256(o + BH * dh * d * 2);
-  w.w3b = o; o = align256(o + BH * dh * d * 2);
-  w.w2b = o; o = align256(o + BH * d * dh * 2);
+  // bf16 operand copies, two buffers (chunk c reads buffer c&1 while its
+  // update writes the other one)
+  w.w1b = o; o = align256(o + 2 * BH * dh * d * 2);
+  w.w3b = o; o = align256(o + 2 * BH * dh * d * 2);
+  w.w2b = o; o = align256(o + 2 * BH * d * dh * 2);
   w.d13 = o; o = align256(o + BH * cmax * 2 * dh * 2);
   w.gm = o; o = align256(o + BH * cmax * dh * 2);
   w.aq = o; o = align256(o + BH * cmax * dh * 2);
@@ -649,9 +678,9 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
   }
   w.w1lo = w.w3lo = w.w2lo = w.d13lo = w.gmlo = w.aqlo = w.nsxlo = w.nsalo = w.nsblo = o;
   if (split) {
-    w.w1lo = o; o = align256(o + BH * dh * d * 2);
-    w.w3lo = o; o = align256(o + BH * dh * d * 2);
-    w.w2lo = o; o = align256(o + BH * d * dh * 2);
+    w.w1lo = o; o = align256(o + 2 * BH * dh * d * 2);
+    w.w3lo = o; o = align256(o + 2 * BH * dh * d * 2);
+    w.w2lo = o; o = align256(o + 2 * BH * d * dh * 2);
     w.d13lo = o; o = align256(o + BH * cmax * 2 * dh * 2);
     w.gmlo = o; o = align256(o + BH * cmax * dh * 2);
     w.aqlo = o; o = align256(o + BH * cmax * dh * 2);
@@ -710,10 +739,18 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt, L.split);
   uint8_t* ws = L.ws;
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
-  __nv_bfloat16 *w1b = bf(w.w1b), *w3b = bf(w.w3b), *w2b = bf(w.w2b);
+  const size_t wsz = (size_t)BH * d * dh;
+  __nv_bfloat16* wbuf[2][3];
+  __nv_bfloat16* lbuf[2][3];
+  for (int b = 0; b < 2; ++b) {
+    wbuf[b][0] = bf(w.w1b) + b * wsz;
+    wbuf[b][1] = bf(w.w3b) + b * wsz;
+    wbuf[b][2] = bf(w.w2b) + b * wsz;
+    lbuf[b][0] = split ? bf(w.w1lo) + b * wsz : nullptr;
+    lbuf[b][1] = split ? bf(w.w3lo) + b * wsz : nullptr;
+    lbuf[b][2] = split ? bf(w.w2lo) + b * wsz : nullptr;
+  }
   __nv_bfloat16 *D13 = bf(w.d13), *Gm = bf(w.gm), *Aq = bf(w.aq);
-  __nv_bfloat16 *w1lo = split ? bf(w.w1lo) : nullptr, *w3lo = split ? bf(w.w3lo) : nullptr,
-                *w2lo = split ? bf(w.w2lo) : nullptr;
   __nv_bfloat16 *D13lo = split ? bf(w.d13lo) : nullptr, *Gmlo = split ? bf(w.gmlo) : nullptr, *Aqlo = split ? bf(w.aqlo) : nullptr;
   float* part = reinterpret_cast<float*>(ws + w.part);
   const size_t mat_elems = (size_t)BH * d * dh;
@@ -730,8 +767,12 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   ra.norm_eps = L.norm_eps; ra.ns_eps = L.ns_eps;
   ra.W[0] = W1; ra.W[1] = W3; ra.W[2] = W2;
   ra.M[0] = M1; ra.M[1] = M3; ra.M[2] = M2;
-  ra.Wb[0] = w1b; ra.Wb[1] = w3b; ra.Wb[2] = w2b;
-  ra.Wlo[0] = w1lo; ra.Wlo[1] = w3lo; ra.Wlo[2] = w2lo;
+  auto set_out_buf = [&](int b) {
+    for (int i = 0; i < 3; ++i) {
+      ra.Wb[i] = wbuf[b][i];
+      ra.Wlo[i] = lbuf[b][i];
+    }
+  };
   ra.part[0] = part;
   ra.part[1] = part + (size_t)w.splits * mat_elems;
   ra.part[2] = part + 2 * (size_t)w.splits * mat_elems;
@@ -740,10 +781,15 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   const int row_warps = BH * (2 * dh + d);
   const int row_blocks = (row_warps * 32 + 255) / 256;
 
-  prof_before(K_LACT_CAST, stream);
-  if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
-    return -1;
-  prof_after(K_LACT_CAST, stream);
+  // both buffers start from the state (matrices excluded by update_mask are
+  // never rewritten and must read the same in either buffer)
+  for (int b = 0; b < 2; ++b) {
+    set_out_buf(b);
+    prof_before(K_LACT_CAST, stream);
+    if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
+      return -1;
+    prof_after(K_LACT_CAST, stream);
+  }
   TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
 
   // ---- tensor maps.  Token tensors {d, rows, BH}; K-major boxes {64, 128},
@@ -775,19 +821,24 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   if (q_rows > 0) TTT_TRY(tok_map(&km.q, L.q, q_rows, 128));
   else km.q = km.k;
   if (L.N_in == 0) { km.k = km.q; km.v = km.q; }
-  TTT_TRY(w13_map(&km.w1, w1b));
-  TTT_TRY(w13_map(&km.w3, w3b));
-  TTT_TRY(w2_mn_map(&km.w2, w2b));
-  if (split) {
-    TTT_TRY(w13_map(&km.w1lo, w1lo));
-    TTT_TRY(w13_map(&km.w3lo, w3lo));
-    TTT_TRY(w2_mn_map(&km.w2lo, w2lo));
-  } else {
-    km.w1lo = km.w1; km.w3lo = km.w3; km.w2lo = km.w2;
+  KeyPassMaps kmb[2] = {km, km};
+  CUtensorMap mw2k[2], mw2klo[2];
+  for (int b = 0; b < 2; ++b) {
+    TTT_TRY(w13_map(&kmb[b].w1, wbuf[b][0]));
+    TTT_TRY(w13_map(&kmb[b].w3, wbuf[b][1]));
+    TTT_TRY(w2_mn_map(&kmb[b].w2, wbuf[b][2]));
+    TTT_TRY(w2_k_map(&mw2k[b], wbuf[b][2]));
+    if (split) {
+      TTT_TRY(w13_map(&kmb[b].w1lo, lbuf[b][0]));
+      TTT_TRY(w13_map(&kmb[b].w3lo, lbuf[b][1]));
+      TTT_TRY(w2_mn_map(&kmb[b].w2lo, lbuf[b][2]));
+      TTT_TRY(w2_k_map(&mw2klo[b], lbuf[b][2]));
+    } else {
+      kmb[b].w1lo = kmb[b].w1; kmb[b].w3lo = kmb[b].w3; kmb[b].w2lo = kmb[b].w2;
+      mw2klo[b] = mw2k[b];
+    }
   }
-  CUtensorMap mw2k, mw2klo;
-  TTT_TRY(w2_k_map(&mw2k, w2b));
-  if (split) TTT_TRY(w2_k_map(&mw2klo, w2lo));
+  int cur = 0;   // buffer holding the chunk-start weights
   CUtensorMap mk_mn{}, mv_mn{};   // token tensors as MN-major operands
   if (L.N_in > 0) {
     TTT_TRY(tok_map(&mk_mn, L.k, L.N_in, 64));
@@ -802,7 +853,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     kp_attr = true;
   }
 
-  auto key_pass = [&](int t0, int C, int nkt, int nqt) -> int {
+  auto key_pass_on = [&](int t0, int C, int nkt, int nqt, cudaStream_t kstream) -> int {
     KeyPassArgs a{};
     a.C = C; a.t0 = t0; a.n_key_tiles = nkt; a.n_q_tiles = nqt; a.n_hb = dh / 64; a.BH = BH;
     a.d_steps = d / 64; a.dh = dh; a.lr_len = L.N_in; a.lr = L.lr;
@@ -811,12 +862,15 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     a.inter_bs = (long long)w.cmax * dh; a.st = L.st;
     const int tiles = (nkt + nqt) * a.n_hb * BH;
     if (tiles <= 0) return 0;
-    prof_before(K_KEYPASS, stream);
+    prof_before(K_KEYPASS, kstream);
     if (launch_pdl(lact_keypass_kernel, dim3(std::min(tiles, num_sms())), dim3(kp::THREADS),
-                   kp::SMEM, stream, km, a) != cudaSuccess)
+                   kp::SMEM, kstream, kmb[cur], a) != cudaSuccess)
       return -1;
-    prof_after(K_KEYPASS, stream);
+    prof_after(K_KEYPASS, kstream);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  };
+  auto key_pass = [&](int t0, int C, int nkt, int nqt) -> int {
+    return key_pass_on(t0, C, nkt, nqt, stream);
   };
   // out rows [t0, t0 + C) = Aq W2^T (split: hi*hi + hi*lo + lo*hi)
   auto read_out = [&](int t0, int C, cudaStream_t rstream) -> int {
@@ -835,13 +889,13 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     }
     GemmMaps m{};
     TTT_TRY(inter_map(&m.a[0], Aq, C, 128));
-    m.b[0] = mw2k;
+    m.b[0] = mw2k[cur];
     if (split) {
       g.npairs = 3;
       m.a[1] = m.a[0];
-      m.b[1] = mw2klo;
+      m.b[1] = mw2klo[cur];
       TTT_TRY(inter_map(&m.a[2], Aqlo, C, 128));
-      m.b[2] = mw2k;
+      m.b[2] = mw2k[cur];
     }
     return run_gemm<128, false, false, 4>(m, g, rstream, K_GEMM_READ);
   };
@@ -879,7 +933,8 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
         GemmArgs g13 = g;
         g13.M = 2 * dh; g13.N = d; g13.ldw = d; g13.rows_first = dh;
         g13.W[0] = W1; g13.W[1] = W3; g13.Mom[0] = M1; g13.Mom[1] = M3;
-        g13.Wb[0] = w1b; g13.Wb[1] = w3b; g13.Wlo[0] = w1lo; g13.Wlo[1] = w3lo;
+        g13.Wb[0] = wbuf[cur ^ 1][0]; g13.Wb[1] = wbuf[cur ^ 1][1];
+        g13.Wlo[0] = lbuf[cur ^ 1][0]; g13.Wlo[1] = lbuf[cur ^ 1][1];
         if ((L.update_mask & 3) == 2) { g13.a_m_off[0] = g13.a_m_off[1] = dh; g13.M = dh; g13.rows_first = 0; }
         if ((L.update_mask & 3) == 1) { g13.M = dh; }
         for (int p = 0; p < np; ++p) {
@@ -887,20 +942,20 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
           m.b[p] = mk_mn;
           g13.b_k_off[p] = t0;
         }
-        if (d == 128) TTT_TRY(run_gemm<128, true, true, 4>(m, g13, mstream[0], K_GEMM_GRAD));
-        else TTT_TRY(run_gemm<256, true, true, 3>(m, g13, mstream[0], K_GEMM_GRAD));
+        if (d == 128) TTT_TRY(run_gemm<128, true, true, 6>(m, g13, mstream[0], K_GEMM_GRAD));
+        else TTT_TRY(run_gemm<256, true, true, 4>(m, g13, mstream[0], K_GEMM_GRAD));
       }
       if (L.update_mask & 4) {
         GemmArgs g2 = g;
         g2.M = d; g2.N = dh; g2.ldw = dh; g2.rows_first = d; g2.cluster_n = dh / 128;
-        g2.W[0] = W2; g2.Mom[0] = M2; g2.Wb[0] = w2b; g2.Wlo[0] = w2lo;
+        g2.W[0] = W2; g2.Mom[0] = M2; g2.Wb[0] = wbuf[cur ^ 1][2]; g2.Wlo[0] = lbuf[cur ^ 1][2];
         for (int p = 0; p < np; ++p) {
           m.a[p] = mv_mn;
           m.b[p] = p == 0 ? mg : mgl;
           g2.a_k_off[p] = t0;
           g2.b_k_off[p] = 0;
         }
-        TTT_TRY(run_gemm<128, true, true, 4>(m, g2, mstream[1], K_GEMM_GRAD));
+        TTT_TRY(run_gemm<128, true, true, 6>(m, g2, mstream[1], K_GEMM_GRAD));
       }
       return 1;
     }
@@ -1043,7 +1098,51 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
         return -1;
     return 0;
   };
-  for (int t0 = 0; t0 < L.N_in; t0 += L.chunk) {
+  // head dim 128 without split operands: the key pass and the gradient
+  // contraction run fused (partial sums per token group), the queries and
+  // the read run concurrently on a helper stream.
+  const bool keygrad = d == 128 && !split && L.opt != 2;
+  // Chunk c: the helper stream runs the queries and the read of chunk c on
+  // the chunk-start weights (buffer cur) while the caller's stream runs the
+  // fused key/gradient kernel; the update of chunk c writes buffer cur^1,
+  // which the read of chunk c-1 used, so it waits only for that read.
+  int ci = 0;
+  for (int t0 = 0; keygrad && t0 < L.N_in; t0 += L.chunk, ++ci) {
+    const int C = std::min(L.chunk, L.N_in - t0);
+    const int nt = (C + 127) / 128;
+    if (L.causal) {
+      if (ss) {
+        TTT_TRY(cudaEventRecord(ss->fork, stream) == cudaSuccess ? 0 : -1);
+        TTT_TRY(cudaStreamWaitEvent(rstream, ss->fork, 0) == cudaSuccess ? 0 : -1);
+      }
+      TTT_TRY(key_pass_on(t0, C, 0, nt, rstream));
+      TTT_TRY(read_out(t0, C, rstream));
+      if (ss) TTT_TRY(cudaEventRecord(ss->read_done[ci & 1], rstream) == cudaSuccess ? 0 : -1);
+    }
+    KeyGradLaunch kgl{};
+    kgl.BH = BH; kgl.N_in = L.N_in; kgl.C = C; kgl.t0 = t0; kgl.dh = dh;
+    kgl.groups = keygrad_groups(BH, dh, C, w.splits);
+    kgl.k = L.k; kgl.v = L.v; kgl.lr = L.lr;
+    kgl.w1b = wbuf[cur][0]; kgl.w3b = wbuf[cur][1]; kgl.w2b = wbuf[cur][2];
+    kgl.part[0] = const_cast<float*>(ra.part[0]);
+    kgl.part[1] = const_cast<float*>(ra.part[1]);
+    kgl.part[2] = const_cast<float*>(ra.part[2]);
+    kgl.st = L.st;
+    TTT_TRY(launch_lact_keygrad(kgl, stream));
+    if (L.causal && ss && ci >= 1)
+      TTT_TRY(cudaStreamWaitEvent(stream, ss->read_done[(ci - 1) & 1], 0) == cudaSuccess ? 0 : -1);
+    ra.splits = kgl.groups;
+    set_out_buf(cur ^ 1);
+    prof_before(K_UPDATE, stream);
+    if (launch_pdl(lact_update_kernel, dim3((row_warps + UPD_ROWS_PER_BLOCK - 1) / UPD_ROWS_PER_BLOCK),
+                   dim3(UPD_ROWS_PER_BLOCK * 32), 0, stream, ra) != cudaSuccess)
+      return -1;
+    prof_after(K_UPDATE, stream);
+    cur ^= 1;
+  }
+  if (keygrad && L.causal && ss && ci >= 1)   // the last read joins the caller's stream
+    TTT_TRY(cudaStreamWaitEvent(stream, ss->read_done[(ci - 1) & 1], 0) == cudaSuccess ? 0 : -1);
+  for (int t0 = 0; !keygrad && t0 < L.N_in; t0 += L.chunk) {
     const int C = std::min(L.chunk, L.N_in - t0);
     const int nt = (C + 127) / 128;
     TTT_TRY(key_pass(t0, C, nt, L.causal ? nt : 0));
@@ -1052,18 +1151,23 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     const int splits = gradients(t0, C, gstream);
     if (splits < 0) return -1;
     TTT_TRY(join());
-    if (fused_update) continue;
+    if (fused_update) {   // the epilogues wrote buffer cur^1
+      cur ^= 1;
+      continue;
+    }
     ra.splits = splits;
+    set_out_buf(cur ^ 1);
     if (L.opt == 2) {
       TTT_TRY(muon());
     } else {
       prof_before(K_UPDATE, stream);
-      if (launch_pdl(lact_update_kernel, dim3(row_warps), dim3(ROW_THREADS), 0, stream, ra) !=
-          cudaSuccess)
+      if (launch_pdl(lact_update_kernel, dim3((row_warps + UPD_ROWS_PER_BLOCK - 1) / UPD_ROWS_PER_BLOCK),
+                     dim3(UPD_ROWS_PER_BLOCK * 32), 0, stream, ra) != cudaSuccess)
         return -1;
       prof_after(K_UPDATE, stream);
       TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     }
+    cur ^= 1;
   }
   if (!L.causal && L.N_q > 0) {
     TTT_TRY(key_pass(0, L.N_q, 0, (L.N_q + 127) / 128));

@@ -1,0 +1,385 @@
+// lact_keygrad.cu -- fused key pass + chunk gradient for head dim d = 128
+// ("Test-Time Training Done Right" review, "Memoria no lineal y atención
+// local": the chunk's lr-weighted gradients of -<f_W(k), v> are summed at
+// the chunk-start weights).
+//
+// One work item = (head, 64 hidden units J, a group of token tiles of the
+// chunk).  For every 128-token tile of the group:
+//   MMA   H13 = K [W1_J; W3_J]^T   (128 x 128),   dGr = V W2[:, J]  (128 x 64)
+//   epi   dG = -eta dGr, dH3 = dG silu(H1), dH1 = dG H3 silu'(H1),
+//         Gm' = -eta silu(H1) H3           -> bf16 operands in shared memory
+//   MMA   G1_J^T += K^T dH1, G3_J^T += K^T dH3, G2[:, J] += V^T Gm'
+// with the K and V tiles reused from shared memory (as MN-major operands)
+// and the three gradient accumulators resident in TMEM across the group.
+// At the end of the item the partial gradients are stored (plain stores,
+// one slot per token group) and the row update kernel sums the groups in a
+// fixed order.  Nothing of the chunk's intermediates goes to global memory.
+#include <algorithm>
+
+#include "kernels.h"
+
+namespace ttt {
+namespace kg {
+constexpr int D = 128, HB = 64, BM = 128;
+constexpr uint32_t HALF = BM * 64 * 2;                 // 16 KB: 128 rows x 64 bf16
+constexpr uint32_t TILE = 2 * HALF;                    // 32 KB: 128 tokens x 128 d
+constexpr uint32_t OFF_KV = 0;                         // 2 stages x (K tile | V tile)
+constexpr uint32_t KV_STAGE = 2 * TILE;                // 64 KB
+constexpr uint32_t OFF_W13 = 2 * KV_STAGE;             // [W1_J | W3_J] x d: two K atoms
+constexpr uint32_t OFF_W2 = OFF_W13 + 2 * HALF;        // W2[:, J]: 128 d-rows x 64 hidden
+constexpr uint32_t OFF_DH = OFF_W2 + 2 * 8192;         // dH1 | dH3 | Gm' (16 KB each)
+constexpr uint32_t OFF_BAR = OFF_DH + 3 * HALF;
+constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
+// TMEM columns
+constexpr uint32_t TM_H13 = 0, TM_DG = 128, TM_G1 = 256, TM_G3 = 320, TM_G2 = 384, TM_COLS = 512;
+}  // namespace kg
+
+struct KeyGradArgs {
+  int BH, C, t0, lr_len, dh;
+  int n_hb, n_groups, tiles_total, tiles_per_group;
+  const float* lr;
+  float* part[3];        // [group][BH][rows][cols] partial gradients (G1, G3, G2)
+  int split;             // exact sigmoid (split-operand mode) instead of tanh.approx
+  DevStatus st;
+};
+struct KeyGradMaps {
+  CUtensorMap k, v, w1, w3, w2;
+};
+
+TTT_DEVICE_INLINE float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+TTT_DEVICE_INLINE float sigmoid_tanh(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
+}
+
+__global__ void __launch_bounds__(kg::THREADS, 1)
+    lact_keygrad_kernel(const __grid_constant__ KeyGradMaps maps, const KeyGradArgs a) {
+  using namespace kg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* kv_full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);   // [2]
+  uint64_t* kv_empty = kv_full + 2;                                   // [2]
+  uint64_t* w_full = kv_empty + 2;
+  uint64_t* w_empty = w_full + 1;
+  uint64_t* acc_full = w_empty + 1;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* dh_ready = acc_empty + 1;
+  uint64_t* dh_free = dh_ready + 1;
+  uint64_t* g_full = dh_free + 1;
+  uint64_t* g_empty = g_full + 1;
+  uint64_t* fin = g_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int items_per_bh = a.n_hb * a.n_groups;
+  const int n_items = items_per_bh * a.BH;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(w_full, 1);
+    mbar_init(w_empty, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, EPI_WARPS * 32);
+    mbar_init(dh_ready, EPI_WARPS * 32);
+    mbar_init(dh_free, 1);
+    mbar_init(g_full, 1);
+    mbar_init(g_empty, EPI_WARPS * 32);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.k);
+    tma_prefetch_desc(&maps.v);
+    tma_prefetch_desc(&maps.w1);
+    tma_prefetch_desc(&maps.w3);
+    tma_prefetch_desc(&maps.w2);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  pdl_launch_dependents();
+  const uint32_t tmem = *tmem_slot;
+  Waiter W{abort_flag, a.st, 300};
+
+  auto decode = [&](int item, int& bh, int& hb, int& grp) {
+    hb = item % a.n_hb;
+    grp = (item / a.n_hb) % a.n_groups;
+    bh = item / items_per_bh;
+  };
+  auto group_tiles = [&](int grp) {
+    const int first = grp * a.tiles_per_group;
+    return std::max(0, std::min(a.tiles_per_group, a.tiles_total - first));
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      uint32_t tile = 0, item_ctr = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++item_ctr) {
+        int bh, hb, grp;
+        decode(item, bh, hb, grp);
+        const int j0 = hb * HB;
+        const int nt = group_tiles(grp);
+        if (item_ctr >= 1 && !W.wait(w_empty, (item_ctr - 1) & 1, 1)) { ok = false; break; }
+        // weights of the item: [W1_J; W3_J] as two K atoms (d 0-63, 64-127),
+        // W2[:, J] as 128 d-rows of 64 hidden units (and the lo copies)
+        mbar_arrive_expect_tx(w_full, 2 * HALF + 2 * 8192);
+        {
+          const CUtensorMap* m1 = &maps.w1;
+          const CUtensorMap* m3 = &maps.w3;
+          const CUtensorMap* m2 = &maps.w2;
+          for (int atom = 0; atom < 2; ++atom) {
+            tma_load_3d(smem + OFF_W13 + atom * HALF, m1, w_full, atom * 64, j0, bh);
+            tma_load_3d(smem + OFF_W13 + atom * HALF + HALF / 2, m3, w_full, atom * 64, j0, bh);
+            tma_load_3d(smem + OFF_W2 + atom * 8192, m2, w_full, j0, atom * 64, bh);
+          }
+        }
+        for (int i = 0; i < nt; ++i, ++tile) {
+          const uint32_t s = tile & 1;
+          if (tile >= 2 && !W.wait(&kv_empty[s], ((tile >> 1) - 1) & 1, 2)) { ok = false; break; }
+          const int row = a.t0 + (grp * a.tiles_per_group + i) * BM;
+          uint8_t* st = smem + OFF_KV + s * KV_STAGE;
+          mbar_arrive_expect_tx(&kv_full[s], KV_STAGE);
+          tma_load_3d(st, &maps.k, &kv_full[s], 0, row, bh);
+          tma_load_3d(st + HALF, &maps.k, &kv_full[s], 64, row, bh);
+          tma_load_3d(st + TILE, &maps.v, &kv_full[s], 0, row, bh);
+          tma_load_3d(st + TILE + HALF, &maps.v, &kv_full[s], 64, row, bh);
+        }
+      }
+      if (W.aborted()) {
+        const uint32_t first = tile > 2 ? tile - 2 : 0;
+        for (uint32_t i = first; i < tile; ++i) W.drain(&kv_full[i & 1], (i >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id_h = make_idesc(128, 128, false, false);
+      const uint32_t id_g = make_idesc(128, 64, false, true);
+      const uint32_t id_grad = make_idesc(128, 64, true, true);
+      const uint32_t kvb = smem_u32(smem + OFF_KV);
+      const uint32_t w13 = smem_u32(smem + OFF_W13), w2 = smem_u32(smem + OFF_W2);
+      const uint32_t dhb = smem_u32(smem + OFF_DH);
+      uint32_t tile = 0, item_ctr = 0;
+      bool ok = true;
+      auto grads = [&](uint32_t t, bool first, uint32_t item_c) -> bool {
+        if (first && item_c >= 1 && !W.wait(g_empty, (item_c - 1) & 1, 3)) return false;
+        if (!W.wait(dh_ready, t & 1, 4)) return false;
+        tc_fence_after();
+        const uint32_t kt = kvb + (t & 1) * KV_STAGE, vt = kt + TILE;
+        // K^T / V^T as MN-major A: M = d in two 64-wide blocks 16 KB apart,
+        // K = tokens (rows of 128 B); dH / Gm' as MN-major B: N = 64 hidden
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+          const uint64_t ka = make_sdesc(kt + kk * 2048, HALF, 1024);
+          const uint64_t va = make_sdesc(vt + kk * 2048, HALF, 1024);
+          mma_bf16(tmem + TM_G1, ka, make_sdesc(dhb + kk * 2048, 8192, 1024), id_grad, acc);
+          mma_bf16(tmem + TM_G3, ka, make_sdesc(dhb + HALF + kk * 2048, 8192, 1024), id_grad, acc);
+          mma_bf16(tmem + TM_G2, va, make_sdesc(dhb + 2 * HALF + kk * 2048, 8192, 1024), id_grad, acc);
+        }
+        mma_commit(dh_free);
+        mma_commit(&kv_empty[t & 1]);
+        return true;
+      };
+      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++item_ctr) {
+        int bh, hb, grp;
+        decode(item, bh, hb, grp);
+        const int nt = group_tiles(grp);
+        if (!W.wait(w_full, item_ctr & 1, 5)) { ok = false; break; }
+        const uint32_t base = tile;
+        for (int i = 0; i < nt; ++i, ++tile) {
+          const uint32_t s = tile & 1;
+          if (!W.wait(&kv_full[s], (tile >> 1) & 1, 6)) { ok = false; break; }
+          if (tile >= 1 && !W.wait(acc_empty, (tile - 1) & 1, 7)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kt = kvb + s * KV_STAGE, vt = kt + TILE;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t atom = kk >> 2, ko = (kk & 3) * 32;
+            mma_bf16(tmem + TM_H13, make_sdesc(kt + atom * HALF + ko, 16, 1024),
+                     make_sdesc(w13 + atom * HALF + ko, 16, 1024), id_h, kk > 0);
+            mma_bf16(tmem + TM_DG, make_sdesc(vt + atom * HALF + ko, 16, 1024),
+                     make_sdesc(w2 + kk * 2048, 8192, 1024), id_g, kk > 0);
+          }
+          mma_commit(acc_full);
+          if (i >= 1 && !grads(tile - 1, i - 1 == 0, item_ctr)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (nt > 0 && !grads(base + nt - 1, nt == 1, item_ctr)) { ok = false; break; }
+        mma_commit(g_full);
+        mma_commit(w_empty);
+      }
+      mma_commit(fin);
+      W.drain(fin, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;
+    const int cg = (warp - 2) >> 2;                 // 32-column group of the 64 hidden
+    const int r = q4 * 32 + lane;                   // token row of the tile / d row of G
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    uint8_t* dh1s = smem + OFF_DH;
+    const uint32_t dh1 = smem_u32(dh1s), dh3 = dh1 + HALF, gms = dh1 + 2 * HALF;
+    uint32_t tile = 0, item_ctr = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
+      int bh, hb, grp;
+      decode(item, bh, hb, grp);
+      const int nt = group_tiles(grp);
+      bool ok = true;
+      for (int i = 0; i < nt; ++i, ++tile) {
+        const int tc = (grp * a.tiles_per_group + i) * BM + r;   // token row in the chunk
+        const bool valid = tc < a.C;
+        const float eta = valid ? a.lr[(size_t)bh * a.lr_len + a.t0 + tc] : 0.f;
+        if (!W.wait(acc_full, tile & 1, 8)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t rh1[32], rh3[32], rg[32];
+        const uint32_t tb = tmem + lane_base + cg * 32;
+        tmem_ld16_issue(tb + TM_H13, rh1);
+        tmem_ld16_issue(tb + TM_H13 + 16, rh1 + 16);
+        tmem_ld16_issue(tb + TM_H13 + 64, rh3);
+        tmem_ld16_issue(tb + TM_H13 + 80, rh3 + 16);
+        tmem_ld16_issue(tb + TM_DG, rg);
+        tmem_ld16_issue(tb + TM_DG + 16, rg + 16);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(acc_empty);
+        uint32_t o1[16], o3[16], om[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          float r1[2], r3[2], rm[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const float x = __uint_as_float(rh1[j + u]), y = __uint_as_float(rh3[j + u]);
+            const float sg = a.split ? sigmoid_fast(x) : sigmoid_tanh(x);
+            const float act = x * sg;
+            const float dg = valid ? -eta * __uint_as_float(rg[j + u]) : 0.f;
+            r3[u] = dg * act;
+            r1[u] = dg * y * (sg * (1.f + x * (1.f - sg)));
+            rm[u] = valid ? -eta * act * y : 0.f;
+          }
+          o1[j >> 1] = pack_bf16x2(r1[0], r1[1]);
+          o3[j >> 1] = pack_bf16x2(r3[0], r3[1]);
+          om[j >> 1] = pack_bf16x2(rm[0], rm[1]);
+        }
+        // the previous tile's gradient MMAs must be done reading dH
+        if (tile >= 1 && !W.wait(dh_free, (tile - 1) & 1, 9)) { ok = false; break; }
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          const uint32_t off = sw128_offset(r, cg * 32 + j);
+          st_shared_v4(dh1 + off, o1[j / 2], o1[j / 2 + 1], o1[j / 2 + 2], o1[j / 2 + 3]);
+          st_shared_v4(dh3 + off, o3[j / 2], o3[j / 2 + 1], o3[j / 2 + 2], o3[j / 2 + 3]);
+          st_shared_v4(gms + off, om[j / 2], om[j / 2 + 1], om[j / 2 + 2], om[j / 2 + 3]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(dh_ready);
+      }
+      if (!ok) break;
+      if (nt == 0) continue;
+      // item done: partial gradients -> their token-group slot
+      if (!W.wait(g_full, item_ctr & 1, 10)) break;
+      tc_fence_after();
+      const int j0 = hb * HB + cg * 32;
+      const size_t mat_stride = (size_t)a.BH * a.dh * D;
+      const size_t slot = (size_t)grp * mat_stride;
+      float g1[32], g3[32], g2[32];
+      tmem_ld32(tmem + lane_base + TM_G1 + cg * 32, g1);
+      tmem_ld32(tmem + lane_base + TM_G3 + cg * 32, g3);
+      tmem_ld32(tmem + lane_base + TM_G2 + cg * 32, g2);
+      tc_fence_before();
+      mbar_arrive(g_empty);
+      // G1, G3 [BH][dh][d]: this thread is d row r -> element (j0 + j, r)
+      float* p1 = a.part[0] + slot + ((size_t)bh * a.dh + j0) * D + r;
+      float* p3 = a.part[1] + slot + ((size_t)bh * a.dh + j0) * D + r;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        p1[(size_t)j * D] = g1[j];
+        p3[(size_t)j * D] = g3[j];
+      }
+      // G2 [BH][d][dh]: row r, columns j0 .. j0 + 31
+      float4* p2 = reinterpret_cast<float4*>(a.part[2] + slot + ((size_t)bh * D + r) * a.dh + j0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) p2[j] = make_float4(g2[4 * j], g2[4 * j + 1], g2[4 * j + 2], g2[4 * j + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
+// Token groups per chunk: enough items (BH x dh/64 x groups) to fill the
+// SMs, and never an empty group (every slot of the partial sums is written).
+int keygrad_groups(int BH, int dh, int C, int max_groups) {
+  const int n_hb = dh / kg::HB;
+  const int tiles = std::max(1, (C + kg::BM - 1) / kg::BM);
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  int g = std::max(1, std::min(sms / std::max(1, BH * n_hb), tiles));
+  if (max_groups > 0) g = std::min(g, max_groups);
+  const int tpg = (tiles + g - 1) / g;
+  return (tiles + tpg - 1) / tpg;
+}
+
+int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream) {
+  KeyGradMaps m{};
+  const uint64_t BH = (uint64_t)L.BH;
+  const uint64_t tok_row = (uint64_t)kg::D * 2;
+  if (make_tmap_bf16_3d(&m.k, L.k, kg::D, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 128) ||
+      make_tmap_bf16_3d(&m.v, L.v, kg::D, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 128) ||
+      make_tmap_bf16_3d(&m.w1, L.w1b, kg::D, L.dh, BH, tok_row, tok_row * L.dh, 64, 64) ||
+      make_tmap_bf16_3d(&m.w3, L.w3b, kg::D, L.dh, BH, tok_row, tok_row * L.dh, 64, 64) ||
+      make_tmap_bf16_3d(&m.w2, L.w2b, L.dh, kg::D, BH, (uint64_t)L.dh * 2, (uint64_t)L.dh * 2 * kg::D,
+                        64, 64))
+    return -1;
+  KeyGradArgs a{};
+  a.BH = L.BH; a.C = L.C; a.t0 = L.t0; a.lr_len = L.N_in; a.dh = L.dh;
+  a.n_hb = L.dh / kg::HB;
+  a.tiles_total = (L.C + kg::BM - 1) / kg::BM;
+  a.n_groups = L.groups;
+  a.tiles_per_group = (a.tiles_total + a.n_groups - 1) / a.n_groups;
+  if ((a.n_groups - 1) * a.tiles_per_group >= a.tiles_total) return -1;   // empty group
+  a.lr = L.lr;
+  a.part[0] = L.part[0]; a.part[1] = L.part[1]; a.part[2] = L.part[2];
+  a.split = 0;
+  a.st = L.st;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(lact_keygrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kg::SMEM) != cudaSuccess)
+      return -1;
+    attr = true;
+  }
+  const int items = a.n_hb * a.n_groups * L.BH;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  prof_before(K_KEYGRAD, stream);
+  if (launch_pdl(lact_keygrad_kernel, dim3(std::min(items, sms)), dim3(kg::THREADS), kg::SMEM, stream,
+                 m, a) != cudaSuccess)
+    return -1;
+  prof_after(K_KEYGRAD, stream);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace ttt

@@ -155,3 +155,11 @@ def test_cuda_graph_replay_matches_eager(cuda_device):
     g.replay()
     torch.cuda.synchronize()
     assert np.array_equal(run.out.cpu().numpy(), eager)
+
+
+def test_causal_many_chunks_multi_tile_groups(cuda_device):
+    """Chunks of 1024 tokens over 8 heads: every fused key/gradient work item
+    covers several token tiles, and the read of each chunk runs beside the
+    gradient of the same chunk."""
+    x = make_lact_inputs(2, 4, 4096, 128, 256, chunk=1024, order="causal", cfg=42)
+    _check(x)
