@@ -102,7 +102,9 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream);
 // Fused key pass + chunk gradient (head dim 128): partial sums per token group.
 struct KeyGradLaunch {
   int BH, N_in, C, t0, dh, groups;
-  const void *k, *v;
+  const void *k, *v, *q;      // q != nullptr: also form Aq for the chunk's queries
+  __nv_bfloat16* Aq;
+  long long aq_bs;
   const float* lr;
   const void *w1b, *w3b, *w2b;
   float* part[3];

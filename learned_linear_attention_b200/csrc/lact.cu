@@ -1102,35 +1102,36 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // contraction run fused (partial sums per token group), the queries and
   // the read run concurrently on a helper stream.
   const bool keygrad = d == 128 && !split && L.opt != 2;
-  // Chunk c: the helper stream runs the queries and the read of chunk c on
-  // the chunk-start weights (buffer cur) while the caller's stream runs the
-  // fused key/gradient kernel; the update of chunk c writes buffer cur^1,
-  // which the read of chunk c-1 used, so it waits only for that read.
+  // Chunk c: the fused kernel forms the gradient partial sums and Aq on the
+  // chunk-start weights (buffer cur); the read of chunk c (helper stream,
+  // buffer cur) then runs beside the update, which writes buffer cur^1; the
+  // next chunk's fused kernel waits for that read before rewriting Aq.
   int ci = 0;
   for (int t0 = 0; keygrad && t0 < L.N_in; t0 += L.chunk, ++ci) {
     const int C = std::min(L.chunk, L.N_in - t0);
-    const int nt = (C + 127) / 128;
-    if (L.causal) {
-      if (ss) {
-        TTT_TRY(cudaEventRecord(ss->fork, stream) == cudaSuccess ? 0 : -1);
-        TTT_TRY(cudaStreamWaitEvent(rstream, ss->fork, 0) == cudaSuccess ? 0 : -1);
-      }
-      TTT_TRY(key_pass_on(t0, C, 0, nt, rstream));
-      TTT_TRY(read_out(t0, C, rstream));
-      if (ss) TTT_TRY(cudaEventRecord(ss->read_done[ci & 1], rstream) == cudaSuccess ? 0 : -1);
-    }
     KeyGradLaunch kgl{};
     kgl.BH = BH; kgl.N_in = L.N_in; kgl.C = C; kgl.t0 = t0; kgl.dh = dh;
     kgl.groups = keygrad_groups(BH, dh, C, w.splits);
     kgl.k = L.k; kgl.v = L.v; kgl.lr = L.lr;
+    kgl.q = L.causal ? L.q : nullptr;
+    kgl.Aq = Aq; kgl.aq_bs = (long long)w.cmax * dh;
     kgl.w1b = wbuf[cur][0]; kgl.w3b = wbuf[cur][1]; kgl.w2b = wbuf[cur][2];
     kgl.part[0] = const_cast<float*>(ra.part[0]);
     kgl.part[1] = const_cast<float*>(ra.part[1]);
     kgl.part[2] = const_cast<float*>(ra.part[2]);
     kgl.st = L.st;
-    TTT_TRY(launch_lact_keygrad(kgl, stream));
+    // Aq of the previous chunk must have been read before this chunk rewrites it
     if (L.causal && ss && ci >= 1)
       TTT_TRY(cudaStreamWaitEvent(stream, ss->read_done[(ci - 1) & 1], 0) == cudaSuccess ? 0 : -1);
+    TTT_TRY(launch_lact_keygrad(kgl, stream));
+    if (L.causal) {   // the read of this chunk runs beside the update
+      if (ss) {
+        TTT_TRY(cudaEventRecord(ss->fork, stream) == cudaSuccess ? 0 : -1);
+        TTT_TRY(cudaStreamWaitEvent(rstream, ss->fork, 0) == cudaSuccess ? 0 : -1);
+      }
+      TTT_TRY(read_out(t0, C, rstream));
+      if (ss) TTT_TRY(cudaEventRecord(ss->read_done[ci & 1], rstream) == cudaSuccess ? 0 : -1);
+    }
     ra.splits = kgl.groups;
     set_out_buf(cur ^ 1);
     prof_before(K_UPDATE, stream);

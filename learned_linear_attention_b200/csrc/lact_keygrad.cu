@@ -30,8 +30,9 @@ constexpr uint32_t OFF_W2 = OFF_W13 + 2 * HALF;        // W2[:, J]: 128 d-rows x
 constexpr uint32_t OFF_DH = OFF_W2 + 2 * 8192;         // dH1 | dH3 | Gm' (16 KB each)
 constexpr uint32_t OFF_BAR = OFF_DH + 3 * HALF;
 constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
-constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARPS = 16;                          // four per TMEM lane quadrant
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr int CW = HB / (EPI_WARPS / 4);              // hidden columns per epilogue warp (16)
 // TMEM columns
 constexpr uint32_t TM_H13 = 0, TM_DG = 128, TM_G1 = 256, TM_G3 = 320, TM_G2 = 384, TM_COLS = 512;
 }  // namespace kg
@@ -42,10 +43,13 @@ struct KeyGradArgs {
   const float* lr;
   float* part[3];        // [group][BH][rows][cols] partial gradients (G1, G3, G2)
   int split;             // exact sigmoid (split-operand mode) instead of tanh.approx
+  int queries;           // causal order: also form Aq = silu(Q W1^T) (Q W3^T) for the tiles
+  __nv_bfloat16* Aq;     // [BH][cmax][dh] (queries)
+  long long aq_bs;       // cmax * dh
   DevStatus st;
 };
 struct KeyGradMaps {
-  CUtensorMap k, v, w1, w3, w2;
+  CUtensorMap k, v, q, w1, w3, w2;
 };
 
 TTT_DEVICE_INLINE float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
@@ -111,7 +115,6 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   pdl_wait();
-  pdl_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   Waiter W{abort_flag, a.st, 300};
 
@@ -149,16 +152,24 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
             tma_load_3d(smem + OFF_W2 + atom * 8192, m2, w_full, j0, atom * 64, bh);
           }
         }
-        for (int i = 0; i < nt; ++i, ++tile) {
+        const int nq = a.queries ? nt : 0;
+        for (int i = 0; ok && i < nt + nq; ++i, ++tile) {
           const uint32_t s = tile & 1;
           if (tile >= 2 && !W.wait(&kv_empty[s], ((tile >> 1) - 1) & 1, 2)) { ok = false; break; }
-          const int row = a.t0 + (grp * a.tiles_per_group + i) * BM;
+          const bool is_q = i >= nt;
+          const int row = a.t0 + (grp * a.tiles_per_group + (is_q ? i - nt : i)) * BM;
           uint8_t* st = smem + OFF_KV + s * KV_STAGE;
-          mbar_arrive_expect_tx(&kv_full[s], KV_STAGE);
-          tma_load_3d(st, &maps.k, &kv_full[s], 0, row, bh);
-          tma_load_3d(st + HALF, &maps.k, &kv_full[s], 64, row, bh);
-          tma_load_3d(st + TILE, &maps.v, &kv_full[s], 0, row, bh);
-          tma_load_3d(st + TILE + HALF, &maps.v, &kv_full[s], 64, row, bh);
+          if (is_q) {   // query tile in the K slot
+            mbar_arrive_expect_tx(&kv_full[s], TILE);
+            tma_load_3d(st, &maps.q, &kv_full[s], 0, row, bh);
+            tma_load_3d(st + HALF, &maps.q, &kv_full[s], 64, row, bh);
+          } else {
+            mbar_arrive_expect_tx(&kv_full[s], KV_STAGE);
+            tma_load_3d(st, &maps.k, &kv_full[s], 0, row, bh);
+            tma_load_3d(st + HALF, &maps.k, &kv_full[s], 64, row, bh);
+            tma_load_3d(st + TILE, &maps.v, &kv_full[s], 0, row, bh);
+            tma_load_3d(st + TILE + HALF, &maps.v, &kv_full[s], 64, row, bh);
+          }
         }
       }
       if (W.aborted()) {
@@ -175,13 +186,14 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
       const uint32_t kvb = smem_u32(smem + OFF_KV);
       const uint32_t w13 = smem_u32(smem + OFF_W13), w2 = smem_u32(smem + OFF_W2);
       const uint32_t dhb = smem_u32(smem + OFF_DH);
-      uint32_t tile = 0, item_ctr = 0;
+      uint32_t tile = 0, ktile = 0, item_ctr = 0;   // all tiles / key tiles of this CTA
       bool ok = true;
-      auto grads = [&](uint32_t t, bool first, uint32_t item_c) -> bool {
+      // gradient MMAs of key tile kt_ (its K/V tiles sit in stage t_ & 1)
+      auto grads = [&](uint32_t t_, uint32_t kt_, bool first, uint32_t item_c) -> bool {
         if (first && item_c >= 1 && !W.wait(g_empty, (item_c - 1) & 1, 3)) return false;
-        if (!W.wait(dh_ready, t & 1, 4)) return false;
+        if (!W.wait(dh_ready, kt_ & 1, 4)) return false;
         tc_fence_after();
-        const uint32_t kt = kvb + (t & 1) * KV_STAGE, vt = kt + TILE;
+        const uint32_t kt = kvb + (t_ & 1) * KV_STAGE, vt = kt + TILE;
         // K^T / V^T as MN-major A: M = d in two 64-wide blocks 16 KB apart,
         // K = tokens (rows of 128 B); dH / Gm' as MN-major B: N = 64 hidden
 #pragma unroll
@@ -194,35 +206,46 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
           mma_bf16(tmem + TM_G2, va, make_sdesc(dhb + 2 * HALF + kk * 2048, 8192, 1024), id_grad, acc);
         }
         mma_commit(dh_free);
-        mma_commit(&kv_empty[t & 1]);
+        mma_commit(&kv_empty[t_ & 1]);
+        return true;
+      };
+      // H13 (+ dG for key tiles) of tile t_ into the shared accumulator
+      auto forward = [&](uint32_t t_, bool is_key) -> bool {
+        const uint32_t s = t_ & 1;
+        if (!W.wait(&kv_full[s], (t_ >> 1) & 1, 6)) return false;
+        if (t_ >= 1 && !W.wait(acc_empty, (t_ - 1) & 1, 7)) return false;
+        tc_fence_after();
+        const uint32_t kt = kvb + s * KV_STAGE, vt = kt + TILE;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t atom = kk >> 2, ko = (kk & 3) * 32;
+          mma_bf16(tmem + TM_H13, make_sdesc(kt + atom * HALF + ko, 16, 1024),
+                   make_sdesc(w13 + atom * HALF + ko, 16, 1024), id_h, kk > 0);
+          if (is_key)
+            mma_bf16(tmem + TM_DG, make_sdesc(vt + atom * HALF + ko, 16, 1024),
+                     make_sdesc(w2 + kk * 2048, 8192, 1024), id_g, kk > 0);
+        }
+        mma_commit(acc_full);
+        if (!is_key) mma_commit(&kv_empty[s]);   // a query tile is done with its stage
         return true;
       };
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++item_ctr) {
         int bh, hb, grp;
         decode(item, bh, hb, grp);
         const int nt = group_tiles(grp);
+        const int nq = a.queries ? nt : 0;
         if (!W.wait(w_full, item_ctr & 1, 5)) { ok = false; break; }
-        const uint32_t base = tile;
-        for (int i = 0; i < nt; ++i, ++tile) {
-          const uint32_t s = tile & 1;
-          if (!W.wait(&kv_full[s], (tile >> 1) & 1, 6)) { ok = false; break; }
-          if (tile >= 1 && !W.wait(acc_empty, (tile - 1) & 1, 7)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kt = kvb + s * KV_STAGE, vt = kt + TILE;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t atom = kk >> 2, ko = (kk & 3) * 32;
-            mma_bf16(tmem + TM_H13, make_sdesc(kt + atom * HALF + ko, 16, 1024),
-                     make_sdesc(w13 + atom * HALF + ko, 16, 1024), id_h, kk > 0);
-            mma_bf16(tmem + TM_DG, make_sdesc(vt + atom * HALF + ko, 16, 1024),
-                     make_sdesc(w2 + kk * 2048, 8192, 1024), id_g, kk > 0);
-          }
-          mma_commit(acc_full);
-          if (i >= 1 && !grads(tile - 1, i - 1 == 0, item_ctr)) { ok = false; break; }
+        const uint32_t base = tile, kbase = ktile;
+        for (int i = 0; i < nt; ++i, ++tile, ++ktile) {
+          if (!forward(tile, true)) { ok = false; break; }
+          if (i >= 1 && !grads(tile - 1, ktile - 1, i - 1 == 0, item_ctr)) { ok = false; break; }
         }
         if (!ok) break;
-        if (nt > 0 && !grads(base + nt - 1, nt == 1, item_ctr)) { ok = false; break; }
+        if (nt > 0 && !grads(base + nt - 1, kbase + nt - 1, nt == 1, item_ctr)) { ok = false; break; }
         mma_commit(g_full);
+        for (int i = 0; i < nq; ++i, ++tile)
+          if (!forward(tile, false)) { ok = false; break; }
+        if (!ok) break;
         mma_commit(w_empty);
       }
       mma_commit(fin);
@@ -231,37 +254,35 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q4 = warp & 3;
-    const int cg = (warp - 2) >> 2;                 // 32-column group of the 64 hidden
+    const int cg = (warp - 2) >> 2;                 // 16-column group of the 64 hidden
     const int r = q4 * 32 + lane;                   // token row of the tile / d row of G
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     uint8_t* dh1s = smem + OFF_DH;
     const uint32_t dh1 = smem_u32(dh1s), dh3 = dh1 + HALF, gms = dh1 + 2 * HALF;
-    uint32_t tile = 0, item_ctr = 0;
+    uint32_t tile = 0, ktile = 0, item_ctr = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
       int bh, hb, grp;
       decode(item, bh, hb, grp);
       const int nt = group_tiles(grp);
+      const int nq = a.queries ? nt : 0;
       bool ok = true;
-      for (int i = 0; i < nt; ++i, ++tile) {
+      for (int i = 0; i < nt; ++i, ++tile, ++ktile) {
         const int tc = (grp * a.tiles_per_group + i) * BM + r;   // token row in the chunk
         const bool valid = tc < a.C;
         const float eta = valid ? a.lr[(size_t)bh * a.lr_len + a.t0 + tc] : 0.f;
         if (!W.wait(acc_full, tile & 1, 8)) { ok = false; break; }
         tc_fence_after();
-        uint32_t rh1[32], rh3[32], rg[32];
-        const uint32_t tb = tmem + lane_base + cg * 32;
+        uint32_t rh1[CW], rh3[CW], rg[CW];
+        const uint32_t tb = tmem + lane_base + cg * CW;
         tmem_ld16_issue(tb + TM_H13, rh1);
-        tmem_ld16_issue(tb + TM_H13 + 16, rh1 + 16);
         tmem_ld16_issue(tb + TM_H13 + 64, rh3);
-        tmem_ld16_issue(tb + TM_H13 + 80, rh3 + 16);
         tmem_ld16_issue(tb + TM_DG, rg);
-        tmem_ld16_issue(tb + TM_DG + 16, rg + 16);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(acc_empty);
-        uint32_t o1[16], o3[16], om[16];
+        uint32_t o1[CW / 2], o3[CW / 2], om[CW / 2];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
+        for (int j = 0; j < CW; j += 2) {
           float r1[2], r3[2], rm[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
@@ -277,11 +298,11 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
           o3[j >> 1] = pack_bf16x2(r3[0], r3[1]);
           om[j >> 1] = pack_bf16x2(rm[0], rm[1]);
         }
-        // the previous tile's gradient MMAs must be done reading dH
-        if (tile >= 1 && !W.wait(dh_free, (tile - 1) & 1, 9)) { ok = false; break; }
+        // the previous key tile's gradient MMAs must be done reading dH
+        if (ktile >= 1 && !W.wait(dh_free, (ktile - 1) & 1, 9)) { ok = false; break; }
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          const uint32_t off = sw128_offset(r, cg * 32 + j);
+        for (int j = 0; j < CW; j += 8) {
+          const uint32_t off = sw128_offset(r, cg * CW + j);
           st_shared_v4(dh1 + off, o1[j / 2], o1[j / 2 + 1], o1[j / 2 + 2], o1[j / 2 + 3]);
           st_shared_v4(dh3 + off, o3[j / 2], o3[j / 2 + 1], o3[j / 2 + 2], o3[j / 2 + 3]);
           st_shared_v4(gms + off, om[j / 2], om[j / 2 + 1], om[j / 2 + 2], om[j / 2 + 3]);
@@ -292,32 +313,65 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
       }
       if (!ok) break;
       if (nt == 0) continue;
-      // item done: partial gradients -> their token-group slot
+      // item's gradients complete: partial sums -> their token-group slot
       if (!W.wait(g_full, item_ctr & 1, 10)) break;
       tc_fence_after();
-      const int j0 = hb * HB + cg * 32;
-      const size_t mat_stride = (size_t)a.BH * a.dh * D;
-      const size_t slot = (size_t)grp * mat_stride;
-      float g1[32], g3[32], g2[32];
-      tmem_ld32(tmem + lane_base + TM_G1 + cg * 32, g1);
-      tmem_ld32(tmem + lane_base + TM_G3 + cg * 32, g3);
-      tmem_ld32(tmem + lane_base + TM_G2 + cg * 32, g2);
-      tc_fence_before();
-      mbar_arrive(g_empty);
-      // G1, G3 [BH][dh][d]: this thread is d row r -> element (j0 + j, r)
-      float* p1 = a.part[0] + slot + ((size_t)bh * a.dh + j0) * D + r;
-      float* p3 = a.part[1] + slot + ((size_t)bh * a.dh + j0) * D + r;
+      {
+        const int j0 = hb * HB + cg * CW;
+        const size_t mat_stride = (size_t)a.BH * a.dh * D;
+        const size_t slot = (size_t)grp * mat_stride;
+        float g1[CW], g3[CW], g2[CW];
+        tmem_ld16(tmem + lane_base + TM_G1 + cg * CW, g1);
+        tmem_ld16(tmem + lane_base + TM_G3 + cg * CW, g3);
+        tmem_ld16(tmem + lane_base + TM_G2 + cg * CW, g2);
+        tc_fence_before();
+        mbar_arrive(g_empty);
+        // G1, G3 [BH][dh][d]: this thread is d row r -> element (j0 + j, r)
+        float* p1 = a.part[0] + slot + ((size_t)bh * a.dh + j0) * D + r;
+        float* p3 = a.part[1] + slot + ((size_t)bh * a.dh + j0) * D + r;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        p1[(size_t)j * D] = g1[j];
-        p3[(size_t)j * D] = g3[j];
+        for (int j = 0; j < CW; ++j) {
+          p1[(size_t)j * D] = g1[j];
+          p3[(size_t)j * D] = g3[j];
+        }
+        // G2 [BH][d][dh]: row r, columns j0 .. j0 + CW - 1
+        float4* p2 = reinterpret_cast<float4*>(a.part[2] + slot + ((size_t)bh * D + r) * a.dh + j0);
+#pragma unroll
+        for (int j = 0; j < CW / 4; ++j) p2[j] = make_float4(g2[4 * j], g2[4 * j + 1], g2[4 * j + 2], g2[4 * j + 3]);
       }
-      // G2 [BH][d][dh]: row r, columns j0 .. j0 + 31
-      float4* p2 = reinterpret_cast<float4*>(a.part[2] + slot + ((size_t)bh * D + r) * a.dh + j0);
+      // query tiles (causal): Aq = silu(Q W1_J^T) * (Q W3_J^T) -> bf16
+      for (int i = 0; i < nq; ++i, ++tile) {
+        const int tc = (grp * a.tiles_per_group + i) * BM + r;
+        const bool valid = tc < a.C;
+        if (!W.wait(acc_full, tile & 1, 11)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t rh1[CW], rh3[CW];
+        const uint32_t tb = tmem + lane_base + cg * CW;
+        tmem_ld16_issue(tb + TM_H13, rh1);
+        tmem_ld16_issue(tb + TM_H13 + 64, rh3);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(acc_empty);
+        if (valid) {
+          uint32_t oq[CW / 2];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) p2[j] = make_float4(g2[4 * j], g2[4 * j + 1], g2[4 * j + 2], g2[4 * j + 3]);
+          for (int j = 0; j < CW; j += 2) {
+            const float x0 = __uint_as_float(rh1[j]), x1 = __uint_as_float(rh1[j + 1]);
+            const float a0 = x0 * (a.split ? sigmoid_fast(x0) : sigmoid_tanh(x0)) * __uint_as_float(rh3[j]);
+            const float a1 = x1 * (a.split ? sigmoid_fast(x1) : sigmoid_tanh(x1)) * __uint_as_float(rh3[j + 1]);
+            oq[j >> 1] = pack_bf16x2(a0, a1);
+          }
+          uint4* dq = reinterpret_cast<uint4*>(a.Aq + (size_t)bh * a.aq_bs + (size_t)tc * a.dh +
+                                               hb * HB + cg * CW);
+#pragma unroll
+          for (int j = 0; j < CW / 8; ++j) dq[j] = make_uint4(oq[4 * j], oq[4 * j + 1], oq[4 * j + 2], oq[4 * j + 3]);
+        }
+      }
+      if (!ok) break;
     }
   }
+  // dependents (the row update) may start launching once this CTA is done
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -347,6 +401,7 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream) {
   const uint64_t tok_row = (uint64_t)kg::D * 2;
   if (make_tmap_bf16_3d(&m.k, L.k, kg::D, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 128) ||
       make_tmap_bf16_3d(&m.v, L.v, kg::D, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 128) ||
+      make_tmap_bf16_3d(&m.q, L.q ? L.q : L.k, kg::D, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 128) ||
       make_tmap_bf16_3d(&m.w1, L.w1b, kg::D, L.dh, BH, tok_row, tok_row * L.dh, 64, 64) ||
       make_tmap_bf16_3d(&m.w3, L.w3b, kg::D, L.dh, BH, tok_row, tok_row * L.dh, 64, 64) ||
       make_tmap_bf16_3d(&m.w2, L.w2b, L.dh, kg::D, BH, (uint64_t)L.dh * 2, (uint64_t)L.dh * 2 * kg::D,
@@ -362,6 +417,9 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream) {
   a.lr = L.lr;
   a.part[0] = L.part[0]; a.part[1] = L.part[1]; a.part[2] = L.part[2];
   a.split = 0;
+  a.queries = L.q != nullptr ? 1 : 0;
+  a.Aq = L.Aq;
+  a.aq_bs = L.aq_bs;
   a.st = L.st;
   static bool attr = false;
   if (!attr) {
