@@ -424,66 +424,90 @@ TTT_DEVICE_INLINE void sum_partials(const RowArgs& a, int mat, size_t off, size_
 }
 
 // GD / momentum: sum the split-K partials, update, normalise the row.  One
-// warp per row, lanes own 4 consecutive columns per 128-column chunk (16-byte
-// loads; every partial sum of a chunk is in flight at once).
-constexpr int UPD_ROWS_PER_BLOCK = 8;
+// warp per UPD_RPW rows; lanes own 4 consecutive columns per 128-column chunk
+// (16-byte loads).  All partial sums of all the warp's rows are requested
+// before any is used, so many loads are in flight per warp.
+constexpr int UPD_ROWS_PER_BLOCK = 8;   // warps per block
+constexpr int UPD_RPW = 1;              // rows per warp
 __global__ void __launch_bounds__(UPD_ROWS_PER_BLOCK * 32) lact_update_kernel(RowArgs a) {
   pdl_wait();
   pdl_launch_dependents();
-  const int gw = blockIdx.x * UPD_ROWS_PER_BLOCK + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (gw >= a.BH * (2 * a.dh + a.d)) return;
-  int mat, bh, row, rows, cols;
-  row_decode(a, gw, mat, bh, row, rows, cols);
-  if (!(a.mask & (1 << mat))) return;
-  const size_t off = ((size_t)bh * rows + row) * cols;
-  const size_t split_stride = (size_t)a.BH * rows * cols;
-  const int nch = cols >> 7;                        // 128-column chunks (cols % 128 == 0)
-  float4 w[8];
+  const int lane = threadIdx.x & 31;
+  const int total = a.BH * (2 * a.dh + a.d);
+  const int gw0 = (blockIdx.x * UPD_ROWS_PER_BLOCK + (threadIdx.x >> 5)) * UPD_RPW;
+  if (gw0 >= total) return;
+  int mat[UPD_RPW], rows[UPD_RPW], cols[UPD_RPW];
+  size_t off[UPD_RPW];
+  bool live[UPD_RPW];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) w[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int q = 0; q < UPD_RPW; ++q) {
+    int bh, row;
+    live[q] = gw0 + q < total;
+    row_decode(a, live[q] ? gw0 + q : gw0, mat[q], bh, row, rows[q], cols[q]);
+    live[q] = live[q] && (a.mask & (1 << mat[q]));
+    off[q] = ((size_t)bh * rows[q] + row) * cols[q];
+  }
+  float4 w[UPD_RPW][8];
+#pragma unroll
+  for (int q = 0; q < UPD_RPW; ++q)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[q][i] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < a.splits; ++s) {
-    const float4* p = reinterpret_cast<const float4*>(a.part[mat] + s * split_stride + off) + lane;
+#pragma unroll
+    for (int q = 0; q < UPD_RPW; ++q) {
+      if (!live[q]) continue;
+      const size_t split_stride = (size_t)a.BH * rows[q] * cols[q];
+      const float4* p = reinterpret_cast<const float4*>(a.part[mat[q]] + s * split_stride + off[q]) + lane;
+      const int nch = cols[q] >> 7;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (i < nch) {
+          const float4 x = __ldcg(p + 32 * i);
+          w[q][i].x += x.x; w[q][i].y += x.y; w[q][i].z += x.z; w[q][i].w += x.w;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < UPD_RPW; ++q) {
+    if (!live[q]) continue;
+    const int nch = cols[q] >> 7;
+    float4* Wr = reinterpret_cast<float4*>(a.W[mat[q]] + off[q]) + lane;
+    float4* Mr = a.opt == 1 ? reinterpret_cast<float4*>(a.M[mat[q]] + off[q]) + lane : nullptr;
+    float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if (i < nch) {
-        const float4 x = __ldcg(p + 32 * i);
-        w[i].x += x.x; w[i].y += x.y; w[i].z += x.z; w[i].w += x.w;
+        float4 u = w[q][i];
+        if (Mr != nullptr) {
+          float4 m = Mr[32 * i];
+          m.x = a.beta * m.x + u.x; m.y = a.beta * m.y + u.y;
+          m.z = a.beta * m.z + u.z; m.w = a.beta * m.w + u.w;
+          Mr[32 * i] = m;
+          u = m;
+        }
+        const float4 x = Wr[32 * i];
+        w[q][i] = make_float4(x.x - u.x, x.y - u.y, x.z - u.z, x.w - u.w);
+        ss += w[q][i].x * w[q][i].x + w[q][i].y * w[q][i].y + w[q][i].z * w[q][i].z +
+              w[q][i].w * w[q][i].w;
       }
     }
-  }
-  float ss = 0.f;
-  float4* Wr = reinterpret_cast<float4*>(a.W[mat] + off) + lane;
-  float4* Mr = a.opt == 1 ? reinterpret_cast<float4*>(a.M[mat] + off) + lane : nullptr;
+    float scale = 1.f;
+    if (a.normalize) scale = 1.f / fmaxf(sqrtf(warp_sum(ss)), a.norm_eps);
+    uint2* Br = reinterpret_cast<uint2*>(a.Wb[mat[q]] + off[q]) + lane;
+    uint2* Lr = a.Wlo[mat[q]] != nullptr ? reinterpret_cast<uint2*>(a.Wlo[mat[q]] + off[q]) + lane : nullptr;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (i < nch) {
-      float4 u = w[i];
-      if (Mr != nullptr) {
-        float4 m = Mr[32 * i];
-        m.x = a.beta * m.x + u.x; m.y = a.beta * m.y + u.y;
-        m.z = a.beta * m.z + u.z; m.w = a.beta * m.w + u.w;
-        Mr[32 * i] = m;
-        u = m;
+    for (int i = 0; i < 8; ++i) {
+      if (i < nch) {
+        const float4 x = make_float4(w[q][i].x * scale, w[q][i].y * scale, w[q][i].z * scale,
+                                     w[q][i].w * scale);
+        Wr[32 * i] = x;
+        const uint32_t h0 = pack_bf16x2(x.x, x.y), h1 = pack_bf16x2(x.z, x.w);
+        Br[32 * i] = make_uint2(h0, h1);
+        if (Lr != nullptr)
+          Lr[32 * i] = make_uint2(pack_bf16x2(x.x - bf16lo(h0), x.y - bf16hi(h0)),
+                                  pack_bf16x2(x.z - bf16lo(h1), x.w - bf16hi(h1)));
       }
-      const float4 x = Wr[32 * i];
-      w[i] = make_float4(x.x - u.x, x.y - u.y, x.z - u.z, x.w - u.w);
-      ss += w[i].x * w[i].x + w[i].y * w[i].y + w[i].z * w[i].z + w[i].w * w[i].w;
-    }
-  }
-  float scale = 1.f;
-  if (a.normalize) scale = 1.f / fmaxf(sqrtf(warp_sum(ss)), a.norm_eps);
-  uint2* Br = reinterpret_cast<uint2*>(a.Wb[mat] + off) + lane;
-  uint2* Lr = a.Wlo[mat] != nullptr ? reinterpret_cast<uint2*>(a.Wlo[mat] + off) + lane : nullptr;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (i < nch) {
-      const float4 x = make_float4(w[i].x * scale, w[i].y * scale, w[i].z * scale, w[i].w * scale);
-      Wr[32 * i] = x;
-      const uint32_t h0 = pack_bf16x2(x.x, x.y), h1 = pack_bf16x2(x.z, x.w);
-      Br[32 * i] = make_uint2(h0, h1);
-      if (Lr != nullptr)
-        Lr[32 * i] = make_uint2(pack_bf16x2(x.x - bf16lo(h0), x.y - bf16hi(h0)),
-                                pack_bf16x2(x.z - bf16lo(h1), x.w - bf16hi(h1)));
     }
   }
 }
@@ -1135,7 +1159,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     ra.splits = kgl.groups;
     set_out_buf(cur ^ 1);
     prof_before(K_UPDATE, stream);
-    if (launch_pdl(lact_update_kernel, dim3((row_warps + UPD_ROWS_PER_BLOCK - 1) / UPD_ROWS_PER_BLOCK),
+    if (launch_pdl(lact_update_kernel, dim3((row_warps + UPD_ROWS_PER_BLOCK * UPD_RPW - 1) / (UPD_ROWS_PER_BLOCK * UPD_RPW)),
                    dim3(UPD_ROWS_PER_BLOCK * 32), 0, stream, ra) != cudaSuccess)
       return -1;
     prof_after(K_UPDATE, stream);
@@ -1162,7 +1186,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       TTT_TRY(muon());
     } else {
       prof_before(K_UPDATE, stream);
-      if (launch_pdl(lact_update_kernel, dim3((row_warps + UPD_ROWS_PER_BLOCK - 1) / UPD_ROWS_PER_BLOCK),
+      if (launch_pdl(lact_update_kernel, dim3((row_warps + UPD_ROWS_PER_BLOCK * UPD_RPW - 1) / (UPD_ROWS_PER_BLOCK * UPD_RPW)),
                      dim3(UPD_ROWS_PER_BLOCK * 32), 0, stream, ra) != cudaSuccess)
         return -1;
       prof_after(K_UPDATE, stream);
