@@ -142,10 +142,14 @@ class LaCTBench:
         return f
 
     def kernel_flops_per_step(self):
+        """Algorithmic FLOPs per step of each kernel kind (per token-head:
+        key forward 4 d dh, dG 2 d dh, three gradient products 6 d dh, query
+        forward 4 d dh, read 2 d dh)."""
         BH, d, dh, N, Nq = self.B * self.H, self.d, self.dh, self.N, self.Nq
         kp = (6 * N + 4 * Nq) * d * dh * BH
+        kg = (12 * N + (4 * Nq if self.causal else 0)) * d * dh * BH
         return {"lact_keypass": kp, "gemm_grad": 6 * d * dh * N * BH,
-                "gemm_read": 2 * d * dh * Nq * BH}
+                "gemm_read": 2 * d * dh * Nq * BH, "lact_keygrad": kg}
 
     def resident_bytes(self):
         return sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v, self.lr,

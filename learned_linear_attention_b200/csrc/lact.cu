@@ -17,7 +17,6 @@
 // Bidirectional order: steps 1 (keys only), 3, 4 for every chunk, then the
 // queries run step 1 (queries only) and step 2 with the final weights.
 #include <algorithm>
-#include <mutex>
 
 #include "gemm.cuh"
 #include "kernels.h"
@@ -642,12 +641,13 @@ struct SideStreams {
   cudaEvent_t fork = nullptr, join[3] = {nullptr, nullptr, nullptr}, read_done[2] = {nullptr, nullptr};
   bool ok = false;
 };
+// Helper streams and their events belong to the calling host thread (one set
+// per device), so calls made concurrently from several threads never record
+// or wait on each other's events.
 static SideStreams* side_streams() {
-  static SideStreams per_dev[64];
-  static std::mutex mu;
+  thread_local SideStreams per_dev[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(mu);
   SideStreams& x = per_dev[dev];
   if (!x.ok) {
     bool good = cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess &&

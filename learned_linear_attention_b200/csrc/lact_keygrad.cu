@@ -8,9 +8,12 @@
 //   MMA   H13 = K [W1_J; W3_J]^T   (128 x 128),   dGr = V W2[:, J]  (128 x 64)
 //   epi   dG = -eta dGr, dH3 = dG silu(H1), dH1 = dG H3 silu'(H1),
 //         Gm' = -eta silu(H1) H3           -> bf16 operands in shared memory
-//   MMA   G1_J^T += K^T dH1, G3_J^T += K^T dH3, G2[:, J] += V^T Gm'
+//   MMA   [G1_J | G3_J]^T += K^T [dH1 | dH3] (one N = 128 product),
+//         G2[:, J] += V^T Gm'
 // with the K and V tiles reused from shared memory (as MN-major operands)
 // and the three gradient accumulators resident in TMEM across the group.
+// H13 alternates between two TMEM buffers, so a tile's forward product runs
+// while the epilogue still works on the previous tile.
 // At the end of the item the partial gradients are stored (plain stores,
 // one slot per token group) and the row update kernel sums the groups in a
 // fixed order.  Nothing of the chunk's intermediates goes to global memory.
@@ -33,8 +36,8 @@ constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 constexpr int EPI_WARPS = 16;                          // four per TMEM lane quadrant
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
 constexpr int CW = HB / (EPI_WARPS / 4);              // hidden columns per epilogue warp (16)
-// TMEM columns
-constexpr uint32_t TM_H13 = 0, TM_DG = 128, TM_G1 = 256, TM_G3 = 320, TM_G2 = 384, TM_COLS = 512;
+// TMEM columns: H13 in two buffers, dGr (key tiles), G2, [G1 | G3]
+constexpr uint32_t TM_H13A = 0, TM_DG = 128, TM_G2 = 192, TM_G13 = 256, TM_H13B = 384, TM_COLS = 512;
 }  // namespace kg
 
 struct KeyGradArgs {
@@ -51,6 +54,24 @@ struct KeyGradArgs {
 struct KeyGradMaps {
   CUtensorMap k, v, q, w1, w3, w2;
 };
+
+TTT_DEVICE_INLINE bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+TTT_DEVICE_INLINE void tma_prefetch_l2_3d(const CUtensorMap* m, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
 
 TTT_DEVICE_INLINE float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 TTT_DEVICE_INLINE float sigmoid_tanh(float x) {
@@ -69,9 +90,9 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
   uint64_t* kv_empty = kv_full + 2;                                   // [2]
   uint64_t* w_full = kv_empty + 2;
   uint64_t* w_empty = w_full + 1;
-  uint64_t* acc_full = w_empty + 1;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* dh_ready = acc_empty + 1;
+  uint64_t* acc_full = w_empty + 1;    // [2]: per H13 buffer
+  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint64_t* dh_ready = acc_empty + 2;
   uint64_t* dh_free = dh_ready + 1;
   uint64_t* g_full = dh_free + 1;
   uint64_t* g_empty = g_full + 1;
@@ -90,8 +111,10 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
     }
     mbar_init(w_full, 1);
     mbar_init(w_empty, 1);
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, EPI_WARPS * 32);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], EPI_WARPS * 32);
+    }
     mbar_init(dh_ready, EPI_WARPS * 32);
     mbar_init(dh_free, 1);
     mbar_init(g_full, 1);
@@ -152,6 +175,13 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
             tma_load_3d(smem + OFF_W2 + atom * 8192, m2, w_full, j0, atom * 64, bh);
           }
         }
+        // warm L2 with the item's later tiles; their loads then hit it
+        for (int i = 2; i < nt; ++i)
+          for (int h = 0; h < 2; ++h) {
+            const int row = a.t0 + (grp * a.tiles_per_group + i) * BM;
+            tma_prefetch_l2_3d(&maps.k, h * 64, row, bh);
+            tma_prefetch_l2_3d(&maps.v, h * 64, row, bh);
+          }
         const int nq = a.queries ? nt : 0;
         for (int i = 0; ok && i < nt + nq; ++i, ++tile) {
           const uint32_t s = tile & 1;
@@ -179,55 +209,64 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
+    // One thread issues every MMA.  Within an item it polls the readiness of
+    // the next forward product and of the next gradient product and issues
+    // whichever can go, so a gradient whose operands are ready never waits
+    // behind a forward product that waits for its tile.
     if (lane == 0) {
       const uint32_t id_h = make_idesc(128, 128, false, false);
       const uint32_t id_g = make_idesc(128, 64, false, true);
-      const uint32_t id_grad = make_idesc(128, 64, true, true);
+      const uint32_t id_g13 = make_idesc(128, 128, true, true);
+      const uint32_t id_g2 = make_idesc(128, 64, true, true);
       const uint32_t kvb = smem_u32(smem + OFF_KV);
       const uint32_t w13 = smem_u32(smem + OFF_W13), w2 = smem_u32(smem + OFF_W2);
       const uint32_t dhb = smem_u32(smem + OFF_DH);
       uint32_t tile = 0, ktile = 0, item_ctr = 0;   // all tiles / key tiles of this CTA
       bool ok = true;
-      // gradient MMAs of key tile kt_ (its K/V tiles sit in stage t_ & 1)
-      auto grads = [&](uint32_t t_, uint32_t kt_, bool first, uint32_t item_c) -> bool {
-        if (first && item_c >= 1 && !W.wait(g_empty, (item_c - 1) & 1, 3)) return false;
-        if (!W.wait(dh_ready, kt_ & 1, 4)) return false;
-        tc_fence_after();
-        const uint32_t kt = kvb + (t_ & 1) * KV_STAGE, vt = kt + TILE;
-        // K^T / V^T as MN-major A: M = d in two 64-wide blocks 16 KB apart,
-        // K = tokens (rows of 128 B); dH / Gm' as MN-major B: N = 64 hidden
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-          const uint64_t ka = make_sdesc(kt + kk * 2048, HALF, 1024);
-          const uint64_t va = make_sdesc(vt + kk * 2048, HALF, 1024);
-          mma_bf16(tmem + TM_G1, ka, make_sdesc(dhb + kk * 2048, 8192, 1024), id_grad, acc);
-          mma_bf16(tmem + TM_G3, ka, make_sdesc(dhb + HALF + kk * 2048, 8192, 1024), id_grad, acc);
-          mma_bf16(tmem + TM_G2, va, make_sdesc(dhb + 2 * HALF + kk * 2048, 8192, 1024), id_grad, acc);
-        }
-        mma_commit(dh_free);
-        mma_commit(&kv_empty[t_ & 1]);
+      // tile t can take its forward product: its tile has landed, its H13
+      // buffer was read by the epilogue (tile t - 2) and, for a key tile, so
+      // was dGr (tile t - 1)
+      auto fwd_ready = [&](uint32_t t, bool is_key) -> bool {
+        if (!mbar_test(&kv_full[t & 1], (t >> 1) & 1)) return false;
+        if (t >= 2 && !mbar_test(&acc_empty[t & 1], ((t >> 1) - 1) & 1)) return false;
+        if (is_key && t >= 1 && !mbar_test(&acc_empty[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
         return true;
       };
-      // H13 (+ dG for key tiles) of tile t_ into the shared accumulator
-      auto forward = [&](uint32_t t_, bool is_key) -> bool {
-        const uint32_t s = t_ & 1;
-        if (!W.wait(&kv_full[s], (t_ >> 1) & 1, 6)) return false;
-        if (t_ >= 1 && !W.wait(acc_empty, (t_ - 1) & 1, 7)) return false;
+      // H13 (+ dGr for key tiles) of tile t into its H13 buffer
+      auto forward = [&](uint32_t t, bool is_key) {
         tc_fence_after();
+        const uint32_t s = t & 1;
         const uint32_t kt = kvb + s * KV_STAGE, vt = kt + TILE;
+        const uint32_t acc = tmem + (s ? TM_H13B : TM_H13A);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t atom = kk >> 2, ko = (kk & 3) * 32;
-          mma_bf16(tmem + TM_H13, make_sdesc(kt + atom * HALF + ko, 16, 1024),
+          mma_bf16(acc, make_sdesc(kt + atom * HALF + ko, 16, 1024),
                    make_sdesc(w13 + atom * HALF + ko, 16, 1024), id_h, kk > 0);
           if (is_key)
             mma_bf16(tmem + TM_DG, make_sdesc(vt + atom * HALF + ko, 16, 1024),
                      make_sdesc(w2 + kk * 2048, 8192, 1024), id_g, kk > 0);
         }
-        mma_commit(acc_full);
+        mma_commit(&acc_full[s]);
         if (!is_key) mma_commit(&kv_empty[s]);   // a query tile is done with its stage
-        return true;
+      };
+      // gradient products of the key tile in stage t & 1
+      auto grads = [&](uint32_t t, bool first) {
+        tc_fence_after();
+        const uint32_t kt = kvb + (t & 1) * KV_STAGE, vt = kt + TILE;
+        // K^T / V^T as MN-major A: M = d in two 64-wide blocks 16 KB apart,
+        // K = tokens (rows of 128 B); [dH1 | dH3] as MN-major B with its two
+        // 64-wide blocks 16 KB apart (N = 128), Gm' as N = 64
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+          mma_bf16(tmem + TM_G13, make_sdesc(kt + kk * 2048, HALF, 1024),
+                   make_sdesc(dhb + kk * 2048, HALF, 1024), id_g13, acc);
+          mma_bf16(tmem + TM_G2, make_sdesc(vt + kk * 2048, HALF, 1024),
+                   make_sdesc(dhb + 2 * HALF + kk * 2048, 8192, 1024), id_g2, acc);
+        }
+        mma_commit(dh_free);
+        mma_commit(&kv_empty[t & 1]);
       };
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++item_ctr) {
         int bh, hb, grp;
@@ -235,17 +274,48 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         const int nt = group_tiles(grp);
         const int nq = a.queries ? nt : 0;
         if (!W.wait(w_full, item_ctr & 1, 5)) { ok = false; break; }
-        const uint32_t base = tile, kbase = ktile;
-        for (int i = 0; i < nt; ++i, ++tile, ++ktile) {
-          if (!forward(tile, true)) { ok = false; break; }
-          if (i >= 1 && !grads(tile - 1, ktile - 1, i - 1 == 0, item_ctr)) { ok = false; break; }
+        // key tiles first, then the query tiles
+        int nf = 0, ng = 0;   // forward / gradient products issued in this item
+        uint64_t t_idle = 0;
+        uint32_t spins = 0;
+        while (nf < nt + nq || ng < nt) {
+          bool prog = false;
+          // the next key tile's gradient: its forward is issued and its dH is
+          // staged (the accumulators were read out after the previous item)
+          if (ng < nt && ng < nf) {
+            const bool first = ng == 0;
+            if ((!first || item_ctr == 0 || mbar_test(g_empty, (item_ctr - 1) & 1)) &&
+                mbar_test(dh_ready, (ktile + ng) & 1)) {
+              grads(tile + ng, first);
+              ++ng;
+              prog = true;
+              if (ng == nt) mma_commit(g_full);
+            }
+          }
+          if (nf < nt + nq) {
+            const bool is_key = nf < nt;
+            if (fwd_ready(tile + nf, is_key)) {
+              forward(tile + nf, is_key);
+              ++nf;
+              prog = true;
+            }
+          }
+          if (prog) {
+            spins = 0;
+            t_idle = 0;
+            continue;
+          }
+          if ((++spins & 255u) == 0u) {   // bounded: give up after the wait timeout
+            if (W.aborted()) { ok = false; break; }
+            const uint64_t now = globaltimer_ns();
+            if (t_idle == 0) t_idle = now;
+            else if (now - t_idle > W.st.timeout_ns) { W.fail(15); ok = false; break; }
+          }
         }
         if (!ok) break;
-        if (nt > 0 && !grads(base + nt - 1, kbase + nt - 1, nt == 1, item_ctr)) { ok = false; break; }
-        mma_commit(g_full);
-        for (int i = 0; i < nq; ++i, ++tile)
-          if (!forward(tile, false)) { ok = false; break; }
-        if (!ok) break;
+        if (nt == 0) mma_commit(g_full);
+        tile += nt + nq;
+        ktile += nt;
         mma_commit(w_empty);
       }
       mma_commit(fin);
@@ -270,16 +340,17 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         const int tc = (grp * a.tiles_per_group + i) * BM + r;   // token row in the chunk
         const bool valid = tc < a.C;
         const float eta = valid ? a.lr[(size_t)bh * a.lr_len + a.t0 + tc] : 0.f;
-        if (!W.wait(acc_full, tile & 1, 8)) { ok = false; break; }
+        if (!W.wait(&acc_full[tile & 1], (tile >> 1) & 1, 8)) { ok = false; break; }
         tc_fence_after();
         uint32_t rh1[CW], rh3[CW], rg[CW];
         const uint32_t tb = tmem + lane_base + cg * CW;
-        tmem_ld16_issue(tb + TM_H13, rh1);
-        tmem_ld16_issue(tb + TM_H13 + 64, rh3);
+        const uint32_t th = tb + ((tile & 1) ? TM_H13B : TM_H13A);
+        tmem_ld16_issue(th, rh1);
+        tmem_ld16_issue(th + 64, rh3);
         tmem_ld16_issue(tb + TM_DG, rg);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(acc_empty);
+        mbar_arrive(&acc_empty[tile & 1]);
         uint32_t o1[CW / 2], o3[CW / 2], om[CW / 2];
 #pragma unroll
         for (int j = 0; j < CW; j += 2) {
@@ -321,8 +392,8 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         const size_t mat_stride = (size_t)a.BH * a.dh * D;
         const size_t slot = (size_t)grp * mat_stride;
         float g1[CW], g3[CW], g2[CW];
-        tmem_ld16(tmem + lane_base + TM_G1 + cg * CW, g1);
-        tmem_ld16(tmem + lane_base + TM_G3 + cg * CW, g3);
+        tmem_ld16(tmem + lane_base + TM_G13 + cg * CW, g1);
+        tmem_ld16(tmem + lane_base + TM_G13 + HB + cg * CW, g3);
         tmem_ld16(tmem + lane_base + TM_G2 + cg * CW, g2);
         tc_fence_before();
         mbar_arrive(g_empty);
@@ -343,15 +414,15 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
       for (int i = 0; i < nq; ++i, ++tile) {
         const int tc = (grp * a.tiles_per_group + i) * BM + r;
         const bool valid = tc < a.C;
-        if (!W.wait(acc_full, tile & 1, 11)) { ok = false; break; }
+        if (!W.wait(&acc_full[tile & 1], (tile >> 1) & 1, 11)) { ok = false; break; }
         tc_fence_after();
         uint32_t rh1[CW], rh3[CW];
-        const uint32_t tb = tmem + lane_base + cg * CW;
-        tmem_ld16_issue(tb + TM_H13, rh1);
-        tmem_ld16_issue(tb + TM_H13 + 64, rh3);
+        const uint32_t tb = tmem + lane_base + cg * CW + ((tile & 1) ? TM_H13B : TM_H13A);
+        tmem_ld16_issue(tb, rh1);
+        tmem_ld16_issue(tb + 64, rh3);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(acc_empty);
+        mbar_arrive(&acc_empty[tile & 1]);
         if (valid) {
           uint32_t oq[CW / 2];
 #pragma unroll

@@ -145,7 +145,7 @@ constexpr uint32_t OFF_SB = OFF_EV + 2 * TILE_BYTES;              // 8 KB (S, bf
 constexpr uint32_t OFF_BAR = OFF_SB + D * D * 2;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;             // + alignment slack
 // TMEM columns
-constexpr uint32_t TM_P0 = 0, TM_P1 = 128, TM_O = 256, TM_S = 320, TM_COLS = 512;
+constexpr uint32_t TM_P0 = 0, TM_P1 = 128, TM_O0 = 256, TM_S = 320, TM_O1 = 384, TM_COLS = 512;
 }  // namespace lin
 
 struct LinUmmaArgs {
@@ -264,13 +264,16 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
         const uint32_t ks = qs + TILE_BYTES;
         const uint32_t pt = pt_base + s * 2 * TILE_BYTES;
         const uint32_t ev = ev_base + s * TILE_BYTES;
-        // O = mask(P) (eta V): K = 128 keys, two 64-key atoms of the P tile
+        // O = mask(P) (eta V): K = 128 keys, two 64-key atoms of the P tile.
+        // O alternates between two TMEM buffers so the epilogue can store the
+        // previous tile's O while this tile's products run.
+        const uint32_t tm_o = s ? TM_O1 : TM_O0;
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + TM_O, make_sdesc(pt + (kk >> 2) * TILE_BYTES + (kk & 3) * 32, 16, 1024),
+          mma_bf16(tmem + tm_o, make_sdesc(pt + (kk >> 2) * TILE_BYTES + (kk & 3) * 32, 16, 1024),
                    make_sdesc(ev + kk * 2048, 8192, 1024), id_o, kk > 0);
         // O += Q S_{prev}
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + TM_O, make_sdesc(qs + kk * 32, 16, 1024),
+          mma_bf16(tmem + tm_o, make_sdesc(qs + kk * 32, 16, 1024),
                    make_sdesc(sb_base + kk * 2048, 8192, 1024), id_o, 1);
         // S += K^T (eta V)   (M = 64: rows live in lanes 0-15 of each quadrant)
         for (int kk = 0; kk < 8; ++kk)
@@ -314,7 +317,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     auto store_out = [&](int tile) {
       const int t = tile * T + r;
       float o[32];
-      tmem_ld32(tmem + lane_base + TM_O + hf * 32, o);
+      tmem_ld32(tmem + lane_base + ((tile & 1) ? TM_O1 : TM_O0) + hf * 32, o);
       if (t < a.N) {
         const size_t base = ((size_t)bh * a.N + t) * D + hf * 32;
         if (a.out_bf16) {
@@ -376,7 +379,6 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       if (i > 0) {
         if (!W.wait(ofull, (i - 1) & 1, 6)) { ok = false; break; }
         tc_fence_after();
-        store_out(i - 1);
         // S after tile i-1 -> bf16 operand copy for tile i
         float sv[32];
         tmem_ld32(tmem + lane_base + TM_S + hf * 32, sv);
@@ -391,6 +393,9 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(ops);
+      // the previous tile's output leaves the critical path: stored while
+      // this tile's products run (its TMEM buffer is next written by tile i+1)
+      if (i > 0) store_out(i - 1);
     }
     if (ok && n_tiles > 0 && W.wait(ofull, (n_tiles - 1) & 1, 7)) {
       tc_fence_after();
