@@ -354,6 +354,9 @@ struct RowArgs {
   const float* part[3];     // split-K partial gradients [splits][BH][rows][cols]
   float* rowss;             // [3][BH][rows] row sums of squares (Muon)
   const float* X32;         // NS result [3][BH][r][c] (Muon apply)
+  DevStatus st;
+  int nbuf;                 // cast: copies written, buf_stride elements apart
+  size_t buf_stride;
 };
 
 constexpr int ROW_MAXV = 32;  // columns per lane (cols <= 1024)
@@ -390,8 +393,10 @@ __global__ void lact_cast_kernel(RowArgs a) {
   for (int c = lane; c < cols; c += 32) {
     const float x = a.W[mat][off + c];
     const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    a.Wb[mat][off + c] = h;
-    if (a.Wlo[mat] != nullptr) a.Wlo[mat][off + c] = bf16_residual(x, h);
+    for (int b = 0; b < a.nbuf; ++b) {
+      a.Wb[mat][b * a.buf_stride + off + c] = h;
+      if (a.Wlo[mat] != nullptr) a.Wlo[mat][b * a.buf_stride + off + c] = bf16_residual(x, h);
+    }
   }
 }
 
@@ -509,6 +514,114 @@ __global__ void __launch_bounds__(UPD_ROWS_PER_BLOCK * 32) lact_update_kernel(Ro
       }
     }
   }
+}
+
+// GD / momentum on slabs of whole rows (about 8 KB of one matrix of one
+// head).  One thread brings the slab's split-K partial sums, its fp32
+// weights and its momentum into shared memory with bulk copies completing
+// on one mbarrier, so every byte a block needs is in flight at once; then
+// each warp sums its rows' partials in split order, updates, normalises
+// and writes fp32 weights and bf16 copies.
+constexpr int UPB_THREADS = 256;
+constexpr uint32_t UPB_SLAB = 8192;
+constexpr int UPB_MAX_SPLITS = 8;
+__host__ __device__ __forceinline__ int upb_rows(int cols) { return cols * 4 >= (int)UPB_SLAB ? 1 : (int)UPB_SLAB / (cols * 4); }
+
+TTT_DEVICE_INLINE void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__global__ void __launch_bounds__(UPB_THREADS) lact_update_bulk_kernel(RowArgs a) {
+  extern __shared__ __align__(128) uint8_t upb_smem[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r13 = upb_rows(a.d), r2 = upb_rows(a.dh);
+  const int s13 = (a.dh + r13 - 1) / r13, s2 = (a.d + r2 - 1) / r2;
+  const int per_bh = 2 * s13 + s2;
+  const int bh = blockIdx.x / per_bh, rr = blockIdx.x % per_bh;
+  const int mat = rr < s13 ? 0 : (rr < 2 * s13 ? 1 : 2);
+  const int slab = mat == 0 ? rr : (mat == 1 ? rr - s13 : rr - 2 * s13);
+  const int rows = mat < 2 ? a.dh : a.d, cols = mat < 2 ? a.d : a.dh;
+  const int R = mat < 2 ? r13 : r2;
+  const int row0 = slab * R, nrows = min(R, rows - row0);
+  if (bh >= a.BH || nrows <= 0 || !(a.mask & (1 << mat))) return;
+  const size_t off = ((size_t)bh * rows + row0) * cols;
+  const uint32_t bytes = (uint32_t)nrows * cols * 4;
+  float* const Wg = mat == 0 ? a.W[0] : (mat == 1 ? a.W[1] : a.W[2]);
+  float* const Mg = a.opt == 1 ? (mat == 0 ? a.M[0] : (mat == 1 ? a.M[1] : a.M[2])) : nullptr;
+  const float* const Pg = mat == 0 ? a.part[0] : (mat == 1 ? a.part[1] : a.part[2]);
+  __nv_bfloat16* const Bg = mat == 0 ? a.Wb[0] : (mat == 1 ? a.Wb[1] : a.Wb[2]);
+  __nv_bfloat16* const Lg = mat == 0 ? a.Wlo[0] : (mat == 1 ? a.Wlo[1] : a.Wlo[2]);
+  const size_t split_stride = (size_t)a.BH * rows * cols;
+  float* sp = reinterpret_cast<float*>(upb_smem);                  // [splits][R][cols]
+  float* sw = sp + (size_t)a.splits * UPB_SLAB / 4;                 // [R][cols]
+  float* sm = sw + UPB_SLAB / 4;                                    // [R][cols]
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar, bytes * (a.splits + 1 + (Mg != nullptr ? 1 : 0)));
+    for (int s = 0; s < a.splits; ++s)
+      bulk_load(sp + (size_t)s * UPB_SLAB / 4, Pg + s * split_stride + off, bytes, &bar);
+    bulk_load(sw, Wg + off, bytes, &bar);
+    if (Mg != nullptr) bulk_load(sm, Mg + off, bytes, &bar);
+  }
+  Waiter W{&abort_flag, a.st, 500};
+  if (!W.wait(&bar, 0, 0)) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = cols >> 7;   // 128-column chunks; lane owns 4 columns of each
+  for (int r = warp; r < nrows; r += UPB_THREADS / 32) {
+    float4 w[8];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i >= nch) break;
+      const int c = r * cols + 128 * i + 4 * lane;
+      float4 u = *reinterpret_cast<const float4*>(sp + c);
+      for (int s = 1; s < a.splits; ++s) {
+        const float4 x = *reinterpret_cast<const float4*>(sp + (size_t)s * UPB_SLAB / 4 + c);
+        u.x += x.x; u.y += x.y; u.z += x.z; u.w += x.w;
+      }
+      if (Mg != nullptr) {
+        float4 m = *reinterpret_cast<const float4*>(sm + c);
+        m.x = a.beta * m.x + u.x; m.y = a.beta * m.y + u.y;
+        m.z = a.beta * m.z + u.z; m.w = a.beta * m.w + u.w;
+        *reinterpret_cast<float4*>(Mg + off + c) = m;
+        u = m;
+      }
+      const float4 x = *reinterpret_cast<const float4*>(sw + c);
+      w[i] = make_float4(x.x - u.x, x.y - u.y, x.z - u.z, x.w - u.w);
+      ss += w[i].x * w[i].x + w[i].y * w[i].y + w[i].z * w[i].z + w[i].w * w[i].w;
+    }
+    float scale = 1.f;
+    if (a.normalize) scale = 1.f / fmaxf(sqrtf(warp_sum(ss)), a.norm_eps);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i >= nch) break;
+      const int c = r * cols + 128 * i + 4 * lane;
+      const float4 x = make_float4(w[i].x * scale, w[i].y * scale, w[i].z * scale, w[i].w * scale);
+      *reinterpret_cast<float4*>(Wg + off + c) = x;
+      const uint32_t h0 = pack_bf16x2(x.x, x.y), h1 = pack_bf16x2(x.z, x.w);
+      *reinterpret_cast<uint2*>(Bg + off + c) = make_uint2(h0, h1);
+      if (Lg != nullptr)
+        *reinterpret_cast<uint2*>(Lg + off + c) =
+            make_uint2(pack_bf16x2(x.x - bf16lo(h0), x.y - bf16hi(h0)),
+                       pack_bf16x2(x.z - bf16lo(h1), x.w - bf16hi(h1)));
+    }
+  }
+}
+static int update_bulk_blocks(int BH, int d, int dh) {
+  const int r13 = upb_rows(d), r2 = upb_rows(dh);
+  return BH * (2 * ((dh + r13 - 1) / r13) + (d + r2 - 1) / r2);
 }
 
 // Muon step 1: M = beta M + G, and the row sums of squares of M.
@@ -788,7 +901,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   RowArgs ra{};
   ra.BH = BH; ra.d = d; ra.dh = dh; ra.splits = w.splits; ra.opt = L.opt;
   ra.normalize = L.normalize_rows; ra.mask = L.update_mask; ra.beta = L.beta;
-  ra.norm_eps = L.norm_eps; ra.ns_eps = L.ns_eps;
+  ra.norm_eps = L.norm_eps; ra.ns_eps = L.ns_eps; ra.st = L.st;
   ra.W[0] = W1; ra.W[1] = W3; ra.W[2] = W2;
   ra.M[0] = M1; ra.M[1] = M3; ra.M[2] = M2;
   auto set_out_buf = [&](int b) {
@@ -804,16 +917,41 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   ra.X32 = reinterpret_cast<float*>(ws + w.nsx32);
   const int row_warps = BH * (2 * dh + d);
   const int row_blocks = (row_warps * 32 + 255) / 256;
+  // GD / momentum row update: slab kernel with bulk copies (split count
+  // bounded by its shared memory), else one warp per row
+  auto row_update = [&](cudaStream_t st) -> int {
+    prof_before(K_UPDATE, st);
+    cudaError_t e;
+    if (ra.splits <= UPB_MAX_SPLITS && d % 128 == 0 && dh % 128 == 0) {
+      static bool upb_attr = false;
+      if (!upb_attr) {
+        if (cudaFuncSetAttribute(lact_update_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)((UPB_MAX_SPLITS + 2) * UPB_SLAB)) != cudaSuccess)
+          return -1;
+        upb_attr = true;
+      }
+      e = launch_pdl(lact_update_bulk_kernel, dim3(update_bulk_blocks(BH, d, dh)), dim3(UPB_THREADS),
+                     (size_t)(ra.splits + 2) * UPB_SLAB, st, ra);
+    } else {
+      e = launch_pdl(lact_update_kernel,
+                     dim3((row_warps + UPD_ROWS_PER_BLOCK * UPD_RPW - 1) / (UPD_ROWS_PER_BLOCK * UPD_RPW)),
+                     dim3(UPD_ROWS_PER_BLOCK * 32), 0, st, ra);
+    }
+    if (e != cudaSuccess) return -1;
+    prof_after(K_UPDATE, st);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  };
 
   // both buffers start from the state (matrices excluded by update_mask are
   // never rewritten and must read the same in either buffer)
-  for (int b = 0; b < 2; ++b) {
-    set_out_buf(b);
-    prof_before(K_LACT_CAST, stream);
-    if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
-      return -1;
-    prof_after(K_LACT_CAST, stream);
-  }
+  set_out_buf(0);
+  ra.nbuf = 2;
+  ra.buf_stride = wsz;
+  prof_before(K_LACT_CAST, stream);
+  if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
+    return -1;
+  prof_after(K_LACT_CAST, stream);
+  ra.nbuf = 1;
   TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
 
   // ---- tensor maps.  Token tensors {d, rows, BH}; K-major boxes {64, 128},
@@ -1158,11 +1296,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     }
     ra.splits = kgl.groups;
     set_out_buf(cur ^ 1);
-    prof_before(K_UPDATE, stream);
-    if (launch_pdl(lact_update_kernel, dim3((row_warps + UPD_ROWS_PER_BLOCK * UPD_RPW - 1) / (UPD_ROWS_PER_BLOCK * UPD_RPW)),
-                   dim3(UPD_ROWS_PER_BLOCK * 32), 0, stream, ra) != cudaSuccess)
-      return -1;
-    prof_after(K_UPDATE, stream);
+    TTT_TRY(row_update(stream));
     cur ^= 1;
   }
   if (keygrad && L.causal && ss && ci >= 1)   // the last read joins the caller's stream
@@ -1185,12 +1319,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     if (L.opt == 2) {
       TTT_TRY(muon());
     } else {
-      prof_before(K_UPDATE, stream);
-      if (launch_pdl(lact_update_kernel, dim3((row_warps + UPD_ROWS_PER_BLOCK * UPD_RPW - 1) / (UPD_ROWS_PER_BLOCK * UPD_RPW)),
-                     dim3(UPD_ROWS_PER_BLOCK * 32), 0, stream, ra) != cudaSuccess)
-        return -1;
-      prof_after(K_UPDATE, stream);
-      TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+      TTT_TRY(row_update(stream));
     }
     cur ^= 1;
   }
