@@ -539,8 +539,6 @@ __global__ void __launch_bounds__(UPB_THREADS) lact_update_bulk_kernel(RowArgs a
   extern __shared__ __align__(128) uint8_t upb_smem[];
   __shared__ uint64_t bar;
   __shared__ uint32_t abort_flag;
-  pdl_wait();
-  pdl_launch_dependents();
   const int r13 = upb_rows(a.d), r2 = upb_rows(a.dh);
   const int s13 = (a.dh + r13 - 1) / r13, s2 = (a.d + r2 - 1) / r2;
   const int per_bh = 2 * s13 + s2;
@@ -550,7 +548,11 @@ __global__ void __launch_bounds__(UPB_THREADS) lact_update_bulk_kernel(RowArgs a
   const int rows = mat < 2 ? a.dh : a.d, cols = mat < 2 ? a.d : a.dh;
   const int R = mat < 2 ? r13 : r2;
   const int row0 = slab * R, nrows = min(R, rows - row0);
-  if (bh >= a.BH || nrows <= 0 || !(a.mask & (1 << mat))) return;
+  if (bh >= a.BH || nrows <= 0 || !(a.mask & (1 << mat))) {
+    pdl_wait();
+    pdl_launch_dependents();
+    return;
+  }
   const size_t off = ((size_t)bh * rows + row0) * cols;
   const uint32_t bytes = (uint32_t)nrows * cols * 4;
   float* const Wg = mat == 0 ? a.W[0] : (mat == 1 ? a.W[1] : a.W[2]);
@@ -568,13 +570,19 @@ __global__ void __launch_bounds__(UPB_THREADS) lact_update_bulk_kernel(RowArgs a
     fence_barrier_init();
   }
   __syncthreads();
+  // The fp32 weights and momentum were last written by an update that had
+  // completed before the preceding kernel started, so their copies go out
+  // before the wait for that kernel (whose partial sums come after it).
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(&bar, bytes * (a.splits + 1 + (Mg != nullptr ? 1 : 0)));
-    for (int s = 0; s < a.splits; ++s)
-      bulk_load(sp + (size_t)s * UPB_SLAB / 4, Pg + s * split_stride + off, bytes, &bar);
     bulk_load(sw, Wg + off, bytes, &bar);
     if (Mg != nullptr) bulk_load(sm, Mg + off, bytes, &bar);
   }
+  pdl_wait();
+  pdl_launch_dependents();
+  if (threadIdx.x == 0)
+    for (int s = 0; s < a.splits; ++s)
+      bulk_load(sp + (size_t)s * UPB_SLAB / 4, Pg + s * split_stride + off, bytes, &bar);
   Waiter W{&abort_flag, a.st, 500};
   if (!W.wait(&bar, 0, 0)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -137,7 +137,10 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_wait();
+  // The TMA thread waits for the preceding kernels after it has issued its
+  // first token tiles (inputs of the call, which no kernel of the call
+  // writes); everything else waits here.
+  if (warp != 0 || lane != 0) pdl_wait();
   const uint32_t tmem = *tmem_slot;
   Waiter W{abort_flag, a.st, 300};
 
@@ -156,6 +159,36 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
     if (lane == 0) {
       uint32_t tile = 0, item_ctr = 0;
       bool ok = true;
+      // tile i of an item: key tiles (K and V) first, then query tiles (Q in
+      // the K slot)
+      auto issue_tile = [&](uint32_t t, int i, int nt, int bh, int grp) {
+        const uint32_t s = t & 1;
+        const bool is_q = i >= nt;
+        const int row = a.t0 + (grp * a.tiles_per_group + (is_q ? i - nt : i)) * BM;
+        uint8_t* st = smem + OFF_KV + s * KV_STAGE;
+        if (is_q) {
+          mbar_arrive_expect_tx(&kv_full[s], TILE);
+          tma_load_3d(st, &maps.q, &kv_full[s], 0, row, bh);
+          tma_load_3d(st + HALF, &maps.q, &kv_full[s], 64, row, bh);
+        } else {
+          mbar_arrive_expect_tx(&kv_full[s], KV_STAGE);
+          tma_load_3d(st, &maps.k, &kv_full[s], 0, row, bh);
+          tma_load_3d(st + HALF, &maps.k, &kv_full[s], 64, row, bh);
+          tma_load_3d(st + TILE, &maps.v, &kv_full[s], 0, row, bh);
+          tma_load_3d(st + TILE + HALF, &maps.v, &kv_full[s], 64, row, bh);
+        }
+      };
+      // the first item's first two tiles go out before the wait for the
+      // preceding kernels: they overlap that kernel's tail
+      int pre = 0;
+      if ((int)blockIdx.x < n_items) {
+        int bh, hb, grp;
+        decode(blockIdx.x, bh, hb, grp);
+        const int nt = group_tiles(grp);
+        const int n_all = nt + (a.queries ? nt : 0);
+        for (; pre < 2 && pre < n_all; ++pre, ++tile) issue_tile(tile, pre, nt, bh, grp);
+      }
+      pdl_wait();
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++item_ctr) {
         int bh, hb, grp;
         decode(item, bh, hb, grp);
@@ -163,17 +196,12 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         const int nt = group_tiles(grp);
         if (item_ctr >= 1 && !W.wait(w_empty, (item_ctr - 1) & 1, 1)) { ok = false; break; }
         // weights of the item: [W1_J; W3_J] as two K atoms (d 0-63, 64-127),
-        // W2[:, J] as 128 d-rows of 64 hidden units (and the lo copies)
+        // W2[:, J] as 128 d-rows of 64 hidden units
         mbar_arrive_expect_tx(w_full, 2 * HALF + 2 * 8192);
-        {
-          const CUtensorMap* m1 = &maps.w1;
-          const CUtensorMap* m3 = &maps.w3;
-          const CUtensorMap* m2 = &maps.w2;
-          for (int atom = 0; atom < 2; ++atom) {
-            tma_load_3d(smem + OFF_W13 + atom * HALF, m1, w_full, atom * 64, j0, bh);
-            tma_load_3d(smem + OFF_W13 + atom * HALF + HALF / 2, m3, w_full, atom * 64, j0, bh);
-            tma_load_3d(smem + OFF_W2 + atom * 8192, m2, w_full, j0, atom * 64, bh);
-          }
+        for (int atom = 0; atom < 2; ++atom) {
+          tma_load_3d(smem + OFF_W13 + atom * HALF, &maps.w1, w_full, atom * 64, j0, bh);
+          tma_load_3d(smem + OFF_W13 + atom * HALF + HALF / 2, &maps.w3, w_full, atom * 64, j0, bh);
+          tma_load_3d(smem + OFF_W2 + atom * 8192, &maps.w2, w_full, j0, atom * 64, bh);
         }
         // warm L2 with the item's later tiles; their loads then hit it
         for (int i = 2; i < nt; ++i)
@@ -183,23 +211,10 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
             tma_prefetch_l2_3d(&maps.v, h * 64, row, bh);
           }
         const int nq = a.queries ? nt : 0;
-        for (int i = 0; ok && i < nt + nq; ++i, ++tile) {
+        for (int i = item_ctr == 0 ? pre : 0; ok && i < nt + nq; ++i, ++tile) {
           const uint32_t s = tile & 1;
           if (tile >= 2 && !W.wait(&kv_empty[s], ((tile >> 1) - 1) & 1, 2)) { ok = false; break; }
-          const bool is_q = i >= nt;
-          const int row = a.t0 + (grp * a.tiles_per_group + (is_q ? i - nt : i)) * BM;
-          uint8_t* st = smem + OFF_KV + s * KV_STAGE;
-          if (is_q) {   // query tile in the K slot
-            mbar_arrive_expect_tx(&kv_full[s], TILE);
-            tma_load_3d(st, &maps.q, &kv_full[s], 0, row, bh);
-            tma_load_3d(st + HALF, &maps.q, &kv_full[s], 64, row, bh);
-          } else {
-            mbar_arrive_expect_tx(&kv_full[s], KV_STAGE);
-            tma_load_3d(st, &maps.k, &kv_full[s], 0, row, bh);
-            tma_load_3d(st + HALF, &maps.k, &kv_full[s], 64, row, bh);
-            tma_load_3d(st + TILE, &maps.v, &kv_full[s], 0, row, bh);
-            tma_load_3d(st + TILE + HALF, &maps.v, &kv_full[s], 64, row, bh);
-          }
+          issue_tile(tile, i, nt, bh, grp);
         }
       }
       if (W.aborted()) {
