@@ -85,7 +85,13 @@ typedef struct {
   ttt_dtype out_dtype;  /* out element type                                  */
 } ttt_linear_desc;
 
-/* Workspace bytes needed by ttt_linear_fwd (status word only). */
+/* Workspace bytes for ttt_linear_fwd at full speed: the status block, plus,
+ * on the tensor-core path (bf16, dk = dv = 64), room for the start states of
+ * the sequence segments that run on separate SMs (the state after a token is
+ * S0 plus the sum of the updates before it, so a head's sequence splits into
+ * segments whose start states a pre-pass sums).  The size depends on the
+ * device's SM count; a workspace of only TTT_STATUS_BYTES is accepted and
+ * runs each head unsplit. */
 int ttt_linear_workspace_bytes(const ttt_linear_desc* desc, size_t* bytes);
 
 /* S <- S0 (device float32 [B,H,dk,dv]); S0 == NULL zero-fills S. */
@@ -97,7 +103,10 @@ int ttt_linear_state_readout(const ttt_linear_desc* desc, const float* S, float*
 /* One call over N tokens.  q, k: [B,H,N,dk]; v: [B,H,N,dv]; lr: [B,H,N];
  * S: in = state before the first token, out = state after the last token;
  * out: [B,H,N,dv].  Supported: in_dtype F32 (any dk, dv <= 128) and BF16
- * (dk = dv = 64 on tensor cores; other dims <= 128 on CUDA cores). */
+ * (dk = dv = 64 on tensor cores; other dims <= 128 on CUDA cores).
+ * ws (>= TTT_STATUS_BYTES, device, caller-owned) holds the status block and
+ * the segment states (see ttt_linear_workspace_bytes); it must not be shared
+ * by calls that overlap in time. */
 int ttt_linear_fwd(const ttt_linear_desc* desc, const void* q, const void* k, const void* v,
                    const float* lr, float* S, void* out, void* ws, size_t ws_bytes, void* stream);
 

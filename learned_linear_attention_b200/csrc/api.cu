@@ -106,11 +106,26 @@ const char* ttt_build_info(void) {
 }
 
 // ------------------------------------------------------------------ linear
+static int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  return sms;
+}
+static bool linear_uses_umma(const ttt_linear_desc* d) {
+  return d->in_dtype == TTT_BF16 && d->dk == 64 && d->dv == 64;
+}
+
 int ttt_linear_workspace_bytes(const ttt_linear_desc* d, size_t* bytes) {
   int e = check_linear(d);
   if (e) return e;
   if (!bytes) return TTT_ERR_ARG;
-  *bytes = TTT_STATUS_BYTES;
+  size_t seg = 0;
+  if (linear_uses_umma(d)) seg = ttt_linear_plan(d->B * d->H, d->N, device_sms()).ws_floats * sizeof(float);
+  *bytes = TTT_STATUS_BYTES + seg;
   return TTT_OK;
 }
 
@@ -149,7 +164,12 @@ int ttt_linear_fwd(const ttt_linear_desc* d, const void* q, const void* k, const
   L.out_bf16 = d->out_dtype == TTT_BF16;
   L.q = q; L.k = k; L.v = v; L.lr = lr; L.S = S; L.out = out;
   L.st = status_of(ws, 1);
-  const bool umma = L.in_bf16 && d->dk == 64 && d->dv == 64;
+  const bool umma = linear_uses_umma(d);
+  if (umma) {
+    L.plan = ttt_linear_plan(d->B * d->H, d->N, device_sms());
+    L.seg_state = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + TTT_STATUS_BYTES);
+    L.seg_state_floats = (ws_bytes - TTT_STATUS_BYTES) / sizeof(float);
+  }
   const int r = umma ? launch_ttt_linear_umma(L, as_stream(stream))
                      : launch_ttt_linear_simt(L, as_stream(stream));
   return r == 0 ? TTT_OK : TTT_ERR_CUDA;

@@ -53,6 +53,12 @@ int make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t
                       uint32_t box_inner, uint32_t box_rows);
 
 // ----------------------------------------------------------------- TTT-linear
+// Sequence split of the tensor-core linear kernel (see ttt_linear.cu).
+struct LinearPlan {
+  int P, R, seg_tiles, unit_tiles;
+  size_t ws_floats;   // segment-state floats the split needs in the workspace
+};
+LinearPlan ttt_linear_plan(int BH, int N, int sms);
 struct LinearLaunch {
   int B, H, N, dk, dv, chunk, include_diag;
   int in_bf16, out_bf16;
@@ -61,6 +67,9 @@ struct LinearLaunch {
   float* S;
   void* out;
   DevStatus st;
+  LinearPlan plan;
+  float* seg_state;           // workspace after the status block
+  size_t seg_state_floats;
 };
 int launch_ttt_linear_simt(const LinearLaunch& L, cudaStream_t stream);
 int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream);
@@ -116,7 +125,7 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream);
 // ----------------------------------------------------------------- profiling
 enum KernelKind {
   K_LIN_SIMT, K_LIN_UMMA, K_LACT_CAST, K_KEYPASS, K_GEMM_READ, K_GEMM_GRAD, K_UPDATE,
-  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_NUM
+  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_LIN_SEG, K_NUM
 };
 void prof_before(int kind, cudaStream_t s);
 void prof_after(int kind, cudaStream_t s);

@@ -11,7 +11,8 @@ namespace ttt {
 static const char* kKindNames[K_NUM] = {
     "ttt_linear_simt", "ttt_linear_umma", "lact_cast",     "lact_keypass",
     "gemm_read",       "gemm_grad",       "lact_update",   "muon_momentum",
-    "ns_prep",         "gemm_ns",         "muon_apply",    "lact_keygrad"};
+    "ns_prep",         "gemm_ns",         "muon_apply",    "lact_keygrad",
+    "ttt_linear_segstate"};
 
 struct ProfRec {
   int kind;

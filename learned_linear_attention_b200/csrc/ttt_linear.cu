@@ -15,6 +15,8 @@
 //    whole sequence, causal mask and per-token lr applied by the epilogue
 //    warps between the MMAs.
 #include "common.cuh"
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace ttt {
@@ -156,6 +158,12 @@ struct LinUmmaArgs {
   int include_diag;
   int out_bf16;
   DevStatus st;
+  // Sequence split: CTA (bh, p) takes tiles [p seg_tiles, (p + 1) seg_tiles)
+  // of head bh.  With P > 1 its start state is S0 (copied to seg_state by
+  // the pre-pass) plus the state increments of the R units of every
+  // earlier segment, and only the last segment writes S.
+  int P, R, seg_tiles;
+  const float* seg_state;   // [BH][1 + (P - 1) R][64][64]: S0, then the units' increments
 };
 
 __global__ void __launch_bounds__(lin::THREADS, 1)
@@ -176,8 +184,9 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
   uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int n_tiles = (a.N + T - 1) / T;
+  const int bh = blockIdx.x / a.P, seg = blockIdx.x % a.P;
+  const int t_first = seg * a.seg_tiles;   // first tile of this CTA's segment
+  const int n_tiles = max(0, min(a.seg_tiles, (a.N + T - 1) / T - t_first));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -215,9 +224,9 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
         if (i >= STAGES && !W.wait(&empty[s], ((i >> 1) - 1) & 1, 1)) break;
         uint8_t* st = smem + OFF_STAGE + s * STAGE_BYTES;
         mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-        tma_load_3d(st, &mapQ, &full[s], 0, i * T, bh);
-        tma_load_3d(st + TILE_BYTES, &mapK, &full[s], 0, i * T, bh);
-        tma_load_3d(st + 2 * TILE_BYTES, &mapV, &full[s], 0, i * T, bh);
+        tma_load_3d(st, &mapQ, &full[s], 0, (t_first + i) * T, bh);
+        tma_load_3d(st + TILE_BYTES, &mapK, &full[s], 0, (t_first + i) * T, bh);
+        tma_load_3d(st + 2 * TILE_BYTES, &mapV, &full[s], 0, (t_first + i) * T, bh);
         issued = i + 1;
       }
       if (W.aborted()) {  // drain the copies still in flight into our smem
@@ -302,8 +311,18 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     const int srow = q4 * 16 + lane;
     {
       float vals[32];
+      if (a.P == 1) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) vals[j] = s_owner ? Sg[srow * D + hf * 32 + j] : 0.f;
+        for (int j = 0; j < 32; ++j) vals[j] = s_owner ? Sg[srow * D + hf * 32 + j] : 0.f;
+      } else {   // S0 + the increments of the earlier segments' units, in order
+        const int nu = 1 + seg * a.R;
+        const float* ss = a.seg_state + (size_t)bh * (1 + (a.P - 1) * a.R) * D * D + srow * D + hf * 32;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) vals[j] = 0.f;
+        for (int u = 0; u < nu; ++u)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) vals[j] += s_owner ? ss[(size_t)u * D * D + j] : 0.f;
+      }
       tmem_st16(tmem + lane_base + TM_S + hf * 32, vals);
       tmem_st16(tmem + lane_base + TM_S + hf * 32 + 16, vals + 16);
       if (s_owner) {
@@ -315,7 +334,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       }
     }
     auto store_out = [&](int tile) {
-      const int t = tile * T + r;
+      const int t = (t_first + tile) * T + r;
       float o[32];
       tmem_ld32(tmem + lane_base + ((tile & 1) ? TM_O1 : TM_O0) + hf * 32, o);
       if (t < a.N) {
@@ -338,7 +357,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       const int s = i & 1;
       if (!W.wait(&pfull[s], (i >> 1) & 1, 5)) { ok = false; break; }
       tc_fence_after();
-      const int t = i * T + r;
+      const int t = (t_first + i) * T + r;
       const float eta = (t < a.N) ? lrg[t] : 0.f;
       // eta * V  -> EV[s]  (same swizzled layout as the TMA-loaded V tile)
       {
@@ -402,7 +421,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       store_out(n_tiles - 1);
       float sv[32];
       tmem_ld32(tmem + lane_base + TM_S + hf * 32, sv);
-      if (s_owner) {
+      if (s_owner && seg == a.P - 1) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) Sg[srow * D + hf * 32 + j] = sv[j];
       }
@@ -416,6 +435,199 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
   }
 }
 
+// =====================================================================
+// sequence split: state increments of the earlier segments
+// =====================================================================
+// Causal linear attention is a prefix scan of S (the state after a token is
+// S0 plus the sum of eta k v^T before it), so a head's sequence can be cut
+// into segments that run on different SMs once each knows its start state.
+// This pre-pass forms, per unit of tiles of every segment but the last,
+// dS_u = sum_t k_t^T (eta_t v_t) with the same bf16 operands and fp32
+// tensor-core accumulation as the main kernel, and copies S0 beside them.
+namespace lss {
+constexpr int T = 128, D = 64;
+constexpr int EPI_WARPS = 4;
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr uint32_t TILE = T * D * 2;                 // 16 KB
+constexpr uint32_t STAGE = 2 * TILE;                 // K, V
+constexpr int STAGES = 3;
+constexpr uint32_t OFF_EV = STAGES * STAGE;          // 2 x 16 KB (eta V, bf16)
+constexpr uint32_t OFF_BAR = OFF_EV + 2 * TILE;
+constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+constexpr uint32_t TM_S = 0, TM_COLS = 64;
+}  // namespace lss
+
+struct SegStateArgs {
+  const float* lr;
+  const float* S0;    // [BH][64][64]
+  float* seg_state;   // [BH][1 + U][64][64]
+  int N, U, R, seg_tiles, unit_tiles;
+  DevStatus st;
+};
+
+__global__ void __launch_bounds__(lss::THREADS, 1)
+    ttt_linear_segstate_kernel(const __grid_constant__ CUtensorMap mapK,
+                               const __grid_constant__ CUtensorMap mapV, SegStateArgs a) {
+  using namespace lss;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);   // [STAGES]
+  uint64_t* empty = full + STAGES;                                  // [STAGES]
+  uint64_t* evfull = empty + STAGES;                                // [2]
+  uint64_t* evempty = evfull + 2;                                   // [2]
+  uint64_t* fin = evempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x / a.U, u = blockIdx.x % a.U;
+  const int p = u / a.R, rr = u % a.R;
+  const int total = (a.N + T - 1) / T;
+  const int t0 = p * a.seg_tiles + rr * a.unit_tiles;
+  const int t1 = min(min(t0 + a.unit_tiles, (p + 1) * a.seg_tiles), total);
+  const int nt = max(0, t1 - t0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&evfull[s], EPI_WARPS * 32);
+      mbar_init(&evempty[s], 1);
+    }
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  Waiter W{abort_flag, a.st, 600};
+  float* out = a.seg_state + (size_t)bh * (1 + a.U) * D * D;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nt; ++i) {
+        const int s = i % STAGES;
+        if (i >= STAGES && !W.wait(&empty[s], ((i / STAGES) - 1) & 1, 1)) break;
+        uint8_t* st = smem + s * STAGE;
+        mbar_arrive_expect_tx(&full[s], STAGE);
+        tma_load_3d(st, &mapK, &full[s], 0, (t0 + i) * T, bh);
+        tma_load_3d(st + TILE, &mapV, &full[s], 0, (t0 + i) * T, bh);
+        issued = i + 1;
+      }
+      if (W.aborted())
+        for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+          W.drain(&full[i % STAGES], (i / STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = make_idesc(64, 64, true, true);
+      for (int i = 0; i < nt; ++i) {
+        const int s = i % STAGES, e = i & 1;
+        if (!W.wait(&evfull[e], (i >> 1) & 1, 2)) break;
+        tc_fence_after();
+        const uint32_t ks = smem_u32(smem + s * STAGE);
+        const uint32_t ev = smem_u32(smem + OFF_EV + e * TILE);
+        // S += K^T (eta V): M = 64 (d), K = 128 tokens, N = 64
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + TM_S, make_sdesc(ks + kk * 2048, 8192, 1024),
+                   make_sdesc(ev + kk * 2048, 8192, 1024), id_s, (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&empty[s]);
+        mma_commit(&evempty[e]);
+      }
+      mma_commit(fin);
+      W.drain(fin, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue: eta V
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;   // token row of the tile
+    const float* lrg = a.lr + (size_t)bh * a.N;
+    bool ok = true;
+    for (int i = 0; i < nt; ++i) {
+      const int s = i % STAGES, e = i & 1;
+      const int t = (t0 + i) * T + r;
+      const float eta = t < a.N ? lrg[t] : 0.f;
+      if (!W.wait(&full[s], (i / STAGES) & 1, 3)) { ok = false; break; }
+      if (i >= 2 && !W.wait(&evempty[e], ((i >> 1) - 1) & 1, 4)) { ok = false; break; }
+      const uint32_t vsrc = smem_u32(smem + s * STAGE + TILE);
+      const uint32_t evdst = smem_u32(smem + OFF_EV + e * TILE);
+#pragma unroll
+      for (int j = 0; j < 64; j += 8) {
+        const uint32_t off = sw128_offset(r, j);
+        uint32_t w0, w1, w2, w3;
+        ld_shared_v4(vsrc + off, w0, w1, w2, w3);
+        st_shared_v4(evdst + off, pack_bf16x2(eta * bf16lo(w0), eta * bf16hi(w0)),
+                     pack_bf16x2(eta * bf16lo(w1), eta * bf16hi(w1)),
+                     pack_bf16x2(eta * bf16lo(w2), eta * bf16hi(w2)),
+                     pack_bf16x2(eta * bf16lo(w3), eta * bf16hi(w3)));
+      }
+      fence_async_smem();
+      mbar_arrive(&evfull[e]);
+    }
+    // increment of the unit (rows of the M = 64 accumulator: lanes 0-15 of
+    // quadrant q4 hold rows 16 q4 + lane)
+    if (ok && W.wait(fin, 0, 5)) {
+      tc_fence_after();
+      const int srow = q4 * 16 + lane;
+      float sv[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + TM_S + h * 32, sv);
+        if (lane < 16) {
+          float* dst = out + (size_t)(1 + u) * D * D + srow * D + h * 32;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + j) =
+                nt > 0 ? make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    }
+    // the first unit of the head also copies S0 beside the increments
+    if (u == 0) {
+      const float4* src = reinterpret_cast<const float4*>(a.S0 + (size_t)bh * D * D);
+      float4* dst = reinterpret_cast<float4*>(out);
+      for (int k = threadIdx.x - 64; k < D * D / 4; k += EPI_WARPS * 32) dst[k] = src[k];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
+// Segments per head P, units per segment R, tiles per segment and per unit.
+// P fills the SMs with one CTA per (head, segment) (at least 8 tiles per
+// segment); the pre-pass fills them again with (head, unit) CTAs.
+LinearPlan ttt_linear_plan(int BH, int N, int sms) {
+  LinearPlan pl{};
+  const int total = (N + 127) / 128;
+  pl.P = std::max(1, std::min(std::min(8, sms / std::max(1, BH)), total / 8));
+  pl.seg_tiles = (total + pl.P - 1) / std::max(1, pl.P);
+  if (pl.seg_tiles < 1) pl.seg_tiles = 1;
+  pl.P = std::max(1, (total + pl.seg_tiles - 1) / pl.seg_tiles);
+  pl.R = 1;
+  if (pl.P > 1) pl.R = std::max(1, std::min(std::min(8, sms / (BH * (pl.P - 1))), pl.seg_tiles / 4));
+  pl.unit_tiles = (pl.seg_tiles + pl.R - 1) / pl.R;
+  pl.ws_floats = pl.P > 1 ? (size_t)BH * (1 + (size_t)(pl.P - 1) * pl.R) * 64 * 64 : 0;
+  return pl;
+}
+
 int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   const uint64_t BH = (uint64_t)L.B * L.H;
@@ -423,12 +635,36 @@ int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream) {
       make_tmap_bf16_3d(&mk, L.k, 64, L.N, BH, 64 * 2, (uint64_t)L.N * 64 * 2, 64, 128) ||
       make_tmap_bf16_3d(&mv, L.v, 64, L.N, BH, 64 * 2, (uint64_t)L.N * 64 * 2, 64, 128))
     return -1;
-  LinUmmaArgs a{L.lr, L.S, L.out, L.N, L.include_diag, L.out_bf16, L.st};
-  if (cudaFuncSetAttribute(ttt_linear_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)lin::SMEM_BYTES) != cudaSuccess)
-    return -1;
+  LinearPlan pl = L.plan;
+  if (pl.P > 1 && (L.seg_state == nullptr || L.seg_state_floats < pl.ws_floats)) {
+    pl.P = 1;   // no room for the segment states: one CTA per head
+    pl.seg_tiles = (L.N + 127) / 128;
+  }
+  LinUmmaArgs a{L.lr, L.S, L.out, L.N, L.include_diag, L.out_bf16, L.st,
+                pl.P, pl.R, pl.seg_tiles, L.seg_state};
+  if (pl.P > 1) {
+    SegStateArgs sa{L.lr, L.S, L.seg_state, L.N, (pl.P - 1) * pl.R, pl.R, pl.seg_tiles, pl.unit_tiles, L.st};
+    static bool ss_attr = false;
+    if (!ss_attr) {
+      if (cudaFuncSetAttribute(ttt_linear_segstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)lss::SMEM) != cudaSuccess)
+        return -1;
+      ss_attr = true;
+    }
+    prof_before(K_LIN_SEG, stream);
+    ttt_linear_segstate_kernel<<<dim3((unsigned)(BH * sa.U)), dim3(lss::THREADS), lss::SMEM, stream>>>(
+        mk, mv, sa);
+    prof_after(K_LIN_SEG, stream);
+  }
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(ttt_linear_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)lin::SMEM_BYTES) != cudaSuccess)
+      return -1;
+    attr = true;
+  }
   prof_before(K_LIN_UMMA, stream);
-  ttt_linear_umma_kernel<<<dim3((unsigned)BH), dim3(lin::THREADS), lin::SMEM_BYTES, stream>>>(
+  ttt_linear_umma_kernel<<<dim3((unsigned)(BH * pl.P)), dim3(lin::THREADS), lin::SMEM_BYTES, stream>>>(
       mq, mk, mv, a);
   prof_after(K_LIN_UMMA, stream);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;

@@ -22,7 +22,8 @@ def rel_err(a, ref):
     return float(np.abs(a - ref).max() / max(np.abs(ref).max(), 1e-300))
 
 
-def run_linear(x, include_diag=True, out_dtype="f32", S0=None, chunk=None, stream=None):
+def run_linear(x, include_diag=True, out_dtype="f32", S0=None, chunk=None, stream=None,
+               ws_bytes=None):
     B, H, N, dk = x.q.values.shape
     dv = x.v.values.shape[-1]
     desc = T.make_linear_desc(B, H, N, dk, dv, chunk or x.chunk, include_diag,
@@ -34,7 +35,7 @@ def run_linear(x, include_diag=True, out_dtype="f32", S0=None, chunk=None, strea
         S.copy_(torch.from_numpy(np.asarray(S0, dtype=np.float32)))
     odt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
     out = torch.full((B, H, N, dv), float("nan"), dtype=odt, device="cuda")
-    ws = T.alloc_workspace(T.ttt_linear_workspace_bytes(desc))
+    ws = T.alloc_workspace(ws_bytes or T.ttt_linear_workspace_bytes(desc))
     T.ttt_linear_fwd(desc, q, k, v, lr, S, out, ws, stream=stream)
     assert T.ttt_check_device_status(ws, stream) == T.TTT_OK
     return out.float().cpu().numpy(), S.cpu().numpy()

@@ -51,6 +51,32 @@ def test_bf16_tensor_core_kernel(cuda_device, include_diag, N):
     assert rel_err(S, Sref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("include_diag", [True, False])
+def test_bf16_sequence_split_matches_oracle(cuda_device, include_diag):
+    """5000 tokens over 3 heads: each head's 40 tiles run as 5 segments on
+    separate SMs, their start states summed by the segment pre-pass from S0
+    and the earlier segments' increments; the last tile is ragged."""
+    x = make_linear_inputs(1, 3, 5000, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=19,
+                           with_S0=True)
+    out, S = run_linear(x, include_diag, S0=x.S0)
+    ref, Sref = _oracle(x, include_diag, x.S0)
+    assert not np.isnan(out).any()
+    assert rel_err(out, ref) <= TOL_BF16
+    assert rel_err(S, Sref) <= TOL_BF16
+
+
+def test_bf16_split_and_unsplit_agree(cuda_device):
+    """A workspace of only the status block runs every head unsplit; the
+    split run differs from it by fp32 summation order and the bf16 rounding
+    of the segments' start states only."""
+    x = make_linear_inputs(2, 2, 4096, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=20,
+                           with_S0=True)
+    o_split, S_split = run_linear(x, S0=x.S0)
+    o_one, S_one = run_linear(x, S0=x.S0, ws_bytes=T.TTT_STATUS_BYTES)
+    assert rel_err(o_split, o_one) <= 1e-2
+    assert rel_err(S_split, S_one) <= 1e-5
+
+
 def test_bf16_output_dtype(cuda_device):
     x = make_linear_inputs(1, 2, 400, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=13)
     out, _ = run_linear(x, out_dtype="bf16")
