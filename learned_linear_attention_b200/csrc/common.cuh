@@ -63,6 +63,20 @@ TTT_DEVICE_INLINE bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase (no suspend): for issuers that poll several
+// barriers and act on whichever is ready.
+TTT_DEVICE_INLINE bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Per-CTA abort flag lives in shared memory; once any thread of the CTA gives
 // up on a wait, every later wait of the CTA returns false immediately so that
 // all roles drain to the common teardown.

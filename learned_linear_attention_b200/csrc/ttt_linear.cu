@@ -236,6 +236,10 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // It polls the next tile's QK^T product (its Q/K tiles landed, its P
+    // buffer was read by the epilogue two tiles back) and the current tile's
+    // O and S products (the epilogue staged its operands) and issues
+    // whichever can go, so the O/S chain never waits for a tile load.
     if (lane == 0 && n_tiles > 0) {
       const uint32_t id_qk = make_idesc(128, 128, false, false);
       const uint32_t id_o = make_idesc(128, 64, false, true);
@@ -243,32 +247,19 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       const uint32_t pt_base = smem_u32(smem + OFF_PT);
       const uint32_t ev_base = smem_u32(smem + OFF_EV);
       const uint32_t sb_base = smem_u32(smem + OFF_SB);
-      bool ok = W.wait(&full[0], 0, 2);
-      if (ok) {
+      auto issue_p = [&](int i) {
         tc_fence_after();
-        const uint32_t qs = smem_u32(smem + OFF_STAGE), ks = qs + TILE_BYTES;
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + TM_P0, make_sdesc(qs + kk * 32, 16, 1024),
-                   make_sdesc(ks + kk * 32, 16, 1024), id_qk, kk > 0);
-        mma_commit(&pfull[0]);
-      }
-      for (int i = 0; ok && i < n_tiles; ++i) {
         const int s = i & 1;
-        // P of the next tile first: the epilogue converts it while this
-        // tile's O and S products run.
-        if (i + 1 < n_tiles) {
-          const int s1 = (i + 1) & 1;
-          if (!W.wait(&full[s1], ((i + 1) >> 1) & 1, 4)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t qs1 = smem_u32(smem + OFF_STAGE + s1 * STAGE_BYTES);
-          const uint32_t ks1 = qs1 + TILE_BYTES;
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + (s1 ? TM_P1 : TM_P0), make_sdesc(qs1 + kk * 32, 16, 1024),
-                     make_sdesc(ks1 + kk * 32, 16, 1024), id_qk, kk > 0);
-          mma_commit(&pfull[s1]);
-        }
-        if (!W.wait(ops, i & 1, 3)) { ok = false; break; }
+        const uint32_t qs = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES);
+        const uint32_t ks = qs + TILE_BYTES;
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + (s ? TM_P1 : TM_P0), make_sdesc(qs + kk * 32, 16, 1024),
+                   make_sdesc(ks + kk * 32, 16, 1024), id_qk, kk > 0);
+        mma_commit(&pfull[s]);
+      };
+      auto issue_o = [&](int i) {
         tc_fence_after();
+        const int s = i & 1;
         const uint32_t qs = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES);
         const uint32_t ks = qs + TILE_BYTES;
         const uint32_t pt = pt_base + s * 2 * TILE_BYTES;
@@ -290,8 +281,34 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
                    make_sdesc(ev + kk * 2048, 8192, 1024), id_s, 1);
         mma_commit(ofull);
         mma_commit(&empty[s]);
+      };
+      int np = 0, no = 0;   // QK^T products / O and S products issued
+      uint64_t t_idle = 0;
+      uint32_t spins = 0;
+      while (no < n_tiles) {
+        bool prog = false;
+        if (no < np && mbar_test(ops, no & 1)) {
+          issue_o(no);
+          ++no;
+          prog = true;
+        }
+        if (np < n_tiles && np <= no + 1 && mbar_test(&full[np & 1], (np >> 1) & 1)) {
+          issue_p(np);
+          ++np;
+          prog = true;
+        }
+        if (prog) {
+          spins = 0;
+          t_idle = 0;
+          continue;
+        }
+        if ((++spins & 255u) == 0u) {   // bounded: give up after the wait timeout
+          if (W.aborted()) break;
+          const uint64_t now = globaltimer_ns();
+          if (t_idle == 0) t_idle = now;
+          else if (now - t_idle > W.st.timeout_ns) { W.fail(3); break; }
+        }
       }
-      (void)ok;
     }
     if (lane == 0) {  // every MMA issued by this thread completes before teardown
       mma_commit(fin);
