@@ -139,11 +139,15 @@ constexpr int NUM_EPI_WARPS = 8;
 constexpr int THREADS = (2 + NUM_EPI_WARPS) * 32;
 constexpr uint32_t TILE_BYTES = T * D * 2;          // 16 KB (Q, K, V, eta*V tiles)
 constexpr uint32_t STAGE_BYTES = 3 * TILE_BYTES;    // Q, K, V
-constexpr int STAGES = 2;
+// Three Q/K/V stages keep about two tiles of loads in flight per SM; the
+// masked P and eta V operands are single-buffered: the epilogue builds the
+// next tile's in registers while this tile's products run and stores them
+// once those products are done.
+constexpr int STAGES = 3;
 constexpr uint32_t OFF_STAGE = 0;
-constexpr uint32_t OFF_PT = OFF_STAGE + STAGES * STAGE_BYTES;      // 2 x 32 KB (masked P, bf16)
-constexpr uint32_t OFF_EV = OFF_PT + 2 * 2 * TILE_BYTES;          // 2 x 16 KB (eta*V, bf16)
-constexpr uint32_t OFF_SB = OFF_EV + 2 * TILE_BYTES;              // 8 KB (S, bf16)
+constexpr uint32_t OFF_PT = OFF_STAGE + STAGES * STAGE_BYTES;      // 32 KB (masked P, bf16)
+constexpr uint32_t OFF_EV = OFF_PT + 2 * TILE_BYTES;              // 16 KB (eta*V, bf16)
+constexpr uint32_t OFF_SB = OFF_EV + TILE_BYTES;                  // 8 KB (S, bf16)
 constexpr uint32_t OFF_BAR = OFF_SB + D * D * 2;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;             // + alignment slack
 // TMEM columns
@@ -174,9 +178,9 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);   // [2]
-  uint64_t* empty = full + 2;                                       // [2]
-  uint64_t* pfull = empty + 2;                                      // [2]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);   // [STAGES]
+  uint64_t* empty = full + STAGES;                                  // [STAGES]
+  uint64_t* pfull = empty + STAGES;                                 // [2]: per P buffer
   uint64_t* ops = pfull + 2;                                        // [1]
   uint64_t* ofull = ops + 1;                                        // [1]
   uint64_t* fin = ofull + 1;                                        // [1]
@@ -189,11 +193,11 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
   const int n_tiles = max(0, min(a.seg_tiles, (a.N + T - 1) / T - t_first));
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&pfull[s], 1);
     }
+    for (int s = 0; s < 2; ++s) mbar_init(&pfull[s], 1);
     mbar_init(ops, NUM_EPI_WARPS * 32);
     mbar_init(ofull, 1);
     mbar_init(fin, 1);
@@ -220,8 +224,8 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < n_tiles; ++i) {
-        const int s = i & 1;
-        if (i >= STAGES && !W.wait(&empty[s], ((i >> 1) - 1) & 1, 1)) break;
+        const int s = i % STAGES;
+        if (i >= STAGES && !W.wait(&empty[s], ((i / STAGES) - 1) & 1, 1)) break;
         uint8_t* st = smem + OFF_STAGE + s * STAGE_BYTES;
         mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
         tma_load_3d(st, &mapQ, &full[s], 0, (t_first + i) * T, bh);
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       }
       if (W.aborted()) {  // drain the copies still in flight into our smem
         for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; ++i)
-          W.drain(&full[i & 1], (i >> 1) & 1);
+          W.drain(&full[i % STAGES], (i / STAGES) & 1);
       }
     }
   } else if (warp == 1) {
@@ -249,25 +253,25 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       const uint32_t sb_base = smem_u32(smem + OFF_SB);
       auto issue_p = [&](int i) {
         tc_fence_after();
-        const int s = i & 1;
+        const int s = i % STAGES, pb = i & 1;
         const uint32_t qs = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES);
         const uint32_t ks = qs + TILE_BYTES;
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + (s ? TM_P1 : TM_P0), make_sdesc(qs + kk * 32, 16, 1024),
+          mma_bf16(tmem + (pb ? TM_P1 : TM_P0), make_sdesc(qs + kk * 32, 16, 1024),
                    make_sdesc(ks + kk * 32, 16, 1024), id_qk, kk > 0);
-        mma_commit(&pfull[s]);
+        mma_commit(&pfull[pb]);
       };
       auto issue_o = [&](int i) {
         tc_fence_after();
-        const int s = i & 1;
+        const int s = i % STAGES;
         const uint32_t qs = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES);
         const uint32_t ks = qs + TILE_BYTES;
-        const uint32_t pt = pt_base + s * 2 * TILE_BYTES;
-        const uint32_t ev = ev_base + s * TILE_BYTES;
+        const uint32_t pt = pt_base;
+        const uint32_t ev = ev_base;
         // O = mask(P) (eta V): K = 128 keys, two 64-key atoms of the P tile.
         // O alternates between two TMEM buffers so the epilogue can store the
         // previous tile's O while this tile's products run.
-        const uint32_t tm_o = s ? TM_O1 : TM_O0;
+        const uint32_t tm_o = (i & 1) ? TM_O1 : TM_O0;
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + tm_o, make_sdesc(pt + (kk >> 2) * TILE_BYTES + (kk & 3) * 32, 16, 1024),
                    make_sdesc(ev + kk * 2048, 8192, 1024), id_o, kk > 0);
@@ -292,7 +296,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
           ++no;
           prog = true;
         }
-        if (np < n_tiles && np <= no + 1 && mbar_test(&full[np & 1], (np >> 1) & 1)) {
+        if (np < n_tiles && np <= no + 1 && mbar_test(&full[np % STAGES], (np / STAGES) & 1)) {
           issue_p(np);
           ++np;
           prog = true;
@@ -371,60 +375,70 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     };
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
-      const int s = i & 1;
-      if (!W.wait(&pfull[s], (i >> 1) & 1, 5)) { ok = false; break; }
+      const int s = i % STAGES, pb = i & 1;
+      if (!W.wait(&pfull[pb], (i >> 1) & 1, 5)) { ok = false; break; }
       tc_fence_after();
       const int t = (t_first + i) * T + r;
       const float eta = (t < a.N) ? lrg[t] : 0.f;
-      // eta * V  -> EV[s]  (same swizzled layout as the TMA-loaded V tile)
+      // eta * V of this row's 32 columns (bf16 pairs), from the stage
+      uint32_t evr[16];
       {
         const uint32_t vsrc = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES + 2 * TILE_BYTES);
-        const uint32_t evdst = smem_u32(smem + OFF_EV + s * TILE_BYTES);
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          const uint32_t off = sw128_offset(r, hf * 32 + j);
+        for (int j = 0; j < 4; ++j) {
           uint32_t w0, w1, w2, w3;
-          ld_shared_v4(vsrc + off, w0, w1, w2, w3);
-          st_shared_v4(evdst + off, pack_bf16x2(eta * bf16lo(w0), eta * bf16hi(w0)),
-                       pack_bf16x2(eta * bf16lo(w1), eta * bf16hi(w1)),
-                       pack_bf16x2(eta * bf16lo(w2), eta * bf16hi(w2)),
-                       pack_bf16x2(eta * bf16lo(w3), eta * bf16hi(w3)));
+          ld_shared_v4(vsrc + sw128_offset(r, hf * 32 + 8 * j), w0, w1, w2, w3);
+          evr[4 * j] = pack_bf16x2(eta * bf16lo(w0), eta * bf16hi(w0));
+          evr[4 * j + 1] = pack_bf16x2(eta * bf16lo(w1), eta * bf16hi(w1));
+          evr[4 * j + 2] = pack_bf16x2(eta * bf16lo(w2), eta * bf16hi(w2));
+          evr[4 * j + 3] = pack_bf16x2(eta * bf16lo(w3), eta * bf16hi(w3));
         }
       }
-      // masked P -> Pt[s] (keys hf*64 .. hf*64+63 form atom hf)
+      // masked P of this row's 64 keys hf*64 .. hf*64+63 (bf16 pairs)
+      uint32_t pr[32];
       {
-        const uint32_t pdst = smem_u32(smem + OFF_PT + s * 2 * TILE_BYTES + hf * TILE_BYTES);
-        const uint32_t pcol = (s ? TM_P1 : TM_P0) + hf * 64;
+        const uint32_t pcol = (pb ? TM_P1 : TM_P0) + hf * 64;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           float p[32];
           tmem_ld32(tmem + lane_base + pcol + h2 * 32, p);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 32; j += 2) {
             const int key = hf * 64 + h2 * 32 + j;
-            const bool keep = a.include_diag ? (key <= r) : (key < r);
-            p[j] = keep ? p[j] : 0.f;
+            const bool k0 = a.include_diag ? (key <= r) : (key < r);
+            const bool k1 = a.include_diag ? (key + 1 <= r) : (key + 1 < r);
+            pr[h2 * 16 + j / 2] = pack_bf16x2(k0 ? p[j] : 0.f, k1 ? p[j + 1] : 0.f);
           }
-#pragma unroll
-          for (int j = 0; j < 32; j += 8)
-            st_shared_v4(pdst + sw128_offset(r, h2 * 32 + j), pack_bf16x2(p[j], p[j + 1]),
-                         pack_bf16x2(p[j + 2], p[j + 3]), pack_bf16x2(p[j + 4], p[j + 5]),
-                         pack_bf16x2(p[j + 6], p[j + 7]));
         }
       }
+      // the previous tile's products are done with the single P, eta V and
+      // S operand buffers; S after tile i-1 becomes tile i's operand
+      float sv[32];
       if (i > 0) {
         if (!W.wait(ofull, (i - 1) & 1, 6)) { ok = false; break; }
         tc_fence_after();
-        // S after tile i-1 -> bf16 operand copy for tile i
-        float sv[32];
         tmem_ld32(tmem + lane_base + TM_S + hf * 32, sv);
-        if (s_owner) {
+      }
+      {
+        const uint32_t evdst = smem_u32(smem + OFF_EV);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          st_shared_v4(evdst + sw128_offset(r, hf * 32 + 8 * j), evr[4 * j], evr[4 * j + 1],
+                       evr[4 * j + 2], evr[4 * j + 3]);
+        const uint32_t pdst = smem_u32(smem + OFF_PT + hf * TILE_BYTES);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
           for (int j = 0; j < 32; j += 8)
-            st_shared_v4(smem_u32(sb) + sw128_offset(srow, hf * 32 + j),
-                         pack_bf16x2(sv[j], sv[j + 1]), pack_bf16x2(sv[j + 2], sv[j + 3]),
-                         pack_bf16x2(sv[j + 4], sv[j + 5]), pack_bf16x2(sv[j + 6], sv[j + 7]));
-        }
+            st_shared_v4(pdst + sw128_offset(r, h2 * 32 + j), pr[h2 * 16 + j / 2], pr[h2 * 16 + j / 2 + 1],
+                         pr[h2 * 16 + j / 2 + 2], pr[h2 * 16 + j / 2 + 3]);
+      }
+      if (i > 0 && s_owner) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 8)
+          st_shared_v4(smem_u32(sb) + sw128_offset(srow, hf * 32 + j),
+                       pack_bf16x2(sv[j], sv[j + 1]), pack_bf16x2(sv[j + 2], sv[j + 3]),
+                       pack_bf16x2(sv[j + 4], sv[j + 5]), pack_bf16x2(sv[j + 6], sv[j + 7]));
       }
       fence_async_smem();
       tc_fence_before();
@@ -467,7 +481,7 @@ constexpr int EPI_WARPS = 4;
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
 constexpr uint32_t TILE = T * D * 2;                 // 16 KB
 constexpr uint32_t STAGE = 2 * TILE;                 // K, V
-constexpr int STAGES = 3;
+constexpr int STAGES = 5;                            // ~128 KB of loads in flight per SM
 constexpr uint32_t OFF_EV = STAGES * STAGE;          // 2 x 16 KB (eta V, bf16)
 constexpr uint32_t OFF_BAR = OFF_EV + 2 * TILE;
 constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
