@@ -45,7 +45,6 @@ struct KeyGradArgs {
   int n_hb, n_groups, tiles_total, tiles_per_group;
   const float* lr;
   float* part[3];        // [group][BH][rows][cols] partial gradients (G1, G3, G2)
-  int split;             // exact sigmoid (split-operand mode) instead of tanh.approx
   int queries;           // causal order: also form Aq = silu(Q W1^T) (Q W3^T) for the tiles
   __nv_bfloat16* Aq;     // [BH][cmax][dh] (queries)
   long long aq_bs;       // cmax * dh
@@ -62,7 +61,6 @@ TTT_DEVICE_INLINE void tma_prefetch_l2_3d(const CUtensorMap* m, int x, int y, in
                : "memory");
 }
 
-TTT_DEVICE_INLINE float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 TTT_DEVICE_INLINE float sigmoid_tanh(float x) {
   float t;
   asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
@@ -343,7 +341,9 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
       for (int i = 0; i < nt; ++i, ++tile, ++ktile) {
         const int tc = (grp * a.tiles_per_group + i) * BM + r;   // token row in the chunk
         const bool valid = tc < a.C;
-        const float eta = valid ? a.lr[(size_t)bh * a.lr_len + a.t0 + tc] : 0.f;
+        // -eta, zero for rows past the chunk (their H and dGr are finite, so
+        // every gradient operand of such a row comes out zero)
+        const float neta = valid ? -a.lr[(size_t)bh * a.lr_len + a.t0 + tc] : 0.f;
         if (!W.wait(&acc_full[tile & 1], (tile >> 1) & 1, 8)) { ok = false; break; }
         tc_fence_after();
         uint32_t rh1[CW], rh3[CW], rg[CW];
@@ -361,13 +361,15 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
           float r1[2], r3[2], rm[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
+            // dG = -eta dGr;  dH3 = dG silu(x) = (dG sg) x;
+            // dH1 = dG y silu'(x) = (dG sg) y (1 + x (1 - sg));  Gm' = -eta silu(x) y
             const float x = __uint_as_float(rh1[j + u]), y = __uint_as_float(rh3[j + u]);
-            const float sg = a.split ? sigmoid_fast(x) : sigmoid_tanh(x);
-            const float act = x * sg;
-            const float dg = valid ? -eta * __uint_as_float(rg[j + u]) : 0.f;
-            r3[u] = dg * act;
-            r1[u] = dg * y * (sg * (1.f + x * (1.f - sg)));
-            rm[u] = valid ? -eta * act * y : 0.f;
+            const float sg = sigmoid_tanh(x);
+            const float p = neta * __uint_as_float(rg[j + u]) * sg;
+            const float py = p * y;
+            r3[u] = p * x;
+            r1[u] = fmaf(py, fmaf(-x, sg, x), py);
+            rm[u] = neta * (x * sg) * y;
           }
           o1[j >> 1] = pack_bf16x2(r1[0], r1[1]);
           o3[j >> 1] = pack_bf16x2(r3[0], r3[1]);
@@ -432,8 +434,8 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
 #pragma unroll
           for (int j = 0; j < CW; j += 2) {
             const float x0 = __uint_as_float(rh1[j]), x1 = __uint_as_float(rh1[j + 1]);
-            const float a0 = x0 * (a.split ? sigmoid_fast(x0) : sigmoid_tanh(x0)) * __uint_as_float(rh3[j]);
-            const float a1 = x1 * (a.split ? sigmoid_fast(x1) : sigmoid_tanh(x1)) * __uint_as_float(rh3[j + 1]);
+            const float a0 = x0 * sigmoid_tanh(x0) * __uint_as_float(rh3[j]);
+            const float a1 = x1 * sigmoid_tanh(x1) * __uint_as_float(rh3[j + 1]);
             oq[j >> 1] = pack_bf16x2(a0, a1);
           }
           uint4* dq = reinterpret_cast<uint4*>(a.Aq + (size_t)bh * a.aq_bs + (size_t)tc * a.dh +
@@ -491,7 +493,6 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream) {
   if ((a.n_groups - 1) * a.tiles_per_group >= a.tiles_total) return -1;   // empty group
   a.lr = L.lr;
   a.part[0] = L.part[0]; a.part[1] = L.part[1]; a.part[2] = L.part[2];
-  a.split = 0;
   a.queries = L.q != nullptr ? 1 : 0;
   a.Aq = L.Aq;
   a.aq_bs = L.aq_bs;
