@@ -280,6 +280,23 @@ def make_bench(name, device, seed):
 
 
 # --------------------------------------------------------------------------- timing
+def max_over_ranks(ms, dist):
+    """The job's time: the slowest rank's (NCCL on the GPU, gloo on the host)."""
+    if dist is None:
+        return ms
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, units_per_step_per_rank, step_ms):
+    """Whole-job throughput under weak scaling: every rank processes its own
+    replica, and the step takes the slowest rank's time."""
+    return world * units_per_step_per_rank / (step_ms * 1e-3)
+
+
 def timed(bench, steps, stream, fn=None, dist=None):
     import torch
     fn = fn or bench.step
@@ -292,12 +309,7 @@ def timed(bench, steps, stream, fn=None, dist=None):
         fn(stream)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(e0.elapsed_time(e1), dist)
 
 
 def profile_kernels(bench, steps, stream):
@@ -485,12 +497,12 @@ def main():
         for _ in range(2):
             bench.step_e2e(stream)
         ems = timed(bench, args.steps, stream, fn=bench.step_e2e, dist=dist)
-        e2e = {"value": world * bench.tokens_per_step() * args.steps / (ems * 1e-3),
+        e2e = {"value": job_value(world, bench.tokens_per_step(), ems / args.steps),
                "unit": "tokens/s", "h2d_bytes_per_step": bench.h2d,
                "d2h_bytes_per_step": bench.d2h, "ms_per_step": ems / args.steps}
 
     step_ms = ms / args.steps
-    value = world * bench.tokens_per_step() / (step_ms * 1e-3)
+    value = job_value(world, bench.tokens_per_step(), step_ms)
     tflops = bench.flops_per_step() / (step_ms * 1e-3) / 1e12
 
     secondary = None
@@ -506,7 +518,7 @@ def main():
         sms = timed(sb, args.steps, stream, fn=sfn, dist=dist) / args.steps
         sprof = profile_kernels(sb, args.steps, stream)
         secondary = {"config": sb.config(),
-                     "value": world * sb.tokens_per_step() / (sms * 1e-3),
+                     "value": job_value(world, sb.tokens_per_step(), sms),
                      "unit": "tokens/s", "ms_per_step": sms,
                      "roofline": roofline_for(sb, sprof, args.steps, pk, pk_kind)}
         del sb
