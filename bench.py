@@ -12,6 +12,11 @@ process per GPU under torchrun) every rank runs its own replica on
 rank-seeded inputs: weak scaling, no data-path collective; the step time is
 the max over ranks.
 
+The line also carries `secondary` (the 32K-token linear layer, HBM-bound,
+with its own roofline) and `extra` (the view-synthesis LaCT shapes: one
+196K-token chunk with GD, and ~1M tokens in 64K chunks with Muon), timed
+over a few host-launched steps each.
+
 `--impl reference` times the CPU oracle (float64 numpy) on the host cores, a
 bounded sample of the same workload per step.
 """
@@ -433,6 +438,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="lact_causal_n32k")
     ap.add_argument("--secondary", default="ttt_linear_bf16_n32k")
+    ap.add_argument("--extra", default="lact_bidir_196k,lact_bidir_muon_1m",
+                    help="further workloads timed once each (comma list, or none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every kernel from the host instead of replaying a CUDA graph")
@@ -523,6 +530,30 @@ def main():
                      "roofline": roofline_for(sb, sprof, args.steps, pk, pk_kind)}
         del sb
 
+    # the other LaCT shapes (view-synthesis sets, Muon): a few eager steps each
+    extra = {}
+    for name in ([] if args.extra in ("", "none") else args.extra.split(",")):
+        if name == args.workload:
+            continue
+        eb = make_bench(name, device, seed=rank)
+        for _ in range(2):
+            eb.step(stream)
+        esteps = 3
+        ems = timed(eb, esteps, stream, dist=dist) / esteps
+        eprof = profile_kernels(eb, 1, stream)
+        etot = sum(v["total_ms"] for v in eprof.values()) or 1.0
+        etf = eb.flops_per_step() / (ems * 1e-3) / 1e12
+        ecfg = eb.config()
+        ecfg["launch"] = "host launches"
+        extra[name] = {"config": ecfg, "value": job_value(world, eb.tokens_per_step(), ems),
+                       "unit": "tokens/s", "ms_per_step": ems, "steps": esteps, "tflops": etf,
+                       "frac_bf16_peak": etf / pk["bf16_tflops"],
+                       "kernels": {k: {"launches_per_step": v["launches"],
+                                       "share": v["total_ms"] / etot}
+                                   for k, v in sorted(eprof.items(), key=lambda kv: -kv[1]["total_ms"])}}
+        del eb
+        torch.cuda.empty_cache()
+
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -539,7 +570,7 @@ def main():
                 "tflops": tflops, "frac_bf16_peak": tflops / pk["bf16_tflops"],
                 "peak_source": pk_kind, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "clocks": clocks, "kernels": kernels,
-                "secondary": secondary}
+                "secondary": secondary, "extra": extra or None}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
