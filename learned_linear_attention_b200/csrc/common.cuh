@@ -225,6 +225,11 @@ TTT_DEVICE_INLINE uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo
   return d;
 }
 
+// The same descriptor for an operand `bytes` further on (the start address
+// field holds addr >> 4 in 14 bits; shared addresses stay below 2^18, so the
+// sum never carries out of the field).
+TTT_DEVICE_INLINE uint64_t sdesc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 // 32 lanes x 32 consecutive 32-bit columns per warp (one row per thread).
 TTT_DEVICE_INLINE void tmem_ld32(uint32_t taddr, float* v) {
   uint32_t r[32];

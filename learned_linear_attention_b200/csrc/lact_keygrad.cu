@@ -235,19 +235,20 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         return true;
       };
       // H13 (+ dGr for key tiles) of tile t into its H13 buffer
+      // descriptor bases, advanced by constant byte offsets
+      const uint64_t dkv_k = make_sdesc(kvb, 16, 1024), dkv_mn = make_sdesc(kvb, HALF, 1024);
+      const uint64_t dw13 = make_sdesc(w13, 16, 1024), dw2 = make_sdesc(w2, 8192, 1024);
+      const uint64_t ddh13 = make_sdesc(dhb, HALF, 1024), dgm = make_sdesc(dhb + 2 * HALF, 8192, 1024);
       auto forward = [&](uint32_t t, bool is_key) {
         tc_fence_after();
         const uint32_t s = t & 1;
-        const uint32_t kt = kvb + s * KV_STAGE, vt = kt + TILE;
+        const uint64_t dk = sdesc_add(dkv_k, s * KV_STAGE), dv = sdesc_add(dk, TILE);
         const uint32_t acc = tmem + (s ? TM_H13B : TM_H13A);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t atom = kk >> 2, ko = (kk & 3) * 32;
-          mma_bf16(acc, make_sdesc(kt + atom * HALF + ko, 16, 1024),
-                   make_sdesc(w13 + atom * HALF + ko, 16, 1024), id_h, kk > 0);
-          if (is_key)
-            mma_bf16(tmem + TM_DG, make_sdesc(vt + atom * HALF + ko, 16, 1024),
-                     make_sdesc(w2 + kk * 2048, 8192, 1024), id_g, kk > 0);
+          const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+          mma_bf16(acc, sdesc_add(dk, off), sdesc_add(dw13, off), id_h, kk > 0);
+          if (is_key) mma_bf16(tmem + TM_DG, sdesc_add(dv, off), sdesc_add(dw2, kk * 2048), id_g, kk > 0);
         }
         mma_commit(&acc_full[s]);
         if (!is_key) mma_commit(&kv_empty[s]);   // a query tile is done with its stage
@@ -255,17 +256,15 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
       // gradient products of the key tile in stage t & 1
       auto grads = [&](uint32_t t, bool first) {
         tc_fence_after();
-        const uint32_t kt = kvb + (t & 1) * KV_STAGE, vt = kt + TILE;
+        const uint64_t dk = sdesc_add(dkv_mn, (t & 1) * KV_STAGE), dv = sdesc_add(dk, TILE);
         // K^T / V^T as MN-major A: M = d in two 64-wide blocks 16 KB apart,
         // K = tokens (rows of 128 B); [dH1 | dH3] as MN-major B with its two
         // 64-wide blocks 16 KB apart (N = 128), Gm' as N = 64
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-          mma_bf16(tmem + TM_G13, make_sdesc(kt + kk * 2048, HALF, 1024),
-                   make_sdesc(dhb + kk * 2048, HALF, 1024), id_g13, acc);
-          mma_bf16(tmem + TM_G2, make_sdesc(vt + kk * 2048, HALF, 1024),
-                   make_sdesc(dhb + 2 * HALF + kk * 2048, 8192, 1024), id_g2, acc);
+          mma_bf16(tmem + TM_G13, sdesc_add(dk, kk * 2048), sdesc_add(ddh13, kk * 2048), id_g13, acc);
+          mma_bf16(tmem + TM_G2, sdesc_add(dv, kk * 2048), sdesc_add(dgm, kk * 2048), id_g2, acc);
         }
         mma_commit(dh_free);
         mma_commit(&kv_empty[t & 1]);
@@ -307,6 +306,8 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
             t_idle = 0;
             continue;
           }
+          // back off: this warp shares its scheduler with epilogue warps
+          __nanosleep(32);
           if ((++spins & 255u) == 0u) {   // bounded: give up after the wait timeout
             if (W.aborted()) { ok = false; break; }
             const uint64_t now = globaltimer_ns();

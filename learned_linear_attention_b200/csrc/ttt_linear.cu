@@ -251,38 +251,43 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       const uint32_t pt_base = smem_u32(smem + OFF_PT);
       const uint32_t ev_base = smem_u32(smem + OFF_EV);
       const uint32_t sb_base = smem_u32(smem + OFF_SB);
+      // descriptors: per-stage bases, advanced by constant byte offsets
+      const uint64_t dq0 = make_sdesc(smem_u32(smem + OFF_STAGE), 16, 1024);
+      const uint64_t dk_mn0 = make_sdesc(smem_u32(smem + OFF_STAGE) + TILE_BYTES, 8192, 1024);
+      const uint64_t dpt = make_sdesc(pt_base, 16, 1024);
+      const uint64_t dev_mn = make_sdesc(ev_base, 8192, 1024);
+      const uint64_t dsb = make_sdesc(sb_base, 8192, 1024);
       auto issue_p = [&](int i) {
         tc_fence_after();
         const int s = i % STAGES, pb = i & 1;
-        const uint32_t qs = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES);
-        const uint32_t ks = qs + TILE_BYTES;
+        const uint64_t dq = sdesc_add(dq0, s * STAGE_BYTES), dk = sdesc_add(dq, TILE_BYTES);
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + (pb ? TM_P1 : TM_P0), make_sdesc(qs + kk * 32, 16, 1024),
-                   make_sdesc(ks + kk * 32, 16, 1024), id_qk, kk > 0);
+          mma_bf16(tmem + (pb ? TM_P1 : TM_P0), sdesc_add(dq, kk * 32), sdesc_add(dk, kk * 32), id_qk,
+                   kk > 0);
         mma_commit(&pfull[pb]);
       };
       auto issue_o = [&](int i) {
         tc_fence_after();
         const int s = i % STAGES;
-        const uint32_t qs = smem_u32(smem + OFF_STAGE + s * STAGE_BYTES);
-        const uint32_t ks = qs + TILE_BYTES;
-        const uint32_t pt = pt_base;
-        const uint32_t ev = ev_base;
+        const uint64_t dq = sdesc_add(dq0, s * STAGE_BYTES);
+        const uint64_t dk = sdesc_add(dk_mn0, s * STAGE_BYTES);
         // O = mask(P) (eta V): K = 128 keys, two 64-key atoms of the P tile.
         // O alternates between two TMEM buffers so the epilogue can store the
         // previous tile's O while this tile's products run.
         const uint32_t tm_o = (i & 1) ? TM_O1 : TM_O0;
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + tm_o, make_sdesc(pt + (kk >> 2) * TILE_BYTES + (kk & 3) * 32, 16, 1024),
-                   make_sdesc(ev + kk * 2048, 8192, 1024), id_o, kk > 0);
+          mma_bf16(tmem + tm_o, sdesc_add(dpt, (kk >> 2) * TILE_BYTES + (kk & 3) * 32),
+                   sdesc_add(dev_mn, kk * 2048), id_o, kk > 0);
         // O += Q S_{prev}
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + tm_o, make_sdesc(qs + kk * 32, 16, 1024),
-                   make_sdesc(sb_base + kk * 2048, 8192, 1024), id_o, 1);
+          mma_bf16(tmem + tm_o, sdesc_add(dq, kk * 32), sdesc_add(dsb, kk * 2048), id_o, 1);
         // S += K^T (eta V)   (M = 64: rows live in lanes 0-15 of each quadrant)
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + TM_S, make_sdesc(ks + kk * 2048, 8192, 1024),
-                   make_sdesc(ev + kk * 2048, 8192, 1024), id_s, 1);
+          mma_bf16(tmem + TM_S, sdesc_add(dk, kk * 2048), sdesc_add(dev_mn, kk * 2048), id_s, 1);
         mma_commit(ofull);
         mma_commit(&empty[s]);
       };
@@ -306,6 +311,8 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
           t_idle = 0;
           continue;
         }
+        // back off: this warp shares its scheduler with epilogue warps
+        __nanosleep(32);
         if ((++spins & 255u) == 0u) {   // bounded: give up after the wait timeout
           if (W.aborted()) break;
           const uint64_t now = globaltimer_ns();
