@@ -64,6 +64,14 @@ struct GemmMaps {
   CUtensorMap a[3], b[3];
 };
 
+// TMEM columns for the two accumulators (allocations are powers of two >= 32)
+template <int BN>
+struct GemmTmem {
+  static constexpr uint32_t COLS = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128
+                                   : 2 * BN <= 256 ? 256 : 512;
+  static_assert(2 * BN <= 512, "two accumulators fit in TMEM");
+};
+
 template <int BN, int STAGES>
 struct GemmSmem {
   static constexpr uint32_t A_BYTES = 128 * 64 * 2;
@@ -236,7 +244,7 @@ __global__ void __launch_bounds__(192, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * BN);
+    tmem_alloc(tmem_slot, GemmTmem<BN>::COLS);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -437,7 +445,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * BN);
+    tmem_dealloc(tmem, GemmTmem<BN>::COLS);
   }
 }
 

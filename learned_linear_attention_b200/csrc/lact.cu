@@ -1153,7 +1153,14 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
         }
       }
       g.o32 = const_cast<float*>(ra.part[mat]);
-      TTT_TRY(run_gemm<128, true, true, 4>(m, g, mstream[mat], K_GEMM_GRAD));
+      // wide N tiles read the long token-major operands fewer times: 192 for
+      // [G1; G3] (N = d), 256 for G2 (N = dh)
+      if (mat < 2 && d % 192 == 0)
+        TTT_TRY(run_gemm<192, true, true, 5>(m, g, mstream[mat], K_GEMM_GRAD));
+      else if (mat == 2 && dh % 256 == 0)
+        TTT_TRY(run_gemm<256, true, true, 4>(m, g, mstream[mat], K_GEMM_GRAD));
+      else
+        TTT_TRY(run_gemm<128, true, true, 4>(m, g, mstream[mat], K_GEMM_GRAD));
     }
     return splits;
   };
