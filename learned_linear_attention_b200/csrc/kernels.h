@@ -103,7 +103,11 @@ struct LactWorkspace {
   size_t w1lo, w3lo, w2lo, d13lo, gmlo, aqlo, nsxlo, nsalo, nsblo;
   int cmax;                // rows of the per-chunk intermediates
   int splits;              // split-K factor of the gradient GEMMs
+  int keygrad;             // head dim 128, GD / momentum: fused key/gradient path
+  int nbuf;                // bf16 weight buffers (3 on the fused causal path, else 2)
+  int naq;                 // Aq buffers (2 on the fused causal path, else 1)
 };
+bool lact_uses_keygrad(int d, int dh, int opt, int split);
 LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
                                     int causal, int opt, int split);
 int launch_lact(const LactLaunch& L, cudaStream_t stream);

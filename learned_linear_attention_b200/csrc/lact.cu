@@ -790,6 +790,12 @@ static int grad_splits(int BH, int d, int dh, int cmax) {
   return s;
 }
 
+// head dim 128 (dh a multiple of 64), no split operands, GD or momentum: the
+// key pass and the chunk gradient run as one fused kernel (lact_keygrad.cu)
+bool lact_uses_keygrad(int d, int dh, int opt, int split) {
+  return d == 128 && dh % 64 == 0 && !split && opt != 2;
+}
+
 LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
                                     int causal, int opt, int split) {
   LactWorkspace w{};
@@ -799,17 +805,25 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
   cmax = (cmax + 127) / 128 * 128;
   w.cmax = cmax;
   w.splits = grad_splits((int)BH, d, dh, cin);
-  if (d == 128 && dh % 64 == 0) w.splits = std::max(w.splits, keygrad_groups((int)BH, dh, cin, 0));
+  w.keygrad = lact_uses_keygrad(d, dh, opt, split) ? 1 : 0;
+  if (w.keygrad) w.splits = std::max(w.splits, keygrad_groups((int)BH, dh, cin, 0));
+  // bf16 operand copies: chunk c reads buffer c mod nbuf while its update
+  // writes the next one.  On the fused causal path the read of chunk c runs
+  // beside the next chunk, so a third buffer (and a second Aq) keeps what it
+  // reads intact.
+  w.nbuf = w.keygrad && causal ? 3 : 2;
+  w.naq = w.keygrad && causal ? 2 : 1;
   size_t o = 0;
   w.status = o; o = align256(o + 256);
-  // bf16 operand copies, two buffers (chunk c reads buffer c&1 while its
-  // update writes the other one)
-  w.w1b = o; o = align256(o + 2 * BH * dh * d * 2);
-  w.w3b = o; o = align256(o + 2 * BH * dh * d * 2);
-  w.w2b = o; o = align256(o + 2 * BH * d * dh * 2);
-  w.d13 = o; o = align256(o + BH * cmax * 2 * dh * 2);
-  w.gm = o; o = align256(o + BH * cmax * dh * 2);
-  w.aq = o; o = align256(o + BH * cmax * dh * 2);
+  w.w1b = o; o = align256(o + w.nbuf * BH * dh * d * 2);
+  w.w3b = o; o = align256(o + w.nbuf * BH * dh * d * 2);
+  w.w2b = o; o = align256(o + w.nbuf * BH * d * dh * 2);
+  w.aq = o; o = align256(o + w.naq * BH * cmax * dh * 2);
+  w.d13 = w.gm = o;
+  if (!w.keygrad) {   // key-pass intermediates of the unfused path
+    w.d13 = o; o = align256(o + BH * cmax * 2 * dh * 2);
+    w.gm = o; o = align256(o + BH * cmax * dh * 2);
+  }
   w.part = o; o = align256(o + (size_t)w.splits * BH * 3 * d * dh * 4);
   w.rowss = w.nsx32 = w.nsxb = w.nsa32 = w.nsab = w.nsbb = o;
   if (opt == 2) {
@@ -841,7 +855,8 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
 }
 
 template <int BN, bool A_MN, bool B_MN, int STAGES>
-static int run_gemm(const GemmMaps& maps, const GemmArgs& g, cudaStream_t stream, int kind) {
+static int run_gemm(const GemmMaps& maps, const GemmArgs& g, cudaStream_t stream, int kind,
+                    int max_grid = 0) {
   auto kfn = gemm_bf16_kernel<BN, A_MN, B_MN, STAGES>;
   const int smem = (int)GemmSmem<BN, STAGES>::BYTES;
   static bool attr_done = false;
@@ -855,7 +870,7 @@ static int run_gemm(const GemmMaps& maps, const GemmArgs& g, cudaStream_t stream
   // cluster mode: one tile per CTA, N tiles of a row block in one cluster
   const int cl = g.cluster_n > 1 ? g.cluster_n : 1;
   if (cl > 1 && (g.N / BN != cl || g.splits != 1)) return -1;
-  const int grid = cl > 1 ? tiles : std::min(tiles, num_sms());
+  const int grid = cl > 1 ? tiles : std::min(tiles, max_grid > 0 ? max_grid : num_sms());
   prof_before(kind, stream);
   if (launch_pdl_cluster(kfn, dim3(grid), dim3(192), smem, stream, cl, maps, g) != cudaSuccess)
     return -1;
@@ -885,9 +900,10 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   uint8_t* ws = L.ws;
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
   const size_t wsz = (size_t)BH * d * dh;
-  __nv_bfloat16* wbuf[2][3];
-  __nv_bfloat16* lbuf[2][3];
-  for (int b = 0; b < 2; ++b) {
+  const int nbuf = w.nbuf;
+  __nv_bfloat16* wbuf[3][3];
+  __nv_bfloat16* lbuf[3][3];
+  for (int b = 0; b < nbuf; ++b) {
     wbuf[b][0] = bf(w.w1b) + b * wsz;
     wbuf[b][1] = bf(w.w3b) + b * wsz;
     wbuf[b][2] = bf(w.w2b) + b * wsz;
@@ -953,7 +969,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // both buffers start from the state (matrices excluded by update_mask are
   // never rewritten and must read the same in either buffer)
   set_out_buf(0);
-  ra.nbuf = 2;
+  ra.nbuf = nbuf;
   ra.buf_stride = wsz;
   prof_before(K_LACT_CAST, stream);
   if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
@@ -991,9 +1007,9 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   if (q_rows > 0) TTT_TRY(tok_map(&km.q, L.q, q_rows, 128));
   else km.q = km.k;
   if (L.N_in == 0) { km.k = km.q; km.v = km.q; }
-  KeyPassMaps kmb[2] = {km, km};
-  CUtensorMap mw2k[2], mw2klo[2];
-  for (int b = 0; b < 2; ++b) {
+  KeyPassMaps kmb[3] = {km, km, km};
+  CUtensorMap mw2k[3], mw2klo[3];
+  for (int b = 0; b < nbuf; ++b) {
     TTT_TRY(w13_map(&kmb[b].w1, wbuf[b][0]));
     TTT_TRY(w13_map(&kmb[b].w3, wbuf[b][1]));
     TTT_TRY(w2_mn_map(&kmb[b].w2, wbuf[b][2]));
@@ -1009,6 +1025,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     }
   }
   int cur = 0;   // buffer holding the chunk-start weights
+  auto nxt = [&](int b) { return b + 1 == nbuf ? 0 : b + 1; };   // buffer its update writes
   CUtensorMap mk_mn{}, mv_mn{};   // token tensors as MN-major operands
   if (L.N_in > 0) {
     TTT_TRY(tok_map(&mk_mn, L.k, L.N_in, 64));
@@ -1043,7 +1060,8 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     return key_pass_on(t0, C, nkt, nqt, stream);
   };
   // out rows [t0, t0 + C) = Aq W2^T (split: hi*hi + hi*lo + lo*hi)
-  auto read_out = [&](int t0, int C, cudaStream_t rstream) -> int {
+  auto read_out = [&](int t0, int C, cudaStream_t rstream, const __nv_bfloat16* aq,
+                      int max_grid = 0) -> int {
     GemmArgs g = gemm_defaults(L.st);
     g.M = C; g.N = d; g.batch = BH; g.k_steps = dh / 64;
     g.out_row_off = t0;
@@ -1058,7 +1076,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       g.ld32 = d;
     }
     GemmMaps m{};
-    TTT_TRY(inter_map(&m.a[0], Aq, C, 128));
+    TTT_TRY(inter_map(&m.a[0], aq, C, 128));
     m.b[0] = mw2k[cur];
     if (split) {
       g.npairs = 3;
@@ -1067,7 +1085,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       TTT_TRY(inter_map(&m.a[2], Aqlo, C, 128));
       m.b[2] = mw2k[cur];
     }
-    return run_gemm<128, false, false, 4>(m, g, rstream, K_GEMM_READ);
+    return run_gemm<128, false, false, 4>(m, g, rstream, K_GEMM_READ, max_grid);
   };
   // Chunk gradients G1 = dH1^T K, G3 = dH3^T K (rows = hidden units, N = d)
   // and G2 = V^T Gm' (rows = d, N = dh), contracted over the chunk's tokens.
@@ -1103,8 +1121,8 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
         GemmArgs g13 = g;
         g13.M = 2 * dh; g13.N = d; g13.ldw = d; g13.rows_first = dh;
         g13.W[0] = W1; g13.W[1] = W3; g13.Mom[0] = M1; g13.Mom[1] = M3;
-        g13.Wb[0] = wbuf[cur ^ 1][0]; g13.Wb[1] = wbuf[cur ^ 1][1];
-        g13.Wlo[0] = lbuf[cur ^ 1][0]; g13.Wlo[1] = lbuf[cur ^ 1][1];
+        g13.Wb[0] = wbuf[nxt(cur)][0]; g13.Wb[1] = wbuf[nxt(cur)][1];
+        g13.Wlo[0] = lbuf[nxt(cur)][0]; g13.Wlo[1] = lbuf[nxt(cur)][1];
         if ((L.update_mask & 3) == 2) { g13.a_m_off[0] = g13.a_m_off[1] = dh; g13.M = dh; g13.rows_first = 0; }
         if ((L.update_mask & 3) == 1) { g13.M = dh; }
         for (int p = 0; p < np; ++p) {
@@ -1118,7 +1136,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       if (L.update_mask & 4) {
         GemmArgs g2 = g;
         g2.M = d; g2.N = dh; g2.ldw = dh; g2.rows_first = d; g2.cluster_n = dh / 128;
-        g2.W[0] = W2; g2.Mom[0] = M2; g2.Wb[0] = wbuf[cur ^ 1][2]; g2.Wlo[0] = lbuf[cur ^ 1][2];
+        g2.W[0] = W2; g2.Mom[0] = M2; g2.Wb[0] = wbuf[nxt(cur)][2]; g2.Wlo[0] = lbuf[nxt(cur)][2];
         for (int p = 0; p < np; ++p) {
           m.a[p] = mv_mn;
           m.b[p] = p == 0 ? mg : mgl;
@@ -1275,72 +1293,72 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
         return -1;
     return 0;
   };
-  // head dim 128 without split operands: the key pass and the gradient
-  // contraction run fused (partial sums per token group), the queries and
-  // the read run concurrently on a helper stream.
-  const bool keygrad = d == 128 && !split && L.opt != 2;
-  // Chunk c: the fused kernel forms the gradient partial sums and Aq on the
-  // chunk-start weights (buffer cur); the read of chunk c (helper stream,
-  // buffer cur) then runs beside the update, which writes buffer cur^1; the
-  // next chunk's fused kernel waits for that read before rewriting Aq.
+  // Head dim 128, GD / momentum: per chunk the fused kernel forms Aq (causal)
+  // and the gradient partial sums on the chunk-start weights (buffer cur);
+  // the row update writes buffer nxt(cur).  The read of chunk c (helper
+  // stream; Aq buffer c % 2, W2 buffer cur) runs beside the update and the
+  // next chunk on the SMs the fused kernel leaves free; the kernel of chunk
+  // c + 2 rewrites both, so it first waits for that read.
+  const bool keygrad = w.keygrad != 0;
   int ci = 0;
   for (int t0 = 0; keygrad && t0 < L.N_in; t0 += L.chunk, ++ci) {
     const int C = std::min(L.chunk, L.N_in - t0);
+    __nv_bfloat16* aq = Aq + (size_t)(ci % w.naq) * BH * w.cmax * dh;
     KeyGradLaunch kgl{};
     kgl.BH = BH; kgl.N_in = L.N_in; kgl.C = C; kgl.t0 = t0; kgl.dh = dh;
     kgl.groups = keygrad_groups(BH, dh, C, w.splits);
     kgl.k = L.k; kgl.v = L.v; kgl.lr = L.lr;
     kgl.q = L.causal ? L.q : nullptr;
-    kgl.Aq = Aq; kgl.aq_bs = (long long)w.cmax * dh;
+    kgl.Aq = aq; kgl.aq_bs = (long long)w.cmax * dh;
     kgl.w1b = wbuf[cur][0]; kgl.w3b = wbuf[cur][1]; kgl.w2b = wbuf[cur][2];
     kgl.part[0] = const_cast<float*>(ra.part[0]);
     kgl.part[1] = const_cast<float*>(ra.part[1]);
     kgl.part[2] = const_cast<float*>(ra.part[2]);
     kgl.st = L.st;
-    // Aq of the previous chunk must have been read before this chunk rewrites it
-    if (L.causal && ss && ci >= 1)
-      TTT_TRY(cudaStreamWaitEvent(stream, ss->read_done[(ci - 1) & 1], 0) == cudaSuccess ? 0 : -1);
+    if (L.causal && ss && ci >= w.naq)
+      TTT_TRY(cudaStreamWaitEvent(stream, ss->read_done[ci & 1], 0) == cudaSuccess ? 0 : -1);
     TTT_TRY(launch_lact_keygrad(kgl, stream));
-    if (L.causal) {   // the read of this chunk runs beside the update
+    if (L.causal) {   // the read of this chunk runs beside the update and the next chunk
       if (ss) {
         TTT_TRY(cudaEventRecord(ss->fork, stream) == cudaSuccess ? 0 : -1);
         TTT_TRY(cudaStreamWaitEvent(rstream, ss->fork, 0) == cudaSuccess ? 0 : -1);
       }
-      TTT_TRY(read_out(t0, C, rstream));
+      const int kg_grid = std::min(BH * (dh / 64) * kgl.groups, num_sms());
+      TTT_TRY(read_out(t0, C, rstream, aq, ss ? std::max(8, num_sms() - kg_grid) : 0));
       if (ss) TTT_TRY(cudaEventRecord(ss->read_done[ci & 1], rstream) == cudaSuccess ? 0 : -1);
     }
     ra.splits = kgl.groups;
-    set_out_buf(cur ^ 1);
+    set_out_buf(nxt(cur));
     TTT_TRY(row_update(stream));
-    cur ^= 1;
+    cur = nxt(cur);
   }
-  if (keygrad && L.causal && ss && ci >= 1)   // the last read joins the caller's stream
+  if (keygrad && L.causal && ss && ci >= 1)   // the reads join the caller's stream
     TTT_TRY(cudaStreamWaitEvent(stream, ss->read_done[(ci - 1) & 1], 0) == cudaSuccess ? 0 : -1);
   for (int t0 = 0; !keygrad && t0 < L.N_in; t0 += L.chunk) {
     const int C = std::min(L.chunk, L.N_in - t0);
     const int nt = (C + 127) / 128;
     TTT_TRY(key_pass(t0, C, nt, L.causal ? nt : 0));
     TTT_TRY(fork());
-    if (L.causal) TTT_TRY(read_out(t0, C, rstream));
+    if (L.causal) TTT_TRY(read_out(t0, C, rstream, Aq));
     const int splits = gradients(t0, C, gstream);
     if (splits < 0) return -1;
     TTT_TRY(join());
-    if (fused_update) {   // the epilogues wrote buffer cur^1
-      cur ^= 1;
+    if (fused_update) {   // the epilogues wrote buffer nxt(cur)
+      cur = nxt(cur);
       continue;
     }
     ra.splits = splits;
-    set_out_buf(cur ^ 1);
+    set_out_buf(nxt(cur));
     if (L.opt == 2) {
       TTT_TRY(muon());
     } else {
       TTT_TRY(row_update(stream));
     }
-    cur ^= 1;
+    cur = nxt(cur);
   }
   if (!L.causal && L.N_q > 0) {
     TTT_TRY(key_pass(0, L.N_q, 0, (L.N_q + 127) / 128));
-    TTT_TRY(read_out(0, L.N_q, stream));
+    TTT_TRY(read_out(0, L.N_q, stream, Aq));
   }
   return 0;
 }
