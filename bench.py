@@ -329,8 +329,18 @@ def profile_kernels(bench, steps, stream):
 
 
 def roofline_for(bench, prof, steps, pk, pk_kind):
+    """Roofline of the dominant kernel: for the LaCT layer the kernel doing the
+    most algorithmic work (the fused key/gradient kernel, on the critical
+    path; the read runs beside it on a helper stream), for the linear layer
+    the kernel taking the most time."""
     total = sum(v["total_ms"] for v in prof.values())
     name, rec = max(prof.items(), key=lambda kv: kv[1]["total_ms"])
+    if not isinstance(bench, LinearBench):
+        kfs = bench.kernel_flops_per_step()
+        cands = [k for k in prof if k in kfs]
+        if cands:
+            name = max(cands, key=lambda k: kfs[k])
+            rec = prof[name]
     per_launch_ms = rec["total_ms"] / rec["launches"]
     launches_per_step = rec["launches"] / steps
     tr = traffic_table().get(name, {}).get(bench.name)
