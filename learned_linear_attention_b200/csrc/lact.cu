@@ -966,10 +966,10 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   };
 
-  // both buffers start from the state (matrices excluded by update_mask are
-  // never rewritten and must read the same in either buffer)
   set_out_buf(0);
-  ra.nbuf = nbuf;
+  // only buffer 0 is read before an update writes it, unless a matrix is
+  // never updated (update_mask): then every buffer must hold it
+  ra.nbuf = (L.update_mask & 7) == 7 ? 1 : nbuf;
   ra.buf_stride = wsz;
   prof_before(K_LACT_CAST, stream);
   if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
