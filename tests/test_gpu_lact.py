@@ -163,3 +163,37 @@ def test_causal_many_chunks_multi_tile_groups(cuda_device):
     gradient of the same chunk."""
     x = make_lact_inputs(2, 4, 4096, 128, 256, chunk=1024, order="causal", cfg=42)
     _check(x)
+
+
+def test_causal_update_mask_w1_w3_with_norm_keeps_w2(cuda_device):
+    """W2 excluded from the update on the fused path: every bf16 buffer must
+    hold the initial W2, which stays exactly unchanged, and the rows of W1
+    and W3 are normalised."""
+    x = make_lact_inputs(1, 2, 640, 128, 256, chunk=128, order="causal", cfg=43)
+    run, *_ = _check(x, update_mask=3)
+    W = run.weights()
+    assert np.array_equal(W[2][0], x.W2)
+    for w in W[:2]:
+        assert np.abs(np.linalg.norm(w.astype(np.float64), axis=-1) - 1).max() < 1e-5
+
+
+def test_causal_chunk_not_a_multiple_of_the_tile(cuda_device):
+    """Chunks of 200 tokens: the last tile of each chunk holds rows of the
+    next chunk, which must not enter this chunk's gradient."""
+    x = make_lact_inputs(1, 2, 600, 128, 256, chunk=200, order="causal", cfg=44)
+    _check(x)
+    _check(x, "momentum")
+
+
+def test_causal_head_dim_256_fused_gemm_update(cuda_device):
+    """d = dh = 256 runs the key pass and the gradient GEMMs with the update
+    fused into their epilogues (momentum)."""
+    x = make_lact_inputs(1, 2, 512, 256, 256, chunk=256, order="causal", cfg=45)
+    _check(x, "momentum")
+
+
+def test_causal_hidden_128_and_many_items_per_cta(cuda_device):
+    """dh = 128 (two hidden blocks per head) over 64 heads: more work items
+    than SMs, so CTAs of the fused kernel run several items."""
+    x = make_lact_inputs(4, 16, 512, 128, 128, chunk=256, order="causal", cfg=46)
+    _check(x)
