@@ -117,10 +117,13 @@ class LaCTBench:
         self.Nq = x.q.values.shape[2]
         self.causal = w["order"] == "causal"
         self.opt = w.get("opt", "gd")
+        self.update_mask = w.get("update_mask", 7)
+        self.normalize_rows = w.get("normalize_rows", True)
         self.desc = T.make_lact_desc(self.B, self.H, self.N, self.d, self.dh, w["chunk"],
                                      N_q=self.Nq, order=w["order"], opt=self.opt,
                                      beta=w.get("beta", 0.9), ns_steps=w.get("ns_steps", 5),
-                                     out_dtype="bf16")
+                                     out_dtype="bf16", update_mask=self.update_mask,
+                                     normalize_rows=self.normalize_rows)
         tok = lambda tt: torch.from_numpy(tt.bits.view("int16")).view(torch.bfloat16)  # noqa
         self.h_q, self.h_k, self.h_v = tok(x.q), tok(x.k), tok(x.v)
         self.h_lr = torch.from_numpy(x.lr)
@@ -139,6 +142,8 @@ class LaCTBench:
 
     def flops_per_step(self):
         BH, d, dh = self.B * self.H, self.d, self.dh
+        if self.update_mask == 4:   # W2 only: phi(k) 4 d dh, its gradient 2, phi(q) 4, read 2
+            return 6 * d * dh * self.N * BH + 6 * d * dh * self.Nq * BH
         f = 12 * d * dh * self.N * BH + 6 * d * dh * self.Nq * BH
         if self.opt == "muon":
             r, c = min(d, dh), max(d, dh)
@@ -186,10 +191,14 @@ class LaCTBench:
 
     def config(self):
         w = self.w
-        return {"workload": self.name, "B": self.B, "H": self.H, "N_in": self.N,
-                "N_q": self.Nq, "d": self.d, "dh": self.dh, "chunk": w["chunk"],
-                "order": w["order"], "optimizer": self.opt, "out_dtype": "bf16",
-                "state_dtype": "f32"}
+        cfg = {"workload": self.name, "B": self.B, "H": self.H, "N_in": self.N,
+               "N_q": self.Nq, "d": self.d, "dh": self.dh, "chunk": w["chunk"],
+               "order": w["order"], "optimizer": self.opt, "out_dtype": "bf16",
+               "state_dtype": "f32"}
+        if self.update_mask != 7 or not self.normalize_rows:
+            cfg["update_mask"] = self.update_mask
+            cfg["normalize_rows"] = self.normalize_rows
+        return cfg
 
     def oracle_sample(self, n_chunks):
         """Oracle on one (b,h) stream and the first n_chunks chunks."""
@@ -448,7 +457,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="lact_causal_n32k")
     ap.add_argument("--secondary", default="ttt_linear_bf16_n32k")
-    ap.add_argument("--extra", default="lact_bidir_196k,lact_bidir_muon_1m",
+    ap.add_argument("--extra", default="lact_bidir_196k,lact_bidir_muon_1m,lact_w2only_causal_n32k",
                     help="further workloads timed once each (comma list, or none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",

@@ -71,7 +71,8 @@ int check_lact(const lact_desc* d) {
 
 LactWorkspace layout_of(const lact_desc* d) {
   return lact_workspace_layout(d->B, d->H, d->N_in, d->N_q, d->d, d->dh, d->chunk,
-                               d->order == TTT_CAUSAL, (int)d->opt, d->split_operands ? 1 : 0);
+                               d->order == TTT_CAUSAL, (int)d->opt, d->split_operands ? 1 : 0,
+                               d->update_mask, d->normalize_rows);
 }
 
 size_t lact_state_elems(const lact_desc* d) {

@@ -104,12 +104,16 @@ struct LactWorkspace {
   int cmax;                // rows of the per-chunk intermediates
   int splits;              // split-K factor of the gradient GEMMs
   int keygrad;             // head dim 128, GD / momentum: fused key/gradient path
+  int w2par;               // W2-only GD without normalisation: parallel form over chunks
+  size_t pmb;              // parallel form: bf16 chunk-start W2 [chunks][BH][d][dh]
   int nbuf;                // bf16 weight buffers (3 on the fused causal path, else 2)
   int naq;                 // Aq buffers (2 on the fused causal path, else 1)
 };
 bool lact_uses_keygrad(int d, int dh, int opt, int split);
+bool lact_uses_w2_parallel(int N_in, int chunk, int d, int dh, int causal, int opt, int split,
+                           int update_mask, int normalize);
 LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
-                                    int causal, int opt, int split);
+                                    int causal, int opt, int split, int update_mask, int normalize);
 int launch_lact(const LactLaunch& L, cudaStream_t stream);
 
 // Fused key pass + chunk gradient (head dim 128): partial sums per token group.

@@ -57,6 +57,9 @@ struct KeyPassArgs {
   // intermediates are written as hi and lo bf16 parts
   int split;
   __nv_bfloat16 *D13lo, *Gmlo, *Aqlo;
+  // key tiles form only Gm' = -eta silu(H1) H3 (no V W2 product, no dH1 and
+  // dH3): only W2 is updated
+  int feat_only;
   long long inter_bs;      // cmax * dh (Gm', Aq); D13 uses twice that
   DevStatus st;
 };
@@ -159,12 +162,13 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
             break;
           }
           uint8_t* st = smem + s * STAGE;
-          mbar_arrive_expect_tx(&full[s], is_key ? STAGE : X_BYTES + W13_BYTES);
+          const bool with_v = is_key && !a.feat_only;
+          mbar_arrive_expect_tx(&full[s], with_v ? STAGE : X_BYTES + W13_BYTES);
           tma_load_3d(st, is_key ? &maps.k : &maps.q, &full[s], ks * 64, row, bh);
           tma_load_3d(st + X_BYTES + V_BYTES, lo ? &maps.w1lo : &maps.w1, &full[s], ks * 64, j0, bh);
           tma_load_3d(st + X_BYTES + V_BYTES + W13_BYTES / 2, lo ? &maps.w3lo : &maps.w3, &full[s],
                       ks * 64, j0, bh);
-          if (is_key) {
+          if (with_v) {
             tma_load_3d(st + X_BYTES, &maps.v, &full[s], ks * 64, row, bh);
             tma_load_3d(st + X_BYTES + V_BYTES + W13_BYTES, lo ? &maps.w2lo : &maps.w2, &full[s],
                         j0, ks * 64, bh);
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
           for (int k4 = 0; k4 < 4; ++k4) {
             mma_bf16(d, make_sdesc(sx + k4 * 32, 16, 1024), make_sdesc(sw13 + k4 * 32, 16, 1024),
                      id_h, (ks | k4) != 0);
-            if (is_key)
+            if (is_key && !a.feat_only)
               mma_bf16(d + 128, make_sdesc(sv + k4 * 32, 16, 1024),
                        make_sdesc(sw2 + k4 * 2048, 8192, 1024), id_g, (ks | k4) != 0);
           }
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
         uint32_t rh1[16], rh3[16], rg[16];
         tmem_ld16_issue(base + jc, rh1);
         tmem_ld16_issue(base + 64 + jc, rh3);
-        if (is_key) tmem_ld16_issue(base + 128 + jc, rg);
+        if (is_key && !a.feat_only) tmem_ld16_issue(base + 128 + jc, rg);
         tmem_wait_ld();
         float h1[16], h3[16];
 #pragma unroll
@@ -254,7 +258,21 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
           h1[j] = __uint_as_float(rh1[j]);
           h3[j] = __uint_as_float(rh3[j]);
         }
-        if (is_key) {
+        if (is_key && a.feat_only) {
+          if (valid) {
+            uint32_t om[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float x0 = h1[2 * j], x1 = h1[2 * j + 1];
+              om[j] = pack_bf16x2(-eta * x0 * sigmoidf_tanh(x0) * h3[2 * j],
+                                  -eta * x1 * sigmoidf_tanh(x1) * h3[2 * j + 1]);
+            }
+            uint4* dm = reinterpret_cast<uint4*>(a.Gm + obase + jc);
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              dm[j] = make_uint4(om[4 * j], om[4 * j + 1], om[4 * j + 2], om[4 * j + 3]);
+          }
+        } else if (is_key) {
           float g[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) g[j] = __uint_as_float(rg[j]);
@@ -277,15 +295,19 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
               o3[j] = pack_bf16x2(r3[2 * j], r3[2 * j + 1]);
               om[j] = pack_bf16x2(rm[2 * j], rm[2 * j + 1]);
             }
-            uint4* d1 = reinterpret_cast<uint4*>(a.D13 + dbase + jc);
-            uint4* d3 = reinterpret_cast<uint4*>(a.D13 + dbase + a.dh + jc);
             uint4* dm = reinterpret_cast<uint4*>(a.Gm + obase + jc);
+            if (a.D13 != nullptr) {   // dH1, dH3 (absent when only W2 is updated)
+              uint4* d1 = reinterpret_cast<uint4*>(a.D13 + dbase + jc);
+              uint4* d3 = reinterpret_cast<uint4*>(a.D13 + dbase + a.dh + jc);
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              d1[j] = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
-              d3[j] = make_uint4(o3[4 * j], o3[4 * j + 1], o3[4 * j + 2], o3[4 * j + 3]);
-              dm[j] = make_uint4(om[4 * j], om[4 * j + 1], om[4 * j + 2], om[4 * j + 3]);
+              for (int j = 0; j < 2; ++j) {
+                d1[j] = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
+                d3[j] = make_uint4(o3[4 * j], o3[4 * j + 1], o3[4 * j + 2], o3[4 * j + 3]);
+              }
             }
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              dm[j] = make_uint4(om[4 * j], om[4 * j + 1], om[4 * j + 2], om[4 * j + 3]);
             if (a.split) {
               uint32_t l1[8], l3[8], lm[8];
 #pragma unroll
@@ -796,14 +818,53 @@ bool lact_uses_keygrad(int d, int dh, int opt, int split) {
   return d == 128 && dh % 64 == 0 && !split && opt != 2;
 }
 
+// W2 alone updated by plain GD without row normalisation, causal order,
+// whole chunks of whole tiles: W1 and W3 stay fixed, so the layer is
+// block-causal linear attention on the features silu(W1 x) * (W3 x) and no
+// chunk depends on an earlier chunk's weights ("Test-Time Training with KV
+// Binding Is Secretly Linear Attention", Resumen técnico §4: with only the
+// last layer updated and no normalisation the layer reduces to linear
+// attention, which has a parallel form).  It runs as one key pass over all
+// tokens, one split-K GEMM whose splits are the chunks (the per-chunk W2
+// increments), a prefix over chunks and one batched read.
+bool lact_uses_w2_parallel(int N_in, int chunk, int d, int dh, int causal, int opt, int split,
+                           int update_mask, int normalize) {
+  return causal && opt == 0 && !split && update_mask == 4 && !normalize && N_in > 0 &&
+         chunk % 128 == 0 && N_in % chunk == 0 && d % 128 == 0 && dh % 128 == 0;
+}
+
 LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
-                                    int causal, int opt, int split) {
+                                    int causal, int opt, int split, int update_mask,
+                                    int normalize) {
   LactWorkspace w{};
   const size_t BH = (size_t)B * H;
   const int cin = std::min(chunk, std::max(N_in, 1));
   int cmax = std::max(cin, causal ? 0 : N_q);
   cmax = (cmax + 127) / 128 * 128;
   w.cmax = cmax;
+  w.w2par = lact_uses_w2_parallel(N_in, chunk, d, dh, causal, opt, split, update_mask, normalize) ? 1 : 0;
+  if (w.w2par) {   // every token at once: features, increments per chunk, chunk-start weights
+    const int nch = N_in / chunk;
+    w.cmax = (N_in + 127) / 128 * 128;
+    w.splits = nch;
+    w.keygrad = 0;
+    w.nbuf = 1;
+    w.naq = 1;
+    size_t o = 0;
+    w.status = o; o = align256(o + 256);
+    w.w1b = o; o = align256(o + BH * dh * d * 2);
+    w.w3b = o; o = align256(o + BH * dh * d * 2);
+    w.w2b = o; o = align256(o + BH * d * dh * 2);
+    w.aq = o; o = align256(o + BH * w.cmax * dh * 2);
+    w.gm = o; o = align256(o + BH * w.cmax * dh * 2);
+    w.d13 = o;
+    w.part = o; o = align256(o + (size_t)nch * BH * d * dh * 4);
+    w.pmb = o; o = align256(o + (size_t)nch * BH * d * dh * 2);
+    w.rowss = w.nsx32 = w.nsxb = w.nsa32 = w.nsab = w.nsbb = o;
+    w.w1lo = w.w3lo = w.w2lo = w.d13lo = w.gmlo = w.aqlo = w.nsxlo = w.nsalo = w.nsblo = o;
+    w.total = o;
+    return w;
+  }
   w.splits = grad_splits((int)BH, d, dh, cin);
   w.keygrad = lact_uses_keygrad(d, dh, opt, split) ? 1 : 0;
   if (w.keygrad) w.splits = std::max(w.splits, keygrad_groups((int)BH, dh, cin, 0));
@@ -892,11 +953,35 @@ static GemmArgs gemm_defaults(const DevStatus& st) {
     if ((__VA_ARGS__) != 0) return -1;    \
   } while (0)
 
+// Parallel form of the W2-only layer: W2 before chunk c (bf16, the read's
+// operand) and W2 after the last chunk, from W2_0 and the chunks' gradient
+// sums part[c] = sum_t (-eta_t v_t) phi(k_t)^T, summed in chunk order.
+__global__ void w2_prefix_kernel(float* W2, const float* part, __nv_bfloat16* Mb, int BH, int dd,
+                                 int nch) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t n4 = (size_t)BH * dd / 4;
+  for (size_t e4 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e4 < n4;
+       e4 += (size_t)gridDim.x * blockDim.x) {
+    const size_t e = e4 * 4;
+    const size_t bh = e / dd, r = e % dd;
+    float4 m = *reinterpret_cast<const float4*>(W2 + e);
+    for (int c = 0; c < nch; ++c) {
+      *reinterpret_cast<uint2*>(Mb + (bh * nch + c) * dd + r) =
+          make_uint2(pack_bf16x2(m.x, m.y), pack_bf16x2(m.z, m.w));
+      const float4 p = __ldcg(reinterpret_cast<const float4*>(part + ((size_t)c * BH + bh) * dd + r));
+      m.x -= p.x; m.y -= p.y; m.z -= p.z; m.w -= p.w;
+    }
+    *reinterpret_cast<float4*>(W2 + e) = m;
+  }
+}
+
 int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   const int BH = L.B * L.H, d = L.d, dh = L.dh;
   const bool split = L.split != 0;
   const LactWorkspace w =
-      lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt, L.split);
+      lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt, L.split,
+                            L.update_mask, L.normalize_rows);
   uint8_t* ws = L.ws;
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
   const size_t wsz = (size_t)BH * d * dh;
@@ -911,7 +996,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     lbuf[b][1] = split ? bf(w.w3lo) + b * wsz : nullptr;
     lbuf[b][2] = split ? bf(w.w2lo) + b * wsz : nullptr;
   }
-  __nv_bfloat16 *D13 = bf(w.d13), *Gm = bf(w.gm), *Aq = bf(w.aq);
+  __nv_bfloat16 *D13 = w.w2par ? nullptr : bf(w.d13), *Gm = bf(w.gm), *Aq = bf(w.aq);
   __nv_bfloat16 *D13lo = split ? bf(w.d13lo) : nullptr, *Gmlo = split ? bf(w.gmlo) : nullptr, *Aqlo = split ? bf(w.aqlo) : nullptr;
   float* part = reinterpret_cast<float*>(ws + w.part);
   const size_t mat_elems = (size_t)BH * d * dh;
@@ -1046,6 +1131,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     a.d_steps = d / 64; a.dh = dh; a.lr_len = L.N_in; a.lr = L.lr;
     a.D13 = D13; a.Gm = Gm; a.Aq = Aq;
     a.split = split ? 1 : 0; a.D13lo = D13lo; a.Gmlo = Gmlo; a.Aqlo = Aqlo;
+    a.feat_only = D13 == nullptr ? 1 : 0;
     a.inter_bs = (long long)w.cmax * dh; a.st = L.st;
     const int tiles = (nkt + nqt) * a.n_hb * BH;
     if (tiles <= 0) return 0;
@@ -1293,6 +1379,54 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
         return -1;
     return 0;
   };
+  if (w.w2par) {
+    // ---- parallel form of the W2-only layer (see lact_uses_w2_parallel)
+    const int nch = L.N_in / L.chunk;
+    const int nt = L.N_in / 128;
+    TTT_TRY(key_pass(0, L.N_in, nt, nt));   // phi(q) -> Aq, -eta phi(k) -> Gm'
+    {   // per-chunk gradient sums G2_c = V_c^T Gm'_c: the chunks are the splits
+      CUtensorMap mg;
+      TTT_TRY(inter_map(&mg, Gm, L.N_in, 64));
+      GemmArgs g = gemm_defaults(L.st);
+      g.M = d; g.N = dh; g.batch = BH; g.splits = nch; g.k_steps = L.chunk / 64; g.npairs = 1;
+      g.o32 = part; g.o32_ss = (long long)BH * d * dh; g.o32_bs = (long long)d * dh; g.ld32 = dh;
+      GemmMaps m{};
+      m.a[0] = mv_mn;
+      m.b[0] = mg;
+      if (dh % 256 == 0) TTT_TRY(run_gemm<256, true, true, 4>(m, g, stream, K_GEMM_GRAD));
+      else TTT_TRY(run_gemm<128, true, true, 4>(m, g, stream, K_GEMM_GRAD));
+    }
+    __nv_bfloat16* Mb = bf(w.pmb);
+    {
+      const int dd = d * dh;
+      const int blocks = std::min(4 * num_sms(), (int)(((size_t)BH * dd / 4 + 255) / 256));
+      prof_before(K_UPDATE, stream);
+      if (launch_pdl(w2_prefix_kernel, dim3(blocks), dim3(256), 0, stream, W2, (const float*)part, Mb, BH,
+                     dd, nch) != cudaSuccess)
+        return -1;
+      prof_after(K_UPDATE, stream);
+    }
+    {   // out rows of chunk c = Aq_c (W2 before chunk c)^T, all chunks at once
+      GemmArgs g = gemm_defaults(L.st);
+      g.M = L.chunk; g.N = d; g.batch = BH * nch; g.k_steps = dh / 64;
+      if (L.out_bf16) {
+        g.o16 = reinterpret_cast<__nv_bfloat16*>(L.out);
+        g.o16_bs = (long long)L.chunk * d;
+        g.ld16 = d;
+      } else {
+        g.o32 = reinterpret_cast<float*>(L.out);
+        g.o32_bs = (long long)L.chunk * d;
+        g.ld32 = d;
+      }
+      GemmMaps m{};
+      TTT_TRY(make_tmap_bf16_3d(&m.a[0], Aq, dh, L.chunk, (uint64_t)BH * nch, (uint64_t)dh * 2,
+                                (uint64_t)L.chunk * dh * 2, 64, 128));
+      TTT_TRY(make_tmap_bf16_3d(&m.b[0], Mb, dh, d, (uint64_t)BH * nch, (uint64_t)dh * 2,
+                                (uint64_t)d * dh * 2, 64, 128));
+      TTT_TRY(run_gemm<128, false, false, 4>(m, g, stream, K_GEMM_READ));
+    }
+    return 0;
+  }
   // Head dim 128, GD / momentum: per chunk the fused kernel forms Aq (causal)
   // and the gradient partial sums on the chunk-start weights (buffer cur);
   // the row update writes buffer nxt(cur).  The read of chunk c (helper

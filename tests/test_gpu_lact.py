@@ -197,3 +197,15 @@ def test_causal_hidden_128_and_many_items_per_cta(cuda_device):
     than SMs, so CTAs of the fused kernel run several items."""
     x = make_lact_inputs(4, 16, 512, 128, 128, chunk=256, order="causal", cfg=46)
     _check(x)
+
+
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+def test_w2_only_parallel_form(cuda_device, out_dtype):
+    """Only W2 updated, plain GD, no row norm: the layer is block-causal linear
+    attention on silu(W1 x) * (W3 x) and runs in its parallel form (one key
+    pass, per-chunk increments as the splits of one GEMM, a prefix over
+    chunks, one batched read).  W1 and W3 stay exactly as given."""
+    x = make_lact_inputs(2, 2, 2048, 128, 256, chunk=256, order="causal", cfg=47)
+    run, *_ = _check(x, out_dtype=out_dtype, update_mask=4, normalize_rows=False)
+    W = run.weights()
+    assert np.array_equal(W[0][0], x.W1) and np.array_equal(W[1][0], x.W3)

@@ -167,6 +167,12 @@ WORKLOADS = {
     "lact_causal_n32k": dict(kind="lact", B=2, H=4, N=32768, d=128, dh=256, chunk=2048,
                              order="causal", qk_norm=True, v_norm=False,
                              lr_kind="0.01softplus", opt="gd", cfg=3),
+    # the 32K causal shape with only W2 updated (plain GD, no row norm): the
+    # layer is block-causal linear attention on silu(W1 x) * (W3 x)
+    "lact_w2only_causal_n32k": dict(kind="lact", B=2, H=4, N=32768, d=128, dh=256, chunk=2048,
+                                    order="causal", qk_norm=True, v_norm=False,
+                                    lr_kind="0.01softplus", opt="gd", update_mask=4,
+                                    normalize_rows=False, cfg=3),
     "lact_bidir_196k": dict(kind="lact", B=1, H=2, N=196608, Nq=4096, d=384, dh=768,
                             chunk=196608, order="bidirectional", qk_norm=True, v_norm=True,
                             lr_kind="0.01sig", opt="gd", cfg=4),
