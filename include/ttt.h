@@ -160,8 +160,21 @@ typedef struct {
 int lact_state_bytes(const lact_desc* desc, size_t* bytes);
 
 /* Workspace bytes for lact_chunk_fwd (status word, bf16 operand copies of
- * the weights, per-chunk intermediates, split-K partial sums, NS buffers). */
+ * the weights, per-chunk intermediates, split-K partial sums, NS buffers):
+ * the size at which the call takes its fastest form. */
 int lact_workspace_bytes(const lact_desc* desc, size_t* bytes);
+
+/* The smallest workspace lact_chunk_fwd accepts.  It equals
+ * lact_workspace_bytes except for the W2-only layer of "Test-Time Training
+ * with KV Binding Is Secretly Linear Attention", summary "Resultados
+ * Experimentales" (component ablation) and "Formulación Paralela" (causal, GD,
+ * update_mask = 4, normalize_rows = 0, no split operands, d and dh
+ * multiples of 128, chunk a multiple of 128 dividing N_in): that layer is
+ * block-causal linear attention on silu(W1 x) * (W3 x) and runs in parallel
+ * over chunks when the workspace holds every chunk's features and W2
+ * increment (lact_workspace_bytes); with less, down to this size, it runs the
+ * chunk loop.  Both give the same result up to rounding. */
+int lact_workspace_bytes_min(const lact_desc* desc, size_t* bytes);
 
 /* Initialise the state from float32 device weights.  w_per_batch = 0: W1,
  * W3 are [H,dh,d] and W2 [H,d,dh], shared by every batch entry; 1: they are
@@ -191,7 +204,7 @@ int lact_chunk_fwd(const lact_desc* desc, const void* q, const void* k, const vo
  * counterpart: this is a deployment variant, not part of the method.
  * The workspace is a file-scope device array of 64 MiB held by every GPU
  * that loads the library until exit; problems needing more (see
- * lact_workspace_bytes) return TTT_ERR_WORKSPACE and nothing runs.  The
+ * lact_workspace_bytes_min) return TTT_ERR_WORKSPACE and nothing runs.  The
  * first call on a device looks up the array's address with that device
  * current.  All calls share the array: each call clears its status block on
  * `stream`; calls whose GPU work overlaps race and must not be issued.  The

@@ -58,6 +58,7 @@ _SIGS = {
                        _VP],
     "lact_state_bytes": [ctypes.POINTER(lact_desc), _SZP],
     "lact_workspace_bytes": [ctypes.POINTER(lact_desc), _SZP],
+    "lact_workspace_bytes_min": [ctypes.POINTER(lact_desc), _SZP],
     "lact_state_init": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _I, _VP, _VP],
     "lact_state_readout": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _VP, _VP, _VP],
     "lact_chunk_fwd": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
@@ -155,6 +156,13 @@ def lact_workspace_bytes(desc: lact_desc) -> int:
     n = ctypes.c_size_t(0)
     _check("lact_workspace_bytes", load().lact_workspace_bytes(ctypes.byref(desc),
                                                               ctypes.byref(n)))
+    return n.value
+
+
+def lact_workspace_bytes_min(desc: lact_desc) -> int:
+    n = ctypes.c_size_t(0)
+    _check("lact_workspace_bytes_min", load().lact_workspace_bytes_min(ctypes.byref(desc),
+                                                                      ctypes.byref(n)))
     return n.value
 
 

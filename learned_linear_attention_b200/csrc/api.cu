@@ -69,10 +69,10 @@ int check_lact(const lact_desc* d) {
   return TTT_OK;
 }
 
-LactWorkspace layout_of(const lact_desc* d) {
+LactWorkspace layout_of(const lact_desc* d, int allow_parallel) {
   return lact_workspace_layout(d->B, d->H, d->N_in, d->N_q, d->d, d->dh, d->chunk,
                                d->order == TTT_CAUSAL, (int)d->opt, d->split_operands ? 1 : 0,
-                               d->update_mask, d->normalize_rows);
+                               d->update_mask, d->normalize_rows, allow_parallel);
 }
 
 size_t lact_state_elems(const lact_desc* d) {
@@ -189,7 +189,15 @@ int lact_workspace_bytes(const lact_desc* d, size_t* bytes) {
   int e = check_lact(d);
   if (e) return e;
   if (!bytes) return TTT_ERR_ARG;
-  *bytes = layout_of(d).total;
+  *bytes = layout_of(d, 1).total;
+  return TTT_OK;
+}
+
+int lact_workspace_bytes_min(const lact_desc* d, size_t* bytes) {
+  int e = check_lact(d);
+  if (e) return e;
+  if (!bytes) return TTT_ERR_ARG;
+  *bytes = layout_of(d, 0).total;
   return TTT_OK;
 }
 
@@ -244,8 +252,9 @@ int lact_chunk_fwd(const lact_desc* d, const void* q, const void* k, const void*
   int e = check_lact(d);
   if (e) return e;
   if (!state || !ws) return TTT_ERR_ARG;
-  const LactWorkspace w = layout_of(d);
-  if (ws_bytes < w.total) return TTT_ERR_WORKSPACE;
+  // the smallest workspace runs the chunk loop; launch_lact takes the
+  // parallel form of the W2-only layer when ws_bytes holds its layout
+  if (ws_bytes < layout_of(d, 0).total) return TTT_ERR_WORKSPACE;
   const bool causal = d->order == TTT_CAUSAL;
   const int n_out = causal ? d->N_in : d->N_q;
   if (d->N_in > 0 && (!k || !v || !lr)) return TTT_ERR_ARG;

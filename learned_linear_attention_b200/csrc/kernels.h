@@ -112,8 +112,11 @@ struct LactWorkspace {
 bool lact_uses_keygrad(int d, int dh, int opt, int split);
 bool lact_uses_w2_parallel(int N_in, int chunk, int d, int dh, int causal, int opt, int split,
                            int update_mask, int normalize);
+// allow_parallel = 0 lays out the chunk loop even where the parallel form of
+// the W2-only layer applies (its workspace holds every chunk at once).
 LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
-                                    int causal, int opt, int split, int update_mask, int normalize);
+                                    int causal, int opt, int split, int update_mask, int normalize,
+                                    int allow_parallel);
 int launch_lact(const LactLaunch& L, cudaStream_t stream);
 
 // Fused key pass + chunk gradient (head dim 128): partial sums per token group.

@@ -835,14 +835,16 @@ bool lact_uses_w2_parallel(int N_in, int chunk, int d, int dh, int causal, int o
 
 LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int dh, int chunk,
                                     int causal, int opt, int split, int update_mask,
-                                    int normalize) {
+                                    int normalize, int allow_parallel) {
   LactWorkspace w{};
   const size_t BH = (size_t)B * H;
   const int cin = std::min(chunk, std::max(N_in, 1));
   int cmax = std::max(cin, causal ? 0 : N_q);
   cmax = (cmax + 127) / 128 * 128;
   w.cmax = cmax;
-  w.w2par = lact_uses_w2_parallel(N_in, chunk, d, dh, causal, opt, split, update_mask, normalize) ? 1 : 0;
+  w.w2par = allow_parallel &&
+                    lact_uses_w2_parallel(N_in, chunk, d, dh, causal, opt, split, update_mask, normalize)
+                ? 1 : 0;
   if (w.w2par) {   // every token at once: features, increments per chunk, chunk-start weights
     const int nch = N_in / chunk;
     w.cmax = (N_in + 127) / 128 * 128;
@@ -979,9 +981,14 @@ __global__ void w2_prefix_kernel(float* W2, const float* part, __nv_bfloat16* Mb
 int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   const int BH = L.B * L.H, d = L.d, dh = L.dh;
   const bool split = L.split != 0;
-  const LactWorkspace w =
+  // the parallel form of the W2-only layer runs when the workspace holds it,
+  // else the chunk loop
+  LactWorkspace w =
       lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt, L.split,
-                            L.update_mask, L.normalize_rows);
+                            L.update_mask, L.normalize_rows, 1);
+  if (w.w2par && w.total > L.ws_bytes)
+    w = lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt, L.split,
+                              L.update_mask, L.normalize_rows, 0);
   uint8_t* ws = L.ws;
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
   const size_t wsz = (size_t)BH * d * dh;

@@ -10,8 +10,9 @@
 //
 // Limits and sharing:
 //   * the scratch array holds kNoAllocScratchBytes (64 MiB); problems whose
-//     lact_workspace_bytes() exceeds it are rejected with TTT_ERR_WORKSPACE
-//     before anything is enqueued;
+//     lact_workspace_bytes_min() exceeds it are rejected with
+//     TTT_ERR_WORKSPACE before anything is enqueued, and a problem whose
+//     fastest form needs more runs the form that fits;
 //   * every GPU on which the library's device code is loaded holds the array
 //     until the process exits;
 //   * all calls share the one array and it keeps the last call's contents:
@@ -57,7 +58,7 @@ extern "C" int lact_chunk_fwd_noalloc(const lact_desc* desc, const void* q, cons
                                       const void* v, const float* lr, void* state, void* out,
                                       void* stream) {
   size_t need = 0;
-  const int e = lact_workspace_bytes(desc, &need);
+  const int e = lact_workspace_bytes_min(desc, &need);
   if (e != TTT_OK) return e;
   if (need > kNoAllocScratchBytes) return TTT_ERR_WORKSPACE;
   void* scratch = scratch_on_current_device();

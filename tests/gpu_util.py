@@ -44,7 +44,7 @@ def run_linear(x, include_diag=True, out_dtype="f32", S0=None, chunk=None, strea
 class LaCTRun:
     """One LaCT problem on the device: descriptor, state, workspace."""
 
-    def __init__(self, x, opt="gd", out_dtype="f32", **kw):
+    def __init__(self, x, opt="gd", out_dtype="f32", min_workspace=False, **kw):
         B, H, N, d = x.k.values.shape
         dh = x.W1.shape[-2]
         nq = x.q.values.shape[2]
@@ -54,7 +54,8 @@ class LaCTRun:
         self.q, self.k, self.v = to_dev(x.q), to_dev(x.k), to_dev(x.v)
         self.lr = torch.from_numpy(x.lr).cuda()
         self.state = T.alloc_lact_state(self.desc)
-        self.ws = T.alloc_workspace(T.lact_workspace_bytes(self.desc))
+        size = T.lact_workspace_bytes_min if min_workspace else T.lact_workspace_bytes
+        self.ws = T.alloc_workspace(size(self.desc))
         odt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
         self.out = torch.full((B, H, nq, d), float("nan"), dtype=odt, device="cuda")
         self.init_state()

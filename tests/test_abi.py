@@ -137,3 +137,25 @@ def test_lact_workspace_sizes_for_the_workloads(lib):
     d5 = T.make_lact_desc(1, 2, 1029120, 384, 768, 65536, N_q=8040, order="bidirectional",
                           opt="muon")
     assert T.lact_workspace_bytes(d5) < 2 << 30
+    for d in (d3, d4, d5):
+        assert T.lact_workspace_bytes_min(d) == T.lact_workspace_bytes(d)
+
+
+def test_w2_only_parallel_form_workspace(lib):
+    # the W2-only GD layer without normalisation holds every chunk's features
+    # ([BH, N, dh] bf16 twice) and W2 increment ([chunks, BH, d, dh] fp32 and
+    # bf16); the chunk loop it falls back to needs the 32K layer's size
+    full = T.make_lact_desc(2, 4, 32768, 128, 256, 2048)
+    w2 = T.make_lact_desc(2, 4, 32768, 128, 256, 2048, update_mask=4, normalize_rows=False)
+    need = T.lact_workspace_bytes(w2)
+    assert need >= 2 * 8 * 32768 * 256 * 2 + 16 * 8 * 128 * 256 * 6
+    assert T.lact_workspace_bytes_min(w2) <= T.lact_workspace_bytes(full) < 64 << 20
+    # not eligible: row norm on, a chunk that does not divide N, momentum
+    for kw in (dict(normalize_rows=True), dict(chunk=3000), dict(opt="momentum")):
+        args = dict(update_mask=4, normalize_rows=False, chunk=2048)
+        args.update(kw)
+        chunk = args.pop("chunk")
+        d = T.make_lact_desc(2, 4, 32768, 128, 256, chunk, **args)
+        assert T.lact_workspace_bytes(d) == T.lact_workspace_bytes_min(d)
+    # a workspace below the minimum is rejected before any launch
+    assert _call_lact(w2, ws_bytes=T.lact_workspace_bytes_min(w2) - 256) == T.TTT_ERR_WORKSPACE

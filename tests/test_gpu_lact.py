@@ -209,3 +209,17 @@ def test_w2_only_parallel_form(cuda_device, out_dtype):
     run, *_ = _check(x, out_dtype=out_dtype, update_mask=4, normalize_rows=False)
     W = run.weights()
     assert np.array_equal(W[0][0], x.W1) and np.array_equal(W[1][0], x.W3)
+
+
+def test_w2_only_chunk_loop_in_the_minimum_workspace(cuda_device):
+    """Given only lact_workspace_bytes_min, the same W2-only layer runs the
+    chunk loop instead of the parallel form; both match the oracle."""
+    x = make_lact_inputs(2, 2, 2048, 128, 256, chunk=256, order="causal", cfg=47)
+    kw = dict(update_mask=4, normalize_rows=False)
+    fast, loop = LaCTRun(x, **kw), LaCTRun(x, min_workspace=True, **kw)
+    assert loop.ws.numel() < fast.ws.numel()
+    a, b = fast.run(), loop.run()
+    ref, st = _oracle(x, "gd", **kw)
+    assert rel_err(b, ref) <= TOL, rel_err(b, ref)
+    assert rel_err(a, ref) <= TOL, rel_err(a, ref)
+    assert rel_err(loop.weights()[2], st.W2) <= TOL
