@@ -10,7 +10,8 @@ the seeded input module ``ttt_synth``.
 Contents
   ttt_linear  -- linear fast weight trained on the negative inner-product
                  binding loss (token-by-token recurrence) and the equivalent
-                 causal linear-attention sum.
+                 causal linear-attention sum; the backward pass (gradients of
+                 a linear functional of the outputs and final state).
   lact        -- large-chunk TTT with a SwiGLU fast-weight memory: chunk
                  gradients, GD / momentum / Muon (Newton-Schulz) updates, row
                  L2 normalisation, causal and bidirectional ordering.
@@ -18,6 +19,7 @@ Contents
 Every function names the passage of the pages it follows.  Pins (checks
 against facts that are not this code) live in ``tests/test_oracle_*.py``.
 """
-from .ttt_linear import ttt_linear_recurrent, ttt_linear_attention_sum  # noqa: F401
+from .ttt_linear import (ttt_linear_recurrent, ttt_linear_attention_sum,  # noqa: F401
+                         ttt_linear_backward)
 from .lact import (lact_forward, lact_read, lact_chunk_gradients, newton_schulz,  # noqa: F401
                    silu, silu_prime, LaCTState)

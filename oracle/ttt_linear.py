@@ -68,3 +68,55 @@ def ttt_linear_attention_sum(q, k, v, lr, S0=None, include_diag=True, t_index=No
         if S0 is not None:
             out[:, :, j] += np.einsum("bhij,bhi->bhj", _f64(S0), q[:, :, t])
     return out
+
+
+def ttt_linear_backward(q, k, v, lr, dout, S0=None, dS_end=None, include_diag=True):
+    """Gradients of the recurrence above for the scalar
+        L = sum_t <dout_t, o_t> + <dS_end, S_end>
+    with respect to q, k, v, lr and S0 (the backward pass of the layer, which
+    the pages' training-speed results rely on: "Test-Time Training with KV
+    Binding Is Secretly Linear Attention", section "Resultados Experimentales").
+
+    Written as the reverse-time recurrence of the definition.  With
+    R_s = dS_end + sum of q_t dout_t^T over the tokens t whose read sees token
+    s's update (t >= s inclusive, t > s exclusive), the token's contributions
+    are
+        dk_s = eta_s R_s v_s,  dv_s = eta_s R_s^T k_s,  dlr_s = k_s^T R_s v_s,
+    and the read gives dq_t = S_t dout_t with S_t the state the token read.
+    dS0 = R after the first token.
+
+    q, k: [B,H,N,dk]; v, dout: [B,H,N,dv]; lr: [B,H,N]; S0, dS_end:
+    [B,H,dk,dv] or None (zeros).  Returns (dq, dk, dv, dlr, dS0) in float64.
+    """
+    q, k, v, lr, dout = _f64(q), _f64(k), _f64(v), _f64(lr), _f64(dout)
+    B, H, N, dk_ = q.shape
+    dv_ = v.shape[-1]
+    # forward: the state each token's read sees, S = W^T [dk, dv]
+    S = np.zeros((B, H, dk_, dv_)) if S0 is None else _f64(S0).copy()
+    dq = np.empty((B, H, N, dk_))
+    for t in range(N):
+        inc = lr[:, :, t, None, None] * (k[:, :, t, :, None] * v[:, :, t, None, :])
+        if include_diag:
+            S += inc
+        # o_t = S^T q_t  =>  d q_t = S dout_t
+        dq[:, :, t] = np.einsum("bhij,bhj->bhi", S, dout[:, :, t])
+        if not include_diag:
+            S += inc
+    # reverse: R accumulates the reads' sensitivities to the state
+    R = np.zeros((B, H, dk_, dv_)) if dS_end is None else _f64(dS_end).copy()
+    dk = np.empty((B, H, N, dk_))
+    dv = np.empty((B, H, N, dv_))
+    dlr = np.empty((B, H, N))
+    for s in range(N - 1, -1, -1):
+        read = q[:, :, s, :, None] * dout[:, :, s, None, :]
+        if include_diag:
+            R += read
+        # token s adds eta_s k_s v_s^T to every later state
+        Rv = np.einsum("bhij,bhj->bhi", R, v[:, :, s])
+        RTk = np.einsum("bhij,bhi->bhj", R, k[:, :, s])
+        dk[:, :, s] = lr[:, :, s, None] * Rv
+        dv[:, :, s] = lr[:, :, s, None] * RTk
+        dlr[:, :, s] = np.einsum("bhi,bhi->bh", k[:, :, s], Rv)
+        if not include_diag:
+            R += read
+    return dq, dk, dv, dlr, R
