@@ -276,6 +276,51 @@ class LinearBench:
                 "out_dtype": "bf16", "state_dtype": "f32"}
 
 
+class LinearBwdBench(LinearBench):
+    """Backward pass of the linear layer: gradients of q, k, v, lr and S0
+    from seeded upstream gradients dout and dS_end; float32 gradients."""
+
+    def __init__(self, name, device, seed):
+        super().__init__(name, device, seed)
+        torch, T = self.torch, self.T
+        from ttt_synth import make_linear_grads
+        g = make_linear_grads(self.x, cfg=self.w["cfg"], seed=seed)
+        if self.bf16:
+            self.dout = torch.from_numpy(g.dout.bits.view("int16")).view(torch.bfloat16).to(device)
+        else:
+            self.dout = torch.from_numpy(g.dout.values).to(device)
+        self.dS_end = torch.from_numpy(g.dS_end).to(device)
+        B, H, N, dk, dv = self.B, self.H, self.N, self.dk, self.dv
+        self.grads = [torch.empty(s, device=device) for s in
+                      ((B, H, N, dk), (B, H, N, dk), (B, H, N, dv), (B, H, N), (B, H, dk, dv))]
+        self.out = None
+        self.ws = T.alloc_workspace(T.ttt_linear_bwd_workspace_bytes(self.desc), device)
+
+    def flops_per_step(self):
+        return 4 * super().flops_per_step()
+
+    def bytes_per_step(self):
+        # read q, k, v, dout, lr; write dq, dk, dv, dlr (float32) and dS0
+        BH, N, dk, dv = self.B * self.H, self.N, self.dk, self.dv
+        el = 2 if self.bf16 else 4
+        return BH * N * ((2 * dk + 2 * dv) * el + 4 + (2 * dk + dv) * 4 + 4) + \
+            2 * BH * dk * dv * 4
+
+    def step(self, stream):
+        self.T.ttt_linear_bwd(self.desc, self.q, self.k, self.v, self.lr, None, self.dout,
+                              self.dS_end, *self.grads, self.ws, stream=stream)
+
+    def resident_bytes(self):
+        return sum(t.numel() * t.element_size() for t in
+                   [self.q, self.k, self.v, self.lr, self.dout] + self.grads)
+
+    def config(self):
+        c = super().config()
+        c["pass"] = "backward"
+        c["out_dtype"] = "f32"
+        return c
+
+
 def capture_graph(bench, stream):
     """Capture one step (state init + layer call) in a CUDA graph; replaying
     it removes host launch overhead from the timed region."""
@@ -290,7 +335,10 @@ def capture_graph(bench, stream):
 
 def make_bench(name, device, seed):
     from ttt_synth import WORKLOADS
-    return (LinearBench if WORKLOADS[name]["kind"] == "linear" else LaCTBench)(name, device, seed)
+    w = WORKLOADS[name]
+    if w["kind"] == "linear":
+        return (LinearBwdBench if w.get("backward") else LinearBench)(name, device, seed)
+    return LaCTBench(name, device, seed)
 
 
 # --------------------------------------------------------------------------- timing
@@ -457,7 +505,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="lact_causal_n32k")
     ap.add_argument("--secondary", default="ttt_linear_bf16_n32k")
-    ap.add_argument("--extra", default="lact_bidir_196k,lact_bidir_muon_1m,lact_w2only_causal_n32k",
+    ap.add_argument("--extra", default="lact_bidir_196k,lact_bidir_muon_1m,lact_w2only_causal_n32k,"
+                    "ttt_linear_bwd_bf16_n32k",
                     help="further workloads timed once each (comma list, or none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
@@ -567,6 +616,10 @@ def main():
         extra[name] = {"config": ecfg, "value": job_value(world, eb.tokens_per_step(), ems),
                        "unit": "tokens/s", "ms_per_step": ems, "steps": esteps, "tflops": etf,
                        "frac_bf16_peak": etf / pk["bf16_tflops"],
+                       "hbm": ({"algorithmic_bytes": eb.bytes_per_step(),
+                                "gbs": eb.bytes_per_step() / (ems * 1e-3) / 1e9,
+                                "frac": eb.bytes_per_step() / (ems * 1e-3) / 1e9 / pk["hbm_gbs"]}
+                               if isinstance(eb, LinearBench) else None),
                        "kernels": {k: {"launches_per_step": v["launches"],
                                        "share": v["total_ms"] / etot}
                                    for k, v in sorted(eprof.items(), key=lambda kv: -kv[1]["total_ms"])}}

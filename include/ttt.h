@@ -110,6 +110,31 @@ int ttt_linear_state_readout(const ttt_linear_desc* desc, const float* S, float*
 int ttt_linear_fwd(const ttt_linear_desc* desc, const void* q, const void* k, const void* v,
                    const float* lr, float* S, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Backward pass of ttt_linear_fwd: the gradients of
+ *   L = sum_t <dout_t, out_t> + <dS_end, S_end>
+ * with respect to q, k, v, lr and the start state S0, for training through
+ * the layer ("Test-Time Training with KV Binding Is Secretly Linear
+ * Attention", summary "Resultados Experimentales": the training-time result).
+ * With R_s = dS_end + sum of q_t dout_t^T over the reads t that see token s,
+ *   dq_t = S_t dout_t,  dk_s = lr_s R_s v_s,  dv_s = lr_s R_s^T k_s,
+ *   dlr_s = k_s^T R_s v_s,  dS0 = dS_end + sum_t q_t dout_t^T,
+ * where S_t is the state token t read (desc->include_diag as in the forward
+ * call).  Each is computed as a forward-time causal scan with the roles of
+ * q, k, v and dout exchanged, on the kernels of ttt_linear_fwd.
+ * Inputs (device): q, k [B,H,N,dk], v [B,H,N,dv], lr [B,H,N] as given to the
+ * forward call; S0 [B,H,dk,dv] float32, the forward call's start state (NULL =
+ * zeros); dout [B,H,N,dv] in desc->in_dtype; dS_end [B,H,dk,dv] float32 (NULL =
+ * zeros).  Outputs (device, float32, written in full): dq, dk [B,H,N,dk],
+ * dv [B,H,N,dv], dlr [B,H,N], dS0 [B,H,dk,dv]; desc->out_dtype is not used.
+ * ws: device workspace of at least ttt_linear_bwd_workspace_bytes, status
+ * block first; it must not be shared by calls that overlap in time.
+ * Errors as ttt_linear_fwd; nothing is enqueued when validation fails. */
+int ttt_linear_bwd_workspace_bytes(const ttt_linear_desc* desc, size_t* bytes);
+int ttt_linear_bwd(const ttt_linear_desc* desc, const void* q, const void* k, const void* v,
+                   const float* lr, const float* S0, const void* dout, const float* dS_end,
+                   float* dq, float* dk, float* dv, float* dlr, float* dS0, void* ws,
+                   size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Case (b): LaCT, SwiGLU fast-weight memory with large chunks.
  * "Test-Time Training Done Right" review, "Memoria no lineal y atención

@@ -14,7 +14,8 @@ from ._lib import (  # noqa: F401
     TTT_F32, TTT_OK, TTT_OPT_GD, TTT_OPT_MOMENTUM, TTT_OPT_MUON, TTT_STATUS_BYTES, TTTError,
     lact_chunk_fwd, lact_chunk_fwd_noalloc, lact_desc, lact_state_bytes, lact_state_init, lact_state_readout,
     lact_workspace_bytes, lact_workspace_bytes_min, load, status_string, ttt_build_info, ttt_check_device_status,
-    ttt_linear_desc, ttt_linear_fwd, ttt_linear_state_init, ttt_linear_state_readout,
+    ttt_linear_bwd, ttt_linear_bwd_workspace_bytes, ttt_linear_desc, ttt_linear_fwd,
+    ttt_linear_state_init, ttt_linear_state_readout,
     ttt_linear_workspace_bytes, ttt_profile_begin, ttt_profile_end, ttt_selftest_wait_timeout)
 
 _DT = {"f32": TTT_F32, "fp32": TTT_F32, "bf16": TTT_BF16}

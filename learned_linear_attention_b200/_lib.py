@@ -56,6 +56,8 @@ _SIGS = {
     "ttt_linear_state_readout": [ctypes.POINTER(ttt_linear_desc), _VP, _VP, _VP],
     "ttt_linear_fwd": [ctypes.POINTER(ttt_linear_desc), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ,
                        _VP],
+    "ttt_linear_bwd_workspace_bytes": [ctypes.POINTER(ttt_linear_desc), _SZP],
+    "ttt_linear_bwd": [ctypes.POINTER(ttt_linear_desc)] + [_VP] * 13 + [_SZ, _VP],
     "lact_state_bytes": [ctypes.POINTER(lact_desc), _SZP],
     "lact_workspace_bytes": [ctypes.POINTER(lact_desc), _SZP],
     "lact_workspace_bytes_min": [ctypes.POINTER(lact_desc), _SZP],
@@ -143,6 +145,24 @@ def ttt_linear_fwd(desc, q, k, v, lr, S, out, ws, ws_bytes=None, stream=None, ch
     st = load().ttt_linear_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lr), _ptr(S),
                                _ptr(out), _ptr(ws), nbytes, _stream(stream))
     return _check("ttt_linear_fwd", st) if check else st
+
+
+def ttt_linear_bwd_workspace_bytes(desc: ttt_linear_desc) -> int:
+    n = ctypes.c_size_t(0)
+    _check("ttt_linear_bwd_workspace_bytes",
+           load().ttt_linear_bwd_workspace_bytes(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
+def ttt_linear_bwd(desc, q, k, v, lr, S0, dout, dS_end, dq, dk, dv, dlr, dS0, ws, ws_bytes=None,
+                   stream=None, check=True):
+    """Gradients of sum <dout, out> + <dS_end, S_end> (see include/ttt.h);
+    S0 and dS_end may be None (zeros)."""
+    nbytes = ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
+    st = load().ttt_linear_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lr), _ptr(S0),
+                               _ptr(dout), _ptr(dS_end), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlr),
+                               _ptr(dS0), _ptr(ws), nbytes, _stream(stream))
+    return _check("ttt_linear_bwd", st) if check else st
 
 
 # ------------------------------------------------------------------ LaCT

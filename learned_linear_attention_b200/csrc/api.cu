@@ -176,6 +176,50 @@ int ttt_linear_fwd(const ttt_linear_desc* d, const void* q, const void* k, const
   return r == 0 ? TTT_OK : TTT_ERR_CUDA;
 }
 
+LinearBwdWorkspace linear_bwd_layout(const ttt_linear_desc* d, LinearPlan* plan) {
+  const bool umma = linear_uses_umma(d);
+  if (umma) *plan = ttt_linear_plan(d->B * d->H, d->N, device_sms());
+  return ttt_linear_bwd_layout(d->B * d->H, d->N, d->dk, d->dv, umma ? plan : nullptr);
+}
+
+int ttt_linear_bwd_workspace_bytes(const ttt_linear_desc* d, size_t* bytes) {
+  int e = check_linear(d);
+  if (e) return e;
+  if (!bytes) return TTT_ERR_ARG;
+  LinearPlan plan{};
+  *bytes = linear_bwd_layout(d, &plan).total;
+  return TTT_OK;
+}
+
+int ttt_linear_bwd(const ttt_linear_desc* d, const void* q, const void* k, const void* v,
+                   const float* lr, const float* S0, const void* dout, const float* dS_end,
+                   float* dq, float* dk, float* dv, float* dlr, float* dS0, void* ws,
+                   size_t ws_bytes, void* stream) {
+  int e = check_linear(d);
+  if (e) return e;
+  if (!ws || !dS0) return TTT_ERR_ARG;
+  LinearPlan plan{};
+  const LinearBwdWorkspace w = linear_bwd_layout(d, &plan);
+  if (ws_bytes < w.total) return TTT_ERR_WORKSPACE;
+  if (d->N > 0 && (!q || !k || !v || !lr || !dout || !dq || !dk || !dv || !dlr))
+    return TTT_ERR_ARG;
+  const void* ptrs[] = {q, k, v, lr, S0, dout, dS_end, dq, dk, dv, dlr, dS0, ws};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGN;
+  LinearBwdLaunch L{};
+  L.B = d->B; L.H = d->H; L.N = d->N; L.dk = d->dk; L.dv = d->dv; L.chunk = d->chunk;
+  L.include_diag = d->include_diag ? 1 : 0;
+  L.in_bf16 = d->in_dtype == TTT_BF16;
+  L.umma = linear_uses_umma(d) ? 1 : 0;
+  L.q = q; L.k = k; L.v = v; L.dout = dout; L.lr = lr; L.S0 = S0; L.dS_end = dS_end;
+  L.gq = dq; L.gk = dk; L.gv = dv; L.glr = dlr; L.gS0 = dS0;
+  L.ws = static_cast<uint8_t*>(ws);
+  L.w = w;
+  L.plan = plan;
+  L.st = status_of(ws, 1);
+  return launch_ttt_linear_bwd(L, as_stream(stream)) == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ LaCT
 int lact_state_bytes(const lact_desc* d, size_t* bytes) {
   int e = check_lact(d);

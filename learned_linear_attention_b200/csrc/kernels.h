@@ -75,6 +75,24 @@ int launch_ttt_linear_simt(const LinearLaunch& L, cudaStream_t stream);
 int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream);
 size_t ttt_linear_simt_smem(int dk, int dv);
 
+// Backward pass (ttt_linear_bwd.cu): four forward scans with exchanged roles.
+struct LinearBwdWorkspace {
+  size_t status, ones, r, neg_rt, neg_r, s0t, seg, total;   // byte offsets
+  size_t seg_floats;                                         // segment states of one scan
+};
+LinearBwdWorkspace ttt_linear_bwd_layout(int BH, int N, int dk, int dv, const LinearPlan* plan);
+struct LinearBwdLaunch {
+  int B, H, N, dk, dv, chunk, include_diag, in_bf16, umma;
+  const void *q, *k, *v, *dout;
+  const float *lr, *S0, *dS_end;       // S0, dS_end nullable (zeros)
+  float *gq, *gk, *gv, *glr, *gS0;     // gradients of q, k, v, lr, S0 (float32)
+  uint8_t* ws;
+  LinearBwdWorkspace w;
+  LinearPlan plan;
+  DevStatus st;
+};
+int launch_ttt_linear_bwd(const LinearBwdLaunch& L, cudaStream_t stream);
+
 // ----------------------------------------------------------------- LaCT
 struct LactLaunch {
   int B, H, N_in, N_q, d, dh, chunk;
@@ -136,7 +154,7 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream);
 // ----------------------------------------------------------------- profiling
 enum KernelKind {
   K_LIN_SIMT, K_LIN_UMMA, K_LACT_CAST, K_KEYPASS, K_GEMM_READ, K_GEMM_GRAD, K_UPDATE,
-  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_LIN_SEG, K_NUM
+  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_LIN_SEG, K_LIN_BWD_EW, K_NUM
 };
 void prof_before(int kind, cudaStream_t s);
 void prof_after(int kind, cudaStream_t s);

@@ -94,6 +94,39 @@ def test_linear_validation_before_launch(lib):
     assert T.ttt_linear_workspace_bytes(good) == T.TTT_STATUS_BYTES
 
 
+def _call_linear_bwd(desc, ws_bytes=1 << 40, **ptrs):
+    p = dict(q=16, k=16, v=16, lr=16, S0=0, dout=16, dS_end=0, dq=16, dk=16, dv=16, dlr=16,
+             dS0=16, ws=16)
+    p.update(ptrs)
+    return T.load().ttt_linear_bwd(ctypes.byref(desc), p["q"], p["k"], p["v"], p["lr"], p["S0"],
+                                   p["dout"], p["dS_end"], p["dq"], p["dk"], p["dv"], p["dlr"],
+                                   p["dS0"], p["ws"], ws_bytes, None)
+
+
+def test_linear_backward_validation_before_launch(lib):
+    good = T.make_linear_desc(1, 2, 8, 64, 64, 16)
+    assert _call_linear_bwd(T.make_linear_desc(0, 2, 8, 64, 64, 16)) == T.TTT_ERR_SHAPE
+    assert _call_linear_bwd(T.make_linear_desc(1, 2, 8, 256, 64, 16)) == T.TTT_ERR_UNSUPPORTED
+    assert _call_linear_bwd(good, ws_bytes=T.TTT_STATUS_BYTES) == T.TTT_ERR_WORKSPACE
+    assert _call_linear_bwd(good, dS0=0) == T.TTT_ERR_ARG
+    assert _call_linear_bwd(good, dq=0) == T.TTT_ERR_ARG
+    assert _call_linear_bwd(good, dout=0) == T.TTT_ERR_ARG
+    assert _call_linear_bwd(good, dv=40) == T.TTT_ERR_ALIGN
+    assert _call_linear_bwd(good, S0=8) == T.TTT_ERR_ALIGN
+
+
+def test_linear_backward_workspace(lib):
+    # 32K tokens x 64 heads of dims 64: a float32 lr = 1 array per token, four
+    # [64][64] float32 states per head and the segment states of one scan
+    d = T.make_linear_desc(4, 16, 32768, 64, 64, 64)
+    need = T.ttt_linear_bwd_workspace_bytes(d)
+    floor = T.TTT_STATUS_BYTES + 64 * 32768 * 4 + 4 * 64 * 64 * 64 * 4
+    assert floor <= need <= floor + T.ttt_linear_workspace_bytes(d) + 4096
+    small = T.make_linear_desc(1, 2, 100, 24, 40, 9, in_dtype="f32")
+    assert T.ttt_linear_bwd_workspace_bytes(small) >= T.TTT_STATUS_BYTES + 2 * 100 * 4 + \
+        4 * 2 * 24 * 40 * 4
+
+
 def _call_lact(desc, ws_bytes=1 << 40, **ptrs):
     p = dict(q=16, k=16, v=16, lr=16, state=16, out=16, ws=16)
     p.update(ptrs)

@@ -7,7 +7,8 @@ Both the CPU oracle (through the tests and the bench's CPU baseline) and the
 GPU path receive the very same bytes from here.
 
 Recipe (one PCG64 stream per tensor): ``numpy.random.default_rng([cfg, tid])``
-with ``tid`` 0:q 1:k 2:v 3:lr 4:W1 5:W3 6:W2; float32 draws; per-token L2
+with ``tid`` 0:q 1:k 2:v 3:lr 4:W1 5:W3 6:W2 7:dout 8:dS_end (the output
+and end-state gradients a backward pass receives); float32 draws; per-token L2
 normalisation where the workload says so; a single round-to-nearest-even cast
 to bfloat16 for bf16 workloads.  The workloads mirror the pages' settings:
 the linear fast weight of "Test-Time Training with KV Binding Is Secretly
@@ -20,7 +21,7 @@ from __future__ import annotations
 import dataclasses
 import numpy as np
 
-TID_Q, TID_K, TID_V, TID_LR, TID_W1, TID_W3, TID_W2 = range(7)
+TID_Q, TID_K, TID_V, TID_LR, TID_W1, TID_W3, TID_W2, TID_DOUT, TID_DSEND = range(9)
 
 
 # ---------------------------------------------------------------- bf16 bits
@@ -127,6 +128,22 @@ def make_linear_inputs(B, H, N, dk, dv, *, chunk, dtype, lr_kind, cfg=100, seed=
                         np.ascontiguousarray(lr, np.float32), S0, chunk)
 
 
+@dataclasses.dataclass
+class LinearGrads:
+    dout: TokenTensor             # [B,H,N,dv], the dtype of the layer's inputs
+    dS_end: np.ndarray            # float32 [B,H,dk,dv]
+
+
+def make_linear_grads(x: LinearInputs, *, cfg=100, seed=0) -> LinearGrads:
+    """Upstream gradients for a backward pass over ``x``: dout ~ N(0,1) in
+    the inputs' dtype and dS_end ~ 0.1 N(0,1)."""
+    B, H, N, dk = x.q.values.shape
+    dv = x.v.values.shape[-1]
+    dout = _normal(cfg, TID_DOUT, (B, H, N, dv), seed)
+    dS_end = np.float32(0.1) * _normal(cfg, TID_DSEND, (B, H, dk, dv), seed)
+    return LinearGrads(_token(dout, x.q.dtype), dS_end)
+
+
 def make_lact_inputs(B, H, N, d, dh, *, chunk, order, Nq=None, qk_norm=True,
                      v_norm=False, lr_kind="0.01softplus", cfg=200, seed=0,
                      dtype="bf16") -> LaCTInputs:
@@ -164,6 +181,9 @@ WORKLOADS = {
                                 dtype="f32", lr_kind="0.1sig", cfg=1),
     "ttt_linear_bf16_n32k": dict(kind="linear", B=4, H=16, N=32768, dk=64, dv=64, chunk=64,
                                  dtype="bf16", lr_kind="sig-2", cfg=2),
+    # backward pass of the 32K linear layer (upstream gradients from make_linear_grads)
+    "ttt_linear_bwd_bf16_n32k": dict(kind="linear", B=4, H=16, N=32768, dk=64, dv=64, chunk=64,
+                                     dtype="bf16", lr_kind="sig-2", cfg=2, backward=True),
     "lact_causal_n32k": dict(kind="lact", B=2, H=4, N=32768, d=128, dh=256, chunk=2048,
                              order="causal", qk_norm=True, v_norm=False,
                              lr_kind="0.01softplus", opt="gd", cfg=3),
