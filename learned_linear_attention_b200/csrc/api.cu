@@ -177,9 +177,13 @@ int ttt_linear_fwd(const ttt_linear_desc* d, const void* q, const void* k, const
 }
 
 LinearBwdWorkspace linear_bwd_layout(const ttt_linear_desc* d, LinearPlan* plan) {
-  const bool umma = linear_uses_umma(d);
-  if (umma) *plan = ttt_linear_plan(d->B * d->H, d->N, device_sms());
-  return ttt_linear_bwd_layout(d->B * d->H, d->N, d->dk, d->dv, umma ? plan : nullptr);
+  const int BH = d->B * d->H, sms = device_sms();
+  size_t seg = 0;
+  if (linear_uses_umma(d)) {
+    *plan = ttt_linear_plan(BH, d->N, sms);
+    seg = std::max(plan->ws_floats, ttt_linear_state_sum_floats(BH, d->N, sms));
+  }
+  return ttt_linear_bwd_layout(BH, d->N, d->dk, d->dv, seg);
 }
 
 int ttt_linear_bwd_workspace_bytes(const ttt_linear_desc* d, size_t* bytes) {
@@ -211,6 +215,7 @@ int ttt_linear_bwd(const ttt_linear_desc* d, const void* q, const void* k, const
   L.include_diag = d->include_diag ? 1 : 0;
   L.in_bf16 = d->in_dtype == TTT_BF16;
   L.umma = linear_uses_umma(d) ? 1 : 0;
+  L.sms = device_sms();
   L.q = q; L.k = k; L.v = v; L.dout = dout; L.lr = lr; L.S0 = S0; L.dS_end = dS_end;
   L.gq = dq; L.gk = dk; L.gv = dv; L.glr = dlr; L.gS0 = dS0;
   L.ws = static_cast<uint8_t*>(ws);

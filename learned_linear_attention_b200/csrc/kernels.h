@@ -70,7 +70,14 @@ struct LinearLaunch {
   LinearPlan plan;
   float* seg_state;           // workspace after the status block
   size_t seg_state_floats;
+  const float* out_scale;     // nullable: output row t is multiplied by out_mul * out_scale[bh][t]
+  float out_mul;
 };
+// S <- S + sum_t lr_t k_t v_t^T over all N tokens (bf16, dk = dv = 64), with
+// no outputs: the segment pre-pass run over the whole sequence, then a sum of
+// its unit increments.  Needs L.seg_state_floats >= ttt_linear_state_sum_floats.
+size_t ttt_linear_state_sum_floats(int BH, int N, int sms);
+int launch_ttt_linear_state_sum(const LinearLaunch& L, int sms, cudaStream_t stream);
 int launch_ttt_linear_simt(const LinearLaunch& L, cudaStream_t stream);
 int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream);
 size_t ttt_linear_simt_smem(int dk, int dv);
@@ -80,9 +87,10 @@ struct LinearBwdWorkspace {
   size_t status, ones, r, neg_rt, neg_r, s0t, seg, total;   // byte offsets
   size_t seg_floats;                                         // segment states of one scan
 };
-LinearBwdWorkspace ttt_linear_bwd_layout(int BH, int N, int dk, int dv, const LinearPlan* plan);
+// seg_floats: segment states of one tensor-core scan or of the state pre-pass
+LinearBwdWorkspace ttt_linear_bwd_layout(int BH, int N, int dk, int dv, size_t seg_floats);
 struct LinearBwdLaunch {
-  int B, H, N, dk, dv, chunk, include_diag, in_bf16, umma;
+  int B, H, N, dk, dv, chunk, include_diag, in_bf16, umma, sms;
   const void *q, *k, *v, *dout;
   const float *lr, *S0, *dS_end;       // S0, dS_end nullable (zeros)
   float *gq, *gk, *gv, *glr, *gS0;     // gradients of q, k, v, lr, S0 (float32)

@@ -41,7 +41,8 @@ __global__ void __launch_bounds__(SIMT_THREADS)
     ttt_linear_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                            const Tin* __restrict__ v, const float* __restrict__ lr,
                            float* __restrict__ S, Tout* __restrict__ out, int N, int dk, int dv,
-                           int C, int include_diag) {
+                           int C, int include_diag, const float* __restrict__ out_scale,
+                           float out_mul) {
   extern __shared__ float sm[];
   float* Ss = sm;                       // [dk][dv]
   float* Qs = Ss + dk * dv;             // [C][dk]
@@ -83,6 +84,7 @@ __global__ void __launch_bounds__(SIMT_THREADS)
       float acc = 0.f;
       for (int r = 0; r < dk; ++r) acc = fmaf(Qs[i * dk + r], Ss[r * dv + c], acc);
       for (int j = 0; j < Cc; ++j) acc = fmaf(Ps[i * SIMT_MAXC + j], Vs[j * dv + c], acc);
+      if (out_scale) acc *= out_mul * out_scale[(size_t)bh * N + t0 + i];
       out[v_base + (size_t)(t0 + i) * dv + c] = static_cast<Tout>(acc);
     }
     __syncthreads();
@@ -115,7 +117,8 @@ int launch_ttt_linear_simt(const LinearLaunch& L, cudaStream_t stream) {
       return -1;                                                                             \
     prof_before(K_LIN_SIMT, stream);                                                         \
     kfn<<<grid, block, smem, stream>>>((const TI*)L.q, (const TI*)L.k, (const TI*)L.v, L.lr, \
-                                       L.S, (TO*)L.out, L.N, L.dk, L.dv, C, L.include_diag); \
+                                       L.S, (TO*)L.out, L.N, L.dk, L.dv, C, L.include_diag,   \
+                                       L.out_scale, L.out_mul);                               \
     prof_after(K_LIN_SIMT, stream);                                                          \
   } while (0)
   if (L.in_bf16) {
@@ -168,6 +171,8 @@ struct LinUmmaArgs {
   // earlier segment, and only the last segment writes S.
   int P, R, seg_tiles;
   const float* seg_state;   // [BH][1 + (P - 1) R][64][64]: S0, then the units' increments
+  const float* out_scale;   // nullable: output row t is multiplied by out_mul * out_scale[bh][t]
+  float out_mul;
 };
 
 __global__ void __launch_bounds__(lin::THREADS, 1)
@@ -366,6 +371,11 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       float o[32];
       tmem_ld32(tmem + lane_base + ((tile & 1) ? TM_O1 : TM_O0) + hf * 32, o);
       if (t < a.N) {
+        if (a.out_scale) {
+          const float f = a.out_mul * a.out_scale[(size_t)bh * a.N + t];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] *= f;
+        }
         const size_t base = ((size_t)bh * a.N + t) * D + hf * 32;
         if (a.out_bf16) {
           uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base);
@@ -679,7 +689,7 @@ int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream) {
     pl.seg_tiles = (L.N + 127) / 128;
   }
   LinUmmaArgs a{L.lr, L.S, L.out, L.N, L.include_diag, L.out_bf16, L.st,
-                pl.P, pl.R, pl.seg_tiles, L.seg_state};
+                pl.P, pl.R, pl.seg_tiles, L.seg_state, L.out_scale, L.out_mul};
   if (pl.P > 1) {
     SegStateArgs sa{L.lr, L.S, L.seg_state, L.N, (pl.P - 1) * pl.R, pl.R, pl.seg_tiles, pl.unit_tiles, L.st};
     static bool ss_attr = false;
@@ -705,6 +715,66 @@ int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream) {
   ttt_linear_umma_kernel<<<dim3((unsigned)(BH * pl.P)), dim3(lin::THREADS), lin::SMEM_BYTES, stream>>>(
       mq, mk, mv, a);
   prof_after(K_LIN_UMMA, stream);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// ---------------------------------------------------------------- state sum
+namespace {
+// Units of the whole-sequence pre-pass: enough (head, unit) CTAs to fill the
+// SMs, at least 4 tiles per unit.
+int state_sum_units(int BH, int N, int sms) {
+  const int total = (N + 127) / 128;
+  return std::max(1, std::min(std::min(8, sms / std::max(1, BH)), total / 4));
+}
+
+// S[bh] = seg[bh][0] + sum_u seg[bh][1 + u]  (slot 0 holds the start state)
+__global__ void lin_state_sum_kernel(const float* __restrict__ seg, float* __restrict__ S, int BH,
+                                     int U) {
+  constexpr int DD = 64 * 64;
+  const size_t n = (size_t)BH * DD;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const size_t bh = e / DD, i = e % DD;
+    const float* p = seg + bh * (size_t)(1 + U) * DD + i;
+    float acc = p[0];
+    for (int u = 1; u <= U; ++u) acc += p[(size_t)u * DD];
+    S[e] = acc;
+  }
+}
+}  // namespace
+
+size_t ttt_linear_state_sum_floats(int BH, int N, int sms) {
+  return (size_t)BH * (1 + state_sum_units(BH, N, sms)) * 64 * 64;
+}
+
+int launch_ttt_linear_state_sum(const LinearLaunch& L, int sms, cudaStream_t stream) {
+  const int BH = L.B * L.H;
+  const int U = state_sum_units(BH, L.N, sms);
+  if (L.seg_state == nullptr || L.seg_state_floats < ttt_linear_state_sum_floats(BH, L.N, sms))
+    return -1;
+  CUtensorMap mk, mv;
+  if (make_tmap_bf16_3d(&mk, L.k, 64, L.N, BH, 64 * 2, (uint64_t)L.N * 64 * 2, 64, 128) ||
+      make_tmap_bf16_3d(&mv, L.v, 64, L.N, BH, 64 * 2, (uint64_t)L.N * 64 * 2, 64, 128))
+    return -1;
+  const int total = (L.N + 127) / 128;
+  // one segment of `total` tiles split into U units
+  SegStateArgs sa{L.lr, L.S, L.seg_state, L.N, U, U, total, (total + U - 1) / U, L.st};
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(ttt_linear_segstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)lss::SMEM) != cudaSuccess)
+      return -1;
+    attr = true;
+  }
+  prof_before(K_LIN_SEG, stream);
+  ttt_linear_segstate_kernel<<<dim3((unsigned)(BH * U)), dim3(lss::THREADS), lss::SMEM, stream>>>(
+      mk, mv, sa);
+  prof_after(K_LIN_SEG, stream);
+  const size_t n = (size_t)BH * 64 * 64;
+  prof_before(K_LIN_BWD_EW, stream);
+  lin_state_sum_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 148 * 8), 256, 0, stream>>>(
+      L.seg_state, L.S, BH, U);
+  prof_after(K_LIN_BWD_EW, stream);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -19,8 +19,9 @@
 //   dq:         queries dout, keys v,  values k,    lr,     start S0^T
 // with the opposite diagonal for the two R_s scans (a read that sees token s
 // is one that the scan leaves out).  So the forward kernels do all the
-// token work; two elementwise kernels prepare the start states and apply the
-// learning rates and signs.
+// token work (R_tot, an end state only, comes from the state pre-pass on
+// tensor cores); the dk scan scales its output rows by -lr, and two small
+// kernels prepare the start states and finish dv and dlr.
 #include "../../include/ttt.h"
 #include "kernels.h"
 
@@ -65,26 +66,39 @@ __device__ __forceinline__ float load_f<__nv_bfloat16>(const __nv_bfloat16* p, s
   return __bfloat162float(p[i]);
 }
 
-// One warp per token row: dk <- -eta * dk (the scan gave -R_s v_s); with
-// u = -dv (the scan gave -R_s^T k_s): dlr = v . u, dv <- eta * u.
+// One warp per token row.  The scan gave w = -R_s^T k_s = -u in dv:
+// dlr = v . u,  dv <- eta * u.  (dk comes out of its scan already scaled.)
 template <typename TV>
 __global__ void lin_bwd_finish_kernel(const float* __restrict__ lr, const TV* __restrict__ v,
-                                      float* __restrict__ dk, float* __restrict__ dv,
-                                      float* __restrict__ dlr, size_t rows, int dk_dim,
+                                      float* __restrict__ dv, float* __restrict__ dlr, size_t rows,
                                       int dv_dim) {
   const int lane = threadIdx.x & 31;
   const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
   for (size_t row = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
        row += warps) {
     const float eta = lr[row];
-    float* dkr = dk + row * dk_dim;
-    for (int c = lane; c < dk_dim; c += 32) dkr[c] = -eta * dkr[c];
     float* dvr = dv + row * dv_dim;
     float dot = 0.f;
-    for (int c = lane; c < dv_dim; c += 32) {
-      const float u = -dvr[c];
-      dot = fmaf(load_f(v, row * dv_dim + c), u, dot);
-      dvr[c] = eta * u;
+    if (dv_dim == 64) {   // two adjacent columns per lane, one pass
+      float2 w = reinterpret_cast<float2*>(dvr)[lane];
+      float v0, v1;
+      if constexpr (sizeof(TV) == 2) {
+        const __nv_bfloat162 b = reinterpret_cast<const __nv_bfloat162*>(v + row * 64)[lane];
+        v0 = __low2float(b);
+        v1 = __high2float(b);
+      } else {
+        const float2 f = reinterpret_cast<const float2*>(v + row * 64)[lane];
+        v0 = f.x;
+        v1 = f.y;
+      }
+      dot = -(v0 * w.x + v1 * w.y);
+      reinterpret_cast<float2*>(dvr)[lane] = make_float2(-eta * w.x, -eta * w.y);
+    } else {
+      for (int c = lane; c < dv_dim; c += 32) {
+        const float u = -dvr[c];
+        dot = fmaf(load_f(v, row * dv_dim + c), u, dot);
+        dvr[c] = eta * u;
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
@@ -99,7 +113,7 @@ unsigned ew_grid(size_t n, int per_block) {
 
 }  // namespace
 
-LinearBwdWorkspace ttt_linear_bwd_layout(int BH, int N, int dk, int dv, const LinearPlan* plan) {
+LinearBwdWorkspace ttt_linear_bwd_layout(int BH, int N, int dk, int dv, size_t seg_floats) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   LinearBwdWorkspace w{};
   size_t o = 0;
@@ -111,7 +125,7 @@ LinearBwdWorkspace ttt_linear_bwd_layout(int BH, int N, int dk, int dv, const Li
   w.neg_r = o; o = up(o + st);
   w.s0t = o; o = up(o + st);
   w.seg = o;
-  w.seg_floats = plan ? plan->ws_floats : 0;
+  w.seg_floats = seg_floats;
   o = up(o + w.seg_floats * sizeof(float));
   w.total = o;
   return w;
@@ -148,7 +162,7 @@ int launch_ttt_linear_bwd(const LinearBwdLaunch& L, cudaStream_t stream) {
 
   // one forward scan; dims are those of its (query/key, value) operands
   auto scan = [&](const void* q, const void* k, const void* v, const float* lr, float* S,
-                  float* out, int dkk, int dvv, int include_diag) -> int {
+                  float* out, int dkk, int dvv, int include_diag, const float* out_scale) -> int {
     LinearLaunch F{};
     F.B = L.B; F.H = L.H; F.N = L.N; F.dk = dkk; F.dv = dvv; F.chunk = L.chunk;
     F.include_diag = include_diag;
@@ -156,6 +170,8 @@ int launch_ttt_linear_bwd(const LinearBwdLaunch& L, cudaStream_t stream) {
     F.out_bf16 = 0;
     F.q = q; F.k = k; F.v = v; F.lr = lr; F.S = S; F.out = out;
     F.st = L.st;
+    F.out_scale = out_scale;
+    F.out_mul = -1.f;
     if (L.umma) {
       F.plan = L.plan;
       F.seg_state = seg;
@@ -165,27 +181,40 @@ int launch_ttt_linear_bwd(const LinearBwdLaunch& L, cudaStream_t stream) {
     return launch_ttt_linear_simt(F, stream);
   };
   const int inc = L.include_diag ? 1 : 0;
-  // R_tot = dS_end + sum_t q_t dout_t^T: end state of the scan with keys q,
-  // values dout; its outputs land in dv, which a later scan overwrites
-  if (scan(L.q, L.q, L.dout, ones, R, L.gv, L.dk, L.dv, 1)) return -1;
+  // R_tot = dS_end + sum_t q_t dout_t^T: on tensor cores the state-only
+  // pre-pass over the whole sequence; otherwise the end state of a scan with
+  // keys q and values dout, whose outputs land in dv (a later scan
+  // overwrites them)
+  if (L.umma) {
+    LinearLaunch F{};
+    F.B = L.B; F.H = L.H; F.N = L.N; F.dk = L.dk; F.dv = L.dv;
+    F.k = L.q; F.v = L.dout; F.lr = ones; F.S = R;
+    F.st = L.st;
+    F.seg_state = seg;
+    F.seg_state_floats = w.seg_floats;
+    if (launch_ttt_linear_state_sum(F, L.sms, stream)) return -1;
+  } else if (scan(L.q, L.q, L.dout, ones, R, L.gv, L.dk, L.dv, 1, nullptr)) {
+    return -1;
+  }
   prof_before(K_LIN_BWD_EW, stream);
   lin_bwd_states_kernel<<<ew_grid(st_elems, EW_THREADS), EW_THREADS, 0, stream>>>(
       R, L.S0, neg_rt, neg_r, s0t, L.gS0, BH, L.dk, L.dv);
   prof_after(K_LIN_BWD_EW, stream);
-  // -R_s v_s -> dk   (queries v, keys dout, values q; state [dv][dk])
-  if (scan(L.v, L.dout, L.q, ones, neg_rt, L.gk, L.dv, L.dk, 1 - inc)) return -1;
+  // dk_s = eta_s R_s v_s: the scan (queries v, keys dout, values q; state
+  // [dv][dk]) gives -R_s v_s and scales its rows by -eta_s
+  if (scan(L.v, L.dout, L.q, ones, neg_rt, L.gk, L.dv, L.dk, 1 - inc, L.lr)) return -1;
   // -R_s^T k_s -> dv (queries k, keys q, values dout; state [dk][dv])
-  if (scan(L.k, L.q, L.dout, ones, neg_r, L.gv, L.dk, L.dv, 1 - inc)) return -1;
+  if (scan(L.k, L.q, L.dout, ones, neg_r, L.gv, L.dk, L.dv, 1 - inc, nullptr)) return -1;
   // dq_t = S_t dout_t (queries dout, keys v, values k, lr; state S0^T [dv][dk])
-  if (scan(L.dout, L.v, L.k, L.lr, s0t, L.gq, L.dv, L.dk, inc)) return -1;
+  if (scan(L.dout, L.v, L.k, L.lr, s0t, L.gq, L.dv, L.dk, inc, nullptr)) return -1;
   prof_before(K_LIN_BWD_EW, stream);
   const unsigned g = ew_grid(rows, EW_THREADS / 32);
   if (L.in_bf16)
     lin_bwd_finish_kernel<<<g, EW_THREADS, 0, stream>>>(
-        L.lr, static_cast<const __nv_bfloat16*>(L.v), L.gk, L.gv, L.glr, rows, L.dk, L.dv);
+        L.lr, static_cast<const __nv_bfloat16*>(L.v), L.gv, L.glr, rows, L.dv);
   else
     lin_bwd_finish_kernel<<<g, EW_THREADS, 0, stream>>>(
-        L.lr, static_cast<const float*>(L.v), L.gk, L.gv, L.glr, rows, L.dk, L.dv);
+        L.lr, static_cast<const float*>(L.v), L.gv, L.glr, rows, L.dv);
   prof_after(K_LIN_BWD_EW, stream);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
