@@ -15,6 +15,8 @@ Contents
   lact        -- large-chunk TTT with a SwiGLU fast-weight memory: chunk
                  gradients, GD / momentum / Muon (Newton-Schulz) updates, row
                  L2 normalisation, causal and bidirectional ordering.
+  window_attention -- causal sliding-window softmax attention, and the LaCT
+                 language layer (memory + window attention, outputs summed).
 
 Every function names the passage of the pages it follows.  Pins (checks
 against facts that are not this code) live in ``tests/test_oracle_*.py``.
@@ -23,3 +25,4 @@ from .ttt_linear import (ttt_linear_recurrent, ttt_linear_attention_sum,  # noqa
                          ttt_linear_backward)
 from .lact import (lact_forward, lact_read, lact_chunk_gradients, newton_schulz,  # noqa: F401
                    silu, silu_prime, LaCTState)
+from .window_attention import sliding_window_attention, lact_layer_forward  # noqa: F401
