@@ -238,6 +238,41 @@ int lact_chunk_fwd_noalloc(const lact_desc* desc, const void* q, const void* k, 
                            const float* lr, void* state, void* out, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Local branch of the LaCT language layer: causal sliding-window attention.
+ * "Test-Time Training Done Right" review, "Memoria no lineal y atención
+ * local", "El orden de lectura evita información futura" and "Lenguaje"
+ * (window 2048 for the 760M model, 4096 for the 3B one):
+ *
+ *   o_i = sum over j in (i - window, i] of softmax_j(scale q_i . k_j) v_j
+ *
+ * The window counts the token itself; scale <= 0 selects 1 / sqrt(d).
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int B, H, N;          /* N >= 0                                            */
+  int d;                /* head dim of q, k and v: 128                       */
+  int window;           /* >= 1                                              */
+  float scale;
+  ttt_dtype in_dtype;   /* TTT_BF16                                          */
+  ttt_dtype out_dtype;  /* TTT_F32 or TTT_BF16                               */
+  int accumulate;       /* 0: out = attention; 1: out += attention           */
+} ttt_window_desc;
+
+/* q, k, v: device [B,H,N,d] bf16; out: device [B,H,N,d] in out_dtype (read
+ * as well when accumulate = 1).  ws: at least TTT_STATUS_BYTES (status
+ * block).  Tensor cores (tcgen05), one CTA per 128-query tile. */
+int ttt_window_attn_fwd(const ttt_window_desc* desc, const void* q, const void* k, const void* v,
+                        void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* The LaCT language layer in causal order: the fast-weight memory of
+ * lact_chunk_fwd and the sliding-window attention above on the same q, k, v,
+ * outputs summed into out (the window branch adds its output in its
+ * epilogue).  desc as for lact_chunk_fwd (causal, d = 128); window and scale
+ * as in ttt_window_desc; ws as for lact_chunk_fwd. */
+int lact_layer_fwd(const lact_desc* desc, int window, float scale, const void* q, const void* k,
+                   const void* v, const float* lr, void* state, void* out, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Status and diagnostics
  * ---------------------------------------------------------------------- */
 

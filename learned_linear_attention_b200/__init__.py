@@ -12,7 +12,8 @@ from ._lib import (  # noqa: F401
     LIB_PATH, TTT_BF16, TTT_BIDIRECTIONAL, TTT_CAUSAL, TTT_ERR_ALIGN, TTT_ERR_ARG, TTT_ERR_CUDA,
     TTT_ERR_DTYPE, TTT_ERR_SHAPE, TTT_ERR_TIMEOUT, TTT_ERR_UNSUPPORTED, TTT_ERR_WORKSPACE,
     TTT_F32, TTT_OK, TTT_OPT_GD, TTT_OPT_MOMENTUM, TTT_OPT_MUON, TTT_STATUS_BYTES, TTTError,
-    lact_chunk_fwd, lact_chunk_fwd_noalloc, lact_desc, lact_state_bytes, lact_state_init, lact_state_readout,
+    lact_chunk_fwd, lact_chunk_fwd_noalloc, lact_desc, lact_layer_fwd, ttt_window_attn_fwd,
+    ttt_window_desc, lact_state_bytes, lact_state_init, lact_state_readout,
     lact_workspace_bytes, lact_workspace_bytes_min, load, status_string, ttt_build_info, ttt_check_device_status,
     ttt_linear_bwd, ttt_linear_bwd_workspace_bytes, ttt_linear_desc, ttt_linear_fwd,
     ttt_linear_state_init, ttt_linear_state_readout,
@@ -45,6 +46,13 @@ def make_lact_desc(B, H, N_in, d, dh, chunk, *, N_q=None, order="causal", opt="g
     desc.update_mask, desc.in_dtype, desc.out_dtype = update_mask, TTT_BF16, _DT[out_dtype]
     desc.split_operands = int(opt == "muon") if split_operands is None else int(bool(split_operands))
     return desc
+
+
+def make_window_desc(B, H, N, d, window, *, scale=0.0, out_dtype="f32",
+                     accumulate=False) -> ttt_window_desc:
+    """Fill a ttt_window_desc (bf16 q, k, v; scale <= 0 selects 1/sqrt(d))."""
+    return ttt_window_desc(B, H, N, d, window, scale, TTT_BF16, _DT[out_dtype],
+                           int(bool(accumulate)))
 
 
 def alloc_workspace(nbytes: int, device="cuda"):

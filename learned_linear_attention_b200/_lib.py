@@ -44,6 +44,12 @@ class lact_desc(ctypes.Structure):
                 ("out_dtype", ctypes.c_int), ("split_operands", ctypes.c_int)]
 
 
+class ttt_window_desc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int),
+                ("window", ctypes.c_int), ("scale", ctypes.c_float), ("in_dtype", ctypes.c_int),
+                ("out_dtype", ctypes.c_int), ("accumulate", ctypes.c_int)]
+
+
 class ttt_prof_entry(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int),
                 ("total_ms", ctypes.c_double)]
@@ -58,6 +64,9 @@ _SIGS = {
                        _VP],
     "ttt_linear_bwd_workspace_bytes": [ctypes.POINTER(ttt_linear_desc), _SZP],
     "ttt_linear_bwd": [ctypes.POINTER(ttt_linear_desc)] + [_VP] * 13 + [_SZ, _VP],
+    "ttt_window_attn_fwd": [ctypes.POINTER(ttt_window_desc), _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "lact_layer_fwd": [ctypes.POINTER(lact_desc), _I, ctypes.c_float, _VP, _VP, _VP, _VP, _VP, _VP,
+                       _VP, _SZ, _VP],
     "lact_state_bytes": [ctypes.POINTER(lact_desc), _SZP],
     "lact_workspace_bytes": [ctypes.POINTER(lact_desc), _SZP],
     "lact_workspace_bytes_min": [ctypes.POINTER(lact_desc), _SZP],
@@ -163,6 +172,22 @@ def ttt_linear_bwd(desc, q, k, v, lr, S0, dout, dS_end, dq, dk, dv, dlr, dS0, ws
                                _ptr(dout), _ptr(dS_end), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlr),
                                _ptr(dS0), _ptr(ws), nbytes, _stream(stream))
     return _check("ttt_linear_bwd", st) if check else st
+
+
+def ttt_window_attn_fwd(desc, q, k, v, out, ws, ws_bytes=None, stream=None, check=True):
+    nbytes = ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
+    st = load().ttt_window_attn_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                    _ptr(ws), nbytes, _stream(stream))
+    return _check("ttt_window_attn_fwd", st) if check else st
+
+
+def lact_layer_fwd(desc, window, scale, q, k, v, lr, state, out, ws, ws_bytes=None, stream=None,
+                   check=True):
+    nbytes = ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
+    st = load().lact_layer_fwd(ctypes.byref(desc), int(window), float(scale), _ptr(q), _ptr(k),
+                               _ptr(v), _ptr(lr), _ptr(state), _ptr(out), _ptr(ws), nbytes,
+                               _stream(stream))
+    return _check("lact_layer_fwd", st) if check else st
 
 
 # ------------------------------------------------------------------ LaCT

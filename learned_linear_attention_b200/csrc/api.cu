@@ -3,6 +3,7 @@
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
+#include <math.h>
 
 #include <algorithm>
 
@@ -225,6 +226,43 @@ int ttt_linear_bwd(const ttt_linear_desc* d, const void* q, const void* k, const
   return launch_ttt_linear_bwd(L, as_stream(stream)) == 0 ? TTT_OK : TTT_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ window attention
+static int check_window(const ttt_window_desc* d) {
+  if (!d) return TTT_ERR_ARG;
+  if (d->B < 1 || d->H < 1 || d->N < 0) return TTT_ERR_SHAPE;
+  if (d->window < 1) return TTT_ERR_ARG;
+  if (d->in_dtype != TTT_BF16) return TTT_ERR_DTYPE;
+  if (d->out_dtype != TTT_F32 && d->out_dtype != TTT_BF16) return TTT_ERR_DTYPE;
+  if (d->d != 128) return TTT_ERR_UNSUPPORTED;
+  if ((long long)d->B * d->H * d->N > (1ll << 31)) return TTT_ERR_SHAPE;
+  return TTT_OK;
+}
+
+static int run_window(const ttt_window_desc* d, const void* q, const void* k, const void* v,
+                      void* out, void* ws, void* stream) {
+  WindowAttnLaunch L{};
+  L.B = d->B; L.H = d->H; L.N = d->N; L.window = d->window;
+  L.scale = d->scale > 0.f ? d->scale : 1.f / sqrtf((float)d->d);
+  L.out_bf16 = d->out_dtype == TTT_BF16;
+  L.accumulate = d->accumulate ? 1 : 0;
+  L.q = q; L.k = k; L.v = v; L.out = out;
+  L.st = status_of(ws, 3);
+  return launch_window_attention(L, as_stream(stream)) == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
+int ttt_window_attn_fwd(const ttt_window_desc* d, const void* q, const void* k, const void* v,
+                        void* out, void* ws, size_t ws_bytes, void* stream) {
+  int e = check_window(d);
+  if (e) return e;
+  if (!ws) return TTT_ERR_ARG;
+  if (ws_bytes < TTT_STATUS_BYTES) return TTT_ERR_WORKSPACE;
+  if (d->N == 0) return TTT_OK;
+  if (!q || !k || !v || !out) return TTT_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
+    return TTT_ERR_ALIGN;
+  return run_window(d, q, k, v, out, ws, stream);
+}
+
 // ------------------------------------------------------------------ LaCT
 int lact_state_bytes(const lact_desc* d, size_t* bytes) {
   int e = check_lact(d);
@@ -327,6 +365,22 @@ int lact_chunk_fwd(const lact_desc* d, const void* q, const void* k, const void*
   L.ws_bytes = ws_bytes;
   L.st = status_of(ws, 2);
   return launch_lact(L, as_stream(stream)) == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
+int lact_layer_fwd(const lact_desc* d, int window, float scale, const void* q, const void* k,
+                   const void* v, const float* lr, void* state, void* out, void* ws,
+                   size_t ws_bytes, void* stream) {
+  int e = check_lact(d);
+  if (e) return e;
+  if (d->order != TTT_CAUSAL) return TTT_ERR_ARG;
+  ttt_window_desc wd{};
+  wd.B = d->B; wd.H = d->H; wd.N = d->N_in; wd.d = d->d; wd.window = window; wd.scale = scale;
+  wd.in_dtype = d->in_dtype; wd.out_dtype = d->out_dtype; wd.accumulate = 1;
+  e = check_window(&wd);
+  if (e) return e;
+  e = lact_chunk_fwd(d, q, k, v, lr, state, out, ws, ws_bytes, stream);
+  if (e || d->N_in == 0) return e;
+  return run_window(&wd, q, k, v, out, ws, stream);
 }
 
 // ------------------------------------------------------------------ status

@@ -101,6 +101,19 @@ struct LinearBwdLaunch {
 };
 int launch_ttt_linear_bwd(const LinearBwdLaunch& L, cudaStream_t stream);
 
+// ----------------------------------------------------------------- window attention
+// Causal sliding-window softmax attention, head dim 128, bf16 q, k, v
+// [B,H,N,128]; out fp32 or bf16, overwritten or (accumulate) added to.
+struct WindowAttnLaunch {
+  int B, H, N, window;
+  float scale;
+  int out_bf16, accumulate;
+  const void *q, *k, *v;
+  void* out;
+  DevStatus st;
+};
+int launch_window_attention(const WindowAttnLaunch& L, cudaStream_t stream);
+
 // ----------------------------------------------------------------- LaCT
 struct LactLaunch {
   int B, H, N_in, N_q, d, dh, chunk;
@@ -162,7 +175,7 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream);
 // ----------------------------------------------------------------- profiling
 enum KernelKind {
   K_LIN_SIMT, K_LIN_UMMA, K_LACT_CAST, K_KEYPASS, K_GEMM_READ, K_GEMM_GRAD, K_UPDATE,
-  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_LIN_SEG, K_LIN_BWD_EW, K_NUM
+  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_LIN_SEG, K_LIN_BWD_EW, K_SWA, K_NUM
 };
 void prof_before(int kind, cudaStream_t s);
 void prof_after(int kind, cudaStream_t s);

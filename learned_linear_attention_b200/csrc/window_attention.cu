@@ -1,0 +1,350 @@
+// window_attention.cu -- causal sliding-window softmax attention, the local
+// branch of the LaCT language layer ("Test-Time Training Done Right" review,
+// "Memoria no lineal y atención local" and "El orden de lectura evita
+// información futura": windowed attention and the fast-weight memory share
+// Q, K and V and their outputs are summed; the causal sliding window keeps
+// future tokens out).
+//
+// o_i = sum over j in (i - W, i] of softmax_j(scale q_i . k_j) v_j, head dim
+// 128, bf16 q, k, v, fp32 accumulation.
+//
+// One CTA per (head, 128-query tile) walks the window's 128-key tiles twice:
+//   pass 1   S = Q K^T (tcgen05, TMEM)  -> row max m and row sum l (online)
+//   pass 2   S = Q K^T again            -> P = exp(S - m) / l, bf16 in smem
+//            O += P V (tcgen05, TMEM)
+// so O accumulates already-normalised terms and is never rescaled.  S
+// alternates between two TMEM buffers and P between two shared buffers, so
+// the tensor cores work on one key tile while the epilogue warps work on the
+// previous one.  K/V tiles are double-buffered by TMA (pass 1 loads K only).
+#include <algorithm>
+
+#include "kernels.h"
+
+namespace ttt {
+namespace swa {
+constexpr int D = 128, BM = 128, BN = 128;
+constexpr uint32_t HALF = 128 * 64 * 2;          // 16 KB: 128 rows x 64 bf16 (one swizzle atom wide)
+constexpr uint32_t TILE = 2 * HALF;              // 32 KB: 128 rows x 128 bf16
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_KV = TILE;                // 2 stages x (K | V)
+constexpr uint32_t KV_STAGE = 2 * TILE;
+constexpr uint32_t OFF_P = OFF_KV + 2 * KV_STAGE;  // 2 x P (128 queries x 128 keys)
+constexpr uint32_t OFF_BAR = OFF_P + 2 * TILE;
+constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+constexpr int EPI_WARPS = 4;                      // one per TMEM lane quadrant; a thread per query row
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_COLS = 512;
+}  // namespace swa
+
+struct SwaArgs {
+  int N, window, n_qt;
+  float scale_log2;     // scale * log2(e): scores go through exp2
+  int out_bf16, accumulate;
+  void* out;            // [BH][N][128]
+  DevStatus st;
+};
+struct SwaMaps {
+  CUtensorMap q, k, v;
+};
+
+__global__ void __launch_bounds__(swa::THREADS, 1)
+    window_attention_kernel(const __grid_constant__ SwaMaps maps, const SwaArgs a) {
+  using namespace swa;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* kv_full = q_full + 1;     // [2]
+  uint64_t* kv_empty = kv_full + 2;   // [2]
+  uint64_t* s_full = kv_empty + 2;    // [2]
+  uint64_t* s_empty = s_full + 2;     // [2]
+  uint64_t* p_full = s_empty + 2;     // [2]
+  uint64_t* p_empty = p_full + 2;     // [2]
+  uint64_t* o_full = p_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the tiles with the most keys (late in the sequence) first
+  const int bh = blockIdx.x / a.n_qt;
+  const int qt = a.n_qt - 1 - (int)(blockIdx.x % a.n_qt);
+  const int q0 = qt * BM;
+  const int kt_lo = max(0, q0 - a.window + 1) / BN;   // first key tile of the window
+  const int nk = qt - kt_lo + 1;                            // key tiles per pass
+  const int G = 2 * nk;                                     // pass 1, then pass 2
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], EPI_WARPS * 32);
+      mbar_init(&p_full[s], EPI_WARPS * 32);
+      mbar_init(&p_empty[s], 1);
+    }
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.q);
+    tma_prefetch_desc(&maps.k);
+    tma_prefetch_desc(&maps.v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  Waiter W{abort_flag, a.st, 400};
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, TILE);
+      tma_load_3d(smem + OFF_Q, &maps.q, q_full, 0, q0, bh);
+      tma_load_3d(smem + OFF_Q + HALF, &maps.q, q_full, 64, q0, bh);
+      int issued = 0;
+      for (int g = 0; g < G; ++g) {
+        const int s = g & 1;
+        if (g >= 2 && !W.wait(&kv_empty[s], ((g >> 1) - 1) & 1, 1)) break;
+        const bool pass2 = g >= nk;
+        const int row = (kt_lo + (pass2 ? g - nk : g)) * BN;
+        uint8_t* st = smem + OFF_KV + s * KV_STAGE;
+        mbar_arrive_expect_tx(&kv_full[s], pass2 ? KV_STAGE : TILE);
+        tma_load_3d(st, &maps.k, &kv_full[s], 0, row, bh);
+        tma_load_3d(st + HALF, &maps.k, &kv_full[s], 64, row, bh);
+        if (pass2) {
+          tma_load_3d(st + TILE, &maps.v, &kv_full[s], 0, row, bh);
+          tma_load_3d(st + TILE + HALF, &maps.v, &kv_full[s], 64, row, bh);
+        }
+        issued = g + 1;
+      }
+      if (W.aborted()) {
+        W.drain(q_full, 0);
+        for (int g = max(0, issued - 2); g < issued; ++g) W.drain(&kv_full[g & 1], (g >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id_s = make_idesc(128, 128, false, false);   // Q, K both K-major (d)
+      const uint32_t id_o = make_idesc(128, 128, false, true);    // P K-major (keys), V MN-major
+      const uint64_t dq = make_sdesc(smem_u32(smem + OFF_Q), 16, 1024);
+      const uint64_t dkv = make_sdesc(smem_u32(smem + OFF_KV), 16, 1024);
+      const uint64_t dv0 = make_sdesc(smem_u32(smem + OFF_KV + TILE), HALF, 1024);
+      const uint64_t dp0 = make_sdesc(smem_u32(smem + OFF_P), 16, 1024);
+      bool ok = W.wait(q_full, 0, 2);
+      tc_fence_after();
+      // S(g) = Q K(g)^T into S buffer g & 1
+      auto issue_s = [&](int g) -> bool {
+        const int s = g & 1;
+        if (!W.wait(&kv_full[s], (g >> 1) & 1, 3)) return false;
+        if (g >= 2 && !W.wait(&s_empty[s], ((g >> 1) - 1) & 1, 4)) return false;
+        tc_fence_after();
+        const uint64_t dk = sdesc_add(dkv, s * KV_STAGE);
+        const uint32_t acc = tmem + (s ? TM_S1 : TM_S0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+          mma_bf16(acc, sdesc_add(dq, off), sdesc_add(dk, off), id_s, kk > 0);
+        }
+        mma_commit(&s_full[s]);
+        if (g < nk) mma_commit(&kv_empty[s]);   // pass 1 is done with this K tile
+        return true;
+      };
+      if (ok && G > 0) ok = issue_s(0);
+      for (int g = 0; ok && g < G; ++g) {
+        // the next tile's scores first, so they run while the epilogue
+        // turns this tile's scores into P
+        if (g + 1 < G && !issue_s(g + 1)) { ok = false; break; }
+        if (g >= nk) {
+          // pass-2 tile i: P buffer i & 1, filled for the (i >> 1)-th time
+          const int i = g - nk, pb = i & 1, s = g & 1;
+          if (!W.wait(&p_full[pb], (i >> 1) & 1, 5)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t dv = sdesc_add(dv0, s * KV_STAGE);
+          const uint64_t dp = sdesc_add(dp0, pb * TILE);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t offp = (kk >> 2) * HALF + (kk & 3) * 32;
+            mma_bf16(tmem + TM_O, sdesc_add(dp, offp), sdesc_add(dv, kk * 2048), id_o,
+                     (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&kv_empty[s]);
+          mma_commit(&p_empty[pb]);
+        }
+      }
+      mma_commit(o_full);
+      W.drain(o_full, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;               // query row of the tile
+    const int qi = q0 + r;                      // query token
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const bool row_ok = qi < a.N;
+    float m = -INFINITY, l = 0.f;               // running max (log2 units) and sum
+    bool ok = true;
+    for (int g = 0; ok && g < G; ++g) {
+      const bool pass2 = g >= nk;
+      const int kt = kt_lo + (pass2 ? g - nk : g);
+      const int sb = g & 1;
+      if (!W.wait(&s_full[sb], (g >> 1) & 1, 6)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sbase = tmem + lane_base + (sb ? TM_S1 : TM_S0);
+      if (!pass2) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float x[32];
+          // tcgen05.ld is warp-collective: every lane reaches it, converged
+          __syncwarp();
+          tmem_ld32(sbase + c, x);
+          float cm = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int kj = kt * BN + c + j;
+            const bool valid = row_ok && kj <= qi && kj > qi - a.window;
+            x[j] = valid ? x[j] * a.scale_log2 : -INFINITY;
+            cm = fmaxf(cm, x[j]);
+          }
+          const float mn = fmaxf(m, cm);
+          if (mn != -INFINITY) {   // no valid key yet: m and l stay as they are
+            float add = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) add += exp2f(x[j] - mn);
+            l = l * exp2f(m - mn) + add;
+            m = mn;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&s_empty[sb]);
+      } else {
+        // pass-2 tile i writes P buffer i & 1, free once the P V product of
+        // pass-2 tile i - 2 is done
+        const int i = g - nk, pb = i & 1;
+        if (i >= 2 && !W.wait(&p_empty[pb], ((i >> 1) - 1) & 1, 7)) { ok = false; break; }
+        const float inv_l = row_ok ? 1.f / l : 0.f;
+        const uint32_t pbase = smem_u32(smem + OFF_P + pb * TILE);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float x[32];
+          __syncwarp();
+          tmem_ld32(sbase + c, x);
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            float p2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int kj = kt * BN + c + j + u;
+              const bool valid = row_ok && kj <= qi && kj > qi - a.window;
+              p2[u] = valid ? exp2f(x[j + u] * a.scale_log2 - m) * inv_l : 0.f;
+            }
+            pk[j >> 1] = pack_bf16x2(p2[0], p2[1]);
+          }
+          // keys c .. c + 31 of row r: half c / 64, columns (c % 64) ..
+          const uint32_t hb = pbase + (uint32_t)(c >> 6) * HALF;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8)
+            st_shared_v4(hb + sw128_offset(r, (c & 63) + j), pk[j / 2], pk[j / 2 + 1], pk[j / 2 + 2],
+                         pk[j / 2 + 3]);
+        }
+        tc_fence_before();
+        mbar_arrive(&s_empty[sb]);
+        fence_async_smem();
+        mbar_arrive(&p_full[pb]);
+      }
+    }
+    if (ok && W.wait(o_full, 0, 8)) {
+      tc_fence_after();
+      const size_t base = ((size_t)bh * a.N + qi) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        float o[32];
+        // every lane loads (warp-collective); only rows inside the sequence store
+        __syncwarp();
+        tmem_ld32(tmem + lane_base + TM_O + c, o);
+        if (row_ok) {
+          if (a.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float v8[8];
+              if (a.accumulate) {
+                const uint4 w = dst[j];
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  v8[2 * u] = o[8 * j + 2 * u] + bf16lo(ww[u]);
+                  v8[2 * u + 1] = o[8 * j + 2 * u + 1] + bf16hi(ww[u]);
+                }
+              } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v8[u] = o[8 * j + u];
+              }
+              dst[j] = make_uint4(pack_bf16x2(v8[0], v8[1]), pack_bf16x2(v8[2], v8[3]),
+                                  pack_bf16x2(v8[4], v8[5]), pack_bf16x2(v8[6], v8[7]));
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base + c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float4 v4 = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+              if (a.accumulate) {
+                const float4 w = dst[j];
+                v4.x += w.x; v4.y += w.y; v4.z += w.z; v4.w += w.w;
+              }
+              dst[j] = v4;
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
+int launch_window_attention(const WindowAttnLaunch& L, cudaStream_t stream) {
+  using namespace swa;
+  const uint64_t BH = (uint64_t)L.B * L.H;
+  if (L.N == 0) return 0;
+  SwaMaps m;
+  const uint64_t row = D * 2;
+  if (make_tmap_bf16_3d(&m.q, L.q, D, L.N, BH, row, row * L.N, 64, 128) ||
+      make_tmap_bf16_3d(&m.k, L.k, D, L.N, BH, row, row * L.N, 64, 128) ||
+      make_tmap_bf16_3d(&m.v, L.v, D, L.N, BH, row, row * L.N, 64, 128))
+    return -1;
+  SwaArgs a{};
+  a.N = L.N;
+  a.window = L.window;
+  a.n_qt = (L.N + BM - 1) / BM;
+  a.scale_log2 = L.scale * 1.4426950408889634f;
+  a.out_bf16 = L.out_bf16;
+  a.accumulate = L.accumulate;
+  a.out = L.out;
+  a.st = L.st;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(window_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SMEM) != cudaSuccess)
+      return -1;
+    attr = true;
+  }
+  prof_before(K_SWA, stream);
+  window_attention_kernel<<<dim3((unsigned)(BH * a.n_qt)), dim3(THREADS), SMEM, stream>>>(m, a);
+  prof_after(K_SWA, stream);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace ttt

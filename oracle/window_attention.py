@@ -20,23 +20,28 @@ from __future__ import annotations
 import numpy as np
 
 
-def sliding_window_attention(q, k, v, window, scale=None):
+def sliding_window_attention(q, k, v, window, scale=None, t_index=None):
     """o_t = sum over s in (t - window, t] of softmax_s(scale q_t . k_s) v_s.
 
-    q, k: [B,H,N,d]; v: [B,H,N,dv].  Token by token, float64.
+    q, k: [B,H,N,d]; v: [B,H,N,dv].  Token by token, float64.  With
+    ``t_index`` only those positions are computed (sampled checks at full
+    sizes); the result is then [B,H,len(t_index),dv].
     """
-    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
-    B, H, N, d = q.shape
+    B, H, N, d = np.shape(q)
     if scale is None:
         scale = 1.0 / np.sqrt(d)
-    out = np.empty(v.shape[:3] + (v.shape[-1],))
-    for t in range(N):
+    idx = range(N) if t_index is None else list(t_index)
+    out = np.empty((B, H, len(idx), np.shape(v)[-1]))
+    for j, t in enumerate(idx):
         s0 = max(0, t - window + 1)
-        scores = scale * np.einsum("bhd,bhsd->bhs", q[:, :, t], k[:, :, s0:t + 1])
+        qt = np.asarray(q[:, :, t], dtype=np.float64)
+        ks = np.asarray(k[:, :, s0:t + 1], dtype=np.float64)
+        vs = np.asarray(v[:, :, s0:t + 1], dtype=np.float64)
+        scores = scale * np.einsum("bhd,bhsd->bhs", qt, ks)
         scores -= scores.max(axis=-1, keepdims=True)
         p = np.exp(scores)
         p /= p.sum(axis=-1, keepdims=True)
-        out[:, :, t] = np.einsum("bhs,bhsd->bhd", p, v[:, :, s0:t + 1])
+        out[:, :, j] = np.einsum("bhs,bhsd->bhd", p, vs)
     return out
 
 

@@ -45,7 +45,8 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_ctypes_structs_match_c_layout(lib):
     fields = {"ttt_linear_desc": [f[0] for f in T.ttt_linear_desc._fields_],
-              "lact_desc": [f[0] for f in T.lact_desc._fields_]}
+              "lact_desc": [f[0] for f in T.lact_desc._fields_],
+              "ttt_window_desc": [f[0] for f in T.ttt_window_desc._fields_]}
     lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', 'int main(void){']
     for s, fl in fields.items():
         lines.append(f'printf("{s} %zu\\n", sizeof({s}));')
@@ -192,3 +193,29 @@ def test_w2_only_parallel_form_workspace(lib):
         assert T.lact_workspace_bytes(d) == T.lact_workspace_bytes_min(d)
     # a workspace below the minimum is rejected before any launch
     assert _call_lact(w2, ws_bytes=T.lact_workspace_bytes_min(w2) - 256) == T.TTT_ERR_WORKSPACE
+
+
+def test_window_attention_validation_before_launch(lib):
+    def call(desc, **p):
+        a = dict(q=16, k=16, v=16, out=16, ws=16, ws_bytes=256)
+        a.update(p)
+        return T.load().ttt_window_attn_fwd(ctypes.byref(desc), a["q"], a["k"], a["v"], a["out"],
+                                            a["ws"], a["ws_bytes"], None)
+    assert call(T.make_window_desc(1, 2, 64, 64, 16)) == T.TTT_ERR_UNSUPPORTED
+    assert call(T.make_window_desc(1, 2, 64, 128, 0)) == T.TTT_ERR_ARG
+    assert call(T.make_window_desc(0, 2, 64, 128, 16)) == T.TTT_ERR_SHAPE
+    d = T.make_window_desc(1, 2, 64, 128, 16)
+    d.in_dtype = T.TTT_F32
+    assert call(d) == T.TTT_ERR_DTYPE
+    good = T.make_window_desc(1, 2, 64, 128, 16)
+    assert call(good, ws_bytes=8) == T.TTT_ERR_WORKSPACE
+    assert call(good, k=0) == T.TTT_ERR_ARG
+    assert call(good, out=24) == T.TTT_ERR_ALIGN
+    assert call(T.make_window_desc(1, 2, 0, 128, 16)) == T.TTT_OK    # empty: nothing launched
+    # the layer: causal order only, and the window's own checks
+    lact = T.make_lact_desc(1, 2, 64, 128, 256, 32, order="bidirectional", N_q=8)
+    assert T.load().lact_layer_fwd(ctypes.byref(lact), 16, ctypes.c_float(0), 16, 16, 16, 16, 16,
+                                   16, 16, 1 << 40, None) == T.TTT_ERR_ARG
+    lact = T.make_lact_desc(1, 2, 64, 128, 256, 32)
+    assert T.load().lact_layer_fwd(ctypes.byref(lact), 0, ctypes.c_float(0), 16, 16, 16, 16, 16,
+                                   16, 16, 1 << 40, None) == T.TTT_ERR_ARG

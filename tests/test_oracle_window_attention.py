@@ -58,3 +58,10 @@ def test_planted_window_off_by_one_is_caught():
     i, j = np.arange(N)[:, None], np.arange(N)[None, :]
     ref = _sdpa(q, k, v, mask=(j <= i) & (j > i - 8))
     assert np.abs(sliding_window_attention(q, k, v, 9) - ref).max() > 1e-3
+
+
+def test_sampled_positions_match_the_full_computation():
+    q, k, v = _rand(N=50, seed=5)
+    full = sliding_window_attention(q, k, v, 9)
+    idx = [0, 8, 9, 31, 49]
+    np.testing.assert_array_equal(sliding_window_attention(q, k, v, 9, t_index=idx), full[:, :, idx])
