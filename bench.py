@@ -119,6 +119,7 @@ class LaCTBench:
         self.opt = w.get("opt", "gd")
         self.update_mask = w.get("update_mask", 7)
         self.normalize_rows = w.get("normalize_rows", True)
+        self.window = w.get("window", 0)   # > 0: the full layer, memory + window attention
         self.desc = T.make_lact_desc(self.B, self.H, self.N, self.d, self.dh, w["chunk"],
                                      N_q=self.Nq, order=w["order"], opt=self.opt,
                                      beta=w.get("beta", 0.9), ns_steps=w.get("ns_steps", 5),
@@ -149,7 +150,15 @@ class LaCTBench:
             r, c = min(d, dh), max(d, dh)
             nch = -(-self.N // self.w["chunk"])
             f += nch * self.w.get("ns_steps", 5) * 3 * BH * (4 * r * r * c + 2 * r ** 3)
-        return f
+        return f + self.window_flops()
+
+    def window_flops(self):
+        # q.k and p v for every (query, key) pair inside the causal window
+        if not self.window:
+            return 0
+        W, N = self.window, self.N
+        pairs = N * W - W * (W - 1) // 2 if N >= W else N * (N + 1) // 2
+        return 4 * self.d * pairs * self.B * self.H
 
     def kernel_flops_per_step(self):
         """Algorithmic FLOPs per step of each kernel kind (per token-head:
@@ -159,7 +168,8 @@ class LaCTBench:
         kp = (6 * N + 4 * Nq) * d * dh * BH
         kg = (12 * N + (4 * Nq if self.causal else 0)) * d * dh * BH
         return {"lact_keypass": kp, "gemm_grad": 6 * d * dh * N * BH,
-                "gemm_read": 2 * d * dh * Nq * BH, "lact_keygrad": kg}
+                "gemm_read": 2 * d * dh * Nq * BH, "lact_keygrad": kg,
+                "window_attention": self.window_flops()}
 
     def resident_bytes(self):
         return sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v, self.lr,
@@ -168,8 +178,12 @@ class LaCTBench:
     def step(self, stream):
         T = self.T
         T.lact_state_init(self.desc, *self.W, 0, self.state, stream)
-        T.lact_chunk_fwd(self.desc, self.q, self.k, self.v, self.lr, self.state, self.out,
-                         self.ws, stream=stream)
+        if self.window:
+            T.lact_layer_fwd(self.desc, self.window, 0.0, self.q, self.k, self.v, self.lr,
+                             self.state, self.out, self.ws, stream=stream)
+        else:
+            T.lact_chunk_fwd(self.desc, self.q, self.k, self.v, self.lr, self.state, self.out,
+                             self.ws, stream=stream)
 
     def setup_e2e(self, step_fn=None):
         self.e2e_step = step_fn or self.step
@@ -198,6 +212,9 @@ class LaCTBench:
         if self.update_mask != 7 or not self.normalize_rows:
             cfg["update_mask"] = self.update_mask
             cfg["normalize_rows"] = self.normalize_rows
+        if self.window:
+            cfg["window"] = self.window
+            cfg["layer"] = "memory + causal sliding-window attention, summed"
         return cfg
 
     def oracle_sample(self, n_chunks):
@@ -506,7 +523,7 @@ def main():
     ap.add_argument("--workload", default="lact_causal_n32k")
     ap.add_argument("--secondary", default="ttt_linear_bf16_n32k")
     ap.add_argument("--extra", default="lact_bidir_196k,lact_bidir_muon_1m,lact_w2only_causal_n32k,"
-                    "ttt_linear_bwd_bf16_n32k",
+                    "ttt_linear_bwd_bf16_n32k,lact_layer_causal_n32k",
                     help="further workloads timed once each (comma list, or none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",

@@ -193,6 +193,11 @@ WORKLOADS = {
                                     order="causal", qk_norm=True, v_norm=False,
                                     lr_kind="0.01softplus", opt="gd", update_mask=4,
                                     normalize_rows=False, cfg=3),
+    # the full language layer at that shape: memory + causal sliding-window
+    # attention with the 760M model's 2048-token window ("Lenguaje")
+    "lact_layer_causal_n32k": dict(kind="lact", B=2, H=4, N=32768, d=128, dh=256, chunk=2048,
+                                   order="causal", qk_norm=True, v_norm=False,
+                                   lr_kind="0.01softplus", opt="gd", window=2048, cfg=3),
     "lact_bidir_196k": dict(kind="lact", B=1, H=2, N=196608, Nq=4096, d=384, dh=768,
                             chunk=196608, order="bidirectional", qk_norm=True, v_norm=True,
                             lr_kind="0.01sig", opt="gd", cfg=4),
