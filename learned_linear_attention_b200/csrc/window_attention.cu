@@ -12,7 +12,10 @@
 //   pass 1   S = Q K^T (tcgen05, TMEM)  -> row max m and row sum l (online)
 //   pass 2   S = Q K^T again            -> P = exp(S - m) / l, bf16 in smem
 //            O += P V (tcgen05, TMEM)
-// so O accumulates already-normalised terms and is never rescaled.  S
+// so O accumulates already-normalised terms and is never rescaled.  Each
+// query row is shared by four epilogue threads (32 key columns each), whose
+// partial row statistics are combined through shared memory between the
+// passes.  S
 // alternates between two TMEM buffers and P between two shared buffers, so
 // the tensor cores work on one key tile while the epilogue warps work on the
 // previous one.  K/V tiles are double-buffered by TMA (pass 1 loads K only).
@@ -31,8 +34,10 @@ constexpr uint32_t KV_STAGE = 2 * TILE;
 constexpr uint32_t OFF_P = OFF_KV + 2 * KV_STAGE;  // 2 x P (128 queries x 128 keys)
 constexpr uint32_t OFF_BAR = OFF_P + 2 * TILE;
 constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
-constexpr int EPI_WARPS = 4;                      // one per TMEM lane quadrant; a thread per query row
+// four per TMEM lane quadrant: a thread takes 32 key columns of one query row
+constexpr int EPI_WARPS = 16;
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr int CW = 32;                            // columns per epilogue thread
 constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_COLS = 512;
 }  // namespace swa
 
@@ -185,123 +190,137 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q4 = warp & 3;
+    const int cg = (warp - 2) >> 2;             // 32-column group of the key tile
+    const int c0 = cg * CW;
     const int r = q4 * 32 + lane;               // query row of the tile
     const int qi = q0 + r;                      // query token
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const bool row_ok = qi < a.N;
-    float m = -INFINITY, l = 0.f;               // running max (log2 units) and sum
+    float m = -INFINITY, l = 0.f;               // running max (log2 units) and sum of this slice
     bool ok = true;
-    for (int g = 0; ok && g < G; ++g) {
-      const bool pass2 = g >= nk;
-      const int kt = kt_lo + (pass2 ? g - nk : g);
-      const int sb = g & 1;
+    // ---- pass 1: statistics of this thread's 32 columns
+    for (int g = 0; ok && g < nk; ++g) {
+      const int kt = kt_lo + g, sb = g & 1;
       if (!W.wait(&s_full[sb], (g >> 1) & 1, 6)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t sbase = tmem + lane_base + (sb ? TM_S1 : TM_S0);
-      if (!pass2) {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float x[32];
-          // tcgen05.ld is warp-collective: every lane reaches it, converged
-          __syncwarp();
-          tmem_ld32(sbase + c, x);
-          float cm = -INFINITY;
+      float x[CW];
+      // tcgen05.ld is warp-collective: every lane reaches it, converged
+      __syncwarp();
+      tmem_ld32(tmem + lane_base + (sb ? TM_S1 : TM_S0) + c0, x);
+      tc_fence_before();
+      mbar_arrive(&s_empty[sb]);
+      float cm = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int kj = kt * BN + c + j;
-            const bool valid = row_ok && kj <= qi && kj > qi - a.window;
-            x[j] = valid ? x[j] * a.scale_log2 : -INFINITY;
-            cm = fmaxf(cm, x[j]);
-          }
-          const float mn = fmaxf(m, cm);
-          if (mn != -INFINITY) {   // no valid key yet: m and l stay as they are
-            float add = 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) add += exp2f(x[j] - mn);
-            l = l * exp2f(m - mn) + add;
-            m = mn;
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&s_empty[sb]);
-      } else {
-        // pass-2 tile i writes P buffer i & 1, free once the P V product of
-        // pass-2 tile i - 2 is done
-        const int i = g - nk, pb = i & 1;
-        if (i >= 2 && !W.wait(&p_empty[pb], ((i >> 1) - 1) & 1, 7)) { ok = false; break; }
-        const float inv_l = row_ok ? 1.f / l : 0.f;
-        const uint32_t pbase = smem_u32(smem + OFF_P + pb * TILE);
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float x[32];
-          __syncwarp();
-          tmem_ld32(sbase + c, x);
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float p2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int kj = kt * BN + c + j + u;
-              const bool valid = row_ok && kj <= qi && kj > qi - a.window;
-              p2[u] = valid ? exp2f(x[j + u] * a.scale_log2 - m) * inv_l : 0.f;
-            }
-            pk[j >> 1] = pack_bf16x2(p2[0], p2[1]);
-          }
-          // keys c .. c + 31 of row r: half c / 64, columns (c % 64) ..
-          const uint32_t hb = pbase + (uint32_t)(c >> 6) * HALF;
-#pragma unroll
-          for (int j = 0; j < 32; j += 8)
-            st_shared_v4(hb + sw128_offset(r, (c & 63) + j), pk[j / 2], pk[j / 2 + 1], pk[j / 2 + 2],
-                         pk[j / 2 + 3]);
-        }
-        tc_fence_before();
-        mbar_arrive(&s_empty[sb]);
-        fence_async_smem();
-        mbar_arrive(&p_full[pb]);
+      for (int j = 0; j < CW; ++j) {
+        const int kj = kt * BN + c0 + j;
+        const bool valid = row_ok && kj <= qi && kj > qi - a.window;
+        x[j] = valid ? x[j] * a.scale_log2 : -INFINITY;
+        cm = fmaxf(cm, x[j]);
       }
+      const float mn = fmaxf(m, cm);
+      if (mn != -INFINITY) {   // no valid key yet: m and l stay as they are
+        float add = 0.f;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) add += exp2f(x[j] - mn);
+        l = l * exp2f(m - mn) + add;
+        m = mn;
+      }
+    }
+    // ---- the row's statistics from its four slices.  Every epilogue thread
+    // passes both barriers exactly once (also after a failed wait), so no
+    // thread is left waiting.  The scratch is P buffer 1, first written by
+    // pass-2 tile 1, after the second barrier.
+    float2* stats = reinterpret_cast<float2*>(smem + OFF_P + TILE);   // [4 slices][128 rows]
+    stats[cg * BM + r] = make_float2(m, l);
+    asm volatile("bar.sync 1, %0;" ::"n"(EPI_WARPS * 32) : "memory");
+    {
+      float M = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) M = fmaxf(M, stats[u * BM + r].x);
+      float L = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 t = stats[u * BM + r];
+          if (t.x != -INFINITY) L += t.y * exp2f(t.x - M);
+        }
+      }
+      m = M;
+      l = L;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(EPI_WARPS * 32) : "memory");
+    // ---- pass 2: P = exp(S - m) / l for this thread's 32 columns
+    const float inv_l = row_ok ? 1.f / l : 0.f;
+    for (int i = 0; ok && i < nk; ++i) {
+      const int g = nk + i, kt = kt_lo + i, sb = g & 1, pb = i & 1;
+      if (!W.wait(&s_full[sb], (g >> 1) & 1, 6)) { ok = false; break; }
+      // P buffer i & 1 is free once the P V product of pass-2 tile i - 2 is done
+      if (i >= 2 && !W.wait(&p_empty[pb], ((i >> 1) - 1) & 1, 7)) { ok = false; break; }
+      tc_fence_after();
+      float x[CW];
+      __syncwarp();
+      tmem_ld32(tmem + lane_base + (sb ? TM_S1 : TM_S0) + c0, x);
+      tc_fence_before();
+      mbar_arrive(&s_empty[sb]);
+      uint32_t pk[CW / 2];
+#pragma unroll
+      for (int j = 0; j < CW; j += 2) {
+        float p2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int kj = kt * BN + c0 + j + u;
+          const bool valid = row_ok && kj <= qi && kj > qi - a.window;
+          p2[u] = valid ? exp2f(x[j + u] * a.scale_log2 - m) * inv_l : 0.f;
+        }
+        pk[j >> 1] = pack_bf16x2(p2[0], p2[1]);
+      }
+      // keys c0 .. c0 + 31 of row r: half c0 / 64, columns (c0 % 64) ..
+      const uint32_t hb = smem_u32(smem + OFF_P + pb * TILE) + (uint32_t)(c0 >> 6) * HALF;
+#pragma unroll
+      for (int j = 0; j < CW; j += 8)
+        st_shared_v4(hb + sw128_offset(r, (c0 & 63) + j), pk[j / 2], pk[j / 2 + 1], pk[j / 2 + 2],
+                     pk[j / 2 + 3]);
+      fence_async_smem();
+      mbar_arrive(&p_full[pb]);
     }
     if (ok && W.wait(o_full, 0, 8)) {
       tc_fence_after();
-      const size_t base = ((size_t)bh * a.N + qi) * D;
-#pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        float o[32];
-        // every lane loads (warp-collective); only rows inside the sequence store
-        __syncwarp();
-        tmem_ld32(tmem + lane_base + TM_O + c, o);
-        if (row_ok) {
-          if (a.out_bf16) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base + c);
+      float o[CW];
+      // every lane loads (warp-collective); only rows inside the sequence store
+      __syncwarp();
+      tmem_ld32(tmem + lane_base + TM_O + c0, o);
+      if (row_ok) {
+        const size_t base = ((size_t)bh * a.N + qi) * D + c0;
+        if (a.out_bf16) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float v8[8];
-              if (a.accumulate) {
-                const uint4 w = dst[j];
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          for (int j = 0; j < CW / 8; ++j) {
+            float v8[8];
+            if (a.accumulate) {
+              const uint4 w = dst[j];
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  v8[2 * u] = o[8 * j + 2 * u] + bf16lo(ww[u]);
-                  v8[2 * u + 1] = o[8 * j + 2 * u + 1] + bf16hi(ww[u]);
-                }
-              } else {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) v8[u] = o[8 * j + u];
+              for (int u = 0; u < 4; ++u) {
+                v8[2 * u] = o[8 * j + 2 * u] + bf16lo(ww[u]);
+                v8[2 * u + 1] = o[8 * j + 2 * u + 1] + bf16hi(ww[u]);
               }
-              dst[j] = make_uint4(pack_bf16x2(v8[0], v8[1]), pack_bf16x2(v8[2], v8[3]),
-                                  pack_bf16x2(v8[4], v8[5]), pack_bf16x2(v8[6], v8[7]));
-            }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base + c);
+            } else {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float4 v4 = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-              if (a.accumulate) {
-                const float4 w = dst[j];
-                v4.x += w.x; v4.y += w.y; v4.z += w.z; v4.w += w.w;
-              }
-              dst[j] = v4;
+              for (int u = 0; u < 8; ++u) v8[u] = o[8 * j + u];
             }
+            dst[j] = make_uint4(pack_bf16x2(v8[0], v8[1]), pack_bf16x2(v8[2], v8[3]),
+                                pack_bf16x2(v8[4], v8[5]), pack_bf16x2(v8[6], v8[7]));
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base);
+#pragma unroll
+          for (int j = 0; j < CW / 4; ++j) {
+            float4 v4 = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            if (a.accumulate) {
+              const float4 w = dst[j];
+              v4.x += w.x; v4.y += w.y; v4.z += w.z; v4.w += w.w;
+            }
+            dst[j] = v4;
           }
         }
       }
