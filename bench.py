@@ -229,7 +229,11 @@ class LaCTBench:
         st = lact_init_state(x.W1[:1], x.W3[:1], x.W2[:1], 1, self.opt)
         t0 = time.perf_counter()
         lact_forward(q, sl(x.k.values), sl(x.v.values), sl(x.lr), st, chunk=C,
-                     order=self.w["order"], opt=self.opt)
+                     order=self.w["order"], opt=self.opt, update_mask=self.update_mask,
+                     normalize_rows=self.normalize_rows)
+        if self.window:
+            from oracle import sliding_window_attention
+            sliding_window_attention(q, sl(x.k.values), sl(x.v.values), self.window)
         dt = time.perf_counter() - t0
         # tokens of the metric: every token counts once across all H heads
         toks = (n if self.causal else n + (self.Nq if n >= self.N else 0)) / self.H
@@ -486,7 +490,9 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": {"workload": name, **{k: v for k, v in WORKLOADS[name].items()
-                                            if k in ("B", "H", "N", "d", "dh", "chunk", "order")},
+                                            if k in ("B", "H", "N", "d", "dh", "dk", "dv", "chunk",
+                                                     "order", "window", "update_mask",
+                                                     "backward")},
                        "parallelism": "cpu"},
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": os.cpu_count(),
                              "kind": "oracle", "sample": sample},
@@ -505,12 +511,42 @@ class _CPUOnlyLaCT(LaCTBench):
         self.Nq = self.x.q.values.shape[2]
         self.causal = w["order"] == "causal"
         self.opt = w.get("opt", "gd")
+        self.update_mask = w.get("update_mask", 7)
+        self.normalize_rows = w.get("normalize_rows", True)
+        self.window = w.get("window", 0)
+
+
+class _CPUOnlyLinear:
+    """Oracle side of a linear workload (forward, or backward when the
+    workload says so): no device needed."""
+
+    def __init__(self, name):
+        from ttt_synth import WORKLOADS, make_linear_grads, make_workload
+        self.name, self.w = name, dict(WORKLOADS[name])
+        self.x = make_workload(name)
+        self.g = make_linear_grads(self.x, cfg=self.w["cfg"]) if self.w.get("backward") else None
+
+    def oracle_sample(self, n_blocks):
+        """Batch entry 0, all heads, the first 512 * n_blocks tokens."""
+        from oracle import ttt_linear_backward, ttt_linear_recurrent
+        x, w = self.x, self.w
+        n = min(w["N"], 512 * n_blocks)
+        sl = lambda a: a[:1, :, :n]  # noqa: E731
+        t0 = time.perf_counter()
+        if self.g is None:
+            ttt_linear_recurrent(sl(x.q.values), sl(x.k.values), sl(x.v.values), sl(x.lr))
+        else:
+            ttt_linear_backward(sl(x.q.values), sl(x.k.values), sl(x.v.values), sl(x.lr),
+                                sl(self.g.dout.values), None, self.g.dS_end[:1])
+        dt = time.perf_counter() - t0
+        what = "backward" if self.g is not None else "forward"
+        return n, dt, f"{what}: batch entry 0 (all {w['H']} heads), first {n} tokens"
 
 
 def make_bench_cpu(name):
     from ttt_synth import WORKLOADS
-    if WORKLOADS[name]["kind"] != "lact":
-        raise SystemExit("reference arm implemented for the LaCT workloads")
+    if WORKLOADS[name]["kind"] == "linear":
+        return _CPUOnlyLinear(name)
     return _CPUOnlyLaCT(name)
 
 

@@ -56,11 +56,12 @@ def test_job_value_single_rank():
     assert bench.job_value(1, 65536, 0.5) == pytest.approx(65536 / 0.5e-3)
 
 
-def _run_reference(rank):
+def _run_reference(rank, workload=None):
     env = dict(os.environ, RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE="2",
                MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    extra = [] if workload is None else ["--workload", workload]
     return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                           "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                           "--gpus", "2", "--steps", "1", "--warmup", "3"] + extra,
                           capture_output=True, text=True, env=env, timeout=600, cwd=ROOT)
 
 
@@ -80,3 +81,16 @@ def test_reference_arm_other_ranks_exit_without_work():
     r = _run_reference(1)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+@pytest.mark.parametrize("workload", ["ttt_linear_f32_n256", "lact_layer_causal_n32k"])
+def test_reference_arm_other_workloads(workload):
+    """The oracle arm also times the linear layer and the full language layer
+    (memory + window attention) on a bounded sample."""
+    r = _run_reference(0, workload)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["config"]["workload"] == workload and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
