@@ -15,6 +15,10 @@ Contents
   lact        -- large-chunk TTT with a SwiGLU fast-weight memory: chunk
                  gradients, GD / momentum / Muon (Newton-Schulz) updates, row
                  L2 normalisation, causal and bidirectional ordering.
+  lact_backward -- gradients of the LaCT layer through its chunk loop
+                 (float64 torch restatement of the forward, differentiated by
+                 torch.autograd; pinned to the numpy oracle and to central
+                 differences).
   window_attention -- causal sliding-window softmax attention, and the LaCT
                  language layer (memory + window attention, outputs summed).
 
