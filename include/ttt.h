@@ -11,18 +11,24 @@
  *     the recurrence W_t = W_{t-1} + eta_t v_t k_t^T, o_t = W_t q_t is causal
  *     linear attention and admits a chunked / prefix-scan form
  *     ("Formulación Paralela").
+ *     Its backward pass is ttt_linear_bwd.
  *   * "Test-Time Training Done Right" (LaCT review): a SwiGLU memory with
  *     three matrices, chunk gradients summed with per-token learning rates,
  *     GD / momentum / Muon (Newton-Schulz) updates followed by L2
  *     normalisation ("Memoria no lineal y atención local"); causal chunks read
  *     the memory of earlier chunks before updating it, posed-image sets are
  *     written first and queried afterwards ("El orden de lectura evita
- *     información futura").
+ *     información futura").  The language layer adds causal sliding-window
+ *     attention on the same q, k, v (ttt_window_attn_fwd, lact_layer_fwd).
  *
  * General conventions for every entry point
  *   * Every tensor pointer is a DEVICE pointer owned by the caller.  The
- *     library never allocates device memory and keeps no global state apart
- *     from a per-process cache of kernel attributes.
+ *     library never allocates device memory (lact_chunk_fwd_noalloc uses a
+ *     file-scope device array instead of a workspace).  Its other state is a
+ *     per-process cache of kernel attributes and, per host thread and
+ *     device, helper streams and events created on first use, on which the
+ *     independent kernels of a call run beside each other (forked from and
+ *     joined back into `stream`).
  *   * Token tensors are [B, H, T, D], contiguous, D innermost.  Learning
  *     rates are float32 [B, H, T].  Pointers must be 16-byte aligned and
  *     D * sizeof(element) a multiple of 16 bytes (TMA rule).
