@@ -18,7 +18,9 @@
 // passes.  S
 // alternates between two TMEM buffers and P between two shared buffers, so
 // the tensor cores work on one key tile while the epilogue warps work on the
-// previous one.  K/V tiles are double-buffered by TMA (pass 1 loads K only).
+// previous one.  K and V tiles sit in separate two-slot rings, so a K slot
+// is refilled as soon as its scores are computed, while the V slot waits for
+// its P V product (pass 1 loads K only).
 #include <algorithm>
 
 #include "kernels.h"
@@ -29,9 +31,9 @@ constexpr int D = 128, BM = 128, BN = 128;
 constexpr uint32_t HALF = 128 * 64 * 2;          // 16 KB: 128 rows x 64 bf16 (one swizzle atom wide)
 constexpr uint32_t TILE = 2 * HALF;              // 32 KB: 128 rows x 128 bf16
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_KV = TILE;                // 2 stages x (K | V)
-constexpr uint32_t KV_STAGE = 2 * TILE;
-constexpr uint32_t OFF_P = OFF_KV + 2 * KV_STAGE;  // 2 x P (128 queries x 128 keys)
+constexpr uint32_t OFF_K = TILE;                 // 2 K slots
+constexpr uint32_t OFF_V = OFF_K + 2 * TILE;     // 2 V slots (pass 2)
+constexpr uint32_t OFF_P = OFF_V + 2 * TILE;     // 2 x P (128 queries x 128 keys)
 constexpr uint32_t OFF_BAR = OFF_P + 2 * TILE;
 constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 // four per TMEM lane quadrant: a thread takes 32 key columns of one query row
@@ -59,9 +61,11 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* kv_full = q_full + 1;     // [2]
-  uint64_t* kv_empty = kv_full + 2;   // [2]
-  uint64_t* s_full = kv_empty + 2;    // [2]
+  uint64_t* k_full = q_full + 1;      // [2]
+  uint64_t* k_empty = k_full + 2;     // [2]
+  uint64_t* v_full = k_empty + 2;     // [2]
+  uint64_t* v_empty = v_full + 2;     // [2]
+  uint64_t* s_full = v_empty + 2;     // [2]
   uint64_t* s_empty = s_full + 2;     // [2]
   uint64_t* p_full = s_empty + 2;     // [2]
   uint64_t* p_empty = p_full + 2;     // [2]
@@ -81,8 +85,10 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], EPI_WARPS * 32);
       mbar_init(&p_full[s], EPI_WARPS * 32);
@@ -113,25 +119,32 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
       mbar_arrive_expect_tx(q_full, TILE);
       tma_load_3d(smem + OFF_Q, &maps.q, q_full, 0, q0, bh);
       tma_load_3d(smem + OFF_Q + HALF, &maps.q, q_full, 64, q0, bh);
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int g = 0; g < G; ++g) {
+        // K of tile g into slot g & 1, free once the scores of tile g - 2 are done
         const int s = g & 1;
-        if (g >= 2 && !W.wait(&kv_empty[s], ((g >> 1) - 1) & 1, 1)) break;
+        if (g >= 2 && !W.wait(&k_empty[s], ((g >> 1) - 1) & 1, 1)) break;
         const bool pass2 = g >= nk;
-        const int row = (kt_lo + (pass2 ? g - nk : g)) * BN;
-        uint8_t* st = smem + OFF_KV + s * KV_STAGE;
-        mbar_arrive_expect_tx(&kv_full[s], pass2 ? KV_STAGE : TILE);
-        tma_load_3d(st, &maps.k, &kv_full[s], 0, row, bh);
-        tma_load_3d(st + HALF, &maps.k, &kv_full[s], 64, row, bh);
+        const int i = g - nk;
+        const int row = (kt_lo + (pass2 ? i : g)) * BN;
+        mbar_arrive_expect_tx(&k_full[s], TILE);
+        tma_load_3d(smem + OFF_K + s * TILE, &maps.k, &k_full[s], 0, row, bh);
+        tma_load_3d(smem + OFF_K + s * TILE + HALF, &maps.k, &k_full[s], 64, row, bh);
+        k_issued = g + 1;
         if (pass2) {
-          tma_load_3d(st + TILE, &maps.v, &kv_full[s], 0, row, bh);
-          tma_load_3d(st + TILE + HALF, &maps.v, &kv_full[s], 64, row, bh);
+          // V of pass-2 tile i into slot i & 1, free once P V of tile i - 2 is done
+          const int sv = i & 1;
+          if (i >= 2 && !W.wait(&v_empty[sv], ((i >> 1) - 1) & 1, 9)) break;
+          mbar_arrive_expect_tx(&v_full[sv], TILE);
+          tma_load_3d(smem + OFF_V + sv * TILE, &maps.v, &v_full[sv], 0, row, bh);
+          tma_load_3d(smem + OFF_V + sv * TILE + HALF, &maps.v, &v_full[sv], 64, row, bh);
+          v_issued = i + 1;
         }
-        issued = g + 1;
       }
       if (W.aborted()) {
         W.drain(q_full, 0);
-        for (int g = max(0, issued - 2); g < issued; ++g) W.drain(&kv_full[g & 1], (g >> 1) & 1);
+        for (int g = max(0, k_issued - 2); g < k_issued; ++g) W.drain(&k_full[g & 1], (g >> 1) & 1);
+        for (int i = max(0, v_issued - 2); i < v_issued; ++i) W.drain(&v_full[i & 1], (i >> 1) & 1);
       }
     }
   } else if (warp == 1) {
@@ -140,18 +153,18 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
       const uint32_t id_s = make_idesc(128, 128, false, false);   // Q, K both K-major (d)
       const uint32_t id_o = make_idesc(128, 128, false, true);    // P K-major (keys), V MN-major
       const uint64_t dq = make_sdesc(smem_u32(smem + OFF_Q), 16, 1024);
-      const uint64_t dkv = make_sdesc(smem_u32(smem + OFF_KV), 16, 1024);
-      const uint64_t dv0 = make_sdesc(smem_u32(smem + OFF_KV + TILE), HALF, 1024);
+      const uint64_t dk0 = make_sdesc(smem_u32(smem + OFF_K), 16, 1024);
+      const uint64_t dv0 = make_sdesc(smem_u32(smem + OFF_V), HALF, 1024);
       const uint64_t dp0 = make_sdesc(smem_u32(smem + OFF_P), 16, 1024);
       bool ok = W.wait(q_full, 0, 2);
       tc_fence_after();
       // S(g) = Q K(g)^T into S buffer g & 1
       auto issue_s = [&](int g) -> bool {
         const int s = g & 1;
-        if (!W.wait(&kv_full[s], (g >> 1) & 1, 3)) return false;
+        if (!W.wait(&k_full[s], (g >> 1) & 1, 3)) return false;
         if (g >= 2 && !W.wait(&s_empty[s], ((g >> 1) - 1) & 1, 4)) return false;
         tc_fence_after();
-        const uint64_t dk = sdesc_add(dkv, s * KV_STAGE);
+        const uint64_t dk = sdesc_add(dk0, s * TILE);
         const uint32_t acc = tmem + (s ? TM_S1 : TM_S0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -159,7 +172,7 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
           mma_bf16(acc, sdesc_add(dq, off), sdesc_add(dk, off), id_s, kk > 0);
         }
         mma_commit(&s_full[s]);
-        if (g < nk) mma_commit(&kv_empty[s]);   // pass 1 is done with this K tile
+        mma_commit(&k_empty[s]);   // the scores are done with this K tile
         return true;
       };
       if (ok && G > 0) ok = issue_s(0);
@@ -169,10 +182,11 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
         if (g + 1 < G && !issue_s(g + 1)) { ok = false; break; }
         if (g >= nk) {
           // pass-2 tile i: P buffer i & 1, filled for the (i >> 1)-th time
-          const int i = g - nk, pb = i & 1, s = g & 1;
+          const int i = g - nk, pb = i & 1, sv = i & 1;
           if (!W.wait(&p_full[pb], (i >> 1) & 1, 5)) { ok = false; break; }
+          if (!W.wait(&v_full[sv], (i >> 1) & 1, 10)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t dv = sdesc_add(dv0, s * KV_STAGE);
+          const uint64_t dv = sdesc_add(dv0, sv * TILE);
           const uint64_t dp = sdesc_add(dp0, pb * TILE);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -180,7 +194,7 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
             mma_bf16(tmem + TM_O, sdesc_add(dp, offp), sdesc_add(dv, kk * 2048), id_o,
                      (i > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&kv_empty[s]);
+          mma_commit(&v_empty[sv]);
           mma_commit(&p_empty[pb]);
         }
       }
