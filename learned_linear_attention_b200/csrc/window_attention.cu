@@ -212,6 +212,11 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
     const bool row_ok = qi < a.N;
     float m = -INFINITY, l = 0.f;               // running max (log2 units) and sum of this slice
     bool ok = true;
+    // key tile kt lies inside every row's window (no mask needed): uniform
+    // across the CTA, so the branches below never split a warp
+    auto inside = [&](int kt) {
+      return kt * BN + BN - 1 <= q0 && kt * BN > q0 + BM - 1 - a.window && q0 + BM <= a.N;
+    };
     // ---- pass 1: statistics of this thread's 32 columns
     for (int g = 0; ok && g < nk; ++g) {
       const int kt = kt_lo + g, sb = g & 1;
@@ -224,12 +229,20 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
       tc_fence_before();
       mbar_arrive(&s_empty[sb]);
       float cm = -INFINITY;
+      if (inside(kt)) {
 #pragma unroll
-      for (int j = 0; j < CW; ++j) {
-        const int kj = kt * BN + c0 + j;
-        const bool valid = row_ok && kj <= qi && kj > qi - a.window;
-        x[j] = valid ? x[j] * a.scale_log2 : -INFINITY;
-        cm = fmaxf(cm, x[j]);
+        for (int j = 0; j < CW; ++j) {
+          x[j] *= a.scale_log2;
+          cm = fmaxf(cm, x[j]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < CW; ++j) {
+          const int kj = kt * BN + c0 + j;
+          const bool valid = row_ok && kj <= qi && kj > qi - a.window;
+          x[j] = valid ? x[j] * a.scale_log2 : -INFINITY;
+          cm = fmaxf(cm, x[j]);
+        }
       }
       const float mn = fmaxf(m, cm);
       if (mn != -INFINITY) {   // no valid key yet: m and l stay as they are
@@ -277,16 +290,23 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
       tc_fence_before();
       mbar_arrive(&s_empty[sb]);
       uint32_t pk[CW / 2];
+      if (inside(kt)) {
 #pragma unroll
-      for (int j = 0; j < CW; j += 2) {
-        float p2[2];
+        for (int j = 0; j < CW; j += 2)
+          pk[j >> 1] = pack_bf16x2(exp2f(x[j] * a.scale_log2 - m) * inv_l,
+                                   exp2f(x[j + 1] * a.scale_log2 - m) * inv_l);
+      } else {
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int kj = kt * BN + c0 + j + u;
-          const bool valid = row_ok && kj <= qi && kj > qi - a.window;
-          p2[u] = valid ? exp2f(x[j + u] * a.scale_log2 - m) * inv_l : 0.f;
+        for (int j = 0; j < CW; j += 2) {
+          float p2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int kj = kt * BN + c0 + j + u;
+            const bool valid = row_ok && kj <= qi && kj > qi - a.window;
+            p2[u] = valid ? exp2f(x[j + u] * a.scale_log2 - m) * inv_l : 0.f;
+          }
+          pk[j >> 1] = pack_bf16x2(p2[0], p2[1]);
         }
-        pk[j >> 1] = pack_bf16x2(p2[0], p2[1]);
       }
       // keys c0 .. c0 + 31 of row r: half c0 / 64, columns (c0 % 64) ..
       const uint32_t hb = smem_u32(smem + OFF_P + pb * TILE) + (uint32_t)(c0 >> 6) * HALF;
