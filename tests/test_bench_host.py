@@ -94,3 +94,17 @@ def test_reference_arm_other_workloads(workload):
     line = json.loads(lines[0])
     assert line["config"]["workload"] == workload and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_window_flop_count_matches_brute_force():
+    """The window branch's algorithmic FLOPs (4 d per in-window (query, key)
+    pair) against a direct count of the pairs."""
+    import types
+    import numpy as np
+    for N, W in ((1000, 300), (300, 1000), (2048, 2048), (4097, 128)):
+        i = np.arange(N)[:, None]
+        j = np.arange(N)[None, :]
+        pairs = int(((j <= i) & (j > i - W)).sum())
+        b = types.SimpleNamespace(window=W, N=N, d=128, B=2, H=3)
+        assert bench.LaCTBench.window_flops(b) == 4 * 128 * pairs * 6
+    assert bench.LaCTBench.window_flops(types.SimpleNamespace(window=0, N=10, d=128, B=1, H=1)) == 0
