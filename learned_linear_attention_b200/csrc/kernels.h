@@ -4,6 +4,7 @@
 
 #include <stdio.h>
 
+#include <atomic>
 #include <utility>
 
 #include "common.cuh"
@@ -42,6 +43,21 @@ template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t stream, Args&&... args) {
   return launch_pdl_cluster(kernel, grid, block, smem, stream, 1, std::forward<Args>(args)...);
+}
+
+// Let `kernel` use `bytes` of dynamic shared memory on the current device.
+// The attribute belongs to each device, so `done` keeps one bit per device
+// that already has it (devices 64 and up are set on every call).
+template <typename... KArgs>
+inline int allow_dynamic_smem(void (*kernel)(KArgs...), int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return 0;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return -1;
+  done.fetch_or(bit, std::memory_order_release);
+  return 0;
 }
 
 // ----------------------------------------------------------------- tensor maps

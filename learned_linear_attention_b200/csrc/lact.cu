@@ -922,12 +922,8 @@ static int run_gemm(const GemmMaps& maps, const GemmArgs& g, cudaStream_t stream
                     int max_grid = 0) {
   auto kfn = gemm_bf16_kernel<BN, A_MN, B_MN, STAGES>;
   const int smem = (int)GemmSmem<BN, STAGES>::BYTES;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return -1;
-    attr_done = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (allow_dynamic_smem(kfn, smem, attr_done)) return -1;
   const int tiles = ((g.M + 127) / 128) * (g.N / BN) * g.splits * g.batch;
   if (tiles <= 0) return 0;
   // cluster mode: one tile per CTA, N tiles of a row block in one cluster
@@ -1039,13 +1035,10 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     prof_before(K_UPDATE, st);
     cudaError_t e;
     if (ra.splits <= UPB_MAX_SPLITS && d % 128 == 0 && dh % 128 == 0) {
-      static bool upb_attr = false;
-      if (!upb_attr) {
-        if (cudaFuncSetAttribute(lact_update_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)((UPB_MAX_SPLITS + 2) * UPB_SLAB)) != cudaSuccess)
-          return -1;
-        upb_attr = true;
-      }
+      static std::atomic<uint64_t> upb_attr{0};
+      if (allow_dynamic_smem(lact_update_bulk_kernel, (int)((UPB_MAX_SPLITS + 2) * UPB_SLAB),
+                             upb_attr))
+        return -1;
       e = launch_pdl(lact_update_bulk_kernel, dim3(update_bulk_blocks(BH, d, dh)), dim3(UPB_THREADS),
                      (size_t)(ra.splits + 2) * UPB_SLAB, st, ra);
     } else {
@@ -1124,13 +1117,8 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     TTT_TRY(tok_map(&mv_mn, L.v, L.N_in, 64));
   }
 
-  static bool kp_attr = false;
-  if (!kp_attr) {
-    if (cudaFuncSetAttribute(lact_keypass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kp::SMEM) != cudaSuccess)
-      return -1;
-    kp_attr = true;
-  }
+  static std::atomic<uint64_t> kp_attr{0};
+  if (allow_dynamic_smem(lact_keypass_kernel, (int)kp::SMEM, kp_attr)) return -1;
 
   auto key_pass_on = [&](int t0, int C, int nkt, int nqt, cudaStream_t kstream) -> int {
     KeyPassArgs a{};

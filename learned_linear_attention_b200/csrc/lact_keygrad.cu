@@ -498,13 +498,8 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream) {
   a.Aq = L.Aq;
   a.aq_bs = L.aq_bs;
   a.st = L.st;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(lact_keygrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kg::SMEM) != cudaSuccess)
-      return -1;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (allow_dynamic_smem(lact_keygrad_kernel, (int)kg::SMEM, attr)) return -1;
   const int items = a.n_hb * a.n_groups * L.BH;
   int sms = 148;
   int dev = 0;

@@ -692,25 +692,15 @@ int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream) {
                 pl.P, pl.R, pl.seg_tiles, L.seg_state, L.out_scale, L.out_mul};
   if (pl.P > 1) {
     SegStateArgs sa{L.lr, L.S, L.seg_state, L.N, (pl.P - 1) * pl.R, pl.R, pl.seg_tiles, pl.unit_tiles, L.st};
-    static bool ss_attr = false;
-    if (!ss_attr) {
-      if (cudaFuncSetAttribute(ttt_linear_segstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)lss::SMEM) != cudaSuccess)
-        return -1;
-      ss_attr = true;
-    }
+    static std::atomic<uint64_t> ss_attr{0};
+    if (allow_dynamic_smem(ttt_linear_segstate_kernel, (int)lss::SMEM, ss_attr)) return -1;
     prof_before(K_LIN_SEG, stream);
     ttt_linear_segstate_kernel<<<dim3((unsigned)(BH * sa.U)), dim3(lss::THREADS), lss::SMEM, stream>>>(
         mk, mv, sa);
     prof_after(K_LIN_SEG, stream);
   }
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(ttt_linear_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)lin::SMEM_BYTES) != cudaSuccess)
-      return -1;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (allow_dynamic_smem(ttt_linear_umma_kernel, (int)lin::SMEM_BYTES, attr)) return -1;
   prof_before(K_LIN_UMMA, stream);
   ttt_linear_umma_kernel<<<dim3((unsigned)(BH * pl.P)), dim3(lin::THREADS), lin::SMEM_BYTES, stream>>>(
       mq, mk, mv, a);
@@ -759,13 +749,8 @@ int launch_ttt_linear_state_sum(const LinearLaunch& L, int sms, cudaStream_t str
   const int total = (L.N + 127) / 128;
   // one segment of `total` tiles split into U units
   SegStateArgs sa{L.lr, L.S, L.seg_state, L.N, U, U, total, (total + U - 1) / U, L.st};
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(ttt_linear_segstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)lss::SMEM) != cudaSuccess)
-      return -1;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (allow_dynamic_smem(ttt_linear_segstate_kernel, (int)lss::SMEM, attr)) return -1;
   prof_before(K_LIN_SEG, stream);
   ttt_linear_segstate_kernel<<<dim3((unsigned)(BH * U)), dim3(lss::THREADS), lss::SMEM, stream>>>(
       mk, mv, sa);

@@ -387,13 +387,8 @@ int launch_window_attention(const WindowAttnLaunch& L, cudaStream_t stream) {
   a.accumulate = L.accumulate;
   a.out = L.out;
   a.st = L.st;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(window_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM) != cudaSuccess)
-      return -1;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (allow_dynamic_smem(window_attention_kernel, (int)SMEM, attr)) return -1;
   prof_before(K_SWA, stream);
   window_attention_kernel<<<dim3((unsigned)(BH * a.n_qt)), dim3(THREADS), SMEM, stream>>>(m, a);
   prof_after(K_SWA, stream);
