@@ -763,15 +763,16 @@ __global__ void muon_apply_kernel(RowArgs a, int r, int c) {
 // =====================================================================
 // host side
 // =====================================================================
-static int g_num_sms = 0;
+// SMs of the current device (asked on every call: a process may drive
+// devices of different sizes)
 static int num_sms() {
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = 148;
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 148;
   }
-  return g_num_sms;
+  return n;
 }
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
