@@ -104,3 +104,23 @@ def test_planted_missing_second_order_term_is_caught():
         lb._chunk_gradients = orig
     assert max(np.abs(b - g).max() for b, g in zip(bad[4:], good[4:])) > 1e-4
     del torch
+
+
+EXPLICIT_CASES = [c for c in CASES if c["opt"] in ("gd", "momentum")] + [
+    dict(chunk=2, order="causal", opt="momentum", beta=0.7, update_mask=5),
+    dict(chunk=7, order="bidirectional", opt="momentum", beta=0.9, normalize_rows=False),
+]
+
+
+@pytest.mark.parametrize("kw", EXPLICIT_CASES)
+def test_written_out_backward_equals_autograd(kw):
+    """The step-by-step backward (read VJP, row-norm VJP, momentum carry and
+    the chunk gradient's vector-Jacobian product) equals autograd."""
+    from oracle.lact_backward import lact_backward_explicit
+    x, dout, dW = _rand(B=2, H=2, N=9, Nq=6 if kw["order"] == "bidirectional" else None, seed=7)
+    args = (x["q"], x["k"], x["v"], x["lr"], x["W1"], x["W3"], x["W2"], dout, dW)
+    ref = lact_backward(*args, **kw)
+    got = lact_backward_explicit(*args, **kw)
+    for name, g, r in zip(("q", "k", "v", "lr", "W1", "W3", "W2"), got, ref):
+        np.testing.assert_allclose(g, r, rtol=0, atol=1e-10 * max(1.0, np.abs(r).max()),
+                                   err_msg=name)
