@@ -21,10 +21,10 @@ differentiates that restatement.  Autograd is the library primitive here;
 the restatement is pinned to the numpy oracle, and the gradients to central
 differences of the numpy oracle, in tests/test_oracle_lact_backward.py.
 
-``lact_backward_explicit`` computes the same gradients step by step for GD
-and momentum (read, row-norm and chunk-gradient vector-Jacobian products,
-the momentum carry), the decomposition a backward kernel follows; it is
-pinned to ``lact_backward``.
+``lact_backward_explicit`` computes the same gradients step by step (read,
+row-norm, Newton-Schulz and chunk-gradient vector-Jacobian products, the
+momentum carry), the decomposition a backward kernel follows; it is pinned
+to ``lact_backward``.
 """
 from __future__ import annotations
 
@@ -146,7 +146,7 @@ def lact_backward(q, k, v, lr, W1, W3, W2, dout, dW_end=None, **kw):
 
 
 # ---------------------------------------------------------------------------
-# The same gradients written out step by step (GD and momentum), float64
+# The same gradients written out step by step (GD, momentum, Muon), float64
 # numpy.  This is the list of products a backward kernel computes; it is
 # pinned to lact_backward above.
 #
@@ -227,6 +227,49 @@ def _chunk_gradient_vjp(W1, W3, W2, k, v, lr, R1, R3, R2):
     return dW1, dW3, dW2, dk, -lr[:, None] * d_dy, -_np.sum(v * d_dy, axis=1)
 
 
+def _newton_schulz_np(G, steps, coef, eps):
+    a, b, c = coef
+    X = G / (_np.sqrt(_np.sum(G * G)) + eps)
+    tall = X.shape[0] > X.shape[1]
+    if tall:
+        X = X.T
+    for _ in range(steps):
+        A = X @ X.T
+        X = a * X + (b * A + c * (A @ A)) @ X
+    return X.T if tall else X
+
+
+def _newton_schulz_vjp(G, dY, steps, coef, eps):
+    """Y = NS(G) (Frobenius normalisation, wide orientation, quintic steps
+    X <- a X + (b A + c A^2) X with A = X X^T): the upstream dY taken back to
+    G.  Each step's A and B = b A + c A^2 are symmetric, so
+        dX_prev = a dX + B dX + (dA + dA^T) X,  dB = dX X^T,
+        dA = b dB + c (dB A + A dB);
+    the normalisation X0 = G / (n + eps), n = ||G||_F, gives
+        dG = dX0 / (n + eps) - G <dX0, G> / (n (n + eps)^2)."""
+    a, b, c = coef
+    n = _np.sqrt(_np.sum(G * G))
+    X = G / (n + eps)
+    tall = X.shape[0] > X.shape[1]
+    if tall:
+        X, dY = X.T, dY.T
+    xs = []
+    for _ in range(steps):
+        xs.append(X)
+        A = X @ X.T
+        X = a * X + (b * A + c * (A @ A)) @ X
+    dX = dY
+    for X in reversed(xs):
+        A = X @ X.T
+        Bm = b * A + c * (A @ A)
+        dB = dX @ X.T
+        dA = b * dB + c * (dB @ A + A @ dB)
+        dX = a * dX + Bm @ dX + (dA + dA.T) @ X
+    if tall:
+        dX = dX.T
+    return dX / (n + eps) - G * (_np.sum(dX * G) / (n * (n + eps) ** 2))
+
+
 def _norm_rows_vjp(U, dW, eps):
     """W = U / max(||U_row||, eps): the upstream dW taken back to U."""
     n = _np.sqrt(_np.sum(U * U, axis=-1, keepdims=True))
@@ -237,12 +280,13 @@ def _norm_rows_vjp(U, dW, eps):
 
 
 def lact_backward_explicit(q, k, v, lr, W1, W3, W2, dout, dW_end=None, *, chunk,
-                           order="causal", opt="gd", beta=0.9, normalize_rows=True,
+                           order="causal", opt="gd", beta=0.9, ns_steps=5,
+                           ns_coef=(3.4445, -4.7750, 2.0315), ns_eps=1e-7, normalize_rows=True,
                            norm_eps=1e-12, update_mask=7):
-    """The gradients of lact_backward, computed by the steps above (GD and
-    momentum).  Same arguments and results."""
-    if opt not in ("gd", "momentum"):
-        raise ValueError("the written-out form covers GD and momentum")
+    """The gradients of lact_backward, computed by the steps above (GD,
+    momentum and Muon).  Same arguments and results."""
+    if opt not in ("gd", "momentum", "muon"):
+        raise ValueError(opt)
     f = lambda a: _np.asarray(a, dtype=_np.float64)  # noqa: E731
     q, k, v, lr, dout = f(q), f(k), f(v), f(lr), f(dout)
     W0 = [f(W1), f(W3), f(W2)]
@@ -261,17 +305,22 @@ def lact_backward_explicit(q, k, v, lr, W1, W3, W2, dout, dW_end=None, *, chunk,
                 G = _chunk_gradients_np(*W, k[b, h, t0:t1], v[b, h, t0:t1], lr[b, h, t0:t1])
                 start = [w.copy() for w in W]
                 Us = [None] * 3
+                Ms = [None] * 3
                 for i in range(3):
                     if not update_mask & bits[i]:
                         continue
                     if opt == "momentum":
                         M[i] = beta * M[i] + G[i]
                         U = W[i] - M[i]
+                    elif opt == "muon":
+                        M[i] = beta * M[i] + G[i]
+                        Ms[i] = M[i].copy()
+                        U = W[i] - _newton_schulz_np(M[i], ns_steps, ns_coef, ns_eps)
                     else:
                         U = W[i] - G[i]
                     Us[i] = U
                     W[i] = _normalize_rows_np(U, norm_eps) if normalize_rows else U
-                saved.append((t0, t1, start, Us))
+                saved.append((t0, t1, start, Us, Ms))
             # reverse
             dW = [_np.zeros_like(w) for w in W] if dW_end is None else \
                 [f(g)[b, h].copy() for g in dW_end]
@@ -281,7 +330,7 @@ def lact_backward_explicit(q, k, v, lr, W1, W3, W2, dout, dW_end=None, *, chunk,
                     dW[i] += r[i]
                 grads[0][b, h] = r[3]
             dM = [_np.zeros_like(w) for w in W]
-            for t0, t1, start, Us in reversed(saved):
+            for t0, t1, start, Us, Ms in reversed(saved):
                 R = [_np.zeros_like(w) for w in W]
                 for i in range(3):
                     if Us[i] is None:
@@ -290,6 +339,10 @@ def lact_backward_explicit(q, k, v, lr, W1, W3, W2, dout, dW_end=None, *, chunk,
                     if opt == "momentum":
                         dM[i] = dM[i] - dU      # U = W - M
                         R[i] = dM[i]            # M = beta M_prev + G
+                        dM[i] = beta * dM[i]
+                    elif opt == "muon":         # U = W - NS(M)
+                        dM[i] = dM[i] + _newton_schulz_vjp(Ms[i], -dU, ns_steps, ns_coef, ns_eps)
+                        R[i] = dM[i]
                         dM[i] = beta * dM[i]
                     else:
                         R[i] = -dU              # U = W - G

@@ -106,9 +106,10 @@ def test_planted_missing_second_order_term_is_caught():
     del torch
 
 
-EXPLICIT_CASES = [c for c in CASES if c["opt"] in ("gd", "momentum")] + [
+EXPLICIT_CASES = CASES + [
     dict(chunk=2, order="causal", opt="momentum", beta=0.7, update_mask=5),
     dict(chunk=7, order="bidirectional", opt="momentum", beta=0.9, normalize_rows=False),
+    dict(chunk=3, order="bidirectional", opt="muon", beta=0.8, ns_steps=5),
 ]
 
 
