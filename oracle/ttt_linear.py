@@ -12,7 +12,15 @@ and the read is o_t = W q_t.  Unrolled, o_t = W_0 q_t + sum_{s<=t} eta_s
 Conventions (readings of the pages, all stated once here):
   * the state handed across calls is S = W^T with shape [dk, dv];
   * ``include_diag=True`` (default): token t reads W after its own update
-    (o_t = W_t q_t, inclusive causal mask); ``False`` reads before it.
+    (o_t = W_t q_t, inclusive causal mask); ``False`` reads before it;
+  * ``order="bidirectional"``: every token's update is applied first and
+    every query then reads the final W, o_t = W_N q_t.  This is the unmasked
+    form that the xiaoxiang.io post on the KV-binding paper (section
+    "线性注意力视角", the linear-attention view) writes as X A X^T X B: linear
+    attention with no causal mask.  It is also the linear counterpart of
+    the write-then-read order of posed-image sets in the "Test-Time Training
+    Done Right" review ("El orden de lectura evita información futura").
+    include_diag plays no role there.
 All arithmetic is float64.
 """
 from __future__ import annotations
@@ -24,18 +32,29 @@ def _f64(x):
     return np.asarray(x, dtype=np.float64)
 
 
-def ttt_linear_recurrent(q, k, v, lr, S0=None, include_diag=True):
+def ttt_linear_recurrent(q, k, v, lr, S0=None, include_diag=True, order="causal"):
     """Token-by-token TTT recurrence (the definition).
 
     q, k: [B,H,N,dk]; v: [B,H,N,dv]; lr: [B,H,N]; S0: [B,H,dk,dv] or None.
+    order: "causal" (each token reads as it goes) or "bidirectional" (every
+    token writes, then every query reads the final weight).
     Returns (out [B,H,N,dv] float64, S_end [B,H,dk,dv] float64).
     """
+    if order not in ("causal", "bidirectional"):
+        raise ValueError(order)
     q, k, v, lr = _f64(q), _f64(k), _f64(v), _f64(lr)
     B, H, N, dk = q.shape
     dv = v.shape[-1]
     # W = S^T  (dv x dk) per (b, h)
     W = np.zeros((B, H, dv, dk)) if S0 is None else np.swapaxes(_f64(S0), -1, -2).copy()
     out = np.empty((B, H, N, dv))
+    if order == "bidirectional":
+        for t in range(N):
+            # the same GD step on -<W k_t, v_t> as the causal order, no reads yet
+            W += lr[:, :, t, None, None] * (v[:, :, t, :, None] * k[:, :, t, None, :])
+        for t in range(N):
+            out[:, :, t] = np.einsum("bhij,bhj->bhi", W, q[:, :, t])
+        return out, np.swapaxes(W, -1, -2).copy()
     for t in range(N):
         # gradient of -<W k_t, v_t> w.r.t. W is -v_t k_t^T; one GD step of size eta_t
         step = lr[:, :, t, None, None] * (v[:, :, t, :, None] * k[:, :, t, None, :])
@@ -48,10 +67,12 @@ def ttt_linear_recurrent(q, k, v, lr, S0=None, include_diag=True):
     return out, np.swapaxes(W, -1, -2).copy()
 
 
-def ttt_linear_attention_sum(q, k, v, lr, S0=None, include_diag=True, t_index=None):
+def ttt_linear_attention_sum(q, k, v, lr, S0=None, include_diag=True, t_index=None,
+                             order="causal"):
     """The same outputs written as the causal linear-attention sum
         o_t = S0^T q_t + sum_{s <= t (or s < t)} eta_s (q_t . k_s) v_s
-    evaluated directly for the token positions in ``t_index`` (all if None).
+    (bidirectional order: the sum runs over every s), evaluated directly for
+    the token positions in ``t_index`` (all if None).
     Cost O(|t_index| * N * d); used for sampled checks at full sizes.
     Returns [B,H,len(t_index),dv] float64.
     """
@@ -62,6 +83,8 @@ def ttt_linear_attention_sum(q, k, v, lr, S0=None, include_diag=True, t_index=No
     out = np.zeros((B, H, len(idx), dv))
     for j, t in enumerate(idx):
         last = t + 1 if include_diag else t
+        if order == "bidirectional":
+            last = N
         if last > 0:
             scores = np.einsum("bhd,bhsd->bhs", q[:, :, t], k[:, :, :last]) * lr[:, :, :last]
             out[:, :, j] = np.einsum("bhs,bhsd->bhd", scores, v[:, :, :last])

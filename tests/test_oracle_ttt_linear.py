@@ -90,3 +90,68 @@ def test_planted_index_mistake_is_caught():
     o_wrong, _ = ttt_linear_recurrent(q, k, v, lr, None, include_diag=False)
     o_sum = ttt_linear_attention_sum(q, k, v, lr, None, include_diag=True)
     assert np.abs(o_wrong - o_sum).max() > 1e-3
+
+
+# ---------------------------------------------------------------- bidirectional order
+# Every token writes, then every query reads the final weight: linear attention
+# with no causal mask (the xiaoxiang.io post on the KV-binding paper, section
+# "线性注意力视角": TTT-KV(X) = X A X^T X B).
+
+@pytest.mark.parametrize("with_s0", [False, True])
+def test_bidirectional_equals_unmasked_attention_sum(with_s0):
+    q, k, v, lr, S0 = _rand()
+    S0 = S0 if with_s0 else None
+    o_rec, _ = ttt_linear_recurrent(q, k, v, lr, S0, order="bidirectional")
+    o_sum = ttt_linear_attention_sum(q, k, v, lr, S0, order="bidirectional")
+    np.testing.assert_allclose(o_rec, o_sum, rtol=0, atol=1e-12 * np.abs(o_sum).max())
+
+
+def test_bidirectional_constant_lr_is_the_matrix_product_form():
+    """With a constant learning rate c and W0 = 0 the layer is c (Q K^T) V,
+    the X A X^T X B form with Q = X A, K = X, V = X B (a matmul identity)."""
+    r = np.random.default_rng(3)
+    X = r.standard_normal((1, 1, 29, 6))
+    A = r.standard_normal((6, 6))
+    Bm = r.standard_normal((6, 4))
+    c = 0.37
+    q, k, v = X @ A, X, X @ Bm
+    lr = np.full((1, 1, 29), c)
+    o, _ = ttt_linear_recurrent(q, k, v, lr, None, order="bidirectional")
+    expect = c * (X[0, 0] @ A @ X[0, 0].T @ X[0, 0] @ Bm)
+    np.testing.assert_allclose(o[0, 0], expect, rtol=0, atol=1e-12 * np.abs(expect).max())
+
+
+def test_bidirectional_read_is_a_causal_read_after_the_sequence():
+    """o_t equals what the causal recurrence reads for a query q_t appended
+    after the whole sequence with a zero update (k = v = 0, eta = 0)."""
+    q, k, v, lr, S0 = _rand(N=17)
+    o_bi, S_bi = ttt_linear_recurrent(q, k, v, lr, S0, order="bidirectional")
+    for t in (0, 5, 16):
+        q2 = np.concatenate([q, q[:, :, t:t + 1]], 2)
+        k2 = np.concatenate([k, np.zeros_like(k[:, :, :1])], 2)
+        v2 = np.concatenate([v, np.zeros_like(v[:, :, :1])], 2)
+        lr2 = np.concatenate([lr, np.zeros_like(lr[:, :, :1])], 2)
+        o_c, S_c = ttt_linear_recurrent(q2, k2, v2, lr2, S0)
+        np.testing.assert_allclose(o_bi[:, :, t], o_c[:, :, -1], rtol=0,
+                                   atol=1e-12 * np.abs(o_c).max())
+    np.testing.assert_allclose(S_bi, S_c, rtol=0, atol=1e-12 * np.abs(S_c).max())
+
+
+def test_bidirectional_is_equivariant_under_token_permutation():
+    q, k, v, lr, S0 = _rand(N=21)
+    perm = np.random.default_rng(5).permutation(21)
+    o, S = ttt_linear_recurrent(q, k, v, lr, S0, order="bidirectional")
+    o_p, S_p = ttt_linear_recurrent(q[:, :, perm], k[:, :, perm], v[:, :, perm], lr[:, :, perm],
+                                    S0, order="bidirectional")
+    np.testing.assert_allclose(o_p, o[:, :, perm], rtol=0, atol=1e-12 * np.abs(o).max())
+    np.testing.assert_allclose(S_p, S, rtol=0, atol=1e-12 * np.abs(S).max())
+
+
+def test_planted_causal_mask_in_bidirectional_is_caught():
+    """The causal recurrence (a mask left in place) disagrees with the
+    unmasked sum everywhere but the last token."""
+    q, k, v, lr, _ = _rand(N=13)
+    o_causal, _ = ttt_linear_recurrent(q, k, v, lr, None)
+    o_sum = ttt_linear_attention_sum(q, k, v, lr, None, order="bidirectional")
+    assert np.abs(o_causal[:, :, :-1] - o_sum[:, :, :-1]).max() > 1e-3
+    np.testing.assert_allclose(o_causal[:, :, -1], o_sum[:, :, -1], rtol=0, atol=1e-12)
