@@ -71,7 +71,11 @@ def _chunk_gradients(W1, W3, W2, k, v, lr):
 
 def _newton_schulz(G, steps, coef, eps):
     a, b, c = coef
-    X = G / (torch.sqrt(torch.sum(G * G, dim=(-2, -1), keepdim=True)) + eps)
+    # X0 = G / (||G||_F + eps) is differentiable at G = 0 (derivative I / eps,
+    # since eps > 0); the clamp keeps autograd's sqrt finite there and changes
+    # the forward value by less than 1e-150
+    n = torch.sqrt(torch.clamp_min(torch.sum(G * G, dim=(-2, -1), keepdim=True), 1e-300))
+    X = G / (n + eps)
     tall = X.shape[-2] > X.shape[-1]
     if tall:
         X = X.transpose(-2, -1)
@@ -267,7 +271,9 @@ def _newton_schulz_vjp(G, dY, steps, coef, eps):
         dX = a * dX + Bm @ dX + (dA + dA.T) @ X
     if tall:
         dX = dX.T
-    return dX / (n + eps) - G * (_np.sum(dX * G) / (n * (n + eps) ** 2))
+    # at G = 0 the second term's limit is 0 (|G| |G| / n -> 0)
+    corr = 0.0 if n == 0 else _np.sum(dX * G) / (n * (n + eps) ** 2)
+    return dX / (n + eps) - G * corr
 
 
 def _norm_rows_vjp(U, dW, eps):

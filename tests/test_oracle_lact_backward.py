@@ -125,3 +125,38 @@ def test_written_out_backward_equals_autograd(kw):
     for name, g, r in zip(("q", "k", "v", "lr", "W1", "W3", "W2"), got, ref):
         np.testing.assert_allclose(g, r, rtol=0, atol=1e-10 * max(1.0, np.abs(r).max()),
                                    err_msg=name)
+
+
+def test_muon_chunk_with_zero_learning_rates():
+    """A first chunk whose learning rates are all zero leaves the momentum
+    buffer at exactly zero, and Newton-Schulz maps it to zero.  X0 = G /
+    (||G||_F + eps) is differentiable there (derivative I / eps), so both
+    backward oracles must stay finite, agree, and match central differences."""
+    from oracle.lact_backward import lact_backward_explicit
+    kw = dict(chunk=3, order="causal", opt="muon", beta=0.9, ns_steps=3)
+    x, dout, dW = _rand(N=7, seed=4)
+    x["lr"][..., :3] = 0.0
+    args = (x["q"], x["k"], x["v"], x["lr"], x["W1"], x["W3"], x["W2"], dout, dW)
+    ref = lact_backward(*args, **kw)
+    got = lact_backward_explicit(*args, **kw)
+    for name, g, r in zip(("q", "k", "v", "lr", "W1", "W3", "W2"), got, ref):
+        assert np.isfinite(g).all() and np.isfinite(r).all(), name
+        np.testing.assert_allclose(g, r, rtol=0, atol=1e-10 * max(1.0, np.abs(r).max()),
+                                   err_msg=name)
+    # Inside the zero chunk the map is linear only while ||G|| << eps = 1e-7,
+    # so the difference step there is 1e-12 (the result is ~1e9, so the
+    # rounding of the loss difference stays far below the tolerance); the
+    # token of the second chunk (a momentum buffer away from zero) takes the
+    # usual step.
+    for idx, h in [((0, 0, 0), 1e-12), ((0, 1, 2), 1e-12), ((0, 0, 5), 2e-4)]:
+        def loss(val):
+            old = x["lr"][idx]
+            x["lr"][idx] = val
+            L = _np_loss(x, dout, dW, **kw)
+            x["lr"][idx] = old
+            return L
+        c = x["lr"][idx]
+        fd1 = (loss(c + h) - loss(c - h)) / (2 * h)
+        fd2 = (loss(c + h / 2) - loss(c - h / 2)) / h
+        fd = (4 * fd2 - fd1) / 3
+        assert abs(got[3][idx] - fd) <= 1e-5 * max(1.0, abs(fd)), (idx, got[3][idx], fd)
