@@ -70,13 +70,20 @@ typedef enum { TTT_OPT_GD = 0, TTT_OPT_MOMENTUM = 1, TTT_OPT_MUON = 2 } ttt_opt;
 #define TTT_STATUS_BYTES 256
 
 /* ------------------------------------------------------------------------
- * Case (a): linear fast weight == causal linear attention.
+ * Case (a): linear fast weight == linear attention.
  * "Test-Time Training with KV Binding Is Secretly Linear Attention",
  * summary "B. Reformulación Teórica" and "Formulación Paralela".
  *
  *   state S = W^T, float32 [B, H, dk, dv]
- *   for t in 0..N-1:  S += lr_t k_t v_t^T ;  out_t = S^T q_t
- *   (include_diag = 0: out_t is read before token t's own update)
+ *   causal:  for t in 0..N-1:  S += lr_t k_t v_t^T ;  out_t = S^T q_t
+ *            (include_diag = 0: out_t is read before token t's own update)
+ *   bidirectional:  S += sum_t lr_t k_t v_t^T over all N tokens, then
+ *            out_t = S^T q_t for every t with that final S.  This is linear
+ *            attention with no causal mask, the X A X^T X B form of the
+ *            xiaoxiang.io post on the same paper (section "线性注意力视角"),
+ *            and the write-then-read order that the "Test-Time Training Done
+ *            Right" review gives posed-image sets ("El orden de lectura
+ *            evita información futura"); include_diag is ignored.
  *
  * `chunk` is the blocking of the chunked form.  Because the gradient of the
  * binding loss does not depend on W, the result is the same for every chunk
@@ -86,30 +93,43 @@ typedef struct {
   int B, H, N;          /* batch, heads, tokens (N >= 0)                     */
   int dk, dv;           /* key/query dim, value dim                          */
   int chunk;            /* > 0                                               */
-  int include_diag;     /* 1: token reads after its own update (default)    */
+  ttt_order order;      /* TTT_CAUSAL or TTT_BIDIRECTIONAL                   */
+  int include_diag;     /* causal: 1 = token reads after its own update     */
   ttt_dtype in_dtype;   /* q, k, v element type (TTT_F32 or TTT_BF16)        */
   ttt_dtype out_dtype;  /* out element type                                  */
 } ttt_linear_desc;
 
-/* Workspace bytes for ttt_linear_fwd at full speed: the status block, plus,
- * on the tensor-core path (bf16, dk = dv = 64), room for the start states of
- * the sequence segments that run on separate SMs (the state after a token is
- * S0 plus the sum of the updates before it, so a head's sequence splits into
- * segments whose start states a pre-pass sums).  The size depends on the
- * device's SM count; a workspace of only TTT_STATUS_BYTES is accepted and
- * runs each head unsplit. */
+/* Workspace bytes for ttt_linear_fwd at full speed (same summary,
+ * "Formulación Paralela": the state after a token is S0 plus the sum of the
+ * updates before it, a prefix scan).  The status block, plus, on the
+ * tensor-core path (bf16, dk = dv = 64), room for partial state sums:
+ *   causal: the start states of the sequence segments that run on separate
+ *     SMs (a pre-pass sums each segment's updates);
+ *   bidirectional: the per-unit sums of the whole-sequence state pass.
+ * The size depends on the device's SM count.  A workspace of only
+ * TTT_STATUS_BYTES is accepted: a causal call then runs each head unsplit,
+ * a bidirectional one runs on CUDA cores.  Errors: TTT_ERR_ARG (null
+ * pointers), the shape and dtype errors of ttt_linear_fwd. */
 int ttt_linear_workspace_bytes(const ttt_linear_desc* desc, size_t* bytes);
 
-/* S <- S0 (device float32 [B,H,dk,dv]); S0 == NULL zero-fills S. */
+/* The state before the first token (same summary, "B. Reformulación
+ * Teórica": the fast weight the recurrence starts from, W0 = S0^T).
+ * S <- S0 (device float32 [B,H,dk,dv], caller-owned); S0 == NULL zero-fills
+ * S.  Enqueued on `stream`; TTT_ERR_CUDA if the copy cannot be enqueued. */
 int ttt_linear_state_init(const ttt_linear_desc* desc, const float* S0, float* S, void* stream);
 
-/* dst <- S; dst may be a device pointer or pinned/registered host memory. */
+/* Readout of the fast weight after a call (same summary: the state the next
+ * call of a streamed sequence continues from).  dst <- S, float32
+ * [B,H,dk,dv]; dst may be a device pointer or pinned/registered host memory.
+ * Enqueued on `stream`; TTT_ERR_CUDA if the copy cannot be enqueued. */
 int ttt_linear_state_readout(const ttt_linear_desc* desc, const float* S, float* dst, void* stream);
 
 /* One call over N tokens.  q, k: [B,H,N,dk]; v: [B,H,N,dv]; lr: [B,H,N];
  * S: in = state before the first token, out = state after the last token;
  * out: [B,H,N,dv].  Supported: in_dtype F32 (any dk, dv <= 128) and BF16
- * (dk = dv = 64 on tensor cores; other dims <= 128 on CUDA cores).
+ * (dk = dv = 64 on tensor cores; other dims <= 128 on CUDA cores), in
+ * either order.  A bidirectional call on tensor cores first sums the whole
+ * sequence's updates into S, then reads every query with that S.
  * ws (>= TTT_STATUS_BYTES, device, caller-owned) holds the status block and
  * the segment states (see ttt_linear_workspace_bytes); it must not be shared
  * by calls that overlap in time. */
@@ -126,7 +146,8 @@ int ttt_linear_fwd(const ttt_linear_desc* desc, const void* q, const void* k, co
  *   dlr_s = k_s^T R_s v_s,  dS0 = dS_end + sum_t q_t dout_t^T,
  * where S_t is the state token t read (desc->include_diag as in the forward
  * call).  Each is computed as a forward-time causal scan with the roles of
- * q, k, v and dout exchanged, on the kernels of ttt_linear_fwd.
+ * q, k, v and dout exchanged, on the kernels of ttt_linear_fwd.  Causal order
+ * only: a bidirectional desc returns TTT_ERR_UNSUPPORTED.
  * Inputs (device): q, k [B,H,N,dk], v [B,H,N,dv], lr [B,H,N] as given to the
  * forward call; S0 [B,H,dk,dv] float32, the forward call's start state (NULL =
  * zeros); dout [B,H,N,dv] in desc->in_dtype; dS_end [B,H,dk,dv] float32 (NULL =
@@ -228,6 +249,72 @@ int lact_chunk_fwd(const lact_desc* desc, const void* q, const void* k, const vo
                    const float* lr, void* state, void* out, void* ws, size_t ws_bytes,
                    void* stream);
 
+/* ------------------------------------------------------------------------
+ * Context parallelism: the tokens of one chunk split across devices.
+ * "Test-Time Training Done Right" review, "Vídeo y cálculo distribuido":
+ * every device computes the gradient of its share of a chunk's tokens, the
+ * shares are summed across devices, and every device applies the same
+ * update to its copy of the weights.  These three calls are the per-device
+ * pieces of lact_chunk_fwd; the sum between them is the caller's collective
+ * (an all-reduce into each device's own G).  Per chunk of a causal call:
+ *   lact_read (the chunk's queries, current weights), lact_chunk_grad (this
+ *   device's tokens of the chunk), all-reduce of G, lact_apply_grad;
+ * a bidirectional call does the last three per chunk and lact_read of the
+ * queries at the end.  desc, state and ws are as for lact_chunk_fwd (ws of
+ * at least lact_workspace_bytes_min); the calls keep no state of their own.
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of a chunk gradient G: [G1 | G3 | G2], each [B,H,rows,cols] float32,
+ * laid out like the weights of the state. */
+int lact_grad_bytes(const lact_desc* desc, size_t* bytes);
+
+/* G <- sum over tokens t in [t0, t0 + n) of lr_t times the gradient of
+ * -<f_W(k_t), v_t> at the state's current weights (no update; G is
+ * overwritten).  k, v: [B,H,N_in,d]; lr: [B,H,N_in]; n <= desc->chunk
+ * (a share of one chunk), t0 + n <= N_in, else TTT_ERR_SHAPE.  n = 0 writes
+ * zeros. */
+int lact_chunk_grad(const lact_desc* desc, int t0, int n, const void* k, const void* v,
+                    const float* lr, const void* state, float* G, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/* The update of one chunk with the (summed) chunk gradient G: GD / momentum /
+ * Muon as in lact_chunk_fwd, then the row normalisation, on `state`. */
+int lact_apply_grad(const lact_desc* desc, const float* G, void* state, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* out rows [t0, t0 + n) <- f_W(q rows [t0, t0 + n)) with the state's current
+ * weights ("El orden de lectura evita información futura": a causal chunk
+ * reads the weights left by earlier chunks, queries of a posed-image set read
+ * the final ones).  q, out: [B,H,R,d] with R = N_in (causal) or N_q
+ * (bidirectional); n at most one chunk (causal) or N_q, else TTT_ERR_SHAPE. */
+int lact_read(const lact_desc* desc, int t0, int n, const void* q, const void* state, void* out,
+              void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Backward pass of lact_chunk_fwd, for training through the layer ("Test-Time
+ * Training Done Right" review, "Lenguaje: calidad y velocidad no son
+ * equivalentes": the layer's training throughput with GD, momentum and Muon
+ * updates).  The gradients of
+ *   L = sum <dout, out> + sum_m <dW_end[m], W_m after the call>
+ * with respect to q, k, v, lr and the weights at the start of the call,
+ * through every chunk's update (chunk gradients at the chunk-start weights,
+ * optimizer step, row normalisation) and every read.  GD and MOMENTUM (the
+ * momentum buffers start at zero, as after lact_state_init); MUON returns
+ * TTT_ERR_UNSUPPORTED.  The call replays the forward chunk loop to keep each
+ * chunk's start weights, then walks the chunks in reverse.
+ * state0: the state the forward call started from (its W1, W3, W2 are read);
+ * dout: [B,H,R,d] bf16 with R = N_in (causal) or N_q (bidirectional);
+ * dW_end: nullable [dW1 | dW3 | dW2] float32 in the state's weight layout.
+ * Outputs, float32, written in full: dq [B,H,R,d], dk, dv [B,H,N_in,d],
+ * dlr [B,H,N_in], dW0 [dW1 | dW3 | dW2] (the state's weight layout).
+ * ws: device workspace of at least lact_bwd_workspace_bytes, status block
+ * first. */
+int lact_bwd_workspace_bytes(const lact_desc* desc, size_t* bytes);
+int lact_chunk_bwd(const lact_desc* desc, const void* q, const void* k, const void* v,
+                   const float* lr, const void* state0, const void* dout, const float* dW_end,
+                   float* dq, float* dk, float* dv, float* dlr, float* dW0, void* ws,
+                   size_t ws_bytes, void* stream);
+
 /* Same computation as lact_chunk_fwd for callers that cannot allocate device
  * memory (code hosted by a program that owns all device allocations and
  * hands it only its tensors; paths where cudaMalloc/cudaFree and their
@@ -237,11 +324,22 @@ int lact_chunk_fwd(const lact_desc* desc, const void* q, const void* k, const vo
  * that loads the library until exit; problems needing more (see
  * lact_workspace_bytes_min) return TTT_ERR_WORKSPACE and nothing runs.  The
  * first call on a device looks up the array's address with that device
- * current.  All calls share the array: each call clears its status block on
- * `stream`; calls whose GPU work overlaps race and must not be issued.  The
- * status block is not readable through ttt_check_device_status. */
+ * current (make that first call before any stream capture); a
+ * cudaDeviceReset of the device invalidates it, so do not call the entry
+ * point after one.  `stream` must belong to the current device
+ * (TTT_ERR_ARG otherwise).  All calls share the array: each call clears its
+ * status block on `stream`; calls whose GPU work overlaps race and must not
+ * be issued.  Read the status block with lact_noalloc_check_status. */
 int lact_chunk_fwd_noalloc(const lact_desc* desc, const void* q, const void* k, const void* v,
                            const float* lr, void* state, void* out, void* stream);
+
+/* ttt_check_device_status for the scratch array of lact_chunk_fwd_noalloc
+ * on the current device: synchronises `stream` (which must belong to the
+ * current device), then reads and clears the status block of the last call.
+ * Returns TTT_OK, TTT_ERR_TIMEOUT (a bounded wait of that call ran out),
+ * TTT_ERR_ARG (stream of another device) or TTT_ERR_CUDA.  Like the entry
+ * point it serves, it has no counterpart in the pages. */
+int lact_noalloc_check_status(void* stream);
 
 /* ------------------------------------------------------------------------
  * Local branch of the LaCT language layer: causal sliding-window attention.

@@ -12,7 +12,9 @@ from ._lib import (  # noqa: F401
     LIB_PATH, TTT_BF16, TTT_BIDIRECTIONAL, TTT_CAUSAL, TTT_ERR_ALIGN, TTT_ERR_ARG, TTT_ERR_CUDA,
     TTT_ERR_DTYPE, TTT_ERR_SHAPE, TTT_ERR_TIMEOUT, TTT_ERR_UNSUPPORTED, TTT_ERR_WORKSPACE,
     TTT_F32, TTT_OK, TTT_OPT_GD, TTT_OPT_MOMENTUM, TTT_OPT_MUON, TTT_STATUS_BYTES, TTTError,
-    lact_chunk_fwd, lact_chunk_fwd_noalloc, lact_desc, lact_layer_fwd, ttt_window_attn_fwd,
+    lact_apply_grad, lact_bwd_workspace_bytes, lact_chunk_bwd, lact_chunk_fwd, lact_chunk_fwd_noalloc, lact_chunk_grad, lact_grad_bytes,
+    lact_noalloc_check_status, lact_desc, lact_read,
+    lact_layer_fwd, ttt_window_attn_fwd,
     ttt_window_desc, lact_state_bytes, lact_state_init, lact_state_readout,
     lact_workspace_bytes, lact_workspace_bytes_min, load, status_string, ttt_build_info, ttt_check_device_status,
     ttt_linear_bwd, ttt_linear_bwd_workspace_bytes, ttt_linear_desc, ttt_linear_fwd,
@@ -25,9 +27,9 @@ _OPT = {"gd": TTT_OPT_GD, "momentum": TTT_OPT_MOMENTUM, "muon": TTT_OPT_MUON}
 
 
 def make_linear_desc(B, H, N, dk, dv, chunk, include_diag=True, in_dtype="bf16",
-                     out_dtype="f32") -> ttt_linear_desc:
-    return ttt_linear_desc(B, H, N, dk, dv, chunk, int(bool(include_diag)), _DT[in_dtype],
-                           _DT[out_dtype])
+                     out_dtype="f32", order="causal") -> ttt_linear_desc:
+    return ttt_linear_desc(B, H, N, dk, dv, chunk, _ORDER[order], int(bool(include_diag)),
+                           _DT[in_dtype], _DT[out_dtype])
 
 
 def make_lact_desc(B, H, N_in, d, dh, chunk, *, N_q=None, order="causal", opt="gd", beta=0.9,

@@ -29,8 +29,8 @@ class TTTError(RuntimeError):
 class ttt_linear_desc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
-                ("include_diag", ctypes.c_int), ("in_dtype", ctypes.c_int),
-                ("out_dtype", ctypes.c_int)]
+                ("order", ctypes.c_int), ("include_diag", ctypes.c_int),
+                ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
 
 
 class lact_desc(ctypes.Structure):
@@ -73,7 +73,14 @@ _SIGS = {
     "lact_state_init": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _I, _VP, _VP],
     "lact_state_readout": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _VP, _VP, _VP],
     "lact_chunk_fwd": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "lact_grad_bytes": [ctypes.POINTER(lact_desc), _SZP],
+    "lact_chunk_grad": [ctypes.POINTER(lact_desc), _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "lact_apply_grad": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _SZ, _VP],
+    "lact_read": [ctypes.POINTER(lact_desc), _I, _I, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "lact_bwd_workspace_bytes": [ctypes.POINTER(lact_desc), _SZP],
+    "lact_chunk_bwd": [ctypes.POINTER(lact_desc)] + [_VP] * 14 + [_SZ, _VP],
     "lact_chunk_fwd_noalloc": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "lact_noalloc_check_status": [_VP],
     "ttt_check_device_status": [_VP, _VP],
     "ttt_selftest_wait_timeout": [_VP, _SZ, _I, _VP],
     "ttt_profile_begin": [],
@@ -230,11 +237,62 @@ def lact_chunk_fwd(desc, q, k, v, lr, state, out, ws, ws_bytes=None, stream=None
     return _check("lact_chunk_fwd", st) if check else st
 
 
+def lact_grad_bytes(desc: lact_desc) -> int:
+    n = ctypes.c_size_t(0)
+    _check("lact_grad_bytes", load().lact_grad_bytes(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
+def _nbytes(ws, ws_bytes):
+    return ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
+
+
+def lact_chunk_grad(desc, t0, n, k, v, lr, state, G, ws, ws_bytes=None, stream=None, check=True):
+    st = load().lact_chunk_grad(ctypes.byref(desc), int(t0), int(n), _ptr(k), _ptr(v), _ptr(lr),
+                                _ptr(state), _ptr(G), _ptr(ws), _nbytes(ws, ws_bytes),
+                                _stream(stream))
+    return _check("lact_chunk_grad", st) if check else st
+
+
+def lact_apply_grad(desc, G, state, ws, ws_bytes=None, stream=None, check=True):
+    st = load().lact_apply_grad(ctypes.byref(desc), _ptr(G), _ptr(state), _ptr(ws),
+                                _nbytes(ws, ws_bytes), _stream(stream))
+    return _check("lact_apply_grad", st) if check else st
+
+
+def lact_read(desc, t0, n, q, state, out, ws, ws_bytes=None, stream=None, check=True):
+    st = load().lact_read(ctypes.byref(desc), int(t0), int(n), _ptr(q), _ptr(state), _ptr(out),
+                          _ptr(ws), _nbytes(ws, ws_bytes), _stream(stream))
+    return _check("lact_read", st) if check else st
+
+
+def lact_bwd_workspace_bytes(desc: lact_desc) -> int:
+    n = ctypes.c_size_t(0)
+    _check("lact_bwd_workspace_bytes",
+           load().lact_bwd_workspace_bytes(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
+def lact_chunk_bwd(desc, q, k, v, lr, state0, dout, dW_end, dq, dk, dv, dlr, dW0, ws,
+                   ws_bytes=None, stream=None, check=True):
+    """Gradients of sum <dout, out> + <dW_end, W_end> (see include/ttt.h)."""
+    st = load().lact_chunk_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lr),
+                               _ptr(state0), _ptr(dout), _ptr(dW_end), _ptr(dq), _ptr(dk),
+                               _ptr(dv), _ptr(dlr), _ptr(dW0), _ptr(ws), _nbytes(ws, ws_bytes),
+                               _stream(stream))
+    return _check("lact_chunk_bwd", st) if check else st
+
+
 def lact_chunk_fwd_noalloc(desc, q, k, v, lr, state, out, stream=None, check=True):
     """lact_chunk_fwd with the library's fixed device scratch as workspace."""
     st = load().lact_chunk_fwd_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lr),
                                        _ptr(state), _ptr(out), _stream(stream))
     return _check("lact_chunk_fwd_noalloc", st) if check else st
+
+
+def lact_noalloc_check_status(stream=None) -> int:
+    """Status of the last lact_chunk_fwd_noalloc call on the current device."""
+    return load().lact_noalloc_check_status(_stream(stream))
 
 
 # ------------------------------------------------------------------ status

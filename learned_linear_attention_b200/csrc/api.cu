@@ -43,6 +43,7 @@ int check_linear(const ttt_linear_desc* d) {
   if (!d) return TTT_ERR_ARG;
   if (d->B < 1 || d->H < 1 || d->N < 0 || d->dk < 1 || d->dv < 1) return TTT_ERR_SHAPE;
   if (d->chunk < 1) return TTT_ERR_ARG;
+  if (d->order != TTT_CAUSAL && d->order != TTT_BIDIRECTIONAL) return TTT_ERR_ARG;
   if ((d->in_dtype != TTT_F32 && d->in_dtype != TTT_BF16) ||
       (d->out_dtype != TTT_F32 && d->out_dtype != TTT_BF16))
     return TTT_ERR_DTYPE;
@@ -126,7 +127,11 @@ int ttt_linear_workspace_bytes(const ttt_linear_desc* d, size_t* bytes) {
   if (e) return e;
   if (!bytes) return TTT_ERR_ARG;
   size_t seg = 0;
-  if (linear_uses_umma(d)) seg = ttt_linear_plan(d->B * d->H, d->N, device_sms()).ws_floats * sizeof(float);
+  if (linear_uses_umma(d))
+    seg = (d->order == TTT_BIDIRECTIONAL
+               ? ttt_linear_state_sum_floats(d->B * d->H, d->N, device_sms())
+               : ttt_linear_plan(d->B * d->H, d->N, device_sms()).ws_floats) *
+          sizeof(float);
   *bytes = TTT_STATUS_BYTES + seg;
   return TTT_OK;
 }
@@ -162,11 +167,18 @@ int ttt_linear_fwd(const ttt_linear_desc* d, const void* q, const void* k, const
   LinearLaunch L{};
   L.B = d->B; L.H = d->H; L.N = d->N; L.dk = d->dk; L.dv = d->dv; L.chunk = d->chunk;
   L.include_diag = d->include_diag ? 1 : 0;
+  L.bidir = d->order == TTT_BIDIRECTIONAL ? 1 : 0;
   L.in_bf16 = d->in_dtype == TTT_BF16;
   L.out_bf16 = d->out_dtype == TTT_BF16;
   L.q = q; L.k = k; L.v = v; L.lr = lr; L.S = S; L.out = out;
   L.st = status_of(ws, 1);
-  const bool umma = linear_uses_umma(d);
+  bool umma = linear_uses_umma(d);
+  // the bidirectional tensor-core path needs the state pass's partial sums
+  // in the workspace; with less it runs on CUDA cores
+  if (umma && L.bidir &&
+      ws_bytes - TTT_STATUS_BYTES <
+          ttt_linear_state_sum_floats(d->B * d->H, d->N, device_sms()) * sizeof(float))
+    umma = false;
   if (umma) {
     L.plan = ttt_linear_plan(d->B * d->H, d->N, device_sms());
     L.seg_state = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + TTT_STATUS_BYTES);
@@ -190,6 +202,7 @@ LinearBwdWorkspace linear_bwd_layout(const ttt_linear_desc* d, LinearPlan* plan)
 int ttt_linear_bwd_workspace_bytes(const ttt_linear_desc* d, size_t* bytes) {
   int e = check_linear(d);
   if (e) return e;
+  if (d->order != TTT_CAUSAL) return TTT_ERR_UNSUPPORTED;
   if (!bytes) return TTT_ERR_ARG;
   LinearPlan plan{};
   *bytes = linear_bwd_layout(d, &plan).total;
@@ -202,6 +215,7 @@ int ttt_linear_bwd(const ttt_linear_desc* d, const void* q, const void* k, const
                    size_t ws_bytes, void* stream) {
   int e = check_linear(d);
   if (e) return e;
+  if (d->order != TTT_CAUSAL) return TTT_ERR_UNSUPPORTED;
   if (!ws || !dS0) return TTT_ERR_ARG;
   LinearPlan plan{};
   const LinearBwdWorkspace w = linear_bwd_layout(d, &plan);
@@ -365,6 +379,137 @@ int lact_chunk_fwd(const lact_desc* d, const void* q, const void* k, const void*
   L.ws_bytes = ws_bytes;
   L.st = status_of(ws, 2);
   return launch_lact(L, as_stream(stream)) == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ context parallelism
+static void fill_lact_launch(const lact_desc* d, LactLaunch& L) {
+  const bool causal = d->order == TTT_CAUSAL;
+  L.B = d->B; L.H = d->H; L.N_in = d->N_in; L.N_q = causal ? d->N_in : d->N_q;
+  L.d = d->d; L.dh = d->dh; L.chunk = d->chunk; L.causal = causal ? 1 : 0;
+  L.opt = (int)d->opt; L.beta = d->beta; L.ns_steps = d->ns_steps;
+  L.ns_a = d->ns_coef[0]; L.ns_b = d->ns_coef[1]; L.ns_c = d->ns_coef[2]; L.ns_eps = d->ns_eps;
+  L.normalize_rows = d->normalize_rows ? 1 : 0; L.norm_eps = d->norm_eps;
+  L.update_mask = d->update_mask; L.out_bf16 = d->out_dtype == TTT_BF16;
+  L.split = d->split_operands ? 1 : 0;
+}
+
+int lact_grad_bytes(const lact_desc* d, size_t* bytes) {
+  int e = check_lact(d);
+  if (e) return e;
+  if (!bytes) return TTT_ERR_ARG;
+  *bytes = 3 * (size_t)d->B * d->H * d->d * d->dh * sizeof(float);
+  return TTT_OK;
+}
+
+int lact_chunk_grad(const lact_desc* d, int t0, int n, const void* k, const void* v,
+                    const float* lr, const void* state, float* G, void* ws, size_t ws_bytes,
+                    void* stream) {
+  int e = check_lact(d);
+  if (e) return e;
+  if (!state || !G || !ws) return TTT_ERR_ARG;
+  if (t0 < 0 || n < 0 || (long long)t0 + n > d->N_in || n > d->chunk) return TTT_ERR_SHAPE;
+  if (ws_bytes < layout_of(d, 0).total) return TTT_ERR_WORKSPACE;
+  if (n > 0 && (!k || !v || !lr)) return TTT_ERR_ARG;
+  if ((k && !aligned16(k)) || (v && !aligned16(v)) || (lr && !aligned16(lr)) ||
+      !aligned16(state) || !aligned16(G) || !aligned16(ws))
+    return TTT_ERR_ALIGN;
+  LactLaunch L{};
+  fill_lact_launch(d, L);
+  L.k = k; L.v = v; L.lr = lr;
+  L.state = reinterpret_cast<float*>(const_cast<void*>(state));
+  L.ws = reinterpret_cast<uint8_t*>(ws);
+  L.ws_bytes = ws_bytes;
+  L.st = status_of(ws, 2);
+  L.mode = LACT_GRAD; L.t0 = t0; L.n = n; L.G = G;
+  return launch_lact(L, as_stream(stream)) == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
+int lact_apply_grad(const lact_desc* d, const float* G, void* state, void* ws, size_t ws_bytes,
+                    void* stream) {
+  int e = check_lact(d);
+  if (e) return e;
+  if (!state || !G || !ws) return TTT_ERR_ARG;
+  if (ws_bytes < layout_of(d, 0).total) return TTT_ERR_WORKSPACE;
+  if (!aligned16(state) || !aligned16(G) || !aligned16(ws)) return TTT_ERR_ALIGN;
+  LactLaunch L{};
+  fill_lact_launch(d, L);
+  L.state = reinterpret_cast<float*>(state);
+  L.ws = reinterpret_cast<uint8_t*>(ws);
+  L.ws_bytes = ws_bytes;
+  L.st = status_of(ws, 2);
+  L.mode = LACT_APPLY; L.G = const_cast<float*>(G);
+  return launch_lact(L, as_stream(stream)) == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
+int lact_read(const lact_desc* d, int t0, int n, const void* q, const void* state, void* out,
+              void* ws, size_t ws_bytes, void* stream) {
+  int e = check_lact(d);
+  if (e) return e;
+  if (!state || !ws) return TTT_ERR_ARG;
+  const int rows = d->order == TTT_CAUSAL ? d->N_in : d->N_q;
+  if (t0 < 0 || n < 0 || (long long)t0 + n > rows) return TTT_ERR_SHAPE;
+  if (ws_bytes < layout_of(d, 0).total) return TTT_ERR_WORKSPACE;
+  if (n == 0) return TTT_OK;
+  if (!q || !out) return TTT_ERR_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(state) || !aligned16(ws)) return TTT_ERR_ALIGN;
+  // the read's intermediates hold at most one chunk (causal) or N_q rows
+  if (n > layout_of(d, 0).cmax) return TTT_ERR_SHAPE;
+  LactLaunch L{};
+  fill_lact_launch(d, L);
+  L.q = q;
+  L.state = reinterpret_cast<float*>(const_cast<void*>(state));
+  L.out = out;
+  L.ws = reinterpret_cast<uint8_t*>(ws);
+  L.ws_bytes = ws_bytes;
+  L.st = status_of(ws, 2);
+  L.mode = LACT_READ; L.t0 = t0; L.n = n;
+  return launch_lact(L, as_stream(stream)) == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ LaCT backward
+static int check_lact_bwd(const lact_desc* d) {
+  int e = check_lact(d);
+  if (e) return e;
+  if (d->opt == TTT_OPT_MUON) return TTT_ERR_UNSUPPORTED;
+  return TTT_OK;
+}
+
+int lact_bwd_workspace_bytes(const lact_desc* d, size_t* bytes) {
+  int e = check_lact_bwd(d);
+  if (e) return e;
+  if (!bytes) return TTT_ERR_ARG;
+  LactLaunch f{};
+  fill_lact_launch(d, f);
+  *bytes = lact_bwd_layout(f).total;
+  return TTT_OK;
+}
+
+int lact_chunk_bwd(const lact_desc* d, const void* q, const void* k, const void* v,
+                   const float* lr, const void* state0, const void* dout, const float* dW_end,
+                   float* dq, float* dk, float* dv, float* dlr, float* dW0, void* ws,
+                   size_t ws_bytes, void* stream) {
+  int e = check_lact_bwd(d);
+  if (e) return e;
+  if (!state0 || !dW0 || !ws) return TTT_ERR_ARG;
+  LactLaunch f{};
+  fill_lact_launch(d, f);
+  if (ws_bytes < lact_bwd_layout(f).total) return TTT_ERR_WORKSPACE;
+  const int rows = d->order == TTT_CAUSAL ? d->N_in : d->N_q;
+  if (d->N_in > 0 && (!k || !v || !lr || !dk || !dv || !dlr)) return TTT_ERR_ARG;
+  if (rows > 0 && (!q || !dout || !dq)) return TTT_ERR_ARG;
+  const void* ptrs[] = {q, k, v, lr, state0, dout, dW_end, dq, dk, dv, dlr, dW0, ws};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGN;
+  f.q = q; f.k = k; f.v = v; f.lr = lr;
+  f.st = status_of(ws, 4);
+  LactBwdLaunch L{};
+  L.f = f;
+  L.W0 = reinterpret_cast<const float*>(state0);
+  L.dout = dout; L.dW_end = dW_end;
+  L.dq = dq; L.dk = dk; L.dv = dv; L.dlr = dlr; L.dW0 = dW0;
+  L.ws = reinterpret_cast<uint8_t*>(ws);
+  L.st = f.st;
+  return launch_lact_bwd(L, as_stream(stream)) == 0 ? TTT_OK : TTT_ERR_CUDA;
 }
 
 int lact_layer_fwd(const lact_desc* d, int window, float scale, const void* q, const void* k,

@@ -77,6 +77,7 @@ struct LinearPlan {
 LinearPlan ttt_linear_plan(int BH, int N, int sms);
 struct LinearLaunch {
   int B, H, N, dk, dv, chunk, include_diag;
+  int bidir;    // bidirectional order: every update first, then every read
   int in_bf16, out_bf16;
   const void *q, *k, *v;
   const float* lr;
@@ -150,7 +151,26 @@ struct LactLaunch {
   uint8_t* ws;             // workspace (status block first)
   size_t ws_bytes;
   DevStatus st;
+  // Pieces of the chunk loop for context parallelism (a chunk's tokens split
+  // across devices): LACT_FULL runs the whole layer; LACT_GRAD writes to G
+  // the lr-weighted gradient sum of tokens [t0, t0 + n) (n <= chunk) at the
+  // current weights; LACT_APPLY applies the optimizer step and row
+  // normalisation with the (summed) chunk gradient G; LACT_READ writes out
+  // rows [t0, t0 + n) = f_W(q rows) with the current weights.
+  int mode;
+  int t0, n;
+  float* G;                // [G1 | G3 | G2] fp32, laid out like the weights of the state
+  float* rownorm_out;      // APPLY, nullable: each updated row's norm before the
+                           // normalisation, [BH][2 dh + d] (W1 rows, W3 rows, W2 rows)
 };
+enum LactMode { LACT_FULL = 0, LACT_GRAD = 1, LACT_APPLY = 2, LACT_READ = 3 };
+// The batched tcgen05 GEMM of gemm.cuh (operand majorness by variant).
+struct GemmMaps;
+struct GemmArgs;
+enum { GEMM_AK_BK = 0, GEMM_AK_BMN = 1, GEMM_AMN_BMN = 2 };
+int gemm_launch(int variant, const GemmMaps& maps, const GemmArgs& g, cudaStream_t stream,
+                int kind);
+GemmArgs gemm_args_default(const DevStatus& st);
 // Workspace layout (byte offsets) for a given problem.
 struct LactWorkspace {
   size_t status, w1b, w3b, w2b, d13, gm, aq, part, rowss, nsx32, nsxb, nsa32, nsab, nsbb, total;
@@ -163,7 +183,22 @@ struct LactWorkspace {
   size_t pmb;              // parallel form: bf16 chunk-start W2 [chunks][BH][d][dh]
   int nbuf;                // bf16 weight buffers (3 on the fused causal path, else 2)
   int naq;                 // Aq buffers (2 on the fused causal path, else 1)
+  size_t nsctr;            // Muon: phase counter of the fused Newton-Schulz kernel
 };
+// The Newton-Schulz loop of the Muon step as one cooperative launch
+// (ns_fused.cu): `steps` quintic steps on nb matrices r x c (r <= c).
+struct NsFusedLaunch {
+  int r, c, nb, steps, split;
+  float coef_a, coef_b, coef_c;
+  float* X32;                       // [nb][r][c] fp32, in/out
+  const __nv_bfloat16* Xb[2];       // bf16 hi copies of X (step parity)
+  const __nv_bfloat16* Xl[2];       // lo copies (split operands)
+  float* A32;                       // [nb][r][r]
+  __nv_bfloat16 *Ab, *Al, *Bb, *Bl;
+  unsigned* counter;                // zeroed before the launch
+  DevStatus st;
+};
+int launch_ns_fused(const NsFusedLaunch& L, cudaStream_t stream);
 bool lact_uses_keygrad(int d, int dh, int opt, int split);
 bool lact_uses_w2_parallel(int N_in, int chunk, int d, int dh, int causal, int opt, int split,
                            int update_mask, int normalize);
@@ -173,6 +208,24 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
                                     int causal, int opt, int split, int update_mask, int normalize,
                                     int allow_parallel);
 int launch_lact(const LactLaunch& L, cudaStream_t stream);
+
+// Backward pass of the LaCT layer (lact_bwd.cu).
+struct LactBwdWorkspace {
+  size_t status, fws, fws_bytes, state, wsave, rn, G, dW, dM, R, Rb, Wb, ddy, total;
+  size_t f32[6], b16[7];   // per-chunk intermediates [BH][cmax][dh]
+  int cmax, nch;
+};
+struct LactBwdLaunch {
+  LactLaunch f;            // the forward problem (shapes, optimizer, q, k, v, lr)
+  const float* W0;         // [W1 | W3 | W2] at the start of the call
+  const void* dout;        // [B,H,R,d] bf16 (R = N_in causal, N_q bidirectional)
+  const float* dW_end;     // nullable: [dW1 | dW3 | dW2] of the end weights
+  float *dq, *dk, *dv, *dlr, *dW0;
+  uint8_t* ws;
+  DevStatus st;
+};
+LactBwdWorkspace lact_bwd_layout(const LactLaunch& f);
+int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream);
 
 // Fused key pass + chunk gradient (head dim 128): partial sums per token group.
 struct KeyGradLaunch {

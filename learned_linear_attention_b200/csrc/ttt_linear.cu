@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(SIMT_THREADS)
     ttt_linear_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                            const Tin* __restrict__ v, const float* __restrict__ lr,
                            float* __restrict__ S, Tout* __restrict__ out, int N, int dk, int dv,
-                           int C, int include_diag, const float* __restrict__ out_scale,
+                           int C, int include_diag, int bidir, const float* __restrict__ out_scale,
                            float out_mul) {
   extern __shared__ float sm[];
   float* Ss = sm;                       // [dk][dv]
@@ -57,6 +57,26 @@ __global__ void __launch_bounds__(SIMT_THREADS)
   for (int i = threadIdx.x; i < dk * dv; i += blockDim.x) Ss[i] = Sg[i];
   __syncthreads();
 
+  // Bidirectional order: every token's update first (S += K^T diag(eta) V
+  // chunk by chunk), then the reads below with the final S and no P term.
+  for (int t0 = 0; bidir && t0 < N; t0 += C) {
+    const int Cc = min(C, N - t0);
+    for (int i = threadIdx.x; i < Cc * dk; i += blockDim.x)
+      Ks[i] = load_in(k, qk_base + (size_t)t0 * dk + i);
+    for (int i = threadIdx.x; i < Cc * dv; i += blockDim.x) {
+      const int t = i / dv;
+      Vs[i] = lr[(size_t)bh * N + t0 + t] * load_in(v, v_base + (size_t)t0 * dv + i);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
+      const int r = e / dv, c = e % dv;
+      float acc = Ss[e];
+      for (int j = 0; j < Cc; ++j) acc = fmaf(Ks[j * dk + r], Vs[j * dv + c], acc);
+      Ss[e] = acc;
+    }
+    __syncthreads();
+  }
+
   for (int t0 = 0; t0 < N; t0 += C) {
     const int Cc = min(C, N - t0);
     for (int i = threadIdx.x; i < Cc * dk; i += blockDim.x) {
@@ -68,11 +88,12 @@ __global__ void __launch_bounds__(SIMT_THREADS)
       Vs[i] = lr[(size_t)bh * N + t0 + t] * load_in(v, v_base + (size_t)t0 * dv + i);
     }
     __syncthreads();
-    // P[i][j] = q_i . k_j for j <= i (j < i without the diagonal)
+    // P[i][j] = q_i . k_j for j <= i (j < i without the diagonal); no
+    // within-chunk term in bidirectional order (S already holds every update)
     for (int e = threadIdx.x; e < Cc * Cc; e += blockDim.x) {
       const int i = e / Cc, j = e % Cc;
       float acc = 0.f;
-      if (j < i || (include_diag && j == i)) {
+      if (!bidir && (j < i || (include_diag && j == i))) {
         for (int r = 0; r < dk; ++r) acc = fmaf(Qs[i * dk + r], Ks[j * dk + r], acc);
       }
       Ps[i * SIMT_MAXC + j] = acc;
@@ -89,7 +110,7 @@ __global__ void __launch_bounds__(SIMT_THREADS)
     }
     __syncthreads();
     // S += K^T diag(eta) V
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
+    for (int e = threadIdx.x; !bidir && e < dk * dv; e += blockDim.x) {
       const int r = e / dv, c = e % dv;
       float acc = Ss[e];
       for (int j = 0; j < Cc; ++j) acc = fmaf(Ks[j * dk + r], Vs[j * dv + c], acc);
@@ -118,7 +139,7 @@ int launch_ttt_linear_simt(const LinearLaunch& L, cudaStream_t stream) {
     prof_before(K_LIN_SIMT, stream);                                                         \
     kfn<<<grid, block, smem, stream>>>((const TI*)L.q, (const TI*)L.k, (const TI*)L.v, L.lr, \
                                        L.S, (TO*)L.out, L.N, L.dk, L.dv, C, L.include_diag,   \
-                                       L.out_scale, L.out_mul);                               \
+                                       L.bidir, L.out_scale, L.out_mul);                      \
     prof_after(K_LIN_SIMT, stream);                                                          \
   } while (0)
   if (L.in_bf16) {
@@ -173,6 +194,11 @@ struct LinUmmaArgs {
   const float* seg_state;   // [BH][1 + (P - 1) R][64][64]: S0, then the units' increments
   const float* out_scale;   // nullable: output row t is multiplied by out_mul * out_scale[bh][t]
   float out_mul;
+  // Reads only: out = Q S with S fixed (the bidirectional order, after the
+  // state pass has summed every update into S).  Only Q is loaded, there is
+  // no masked term and no state update, every segment starts from S and
+  // none writes it back.
+  int read_only;
 };
 
 __global__ void __launch_bounds__(lin::THREADS, 1)
@@ -232,10 +258,12 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
         const int s = i % STAGES;
         if (i >= STAGES && !W.wait(&empty[s], ((i / STAGES) - 1) & 1, 1)) break;
         uint8_t* st = smem + OFF_STAGE + s * STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+        mbar_arrive_expect_tx(&full[s], a.read_only ? TILE_BYTES : STAGE_BYTES);
         tma_load_3d(st, &mapQ, &full[s], 0, (t_first + i) * T, bh);
-        tma_load_3d(st + TILE_BYTES, &mapK, &full[s], 0, (t_first + i) * T, bh);
-        tma_load_3d(st + 2 * TILE_BYTES, &mapV, &full[s], 0, (t_first + i) * T, bh);
+        if (!a.read_only) {
+          tma_load_3d(st + TILE_BYTES, &mapK, &full[s], 0, (t_first + i) * T, bh);
+          tma_load_3d(st + 2 * TILE_BYTES, &mapV, &full[s], 0, (t_first + i) * T, bh);
+        }
         issued = i + 1;
       }
       if (W.aborted()) {  // drain the copies still in flight into our smem
@@ -266,11 +294,13 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
         tc_fence_after();
         const int s = i % STAGES, pb = i & 1;
         const uint64_t dq = sdesc_add(dq0, s * STAGE_BYTES), dk = sdesc_add(dq, TILE_BYTES);
+        if (!a.read_only) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + (pb ? TM_P1 : TM_P0), sdesc_add(dq, kk * 32), sdesc_add(dk, kk * 32), id_qk,
-                   kk > 0);
-        mma_commit(&pfull[pb]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + (pb ? TM_P1 : TM_P0), sdesc_add(dq, kk * 32), sdesc_add(dk, kk * 32),
+                     id_qk, kk > 0);
+        }
+        mma_commit(&pfull[pb]);   // read-only: only tells the epilogue the tile is in
       };
       auto issue_o = [&](int i) {
         tc_fence_after();
@@ -281,18 +311,23 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
         // O alternates between two TMEM buffers so the epilogue can store the
         // previous tile's O while this tile's products run.
         const uint32_t tm_o = (i & 1) ? TM_O1 : TM_O0;
+        if (!a.read_only) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + tm_o, sdesc_add(dpt, (kk >> 2) * TILE_BYTES + (kk & 3) * 32),
-                   sdesc_add(dev_mn, kk * 2048), id_o, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16(tmem + tm_o, sdesc_add(dpt, (kk >> 2) * TILE_BYTES + (kk & 3) * 32),
+                     sdesc_add(dev_mn, kk * 2048), id_o, kk > 0);
+        }
         // O += Q S_{prev}
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + tm_o, sdesc_add(dq, kk * 32), sdesc_add(dsb, kk * 2048), id_o, 1);
+          mma_bf16(tmem + tm_o, sdesc_add(dq, kk * 32), sdesc_add(dsb, kk * 2048), id_o,
+                   (a.read_only && kk == 0) ? 0u : 1u);
         // S += K^T (eta V)   (M = 64: rows live in lanes 0-15 of each quadrant)
+        if (!a.read_only) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + TM_S, sdesc_add(dk, kk * 2048), sdesc_add(dev_mn, kk * 2048), id_s, 1);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16(tmem + TM_S, sdesc_add(dk, kk * 2048), sdesc_add(dev_mn, kk * 2048), id_s, 1);
+        }
         mma_commit(ofull);
         mma_commit(&empty[s]);
       };
@@ -344,7 +379,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     const int srow = q4 * 16 + lane;
     {
       float vals[32];
-      if (a.P == 1) {
+      if (a.P == 1 || a.read_only) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) vals[j] = s_owner ? Sg[srow * D + hf * 32 + j] : 0.f;
       } else {   // S0 + the increments of the earlier segments' units, in order
@@ -391,7 +426,20 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       }
     };
     bool ok = true;
-    for (int i = 0; i < n_tiles; ++i) {
+    for (int i = 0; a.read_only && i < n_tiles; ++i) {
+      // reads only: the operands (Q in the stage, S in shared memory) are in
+      // place; keep the O buffers' order and store the previous tile's O
+      if (!W.wait(&pfull[i & 1], (i >> 1) & 1, 5)) { ok = false; break; }
+      if (i > 0 && !W.wait(ofull, (i - 1) & 1, 6)) { ok = false; break; }
+      tc_fence_after();
+      // the bf16 S operand this thread stored before the loop must be visible
+      // to the tensor core (async proxy) before the first product reads it
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(ops);
+      if (i > 0) store_out(i - 1);
+    }
+    for (int i = 0; !a.read_only && i < n_tiles; ++i) {
       const int s = i % STAGES, pb = i & 1;
       if (!W.wait(&pfull[pb], (i >> 1) & 1, 5)) { ok = false; break; }
       tc_fence_after();
@@ -469,7 +517,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       store_out(n_tiles - 1);
       float sv[32];
       tmem_ld32(tmem + lane_base + TM_S + hf * 32, sv);
-      if (s_owner && seg == a.P - 1) {
+      if (s_owner && seg == a.P - 1 && !a.read_only) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) Sg[srow * D + hf * 32 + j] = sv[j];
       }
@@ -676,6 +724,17 @@ LinearPlan ttt_linear_plan(int BH, int N, int sms) {
   return pl;
 }
 
+// SMs of the current device
+static int num_sms_current() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 148;
+  }
+  return n;
+}
+
 int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   const uint64_t BH = (uint64_t)L.B * L.H;
@@ -689,7 +748,19 @@ int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream) {
     pl.seg_tiles = (L.N + 127) / 128;
   }
   LinUmmaArgs a{L.lr, L.S, L.out, L.N, L.include_diag, L.out_bf16, L.st,
-                pl.P, pl.R, pl.seg_tiles, L.seg_state, L.out_scale, L.out_mul};
+                pl.P, pl.R, pl.seg_tiles, L.seg_state, L.out_scale, L.out_mul, 0};
+  if (L.bidir) {
+    // every update first: S <- S + sum over all tokens (state pass), then
+    // reads only, in segments that all start from that S
+    if (launch_ttt_linear_state_sum(L, num_sms_current(), stream) != 0) return -1;
+    const int total = (L.N + 127) / 128;
+    a.read_only = 1;
+    a.P = std::max(1, std::min(total, num_sms_current() / (int)BH));
+    a.seg_tiles = (total + a.P - 1) / a.P;
+    a.P = (total + a.seg_tiles - 1) / a.seg_tiles;
+    a.R = 1;
+    pl.P = 1;   // no segment pre-pass
+  }
   if (pl.P > 1) {
     SegStateArgs sa{L.lr, L.S, L.seg_state, L.N, (pl.P - 1) * pl.R, pl.R, pl.seg_tiles, pl.unit_tiles, L.st};
     static std::atomic<uint64_t> ss_attr{0};
@@ -702,7 +773,7 @@ int launch_ttt_linear_umma(const LinearLaunch& L, cudaStream_t stream) {
   static std::atomic<uint64_t> attr{0};
   if (allow_dynamic_smem(ttt_linear_umma_kernel, (int)lin::SMEM_BYTES, attr)) return -1;
   prof_before(K_LIN_UMMA, stream);
-  ttt_linear_umma_kernel<<<dim3((unsigned)(BH * pl.P)), dim3(lin::THREADS), lin::SMEM_BYTES, stream>>>(
+  ttt_linear_umma_kernel<<<dim3((unsigned)(BH * a.P)), dim3(lin::THREADS), lin::SMEM_BYTES, stream>>>(
       mq, mk, mv, a);
   prof_after(K_LIN_UMMA, stream);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;

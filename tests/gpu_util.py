@@ -11,8 +11,9 @@ import learned_linear_attention_b200 as T
 def to_dev(tt, device="cuda"):
     """TokenTensor -> device tensor with the exact values (bf16 bits or f32)."""
     if tt.dtype == "bf16":
-        return torch.from_numpy(tt.bits.view(np.int16)).view(torch.bfloat16).to(device)
-    return torch.from_numpy(tt.values).to(device)
+        bits = np.ascontiguousarray(tt.bits).view(np.int16)
+        return torch.from_numpy(bits).view(torch.bfloat16).to(device).contiguous()
+    return torch.from_numpy(np.ascontiguousarray(tt.values)).to(device).contiguous()
 
 
 def rel_err(a, ref):
@@ -22,14 +23,21 @@ def rel_err(a, ref):
     return float(np.abs(a - ref).max() / max(np.abs(ref).max(), 1e-300))
 
 
+def elem_err(a, ref):
+    """Elementwise relative error, max_i |a_i - ref_i| / (|ref_i| + 1e-3 max|ref|)."""
+    a = np.asarray(a, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float((np.abs(a - ref) / (np.abs(ref) + 1e-3 * np.abs(ref).max())).max())
+
+
 def run_linear(x, include_diag=True, out_dtype="f32", S0=None, chunk=None, stream=None,
-               ws_bytes=None):
+               ws_bytes=None, order="causal"):
     B, H, N, dk = x.q.values.shape
     dv = x.v.values.shape[-1]
     desc = T.make_linear_desc(B, H, N, dk, dv, chunk or x.chunk, include_diag,
-                              in_dtype=x.q.dtype, out_dtype=out_dtype)
+                              in_dtype=x.q.dtype, out_dtype=out_dtype, order=order)
     q, k, v = to_dev(x.q), to_dev(x.k), to_dev(x.v)
-    lr = torch.from_numpy(x.lr).cuda()
+    lr = torch.from_numpy(np.ascontiguousarray(x.lr)).cuda()
     S = torch.zeros(B, H, dk, dv, dtype=torch.float32, device="cuda")
     if S0 is not None:
         S.copy_(torch.from_numpy(np.asarray(S0, dtype=np.float32)))

@@ -93,6 +93,28 @@ def test_linear_validation_before_launch(lib):
     # N = 0 is a valid empty call and launches nothing
     assert _call_linear_fwd(T.make_linear_desc(1, 2, 0, 64, 64, 16)) == T.TTT_OK
     assert T.ttt_linear_workspace_bytes(good) == T.TTT_STATUS_BYTES
+    d = T.make_linear_desc(1, 2, 8, 64, 64, 16)
+    d.order = 5
+    assert _call_linear_fwd(d) == T.TTT_ERR_ARG
+
+
+def test_linear_bidirectional_desc(lib):
+    """order sits between chunk and include_diag, as the boundary table has it;
+    the bidirectional tensor-core path sizes room for the state pass's
+    partial sums (a CUDA-core fallback runs with less), and the backward pass
+    is causal only."""
+    d = T.make_linear_desc(1, 2, 8, 64, 64, 16, order="bidirectional")
+    assert d.order == T.TTT_BIDIRECTIONAL
+    assert [f[0] for f in T.ttt_linear_desc._fields_][6] == "order"
+    assert _call_linear_fwd(T.make_linear_desc(1, 2, 0, 64, 64, 16, order="bidirectional")) == \
+        T.TTT_OK
+    assert T.ttt_linear_workspace_bytes(d) > T.TTT_STATUS_BYTES
+    f32 = T.make_linear_desc(1, 2, 8, 32, 32, 16, in_dtype="f32", order="bidirectional")
+    assert T.ttt_linear_workspace_bytes(f32) == T.TTT_STATUS_BYTES
+    assert _call_linear_bwd(d) == T.TTT_ERR_UNSUPPORTED
+    n = ctypes.c_size_t(0)
+    assert T.load().ttt_linear_bwd_workspace_bytes(ctypes.byref(d), ctypes.byref(n)) == \
+        T.TTT_ERR_UNSUPPORTED
 
 
 def _call_linear_bwd(desc, ws_bytes=1 << 40, **ptrs):
@@ -219,3 +241,28 @@ def test_window_attention_validation_before_launch(lib):
     lact = T.make_lact_desc(1, 2, 64, 128, 256, 32)
     assert T.load().lact_layer_fwd(ctypes.byref(lact), 0, ctypes.c_float(0), 16, 16, 16, 16, 16,
                                    16, 16, 1 << 40, None) == T.TTT_ERR_ARG
+
+
+def test_context_parallel_pieces_validate_before_launch(lib):
+    """lact_chunk_grad / lact_apply_grad / lact_read reject bad ranges, null
+    buffers and short workspaces on the host, before anything is enqueued."""
+    L = T.load()
+    d = T.make_lact_desc(1, 2, 512, 128, 256, 256)
+    assert T.lact_grad_bytes(d) == 3 * 2 * 128 * 256 * 4
+    ws = T.lact_workspace_bytes(d)
+    g = lambda t0, n, G=16, w=ws: L.lact_chunk_grad(ctypes.byref(d), t0, n, 16, 16, 16, 16, G, 16,  # noqa: E731,E501
+                                                    w, None)
+    assert g(500, 20) == T.TTT_ERR_SHAPE           # past N_in
+    assert g(0, 300) == T.TTT_ERR_SHAPE            # more than one chunk
+    assert g(-1, 10) == T.TTT_ERR_SHAPE
+    assert g(0, 10, G=0) == T.TTT_ERR_ARG
+    assert g(0, 10, w=64) == T.TTT_ERR_WORKSPACE
+    assert g(0, 10, G=24) == T.TTT_ERR_ALIGN
+    assert L.lact_apply_grad(ctypes.byref(d), 0, 16, 16, ws, None) == T.TTT_ERR_ARG
+    assert L.lact_apply_grad(ctypes.byref(d), 16, 16, 16, 64, None) == T.TTT_ERR_WORKSPACE
+    r = lambda t0, n: L.lact_read(ctypes.byref(d), t0, n, 16, 16, 16, 16, ws, None)  # noqa: E731
+    assert r(400, 200) == T.TTT_ERR_SHAPE
+    assert r(0, 0) == T.TTT_OK                     # nothing to read
+    bi = T.make_lact_desc(1, 2, 512, 128, 256, 256, N_q=100, order="bidirectional")
+    assert L.lact_read(ctypes.byref(bi), 50, 60, 16, 16, 16, 16, T.lact_workspace_bytes(bi),
+                       None) == T.TTT_ERR_SHAPE

@@ -158,3 +158,82 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
     x = make_linear_inputs(1, 1, 64, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=18)
     out, _ = run_linear(x)
     assert rel_err(out, _oracle(x)[0]) <= TOL_BF16
+
+
+# ---------------------------------------------------------------- bidirectional order
+# Every token writes, then every query reads the final state: linear attention
+# with no causal mask.
+
+def _oracle_bi(x, S0=None):
+    return ttt_linear_recurrent(x.q.values, x.k.values, x.v.values, x.lr, S0,
+                                order="bidirectional")
+
+
+def test_bidirectional_f32_n256_workload_shape(cuda_device):
+    """The fp32 configuration's shapes (B1 H2 N256 d32, chunk 16) in
+    bidirectional order, on the CUDA-core kernel."""
+    x = make_workload("ttt_linear_f32_n256")
+    out, S = run_linear(x, order="bidirectional")
+    ref, Sref = _oracle_bi(x)
+    assert rel_err(out, ref) <= TOL_F32
+    assert rel_err(S, Sref) <= TOL_F32
+
+
+def test_bidirectional_f32_ragged_with_initial_state(cuda_device):
+    x = make_linear_inputs(2, 3, 77, 24, 40, chunk=9, dtype="f32", lr_kind="0.1sig", cfg=21,
+                           with_S0=True)
+    out, S = run_linear(x, S0=x.S0, order="bidirectional")
+    ref, Sref = _oracle_bi(x, x.S0)
+    assert rel_err(out, ref) <= TOL_F32
+    assert rel_err(S, Sref) <= TOL_F32
+
+
+@pytest.mark.parametrize("N", [1, 128, 300, 5000])
+def test_bidirectional_bf16_tensor_core(cuda_device, N):
+    """State pass over the whole sequence, then reads only, in segments that
+    all start from the final state; ragged last tile for N = 300, 5000."""
+    x = make_linear_inputs(2, 3, N, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=22,
+                           with_S0=True)
+    out, S = run_linear(x, S0=x.S0, order="bidirectional")
+    ref, Sref = _oracle_bi(x, x.S0)
+    assert not np.isnan(out).any()
+    assert rel_err(out, ref) <= TOL_BF16
+    assert rel_err(S, Sref) <= TOL_BF16
+
+
+def test_bidirectional_bf16_small_workspace_runs_on_cuda_cores(cuda_device):
+    x = make_linear_inputs(1, 2, 700, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=23,
+                           with_S0=True)
+    out, S = run_linear(x, S0=x.S0, order="bidirectional", ws_bytes=T.TTT_STATUS_BYTES)
+    ref, Sref = _oracle_bi(x, x.S0)
+    assert rel_err(out, ref) <= TOL_BF16
+    assert rel_err(S, Sref) <= TOL_BF16
+    o_tc, S_tc = run_linear(x, S0=x.S0, order="bidirectional")
+    assert rel_err(o_tc, out) <= 1e-2
+
+
+def test_bidirectional_bf16_other_dims_and_bf16_out(cuda_device):
+    x = make_linear_inputs(1, 2, 150, 32, 48, chunk=16, dtype="bf16", lr_kind="sig-2", cfg=24)
+    out, S = run_linear(x, order="bidirectional", out_dtype="bf16")
+    ref, Sref = _oracle_bi(x)
+    assert rel_err(out, ref) <= TOL_BF16 and rel_err(S, Sref) <= TOL_BF16
+    y = make_linear_inputs(1, 2, 400, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=25)
+    out, _ = run_linear(y, order="bidirectional", out_dtype="bf16")
+    assert rel_err(out, _oracle_bi(y)[0]) <= TOL_BF16
+
+
+def test_bidirectional_output_is_permutation_equivariant(cuda_device):
+    """Permuting the tokens permutes the outputs and leaves the state (up to
+    fp32 summation order), as the unmasked form requires."""
+    x = make_linear_inputs(1, 2, 384, 64, 64, chunk=64, dtype="bf16", lr_kind="sig-2", cfg=26)
+    o, S = run_linear(x, order="bidirectional")
+    import copy
+    perm = np.random.default_rng(0).permutation(384)
+    y = copy.deepcopy(x)
+    for tt in (y.q, y.k, y.v):
+        tt.values = np.ascontiguousarray(tt.values[:, :, perm])
+        tt.bits = np.ascontiguousarray(tt.bits[:, :, perm])
+    y.lr = np.ascontiguousarray(x.lr[:, :, perm])
+    o_p, S_p = run_linear(y, order="bidirectional")
+    assert rel_err(o_p, o[:, :, perm]) <= 1e-2
+    assert rel_err(S_p, S) <= 1e-5
