@@ -21,7 +21,13 @@
 //     whose GPU work overlaps -- on different streams or host threads -- race
 //     on it and must not be issued that way;
 //   * the first call on each device looks up the array's device address
-//     (cudaGetSymbolAddress, with that device current) and caches it.
+//     (cudaGetSymbolAddress, with that device current) and caches it; a
+//     cudaDeviceReset of that device invalidates the cached address, so the
+//     entry point must not be used after one;
+//   * the stream must belong to the current device (checked: the address
+//     is that device's copy of the array);
+//   * a bounded in-kernel wait that runs out records its code in the
+//     array's status block, which lact_noalloc_check_status() reads.
 #include <mutex>
 
 #include "../../include/ttt.h"
@@ -52,19 +58,42 @@ void* scratch_on_current_device() {
   return g_scratch_addr[dev];
 }
 
+// The stream's device must be the current one: the scratch address looked up
+// for the current device names another GPU's copy of the array otherwise.
+int check_stream_device(void* stream) {
+  int cur = 0, sdev = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return TTT_ERR_CUDA;
+  if (stream == nullptr) return TTT_OK;   // legacy default stream: the current device's
+  if (cudaStreamGetDevice(reinterpret_cast<cudaStream_t>(stream), &sdev) != cudaSuccess) {
+    cudaGetLastError();
+    return TTT_ERR_ARG;
+  }
+  return sdev == cur ? TTT_OK : TTT_ERR_ARG;
+}
+
 }  // namespace
 
 extern "C" int lact_chunk_fwd_noalloc(const lact_desc* desc, const void* q, const void* k,
                                       const void* v, const float* lr, void* state, void* out,
                                       void* stream) {
   size_t need = 0;
-  const int e = lact_workspace_bytes_min(desc, &need);
+  int e = lact_workspace_bytes_min(desc, &need);
   if (e != TTT_OK) return e;
   if (need > kNoAllocScratchBytes) return TTT_ERR_WORKSPACE;
+  e = check_stream_device(stream);
+  if (e != TTT_OK) return e;
   void* scratch = scratch_on_current_device();
   if (scratch == nullptr) return TTT_ERR_CUDA;
   if (cudaMemsetAsync(scratch, 0, TTT_STATUS_BYTES, reinterpret_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return TTT_ERR_CUDA;
   return lact_chunk_fwd(desc, q, k, v, lr, state, out, scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" int lact_noalloc_check_status(void* stream) {
+  const int e = check_stream_device(stream);
+  if (e != TTT_OK) return e;
+  void* scratch = scratch_on_current_device();
+  if (scratch == nullptr) return TTT_ERR_CUDA;
+  return ttt_check_device_status(scratch, stream);
 }
