@@ -379,6 +379,7 @@ struct RowArgs {
   DevStatus st;
   int nbuf;                 // cast: copies written, buf_stride elements apart
   size_t buf_stride;
+  float* rownorm;           // nullable: norm of each updated row before normalisation
 };
 
 constexpr int ROW_MAXV = 32;  // columns per lane (cols <= 1024)
@@ -519,7 +520,11 @@ __global__ void __launch_bounds__(UPD_ROWS_PER_BLOCK * 32) lact_update_kernel(Ro
       }
     }
     float scale = 1.f;
-    if (a.normalize) scale = 1.f / fmaxf(sqrtf(warp_sum(ss)), a.norm_eps);
+    if (a.normalize) {
+      const float nrm = sqrtf(warp_sum(ss));
+      scale = 1.f / fmaxf(nrm, a.norm_eps);
+      if (a.rownorm != nullptr && lane == 0) a.rownorm[gw0 + q] = nrm;
+    }
     uint2* Br = reinterpret_cast<uint2*>(a.Wb[mat[q]] + off[q]) + lane;
     uint2* Lr = a.Wlo[mat[q]] != nullptr ? reinterpret_cast<uint2*>(a.Wlo[mat[q]] + off[q]) + lane : nullptr;
 #pragma unroll
@@ -633,7 +638,13 @@ __global__ void __launch_bounds__(UPB_THREADS) lact_update_bulk_kernel(RowArgs a
       ss += w[i].x * w[i].x + w[i].y * w[i].y + w[i].z * w[i].z + w[i].w * w[i].w;
     }
     float scale = 1.f;
-    if (a.normalize) scale = 1.f / fmaxf(sqrtf(warp_sum(ss)), a.norm_eps);
+    if (a.normalize) {
+      const float nrm = sqrtf(warp_sum(ss));
+      scale = 1.f / fmaxf(nrm, a.norm_eps);
+      if (a.rownorm != nullptr && lane == 0)
+        a.rownorm[(size_t)bh * (2 * a.dh + a.d) + (mat == 0 ? 0 : mat == 1 ? a.dh : 2 * a.dh) +
+                  row0 + r] = nrm;
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if (i >= nch) break;
@@ -690,10 +701,12 @@ struct NsPrepArgs {
   float* X32;              // [3*BH][r][c]
   __nv_bfloat16* Xb;       // [3*BH][r][c]
   __nv_bfloat16* Xlo;      // residual (split operands; nullable)
+  unsigned* counter;       // phase counter of the fused Newton-Schulz kernel (zeroed here)
 };
 __global__ void ns_prep_kernel(NsPrepArgs a) {
   pdl_wait();
   pdl_launch_dependents();
+  if (a.counter != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *a.counter = 0u;
   const int mb = blockIdx.y;                 // mat * BH + bh
   const int mat = mb / a.BH, bh = mb % a.BH;
   const int rows = mat < 2 ? a.dh : a.d, cols = mat < 2 ? a.d : a.dh;
@@ -898,6 +911,7 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
     w.nsa32 = o; o = align256(o + 3 * BH * r * r * 4);
     w.nsab = o; o = align256(o + 3 * BH * r * r * 2);
     w.nsbb = o; o = align256(o + 3 * BH * r * r * 2);
+    w.nsctr = o; o = align256(o + 256);
   }
   w.w1lo = w.w3lo = w.w2lo = w.d13lo = w.gmlo = w.aqlo = w.nsxlo = w.nsalo = w.nsblo = o;
   if (split) {
@@ -947,6 +961,19 @@ static GemmArgs gemm_defaults(const DevStatus& st) {
   return g;
 }
 
+// The batched GEMM for other files of the library (the LaCT backward pass):
+// operand majorness by variant, 128-wide N tiles, four stages.
+int gemm_launch(int variant, const GemmMaps& maps, const GemmArgs& g, cudaStream_t stream,
+                int kind) {
+  switch (variant) {
+    case GEMM_AK_BK: return run_gemm<128, false, false, 4>(maps, g, stream, kind);
+    case GEMM_AK_BMN: return run_gemm<128, false, true, 4>(maps, g, stream, kind);
+    case GEMM_AMN_BMN: return run_gemm<128, true, true, 4>(maps, g, stream, kind);
+    default: return -1;
+  }
+}
+GemmArgs gemm_args_default(const DevStatus& st) { return gemm_defaults(st); }
+
 #define TTT_TRY(...)                      \
   do {                                    \
     if ((__VA_ARGS__) != 0) return -1;    \
@@ -972,6 +999,26 @@ __global__ void w2_prefix_kernel(float* W2, const float* part, __nv_bfloat16* Mb
       m.x -= p.x; m.y -= p.y; m.z -= p.z; m.w -= p.w;
     }
     *reinterpret_cast<float4*>(W2 + e) = m;
+  }
+}
+
+// Chunk gradient of a token range: G[m] = sum over the partial-sum slots of
+// matrix m, in slot order (the update kernels sum them the same way).
+__global__ void lact_grad_sum_kernel_strided(const float* __restrict__ part, float* __restrict__ G,
+                                             size_t mat_elems, int slots, int used) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t n4 = mat_elems / 4;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < 3 * n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t m = i / n4, e = (i % n4) * 4;
+    const float* p = part + m * (size_t)slots * mat_elems + e;
+    float4 acc = __ldcg(reinterpret_cast<const float4*>(p));
+    for (int sp = 1; sp < used; ++sp) {
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(p + (size_t)sp * mat_elems));
+      acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+    }
+    *reinterpret_cast<float4*>(G + m * mat_elems + e) = acc;
   }
 }
 
@@ -1057,10 +1104,12 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // never updated (update_mask): then every buffer must hold it
   ra.nbuf = (L.update_mask & 7) == 7 ? 1 : nbuf;
   ra.buf_stride = wsz;
-  prof_before(K_LACT_CAST, stream);
-  if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
-    return -1;
-  prof_after(K_LACT_CAST, stream);
+  if (L.mode != LACT_APPLY) {   // the update of an APPLY call writes its own copies
+    prof_before(K_LACT_CAST, stream);
+    if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
+      return -1;
+    prof_after(K_LACT_CAST, stream);
+  }
   ra.nbuf = 1;
   TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
 
@@ -1085,14 +1134,18 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     return make_tmap_bf16_3d(m, p, dh, rows, BH, (uint64_t)dh * 2, (uint64_t)w.cmax * dh * 2, 64,
                              box_rows);
   };
+  // which token tensors this call reads (the context-parallel pieces read a
+  // subset and may leave the others null)
+  const bool uses_kv = L.N_in > 0 && (L.mode == LACT_FULL || L.mode == LACT_GRAD);
+  const bool uses_q = q_rows > 0 && (L.mode == LACT_FULL || L.mode == LACT_READ);
   KeyPassMaps km{};
-  if (L.N_in > 0) {
+  if (uses_kv) {
     TTT_TRY(tok_map(&km.k, L.k, L.N_in, 128));
     TTT_TRY(tok_map(&km.v, L.v, L.N_in, 128));
   }
-  if (q_rows > 0) TTT_TRY(tok_map(&km.q, L.q, q_rows, 128));
+  if (uses_q) TTT_TRY(tok_map(&km.q, L.q, q_rows, 128));
   else km.q = km.k;
-  if (L.N_in == 0) { km.k = km.q; km.v = km.q; }
+  if (!uses_kv) { km.k = km.q; km.v = km.q; }
   KeyPassMaps kmb[3] = {km, km, km};
   CUtensorMap mw2k[3], mw2klo[3];
   for (int b = 0; b < nbuf; ++b) {
@@ -1113,7 +1166,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   int cur = 0;   // buffer holding the chunk-start weights
   auto nxt = [&](int b) { return b + 1 == nbuf ? 0 : b + 1; };   // buffer its update writes
   CUtensorMap mk_mn{}, mv_mn{};   // token tensors as MN-major operands
-  if (L.N_in > 0) {
+  if (uses_kv) {
     TTT_TRY(tok_map(&mk_mn, L.k, L.N_in, 64));
     TTT_TRY(tok_map(&mv_mn, L.v, L.N_in, 64));
   }
@@ -1183,7 +1236,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     return make_tmap_bf16_3d(m, p, 2 * dh, rows, BH, (uint64_t)dh * 4, (uint64_t)w.cmax * dh * 4,
                              64, 64);
   };
-  auto gradients = [&](int t0, int C, cudaStream_t* mstream) -> int {
+  auto gradients = [&](int t0, int C, cudaStream_t* mstream, bool partials_only) -> int {
     CUtensorMap md, mdl, mg, mgl;
     TTT_TRY(d13_map(&md, D13, C));
     TTT_TRY(inter_map(&mg, Gm, C, 64));
@@ -1193,7 +1246,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     }
     const int ksteps_total = (C + 63) / 64;
     const int np = split ? 2 : 1;
-    if (fused_update) {
+    if (fused_update && !partials_only) {
       GemmArgs g = gemm_defaults(L.st);
       g.batch = BH; g.splits = 1; g.k_steps = ksteps_total; g.npairs = np; g.epi = 1;
       g.mom_beta = L.beta; g.norm_eps = L.norm_eps; g.normalize = L.normalize_rows;
@@ -1284,11 +1337,25 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     pa.BH = BH; pa.d = d; pa.dh = dh; pa.r = r; pa.c = c; pa.eps = L.ns_eps;
     pa.M[0] = M1; pa.M[1] = M3; pa.M[2] = M2; pa.rowss = ra.rowss; pa.X32 = X32;
     pa.Xb = Xb[0]; pa.Xlo = Xl[0];
+    unsigned* ctr = reinterpret_cast<unsigned*>(ws + w.nsctr);
+    pa.counter = ctr;
     prof_before(K_NS_PREP, stream);
     if (launch_pdl(ns_prep_kernel, dim3(r, nb), dim3(256), 0, stream, pa) != cudaSuccess)
       return -1;
     prof_after(K_NS_PREP, stream);
     TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    bool fused_ns = L.ns_steps > 0;
+    if (fused_ns) {   // every Newton-Schulz step in one cooperative launch
+      NsFusedLaunch nl{};
+      nl.r = r; nl.c = c; nl.nb = nb; nl.steps = L.ns_steps; nl.split = split ? 1 : 0;
+      nl.coef_a = L.ns_a; nl.coef_b = L.ns_b; nl.coef_c = L.ns_c;
+      nl.X32 = X32;
+      nl.Xb[0] = Xb[0]; nl.Xb[1] = Xb[1]; nl.Xl[0] = Xl[0]; nl.Xl[1] = Xl[1];
+      nl.A32 = A32; nl.Ab = Ab; nl.Al = Al; nl.Bb = Bb; nl.Bl = Bl;
+      nl.counter = ctr;
+      nl.st = L.st;
+      TTT_TRY(launch_ns_fused(nl, stream));
+    }
     auto sq_map = [&](CUtensorMap* m, const void* p) {
       return make_tmap_bf16_3d(m, p, r, r, nb, (uint64_t)r * 2, (uint64_t)r * r * 2, 64, 128);
     };
@@ -1317,7 +1384,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
         g.npairs = 3;
       }
     };
-    for (int it = 0; it < L.ns_steps; ++it) {
+    for (int it = 0; !fused_ns && it < L.ns_steps; ++it) {
       const int cur = it & 1;
       GemmMaps m{};
       // A = X X^T  (fp32 + bf16 hi/lo)
@@ -1375,6 +1442,57 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
         return -1;
     return 0;
   };
+  // ------------------------------------------------------------ context-parallel pieces
+  if (L.mode == LACT_APPLY) {
+    // the optimizer step and row normalisation with the caller's summed chunk
+    // gradient, which takes the place of the partial sums (one slot)
+    ra.part[0] = L.G;
+    ra.part[1] = L.G + mat_elems;
+    ra.part[2] = L.G + 2 * mat_elems;
+    ra.splits = 1;
+    ra.rownorm = L.rownorm_out;
+    set_out_buf(nxt(cur));
+    return L.opt == 2 ? muon() : row_update(stream);
+  }
+  if (L.mode == LACT_READ) {   // queries [t0, t0 + n) read the current weights
+    if (L.n <= 0) return 0;
+    TTT_TRY(key_pass(L.t0, L.n, 0, (L.n + 127) / 128));
+    return read_out(L.t0, L.n, stream, Aq);
+  }
+  if (L.mode == LACT_GRAD) {   // gradient sum of tokens [t0, t0 + n), no update
+    int splits = 1;
+    if (L.n > 0 && w.keygrad) {
+      KeyGradLaunch kgl{};
+      kgl.BH = BH; kgl.N_in = L.N_in; kgl.C = L.n; kgl.t0 = L.t0; kgl.dh = dh;
+      kgl.groups = keygrad_groups(BH, dh, L.n, w.splits);
+      kgl.k = L.k; kgl.v = L.v; kgl.lr = L.lr; kgl.q = nullptr;
+      kgl.Aq = Aq; kgl.aq_bs = (long long)w.cmax * dh;
+      kgl.w1b = wbuf[cur][0]; kgl.w3b = wbuf[cur][1]; kgl.w2b = wbuf[cur][2];
+      kgl.part[0] = const_cast<float*>(ra.part[0]);
+      kgl.part[1] = const_cast<float*>(ra.part[1]);
+      kgl.part[2] = const_cast<float*>(ra.part[2]);
+      kgl.st = L.st;
+      TTT_TRY(launch_lact_keygrad(kgl, stream));
+      splits = kgl.groups;
+    } else if (L.n > 0) {
+      const int nt = (L.n + 127) / 128;
+      TTT_TRY(key_pass(L.t0, L.n, nt, 0));
+      TTT_TRY(fork());
+      splits = gradients(L.t0, L.n, gstream, /*partials_only=*/true);
+      if (splits < 0) return -1;
+      TTT_TRY(join());
+    } else {   // no tokens: a zero gradient
+      return cudaMemsetAsync(L.G, 0, 3 * mat_elems * sizeof(float), stream) == cudaSuccess ? 0 : -1;
+    }
+    // slot s of matrix m sits at part + (m * w.splits + s) * mat_elems
+    const size_t n4 = 3 * mat_elems / 4;
+    const int blocks = (int)std::min<size_t>((n4 + 255) / 256, 8 * (size_t)num_sms());
+    if (launch_pdl(lact_grad_sum_kernel_strided, dim3(blocks), dim3(256), 0, stream,
+                   (const float*)part, L.G, mat_elems, w.splits, splits) != cudaSuccess)
+      return -1;
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  }
+
   if (w.w2par) {
     // ---- parallel form of the W2-only layer (see lact_uses_w2_parallel)
     const int nch = L.N_in / L.chunk;
@@ -1470,7 +1588,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     TTT_TRY(key_pass(t0, C, nt, L.causal ? nt : 0));
     TTT_TRY(fork());
     if (L.causal) TTT_TRY(read_out(t0, C, rstream, Aq));
-    const int splits = gradients(t0, C, gstream);
+    const int splits = gradients(t0, C, gstream, false);
     if (splits < 0) return -1;
     TTT_TRY(join());
     if (fused_update) {   // the epilogues wrote buffer nxt(cur)

@@ -223,3 +223,41 @@ def test_w2_only_chunk_loop_in_the_minimum_workspace(cuda_device):
     assert rel_err(b, ref) <= TOL, rel_err(b, ref)
     assert rel_err(a, ref) <= TOL, rel_err(a, ref)
     assert rel_err(loop.weights()[2], st.W2) <= TOL
+
+
+# ---------------------------------------------------------------- fused Newton-Schulz
+# The Muon step runs every Newton-Schulz step of a chunk in one cooperative
+# launch with grid-wide barriers between its phases.
+
+@pytest.mark.parametrize("ns_steps", [1, 2, 5])
+def test_muon_fused_newton_schulz_view_synthesis_dims(cuda_device, ns_steps):
+    """d = 384, dh = 768 (the view-synthesis shapes): six 384 x 768 matrices
+    per chunk, three chunks, the last ragged."""
+    x = make_lact_inputs(1, 2, 600, 384, 768, chunk=256, order="bidirectional", Nq=150,
+                         v_norm=True, lr_kind="0.01sig", cfg=43)
+    _check(x, "muon", beta=0.9, ns_steps=ns_steps)
+
+
+def test_muon_fused_newton_schulz_plain_bf16_operands(cuda_device):
+    x = make_lact_inputs(1, 2, 512, 128, 256, chunk=256, order="bidirectional", Nq=128,
+                         v_norm=True, lr_kind="0.01sig", cfg=44)
+    _check(x, "muon", beta=0.9, ns_steps=5, split_operands=False)
+
+
+def test_muon_cuda_graph_replay_matches_eager(cuda_device):
+    """The cooperative Newton-Schulz launch is capturable; replay is bit-exact."""
+    import torch
+    import learned_linear_attention_b200 as T
+    x = make_lact_inputs(1, 2, 512, 128, 256, chunk=256, order="bidirectional", Nq=128,
+                         v_norm=True, lr_kind="0.01sig", cfg=45)
+    run = LaCTRun(x, opt="muon")
+    eager = run.run()
+    W0 = [torch.from_numpy(w).cuda() for w in (x.W1, x.W3, x.W2)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        T.lact_state_init(run.desc, *W0, 0, run.state)
+        T.lact_chunk_fwd(run.desc, run.q, run.k, run.v, run.lr, run.state, run.out, run.ws)
+    run.out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(run.out.cpu().numpy(), eager)
