@@ -1,0 +1,445 @@
+// lact_bwd.cu -- backward pass of the LaCT layer through its chunk loop
+// ("Test-Time Training Done Right" review: the layer is trained end to end,
+// "Lenguaje: calidad y velocidad no son equivalentes" reports its training
+// throughput with GD, momentum and Muon updates).
+//
+// Gradients of  L = sum <dout, out> + sum_m <dW_end[m], W_m(end)>  with
+// respect to q, k, v, lr and the start weights W0 (GD and momentum, causal
+// or bidirectional, with or without row normalisation, any update mask).
+//
+// 1. Forward replay, chunk by chunk, with the layer's own pieces (the chunk
+//    gradient and the update of the context-parallel calls): it keeps every
+//    chunk's start weights W_c and the row norms of the pre-normalisation
+//    update U_c = W_c - (G_c or M_c).
+// 2. Reverse over the chunks, per chunk c with upstream dW = dL/dW_{c+1}:
+//      row step   dU = (dW - w <w, dW>) / |U| (w = W_{c+1} rows; dW / eps
+//                 for a row whose norm was below eps; dU = dW without the
+//                 normalisation); momentum: dM -= dU, R = dM, dM *= beta;
+//                 GD: R = -dU; then dW = dU.  R = dL/dG_c.
+//      chunk gradient VJP at W_c over the chunk's tokens (per token: h1 = W1 k,
+//                 h3 = W3 k, a = silu(h1), s = silu'(h1), g = a h3,
+//                 dy = -lr v, dg = W2^T dy; r1 = R1 k, r3 = R3 k, r2 = R2^T dy):
+//                 d_h3 = r2 a + dg s r1,
+//                 d_h1 = (r2 h3 + dg r3) s + dg h3 r1 silu''(h1),
+//                 d_dg = a r3 + h3 s r1,
+//                 dW1 += d_h1^T K, dW3 += d_h3^T K, dW2 += V^T (-lr d_dg),
+//                 dk = d_h1 W1 + d_h3 W3 + (dg h3 s) R1 + (dg a) R3,
+//                 d_dy = d_dg W2^T + g R2^T, dv = -lr d_dy, dlr = -v . d_dy;
+//      causal read VJP at W_c for the chunk's queries (per query: hq1, hq3,
+//                 aq = silu(hq1), gq = aq hq3, dgq = W2^T dout):
+//                 dW1 += (dgq hq3 s)^T Q, dW3 += (dgq aq)^T Q,
+//                 dW2 += dout^T gq, dq = (dgq hq3 s) W1 + (dgq aq) W3.
+//    The bidirectional read VJP runs once, before the reverse loop, with the
+//    final weights.  dW0 = dW after the first chunk.
+// Every product is a batched tcgen05 GEMM (bf16 operands, fp32 accumulators)
+// of gemm.cuh; the elementwise steps are the kernels below.
+#include <algorithm>
+
+#include "gemm.cuh"
+#include "kernels.h"
+
+namespace ttt {
+
+namespace {
+
+TTT_DEVICE_INLINE float sig(float x) { return 1.f / (1.f + __expf(-x)); }
+
+// bf16 copies of fp32 matrices (the GEMMs' weight and R operands)
+__global__ void bwd_cast_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                                size_t n4) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float4 x = reinterpret_cast<const float4*>(src)[i];
+    reinterpret_cast<uint2*>(dst)[i] = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+  }
+}
+
+struct RowStepArgs {
+  int BH, d, dh, mask, normalize, momentum;
+  float beta, norm_eps;
+  float* dW;             // [3 mats][BH][rows][cols], in: dL/dW_{c+1}, out: dL/dU
+  float* dM;             // momentum carry (momentum only)
+  const float* Wn;       // W_{c+1}
+  const float* rn;       // row norms of U_c, [BH][2 dh + d]
+  float* R;              // out: dL/dG_c (fp32)
+  __nv_bfloat16* Rb;     // out: bf16 copy
+};
+// One warp per row of one matrix of one head (rows of up to 1024 columns).
+__global__ void bwd_row_step_kernel(RowStepArgs a) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int per = 2 * a.dh + a.d;
+  if (gw >= a.BH * per) return;
+  const int bh = gw / per, rr = gw % per;
+  const int mat = rr < a.dh ? 0 : (rr < 2 * a.dh ? 1 : 2);
+  const int row = mat == 0 ? rr : (mat == 1 ? rr - a.dh : rr - 2 * a.dh);
+  const int rows = mat < 2 ? a.dh : a.d, cols = mat < 2 ? a.d : a.dh;
+  const size_t mat_elems = (size_t)a.BH * a.d * a.dh;
+  const size_t off = mat * mat_elems + ((size_t)bh * rows + row) * cols;
+  if (!(a.mask & (1 << mat))) {   // not updated: no dependence on G, dW passes through
+    for (int c = lane; c < cols; c += 32) {
+      a.R[off + c] = 0.f;
+      a.Rb[off + c] = __float2bfloat16_rn(0.f);
+    }
+    return;
+  }
+  float* dW = a.dW + off;
+  float proj = 0.f, inv = 1.f;
+  bool big = true;
+  if (a.normalize) {
+    const float n = a.rn[gw];
+    big = n > a.norm_eps;
+    inv = 1.f / (big ? n : a.norm_eps);
+    for (int c = lane; c < cols; c += 32) proj += a.Wn[off + c] * dW[c];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) proj += __shfl_xor_sync(0xffffffffu, proj, o);
+  }
+  for (int c = lane; c < cols; c += 32) {
+    float du = dW[c];
+    if (a.normalize) du = big ? (du - a.Wn[off + c] * proj) * inv : du * inv;
+    float r;
+    if (a.momentum) {
+      const float m = a.dM[off + c] - du;
+      r = m;
+      a.dM[off + c] = a.beta * m;
+    } else {
+      r = -du;
+    }
+    dW[c] = du;
+    a.R[off + c] = r;
+    a.Rb[off + c] = __float2bfloat16_rn(r);
+  }
+}
+
+struct KeyEwArgs {
+  int BH, C, cmax, dh, lr_len, t0;
+  const float* lr;       // [BH][lr_len]
+  // fp32 [BH][cmax][dh]: K W1^T, K W3^T, V W2, K R1^T, K R3^T, V R2
+  const float *h1, *h3, *vw2, *r1, *r3, *vr2;
+  // bf16 [BH][cmax][dh] outputs
+  __nv_bfloat16 *d_h1, *d_h3, *d_dg, *d_dgn, *e1, *e3, *g;
+};
+// The chunk gradient's elementwise VJP step; rows past the chunk are zero.
+__global__ void bwd_key_ew_kernel(KeyEwArgs a) {
+  const size_t n = (size_t)a.BH * a.cmax * a.dh;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t bh = i / ((size_t)a.cmax * a.dh);
+    const int t = (int)((i / a.dh) % a.cmax);
+    float vdh1 = 0.f, vdh3 = 0.f, vddg = 0.f, vddgn = 0.f, ve1 = 0.f, ve3 = 0.f, vg = 0.f;
+    if (t < a.C) {
+      const float eta = a.lr[bh * a.lr_len + a.t0 + t];
+      const float x = a.h1[i], y = a.h3[i];
+      const float sg = sig(x);
+      const float act = x * sg;                                   // silu
+      const float s1 = sg * (1.f + x * (1.f - sg));               // silu'
+      const float s2 = sg * (1.f - sg) * (2.f + x * (1.f - 2.f * sg));   // silu''
+      const float dg = -eta * a.vw2[i], r2 = -eta * a.vr2[i];
+      const float r1 = a.r1[i], r3 = a.r3[i];
+      vdh3 = r2 * act + dg * s1 * r1;
+      vdh1 = (r2 * y + dg * r3) * s1 + dg * y * r1 * s2;
+      vddg = act * r3 + y * s1 * r1;
+      vddgn = -eta * vddg;
+      ve1 = dg * y * s1;
+      ve3 = dg * act;
+      vg = act * y;
+    }
+    a.d_h1[i] = __float2bfloat16_rn(vdh1);
+    a.d_h3[i] = __float2bfloat16_rn(vdh3);
+    a.d_dg[i] = __float2bfloat16_rn(vddg);
+    a.d_dgn[i] = __float2bfloat16_rn(vddgn);
+    a.e1[i] = __float2bfloat16_rn(ve1);
+    a.e3[i] = __float2bfloat16_rn(ve3);
+    a.g[i] = __float2bfloat16_rn(vg);
+  }
+}
+
+struct ReadEwArgs {
+  int BH, C, cmax, dh;
+  const float *hq1, *hq3, *dgq;   // fp32 [BH][cmax][dh]: Q W1^T, Q W3^T, dout W2
+  __nv_bfloat16 *dhq1, *dhq3, *gq;
+};
+__global__ void bwd_read_ew_kernel(ReadEwArgs a) {
+  const size_t n = (size_t)a.BH * a.cmax * a.dh;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)((i / a.dh) % a.cmax);
+    float v1 = 0.f, v3 = 0.f, vg = 0.f;
+    if (t < a.C) {
+      const float x = a.hq1[i], y = a.hq3[i], dg = a.dgq[i];
+      const float sg = sig(x);
+      const float act = x * sg;
+      v1 = dg * y * sg * (1.f + x * (1.f - sg));
+      v3 = dg * act;
+      vg = act * y;
+    }
+    a.dhq1[i] = __float2bfloat16_rn(v1);
+    a.dhq3[i] = __float2bfloat16_rn(v3);
+    a.gq[i] = __float2bfloat16_rn(vg);
+  }
+}
+
+// dv = -lr d_dy, dlr = -v . d_dy for the chunk's tokens (one warp per token).
+__global__ void bwd_dv_kernel(int BH, int C, int cmax, int d, int N, int t0, const float* lr,
+                              const __nv_bfloat16* v, const float* ddy, float* dv, float* dlr) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= BH * C) return;
+  const int bh = gw / C, t = gw % C;
+  const size_t tok = (size_t)bh * N + t0 + t;
+  const float eta = lr[tok];
+  const float* src = ddy + ((size_t)bh * cmax + t) * d;
+  float acc = 0.f;
+  for (int c = lane; c < d; c += 32) {
+    const float x = src[c];
+    dv[tok * d + c] = -eta * x;
+    acc += __bfloat162float(v[tok * d + c]) * x;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) dlr[tok] = -acc;
+}
+
+}  // namespace
+
+LactBwdWorkspace lact_bwd_layout(const LactLaunch& f) {
+  LactBwdWorkspace w{};
+  const size_t BH = (size_t)f.B * f.H, mat = BH * f.d * f.dh;
+  const int nch = f.N_in > 0 ? (f.N_in + f.chunk - 1) / f.chunk : 0;
+  const int cin = std::min(f.chunk, std::max(f.N_in, 1));
+  w.cmax = (std::max(cin, f.causal ? 0 : f.N_q) + 127) / 128 * 128;
+  w.nch = nch;
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  size_t o = 0;
+  w.status = o; o = al(o + 256);
+  w.fws_bytes = lact_workspace_layout(f.B, f.H, f.N_in, f.N_q, f.d, f.dh, f.chunk, f.causal,
+                                      f.opt, 0, f.update_mask, f.normalize_rows, 0).total;
+  w.fws = o; o = al(o + w.fws_bytes);
+  w.state = o; o = al(o + (f.opt == 0 ? 3 : 6) * mat * 4);
+  w.wsave = o; o = al(o + (size_t)(nch + 1) * 3 * mat * 4);
+  w.rn = o; o = al(o + (size_t)std::max(nch, 1) * BH * (2 * f.dh + f.d) * 4);
+  w.G = o; o = al(o + 3 * mat * 4);
+  w.dW = o; o = al(o + 3 * mat * 4);
+  w.dM = o; o = al(o + 3 * mat * 4);
+  w.R = o; o = al(o + 3 * mat * 4);
+  w.Rb = o; o = al(o + 3 * mat * 2);
+  w.Wb = o; o = al(o + 3 * mat * 2);
+  const size_t inter = BH * w.cmax * f.dh;
+  for (int i = 0; i < 6; ++i) { w.f32[i] = o; o = al(o + inter * 4); }
+  for (int i = 0; i < 7; ++i) { w.b16[i] = o; o = al(o + inter * 2); }
+  w.ddy = o; o = al(o + BH * w.cmax * f.d * 4);
+  w.total = o;
+  return w;
+}
+
+#define BWD_TRY(...)                      \
+  do {                                    \
+    if ((__VA_ARGS__) != 0) return -1;    \
+  } while (0)
+
+int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
+  const LactLaunch& f = L.f;
+  const LactBwdWorkspace w = lact_bwd_layout(f);
+  const int BH = f.B * f.H, d = f.d, dh = f.dh;
+  const size_t mat = (size_t)BH * d * dh;
+  uint8_t* ws = L.ws;
+  auto F = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  auto Hb = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
+  float* state = F(w.state);
+  float* wsave = F(w.wsave);
+  float* rn = F(w.rn);
+  const int nch = w.nch;
+  const int q_rows = f.causal ? f.N_in : f.N_q;
+
+  // ---------------------------------------------------------------- 1. forward replay
+  BWD_TRY(cudaMemcpyAsync(state, L.W0, 3 * mat * 4, cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1);
+  if (f.opt != 0)
+    BWD_TRY(cudaMemsetAsync(state + 3 * mat, 0, 3 * mat * 4, stream) == cudaSuccess ? 0 : -1);
+  LactLaunch p = f;
+  p.state = state;
+  p.ws = ws + w.fws;
+  p.ws_bytes = w.fws_bytes;
+  p.split = 0;
+  p.rownorm_out = nullptr;
+  for (int c = 0; c < nch; ++c) {
+    const int t0 = c * f.chunk, C = std::min(f.chunk, f.N_in - t0);
+    BWD_TRY(cudaMemcpyAsync(wsave + (size_t)c * 3 * mat, state, 3 * mat * 4,
+                            cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1);
+    p.mode = LACT_GRAD; p.t0 = t0; p.n = C; p.G = F(w.G);
+    BWD_TRY(launch_lact(p, stream));
+    p.mode = LACT_APPLY; p.rownorm_out = rn + (size_t)c * BH * (2 * dh + d);
+    BWD_TRY(launch_lact(p, stream));
+    p.rownorm_out = nullptr;
+  }
+  BWD_TRY(cudaMemcpyAsync(wsave + (size_t)nch * 3 * mat, state, 3 * mat * 4,
+                          cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1);
+
+  // ---------------------------------------------------------------- maps and helpers
+  const uint64_t BHu = (uint64_t)BH;
+  auto tok = [&](CUtensorMap* m, const void* ptr, int rows, uint32_t box_rows) {   // [BH][rows][d]
+    return make_tmap_bf16_3d(m, ptr, d, rows, BHu, (uint64_t)d * 2, (uint64_t)d * 2 * rows, 64, box_rows);
+  };
+  auto inter = [&](CUtensorMap* m, const void* ptr, uint32_t box_rows) {            // [BH][cmax][dh]
+    return make_tmap_bf16_3d(m, ptr, dh, w.cmax, BHu, (uint64_t)dh * 2, (uint64_t)dh * 2 * w.cmax, 64,
+                             box_rows);
+  };
+  // weights and R, bf16 [BH][rows][cols]: W1/W3-shaped [dh][d], W2-shaped [d][dh]
+  auto w13 = [&](CUtensorMap* m, const void* ptr, uint32_t box_rows) {
+    return make_tmap_bf16_3d(m, ptr, d, dh, BHu, (uint64_t)d * 2, (uint64_t)d * dh * 2, 64, box_rows);
+  };
+  auto w2m = [&](CUtensorMap* m, const void* ptr, uint32_t box_rows) {
+    return make_tmap_bf16_3d(m, ptr, dh, d, BHu, (uint64_t)dh * 2, (uint64_t)d * dh * 2, 64, box_rows);
+  };
+  __nv_bfloat16* Wb = Hb(w.Wb);
+  __nv_bfloat16* Rb = Hb(w.Rb);
+  auto cast = [&](const float* src, __nv_bfloat16* dst, size_t n) -> int {
+    const size_t n4 = n / 4;
+    bwd_cast_kernel<<<(unsigned)std::min<size_t>((n4 + 255) / 256, 4096), 256, 0, stream>>>(src, dst, n4);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  };
+  float* dW = F(w.dW);
+  float* dM = F(w.dM);
+  // C[b][m][n] (+)= sum_p A_p B_p^T  into fp32 `o` (ld, batch stride), optionally accumulating
+  // TMA coordinate offsets: am (A rows, K-major A), ak / bk (the K coordinate
+  // of an MN-major A / B: token rows of a token tensor)
+  auto gemm = [&](int variant, const CUtensorMap* A, const CUtensorMap* B, int np, int M, int N,
+                  int ksteps, float* o, int ld, long long bs, bool acc, int row_off, int am,
+                  int ak, int bk) -> int {
+    GemmMaps m{};
+    GemmArgs g = gemm_args_default(L.st);
+    for (int i = 0; i < np; ++i) {
+      m.a[i] = A[i];
+      m.b[i] = B[i];
+      g.a_m_off[i] = am;
+      g.a_k_off[i] = ak;
+      g.b_k_off[i] = bk;
+    }
+    g.npairs = np; g.M = M; g.N = N; g.batch = BH; g.k_steps = ksteps;
+    g.o32 = o; g.ld32 = ld; g.o32_bs = bs; g.out_row_off = row_off;
+    if (acc) { g.beta = 1.f; g.cin = o + 0; g.cin_bs = bs; g.ldc = ld; }
+    return gemm_launch(variant, m, g, stream, K_GEMM_GRAD);
+  };
+  // cin of an accumulating GEMM is read at row m (no row offset), so
+  // accumulating outputs always start at row 0 of their buffer
+
+  CUtensorMap mq_k{}, mq_mn{}, mk_k{}, mk_mn{}, mv_k{}, mv_mn{}, mdo_k{}, mdo_mn{};
+  if (f.N_in > 0) {
+    BWD_TRY(tok(&mk_k, f.k, f.N_in, 128));
+    BWD_TRY(tok(&mk_mn, f.k, f.N_in, 64));
+    BWD_TRY(tok(&mv_k, f.v, f.N_in, 128));
+    BWD_TRY(tok(&mv_mn, f.v, f.N_in, 64));
+  }
+  if (q_rows > 0) {
+    BWD_TRY(tok(&mq_k, f.q, q_rows, 128));
+    BWD_TRY(tok(&mq_mn, f.q, q_rows, 64));
+    BWD_TRY(tok(&mdo_k, L.dout, q_rows, 128));
+    BWD_TRY(tok(&mdo_mn, L.dout, q_rows, 64));
+  }
+  CUtensorMap mW1k, mW3k, mW2mn, mW1mn, mW3mn, mW2k, mR1k, mR3k, mR2mn, mR1mn, mR3mn, mR2k;
+  BWD_TRY(w13(&mW1k, Wb, 128) | w13(&mW3k, Wb + mat, 128) | w2m(&mW2mn, Wb + 2 * mat, 64));
+  BWD_TRY(w13(&mW1mn, Wb, 64) | w13(&mW3mn, Wb + mat, 64) | w2m(&mW2k, Wb + 2 * mat, 128));
+  BWD_TRY(w13(&mR1k, Rb, 128) | w13(&mR3k, Rb + mat, 128) | w2m(&mR2mn, Rb + 2 * mat, 64));
+  BWD_TRY(w13(&mR1mn, Rb, 64) | w13(&mR3mn, Rb + mat, 64) | w2m(&mR2k, Rb + 2 * mat, 128));
+  float* f32[6];
+  __nv_bfloat16* b16[7];
+  for (int i = 0; i < 6; ++i) f32[i] = F(w.f32[i]);
+  for (int i = 0; i < 7; ++i) b16[i] = Hb(w.b16[i]);
+  CUtensorMap mb_k[7], mb_mn[7];
+  for (int i = 0; i < 7; ++i) BWD_TRY(inter(&mb_k[i], b16[i], 128) | inter(&mb_mn[i], b16[i], 64));
+  const long long ibs = (long long)w.cmax * dh;
+  float* dW1 = dW;
+  float* dW3 = dW + mat;
+  float* dW2 = dW + 2 * mat;
+  const long long w13bs = (long long)dh * d, w2bs = (long long)d * dh;
+
+  // read VJP for query rows [t0, t0 + C) with the weights in Wb: dq rows and dW
+  auto read_vjp = [&](int t0, int C) -> int {
+    const int ks = (C + 63) / 64;
+    // hq1 = Q W1^T, hq3 = Q W3^T, dgq = dout W2   (M = C, N = dh, K = d)
+    BWD_TRY(gemm(GEMM_AK_BK, &mq_k, &mW1k, 1, C, dh, d / 64, f32[0], dh, ibs, false, 0, t0, 0, 0));
+    BWD_TRY(gemm(GEMM_AK_BK, &mq_k, &mW3k, 1, C, dh, d / 64, f32[1], dh, ibs, false, 0, t0, 0, 0));
+    BWD_TRY(gemm(GEMM_AK_BMN, &mdo_k, &mW2mn, 1, C, dh, d / 64, f32[2], dh, ibs, false, 0, t0, 0, 0));
+    ReadEwArgs ra{BH, C, w.cmax, dh, f32[0], f32[1], f32[2], b16[0], b16[1], b16[6]};
+    const size_t n = (size_t)BH * w.cmax * dh;
+    bwd_read_ew_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 8192), 256, 0, stream>>>(ra);
+    BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    // dW1 += dhq1^T Q, dW3 += dhq3^T Q  (M = dh, N = d, K = C tokens)
+    BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[0], &mq_mn, 1, dh, d, ks, dW1, d, w13bs, true, 0, 0, 0, t0));
+    BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[1], &mq_mn, 1, dh, d, ks, dW3, d, w13bs, true, 0, 0, 0, t0));
+    // dW2 += dout^T gq  (M = d, N = dh)
+    BWD_TRY(gemm(GEMM_AMN_BMN, &mdo_mn, &mb_mn[6], 1, d, dh, ks, dW2, dh, w2bs, true, 0, 0, t0, 0));
+    // dq rows = dhq1 W1 + dhq3 W3  (M = C, N = d, K = dh)
+    const CUtensorMap A[2] = {mb_k[0], mb_k[1]}, B[2] = {mW1mn, mW3mn};
+    return gemm(GEMM_AK_BMN, A, B, 2, C, d, dh / 64, L.dq, d, (long long)q_rows * d, false, t0,
+                0, 0, 0);
+  };
+
+  // ---------------------------------------------------------------- 2. reverse
+  if (L.dW_end)
+    BWD_TRY(cudaMemcpyAsync(dW, L.dW_end, 3 * mat * 4, cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1);
+  else
+    BWD_TRY(cudaMemsetAsync(dW, 0, 3 * mat * 4, stream) == cudaSuccess ? 0 : -1);
+  BWD_TRY(cudaMemsetAsync(dM, 0, 3 * mat * 4, stream) == cudaSuccess ? 0 : -1);
+  if (!f.causal && f.N_q > 0) {   // the queries read the final weights
+    BWD_TRY(cast(wsave + (size_t)nch * 3 * mat, Wb, 3 * mat));
+    BWD_TRY(read_vjp(0, f.N_q));
+  }
+  RowStepArgs rs{};
+  rs.BH = BH; rs.d = d; rs.dh = dh; rs.mask = f.update_mask; rs.normalize = f.normalize_rows;
+  rs.momentum = f.opt == 1; rs.beta = f.beta; rs.norm_eps = f.norm_eps;
+  rs.dW = dW; rs.dM = dM; rs.R = F(w.R); rs.Rb = Rb;
+  const int row_warps = BH * (2 * dh + d);
+  for (int c = nch - 1; c >= 0; --c) {
+    const int t0 = c * f.chunk, C = std::min(f.chunk, f.N_in - t0);
+    const int ks = (C + 63) / 64;
+    rs.Wn = wsave + (size_t)(c + 1) * 3 * mat;
+    rs.rn = rn + (size_t)c * BH * (2 * dh + d);
+    bwd_row_step_kernel<<<(row_warps * 32 + 255) / 256, 256, 0, stream>>>(rs);
+    BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    BWD_TRY(cast(wsave + (size_t)c * 3 * mat, Wb, 3 * mat));
+    // h1 = K W1^T, h3 = K W3^T, vw2 = V W2, r1 = K R1^T, r3 = K R3^T, vr2 = V R2
+    BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mW1k, 1, C, dh, d / 64, f32[0], dh, ibs, false, 0, t0, 0, 0));
+    BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mW3k, 1, C, dh, d / 64, f32[1], dh, ibs, false, 0, t0, 0, 0));
+    BWD_TRY(gemm(GEMM_AK_BMN, &mv_k, &mW2mn, 1, C, dh, d / 64, f32[2], dh, ibs, false, 0, t0, 0, 0));
+    BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mR1k, 1, C, dh, d / 64, f32[3], dh, ibs, false, 0, t0, 0, 0));
+    BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mR3k, 1, C, dh, d / 64, f32[4], dh, ibs, false, 0, t0, 0, 0));
+    BWD_TRY(gemm(GEMM_AK_BMN, &mv_k, &mR2mn, 1, C, dh, d / 64, f32[5], dh, ibs, false, 0, t0, 0, 0));
+    KeyEwArgs ka{BH, C, w.cmax, dh, f.N_in, t0, f.lr, f32[0], f32[1], f32[2], f32[3], f32[4], f32[5],
+                 b16[0], b16[1], b16[2], b16[3], b16[4], b16[5], b16[6]};
+    const size_t n = (size_t)BH * w.cmax * dh;
+    bwd_key_ew_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 8192), 256, 0, stream>>>(ka);
+    BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    // dk rows = d_h1 W1 + d_h3 W3 + e1 R1, then + e3 R3   (M = C, N = d, K = dh)
+    {
+      const CUtensorMap A[3] = {mb_k[0], mb_k[1], mb_k[4]}, B[3] = {mW1mn, mW3mn, mR1mn};
+      BWD_TRY(gemm(GEMM_AK_BMN, A, B, 3, C, d, dh / 64, F(w.ddy), d, (long long)w.cmax * d, false, 0,
+                   0, 0, 0));
+      BWD_TRY(gemm(GEMM_AK_BMN, &mb_k[5], &mR3mn, 1, C, d, dh / 64, F(w.ddy), d, (long long)w.cmax * d,
+                   true, 0, 0, 0, 0));
+    }
+    // the chunk's dk rows: copy out of the temporary (rows t0.. of dk)
+    BWD_TRY(cudaMemcpy2DAsync(L.dk + (size_t)t0 * d, (size_t)f.N_in * d * 4, F(w.ddy),
+                              (size_t)w.cmax * d * 4, (size_t)C * d * 4, BH, cudaMemcpyDeviceToDevice,
+                              stream) == cudaSuccess ? 0 : -1);
+    // weight gradients: dW1 += d_h1^T K, dW3 += d_h3^T K, dW2 += V^T (-lr d_dg)
+    BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[0], &mk_mn, 1, dh, d, ks, dW1, d, w13bs, true, 0, 0, 0, t0));
+    BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[1], &mk_mn, 1, dh, d, ks, dW3, d, w13bs, true, 0, 0, 0, t0));
+    BWD_TRY(gemm(GEMM_AMN_BMN, &mv_mn, &mb_mn[3], 1, d, dh, ks, dW2, dh, w2bs, true, 0, 0, t0, 0));
+    // d_dy = d_dg W2^T + g R2^T   (M = C, N = d, K = dh)
+    {
+      const CUtensorMap A[2] = {mb_k[2], mb_k[6]}, B[2] = {mW2k, mR2k};
+      BWD_TRY(gemm(GEMM_AK_BK, A, B, 2, C, d, dh / 64, F(w.ddy), d, (long long)w.cmax * d, false, 0,
+                   0, 0, 0));
+    }
+    {
+      const int warps = BH * C;
+      bwd_dv_kernel<<<(warps * 32 + 255) / 256, 256, 0, stream>>>(
+          BH, C, w.cmax, d, f.N_in, t0, f.lr, reinterpret_cast<const __nv_bfloat16*>(f.v), F(w.ddy),
+          L.dv, L.dlr);
+      BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    }
+    if (f.causal) BWD_TRY(read_vjp(t0, C));
+  }
+  return cudaMemcpyAsync(L.dW0, dW, 3 * mat * 4, cudaMemcpyDeviceToDevice, stream) == cudaSuccess
+             ? 0 : -1;
+}
+
+}  // namespace ttt

@@ -1,0 +1,96 @@
+"""GPU parity for the backward pass of the LaCT layer (lact_chunk_bwd)
+against the written-out backward oracle (oracle.lact_backward, itself pinned
+to autograd and to central differences of the forward oracle).  Tolerance:
+normwise 2e-2 per gradient (bf16 operands, fp32 accumulation)."""
+import numpy as np
+import pytest
+import torch
+
+import learned_linear_attention_b200 as T
+from oracle.lact_backward import lact_backward_explicit
+from ttt_synth import make_lact_grads, make_lact_inputs
+from gpu_util import rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+NAMES = ("q", "k", "v", "lr", "W1", "W3", "W2")
+
+
+def _run(x, g, opt="gd", with_dw=True, **kw):
+    B, H, N, d = x.k.values.shape
+    dh = x.W1.shape[-2]
+    R = x.q.values.shape[2]
+    desc = T.make_lact_desc(B, H, N, d, dh, x.chunk, N_q=R, order=x.order, opt=opt,
+                            split_operands=False, **kw)
+    state0 = T.alloc_lact_state(desc)
+    T.lact_state_init(desc, *[torch.from_numpy(w).cuda() for w in (x.W1, x.W3, x.W2)], 0, state0)
+    mat = B * H * d * dh
+    dW_end = None
+    if with_dw:
+        dW_end = torch.from_numpy(np.concatenate([w.ravel() for w in g.dW_end])).cuda()
+    grads = [torch.full((B, H, R, d), float("nan"), device="cuda"),
+             torch.full((B, H, N, d), float("nan"), device="cuda"),
+             torch.full((B, H, N, d), float("nan"), device="cuda"),
+             torch.full((B, H, N), float("nan"), device="cuda"),
+             torch.full((3 * mat,), float("nan"), device="cuda")]
+    ws = T.alloc_workspace(T.lact_bwd_workspace_bytes(desc))
+    T.lact_chunk_bwd(desc, to_dev(x.q), to_dev(x.k), to_dev(x.v), torch.from_numpy(x.lr).cuda(),
+                     state0, to_dev(g.dout), dW_end, *grads, ws)
+    assert T.ttt_check_device_status(ws) == T.TTT_OK
+    out = [t.cpu().numpy() for t in grads[:4]]
+    dW = grads[4].cpu().numpy()
+    out += [dW[:mat].reshape(B, H, dh, d), dW[mat:2 * mat].reshape(B, H, dh, d),
+            dW[2 * mat:].reshape(B, H, d, dh)]
+    return out
+
+
+def _oracle(x, g, opt="gd", with_dw=True, **kw):
+    B = x.k.values.shape[0]
+    W = [np.broadcast_to(w[None], (B,) + w.shape).astype(np.float64) for w in (x.W1, x.W3, x.W2)]
+    okw = {k: v for k, v in kw.items() if k in ("beta", "normalize_rows", "update_mask")}
+    return lact_backward_explicit(x.q.values, x.k.values, x.v.values, x.lr, *W, g.dout.values,
+                                  g.dW_end if with_dw else None, chunk=x.chunk, order=x.order,
+                                  opt=opt, **okw)
+
+
+def _check(x, g, opt="gd", with_dw=True, **kw):
+    got = _run(x, g, opt, with_dw, **kw)
+    ref = _oracle(x, g, opt, with_dw, **kw)
+    for name, a, r in zip(NAMES, got, ref):
+        assert not np.isnan(a).any(), name
+        assert rel_err(a, r) <= TOL, (name, rel_err(a, r))
+
+
+@pytest.mark.parametrize("opt", ["gd", "momentum"])
+def test_causal_chunks(cuda_device, opt):
+    """Three chunks (128, 128, 72 tokens: the last ragged), d = 128, dh = 256."""
+    x = make_lact_inputs(1, 2, 328, 128, 256, chunk=128, order="causal", cfg=81)
+    _check(x, make_lact_grads(x, cfg=81), opt, beta=0.9)
+
+
+def test_causal_without_end_gradient(cuda_device):
+    x = make_lact_inputs(2, 1, 256, 128, 256, chunk=128, order="causal", cfg=82)
+    _check(x, make_lact_grads(x, cfg=82), with_dw=False)
+
+
+def test_bidirectional(cuda_device):
+    x = make_lact_inputs(1, 2, 300, 128, 256, chunk=128, order="bidirectional", Nq=90,
+                         v_norm=True, lr_kind="0.01sig", cfg=83)
+    _check(x, make_lact_grads(x, cfg=83), "momentum", beta=0.8)
+
+
+def test_w2_only_without_normalisation(cuda_device):
+    x = make_lact_inputs(1, 2, 256, 128, 256, chunk=128, order="causal", cfg=84)
+    _check(x, make_lact_grads(x, cfg=84), update_mask=4, normalize_rows=False)
+
+
+def test_view_synthesis_dims(cuda_device):
+    x = make_lact_inputs(1, 1, 256, 384, 768, chunk=128, order="bidirectional", Nq=64,
+                         v_norm=True, lr_kind="0.01sig", cfg=85)
+    _check(x, make_lact_grads(x, cfg=85))
+
+
+def test_muon_is_rejected(cuda_device):
+    d = T.make_lact_desc(1, 1, 128, 128, 256, 128, opt="muon")
+    with pytest.raises(T.TTTError):
+        T.lact_bwd_workspace_bytes(d)

@@ -7,8 +7,9 @@ Both the CPU oracle (through the tests and the bench's CPU baseline) and the
 GPU path receive the very same bytes from here.
 
 Recipe (one PCG64 stream per tensor): ``numpy.random.default_rng([cfg, tid])``
-with ``tid`` 0:q 1:k 2:v 3:lr 4:W1 5:W3 6:W2 7:dout 8:dS_end (the output
-and end-state gradients a backward pass receives); float32 draws; per-token L2
+with ``tid`` 0:q 1:k 2:v 3:lr 4:W1 5:W3 6:W2 7:dout 8:dS_end (or dW1_end)
+9:dW3_end 10:dW2_end (the output and end-state gradients a backward pass
+receives); float32 draws; per-token L2
 normalisation where the workload says so; a single round-to-nearest-even cast
 to bfloat16 for bf16 workloads.  The workloads mirror the pages' settings:
 the linear fast weight of "Test-Time Training with KV Binding Is Secretly
@@ -21,7 +22,7 @@ from __future__ import annotations
 import dataclasses
 import numpy as np
 
-TID_Q, TID_K, TID_V, TID_LR, TID_W1, TID_W3, TID_W2, TID_DOUT, TID_DSEND = range(9)
+TID_Q, TID_K, TID_V, TID_LR, TID_W1, TID_W3, TID_W2, TID_DOUT, TID_DSEND, TID_DW3, TID_DW2 = range(11)
 
 
 # ---------------------------------------------------------------- bf16 bits
@@ -142,6 +143,23 @@ def make_linear_grads(x: LinearInputs, *, cfg=100, seed=0) -> LinearGrads:
     dout = _normal(cfg, TID_DOUT, (B, H, N, dv), seed)
     dS_end = np.float32(0.1) * _normal(cfg, TID_DSEND, (B, H, dk, dv), seed)
     return LinearGrads(_token(dout, x.q.dtype), dS_end)
+
+
+@dataclasses.dataclass
+class LaCTGrads:
+    dout: TokenTensor             # [B,H,R,d] bf16 (R: the output rows of the layer)
+    dW_end: tuple                 # float32 ([B,H,dh,d], [B,H,dh,d], [B,H,d,dh])
+
+
+def make_lact_grads(x: LaCTInputs, *, cfg=200, seed=0) -> LaCTGrads:
+    """Upstream gradients for a backward pass over ``x``: dout ~ N(0,1) (bf16)
+    and dW_end ~ 0.1 N(0,1) per weight (ids 8, 9, 10)."""
+    B, H, R, d = x.q.values.shape
+    dh = x.W1.shape[-2]
+    dout = _normal(cfg, TID_DOUT, (B, H, R, d), seed)
+    dW = tuple(np.float32(0.1) * _normal(cfg, tid, shp, seed) for tid, shp in
+               ((TID_DSEND, (B, H, dh, d)), (TID_DW3, (B, H, dh, d)), (TID_DW2, (B, H, d, dh))))
+    return LaCTGrads(_token(dout, "bf16"), dW)
 
 
 def make_lact_inputs(B, H, N, d, dh, *, chunk, order, Nq=None, qk_norm=True,
