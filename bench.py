@@ -469,6 +469,37 @@ def cpu_baseline(bench, budget_s=12.0):
             "kind": "oracle", "sample": sample, "seconds": t_all}
 
 
+def parallelism(world):
+    return "replicas" if world == 1 else f"dp{world} (independent replicas)"
+
+
+def l2_note(resident):
+    return (f"inputs larger than L2: {resident / 2**20:.0f} MiB touched per step vs "
+            f"{L2_BYTES / 2**20:.0f} MiB L2; no flush")
+
+
+def per_config_summary(name, value, step_ms, tflops, peak, secondary, extra):
+    """One compact entry per workload timed in this run: tokens/s, ms per
+    step, TFLOP/s and its fraction of the bf16 peak, and for the HBM-bound
+    linear layers GB/s and its fraction of the HBM peak."""
+    r = lambda x, n=4: None if x is None else float(f"{x:.{n}g}")  # noqa: E731
+    out = {name: {"tok_s": r(value), "ms": r(step_ms), "tflops": r(tflops),
+                  "frac_bf16": r(tflops / peak, 3)}}
+    if secondary:
+        rf = secondary["roofline"]
+        out[secondary["config"]["workload"]] = {
+            "tok_s": r(secondary["value"]), "ms": r(secondary["ms_per_step"]),
+            "gbs": r(rf.get("achieved")), "frac_hbm": r(rf.get("frac"), 3),
+            "kernel": rf.get("kernel")}
+    for k, e in (extra or {}).items():
+        d = {"tok_s": r(e["value"]), "ms": r(e["ms_per_step"]), "tflops": r(e["tflops"]),
+             "frac_bf16": r(e["frac_bf16_peak"], 3)}
+        if e.get("hbm"):
+            d["gbs"], d["frac_hbm"] = r(e["hbm"]["gbs"]), r(e["hbm"]["frac"], 3)
+        out[k] = d
+    return out
+
+
 # --------------------------------------------------------------------------- arms
 def run_reference(args):
     """CPU oracle on the host cores: each step is a bounded sample."""
@@ -489,11 +520,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": name, **{k: v for k, v in WORKLOADS[name].items()
-                                            if k in ("B", "H", "N", "d", "dh", "dk", "dv", "chunk",
-                                                     "order", "window", "update_mask",
-                                                     "backward")},
-                       "parallelism": "cpu"},
+            "config": {**bench.config(), "parallelism": parallelism(args.gpus),
+                       "l2": l2_note(bench.resident_bytes())},
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": os.cpu_count(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -515,6 +543,12 @@ class _CPUOnlyLaCT(LaCTBench):
         self.normalize_rows = w.get("normalize_rows", True)
         self.window = w.get("window", 0)
 
+    def resident_bytes(self):
+        """Bytes the GPU arm keeps resident for this workload (same tensors:
+        bf16 q, k, v and out, fp32 lr)."""
+        BH = self.B * self.H
+        return BH * (self.Nq * self.d * 2 * 2 + self.N * (2 * self.d * 2 + 4))
+
 
 class _CPUOnlyLinear:
     """Oracle side of a linear workload (forward, or backward when the
@@ -525,6 +559,24 @@ class _CPUOnlyLinear:
         self.name, self.w = name, dict(WORKLOADS[name])
         self.x = make_workload(name)
         self.g = make_linear_grads(self.x, cfg=self.w["cfg"]) if self.w.get("backward") else None
+        w = self.w
+        self.B, self.H, self.N, self.dk, self.dv = w["B"], w["H"], w["N"], w["dk"], w["dv"]
+
+    def config(self):
+        """The same workload description as the GPU arm's."""
+        c = LinearBench.config(self)
+        if self.g is not None:
+            c["pass"], c["out_dtype"] = "backward", "f32"
+        return c
+
+    def resident_bytes(self):
+        """Bytes the GPU arm keeps resident for this workload (same tensors)."""
+        el = 2 if self.w["dtype"] == "bf16" else 4
+        tok = self.B * self.H * self.N
+        if self.g is None:   # q, k, v, lr, bf16 out
+            return tok * ((2 * self.dk + self.dv) * el + 4 + 2 * self.dv)
+        return tok * ((2 * self.dk + 2 * self.dv) * el + 4 + (2 * self.dk + self.dv) * 4 + 4) + \
+            self.B * self.H * self.dk * self.dv * 4
 
     def oracle_sample(self, n_blocks):
         """Batch entry 0, all heads, the first 512 * n_blocks tokens."""
@@ -684,10 +736,8 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_baseline(bench)
         cfg = bench.config()
-        cfg["parallelism"] = "replicas" if world == 1 else f"dp{world} (independent replicas)"
-        cfg["launch"] = "host launches" if args.no_graph else "CUDA graph replay of one step"
-        cfg["l2"] = (f"inputs larger than L2: {bench.resident_bytes() / 2**20:.0f} MiB touched "
-                     f"per step vs {L2_BYTES / 2**20:.0f} MiB L2; no flush")
+        cfg["parallelism"] = parallelism(world)
+        cfg["l2"] = l2_note(bench.resident_bytes())
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -695,7 +745,12 @@ def main():
                 "tflops": tflops, "frac_bf16_peak": tflops / pk["bf16_tflops"],
                 "peak_source": pk_kind, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "clocks": clocks, "kernels": kernels,
+                "launch": "host launches" if args.no_graph else "CUDA graph replay of one step",
                 "secondary": secondary, "extra": extra or None}
+        # last, so that a record keeping only the end of the line still holds
+        # every workload's figures
+        line["per_config"] = per_config_summary(args.workload, value, step_ms, tflops,
+                                                pk["bf16_tflops"], secondary, extra)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
