@@ -290,7 +290,9 @@ int lact_workspace_bytes(const lact_desc* d, size_t* bytes) {
   int e = check_lact(d);
   if (e) return e;
   if (!bytes) return TTT_ERR_ARG;
-  *bytes = layout_of(d, 1).total;
+  // the fastest form's layout, and never less than the chunk loop's, which
+  // every call accepts (for short sequences the parallel form can be smaller)
+  *bytes = std::max(layout_of(d, 1).total, layout_of(d, 0).total);
   return TTT_OK;
 }
 

@@ -795,7 +795,8 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // ordered on the caller's stream.
 struct SideStreams {
   cudaStream_t s[3] = {nullptr, nullptr, nullptr};
-  cudaEvent_t fork = nullptr, join[3] = {nullptr, nullptr, nullptr}, read_done[2] = {nullptr, nullptr};
+  cudaEvent_t fork = nullptr, join[3] = {nullptr, nullptr, nullptr},
+              read_done[3] = {nullptr, nullptr, nullptr};
   bool ok = false;
 };
 // Helper streams and their events belong to the calling host thread (one set
@@ -809,7 +810,8 @@ static SideStreams* side_streams() {
   if (!x.ok) {
     bool good = cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess &&
                 cudaEventCreateWithFlags(&x.read_done[0], cudaEventDisableTiming) == cudaSuccess &&
-                cudaEventCreateWithFlags(&x.read_done[1], cudaEventDisableTiming) == cudaSuccess;
+                cudaEventCreateWithFlags(&x.read_done[1], cudaEventDisableTiming) == cudaSuccess &&
+                cudaEventCreateWithFlags(&x.read_done[2], cudaEventDisableTiming) == cudaSuccess;
     for (int i = 0; i < 3 && good; ++i)
       good = cudaStreamCreateWithFlags(&x.s[i], cudaStreamNonBlocking) == cudaSuccess &&
              cudaEventCreateWithFlags(&x.join[i], cudaEventDisableTiming) == cudaSuccess;
@@ -1026,10 +1028,11 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   const int BH = L.B * L.H, d = L.d, dh = L.dh;
   const bool split = L.split != 0;
   // the parallel form of the W2-only layer runs when the workspace holds it,
-  // else the chunk loop
+  // else the chunk loop; the per-chunk pieces of context parallelism (and the
+  // backward pass built on them) always use the chunk loop's layout
   LactWorkspace w =
       lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt, L.split,
-                            L.update_mask, L.normalize_rows, 1);
+                            L.update_mask, L.normalize_rows, L.mode == LACT_FULL ? 1 : 0);
   if (w.w2par && w.total > L.ws_bytes)
     w = lact_workspace_layout(L.B, L.H, L.N_in, L.N_q, d, dh, L.chunk, L.causal, L.opt, L.split,
                               L.update_mask, L.normalize_rows, 0);
@@ -1456,6 +1459,14 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   }
   if (L.mode == LACT_READ) {   // queries [t0, t0 + n) read the current weights
     if (L.n <= 0) return 0;
+    if (d == 128 && !split) {
+      ReadFusedLaunch rl{};
+      rl.BH = BH; rl.rows = q_rows; rl.t0 = L.t0; rl.C = L.n; rl.dh = dh; rl.out_bf16 = L.out_bf16;
+      rl.max_grid = num_sms();
+      rl.q = L.q; rl.w1b = wbuf[cur][0]; rl.w3b = wbuf[cur][1]; rl.w2b = wbuf[cur][2];
+      rl.out = L.out; rl.st = L.st;
+      return launch_lact_read_fused(rl, stream);
+    }
     TTT_TRY(key_pass(L.t0, L.n, 0, (L.n + 127) / 128));
     return read_out(L.t0, L.n, stream, Aq);
   }
@@ -1546,7 +1557,9 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // the row update writes buffer nxt(cur).  The read of chunk c (helper
   // stream; Aq buffer c % 2, W2 buffer cur) runs beside the update and the
   // next chunk on the SMs the fused kernel leaves free; the kernel of chunk
-  // c + 2 rewrites both, so it first waits for that read.
+  // c + 2 rewrites both, so it first waits for that read.  (Forming Aq in the
+  // fused kernel reuses the [W1_J; W3_J] tiles already in its shared memory:
+  // measured faster than a separate Q -> out read kernel on the free SMs.)
   const bool keygrad = w.keygrad != 0;
   int ci = 0;
   for (int t0 = 0; keygrad && t0 < L.N_in; t0 += L.chunk, ++ci) {
@@ -1605,8 +1618,17 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     cur = nxt(cur);
   }
   if (!L.causal && L.N_q > 0) {
-    TTT_TRY(key_pass(0, L.N_q, 0, (L.N_q + 127) / 128));
-    TTT_TRY(read_out(0, L.N_q, stream, Aq));
+    if (d == 128 && !split) {   // the fused read: Q -> out in one kernel
+      ReadFusedLaunch rl{};
+      rl.BH = BH; rl.rows = L.N_q; rl.t0 = 0; rl.C = L.N_q; rl.dh = dh; rl.out_bf16 = L.out_bf16;
+      rl.max_grid = num_sms();
+      rl.q = L.q; rl.w1b = wbuf[cur][0]; rl.w3b = wbuf[cur][1]; rl.w2b = wbuf[cur][2];
+      rl.out = L.out; rl.st = L.st;
+      TTT_TRY(launch_lact_read_fused(rl, stream));
+    } else {
+      TTT_TRY(key_pass(0, L.N_q, 0, (L.N_q + 127) / 128));
+      TTT_TRY(read_out(0, L.N_q, stream, Aq));
+    }
   }
   return 0;
 }

@@ -25,6 +25,8 @@ int make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t
                       uint32_t box_inner, uint32_t box_rows) {
   std::call_once(g_encode_once, load_encode);
   if (g_encode == nullptr) return -1;
+  // a map over no buffer would let a TMA load read address 0: refuse it
+  if (base == nullptr) return -1;
   if (rows == 0) rows = 1;
   if (batch == 0) batch = 1;
   cuuint64_t dims[3] = {inner, rows, batch};

@@ -186,6 +186,10 @@ def test_lact_workspace_sizes_for_the_workloads(lib):
     d3 = T.make_lact_desc(2, 4, 32768, 128, 256, 2048)
     ws3 = T.lact_workspace_bytes(d3)
     assert 4 * 8 * 2048 * 256 * 2 < ws3 < 64 << 20
+    # a short W2-only layer: the workspace of its fastest form is never
+    # smaller than the chunk loop's, which every call accepts
+    dw = T.make_lact_desc(1, 2, 256, 128, 256, 128, update_mask=4, normalize_rows=False)
+    assert T.lact_workspace_bytes(dw) >= T.lact_workspace_bytes_min(dw)
     # 196K-token view-synthesis set in one chunk: intermediates dominate
     d4 = T.make_lact_desc(1, 2, 196608, 384, 768, 196608, N_q=4096, order="bidirectional")
     assert T.lact_workspace_bytes(d4) > 3 * 2 * 196608 * 768 * 2
