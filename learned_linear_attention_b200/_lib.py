@@ -78,7 +78,7 @@ _SIGS = {
     "lact_apply_grad": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _SZ, _VP],
     "lact_read": [ctypes.POINTER(lact_desc), _I, _I, _VP, _VP, _VP, _VP, _SZ, _VP],
     "lact_bwd_workspace_bytes": [ctypes.POINTER(lact_desc), _SZP],
-    "lact_chunk_bwd": [ctypes.POINTER(lact_desc)] + [_VP] * 14 + [_SZ, _VP],
+    "lact_chunk_bwd": [ctypes.POINTER(lact_desc)] + [_VP] * 13 + [_SZ, _VP],
     "lact_chunk_fwd_noalloc": [ctypes.POINTER(lact_desc), _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "lact_noalloc_check_status": [_VP],
     "ttt_check_device_status": [_VP, _VP],

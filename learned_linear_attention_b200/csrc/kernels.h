@@ -239,6 +239,16 @@ struct KeyGradLaunch {
   DevStatus st;
 };
 int keygrad_groups(int BH, int dh, int C, int max_groups);
+// The fused memory read for head dim 128 (lact_read.cu): out rows [t0, t0 + C)
+// = W2 (silu(W1 q) * (W3 q)) with bf16 weight copies, on at most max_grid CTAs.
+struct ReadFusedLaunch {
+  int BH, rows, t0, C, dh, out_bf16, max_grid;
+  const void* q;                       // [BH][rows][128] bf16
+  const __nv_bfloat16 *w1b, *w3b, *w2b;
+  void* out;                           // [BH][rows][128]
+  DevStatus st;
+};
+int launch_lact_read_fused(const ReadFusedLaunch& L, cudaStream_t stream);
 int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream);
 
 // ----------------------------------------------------------------- profiling
