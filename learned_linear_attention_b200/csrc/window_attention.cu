@@ -368,6 +368,329 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Single pass with an online softmax.  One thread per query row holds the
+// row's 128 scores of a key tile; the row keeps a running maximum m (log2
+// units) and sum l, and P = exp2(s - m) goes straight into the P V product.
+// When a tile raises a row's maximum by more than 8 (a factor 256), the row
+// of O accumulated so far in TMEM is rescaled by exp2(m_old - m_new) before
+// that tile's P V product; smaller rises keep the old m (P stays below 256).
+// O is divided by l once, at the end.  Each key tile costs one Q K^T and one
+// P V product and one exponential per score.
+// ---------------------------------------------------------------------------
+namespace swa1 {
+constexpr int D = 128, BM = 128, BN = 128;
+constexpr uint32_t HALF = 128 * 64 * 2;
+constexpr uint32_t TILE = 2 * HALF;
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = TILE;                 // 2 K slots
+constexpr uint32_t OFF_V = OFF_K + 2 * TILE;     // 2 V slots
+constexpr uint32_t OFF_P = OFF_V + 2 * TILE;     // 2 P buffers
+constexpr uint32_t OFF_BAR = OFF_P + 2 * TILE;
+constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+constexpr int EPI_WARPS = 4;                      // one per TMEM lane quadrant: a thread per row
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr float RESCALE = 8.f;                    // lazy rescale threshold (log2 units)
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_COLS = 512;
+}  // namespace swa1
+
+__global__ void __launch_bounds__(swa1::THREADS, 1)
+    window_attention_1p_kernel(const __grid_constant__ SwaMaps maps, const SwaArgs a) {
+  using namespace swa1;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* k_full = q_full + 1;      // [2]
+  uint64_t* k_empty = k_full + 2;     // [2]
+  uint64_t* v_full = k_empty + 2;     // [2]
+  uint64_t* v_empty = v_full + 2;     // [2]
+  uint64_t* s_full = v_empty + 2;     // [2]
+  uint64_t* s_empty = s_full + 2;     // [2]
+  uint64_t* p_full = s_empty + 2;     // [2]
+  uint64_t* p_empty = p_full + 2;     // [2]
+  uint64_t* o_done = p_empty + 2;     // one phase per P V product
+  uint64_t* fin = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x / a.n_qt;
+  const int qt = a.n_qt - 1 - (int)(blockIdx.x % a.n_qt);   // the longest windows first
+  const int q0 = qt * BM;
+  const int kt_lo = max(0, q0 - a.window + 1) / BN;
+  const int nk = qt - kt_lo + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], EPI_WARPS * 32);
+      mbar_init(&p_full[s], EPI_WARPS * 32);
+      mbar_init(&p_empty[s], 1);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.q);
+    tma_prefetch_desc(&maps.k);
+    tma_prefetch_desc(&maps.v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  Waiter W{abort_flag, a.st, 450};
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, TILE);
+      tma_load_3d(smem + OFF_Q, &maps.q, q_full, 0, q0, bh);
+      tma_load_3d(smem + OFF_Q + HALF, &maps.q, q_full, 64, q0, bh);
+      int k_issued = 0, v_issued = 0;
+      for (int g = 0; g < nk; ++g) {
+        const int s = g & 1, row = (kt_lo + g) * BN;
+        // K slot free once the scores of tile g - 2 are done
+        if (g >= 2 && !W.wait(&k_empty[s], ((g >> 1) - 1) & 1, 1)) break;
+        mbar_arrive_expect_tx(&k_full[s], TILE);
+        tma_load_3d(smem + OFF_K + s * TILE, &maps.k, &k_full[s], 0, row, bh);
+        tma_load_3d(smem + OFF_K + s * TILE + HALF, &maps.k, &k_full[s], 64, row, bh);
+        k_issued = g + 1;
+        // V slot free once the P V product of tile g - 2 is done
+        if (g >= 2 && !W.wait(&v_empty[s], ((g >> 1) - 1) & 1, 2)) break;
+        mbar_arrive_expect_tx(&v_full[s], TILE);
+        tma_load_3d(smem + OFF_V + s * TILE, &maps.v, &v_full[s], 0, row, bh);
+        tma_load_3d(smem + OFF_V + s * TILE + HALF, &maps.v, &v_full[s], 64, row, bh);
+        v_issued = g + 1;
+      }
+      if (W.aborted()) {
+        W.drain(q_full, 0);
+        for (int g = max(0, k_issued - 2); g < k_issued; ++g) W.drain(&k_full[g & 1], (g >> 1) & 1);
+        for (int g = max(0, v_issued - 2); g < v_issued; ++g) W.drain(&v_full[g & 1], (g >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id_s = make_idesc(128, 128, false, false);
+      const uint32_t id_o = make_idesc(128, 128, false, true);
+      const uint64_t dq = make_sdesc(smem_u32(smem + OFF_Q), 16, 1024);
+      const uint64_t dk0 = make_sdesc(smem_u32(smem + OFF_K), 16, 1024);
+      const uint64_t dv0 = make_sdesc(smem_u32(smem + OFF_V), HALF, 1024);
+      const uint64_t dp0 = make_sdesc(smem_u32(smem + OFF_P), 16, 1024);
+      bool ok = W.wait(q_full, 0, 3);
+      tc_fence_after();
+      auto issue_s = [&](int g) -> bool {
+        const int s = g & 1;
+        if (!W.wait(&k_full[s], (g >> 1) & 1, 4)) return false;
+        if (g >= 2 && !W.wait(&s_empty[s], ((g >> 1) - 1) & 1, 5)) return false;
+        tc_fence_after();
+        const uint64_t dk = sdesc_add(dk0, s * TILE);
+        const uint32_t acc = tmem + (s ? TM_S1 : TM_S0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+          mma_bf16(acc, sdesc_add(dq, off), sdesc_add(dk, off), id_s, kk > 0);
+        }
+        mma_commit(&s_full[s]);
+        mma_commit(&k_empty[s]);
+        return true;
+      };
+      if (ok && nk > 0) ok = issue_s(0);
+      for (int g = 0; ok && g < nk; ++g) {
+        // the next tile's scores run while the softmax warps work on this one
+        if (g + 1 < nk && !issue_s(g + 1)) { ok = false; break; }
+        const int s = g & 1;
+        if (!W.wait(&p_full[s], (g >> 1) & 1, 6)) { ok = false; break; }
+        if (!W.wait(&v_full[s], (g >> 1) & 1, 7)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t dv = sdesc_add(dv0, s * TILE);
+        const uint64_t dp = sdesc_add(dp0, s * TILE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t offp = (kk >> 2) * HALF + (kk & 3) * 32;
+          mma_bf16(tmem + TM_O, sdesc_add(dp, offp), sdesc_add(dv, kk * 2048), id_o,
+                   (g > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&v_empty[s]);
+        mma_commit(&p_empty[s]);
+        mma_commit(o_done);
+      }
+      mma_commit(fin);
+      W.drain(fin, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;                // query row of the tile
+    const int qi = q0 + r;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const bool row_ok = qi < a.N;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    auto inside = [&](int kt) {
+      return kt * BN + BN - 1 <= q0 && kt * BN > q0 + BM - 1 - a.window && q0 + BM <= a.N;
+    };
+    for (int g = 0; ok && g < nk; ++g) {
+      const int kt = kt_lo + g, s = g & 1;
+      if (!W.wait(&s_full[s], (g >> 1) & 1, 8)) { ok = false; break; }
+      tc_fence_after();
+      float x[BN];
+      {
+        uint32_t xr[BN];
+        __syncwarp();   // tcgen05.ld is warp-collective: every lane, converged
+        // all eight loads in flight before one wait
+#pragma unroll
+        for (int c = 0; c < BN; c += 16) tmem_ld16_issue(tmem + lane_base + (s ? TM_S1 : TM_S0) + c, xr + c);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < BN; ++j) x[j] = __uint_as_float(xr[j]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_empty[s]);
+      float mx = -INFINITY;
+      if (inside(kt)) {
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+          x[j] *= a.scale_log2;
+          mx = fmaxf(mx, x[j]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+          const int kj = kt * BN + j;
+          const bool valid = row_ok && kj <= qi && kj > qi - a.window;
+          x[j] = valid ? x[j] * a.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, x[j]);
+        }
+      }
+      // lazy rescale: keep m unless the tile raises it by more than RESCALE
+      float alpha = 1.f;
+      if (mx > m + RESCALE || (m == -INFINITY && mx != -INFINITY)) {
+        alpha = m == -INFINITY ? 0.f : exp2f(m - mx);
+        m = mx;
+      }
+      // the rows of O a warp rescales: P V of tile g - 1 must be done first;
+      // every lane of the warp takes part in the TMEM load and store
+      const bool any = __any_sync(0xffffffffu, alpha != 1.f) && g > 0;
+      if (any) {
+        if (!W.wait(o_done, (g - 1) & 1, 9)) { ok = false; }
+        __syncwarp();
+        if (ok) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + TM_O + c, o);
+#pragma unroll
+            for (int j = 0; j < 32; j += 16) {
+              float t16[16];
+#pragma unroll
+              for (int u = 0; u < 16; ++u) t16[u] = o[j + u] * alpha;
+              tmem_st16(tmem + lane_base + TM_O + c + j, t16);
+            }
+          }
+          tc_fence_before();
+        }
+      }
+      if (!ok) break;
+      l *= alpha;
+      // P = exp2(s - m) (zero where masked or before any valid key)
+      uint32_t pk[BN / 2];
+      float add = 0.f;
+      if (m == -INFINITY) {
+#pragma unroll
+        for (int j = 0; j < BN / 2; ++j) pk[j] = 0u;
+      } else {
+#pragma unroll
+        for (int j = 0; j < BN; j += 2) {
+          const float p0 = exp2f(x[j] - m), p1 = exp2f(x[j + 1] - m);
+          add += p0 + p1;
+          pk[j >> 1] = pack_bf16x2(p0, p1);
+        }
+      }
+      l += add;
+      // P buffer s is free once the P V product of tile g - 2 is done (its own
+      // barrier: o_done may already be a phase further on)
+      if (g >= 2 && !W.wait(&p_empty[s], ((g >> 1) - 1) & 1, 10)) { ok = false; break; }
+      const uint32_t pb = smem_u32(smem + OFF_P + s * TILE);
+#pragma unroll
+      for (int j = 0; j < BN; j += 8)
+        st_shared_v4(pb + (uint32_t)(j >> 6) * HALF + sw128_offset(r, j & 63), pk[j / 2],
+                     pk[j / 2 + 1], pk[j / 2 + 2], pk[j / 2 + 3]);
+      fence_async_smem();
+      mbar_arrive(&p_full[s]);
+    }
+    if (ok && nk > 0 && W.wait(o_done, (nk - 1) & 1, 11)) {
+      tc_fence_after();
+      const float inv_l = (row_ok && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        float o[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_base + TM_O + c, o);   // every lane (warp-collective)
+        if (!row_ok) continue;
+        const size_t base = ((size_t)bh * a.N + qi) * D + c;
+        if (a.out_bf16) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float v8[8];
+            if (a.accumulate) {
+              const uint4 w = dst[j];
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                v8[2 * u] = o[8 * j + 2 * u] * inv_l + bf16lo(ww[u]);
+                v8[2 * u + 1] = o[8 * j + 2 * u + 1] * inv_l + bf16hi(ww[u]);
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < 8; ++u) v8[u] = o[8 * j + u] * inv_l;
+            }
+            dst[j] = make_uint4(pack_bf16x2(v8[0], v8[1]), pack_bf16x2(v8[2], v8[3]),
+                                pack_bf16x2(v8[4], v8[5]), pack_bf16x2(v8[6], v8[7]));
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 v4 = make_float4(o[4 * j] * inv_l, o[4 * j + 1] * inv_l, o[4 * j + 2] * inv_l,
+                                    o[4 * j + 3] * inv_l);
+            if (a.accumulate) {
+              const float4 w = dst[j];
+              v4.x += w.x; v4.y += w.y; v4.z += w.z; v4.w += w.w;
+            }
+            dst[j] = v4;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
+// The single-pass kernel is the default; the two-pass kernel is kept as the
+// reference design it replaced.
+constexpr bool kSinglePass = true;
+
 int launch_window_attention(const WindowAttnLaunch& L, cudaStream_t stream) {
   using namespace swa;
   const uint64_t BH = (uint64_t)L.B * L.H;
@@ -387,10 +710,17 @@ int launch_window_attention(const WindowAttnLaunch& L, cudaStream_t stream) {
   a.accumulate = L.accumulate;
   a.out = L.out;
   a.st = L.st;
-  static std::atomic<uint64_t> attr{0};
-  if (allow_dynamic_smem(window_attention_kernel, (int)SMEM, attr)) return -1;
   prof_before(K_SWA, stream);
-  window_attention_kernel<<<dim3((unsigned)(BH * a.n_qt)), dim3(THREADS), SMEM, stream>>>(m, a);
+  if (kSinglePass) {
+    static std::atomic<uint64_t> attr1{0};
+    if (allow_dynamic_smem(window_attention_1p_kernel, (int)swa1::SMEM, attr1)) return -1;
+    window_attention_1p_kernel<<<dim3((unsigned)(BH * a.n_qt)), dim3(swa1::THREADS), swa1::SMEM,
+                                 stream>>>(m, a);
+  } else {
+    static std::atomic<uint64_t> attr{0};
+    if (allow_dynamic_smem(window_attention_kernel, (int)SMEM, attr)) return -1;
+    window_attention_kernel<<<dim3((unsigned)(BH * a.n_qt)), dim3(THREADS), SMEM, stream>>>(m, a);
+  }
   prof_after(K_SWA, stream);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
