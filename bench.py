@@ -342,6 +342,50 @@ class LinearBwdBench(LinearBench):
         return c
 
 
+class LaCTBwdBench(LaCTBench):
+    """Backward pass of the LaCT layer (lact_chunk_bwd): gradients of q, k,
+    v, lr and the start weights from seeded upstream gradients dout and
+    dW_end.  Algorithmic work per token-head: 30 d dh for the chunk
+    gradient's vector-Jacobian product and 16 d dh for the read's (the
+    forward replay that keeps each chunk's start weights is not counted)."""
+
+    def __init__(self, name, device, seed):
+        super().__init__(name, device, seed)
+        torch, T = self.torch, self.T
+        from ttt_synth import make_lact_grads
+        g = make_lact_grads(self.x, cfg=self.w["cfg"], seed=seed)
+        B, H, N, d, dh = self.B, self.H, self.N, self.d, self.dh
+        self.dout = torch.from_numpy(g.dout.bits.view("int16")).view(torch.bfloat16).to(device)
+        self.dW_end = torch.from_numpy(
+            __import__("numpy").concatenate([w.ravel() for w in g.dW_end])).to(device)
+        self.state0 = T.alloc_lact_state(self.desc, device)
+        T.lact_state_init(self.desc, *self.W, 0, self.state0)
+        self.grads = [torch.empty(B, H, N, d, device=device), torch.empty(B, H, N, d, device=device),
+                      torch.empty(B, H, N, d, device=device), torch.empty(B, H, N, device=device),
+                      torch.empty(3 * B * H * d * dh, device=device)]
+        self.ws = T.alloc_workspace(T.lact_bwd_workspace_bytes(self.desc), device)
+        self.out = None
+
+    def flops_per_step(self):
+        return 46 * self.d * self.dh * self.N * self.B * self.H
+
+    def kernel_flops_per_step(self):
+        return {}
+
+    def step(self, stream):
+        self.T.lact_chunk_bwd(self.desc, self.q, self.k, self.v, self.lr, self.state0, self.dout,
+                              self.dW_end, *self.grads, self.ws, stream=stream)
+
+    def resident_bytes(self):
+        return sum(t.numel() * t.element_size() for t in
+                   [self.q, self.k, self.v, self.lr, self.dout] + self.grads)
+
+    def config(self):
+        c = super().config()
+        c["pass"] = "backward"
+        return c
+
+
 def capture_graph(bench, stream):
     """Capture one step (state init + layer call) in a CUDA graph; replaying
     it removes host launch overhead from the timed region."""
@@ -359,7 +403,7 @@ def make_bench(name, device, seed):
     w = WORKLOADS[name]
     if w["kind"] == "linear":
         return (LinearBwdBench if w.get("backward") else LinearBench)(name, device, seed)
-    return LaCTBench(name, device, seed)
+    return (LaCTBwdBench if w.get("backward") else LaCTBench)(name, device, seed)
 
 
 # --------------------------------------------------------------------------- timing
@@ -611,7 +655,7 @@ def main():
     ap.add_argument("--workload", default="lact_causal_n32k")
     ap.add_argument("--secondary", default="ttt_linear_bf16_n32k")
     ap.add_argument("--extra", default="lact_bidir_196k,lact_bidir_muon_1m,lact_w2only_causal_n32k,"
-                    "ttt_linear_bwd_bf16_n32k,lact_layer_causal_n32k",
+                    "ttt_linear_bwd_bf16_n32k,lact_layer_causal_n32k,lact_bwd_causal_n32k",
                     help="further workloads timed once each (comma list, or none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",

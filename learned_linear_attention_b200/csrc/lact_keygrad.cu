@@ -120,7 +120,6 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
     tma_prefetch_desc(&maps.w1);
     tma_prefetch_desc(&maps.w3);
     tma_prefetch_desc(&maps.w2);
-    tma_prefetch_desc(&maps.q);
   }
   tc_fence_before();
   __syncthreads();
@@ -191,18 +190,14 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
           tma_load_3d(smem + OFF_W13 + atom * HALF + HALF / 2, &maps.w3, w_full, atom * 64, j0, bh);
           tma_load_3d(smem + OFF_W2 + atom * 8192, &maps.w2, w_full, j0, atom * 64, bh);
         }
-        // warm L2 with the item's later tiles, key tiles and then query
-        // tiles; their loads then hit it
-        const int nq = a.queries ? nt : 0;
+        // warm L2 with the item's later tiles; their loads then hit it
         for (int i = 2; i < nt; ++i)
           for (int h = 0; h < 2; ++h) {
             const int row = a.t0 + (grp * a.tiles_per_group + i) * BM;
             tma_prefetch_l2_3d(&maps.k, h * 64, row, bh);
             tma_prefetch_l2_3d(&maps.v, h * 64, row, bh);
           }
-        for (int i = 0; i < nq; ++i)
-          for (int h = 0; h < 2; ++h)
-            tma_prefetch_l2_3d(&maps.q, h * 64, a.t0 + (grp * a.tiles_per_group + i) * BM, bh);
+        const int nq = a.queries ? nt : 0;
         for (int i = item_ctr == 0 ? pre : 0; ok && i < nt + nq; ++i, ++tile) {
           const uint32_t s = tile & 1;
           if (tile >= 2 && !W.wait(&kv_empty[s], ((tile >> 1) - 1) & 1, 2)) { ok = false; break; }

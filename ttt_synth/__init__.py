@@ -211,6 +211,10 @@ WORKLOADS = {
                                     order="causal", qk_norm=True, v_norm=False,
                                     lr_kind="0.01softplus", opt="gd", update_mask=4,
                                     normalize_rows=False, cfg=3),
+    # the backward pass of that layer (upstream gradients from make_lact_grads)
+    "lact_bwd_causal_n32k": dict(kind="lact", B=2, H=4, N=32768, d=128, dh=256, chunk=2048,
+                                 order="causal", qk_norm=True, v_norm=False,
+                                 lr_kind="0.01softplus", opt="gd", backward=True, cfg=3),
     # the full language layer at that shape: memory + causal sliding-window
     # attention with the 760M model's 2048-token window ("Lenguaje")
     "lact_layer_causal_n32k": dict(kind="lact", B=2, H=4, N=32768, d=128, dh=256, chunk=2048,
@@ -223,6 +227,12 @@ WORKLOADS = {
                                chunk=65536, order="bidirectional", qk_norm=True, v_norm=True,
                                lr_kind="0.01sig", opt="muon", beta=0.9, ns_steps=5,
                                cfg=5),
+    # the first two 64K chunks of that scene: the same kernels on a case small
+    # enough to profile (a few hundred MB on the device)
+    "lact_bidir_muon_128k": dict(kind="lact", B=1, H=2, N=131072, Nq=8040, d=384, dh=768,
+                                 chunk=65536, order="bidirectional", qk_norm=True, v_norm=True,
+                                 lr_kind="0.01sig", opt="muon", beta=0.9, ns_steps=5,
+                                 cfg=5),
 }
 
 
