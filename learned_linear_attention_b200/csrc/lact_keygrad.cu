@@ -67,6 +67,12 @@ TTT_DEVICE_INLINE float sigmoid_tanh(float x) {
   return fmaf(0.5f, t, 0.5f);
 }
 
+TTT_DEVICE_INLINE void mbar_arrive_n(uint64_t* bar, uint32_t n) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
+}
+TTT_DEVICE_INLINE void named_bar_sync(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 __global__ void __launch_bounds__(kg::THREADS, 1)
     lact_keygrad_kernel(const __grid_constant__ KeyGradMaps maps, const KeyGradArgs a) {
   using namespace kg;
@@ -165,15 +171,17 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
           tma_load_3d(st + TILE + HALF, &maps.v, &kv_full[s], 64, row, bh);
         }
       };
-      // the first item's first two tiles go out before the wait for the
-      // preceding kernels: they overlap that kernel's tail
+      // the first item's first tile goes out before the wait for the
+      // preceding kernels (it overlaps that kernel's tail); its second one
+      // follows the weights, so the weights do not queue behind 128 KB of
+      // token tiles
       int pre = 0;
       if ((int)blockIdx.x < n_items) {
         int bh, hb, grp;
         decode(blockIdx.x, bh, hb, grp);
         const int nt = group_tiles(grp);
         const int n_all = nt + (a.queries ? nt : 0);
-        for (; pre < 2 && pre < n_all; ++pre, ++tile) issue_tile(tile, pre, nt, bh, grp);
+        for (; pre < 1 && pre < n_all; ++pre, ++tile) issue_tile(tile, pre, nt, bh, grp);
       }
       pdl_wait();
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++item_ctr) {
@@ -189,6 +197,11 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
           tma_load_3d(smem + OFF_W13 + atom * HALF, &maps.w1, w_full, atom * 64, j0, bh);
           tma_load_3d(smem + OFF_W13 + atom * HALF + HALF / 2, &maps.w3, w_full, atom * 64, j0, bh);
           tma_load_3d(smem + OFF_W2 + atom * 8192, &maps.w2, w_full, j0, atom * 64, bh);
+        }
+        if (item_ctr == 0 && pre == 1 && nt + (a.queries ? nt : 0) > 1) {   // second tile
+          issue_tile(tile, 1, nt, bh, grp);
+          ++tile;
+          ++pre;
         }
         // warm L2 with the item's later tiles; their loads then hit it
         for (int i = 2; i < nt; ++i)
@@ -306,8 +319,8 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
             t_idle = 0;
             continue;
           }
-          // back off: this warp shares its scheduler with epilogue warps
-          __nanosleep(32);
+          // plain polling (a short sleep here measured slower: every issue on
+          // the per-tile chain waits for the wake-up)
           if ((++spins & 255u) == 0u) {   // bounded: give up after the wait timeout
             if (W.aborted()) { ok = false; break; }
             const uint64_t now = globaltimer_ns();
@@ -389,63 +402,90 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         tc_fence_before();
         mbar_arrive(dh_ready);
       }
-      if (!ok) break;
-      if (nt == 0) continue;
-      // item's gradients complete: partial sums -> their token-group slot
-      if (!W.wait(g_full, item_ctr & 1, 10)) break;
-      tc_fence_after();
-      {
-        const int j0 = hb * HB + cg * CW;
-        const size_t mat_stride = (size_t)a.BH * a.dh * D;
-        const size_t slot = (size_t)grp * mat_stride;
-        float g1[CW], g3[CW], g2[CW];
-        tmem_ld16(tmem + lane_base + TM_G13 + cg * CW, g1);
-        tmem_ld16(tmem + lane_base + TM_G13 + HB + cg * CW, g3);
-        tmem_ld16(tmem + lane_base + TM_G2 + cg * CW, g2);
-        tc_fence_before();
-        mbar_arrive(g_empty);
-        // G1, G3 [BH][dh][d]: this thread is d row r -> element (j0 + j, r)
-        float* p1 = a.part[0] + slot + ((size_t)bh * a.dh + j0) * D + r;
-        float* p3 = a.part[1] + slot + ((size_t)bh * a.dh + j0) * D + r;
+      // After the key tiles the epilogue splits: column groups 0-1 move the
+      // item's gradient sums to its token-group slot while groups 2-3 form
+      // the query tiles' Aq, each for all 64 hidden columns (two 16-column
+      // blocks per warp), so the two streams of stores overlap.
+      if (ok && nt > 0) {
+        if (cg < 2) {
+          if (!W.wait(g_full, item_ctr & 1, 10)) {
+            ok = false;
+          } else {
+            tc_fence_after();
+            const size_t mat_stride = (size_t)a.BH * a.dh * D;
+            const size_t slot = (size_t)grp * mat_stride;
 #pragma unroll
-        for (int j = 0; j < CW; ++j) {
-          p1[(size_t)j * D] = g1[j];
-          p3[(size_t)j * D] = g3[j];
-        }
-        // G2 [BH][d][dh]: row r, columns j0 .. j0 + CW - 1
-        float4* p2 = reinterpret_cast<float4*>(a.part[2] + slot + ((size_t)bh * D + r) * a.dh + j0);
+            for (int h = 0; h < 2; ++h) {
+              const int c0 = (cg * 2 + h) * CW;
+              const int j0 = hb * HB + c0;
+              uint32_t g1[CW], g3[CW], g2[CW];
+              tmem_ld16_issue(tmem + lane_base + TM_G13 + c0, g1);
+              tmem_ld16_issue(tmem + lane_base + TM_G13 + HB + c0, g3);
+              tmem_ld16_issue(tmem + lane_base + TM_G2 + c0, g2);
+              tmem_wait_ld();
+              if (h == 1) {
+                tc_fence_before();
+                mbar_arrive_n(g_empty, 2);
+              }
+              // G1, G3 [BH][dh][d]: this thread is d row r -> element (j0 + j, r)
+              float* p1 = a.part[0] + slot + ((size_t)bh * a.dh + j0) * D + r;
+              float* p3 = a.part[1] + slot + ((size_t)bh * a.dh + j0) * D + r;
 #pragma unroll
-        for (int j = 0; j < CW / 4; ++j) p2[j] = make_float4(g2[4 * j], g2[4 * j + 1], g2[4 * j + 2], g2[4 * j + 3]);
-      }
-      // query tiles (causal): Aq = silu(Q W1_J^T) * (Q W3_J^T) -> bf16
-      for (int i = 0; i < nq; ++i, ++tile) {
-        const int tc = (grp * a.tiles_per_group + i) * BM + r;
-        const bool valid = tc < a.C;
-        if (!W.wait(&acc_full[tile & 1], (tile >> 1) & 1, 11)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t rh1[CW], rh3[CW];
-        const uint32_t tb = tmem + lane_base + cg * CW + ((tile & 1) ? TM_H13B : TM_H13A);
-        tmem_ld16_issue(tb, rh1);
-        tmem_ld16_issue(tb + 64, rh3);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&acc_empty[tile & 1]);
-        if (valid) {
-          uint32_t oq[CW / 2];
+              for (int j = 0; j < CW; ++j) {
+                p1[(size_t)j * D] = __uint_as_float(g1[j]);
+                p3[(size_t)j * D] = __uint_as_float(g3[j]);
+              }
+              // G2 [BH][d][dh]: row r, columns j0 .. j0 + CW - 1
+              float4* p2 = reinterpret_cast<float4*>(a.part[2] + slot + ((size_t)bh * D + r) * a.dh + j0);
 #pragma unroll
-          for (int j = 0; j < CW; j += 2) {
-            const float x0 = __uint_as_float(rh1[j]), x1 = __uint_as_float(rh1[j + 1]);
-            const float a0 = x0 * sigmoid_tanh(x0) * __uint_as_float(rh3[j]);
-            const float a1 = x1 * sigmoid_tanh(x1) * __uint_as_float(rh3[j + 1]);
-            oq[j >> 1] = pack_bf16x2(a0, a1);
+              for (int j = 0; j < CW / 4; ++j)
+                p2[j] = make_float4(__uint_as_float(g2[4 * j]), __uint_as_float(g2[4 * j + 1]),
+                                    __uint_as_float(g2[4 * j + 2]), __uint_as_float(g2[4 * j + 3]));
+            }
           }
-          uint4* dq = reinterpret_cast<uint4*>(a.Aq + (size_t)bh * a.aq_bs + (size_t)tc * a.dh +
-                                               hb * HB + cg * CW);
+          tile += nq;
+        } else {
+          // query tiles (causal): Aq = silu(Q W1^T) * (Q W3^T) -> bf16
+          for (int i = 0; i < nq; ++i, ++tile) {
+            const int tc = (grp * a.tiles_per_group + i) * BM + r;
+            const bool valid = tc < a.C;
+            if (!W.wait(&acc_full[tile & 1], (tile >> 1) & 1, 11)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-          for (int j = 0; j < CW / 8; ++j) dq[j] = make_uint4(oq[4 * j], oq[4 * j + 1], oq[4 * j + 2], oq[4 * j + 3]);
+            for (int h = 0; h < 2; ++h) {
+              const int c0 = ((cg - 2) * 2 + h) * CW;
+              uint32_t rh1[CW], rh3[CW];
+              const uint32_t tb = tmem + lane_base + c0 + ((tile & 1) ? TM_H13B : TM_H13A);
+              tmem_ld16_issue(tb, rh1);
+              tmem_ld16_issue(tb + 64, rh3);
+              tmem_wait_ld();
+              if (h == 1) {
+                tc_fence_before();
+                mbar_arrive_n(&acc_empty[tile & 1], 2);
+              }
+              if (valid) {
+                uint32_t oq[CW / 2];
+#pragma unroll
+                for (int j = 0; j < CW; j += 2) {
+                  const float x0 = __uint_as_float(rh1[j]), x1 = __uint_as_float(rh1[j + 1]);
+                  const float a0 = x0 * sigmoid_tanh(x0) * __uint_as_float(rh3[j]);
+                  const float a1 = x1 * sigmoid_tanh(x1) * __uint_as_float(rh3[j + 1]);
+                  oq[j >> 1] = pack_bf16x2(a0, a1);
+                }
+                uint4* dq = reinterpret_cast<uint4*>(a.Aq + (size_t)bh * a.aq_bs + (size_t)tc * a.dh +
+                                                     hb * HB + c0);
+#pragma unroll
+                for (int j = 0; j < CW / 8; ++j) dq[j] = make_uint4(oq[4 * j], oq[4 * j + 1], oq[4 * j + 2], oq[4 * j + 3]);
+              }
+            }
+          }
         }
       }
-      if (!ok) break;
+      // both halves finish the item before either starts the next one, so no
+      // epilogue warp waits on an accumulator phase two uses ahead; every
+      // epilogue thread reaches this barrier, also after a failed wait
+      named_bar_sync(1, EPI_WARPS * 32);
+      if (!ok || W.aborted()) break;
     }
   }
   // dependents (the row update) may start launching once this CTA is done
