@@ -61,12 +61,77 @@ TTT_DEVICE_INLINE void tma_prefetch_l2_3d(const CUtensorMap* m, int x, int y, in
                : "memory");
 }
 
-TTT_DEVICE_INLINE float sigmoid_tanh(float x) {
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
-  return fmaf(0.5f, t, 0.5f);
-}
 
+// Epilogue operand arithmetic on two hidden columns of one token row at a
+// time, with the packed two-lane fp32 instructions of sm_100 (each lane
+// rounds exactly like the scalar instruction), so the per-tile math issues
+// about half as many instructions.  sg = sigmoid(x) = 0.5 tanh(x / 2) + 0.5.
+// Key tiles, with the row's -eta and dGr = g:
+//   dH3 = -eta g silu(x),  Gm' = -eta silu(x) y,
+//   dH1 = -eta g sg y (1 + x (1 - sg))  (x (1 - sg) = x - silu(x)).
+TTT_DEVICE_INLINE void key_ops_x2(uint32_t x0, uint32_t x1, uint32_t y0, uint32_t y1, uint32_t g0,
+                                  uint32_t g1, float neta, uint32_t& o1, uint32_t& o3, uint32_t& om) {
+  asm("{\n\t"
+      ".reg .b64 X, Y, G, N, HF, H, T, SG, XS, NX, NG, Q, QY, U, A;\n\t"
+      ".reg .f32 h0, h1, t0, t1, a0, a1;\n\t"
+      ".reg .b32 c;\n\t"
+      "mov.b32 c, 0f3F000000;\n\t"
+      "mov.b64 HF, {c, c};\n\t"
+      "mov.b64 X, {%3, %4};\n\t"
+      "mov.b64 Y, {%5, %6};\n\t"
+      "mov.b64 G, {%7, %8};\n\t"
+      "mov.b64 N, {%9, %9};\n\t"
+      "mul.rn.f32x2 H, X, HF;\n\t"
+      "mov.b64 {h0, h1}, H;\n\t"
+      "tanh.approx.f32 t0, h0;\n\t"
+      "tanh.approx.f32 t1, h1;\n\t"
+      "mov.b64 T, {t0, t1};\n\t"
+      "fma.rn.f32x2 SG, T, HF, HF;\n\t"
+      "mul.rn.f32x2 XS, X, SG;\n\t"
+      "mul.rn.f32x2 NX, N, XS;\n\t"
+      "mul.rn.f32x2 A, NX, G;\n\t"
+      "mov.b64 {a0, a1}, A;\n\t"
+      "cvt.rn.bf16x2.f32 %1, a1, a0;\n\t"
+      "mul.rn.f32x2 A, NX, Y;\n\t"
+      "mov.b64 {a0, a1}, A;\n\t"
+      "cvt.rn.bf16x2.f32 %2, a1, a0;\n\t"
+      "mul.rn.f32x2 NG, N, G;\n\t"
+      "mul.rn.f32x2 Q, NG, SG;\n\t"
+      "mul.rn.f32x2 QY, Q, Y;\n\t"
+      "sub.rn.f32x2 U, X, XS;\n\t"
+      "fma.rn.f32x2 A, QY, U, QY;\n\t"
+      "mov.b64 {a0, a1}, A;\n\t"
+      "cvt.rn.bf16x2.f32 %0, a1, a0;\n\t"
+      "}"
+      : "=r"(o1), "=r"(o3), "=r"(om)
+      : "r"(x0), "r"(x1), "r"(y0), "r"(y1), "r"(g0), "r"(g1), "f"(neta));
+}
+// Query tiles: Aq = silu(x) y.
+TTT_DEVICE_INLINE uint32_t query_ops_x2(uint32_t x0, uint32_t x1, uint32_t y0, uint32_t y1) {
+  uint32_t o;
+  asm("{\n\t"
+      ".reg .b64 X, Y, HF, H, T, SG, A;\n\t"
+      ".reg .f32 h0, h1, t0, t1, a0, a1;\n\t"
+      ".reg .b32 c;\n\t"
+      "mov.b32 c, 0f3F000000;\n\t"
+      "mov.b64 HF, {c, c};\n\t"
+      "mov.b64 X, {%1, %2};\n\t"
+      "mov.b64 Y, {%3, %4};\n\t"
+      "mul.rn.f32x2 H, X, HF;\n\t"
+      "mov.b64 {h0, h1}, H;\n\t"
+      "tanh.approx.f32 t0, h0;\n\t"
+      "tanh.approx.f32 t1, h1;\n\t"
+      "mov.b64 T, {t0, t1};\n\t"
+      "fma.rn.f32x2 SG, T, HF, HF;\n\t"
+      "mul.rn.f32x2 A, X, SG;\n\t"
+      "mul.rn.f32x2 A, A, Y;\n\t"
+      "mov.b64 {a0, a1}, A;\n\t"
+      "cvt.rn.bf16x2.f32 %0, a1, a0;\n\t"
+      "}"
+      : "=r"(o)
+      : "r"(x0), "r"(x1), "r"(y0), "r"(y1));
+  return o;
+}
 TTT_DEVICE_INLINE void mbar_arrive_n(uint64_t* bar, uint32_t n) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
 }
@@ -222,6 +287,8 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         for (uint32_t i = first; i < tile; ++i) W.drain(&kv_full[i & 1], (i >> 1) & 1);
       }
     }
+    // the other lanes wait here for lane 0 (not at the block barrier below)
+    __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     // One thread issues every MMA.  Within an item it polls the readiness of
@@ -337,6 +404,7 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
       mma_commit(fin);
       W.drain(fin, 0);
     }
+    __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q4 = warp & 3;
@@ -371,24 +439,9 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         mbar_arrive(&acc_empty[tile & 1]);
         uint32_t o1[CW / 2], o3[CW / 2], om[CW / 2];
 #pragma unroll
-        for (int j = 0; j < CW; j += 2) {
-          float r1[2], r3[2], rm[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            // dG = -eta dGr;  dH3 = dG silu(x) = (dG sg) x;
-            // dH1 = dG y silu'(x) = (dG sg) y (1 + x (1 - sg));  Gm' = -eta silu(x) y
-            const float x = __uint_as_float(rh1[j + u]), y = __uint_as_float(rh3[j + u]);
-            const float sg = sigmoid_tanh(x);
-            const float p = neta * __uint_as_float(rg[j + u]) * sg;
-            const float py = p * y;
-            r3[u] = p * x;
-            r1[u] = fmaf(py, fmaf(-x, sg, x), py);
-            rm[u] = neta * (x * sg) * y;
-          }
-          o1[j >> 1] = pack_bf16x2(r1[0], r1[1]);
-          o3[j >> 1] = pack_bf16x2(r3[0], r3[1]);
-          om[j >> 1] = pack_bf16x2(rm[0], rm[1]);
-        }
+        for (int j = 0; j < CW; j += 2)
+          key_ops_x2(rh1[j], rh1[j + 1], rh3[j], rh3[j + 1], rg[j], rg[j + 1], neta, o1[j >> 1],
+                     o3[j >> 1], om[j >> 1]);
         // the previous key tile's gradient MMAs must be done reading dH
         if (ktile >= 1 && !W.wait(dh_free, (ktile - 1) & 1, 9)) { ok = false; break; }
 #pragma unroll
@@ -466,12 +519,8 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
               if (valid) {
                 uint32_t oq[CW / 2];
 #pragma unroll
-                for (int j = 0; j < CW; j += 2) {
-                  const float x0 = __uint_as_float(rh1[j]), x1 = __uint_as_float(rh1[j + 1]);
-                  const float a0 = x0 * sigmoid_tanh(x0) * __uint_as_float(rh3[j]);
-                  const float a1 = x1 * sigmoid_tanh(x1) * __uint_as_float(rh3[j + 1]);
-                  oq[j >> 1] = pack_bf16x2(a0, a1);
-                }
+                for (int j = 0; j < CW; j += 2)
+                  oq[j >> 1] = query_ops_x2(rh1[j], rh1[j + 1], rh3[j], rh3[j + 1]);
                 uint4* dq = reinterpret_cast<uint4*>(a.Aq + (size_t)bh * a.aq_bs + (size_t)tc * a.dh +
                                                      hb * HB + c0);
 #pragma unroll

@@ -150,6 +150,22 @@ def test_bf16_n32k_workload_sampled(cuda_device, out_dtype):
     assert not np.isnan(out).any()
 
 
+@pytest.mark.slow
+def test_bf16_n32k_workload_two_heads_in_full(cuda_device):
+    """Full 4x16x32768 (d = 64) workload in the launch configuration the
+    benchmark times (bf16 output, 64-token chunks): two whole (b, h) heads,
+    every token, against the token-by-token recurrence, and their end states."""
+    x = make_workload("ttt_linear_bf16_n32k")
+    out, S = run_linear(x, out_dtype="bf16")
+    for b, h in ((0, 0), (3, 15)):
+        def sl(t):
+            return t[b:b + 1, h:h + 1]
+        ref, Sref = ttt_linear_recurrent(sl(x.q.values), sl(x.k.values), sl(x.v.values), sl(x.lr))
+        assert rel_err(sl(out), ref) <= TOL_BF16
+        assert rel_err(sl(S), Sref) <= TOL_BF16
+        assert not np.isnan(sl(out)).any()
+
+
 def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
     ws = T.alloc_workspace(256)
     assert T.ttt_selftest_wait_timeout(ws, 2000) == T.TTT_OK

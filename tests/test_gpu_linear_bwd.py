@@ -107,10 +107,11 @@ def test_empty_sequence_passes_the_end_state_gradient(cuda_device):
 
 @pytest.mark.slow
 def test_bf16_n32k_workload_sampled_heads(cuda_device):
-    """The 32K-token, 64-head shape; the oracle recomputes two heads."""
+    """The 32K-token, 64-head shape; the oracle recomputes eight whole heads,
+    two per batch row, spread over the head index."""
     x = make_workload("ttt_linear_bf16_n32k")
     g = make_linear_grads(x, cfg=2)
     got = run_bwd(x, g)
-    heads = [(0, 0), (3, 15)]
+    heads = [(0, 0), (0, 9), (1, 4), (1, 13), (2, 2), (2, 11), (3, 7), (3, 15)]
     ref = oracle_bwd(x, g, heads=heads)
     _compare([np.stack([a[b, h] for b, h in heads])[None] for a in got], ref, TOL_BF16)

@@ -90,9 +90,13 @@ def test_lact_layer_memory_plus_window(cuda_device):
 @pytest.mark.slow
 def test_n32k_window_2048_sampled_positions(cuda_device):
     """The 32K-token, 8-head shape with the pages' 2048-token window; the
-    oracle recomputes sampled positions (tile edges, window edges, the end)."""
+    oracle recomputes tile edges, window edges and the end, every 61st token
+    (a stride that walks through all rows of the 128-token query tiles), and
+    two whole query tiles, one inside the first window and one far past it."""
     x = make_workload("lact_causal_n32k")
     got = run_window(x, 2048)
-    idx = [0, 127, 128, 2046, 2047, 2048, 2049, 4095, 17000, 32767]
+    edges = [0, 127, 128, 2046, 2047, 2048, 2049, 4095, 17000, 32767]
+    idx = sorted(set(edges) | set(range(0, 32768, 61)) | set(range(1024, 1152)) |
+                 set(range(20480, 20608)))
     ref = sliding_window_attention(x.q.values, x.k.values, x.v.values, 2048, t_index=idx)
     assert rel_err(got[:, :, idx], ref) <= TOL, rel_err(got[:, :, idx], ref)
