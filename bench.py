@@ -167,8 +167,11 @@ class LaCTBench:
         BH, d, dh, N, Nq = self.B * self.H, self.d, self.dh, self.N, self.Nq
         kp = (6 * N + 4 * Nq) * d * dh * BH
         kg = (12 * N + (4 * Nq if self.causal else 0)) * d * dh * BH
+        read = 2 * d * dh * Nq * BH
         return {"lact_keypass": kp, "gemm_grad": 6 * d * dh * N * BH,
-                "gemm_read": 2 * d * dh * Nq * BH, "lact_keygrad": kg,
+                "gemm_read": read, "lact_keygrad": kg,
+                # the causal chunk loop in one launch: key/gradient work and read
+                "lact_loop": kg + (read if self.causal else 0),
                 "window_attention": self.window_flops()}
 
     def resident_bytes(self):

@@ -123,6 +123,49 @@ struct Waiter {
   TTT_DEVICE_INLINE bool aborted() const { return *abort_flag != 0u; }
 };
 
+// ------------------------------------------------- grid-wide counters
+// Monotone arrival counters in global memory: a CTA publishes its writes
+// with a release add, a waiter polls with acquire loads.  Generic-proxy
+// writes that a TMA load reads later are ordered by a proxy fence on both
+// sides.
+TTT_DEVICE_INLINE unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+TTT_DEVICE_INLINE void red_release_gpu_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+TTT_DEVICE_INLINE void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until the counter reaches `target`.  False on abort (this
+// CTA's flag, or the grid-wide word `gabort` when given) or timeout; a
+// timeout records the site and raises `gabort`, so the other CTAs stop
+// waiting too.
+TTT_DEVICE_INLINE bool grid_wait(const unsigned* ctr, unsigned target, const Waiter& W,
+                                 uint32_t site, unsigned* gabort = nullptr) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if ((it & 63u) == 0u) {
+      if (W.aborted()) return false;
+      if (gabort != nullptr && *reinterpret_cast<volatile unsigned*>(gabort) != 0u) {
+        *W.abort_flag = 1u;
+        return false;
+      }
+      if (globaltimer_ns() - t0 > W.st.timeout_ns) {
+        W.fail(site);
+        if (gabort != nullptr) atomicExch(gabort, 1u);
+        return false;
+      }
+    }
+  }
+}
+
 // ----------------------------------------------------------------- PDL
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialisation may start while its predecessor drains; it must wait for the

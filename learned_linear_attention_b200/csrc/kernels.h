@@ -184,6 +184,7 @@ struct LactWorkspace {
   int nbuf;                // bf16 weight buffers (3 on the fused causal path, else 2)
   int naq;                 // Aq buffers (2 on the fused causal path, else 1)
   size_t nsctr;            // Muon: phase counter of the fused Newton-Schulz kernel
+  size_t loopctr;          // causal chunk loop: per-head arrival counters (3 BH + 2 words)
 };
 // The Newton-Schulz loop of the Muon step as one cooperative launch
 // (ns_fused.cu): `steps` quintic steps on nb matrices r x c (r <= c).
@@ -239,6 +240,31 @@ struct KeyGradLaunch {
   DevStatus st;
 };
 int keygrad_groups(int BH, int dh, int C, int max_groups);
+// The whole causal chunk sequence of a head-dim-128 GD / momentum layer in
+// one cooperative launch (lact_keygrad.cu): the fused key/gradient work, the
+// row update and the read, with grid counters between the chunks.
+struct KeyGradLoopLaunch {
+  int BH, N_in, C, dh, max_groups, cmax;
+  const void *k, *v, *q;
+  const float* lr;
+  __nv_bfloat16* Aq;          // two buffers of [BH][cmax][dh], aq_buf elements apart
+  long long aq_buf;
+  __nv_bfloat16* Wb[3][3];    // [buffer][matrix] bf16 copies, buffer 0 holds the start weights
+  float* W[3];
+  float* M[3];
+  float* part[3];             // >= groups slots of partial sums
+  int opt, normalize, mask;
+  float beta, norm_eps;
+  void* out;
+  int out_bf16;
+  unsigned* ctr;              // 3 BH + 2 words of workspace (zeroed by the launch)
+  DevStatus st;
+};
+// 0 when the chunk loop can run this shape on the current device (groups,
+// worker and reader CTA counts returned), -1 otherwise.
+int lact_loop_plan(int BH, int N_in, int C, int dh, int max_groups, int* groups, int* workers,
+                   int* readers);
+int launch_lact_loop(const KeyGradLoopLaunch& L, cudaStream_t stream);
 // The fused memory read for head dim 128 (lact_read.cu): out rows [t0, t0 + C)
 // = W2 (silu(W1 q) * (W3 q)) with bf16 weight copies, on at most max_grid CTAs.
 struct ReadFusedLaunch {
@@ -254,7 +280,8 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream);
 // ----------------------------------------------------------------- profiling
 enum KernelKind {
   K_LIN_SIMT, K_LIN_UMMA, K_LACT_CAST, K_KEYPASS, K_GEMM_READ, K_GEMM_GRAD, K_UPDATE,
-  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_LIN_SEG, K_LIN_BWD_EW, K_SWA, K_NUM
+  K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_LIN_SEG, K_LIN_BWD_EW, K_SWA, K_LOOP,
+  K_NUM
 };
 void prof_before(int kind, cudaStream_t s);
 void prof_after(int kind, cudaStream_t s);

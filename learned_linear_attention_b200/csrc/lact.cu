@@ -17,6 +17,7 @@
 // Bidirectional order: steps 1 (keys only), 3, 4 for every chunk, then the
 // queries run step 1 (queries only) and step 2 with the final weights.
 #include <algorithm>
+#include <cstdlib>
 
 #include "gemm.cuh"
 #include "kernels.h"
@@ -830,6 +831,15 @@ static int grad_splits(int BH, int d, int dh, int cmax) {
 
 // head dim 128 (dh a multiple of 64), no split operands, GD or momentum: the
 // key pass and the chunk gradient run as one fused kernel (lact_keygrad.cu)
+// The chunk-loop launch is on unless TTT_LACT_CHUNK_LOOP=0 (read once).
+bool lact_chunk_loop_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("TTT_LACT_CHUNK_LOOP");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+
 bool lact_uses_keygrad(int d, int dh, int opt, int split) {
   return d == 128 && dh % 64 == 0 && !split && opt != 2;
 }
@@ -904,6 +914,8 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
     w.gm = o; o = align256(o + BH * cmax * dh * 2);
   }
   w.part = o; o = align256(o + (size_t)w.splits * BH * 3 * d * dh * 4);
+  w.loopctr = o;
+  if (w.keygrad && causal) o = align256(o + 4 * (3 * BH + 2));
   w.rowss = w.nsx32 = w.nsxb = w.nsa32 = w.nsab = w.nsbb = o;
   if (opt == 2) {
     const size_t r = std::min(d, dh), c = std::max(d, dh);
@@ -1562,7 +1574,38 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // measured faster than a separate Q -> out read kernel on the free SMs.)
   const bool keygrad = w.keygrad != 0;
   int ci = 0;
-  for (int t0 = 0; keygrad && t0 < L.N_in; t0 += L.chunk, ++ci) {
+  // Where the shape allows, one cooperative launch runs the whole causal
+  // sequence (lact_keygrad.cu): no kernel boundary between a chunk's
+  // gradient, its row update and the next chunk, and the reads on the spare
+  // SMs.  TTT_LACT_CHUNK_LOOP=0 in the environment keeps the per-chunk
+  // launches below.
+  bool looped = false;
+  if (keygrad && L.causal && L.mode == LACT_FULL && !split && L.opt != 2 && L.N_in > 0 &&
+      L.out != nullptr && w.nbuf == 3 && w.naq == 2 && lact_chunk_loop_enabled()) {
+    int g = 0, nw = 0, nr = 0;
+    if (lact_loop_plan(BH, L.N_in, L.chunk, dh, w.splits, &g, &nw, &nr) == 0) {
+      KeyGradLoopLaunch ll{};
+      ll.BH = BH; ll.N_in = L.N_in; ll.C = L.chunk; ll.dh = dh; ll.max_groups = w.splits;
+      ll.cmax = w.cmax;
+      ll.k = L.k; ll.v = L.v; ll.q = L.q; ll.lr = L.lr;
+      ll.Aq = Aq; ll.aq_buf = (long long)BH * w.cmax * dh;
+      for (int b = 0; b < 3; ++b)
+        for (int i = 0; i < 3; ++i) ll.Wb[b][i] = wbuf[b][i];
+      for (int i = 0; i < 3; ++i) {
+        ll.W[i] = ra.W[i];
+        ll.M[i] = ra.M[i];
+        ll.part[i] = const_cast<float*>(ra.part[i]);
+      }
+      ll.opt = L.opt; ll.normalize = L.normalize_rows; ll.mask = L.update_mask;
+      ll.beta = L.beta; ll.norm_eps = L.norm_eps;
+      ll.out = L.out; ll.out_bf16 = L.out_bf16;
+      ll.ctr = reinterpret_cast<unsigned*>(ws + w.loopctr);
+      ll.st = L.st;
+      TTT_TRY(launch_lact_loop(ll, stream));
+      looped = true;
+    }
+  }
+  for (int t0 = 0; keygrad && !looped && t0 < L.N_in; t0 += L.chunk, ++ci) {
     const int C = std::min(L.chunk, L.N_in - t0);
     __nv_bfloat16* aq = Aq + (size_t)(ci % w.naq) * BH * w.cmax * dh;
     KeyGradLaunch kgl{};

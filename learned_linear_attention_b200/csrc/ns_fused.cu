@@ -60,38 +60,8 @@ struct NsFusedParams {
   DevStatus st;
 };
 
-TTT_DEVICE_INLINE unsigned ld_acquire_gpu(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-TTT_DEVICE_INLINE void red_release_gpu_add(unsigned* p, unsigned v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-TTT_DEVICE_INLINE void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 // the epilogue warps (threads 64..191) only
 TTT_DEVICE_INLINE void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-// Bounded wait until the phase counter reaches `target` (every CTA finished
-// the previous phase).  False on abort or timeout.
-TTT_DEVICE_INLINE bool grid_wait(const unsigned* ctr, unsigned target, const Waiter& W,
-                                 uint32_t site) {
-  if (ld_acquire_gpu(ctr) >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(64);
-    if (ld_acquire_gpu(ctr) >= target) return true;
-    if ((it & 63u) == 0u) {
-      if (W.aborted()) return false;
-      if (globaltimer_ns() - t0 > W.st.timeout_ns) {
-        W.fail(site);
-        return false;
-      }
-    }
-  }
-}
 
 __global__ void __launch_bounds__(nsf::THREADS, 1)
     ns_fused_kernel(const __grid_constant__ NsFusedParams P) {

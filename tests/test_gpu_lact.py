@@ -272,3 +272,66 @@ def test_muon_cuda_graph_replay_matches_eager(cuda_device):
     g.replay()
     torch.cuda.synchronize()
     assert np.array_equal(run.out.cpu().numpy(), eager)
+
+
+# ---------------------------------------------------------------- chunk loop
+# A causal head-dim-128 GD / momentum call whose items leave spare SMs runs as
+# one cooperative launch over all chunks; TTT_LACT_CHUNK_LOOP=0 keeps one
+# launch per chunk.  Both must agree.
+
+_LOOP_SCRIPT = r"""
+import sys, numpy as np
+sys.path.insert(0, sys.argv[1])
+from ttt_synth import make_lact_inputs
+from gpu_util import LaCTRun
+x = make_lact_inputs(2, 4, int(sys.argv[3]), 128, 256, chunk=1024, order="causal", cfg=47)
+run = LaCTRun(x, opt="momentum")
+out = run.run()
+W = run.weights()
+np.savez(sys.argv[2], out=out, W1=W[0], W3=W[1], W2=W[2])
+"""
+
+
+@pytest.mark.parametrize("n", [4096, 4096 + 1000])
+def test_chunk_loop_matches_per_chunk_launches(cuda_device, tmp_path, n):
+    """The same call with the chunk loop and with per-chunk launches, each
+    in a fresh process: identical arithmetic, so the outputs and weights
+    agree to rounding (bit for bit when every chunk is full), and both match
+    the oracle."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = {}
+    for mode in ("1", "0"):
+        path = tmp_path / f"loop{mode}.npz"
+        env = dict(os.environ, TTT_LACT_CHUNK_LOOP=mode)
+        r = subprocess.run([sys.executable, "-c", _LOOP_SCRIPT, os.path.join(root, "tests"), str(path), str(n)],
+                           env=env, cwd=root, capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stderr[-2000:]
+        res[mode] = np.load(path)
+    for key in ("out", "W1", "W3", "W2"):
+        a, b = res["1"][key], res["0"][key]
+        if n % 1024 == 0:
+            assert np.array_equal(a, b), (key, rel_err(a, b))
+        else:
+            assert rel_err(a, b) <= 1e-5, (key, rel_err(a, b))
+    x = make_lact_inputs(2, 4, n, 128, 256, chunk=1024, order="causal", cfg=47)
+    ref, st = _oracle(x, "momentum")
+    assert rel_err(res["1"]["out"], ref) <= TOL
+    for key, r in (("W1", st.W1), ("W3", st.W3), ("W2", st.W2)):
+        assert rel_err(res["1"][key], r) <= TOL
+
+
+def test_chunk_loop_is_one_launch(cuda_device):
+    """An eligible causal call runs as one chunk-loop launch (plus the bf16
+    weight copy), not as per-chunk kernels."""
+    import learned_linear_attention_b200 as T
+    x = make_lact_inputs(1, 2, 4096, 128, 256, chunk=1024, order="causal", cfg=48)
+    run = LaCTRun(x)
+    run.run()
+    T.ttt_profile_begin()
+    run.run()
+    prof = T.ttt_profile_end()
+    assert prof.get("lact_loop", {}).get("launches") == 1, prof
+    assert "lact_keygrad" not in prof and "lact_update" not in prof, prof
