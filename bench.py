@@ -290,6 +290,24 @@ class LinearBench:
         T.ttt_linear_fwd(self.desc, self.q, self.k, self.v, self.lr, self.S, self.out, self.ws,
                          stream=stream)
 
+    def setup_e2e(self, step_fn=None):
+        self.e2e_step = step_fn or self.step
+        torch = self.torch
+        self.p_q, self.p_k, self.p_v = (t.pin_memory() for t in (self.h_q, self.h_k, self.h_v))
+        self.p_lr = self.h_lr.pin_memory()
+        self.p_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in (self.p_q, self.p_k, self.p_v,
+                                                               self.p_lr))
+        self.d2h = self.p_out.numel() * self.p_out.element_size()
+
+    def step_e2e(self, stream):
+        self.q.copy_(self.p_q, non_blocking=True)
+        self.k.copy_(self.p_k, non_blocking=True)
+        self.v.copy_(self.p_v, non_blocking=True)
+        self.lr.copy_(self.p_lr, non_blocking=True)
+        self.e2e_step(stream)
+        self.p_out.copy_(self.out, non_blocking=True)
+
     def resident_bytes(self):
         return sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v, self.lr,
                                                           self.out))
@@ -317,8 +335,18 @@ class LinearBwdBench(LinearBench):
         B, H, N, dk, dv = self.B, self.H, self.N, self.dk, self.dv
         self.grads = [torch.empty(s, device=device) for s in
                       ((B, H, N, dk), (B, H, N, dk), (B, H, N, dv), (B, H, N), (B, H, dk, dv))]
-        self.out = None
+        self.out = self.grads[0]   # dq: the result read back in the end-to-end timing
+        self.h_dout = self.dout.cpu()
         self.ws = T.alloc_workspace(T.ttt_linear_bwd_workspace_bytes(self.desc), device)
+
+    def setup_e2e(self, step_fn=None):
+        super().setup_e2e(step_fn)
+        self.p_dout = self.h_dout.pin_memory()
+        self.h2d += self.p_dout.numel() * self.p_dout.element_size()
+
+    def step_e2e(self, stream):
+        self.dout.copy_(self.p_dout, non_blocking=True)
+        super().step_e2e(stream)
 
     def flops_per_step(self):
         return 4 * super().flops_per_step()
@@ -367,7 +395,17 @@ class LaCTBwdBench(LaCTBench):
                       torch.empty(B, H, N, d, device=device), torch.empty(B, H, N, device=device),
                       torch.empty(3 * B * H * d * dh, device=device)]
         self.ws = T.alloc_workspace(T.lact_bwd_workspace_bytes(self.desc), device)
-        self.out = None
+        self.h_dout = self.dout.cpu()
+        self.out = self.grads[0]   # dq: the result read back in the end-to-end timing
+
+    def setup_e2e(self, step_fn=None):
+        super().setup_e2e(step_fn)
+        self.p_dout = self.h_dout.pin_memory()
+        self.h2d += self.p_dout.numel() * self.p_dout.element_size()
+
+    def step_e2e(self, stream):
+        self.dout.copy_(self.p_dout, non_blocking=True)
+        super().step_e2e(stream)
 
     def flops_per_step(self):
         return 46 * self.d * self.dh * self.N * self.B * self.H

@@ -51,7 +51,10 @@ struct KeyGradArgs {
   __nv_bfloat16* Aq;     // [BH][cmax][dh] (queries)
   long long aq_bs;       // cmax * dh
   DevStatus st;
-  // ---- chunk loop (one launch runs the whole causal chunk sequence)
+};
+// Chunk loop only (one launch runs the whole causal chunk sequence); a
+// separate parameter, so the one-chunk kernel's arguments stay small.
+struct KeyGradLoopArgs {
   int n_chunks, N;       // chunks of C tokens (the last one may be shorter); tokens
   int n_workers;         // CTAs [0, n_workers) take the items, the others read out
   long long aq_buf;      // elements between the two Aq buffers
@@ -172,25 +175,25 @@ TTT_DEVICE_INLINE float kg_warp_sum(float x) {
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
 }
-TTT_DEVICE_INLINE float4 row_step(const KeyGradArgs& a, int m, size_t c, float4 u, float4 w, float& ss) {
-  if (a.opt == 1) {
-    float4 mo = *reinterpret_cast<const float4*>(a.M[m] + c);
-    mo.x = a.beta * mo.x + u.x; mo.y = a.beta * mo.y + u.y;
-    mo.z = a.beta * mo.z + u.z; mo.w = a.beta * mo.w + u.w;
-    *reinterpret_cast<float4*>(a.M[m] + c) = mo;
+TTT_DEVICE_INLINE float4 row_step(const KeyGradArgs& a, const KeyGradLoopArgs& la, int m, size_t c, float4 u, float4 w, float& ss) {
+  if (la.opt == 1) {
+    float4 mo = *reinterpret_cast<const float4*>(la.M[m] + c);
+    mo.x = la.beta * mo.x + u.x; mo.y = la.beta * mo.y + u.y;
+    mo.z = la.beta * mo.z + u.z; mo.w = la.beta * mo.w + u.w;
+    *reinterpret_cast<float4*>(la.M[m] + c) = mo;
     u = mo;
   }
   w = make_float4(w.x - u.x, w.y - u.y, w.z - u.z, w.w - u.w);
   ss += w.x * w.x + w.y * w.y + w.z * w.z + w.w * w.w;
   return w;
 }
-TTT_DEVICE_INLINE float row_scale(const KeyGradArgs& a, float ss) {
-  return a.normalize ? 1.f / fmaxf(sqrtf(kg_warp_sum(ss)), a.norm_eps) : 1.f;
+TTT_DEVICE_INLINE float row_scale(const KeyGradArgs& a, const KeyGradLoopArgs& la, float ss) {
+  return la.normalize ? 1.f / fmaxf(sqrtf(kg_warp_sum(ss)), la.norm_eps) : 1.f;
 }
-TTT_DEVICE_INLINE void row_store(const KeyGradArgs& a, int m, int nb, size_t c, float4 w, float scale) {
+TTT_DEVICE_INLINE void row_store(const KeyGradArgs& a, const KeyGradLoopArgs& la, int m, int nb, size_t c, float4 w, float scale) {
   const float4 x = make_float4(w.x * scale, w.y * scale, w.z * scale, w.w * scale);
-  *reinterpret_cast<float4*>(a.W[m] + c) = x;
-  *reinterpret_cast<uint2*>(a.Wb[nb][m] + c) = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+  *reinterpret_cast<float4*>(la.W[m] + c) = x;
+  *reinterpret_cast<uint2*>(la.Wb[nb][m] + c) = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
 }
 TTT_DEVICE_INLINE void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -204,7 +207,7 @@ TTT_DEVICE_INLINE void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint
 struct OwnRows {
   int lo13, n13, lo2, n2;
 };
-__host__ __device__ __forceinline__ OwnRows own_rows(const KeyGradArgs& a, int hb, int grp) {
+__host__ __device__ __forceinline__ OwnRows own_rows(const KeyGradArgs& a, const KeyGradLoopArgs& la, int hb, int grp) {
   const int G = a.n_groups, K = a.n_hb * G, k = hb * G + grp;
   OwnRows o;
   o.lo13 = hb * kg::HB + kg::HB * grp / G;
@@ -215,21 +218,21 @@ __host__ __device__ __forceinline__ OwnRows own_rows(const KeyGradArgs& a, int h
 }
 // bytes of one token group's partial sums for the owned rows (masked
 // matrices take no room): [W1 rows | W3 rows | W2 rows], fp32
-__host__ __device__ __forceinline__ uint32_t own_group_bytes(const KeyGradArgs& a, const OwnRows& o) {
-  return (uint32_t)(((a.mask & 1) ? o.n13 * kg::D : 0) + ((a.mask & 2) ? o.n13 * kg::D : 0) +
-                    ((a.mask & 4) ? o.n2 * a.dh : 0)) * 4u;
+__host__ __device__ __forceinline__ uint32_t own_group_bytes(const KeyGradArgs& a, const KeyGradLoopArgs& la, const OwnRows& o) {
+  return (uint32_t)(((la.mask & 1) ? o.n13 * kg::D : 0) + ((la.mask & 2) ? o.n13 * kg::D : 0) +
+                    ((la.mask & 4) ? o.n2 * a.dh : 0)) * 4u;
 }
 // one thread: bring every token group's partial sums of the owned rows into
 // shared memory (one bulk copy per group and matrix, completing on `bar`)
-TTT_DEVICE_INLINE void own_partials_load(const KeyGradArgs& a, int bh, const OwnRows& o, uint8_t* dst,
+TTT_DEVICE_INLINE void own_partials_load(const KeyGradArgs& a, const KeyGradLoopArgs& la, int bh, const OwnRows& o, uint8_t* dst,
                                          uint64_t* bar) {
   const size_t mat_stride = (size_t)a.BH * a.dh * kg::D;
-  const uint32_t gb = own_group_bytes(a, o);
+  const uint32_t gb = own_group_bytes(a, la, o);
   mbar_arrive_expect_tx(bar, gb * (uint32_t)a.n_groups);
   for (int sp = 0; sp < a.n_groups; ++sp) {
     uint8_t* d = dst + (size_t)sp * gb;
     for (int m = 0; m < 3; ++m) {
-      if (!(a.mask & (1 << m))) continue;
+      if (!(la.mask & (1 << m))) continue;
       const size_t off = m < 2 ? ((size_t)bh * a.dh + o.lo13) * kg::D : ((size_t)bh * kg::D + o.lo2) * a.dh;
       const uint32_t bytes = (uint32_t)(m < 2 ? o.n13 * kg::D : o.n2 * a.dh) * 4u;
       bulk_g2s(d, a.part[m] + sp * mat_stride + off, bytes, bar);
@@ -242,9 +245,9 @@ TTT_DEVICE_INLINE void own_partials_load(const KeyGradArgs& a, int bh, const Own
 // memory (added in token-group order): momentum, the step, the row L2 norm
 // and the fp32 / bf16 stores, the arithmetic of the stand-alone GD /
 // momentum row update.
-TTT_DEVICE_INLINE void loop_row_update(const KeyGradArgs& a, int bh, const OwnRows& o, int e, int lane,
+TTT_DEVICE_INLINE void loop_row_update(const KeyGradArgs& a, const KeyGradLoopArgs& la, int bh, const OwnRows& o, int e, int lane,
                                        int nb, const uint8_t* sp0) {
-  const uint32_t gb = own_group_bytes(a, o);
+  const uint32_t gb = own_group_bytes(a, la, o);
   auto psum = [&](uint32_t byte_off) {   // byte offset within one group's block
     float4 u = *reinterpret_cast<const float4*>(sp0 + byte_off);
     for (int sp = 1; sp < a.n_groups; ++sp) {
@@ -255,32 +258,32 @@ TTT_DEVICE_INLINE void loop_row_update(const KeyGradArgs& a, int bh, const OwnRo
   };
   uint32_t base = 0;   // this matrix's rows within a group's block
   for (int m = 0; m < 2; ++m) {
-    if (!(a.mask & (1 << m))) continue;
+    if (!(la.mask & (1 << m))) continue;
     for (int i = e; i < o.n13; i += kg::EPI_WARPS) {
       const size_t c = ((size_t)bh * a.dh + o.lo13 + i) * kg::D + 4 * lane;
-      const float4 w = *reinterpret_cast<const float4*>(a.W[m] + c);
+      const float4 w = *reinterpret_cast<const float4*>(la.W[m] + c);
       const float4 u = psum(base + (uint32_t)(i * kg::D + 4 * lane) * 4u);
       float ss = 0.f;
-      const float4 x = row_step(a, m, c, u, w, ss);
-      row_store(a, m, nb, c, x, row_scale(a, ss));
+      const float4 x = row_step(a, la, m, c, u, w, ss);
+      row_store(a, la, m, nb, c, x, row_scale(a, la, ss));
     }
     base += (uint32_t)o.n13 * kg::D * 4u;
   }
-  if (a.mask & 4) {
+  if (la.mask & 4) {
     const bool two = a.dh > 128;
     for (int i = e; i < o.n2; i += kg::EPI_WARPS) {
       const size_t c0 = ((size_t)bh * kg::D + o.lo2 + i) * a.dh + 4 * lane, c1 = c0 + 128;
       const uint32_t b0 = base + (uint32_t)(i * a.dh + 4 * lane) * 4u, b1 = b0 + 512u;
-      float4 w0 = *reinterpret_cast<const float4*>(a.W[2] + c0);
-      float4 w1 = two ? *reinterpret_cast<const float4*>(a.W[2] + c1) : w0;
+      float4 w0 = *reinterpret_cast<const float4*>(la.W[2] + c0);
+      float4 w1 = two ? *reinterpret_cast<const float4*>(la.W[2] + c1) : w0;
       const float4 u0 = psum(b0);
       const float4 u1 = two ? psum(b1) : u0;
       float ss = 0.f;
-      w0 = row_step(a, 2, c0, u0, w0, ss);
-      if (two) w1 = row_step(a, 2, c1, u1, w1, ss);
-      const float sc = row_scale(a, ss);
-      row_store(a, 2, nb, c0, w0, sc);
-      if (two) row_store(a, 2, nb, c1, w1, sc);
+      w0 = row_step(a, la, 2, c0, u0, w0, ss);
+      if (two) w1 = row_step(a, la, 2, c1, u1, w1, ss);
+      const float sc = row_scale(a, la, ss);
+      row_store(a, la, 2, nb, c0, w0, sc);
+      if (two) row_store(a, la, 2, nb, c1, w1, sc);
     }
   }
 }
@@ -299,7 +302,8 @@ TTT_DEVICE_INLINE void loop_row_update(const KeyGradArgs& a, int bh, const OwnRo
 // chunk c reuses.
 template <bool LOOP>
 __global__ void __launch_bounds__(kg::THREADS, 1)
-    lact_keygrad_kernel(const __grid_constant__ KeyGradMaps maps, const KeyGradArgs a) {
+    lact_keygrad_kernel(const __grid_constant__ KeyGradMaps maps, const KeyGradArgs a,
+                        const __grid_constant__ KeyGradLoopArgs la) {
   using namespace kg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -330,14 +334,14 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int items_per_bh = a.n_hb * a.n_groups;
   const int n_items = items_per_bh * a.BH;
-  const int n_chunks = LOOP ? a.n_chunks : 1;
-  const int stride = LOOP ? a.n_workers : (int)gridDim.x;
-  const bool reader = LOOP && (int)blockIdx.x >= a.n_workers;
-  unsigned* const gabort = LOOP ? a.ctr + 3 * a.BH + 1 : nullptr;
-  auto ctr_part = [&](int bh) { return a.ctr + bh; };
-  auto ctr_upd = [&](int bh) { return a.ctr + a.BH + bh; };
-  auto ctr_aq = [&](int bh) { return a.ctr + 2 * a.BH + bh; };
-  unsigned* const ctr_read = LOOP ? a.ctr + 3 * a.BH : nullptr;
+  const int n_chunks = LOOP ? la.n_chunks : 1;
+  const int stride = LOOP ? la.n_workers : (int)gridDim.x;
+  const bool reader = LOOP && (int)blockIdx.x >= la.n_workers;
+  unsigned* const gabort = LOOP ? la.ctr + 3 * a.BH + 1 : nullptr;
+  auto ctr_part = [&](int bh) { return la.ctr + bh; };
+  auto ctr_upd = [&](int bh) { return la.ctr + a.BH + bh; };
+  auto ctr_aq = [&](int bh) { return la.ctr + 2 * a.BH + bh; };
+  unsigned* const ctr_read = LOOP ? la.ctr + 3 * a.BH : nullptr;
   const unsigned per_head = (unsigned)items_per_bh;   // items (worker CTAs) of one head
 
   if (threadIdx.x == 0) {
@@ -396,11 +400,11 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
   // the chunk a loop iteration works on (without the loop these read the
   // arguments directly, so nothing extra stays in registers)
   auto ct0 = [&](int c) { return LOOP ? a.t0 + c * a.C : a.t0; };
-  auto cC = [&](int c) { return LOOP ? min(a.C, a.N - ct0(c)) : a.C; };
+  auto cC = [&](int c) { return LOOP ? min(a.C, la.N - ct0(c)) : a.C; };
   auto ctiles = [&](int c) { return LOOP ? (cC(c) + BM - 1) / BM : a.tiles_total; };
   auto ctpg = [&](int c) { return LOOP ? (ctiles(c) + a.n_groups - 1) / a.n_groups : a.tiles_per_group; };
   auto cwb = [&](int c) { return LOOP ? c % 3 : 0; };
-  auto caq = [&](int c) { return LOOP ? a.Aq + (size_t)(c & 1) * a.aq_buf : a.Aq; };
+  auto caq = [&](int c) { return LOOP ? a.Aq + (size_t)(c & 1) * la.aq_buf : a.Aq; };
   auto decode = [&](int item, int& bh, int& hb, int& grp) {
     hb = item % a.n_hb;
     grp = (item / a.n_hb) % a.n_groups;
@@ -416,7 +420,7 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
     // Per tile of 128 tokens: out = Aq [128 x dh] W2^T [dh -> 128], K-major
     // operands (Aq rows, W2 rows of the bf16 copy), fp32 accumulator in
     // TMEM (two buffers), 16 epilogue warps convert and store.
-    const int rr = (int)blockIdx.x - a.n_workers, R = (int)gridDim.x - a.n_workers;
+    const int rr = (int)blockIdx.x - la.n_workers, R = (int)gridDim.x - la.n_workers;
     const uint32_t A_OFF = 65536, A_STAGE = 65536;   // W2 at 0 (64 KB), two Aq stages
     const int kblocks = a.dh / 64;
     auto tile_range = [&](int c, int& lo, int& hi) {
@@ -519,15 +523,15 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
           mbar_arrive(&r_acc_empty[s]);
           const int row = mt * BM + r;
           if (row < cC(c)) {
-            const size_t base = (size_t)bh * a.out_bs + (size_t)(ct0(c) + row) * D + cg * 32;
-            if (a.out_bf16) {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base);
+            const size_t base = (size_t)bh * la.out_bs + (size_t)(ct0(c) + row) * D + cg * 32;
+            if (la.out_bf16) {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(la.out) + base);
 #pragma unroll
               for (int j = 0; j < 4; ++j)
                 dst[j] = make_uint4(pack_bf16x2(o[8 * j], o[8 * j + 1]), pack_bf16x2(o[8 * j + 2], o[8 * j + 3]),
                                     pack_bf16x2(o[8 * j + 4], o[8 * j + 5]), pack_bf16x2(o[8 * j + 6], o[8 * j + 7]));
             } else {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base);
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(la.out) + base);
 #pragma unroll
               for (int j = 0; j < 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
             }
@@ -746,7 +750,7 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         // chunk c rewrites the Aq buffer and (in its update) the W buffer of
         // chunk c - 2: the readers must be done with that chunk
         if (threadIdx.x == 64)
-          grid_wait(ctr_read, (unsigned)((int)gridDim.x - a.n_workers) * (c - 1), W, 12, gabort);
+          grid_wait(ctr_read, (unsigned)((int)gridDim.x - la.n_workers) * (c - 1), W, 12, gabort);
         named_bar_sync(1, EPI_WARPS * 32);
         if (W.aborted()) break;
       }
@@ -896,19 +900,19 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         // which waits for this update)
         int bh, hb, grp;
         decode((int)blockIdx.x, bh, hb, grp);
-        const OwnRows own = own_rows(a, hb, grp);
+        const OwnRows own = own_rows(a, la, hb, grp);
         if (threadIdx.x == 64) {
-          if (own_group_bytes(a, own) * (uint32_t)a.n_groups > LOOP_PART_BYTES) {
+          if (own_group_bytes(a, la, own) * (uint32_t)a.n_groups > LOOP_PART_BYTES) {
             W.fail(16);   // the host plan rules this out
           } else if (grid_wait(ctr_part(bh), per_head * (c + 1), W, 13, gabort)) {
             fence_proxy_async_global();
-            own_partials_load(a, bh, own, smem + OFF_W13, upd_full);
+            own_partials_load(a, la, bh, own, smem + OFF_W13, upd_full);
           }
         }
         named_bar_sync(1, EPI_WARPS * 32);
         if (W.aborted()) break;
         if (!W.wait(upd_full, c & 1, 14)) break;
-        loop_row_update(a, bh, own, warp - 2, lane, (c + 1) % 3, smem + OFF_W13);
+        loop_row_update(a, la, bh, own, warp - 2, lane, (c + 1) % 3, smem + OFF_W13);
         // the next chunk's weights: read by TMA in the head's workers
         fence_proxy_async_global();
         named_bar_sync(1, EPI_WARPS * 32);
@@ -983,7 +987,6 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream) {
   a.Aq = L.Aq;
   a.aq_bs = L.aq_bs;
   a.st = L.st;
-  a.n_chunks = 1;
   static std::atomic<uint64_t> attr{0};
   if (allow_dynamic_smem(lact_keygrad_kernel<false>, (int)kg::SMEM, attr)) return -1;
   const int items = a.n_hb * a.n_groups * L.BH;
@@ -992,7 +995,7 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream) {
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   prof_before(K_KEYGRAD, stream);
   if (launch_pdl(lact_keygrad_kernel<false>, dim3(std::min(items, sms)), dim3(kg::THREADS), kg::SMEM,
-                 stream, m, a) != cudaSuccess)
+                 stream, m, a, KeyGradLoopArgs{}) != cudaSuccess)
     return -1;
   prof_after(K_KEYGRAD, stream);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
@@ -1026,10 +1029,11 @@ int lact_loop_plan(int BH, int N_in, int C, int dh, int max_groups, int* groups,
   // update uses (all three matrices counted)
   {
     KeyGradArgs t{};
-    t.BH = BH; t.dh = dh; t.n_hb = dh / kg::HB; t.n_groups = g; t.mask = 7;
+    KeyGradLoopArgs tl{};
+    t.BH = BH; t.dh = dh; t.n_hb = dh / kg::HB; t.n_groups = g; tl.mask = 7;
     for (int hb = 0; hb < t.n_hb; ++hb)
       for (int grp = 0; grp < g; ++grp)
-        if (own_group_bytes(t, own_rows(t, hb, grp)) * (uint32_t)g > kg::LOOP_PART_BYTES) return -1;
+        if (own_group_bytes(t, tl, own_rows(t, tl, hb, grp)) * (uint32_t)g > kg::LOOP_PART_BYTES) return -1;
   }
   static std::atomic<uint64_t> attr{0};
   if (allow_dynamic_smem(lact_keygrad_kernel<true>, (int)kg::SMEM, attr)) return -1;
@@ -1062,28 +1066,29 @@ int launch_lact_loop(const KeyGradLoopLaunch& L, cudaStream_t stream) {
                           (uint64_t)L.dh * 2, (uint64_t)L.cmax * L.dh * 2, 64, 128))
       return -1;
   KeyGradArgs a{};
+  KeyGradLoopArgs la{};
   a.BH = L.BH; a.C = L.C; a.t0 = 0; a.lr_len = L.N_in; a.dh = L.dh;
   a.n_hb = L.dh / kg::HB;
   a.n_groups = g;
   a.lr = L.lr;
   for (int i = 0; i < 3; ++i) {
     a.part[i] = L.part[i];
-    a.W[i] = L.W[i];
-    a.M[i] = L.M[i];
-    for (int b = 0; b < 3; ++b) a.Wb[b][i] = L.Wb[b][i];
+    la.W[i] = L.W[i];
+    la.M[i] = L.M[i];
+    for (int b = 0; b < 3; ++b) la.Wb[b][i] = L.Wb[b][i];
   }
   a.queries = 1;
   a.Aq = L.Aq;
   a.aq_bs = (long long)L.cmax * L.dh;
-  a.aq_buf = L.aq_buf;
+  la.aq_buf = L.aq_buf;
   a.st = L.st;
-  a.n_chunks = (L.N_in + L.C - 1) / L.C;
-  a.N = L.N_in;
-  a.n_workers = nw;
-  a.ctr = L.ctr;
-  a.opt = L.opt; a.normalize = L.normalize; a.mask = L.mask;
-  a.beta = L.beta; a.norm_eps = L.norm_eps;
-  a.out = L.out; a.out_bf16 = L.out_bf16; a.out_bs = (long long)L.N_in * kg::D;
+  la.n_chunks = (L.N_in + L.C - 1) / L.C;
+  la.N = L.N_in;
+  la.n_workers = nw;
+  la.ctr = L.ctr;
+  la.opt = L.opt; la.normalize = L.normalize; la.mask = L.mask;
+  la.beta = L.beta; la.norm_eps = L.norm_eps;
+  la.out = L.out; la.out_bf16 = L.out_bf16; la.out_bs = (long long)L.N_in * kg::D;
   if (cudaMemsetAsync(L.ctr, 0, (3 * (size_t)L.BH + 2) * sizeof(unsigned), stream) != cudaSuccess) return -1;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(nw + nr);
@@ -1096,7 +1101,7 @@ int launch_lact_loop(const KeyGradLoopLaunch& L, cudaStream_t stream) {
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
   prof_before(K_LOOP, stream);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, lact_keygrad_kernel<true>, m, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, lact_keygrad_kernel<true>, m, a, la);
   prof_after(K_LOOP, stream);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
