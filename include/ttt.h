@@ -244,7 +244,13 @@ int lact_state_readout(const lact_desc* desc, const void* state, float* W1, floa
  * k, v: [B,H,N_in,d]; lr: [B,H,N_in]; state in/out; out: [B,H,N_in,d]
  * (causal) or [B,H,N_q,d] (bidirectional).  A causal call may be followed by
  * another call on the continuation of the sequence with the same state;
- * chunk boundaries restart at every call. */
+ * chunk boundaries restart at every call.  A causal call with d = 128, GD
+ * or momentum and no split operands runs every chunk in one cooperative
+ * launch that takes every SM of the device (its CTAs wait on one another
+ * through counters in the workspace, each wait bounded); the environment
+ * variable TTT_LACT_CHUNK_LOOP=0, read once per process, keeps one launch
+ * per chunk.  Both give the same result (bit for bit when every chunk is
+ * full). */
 int lact_chunk_fwd(const lact_desc* desc, const void* q, const void* k, const void* v,
                    const float* lr, void* state, void* out, void* ws, size_t ws_bytes,
                    void* stream);
