@@ -198,6 +198,250 @@ __global__ void bwd_dv_kernel(int BH, int C, int cmax, int d, int N, int t0, con
   if (lane == 0) dlr[tok] = -acc;
 }
 
+
+// dW[m] += sum over the splits of the split-K partial products (the three
+// weight-gradient matrices of a chunk, each [BH][splits][rows x cols]).
+struct WgradSumArgs {
+  int BH, splits;
+  long long mat;             // rows x cols of one head's matrix (equal for the three)
+  const float* part[3];
+  float* dW[3];              // [BH][rows x cols]
+};
+__global__ void bwd_wgrad_sum_kernel(WgradSumArgs a) {
+  const long long per = (long long)a.BH * a.mat / 4;   // float4 per matrix
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < 3 * per;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int m = (int)(i / per);
+    const long long e = (i % per) * 4;
+    const long long b = e / a.mat, o = e % a.mat;
+    const float* src = a.part[m] + (b * a.splits) * a.mat + o;
+    float4 u = *reinterpret_cast<float4*>(a.dW[m] + e);
+    for (int sp = 0; sp < a.splits; ++sp) {
+      const float4 x = *reinterpret_cast<const float4*>(src + sp * a.mat);
+      u.x += x.x; u.y += x.y; u.z += x.z; u.w += x.w;
+    }
+    *reinterpret_cast<float4*>(a.dW[m] + e) = u;
+  }
+}
+
+// ---------------------------------------------------------------- fused forward products + elementwise step
+// d = 128.  One CTA per (head, 128-token tile, 64 hidden units J): all
+// operands in shared memory at once, the products into TMEM, then the
+// elementwise step of the chain rule straight from TMEM to the bf16 outputs
+// (no fp32 intermediates in memory).
+//   key:  [h1 | h3] = K [W1_J; W3_J]^T, [r1 | r3] = K [R1_J; R3_J]^T,
+//         [vw2 | vr2] = V [W2[:, J] | R2[:, J]]  -> d_h1, d_h3, d_dg, -lr d_dg,
+//         e1, e3, g (the chunk gradient's VJP step above)
+//   read: [hq1 | hq3] = Q [W1_J; W3_J]^T, dgq = dout W2[:, J] -> (dgq hq3 s),
+//         (dgq aq), gq
+namespace bf {
+constexpr int BM = 128, HB = 64, D = 128;
+constexpr uint32_t ATILE = BM * D * 2;      // 32 KB: 128 token rows x 128 d, two 64-column boxes
+constexpr uint32_t B2 = 2 * HB * D * 2;     // 32 KB: two weight blocks of 64 hidden x 128 d
+constexpr uint32_t OFF_A0 = 0, OFF_A1 = ATILE, OFF_B13 = 2 * ATILE, OFF_R13 = OFF_B13 + B2,
+                   OFF_B2 = OFF_R13 + B2;
+constexpr uint32_t OFF_BAR_KEY = OFF_B2 + B2, OFF_BAR_READ = OFF_R13;   // read: [W1|W3], then W2 alone
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr uint32_t SMEM_KEY = OFF_BAR_KEY + 256 + 1024, SMEM_READ = OFF_BAR_READ + 16384 + 256 + 1024;
+constexpr uint32_t TM_COLS = 512;
+}  // namespace bf
+
+struct BwdFwdMaps {
+  CUtensorMap a0, a1;        // K / V (key) or Q / dout (read): token maps, box {64, 128}
+  CUtensorMap w1, w3, w2;    // bf16 weights: W1, W3 box {64 d, 64 rows}; W2 box {64 hidden, 64 d rows}
+  CUtensorMap r1, r3, r2;    // key: bf16 R (same shapes)
+};
+struct BwdFwdArgs {
+  int BH, C, cmax, dh, t0, lr_len, n_mt, key;
+  const float* lr;           // key: [BH][lr_len]
+  __nv_bfloat16* out[7];     // [BH][cmax][dh]: key d_h1, d_h3, d_dg, d_dgn, e1, e3, g; read dhq1, dhq3, gq
+  DevStatus st;
+};
+
+__global__ void __launch_bounds__(bf::THREADS, 1)
+    bwd_fwd_fused_kernel(const __grid_constant__ BwdFwdMaps maps, const BwdFwdArgs a) {
+  using namespace bf;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const bool key = a.key != 0;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (key ? OFF_BAR_KEY : OFF_BAR_READ + 16384));
+  uint64_t* acc_full = full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_hb = a.dh / HB;
+  const int mt = blockIdx.x % a.n_mt, hb = (blockIdx.x / a.n_mt) % n_hb, bh = blockIdx.x / (a.n_mt * n_hb);
+  const int j0 = hb * HB;
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  Waiter W{abort_flag, a.st, 400};
+  if (warp == 0) {
+    if (lane == 0) {
+      const int row = a.t0 + mt * BM;
+      const uint32_t bytes = key ? 2 * ATILE + 3 * B2 : 2 * ATILE + B2 + B2 / 2;
+      mbar_arrive_expect_tx(full, bytes);
+      for (int h = 0; h < 2; ++h) {
+        tma_load_3d(smem + OFF_A0 + h * (ATILE / 2), &maps.a0, full, h * 64, row, bh);
+        tma_load_3d(smem + OFF_A1 + h * (ATILE / 2), &maps.a1, full, h * 64, row, bh);
+      }
+      // K-major weight blocks: atom h (d 64h .. 64h + 63) = [first 64 rows | second 64 rows]
+      for (int h = 0; h < 2; ++h) {
+        tma_load_3d(smem + OFF_B13 + h * (B2 / 2), &maps.w1, full, h * 64, j0, bh);
+        tma_load_3d(smem + OFF_B13 + h * (B2 / 2) + B2 / 4, &maps.w3, full, h * 64, j0, bh);
+      }
+      // MN-major W2[:, J] (and R2[:, J]): 128 d rows of 64 hidden units, two 64-row boxes
+      uint8_t* b2 = smem + (key ? OFF_B2 : OFF_R13);
+      for (int h = 0; h < 2; ++h) tma_load_3d(b2 + h * (B2 / 4), &maps.w2, full, j0, h * 64, bh);
+      if (key) {
+        for (int h = 0; h < 2; ++h) {
+          tma_load_3d(smem + OFF_R13 + h * (B2 / 2), &maps.r1, full, h * 64, j0, bh);
+          tma_load_3d(smem + OFF_R13 + h * (B2 / 2) + B2 / 4, &maps.r3, full, h * 64, j0, bh);
+          tma_load_3d(b2 + B2 / 2 + h * (B2 / 4), &maps.r2, full, j0, h * 64, bh);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      if (W.wait(full, 0, 1)) {
+        tc_fence_after();
+        const uint32_t id_k = make_idesc(128, 128, false, false);          // K-major B, N = 128
+        const uint32_t id_mn = make_idesc(128, key ? 128 : 64, false, true);   // MN-major B
+        const uint64_t da0 = make_sdesc(smem_u32(smem + OFF_A0), 16, 1024);
+        const uint64_t da1 = make_sdesc(smem_u32(smem + OFF_A1), 16, 1024);
+        const uint64_t db13 = make_sdesc(smem_u32(smem + OFF_B13), 16, 1024);
+        const uint64_t dr13 = make_sdesc(smem_u32(smem + OFF_R13), 16, 1024);
+        // [W2_J | R2_J]: two 64-wide N blocks 16 KB apart
+        const uint64_t db2 = make_sdesc(smem_u32(smem + (key ? OFF_B2 : OFF_R13)), B2 / 2, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * (ATILE / 2) + (kk & 3) * 32;
+          const uint32_t offb = (kk >> 2) * (B2 / 2) + (kk & 3) * 32;
+          mma_bf16(tmem, sdesc_add(da0, off), sdesc_add(db13, offb), id_k, kk > 0);
+          if (key) mma_bf16(tmem + 128, sdesc_add(da0, off), sdesc_add(dr13, offb), id_k, kk > 0);
+          mma_bf16(tmem + 256, sdesc_add(da1, off), sdesc_add(db2, kk * 2048), id_mn, kk > 0);
+        }
+        mma_commit(acc_full);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q4 = warp & 3;
+    const int cg = (warp - 2) >> 2;                 // 32 hidden columns of the 64
+    const int r = q4 * 32 + lane;
+    const int tok = mt * BM + r;                    // row of the chunk
+    const bool valid = tok < a.C;
+    const uint32_t lb = (uint32_t)(q4 * 32) << 16;
+    const float eta = (key && valid) ? a.lr[(size_t)bh * a.lr_len + a.t0 + tok] : 0.f;
+    const bool ok = W.wait(acc_full, 0, 2);
+    if (ok) tc_fence_after();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t c0 = (uint32_t)(cg * 32 + h * 16);
+      uint32_t x1[16], x3[16], x5[16], y1[16], y3[16], y5[16];
+      // every lane takes part in the warp-collective loads
+      tmem_ld16_issue(tmem + lb + c0, x1);            // h1 / hq1
+      tmem_ld16_issue(tmem + lb + 64 + c0, x3);       // h3 / hq3
+      tmem_ld16_issue(tmem + lb + 256 + c0, x5);      // vw2 / dgq
+      if (key) {
+        tmem_ld16_issue(tmem + lb + 128 + c0, y1);    // r1
+        tmem_ld16_issue(tmem + lb + 192 + c0, y3);    // r3
+        tmem_ld16_issue(tmem + lb + 320 + c0, y5);    // vr2
+      }
+      tmem_wait_ld();
+      const size_t base = ((size_t)bh * a.cmax + tok) * a.dh + j0 + c0;
+      if (key) {
+        uint32_t o[7][8];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          float v[7][2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            float vdh1 = 0.f, vdh3 = 0.f, vddg = 0.f, vddgn = 0.f, ve1 = 0.f, ve3 = 0.f, vg = 0.f;
+            if (valid && ok) {
+              const float x = __uint_as_float(x1[j + u]), y = __uint_as_float(x3[j + u]);
+              const float sg = sig(x);
+              const float act = x * sg;
+              const float s1 = sg * (1.f + x * (1.f - sg));
+              const float s2 = sg * (1.f - sg) * (2.f + x * (1.f - 2.f * sg));
+              const float dg = -eta * __uint_as_float(x5[j + u]), r2 = -eta * __uint_as_float(y5[j + u]);
+              const float r1 = __uint_as_float(y1[j + u]), r3 = __uint_as_float(y3[j + u]);
+              vdh3 = r2 * act + dg * s1 * r1;
+              vdh1 = (r2 * y + dg * r3) * s1 + dg * y * r1 * s2;
+              vddg = act * r3 + y * s1 * r1;
+              vddgn = -eta * vddg;
+              ve1 = dg * y * s1;
+              ve3 = dg * act;
+              vg = act * y;
+            }
+            v[0][u] = vdh1; v[1][u] = vdh3; v[2][u] = vddg; v[3][u] = vddgn;
+            v[4][u] = ve1; v[5][u] = ve3; v[6][u] = vg;
+          }
+#pragma unroll
+          for (int q = 0; q < 7; ++q) o[q][j >> 1] = pack_bf16x2(v[q][0], v[q][1]);
+        }
+#pragma unroll
+        for (int q = 0; q < 7; ++q) {
+          uint4* dst = reinterpret_cast<uint4*>(a.out[q] + base);
+          dst[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
+          dst[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
+        }
+      } else {
+        uint32_t o[3][8];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          float v[3][2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            float v1 = 0.f, v3 = 0.f, vg = 0.f;
+            if (valid && ok) {
+              const float x = __uint_as_float(x1[j + u]), y = __uint_as_float(x3[j + u]);
+              const float dg = __uint_as_float(x5[j + u]);
+              const float sg = sig(x);
+              const float act = x * sg;
+              v1 = dg * y * sg * (1.f + x * (1.f - sg));
+              v3 = dg * act;
+              vg = act * y;
+            }
+            v[0][u] = v1; v[1][u] = v3; v[2][u] = vg;
+          }
+#pragma unroll
+          for (int q = 0; q < 3; ++q) o[q][j >> 1] = pack_bf16x2(v[q][0], v[q][1]);
+        }
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+          uint4* dst = reinterpret_cast<uint4*>(a.out[q] + base);
+          dst[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
+          dst[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    // an aborted CTA: the copies it issued land before it leaves
+    if (*abort_flag && lane == 0) W.drain(full, 0);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
 }  // namespace
 
 LactBwdWorkspace lact_bwd_layout(const LactLaunch& f) {
@@ -320,6 +564,22 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
   // cin of an accumulating GEMM is read at row m (no row offset), so
   // accumulating outputs always start at row 0 of their buffer
 
+  // split-K MN-major product into `o` [BH][splits][M][N] (no accumulation)
+  auto gemm_split = [&](const CUtensorMap* A, const CUtensorMap* B, int np, int M, int N, int kps,
+                        int S, float* o, int ak, int bk) -> int {
+    GemmMaps m{};
+    GemmArgs g = gemm_args_default(L.st);
+    for (int i = 0; i < np; ++i) {
+      m.a[i] = A[i];
+      m.b[i] = B[i];
+      g.a_k_off[i] = ak;
+      g.b_k_off[i] = bk;
+    }
+    g.npairs = np; g.M = M; g.N = N; g.batch = BH; g.k_steps = kps; g.splits = S;
+    g.o32 = o; g.ld32 = N; g.o32_ss = (long long)M * N; g.o32_bs = (long long)S * M * N;
+    return gemm_launch(GEMM_AMN_BMN, m, g, stream, K_GEMM_GRAD);
+  };
+
   CUtensorMap mq_k{}, mq_mn{}, mk_k{}, mk_mn{}, mv_k{}, mv_mn{}, mdo_k{}, mdo_mn{};
   if (f.N_in > 0) {
     BWD_TRY(tok(&mk_k, f.k, f.N_in, 128));
@@ -345,31 +605,73 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
   CUtensorMap mb_k[7], mb_mn[7];
   for (int i = 0; i < 7; ++i) BWD_TRY(inter(&mb_k[i], b16[i], 128) | inter(&mb_mn[i], b16[i], 64));
   const long long ibs = (long long)w.cmax * dh;
+  // d = 128: the forward products and the elementwise step of a chunk in one
+  // kernel (bwd_fwd_fused_kernel); other shapes take the GEMMs + elementwise
+  // kernels below
+  const bool fused_fwd = d == 128 && dh % 64 == 0;
+  // the read VJP's bf16 dhq1, dhq3, gq on the fused path: in the fp32
+  // intermediates' memory (each region holds two bf16 buffers), so a causal
+  // chunk's key and read steps can feed the same weight-gradient products
+  __nv_bfloat16* rb16[3];
+  CUtensorMap mrb_k[3], mrb_mn[3];
+  for (int i = 0; i < 3; ++i) {
+    rb16[i] = reinterpret_cast<__nv_bfloat16*>(f32[i]);
+    BWD_TRY(inter(&mrb_k[i], rb16[i], 128) | inter(&mrb_mn[i], rb16[i], 64));
+  }
+  static std::atomic<uint64_t> fused_attr{0};
+  if (fused_fwd && allow_dynamic_smem(bwd_fwd_fused_kernel, (int)bf::SMEM_KEY, fused_attr)) return -1;
+  auto fused = [&](bool key, const CUtensorMap& a0, const CUtensorMap& a1, int t0, int C) -> int {
+    BwdFwdMaps m{};
+    m.a0 = a0; m.a1 = a1;
+    m.w1 = mW1mn; m.w3 = mW3mn; m.w2 = mW2mn;
+    m.r1 = mR1mn; m.r3 = mR3mn; m.r2 = mR2mn;
+    BwdFwdArgs ba{};
+    ba.BH = BH; ba.C = C; ba.cmax = w.cmax; ba.dh = dh; ba.t0 = t0; ba.lr_len = f.N_in;
+    ba.n_mt = w.cmax / bf::BM; ba.key = key ? 1 : 0; ba.lr = f.lr; ba.st = L.st;
+    for (int i = 0; i < 7; ++i) ba.out[i] = key ? Hb(w.b16[i]) : (i < 3 ? rb16[i] : nullptr);
+    prof_before(K_BWD_FWD, stream);
+    bwd_fwd_fused_kernel<<<dim3((unsigned)(ba.n_mt * (dh / bf::HB) * BH)), dim3(bf::THREADS),
+                           key ? bf::SMEM_KEY : bf::SMEM_READ, stream>>>(m, ba);
+    prof_after(K_BWD_FWD, stream);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  };
+
   float* dW1 = dW;
   float* dW3 = dW + mat;
   float* dW2 = dW + 2 * mat;
   const long long w13bs = (long long)dh * d, w2bs = (long long)d * dh;
 
+  // dq rows [t0, t0 + C) = dhq1 W1 + dhq3 W3  (M = C, N = d, K = dh)
+  auto read_dq = [&](int t0, int C) -> int {
+    const CUtensorMap A[2] = {fused_fwd ? mrb_k[0] : mb_k[0], fused_fwd ? mrb_k[1] : mb_k[1]},
+                      B[2] = {mW1mn, mW3mn};
+    return gemm(GEMM_AK_BMN, A, B, 2, C, d, dh / 64, L.dq, d, (long long)q_rows * d, false, t0,
+                0, 0, 0);
+  };
   // read VJP for query rows [t0, t0 + C) with the weights in Wb: dq rows and dW
   auto read_vjp = [&](int t0, int C) -> int {
     const int ks = (C + 63) / 64;
-    // hq1 = Q W1^T, hq3 = Q W3^T, dgq = dout W2   (M = C, N = dh, K = d)
-    BWD_TRY(gemm(GEMM_AK_BK, &mq_k, &mW1k, 1, C, dh, d / 64, f32[0], dh, ibs, false, 0, t0, 0, 0));
-    BWD_TRY(gemm(GEMM_AK_BK, &mq_k, &mW3k, 1, C, dh, d / 64, f32[1], dh, ibs, false, 0, t0, 0, 0));
-    BWD_TRY(gemm(GEMM_AK_BMN, &mdo_k, &mW2mn, 1, C, dh, d / 64, f32[2], dh, ibs, false, 0, t0, 0, 0));
-    ReadEwArgs ra{BH, C, w.cmax, dh, f32[0], f32[1], f32[2], b16[0], b16[1], b16[6]};
-    const size_t n = (size_t)BH * w.cmax * dh;
-    bwd_read_ew_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 8192), 256, 0, stream>>>(ra);
-    BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    if (fused_fwd) {
+      BWD_TRY(fused(false, mq_k, mdo_k, t0, C));
+    } else {
+      // hq1 = Q W1^T, hq3 = Q W3^T, dgq = dout W2   (M = C, N = dh, K = d)
+      BWD_TRY(gemm(GEMM_AK_BK, &mq_k, &mW1k, 1, C, dh, d / 64, f32[0], dh, ibs, false, 0, t0, 0, 0));
+      BWD_TRY(gemm(GEMM_AK_BK, &mq_k, &mW3k, 1, C, dh, d / 64, f32[1], dh, ibs, false, 0, t0, 0, 0));
+      BWD_TRY(gemm(GEMM_AK_BMN, &mdo_k, &mW2mn, 1, C, dh, d / 64, f32[2], dh, ibs, false, 0, t0, 0, 0));
+      ReadEwArgs ra{BH, C, w.cmax, dh, f32[0], f32[1], f32[2], b16[0], b16[1], b16[6]};
+      const size_t n = (size_t)BH * w.cmax * dh;
+      bwd_read_ew_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 8192), 256, 0, stream>>>(ra);
+      BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    }
+    const CUtensorMap& dhq1_mn = fused_fwd ? mrb_mn[0] : mb_mn[0];
+    const CUtensorMap& dhq3_mn = fused_fwd ? mrb_mn[1] : mb_mn[1];
+    const CUtensorMap& gq_mn = fused_fwd ? mrb_mn[2] : mb_mn[6];
     // dW1 += dhq1^T Q, dW3 += dhq3^T Q  (M = dh, N = d, K = C tokens)
-    BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[0], &mq_mn, 1, dh, d, ks, dW1, d, w13bs, true, 0, 0, 0, t0));
-    BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[1], &mq_mn, 1, dh, d, ks, dW3, d, w13bs, true, 0, 0, 0, t0));
+    BWD_TRY(gemm(GEMM_AMN_BMN, &dhq1_mn, &mq_mn, 1, dh, d, ks, dW1, d, w13bs, true, 0, 0, 0, t0));
+    BWD_TRY(gemm(GEMM_AMN_BMN, &dhq3_mn, &mq_mn, 1, dh, d, ks, dW3, d, w13bs, true, 0, 0, 0, t0));
     // dW2 += dout^T gq  (M = d, N = dh)
-    BWD_TRY(gemm(GEMM_AMN_BMN, &mdo_mn, &mb_mn[6], 1, d, dh, ks, dW2, dh, w2bs, true, 0, 0, t0, 0));
-    // dq rows = dhq1 W1 + dhq3 W3  (M = C, N = d, K = dh)
-    const CUtensorMap A[2] = {mb_k[0], mb_k[1]}, B[2] = {mW1mn, mW3mn};
-    return gemm(GEMM_AK_BMN, A, B, 2, C, d, dh / 64, L.dq, d, (long long)q_rows * d, false, t0,
-                0, 0, 0);
+    BWD_TRY(gemm(GEMM_AMN_BMN, &mdo_mn, &gq_mn, 1, d, dh, ks, dW2, dh, w2bs, true, 0, 0, t0, 0));
+    return read_dq(t0, C);
   };
 
   // ---------------------------------------------------------------- 2. reverse
@@ -395,18 +697,26 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     bwd_row_step_kernel<<<(row_warps * 32 + 255) / 256, 256, 0, stream>>>(rs);
     BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     BWD_TRY(cast(wsave + (size_t)c * 3 * mat, Wb, 3 * mat));
-    // h1 = K W1^T, h3 = K W3^T, vw2 = V W2, r1 = K R1^T, r3 = K R3^T, vr2 = V R2
-    BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mW1k, 1, C, dh, d / 64, f32[0], dh, ibs, false, 0, t0, 0, 0));
-    BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mW3k, 1, C, dh, d / 64, f32[1], dh, ibs, false, 0, t0, 0, 0));
-    BWD_TRY(gemm(GEMM_AK_BMN, &mv_k, &mW2mn, 1, C, dh, d / 64, f32[2], dh, ibs, false, 0, t0, 0, 0));
-    BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mR1k, 1, C, dh, d / 64, f32[3], dh, ibs, false, 0, t0, 0, 0));
-    BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mR3k, 1, C, dh, d / 64, f32[4], dh, ibs, false, 0, t0, 0, 0));
-    BWD_TRY(gemm(GEMM_AK_BMN, &mv_k, &mR2mn, 1, C, dh, d / 64, f32[5], dh, ibs, false, 0, t0, 0, 0));
-    KeyEwArgs ka{BH, C, w.cmax, dh, f.N_in, t0, f.lr, f32[0], f32[1], f32[2], f32[3], f32[4], f32[5],
-                 b16[0], b16[1], b16[2], b16[3], b16[4], b16[5], b16[6]};
-    const size_t n = (size_t)BH * w.cmax * dh;
-    bwd_key_ew_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 8192), 256, 0, stream>>>(ka);
-    BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    // a causal chunk on the fused path: the read's elementwise step too, so
+    // both feed the weight-gradient products below
+    const bool both = fused_fwd && f.causal;
+    if (fused_fwd) {
+      BWD_TRY(fused(true, mk_k, mv_k, t0, C));
+      if (both) BWD_TRY(fused(false, mq_k, mdo_k, t0, C));
+    } else {
+      // h1 = K W1^T, h3 = K W3^T, vw2 = V W2, r1 = K R1^T, r3 = K R3^T, vr2 = V R2
+      BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mW1k, 1, C, dh, d / 64, f32[0], dh, ibs, false, 0, t0, 0, 0));
+      BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mW3k, 1, C, dh, d / 64, f32[1], dh, ibs, false, 0, t0, 0, 0));
+      BWD_TRY(gemm(GEMM_AK_BMN, &mv_k, &mW2mn, 1, C, dh, d / 64, f32[2], dh, ibs, false, 0, t0, 0, 0));
+      BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mR1k, 1, C, dh, d / 64, f32[3], dh, ibs, false, 0, t0, 0, 0));
+      BWD_TRY(gemm(GEMM_AK_BK, &mk_k, &mR3k, 1, C, dh, d / 64, f32[4], dh, ibs, false, 0, t0, 0, 0));
+      BWD_TRY(gemm(GEMM_AK_BMN, &mv_k, &mR2mn, 1, C, dh, d / 64, f32[5], dh, ibs, false, 0, t0, 0, 0));
+      KeyEwArgs ka{BH, C, w.cmax, dh, f.N_in, t0, f.lr, f32[0], f32[1], f32[2], f32[3], f32[4], f32[5],
+                   b16[0], b16[1], b16[2], b16[3], b16[4], b16[5], b16[6]};
+      const size_t n = (size_t)BH * w.cmax * dh;
+      bwd_key_ew_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 8192), 256, 0, stream>>>(ka);
+      BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+    }
     // dk rows = d_h1 W1 + d_h3 W3 + e1 R1, then + e3 R3   (M = C, N = d, K = dh)
     {
       const CUtensorMap A[3] = {mb_k[0], mb_k[1], mb_k[4]}, B[3] = {mW1mn, mW3mn, mR1mn};
@@ -419,10 +729,31 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     BWD_TRY(cudaMemcpy2DAsync(L.dk + (size_t)t0 * d, (size_t)f.N_in * d * 4, F(w.ddy),
                               (size_t)w.cmax * d * 4, (size_t)C * d * 4, BH, cudaMemcpyDeviceToDevice,
                               stream) == cudaSuccess ? 0 : -1);
-    // weight gradients: dW1 += d_h1^T K, dW3 += d_h3^T K, dW2 += V^T (-lr d_dg)
-    BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[0], &mk_mn, 1, dh, d, ks, dW1, d, w13bs, true, 0, 0, 0, t0));
-    BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[1], &mk_mn, 1, dh, d, ks, dW3, d, w13bs, true, 0, 0, 0, t0));
-    BWD_TRY(gemm(GEMM_AMN_BMN, &mv_mn, &mb_mn[3], 1, d, dh, ks, dW2, dh, w2bs, true, 0, 0, t0, 0));
+    // weight gradients: dW1 += d_h1^T K, dW3 += d_h3^T K, dW2 += V^T (-lr d_dg);
+    // with `both`, plus the read's dhq1^T Q, dhq3^T Q, dout^T gq as second pairs
+    {
+      const int np = both ? 2 : 1;
+      const CUtensorMap A1[2] = {mb_mn[0], mrb_mn[0]}, A3[2] = {mb_mn[1], mrb_mn[1]}, B13[2] = {mk_mn, mq_mn};
+      const CUtensorMap A2[2] = {mv_mn, mdo_mn}, B2m[2] = {mb_mn[3], mrb_mn[2]};
+      if (fused_fwd) {
+        // split-K over the chunk's tokens into the (free) fp32 intermediates,
+        // then one pass adds the splits to dW: 16 output tiles per matrix
+        // would leave most SMs idle.  Steps past the chunk read zero rows.
+        // (each split's partial is d x dh per head: S splits fit the region while S d <= cmax)
+        const int S = std::max(1, std::min(std::min(8, ks), w.cmax / d)), kps = (ks + S - 1) / S;
+        BWD_TRY(gemm_split(A1, B13, np, dh, d, kps, S, f32[3], 0, t0));
+        BWD_TRY(gemm_split(A3, B13, np, dh, d, kps, S, f32[4], 0, t0));
+        BWD_TRY(gemm_split(A2, B2m, np, d, dh, kps, S, f32[5], t0, 0));
+        WgradSumArgs sa{BH, S, (long long)d * dh, {f32[3], f32[4], f32[5]}, {dW1, dW3, dW2}};
+        const long long n4 = 3LL * BH * d * dh / 4;
+        bwd_wgrad_sum_kernel<<<(unsigned)std::min<long long>((n4 + 255) / 256, 4096), 256, 0, stream>>>(sa);
+        BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+      } else {
+        BWD_TRY(gemm(GEMM_AMN_BMN, A1, B13, np, dh, d, ks, dW1, d, w13bs, true, 0, 0, 0, t0));
+        BWD_TRY(gemm(GEMM_AMN_BMN, A3, B13, np, dh, d, ks, dW3, d, w13bs, true, 0, 0, 0, t0));
+        BWD_TRY(gemm(GEMM_AMN_BMN, A2, B2m, np, d, dh, ks, dW2, dh, w2bs, true, 0, 0, t0, 0));
+      }
+    }
     // d_dy = d_dg W2^T + g R2^T   (M = C, N = d, K = dh)
     {
       const CUtensorMap A[2] = {mb_k[2], mb_k[6]}, B[2] = {mW2k, mR2k};
@@ -436,7 +767,8 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
           L.dv, L.dlr);
       BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     }
-    if (f.causal) BWD_TRY(read_vjp(t0, C));
+    if (both) BWD_TRY(read_dq(t0, C));
+    else if (f.causal) BWD_TRY(read_vjp(t0, C));
   }
   return cudaMemcpyAsync(L.dW0, dW, 3 * mat * 4, cudaMemcpyDeviceToDevice, stream) == cudaSuccess
              ? 0 : -1;

@@ -12,7 +12,7 @@ static const char* kKindNames[K_NUM] = {
     "ttt_linear_simt", "ttt_linear_umma", "lact_cast",     "lact_keypass",
     "gemm_read",       "gemm_grad",       "lact_update",   "muon_momentum",
     "ns_prep",         "gemm_ns",         "muon_apply",    "lact_keygrad",
-    "ttt_linear_segstate", "ttt_linear_bwd_ew", "window_attention", "lact_loop"};
+    "ttt_linear_segstate", "ttt_linear_bwd_ew", "window_attention", "lact_loop", "lact_bwd_fwd"};
 
 struct ProfRec {
   int kind;
