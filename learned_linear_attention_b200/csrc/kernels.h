@@ -258,6 +258,8 @@ struct KeyGradLoopLaunch {
   void* out;
   int out_bf16;
   unsigned* ctr;              // 3 BH + 2 words of workspace (zeroed by the launch)
+  int cast_first;             // the kernel writes the start weights' bf16 copies (every buffer
+                              // for a matrix the update leaves alone) before the first chunk
   DevStatus st;
 };
 // 0 when the chunk loop can run this shape on the current device (groups,

@@ -1119,7 +1119,17 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // never updated (update_mask): then every buffer must hold it
   ra.nbuf = (L.update_mask & 7) == 7 ? 1 : nbuf;
   ra.buf_stride = wsz;
-  if (L.mode != LACT_APPLY) {   // the update of an APPLY call writes its own copies
+  // Where the shape allows, one cooperative launch runs the whole causal
+  // sequence (lact_keygrad.cu): no kernel boundary between a chunk's
+  // gradient, its row update and the next chunk, and the reads on the spare
+  // SMs; it also makes the start weights' bf16 copies itself.
+  // TTT_LACT_CHUNK_LOOP=0 in the environment keeps the per-chunk launches.
+  int loop_g = 0, loop_nw = 0, loop_nr = 0;
+  const bool use_loop = w.keygrad && L.causal && L.mode == LACT_FULL && !split && L.opt != 2 &&
+                        L.N_in > 0 && L.out != nullptr && w.nbuf == 3 && w.naq == 2 &&
+                        lact_chunk_loop_enabled() &&
+                        lact_loop_plan(BH, L.N_in, L.chunk, dh, w.splits, &loop_g, &loop_nw, &loop_nr) == 0;
+  if (L.mode != LACT_APPLY && !use_loop) {   // the update of an APPLY call writes its own copies
     prof_before(K_LACT_CAST, stream);
     if (launch_pdl(lact_cast_kernel, dim3(row_blocks), dim3(256), 0, stream, ra) != cudaSuccess)
       return -1;
@@ -1574,16 +1584,10 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // measured faster than a separate Q -> out read kernel on the free SMs.)
   const bool keygrad = w.keygrad != 0;
   int ci = 0;
-  // Where the shape allows, one cooperative launch runs the whole causal
-  // sequence (lact_keygrad.cu): no kernel boundary between a chunk's
-  // gradient, its row update and the next chunk, and the reads on the spare
-  // SMs.  TTT_LACT_CHUNK_LOOP=0 in the environment keeps the per-chunk
-  // launches below.
+  // the chunk loop (decided above, before the bf16 copies)
   bool looped = false;
-  if (keygrad && L.causal && L.mode == LACT_FULL && !split && L.opt != 2 && L.N_in > 0 &&
-      L.out != nullptr && w.nbuf == 3 && w.naq == 2 && lact_chunk_loop_enabled()) {
-    int g = 0, nw = 0, nr = 0;
-    if (lact_loop_plan(BH, L.N_in, L.chunk, dh, w.splits, &g, &nw, &nr) == 0) {
+  if (use_loop) {
+    {
       KeyGradLoopLaunch ll{};
       ll.BH = BH; ll.N_in = L.N_in; ll.C = L.chunk; ll.dh = dh; ll.max_groups = w.splits;
       ll.cmax = w.cmax;
@@ -1600,6 +1604,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       ll.beta = L.beta; ll.norm_eps = L.norm_eps;
       ll.out = L.out; ll.out_bf16 = L.out_bf16;
       ll.ctr = reinterpret_cast<unsigned*>(ws + w.loopctr);
+      ll.cast_first = 1;
       ll.st = L.st;
       TTT_TRY(launch_lact_loop(ll, stream));
       looped = true;

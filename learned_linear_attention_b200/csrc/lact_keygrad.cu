@@ -70,6 +70,8 @@ struct KeyGradLoopArgs {
   void* out;             // [BH][N][128] bf16 or fp32
   int out_bf16;
   long long out_bs;      // N * 128
+  int cast_first;        // workers write the start weights' bf16 copies first (counted
+                         // on the heads' update counters like an update)
 };
 struct KeyGradMaps {
   CUtensorMap k, v, q;
@@ -245,6 +247,21 @@ TTT_DEVICE_INLINE void own_partials_load(const KeyGradArgs& a, const KeyGradLoop
 // memory (added in token-group order): momentum, the step, the row L2 norm
 // and the fp32 / bf16 stores, the arithmetic of the stand-alone GD /
 // momentum row update.
+TTT_DEVICE_INLINE void loop_cast_rows(const KeyGradArgs& a, const KeyGradLoopArgs& la, int bh,
+                                      const OwnRows& o, int e, int lane) {
+  for (int m = 0; m < 3; ++m) {
+    const int n = m < 2 ? o.n13 : o.n2, cols = m < 2 ? kg::D : a.dh;
+    const size_t row0 = m < 2 ? (size_t)bh * a.dh + o.lo13 : (size_t)bh * kg::D + o.lo2;
+    const int nb = (la.mask & (1 << m)) ? 1 : 3;
+    for (int i = e; i < n; i += kg::EPI_WARPS)
+      for (int c = 4 * lane; c < cols; c += 128) {
+        const size_t off = (row0 + i) * cols + c;
+        const float4 x = *reinterpret_cast<const float4*>(la.W[m] + off);
+        const uint2 h = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+        for (int b = 0; b < nb; ++b) *reinterpret_cast<uint2*>(la.Wb[b][m] + off) = h;
+      }
+  }
+}
 TTT_DEVICE_INLINE void loop_row_update(const KeyGradArgs& a, const KeyGradLoopArgs& la, int bh, const OwnRows& o, int e, int lane,
                                        int nb, const uint8_t* sp0) {
   const uint32_t gb = own_group_bytes(a, la, o);
@@ -584,8 +601,9 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
             ++tile;
           }
           if (c == 0 && item_ctr == 0) pdl_wait();
-          if (LOOP && c > 0 && item == (int)blockIdx.x) {   // the head's row updates of chunk c - 1
-            if (!grid_wait(ctr_upd(bh), per_head * c, W, 3, gabort)) { ok = false; break; }
+          if (LOOP && (c > 0 || la.cast_first) && item == (int)blockIdx.x) {
+            // the head's row updates of chunk c - 1 (and the start copies)
+            if (!grid_wait(ctr_upd(bh), per_head * (c + la.cast_first), W, 3, gabort)) { ok = false; break; }
             fence_proxy_async_global();
           }
           if (item_ctr >= 1 && !W.wait(w_empty, (item_ctr - 1) & 1, 1)) { ok = false; break; }
@@ -745,6 +763,16 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
     uint8_t* dh1s = smem + OFF_DH;
     const uint32_t dh1 = smem_u32(dh1s), dh3 = dh1 + HALF, gms = dh1 + 2 * HALF;
     uint32_t tile = 0, ktile = 0, item_ctr = 0;
+    if (LOOP && la.cast_first) {
+      // the start weights' bf16 copies of the owned rows (buffer 0, and every
+      // buffer for a matrix the update leaves alone), published like an update
+      int bh, hb, grp;
+      decode((int)blockIdx.x, bh, hb, grp);
+      loop_cast_rows(a, la, bh, own_rows(a, la, hb, grp), warp - 2, lane);
+      fence_proxy_async_global();
+      named_bar_sync(1, EPI_WARPS * 32);
+      if (threadIdx.x == 64) red_release_gpu_add(ctr_upd(bh), 1u);
+    }
     for (int c = 0; c < n_chunks; ++c) {
       if (LOOP && c >= 2) {
         // chunk c rewrites the Aq buffer and (in its update) the W buffer of
@@ -1089,6 +1117,7 @@ int launch_lact_loop(const KeyGradLoopLaunch& L, cudaStream_t stream) {
   la.opt = L.opt; la.normalize = L.normalize; la.mask = L.mask;
   la.beta = L.beta; la.norm_eps = L.norm_eps;
   la.out = L.out; la.out_bf16 = L.out_bf16; la.out_bs = (long long)L.N_in * kg::D;
+  la.cast_first = L.cast_first;
   if (cudaMemsetAsync(L.ctr, 0, (3 * (size_t)L.BH + 2) * sizeof(unsigned), stream) != cudaSuccess) return -1;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(nw + nr);
