@@ -378,6 +378,36 @@ __global__ void __launch_bounds__(swa::THREADS, 1)
 // O is divided by l once, at the end.  Each key tile costs one Q K^T and one
 // P V product and one exponential per score.
 // ---------------------------------------------------------------------------
+// (x0, x1) -> (2^(s x0 + b), 2^(s x1 + b)): one packed two-lane fp32 FMA
+// (sm_100 f32x2, each lane rounded like the scalar instruction) and the
+// hardware base-2 exponential per lane (ex2.approx, a few ulp; the result
+// is rounded to bf16 next).  2^-inf = 0 for masked columns.
+TTT_DEVICE_INLINE float2 exp2_scaled_x2(float x0, float x1, float sc, float b) {
+  float2 r;
+  asm("{\n\t.reg .b64 X, S, B, T;\n\t.reg .f32 t0, t1;\n\t"
+      "mov.b64 X, {%2, %3};\n\t"
+      "mov.b64 S, {%4, %4};\n\t"
+      "mov.b64 B, {%5, %5};\n\t"
+      "fma.rn.f32x2 T, X, S, B;\n\t"
+      "mov.b64 {t0, t1}, T;\n\t"
+      "ex2.approx.ftz.f32 %0, t0;\n\t"
+      "ex2.approx.ftz.f32 %1, t1;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(x0), "f"(x1), "f"(sc), "f"(b));
+  return r;
+}
+TTT_DEVICE_INLINE float2 add_x2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 A, B, R;\n\t"
+      "mov.b64 A, {%2, %3};\n\t"
+      "mov.b64 B, {%4, %5};\n\t"
+      "add.rn.f32x2 R, A, B;\n\t"
+      "mov.b64 {%0, %1}, R;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
 namespace swa1 {
 constexpr int D = 128, BM = 128, BN = 128;
 constexpr uint32_t HALF = 128 * 64 * 2;
@@ -560,22 +590,22 @@ __global__ void __launch_bounds__(swa1::THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&s_empty[s]);
+      // the row maximum on the raw scores (the scale is positive), masked
+      // keys set to -inf
       float mx = -INFINITY;
       if (inside(kt)) {
 #pragma unroll
-        for (int j = 0; j < BN; ++j) {
-          x[j] *= a.scale_log2;
-          mx = fmaxf(mx, x[j]);
-        }
+        for (int j = 0; j < BN; ++j) mx = fmaxf(mx, x[j]);
       } else {
 #pragma unroll
         for (int j = 0; j < BN; ++j) {
           const int kj = kt * BN + j;
           const bool valid = row_ok && kj <= qi && kj > qi - a.window;
-          x[j] = valid ? x[j] * a.scale_log2 : -INFINITY;
+          x[j] = valid ? x[j] : -INFINITY;
           mx = fmaxf(mx, x[j]);
         }
       }
+      mx *= a.scale_log2;
       // lazy rescale: keep m unless the tile raises it by more than RESCALE
       float alpha = 1.f;
       if (mx > m + RESCALE || (m == -INFINITY && mx != -INFINITY)) {
@@ -614,12 +644,16 @@ __global__ void __launch_bounds__(swa1::THREADS, 1)
 #pragma unroll
         for (int j = 0; j < BN / 2; ++j) pk[j] = 0u;
       } else {
+        // two columns per packed fp32 instruction: t = scale x - m, then
+        // the hardware base-2 exponential of each lane
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < BN; j += 2) {
-          const float p0 = exp2f(x[j] - m), p1 = exp2f(x[j + 1] - m);
-          add += p0 + p1;
-          pk[j >> 1] = pack_bf16x2(p0, p1);
+          const float2 p = exp2_scaled_x2(x[j], x[j + 1], a.scale_log2, -m);
+          acc = add_x2(acc, p);
+          pk[j >> 1] = pack_bf16x2(p.x, p.y);
         }
+        add = acc.x + acc.y;
       }
       l += add;
       // P buffer s is free once the P V product of tile g - 2 is done (its own
