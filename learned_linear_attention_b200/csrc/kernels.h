@@ -258,6 +258,7 @@ struct KeyGradLoopLaunch {
   void* out;
   int out_bf16;
   unsigned* ctr;              // 3 BH + 2 words of workspace (zeroed by the launch)
+  int groups, workers, readers;   // from lact_loop_plan (0: the launch plans itself)
   int cast_first;             // the kernel writes the start weights' bf16 copies (every buffer
                               // for a matrix the update leaves alone) before the first chunk
   DevStatus st;

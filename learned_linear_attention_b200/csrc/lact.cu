@@ -1605,6 +1605,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       ll.out = L.out; ll.out_bf16 = L.out_bf16;
       ll.ctr = reinterpret_cast<unsigned*>(ws + w.loopctr);
       ll.cast_first = 1;
+      ll.groups = loop_g; ll.workers = loop_nw; ll.readers = loop_nr;
       ll.st = L.st;
       TTT_TRY(launch_lact_loop(ll, stream));
       looped = true;

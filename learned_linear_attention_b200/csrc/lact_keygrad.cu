@@ -1077,8 +1077,10 @@ int lact_loop_plan(int BH, int N_in, int C, int dh, int max_groups, int* groups,
 }
 
 int launch_lact_loop(const KeyGradLoopLaunch& L, cudaStream_t stream) {
-  int g = 0, nw = 0, nr = 0;
-  if (lact_loop_plan(L.BH, L.N_in, L.C, L.dh, L.max_groups, &g, &nw, &nr)) return -1;
+  // the caller's plan (lact_loop_plan), else this call's
+  int g = L.groups, nw = L.workers, nr = L.readers;
+  if ((g <= 0 || nw <= 0 || nr <= 0) && lact_loop_plan(L.BH, L.N_in, L.C, L.dh, L.max_groups, &g, &nw, &nr))
+    return -1;
   KeyGradMaps m{};
   if (keygrad_maps(m, L.BH, L.N_in, L.dh, L.k, L.v, L.q)) return -1;
   const uint64_t BH = (uint64_t)L.BH;
