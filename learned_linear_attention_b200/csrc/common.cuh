@@ -148,8 +148,8 @@ TTT_DEVICE_INLINE bool grid_wait(const unsigned* ctr, unsigned target, const Wai
                                  uint32_t site, unsigned* gabort = nullptr) {
   if (ld_acquire_gpu(ctr) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
+  // plain polling (one thread per CTA waits)
   for (uint32_t it = 1;; ++it) {
-    __nanosleep(64);
     if (ld_acquire_gpu(ctr) >= target) return true;
     if ((it & 63u) == 0u) {
       if (W.aborted()) return false;

@@ -351,8 +351,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
           t_idle = 0;
           continue;
         }
-        // back off: this warp shares its scheduler with epilogue warps
-        __nanosleep(32);
+        // plain polling: a sleep here put its wake-up on the per-tile chain
         if ((++spins & 255u) == 0u) {   // bounded: give up after the wait timeout
           if (W.aborted()) break;
           const uint64_t now = globaltimer_ns();
