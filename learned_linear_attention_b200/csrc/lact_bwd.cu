@@ -44,6 +44,12 @@ namespace {
 
 TTT_DEVICE_INLINE float sig(float x) { return 1.f / (1.f + __expf(-x)); }
 
+int num_sms_bwd() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 // bf16 copies of fp32 matrices (the GEMMs' weight and R operands)
 __global__ void bwd_cast_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
                                 size_t n4) {
@@ -237,13 +243,14 @@ __global__ void bwd_wgrad_sum_kernel(WgradSumArgs a) {
 namespace bf {
 constexpr int BM = 128, HB = 64, D = 128;
 constexpr uint32_t ATILE = BM * D * 2;      // 32 KB: 128 token rows x 128 d, two 64-column boxes
+constexpr uint32_t ASTAGE = 2 * ATILE;      // K | V (key) or Q | dout (read)
 constexpr uint32_t B2 = 2 * HB * D * 2;     // 32 KB: two weight blocks of 64 hidden x 128 d
-constexpr uint32_t OFF_A0 = 0, OFF_A1 = ATILE, OFF_B13 = 2 * ATILE, OFF_R13 = OFF_B13 + B2,
-                   OFF_B2 = OFF_R13 + B2;
-constexpr uint32_t OFF_BAR_KEY = OFF_B2 + B2, OFF_BAR_READ = OFF_R13;   // read: [W1|W3], then W2 alone
+constexpr uint32_t OFF_A = 0;                               // two A stages
+constexpr uint32_t OFF_B13 = 2 * ASTAGE, OFF_R13 = OFF_B13 + B2, OFF_B2 = OFF_R13 + B2;
+constexpr uint32_t OFF_BAR_KEY = OFF_B2 + B2, OFF_BAR_READ = OFF_R13 + B2 / 2;   // read: [W1|W3], then W2 alone
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
-constexpr uint32_t SMEM_KEY = OFF_BAR_KEY + 256 + 1024, SMEM_READ = OFF_BAR_READ + 16384 + 256 + 1024;
+constexpr uint32_t SMEM_KEY = OFF_BAR_KEY + 256 + 1024, SMEM_READ = OFF_BAR_READ + 256 + 1024;
 constexpr uint32_t TM_COLS = 512;
 }  // namespace bf
 
@@ -259,6 +266,12 @@ struct BwdFwdArgs {
   DevStatus st;
 };
 
+// Persistent: CTA c takes a contiguous range of the (head, hidden block,
+// token tile) tiles, token tile fastest, so consecutive tiles share their
+// weight blocks (reloaded only when the block changes).  Token tiles are
+// double-buffered, so the next tile's loads and products overlap this
+// tile's elementwise step and stores; one set of accumulators in TMEM (the
+// next tile's products wait until the epilogue has read them out).
 __global__ void __launch_bounds__(bf::THREADS, 1)
     bwd_fwd_fused_kernel(const __grid_constant__ BwdFwdMaps maps, const BwdFwdArgs a) {
   using namespace bf;
@@ -266,17 +279,35 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const bool key = a.key != 0;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (key ? OFF_BAR_KEY : OFF_BAR_READ + 16384));
-  uint64_t* acc_full = full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + (key ? OFF_BAR_KEY : OFF_BAR_READ));   // [2]
+  uint64_t* a_empty = a_full + 2;     // [2]
+  uint64_t* w_full = a_empty + 2;
+  uint64_t* w_empty = w_full + 1;
+  uint64_t* acc_full = w_empty + 1;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* fin = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   uint32_t* abort_flag = tmem_slot + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_hb = a.dh / HB;
-  const int mt = blockIdx.x % a.n_mt, hb = (blockIdx.x / a.n_mt) % n_hb, bh = blockIdx.x / (a.n_mt * n_hb);
-  const int j0 = hb * HB;
+  const int total = a.n_mt * n_hb * a.BH;
+  const int lo = (int)((long long)blockIdx.x * total / gridDim.x);
+  const int hi = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
+  auto decode = [&](int t, int& bh, int& hb, int& mt) {
+    mt = t % a.n_mt;
+    hb = (t / a.n_mt) % n_hb;
+    bh = t / (a.n_mt * n_hb);
+  };
   if (threadIdx.x == 0) {
-    mbar_init(full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&a_full[b], 1);
+      mbar_init(&a_empty[b], 1);
+    }
+    mbar_init(w_full, 1);
+    mbar_init(w_empty, 1);
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, EPI_WARPS * 32);
+    mbar_init(fin, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -289,44 +320,78 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   Waiter W{abort_flag, a.st, 400};
+  const uint32_t wbytes = key ? 3 * B2 : B2 + B2 / 2;
+  uint32_t at = 0, wl = 0;   // copies issued (producer lane)
   if (warp == 0) {
     if (lane == 0) {
-      const int row = a.t0 + mt * BM;
-      const uint32_t bytes = key ? 2 * ATILE + 3 * B2 : 2 * ATILE + B2 + B2 / 2;
-      mbar_arrive_expect_tx(full, bytes);
-      for (int h = 0; h < 2; ++h) {
-        tma_load_3d(smem + OFF_A0 + h * (ATILE / 2), &maps.a0, full, h * 64, row, bh);
-        tma_load_3d(smem + OFF_A1 + h * (ATILE / 2), &maps.a1, full, h * 64, row, bh);
-      }
-      // K-major weight blocks: atom h (d 64h .. 64h + 63) = [first 64 rows | second 64 rows]
-      for (int h = 0; h < 2; ++h) {
-        tma_load_3d(smem + OFF_B13 + h * (B2 / 2), &maps.w1, full, h * 64, j0, bh);
-        tma_load_3d(smem + OFF_B13 + h * (B2 / 2) + B2 / 4, &maps.w3, full, h * 64, j0, bh);
-      }
-      // MN-major W2[:, J] (and R2[:, J]): 128 d rows of 64 hidden units, two 64-row boxes
-      uint8_t* b2 = smem + (key ? OFF_B2 : OFF_R13);
-      for (int h = 0; h < 2; ++h) tma_load_3d(b2 + h * (B2 / 4), &maps.w2, full, j0, h * 64, bh);
-      if (key) {
-        for (int h = 0; h < 2; ++h) {
-          tma_load_3d(smem + OFF_R13 + h * (B2 / 2), &maps.r1, full, h * 64, j0, bh);
-          tma_load_3d(smem + OFF_R13 + h * (B2 / 2) + B2 / 4, &maps.r3, full, h * 64, j0, bh);
-          tma_load_3d(b2 + B2 / 2 + h * (B2 / 4), &maps.r2, full, j0, h * 64, bh);
+      int cur = -1;
+      bool ok = true;
+      for (int t = lo; ok && t < hi; ++t) {
+        int bh, hb, mt;
+        decode(t, bh, hb, mt);
+        const int grpw = bh * n_hb + hb;
+        if (grpw != cur) {   // the weight blocks of (head, hidden block)
+          if (wl >= 1 && !W.wait(w_empty, (wl - 1) & 1, 1)) { ok = false; break; }
+          const int j0 = hb * HB;
+          mbar_arrive_expect_tx(w_full, wbytes);
+          // K-major weight blocks: atom h (d 64h .. 64h + 63) = [first 64 rows | second 64 rows]
+          for (int h = 0; h < 2; ++h) {
+            tma_load_3d(smem + OFF_B13 + h * (B2 / 2), &maps.w1, w_full, h * 64, j0, bh);
+            tma_load_3d(smem + OFF_B13 + h * (B2 / 2) + B2 / 4, &maps.w3, w_full, h * 64, j0, bh);
+          }
+          // MN-major W2[:, J] (and R2[:, J]): 128 d rows of 64 hidden units, two 64-row boxes
+          uint8_t* b2 = smem + (key ? OFF_B2 : OFF_R13);
+          for (int h = 0; h < 2; ++h) tma_load_3d(b2 + h * (B2 / 4), &maps.w2, w_full, j0, h * 64, bh);
+          if (key) {
+            for (int h = 0; h < 2; ++h) {
+              tma_load_3d(smem + OFF_R13 + h * (B2 / 2), &maps.r1, w_full, h * 64, j0, bh);
+              tma_load_3d(smem + OFF_R13 + h * (B2 / 2) + B2 / 4, &maps.r3, w_full, h * 64, j0, bh);
+              tma_load_3d(b2 + B2 / 2 + h * (B2 / 4), &maps.r2, w_full, j0, h * 64, bh);
+            }
+          }
+          ++wl;
+          cur = grpw;
         }
+        const uint32_t s = at & 1;
+        if (at >= 2 && !W.wait(&a_empty[s], ((at >> 1) - 1) & 1, 2)) { ok = false; break; }
+        const int row = a.t0 + mt * BM;
+        uint8_t* st = smem + OFF_A + s * ASTAGE;
+        mbar_arrive_expect_tx(&a_full[s], ASTAGE);
+        for (int h = 0; h < 2; ++h) {
+          tma_load_3d(st + h * (ATILE / 2), &maps.a0, &a_full[s], h * 64, row, bh);
+          tma_load_3d(st + ATILE + h * (ATILE / 2), &maps.a1, &a_full[s], h * 64, row, bh);
+        }
+        ++at;
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      if (W.wait(full, 0, 1)) {
+      const uint32_t id_k = make_idesc(128, 128, false, false);          // K-major B, N = 128
+      const uint32_t id_mn = make_idesc(128, key ? 128 : 64, false, true);   // MN-major B
+      const uint64_t da = make_sdesc(smem_u32(smem + OFF_A), 16, 1024);
+      const uint64_t db13 = make_sdesc(smem_u32(smem + OFF_B13), 16, 1024);
+      const uint64_t dr13 = make_sdesc(smem_u32(smem + OFF_R13), 16, 1024);
+      // [W2_J | R2_J]: two 64-wide N blocks 16 KB apart
+      const uint64_t db2 = make_sdesc(smem_u32(smem + (key ? OFF_B2 : OFF_R13)), B2 / 2, 1024);
+      uint32_t am = 0, wu = 0;
+      int cur = -1;
+      bool ok = true;
+      for (int t = lo; ok && t < hi; ++t) {
+        int bh, hb, mt;
+        decode(t, bh, hb, mt);
+        const int grpw = bh * n_hb + hb;
+        if (grpw != cur) {
+          if (wu >= 1) mma_commit(w_empty);   // after every product on the previous blocks
+          if (!W.wait(w_full, wu & 1, 3)) { ok = false; break; }
+          ++wu;
+          cur = grpw;
+        }
+        const uint32_t s = am & 1;
+        if (!W.wait(&a_full[s], (am >> 1) & 1, 4)) { ok = false; break; }
+        if (am >= 1 && !W.wait(acc_empty, (am - 1) & 1, 5)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t id_k = make_idesc(128, 128, false, false);          // K-major B, N = 128
-        const uint32_t id_mn = make_idesc(128, key ? 128 : 64, false, true);   // MN-major B
-        const uint64_t da0 = make_sdesc(smem_u32(smem + OFF_A0), 16, 1024);
-        const uint64_t da1 = make_sdesc(smem_u32(smem + OFF_A1), 16, 1024);
-        const uint64_t db13 = make_sdesc(smem_u32(smem + OFF_B13), 16, 1024);
-        const uint64_t dr13 = make_sdesc(smem_u32(smem + OFF_R13), 16, 1024);
-        // [W2_J | R2_J]: two 64-wide N blocks 16 KB apart
-        const uint64_t db2 = make_sdesc(smem_u32(smem + (key ? OFF_B2 : OFF_R13)), B2 / 2, 1024);
+        const uint64_t da0 = sdesc_add(da, s * ASTAGE), da1 = sdesc_add(da0, ATILE);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * (ATILE / 2) + (kk & 3) * 32;
@@ -335,108 +400,123 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
           if (key) mma_bf16(tmem + 128, sdesc_add(da0, off), sdesc_add(dr13, offb), id_k, kk > 0);
           mma_bf16(tmem + 256, sdesc_add(da1, off), sdesc_add(db2, kk * 2048), id_mn, kk > 0);
         }
+        mma_commit(&a_empty[s]);
         mma_commit(acc_full);
+        ++am;
       }
+      mma_commit(fin);
+      W.drain(fin, 0);
     }
     __syncwarp();
   } else {
     const int q4 = warp & 3;
     const int cg = (warp - 2) >> 2;                 // 32 hidden columns of the 64
     const int r = q4 * 32 + lane;
-    const int tok = mt * BM + r;                    // row of the chunk
-    const bool valid = tok < a.C;
     const uint32_t lb = (uint32_t)(q4 * 32) << 16;
-    const float eta = (key && valid) ? a.lr[(size_t)bh * a.lr_len + a.t0 + tok] : 0.f;
-    const bool ok = W.wait(acc_full, 0, 2);
-    if (ok) tc_fence_after();
+    uint32_t ae = 0;
+    for (int t = lo; t < hi; ++t, ++ae) {
+      int bh, hb, mt;
+      decode(t, bh, hb, mt);
+      const int j0 = hb * HB;
+      const int tok = mt * BM + r;                  // row of the chunk
+      const bool valid = tok < a.C;
+      const float eta = (key && valid) ? a.lr[(size_t)bh * a.lr_len + a.t0 + tok] : 0.f;
+      if (!W.wait(acc_full, ae & 1, 6)) break;
+      tc_fence_after();
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t c0 = (uint32_t)(cg * 32 + h * 16);
-      uint32_t x1[16], x3[16], x5[16], y1[16], y3[16], y5[16];
-      // every lane takes part in the warp-collective loads
-      tmem_ld16_issue(tmem + lb + c0, x1);            // h1 / hq1
-      tmem_ld16_issue(tmem + lb + 64 + c0, x3);       // h3 / hq3
-      tmem_ld16_issue(tmem + lb + 256 + c0, x5);      // vw2 / dgq
-      if (key) {
-        tmem_ld16_issue(tmem + lb + 128 + c0, y1);    // r1
-        tmem_ld16_issue(tmem + lb + 192 + c0, y3);    // r3
-        tmem_ld16_issue(tmem + lb + 320 + c0, y5);    // vr2
-      }
-      tmem_wait_ld();
-      const size_t base = ((size_t)bh * a.cmax + tok) * a.dh + j0 + c0;
-      if (key) {
-        uint32_t o[7][8];
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t c0 = (uint32_t)(cg * 32 + h * 16);
+        uint32_t x1[16], x3[16], x5[16], y1[16], y3[16], y5[16];
+        // every lane takes part in the warp-collective loads
+        tmem_ld16_issue(tmem + lb + c0, x1);            // h1 / hq1
+        tmem_ld16_issue(tmem + lb + 64 + c0, x3);       // h3 / hq3
+        tmem_ld16_issue(tmem + lb + 256 + c0, x5);      // vw2 / dgq
+        if (key) {
+          tmem_ld16_issue(tmem + lb + 128 + c0, y1);    // r1
+          tmem_ld16_issue(tmem + lb + 192 + c0, y3);    // r3
+          tmem_ld16_issue(tmem + lb + 320 + c0, y5);    // vr2
+        }
+        tmem_wait_ld();
+        if (h == 1) {   // the accumulators are read out: the next tile's products may start
+          tc_fence_before();
+          mbar_arrive(acc_empty);
+        }
+        const size_t base = ((size_t)bh * a.cmax + tok) * a.dh + j0 + c0;
+        if (key) {
+          uint32_t o[7][8];
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          float v[7][2];
+          for (int j = 0; j < 16; j += 2) {
+            float v[7][2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            float vdh1 = 0.f, vdh3 = 0.f, vddg = 0.f, vddgn = 0.f, ve1 = 0.f, ve3 = 0.f, vg = 0.f;
-            if (valid && ok) {
-              const float x = __uint_as_float(x1[j + u]), y = __uint_as_float(x3[j + u]);
-              const float sg = sig(x);
-              const float act = x * sg;
-              const float s1 = sg * (1.f + x * (1.f - sg));
-              const float s2 = sg * (1.f - sg) * (2.f + x * (1.f - 2.f * sg));
-              const float dg = -eta * __uint_as_float(x5[j + u]), r2 = -eta * __uint_as_float(y5[j + u]);
-              const float r1 = __uint_as_float(y1[j + u]), r3 = __uint_as_float(y3[j + u]);
-              vdh3 = r2 * act + dg * s1 * r1;
-              vdh1 = (r2 * y + dg * r3) * s1 + dg * y * r1 * s2;
-              vddg = act * r3 + y * s1 * r1;
-              vddgn = -eta * vddg;
-              ve1 = dg * y * s1;
-              ve3 = dg * act;
-              vg = act * y;
+            for (int u = 0; u < 2; ++u) {
+              float vdh1 = 0.f, vdh3 = 0.f, vddg = 0.f, vddgn = 0.f, ve1 = 0.f, ve3 = 0.f, vg = 0.f;
+              if (valid) {
+                const float x = __uint_as_float(x1[j + u]), y = __uint_as_float(x3[j + u]);
+                const float sg = sig(x);
+                const float act = x * sg;
+                const float s1 = sg * (1.f + x * (1.f - sg));
+                const float s2 = sg * (1.f - sg) * (2.f + x * (1.f - 2.f * sg));
+                const float dg = -eta * __uint_as_float(x5[j + u]), r2 = -eta * __uint_as_float(y5[j + u]);
+                const float r1 = __uint_as_float(y1[j + u]), r3 = __uint_as_float(y3[j + u]);
+                vdh3 = r2 * act + dg * s1 * r1;
+                vdh1 = (r2 * y + dg * r3) * s1 + dg * y * r1 * s2;
+                vddg = act * r3 + y * s1 * r1;
+                vddgn = -eta * vddg;
+                ve1 = dg * y * s1;
+                ve3 = dg * act;
+                vg = act * y;
+              }
+              v[0][u] = vdh1; v[1][u] = vdh3; v[2][u] = vddg; v[3][u] = vddgn;
+              v[4][u] = ve1; v[5][u] = ve3; v[6][u] = vg;
             }
-            v[0][u] = vdh1; v[1][u] = vdh3; v[2][u] = vddg; v[3][u] = vddgn;
-            v[4][u] = ve1; v[5][u] = ve3; v[6][u] = vg;
+#pragma unroll
+            for (int q = 0; q < 7; ++q) o[q][j >> 1] = pack_bf16x2(v[q][0], v[q][1]);
           }
 #pragma unroll
-          for (int q = 0; q < 7; ++q) o[q][j >> 1] = pack_bf16x2(v[q][0], v[q][1]);
-        }
+          for (int q = 0; q < 7; ++q) {
+            uint4* dst = reinterpret_cast<uint4*>(a.out[q] + base);
+            dst[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
+            dst[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
+          }
+        } else {
+          uint32_t o[3][8];
 #pragma unroll
-        for (int q = 0; q < 7; ++q) {
-          uint4* dst = reinterpret_cast<uint4*>(a.out[q] + base);
-          dst[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
-          dst[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
-        }
-      } else {
-        uint32_t o[3][8];
+          for (int j = 0; j < 16; j += 2) {
+            float v[3][2];
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          float v[3][2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            float v1 = 0.f, v3 = 0.f, vg = 0.f;
-            if (valid && ok) {
-              const float x = __uint_as_float(x1[j + u]), y = __uint_as_float(x3[j + u]);
-              const float dg = __uint_as_float(x5[j + u]);
-              const float sg = sig(x);
-              const float act = x * sg;
-              v1 = dg * y * sg * (1.f + x * (1.f - sg));
-              v3 = dg * act;
-              vg = act * y;
+            for (int u = 0; u < 2; ++u) {
+              float v1 = 0.f, v3 = 0.f, vg = 0.f;
+              if (valid) {
+                const float x = __uint_as_float(x1[j + u]), y = __uint_as_float(x3[j + u]);
+                const float dg = __uint_as_float(x5[j + u]);
+                const float sg = sig(x);
+                const float act = x * sg;
+                v1 = dg * y * sg * (1.f + x * (1.f - sg));
+                v3 = dg * act;
+                vg = act * y;
+              }
+              v[0][u] = v1; v[1][u] = v3; v[2][u] = vg;
             }
-            v[0][u] = v1; v[1][u] = v3; v[2][u] = vg;
+#pragma unroll
+            for (int q = 0; q < 3; ++q) o[q][j >> 1] = pack_bf16x2(v[q][0], v[q][1]);
           }
 #pragma unroll
-          for (int q = 0; q < 3; ++q) o[q][j >> 1] = pack_bf16x2(v[q][0], v[q][1]);
-        }
-#pragma unroll
-        for (int q = 0; q < 3; ++q) {
-          uint4* dst = reinterpret_cast<uint4*>(a.out[q] + base);
-          dst[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
-          dst[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
+          for (int q = 0; q < 3; ++q) {
+            uint4* dst = reinterpret_cast<uint4*>(a.out[q] + base);
+            dst[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
+            dst[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
+          }
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (warp == 0 && lane == 0 && W.aborted()) {   // an aborted CTA: its copies land before it leaves
+    for (uint32_t i = at > 2 ? at - 2 : 0; i < at; ++i) W.drain(&a_full[i & 1], (i >> 1) & 1);
+    if (wl >= 1) W.drain(w_full, (wl - 1) & 1);
+  }
   if (warp == 1) {
-    // an aborted CTA: the copies it issued land before it leaves
-    if (*abort_flag && lane == 0) W.drain(full, 0);
-    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
   }
@@ -630,8 +710,8 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     ba.n_mt = w.cmax / bf::BM; ba.key = key ? 1 : 0; ba.lr = f.lr; ba.st = L.st;
     for (int i = 0; i < 7; ++i) ba.out[i] = key ? Hb(w.b16[i]) : (i < 3 ? rb16[i] : nullptr);
     prof_before(K_BWD_FWD, stream);
-    bwd_fwd_fused_kernel<<<dim3((unsigned)(ba.n_mt * (dh / bf::HB) * BH)), dim3(bf::THREADS),
-                           key ? bf::SMEM_KEY : bf::SMEM_READ, stream>>>(m, ba);
+    bwd_fwd_fused_kernel<<<dim3((unsigned)std::min(ba.n_mt * (dh / bf::HB) * BH, num_sms_bwd())),
+                           dim3(bf::THREADS), key ? bf::SMEM_KEY : bf::SMEM_READ, stream>>>(m, ba);
     prof_after(K_BWD_FWD, stream);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   };
