@@ -411,7 +411,19 @@ class LaCTBwdBench(LaCTBench):
         return 46 * self.d * self.dh * self.N * self.B * self.H
 
     def kernel_flops_per_step(self):
-        return {}
+        """Per token-head, causal order: the fused forward products of the
+        key step ([h1|h3], [r1|r3], [vw2|vr2]: 12 d dh) and of the read step
+        ([hq1|hq3], dgq: 6 d dh); the grouped chunk products (dk 8 d dh, d_dy
+        4, dq 4, the three weight gradients 12).  The forward replay's
+        key/gradient kernel: 12 d dh per key token."""
+        BH, d, dh, N, Nq = self.B * self.H, self.d, self.dh, self.N, self.Nq
+        f = {"lact_keygrad": 12 * d * dh * N * BH}
+        if self.causal:
+            f.update({"lact_bwd_fwd": 18 * d * dh * N * BH, "lact_bwd_gemm": 28 * d * dh * N * BH})
+        else:
+            f.update({"lact_bwd_fwd": (12 * N + 6 * Nq) * d * dh * BH,
+                      "lact_bwd_gemm": 18 * d * dh * N * BH})
+        return f
 
     def step(self, stream):
         self.T.lact_chunk_bwd(self.desc, self.q, self.k, self.v, self.lr, self.state0, self.dout,

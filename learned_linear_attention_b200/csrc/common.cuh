@@ -342,6 +342,51 @@ TTT_DEVICE_INLINE uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Two-lane fp32 arithmetic with sm_100's packed instructions (each lane
+// rounds exactly like the scalar instruction): half the issue slots.
+TTT_DEVICE_INLINE float2 x2_mul(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 A, B, R;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "mul.rn.f32x2 R, A, B;\n\tmov.b64 {%0, %1}, R;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+TTT_DEVICE_INLINE float2 x2_fma(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 A, B, C, R;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "mov.b64 C, {%6, %7};\n\tfma.rn.f32x2 R, A, B, C;\n\tmov.b64 {%0, %1}, R;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+TTT_DEVICE_INLINE float2 x2_sub(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 A, B, R;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "sub.rn.f32x2 R, A, B;\n\tmov.b64 {%0, %1}, R;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+TTT_DEVICE_INLINE float2 x2_splat(float a) { return make_float2(a, a); }
+// sigmoid(x) = 0.5 tanh(x / 2) + 0.5 on both lanes (hardware tanh
+// approximation, relative error about 2^-11)
+TTT_DEVICE_INLINE float2 x2_sigmoid(float2 x) {
+  const float2 h = x2_mul(x, x2_splat(0.5f));
+  float2 t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(h.x));
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(h.y));
+  return x2_fma(t, x2_splat(0.5f), x2_splat(0.5f));
+}
+
+// 32 bytes to global memory in one 256-bit access (dst 32-byte aligned):
+// a warp storing one row per thread then writes whole 32-byte sectors
+TTT_DEVICE_INLINE void st_global_v8(void* dst, const uint32_t* a) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(a[0]),
+               "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7])
+               : "memory");
+}
+
 TTT_DEVICE_INLINE void st_shared_v4(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c,
                                     uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c),

@@ -284,7 +284,7 @@ int launch_lact_keygrad(const KeyGradLaunch& L, cudaStream_t stream);
 enum KernelKind {
   K_LIN_SIMT, K_LIN_UMMA, K_LACT_CAST, K_KEYPASS, K_GEMM_READ, K_GEMM_GRAD, K_UPDATE,
   K_MUON_MOM, K_NS_PREP, K_GEMM_NS, K_MUON_APPLY, K_KEYGRAD, K_LIN_SEG, K_LIN_BWD_EW, K_SWA, K_LOOP,
-  K_BWD_FWD, K_NUM
+  K_BWD_FWD, K_BWD_GROUP, K_NUM
 };
 void prof_before(int kind, cudaStream_t s);
 void prof_after(int kind, cudaStream_t s);

@@ -37,6 +37,7 @@
 
 #include "gemm.cuh"
 #include "kernels.h"
+#include "gemm_group.cuh"
 
 namespace ttt {
 
@@ -263,8 +264,20 @@ struct BwdFwdArgs {
   int BH, C, cmax, dh, t0, lr_len, n_mt, key;
   const float* lr;           // key: [BH][lr_len]
   __nv_bfloat16* out[7];     // [BH][cmax][dh]: key d_h1, d_h3, d_dg, d_dgn, e1, e3, g; read dhq1, dhq3, gq
+  int v8;                    // every output starts on a 32-byte boundary: 256-bit stores
   DevStatus st;
 };
+
+// 16 bf16 pairs' worth (32 bytes) of one output row
+TTT_DEVICE_INLINE void store_row32(__nv_bfloat16* dst, const uint32_t* o, bool v8) {
+  if (v8) {
+    st_global_v8(dst, o);
+  } else {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
 
 // Persistent: CTA c takes a contiguous range of the (head, hidden block,
 // token tile) tiles, token tile fastest, so consecutive tiles share their
@@ -442,70 +455,72 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
           mbar_arrive(acc_empty);
         }
         const size_t base = ((size_t)bh * a.cmax + tok) * a.dh + j0 + c0;
+        auto f2 = [](const uint32_t* r, int j) {
+          return make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+        };
+        const float2 one = x2_splat(1.f);
         if (key) {
+          // pairs of adjacent hidden columns on the packed fp32 instructions
           uint32_t o[7][8];
+          const float2 ne = x2_splat(-eta);
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
-            float v[7][2];
+            const float2 x = f2(x1, j), y = f2(x3, j);
+            const float2 r1 = f2(y1, j), r3 = f2(y3, j);
+            const float2 sg = x2_sigmoid(x);
+            const float2 act = x2_mul(x, sg);
+            const float2 oms = x2_sub(one, sg);
+            const float2 s1 = x2_fma(sg, x2_mul(x, oms), sg);                       // sg (1 + x (1 - sg))
+            const float2 w = x2_fma(x, x2_fma(sg, x2_splat(-2.f), one), x2_splat(2.f));   // 2 + x (1 - 2 sg)
+            const float2 s2 = x2_mul(x2_mul(sg, oms), w);
+            const float2 dg = x2_mul(ne, f2(x5, j)), r2 = x2_mul(ne, f2(y5, j));
+            const float2 dgy = x2_mul(dg, y);
+            const float2 vdh3 = x2_fma(r2, act, x2_mul(x2_mul(dg, s1), r1));
+            const float2 vdh1 = x2_fma(x2_fma(r2, y, x2_mul(dg, r3)), s1, x2_mul(x2_mul(dgy, r1), s2));
+            const float2 vddg = x2_fma(act, r3, x2_mul(x2_mul(y, s1), r1));
+            const float2 vddgn = x2_mul(ne, vddg);
+            const float2 ve1 = x2_mul(dgy, s1);
+            const float2 ve3 = x2_mul(dg, act);
+            const float2 vg = x2_mul(act, y);
+            o[0][j >> 1] = pack_bf16x2(vdh1.x, vdh1.y);
+            o[1][j >> 1] = pack_bf16x2(vdh3.x, vdh3.y);
+            o[2][j >> 1] = pack_bf16x2(vddg.x, vddg.y);
+            o[3][j >> 1] = pack_bf16x2(vddgn.x, vddgn.y);
+            o[4][j >> 1] = pack_bf16x2(ve1.x, ve1.y);
+            o[5][j >> 1] = pack_bf16x2(ve3.x, ve3.y);
+            o[6][j >> 1] = pack_bf16x2(vg.x, vg.y);
+          }
+          if (!valid) {   // rows past the chunk hold zeros
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              float vdh1 = 0.f, vdh3 = 0.f, vddg = 0.f, vddgn = 0.f, ve1 = 0.f, ve3 = 0.f, vg = 0.f;
-              if (valid) {
-                const float x = __uint_as_float(x1[j + u]), y = __uint_as_float(x3[j + u]);
-                const float sg = sig(x);
-                const float act = x * sg;
-                const float s1 = sg * (1.f + x * (1.f - sg));
-                const float s2 = sg * (1.f - sg) * (2.f + x * (1.f - 2.f * sg));
-                const float dg = -eta * __uint_as_float(x5[j + u]), r2 = -eta * __uint_as_float(y5[j + u]);
-                const float r1 = __uint_as_float(y1[j + u]), r3 = __uint_as_float(y3[j + u]);
-                vdh3 = r2 * act + dg * s1 * r1;
-                vdh1 = (r2 * y + dg * r3) * s1 + dg * y * r1 * s2;
-                vddg = act * r3 + y * s1 * r1;
-                vddgn = -eta * vddg;
-                ve1 = dg * y * s1;
-                ve3 = dg * act;
-                vg = act * y;
-              }
-              v[0][u] = vdh1; v[1][u] = vdh3; v[2][u] = vddg; v[3][u] = vddgn;
-              v[4][u] = ve1; v[5][u] = ve3; v[6][u] = vg;
-            }
+            for (int q = 0; q < 7; ++q)
 #pragma unroll
-            for (int q = 0; q < 7; ++q) o[q][j >> 1] = pack_bf16x2(v[q][0], v[q][1]);
+              for (int u = 0; u < 8; ++u) o[q][u] = 0u;
           }
 #pragma unroll
-          for (int q = 0; q < 7; ++q) {
-            uint4* dst = reinterpret_cast<uint4*>(a.out[q] + base);
-            dst[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
-            dst[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
-          }
+          for (int q = 0; q < 7; ++q) store_row32(a.out[q] + base, o[q], a.v8 != 0);
         } else {
           uint32_t o[3][8];
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
-            float v[3][2];
+            const float2 x = f2(x1, j), y = f2(x3, j), dg = f2(x5, j);
+            const float2 sg = x2_sigmoid(x);
+            const float2 act = x2_mul(x, sg);
+            const float2 s1 = x2_fma(sg, x2_mul(x, x2_sub(one, sg)), sg);
+            const float2 v1 = x2_mul(x2_mul(dg, y), s1);
+            const float2 v3 = x2_mul(dg, act);
+            const float2 vg = x2_mul(act, y);
+            o[0][j >> 1] = pack_bf16x2(v1.x, v1.y);
+            o[1][j >> 1] = pack_bf16x2(v3.x, v3.y);
+            o[2][j >> 1] = pack_bf16x2(vg.x, vg.y);
+          }
+          if (!valid) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              float v1 = 0.f, v3 = 0.f, vg = 0.f;
-              if (valid) {
-                const float x = __uint_as_float(x1[j + u]), y = __uint_as_float(x3[j + u]);
-                const float dg = __uint_as_float(x5[j + u]);
-                const float sg = sig(x);
-                const float act = x * sg;
-                v1 = dg * y * sg * (1.f + x * (1.f - sg));
-                v3 = dg * act;
-                vg = act * y;
-              }
-              v[0][u] = v1; v[1][u] = v3; v[2][u] = vg;
-            }
+            for (int q = 0; q < 3; ++q)
 #pragma unroll
-            for (int q = 0; q < 3; ++q) o[q][j >> 1] = pack_bf16x2(v[q][0], v[q][1]);
+              for (int u = 0; u < 8; ++u) o[q][u] = 0u;
           }
 #pragma unroll
-          for (int q = 0; q < 3; ++q) {
-            uint4* dst = reinterpret_cast<uint4*>(a.out[q] + base);
-            dst[0] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
-            dst[1] = make_uint4(o[q][4], o[q][5], o[q][6], o[q][7]);
-          }
+          for (int q = 0; q < 3; ++q) store_row32(a.out[q] + base, o[q], a.v8 != 0);
         }
       }
     }
@@ -644,21 +659,6 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
   // cin of an accumulating GEMM is read at row m (no row offset), so
   // accumulating outputs always start at row 0 of their buffer
 
-  // split-K MN-major product into `o` [BH][splits][M][N] (no accumulation)
-  auto gemm_split = [&](const CUtensorMap* A, const CUtensorMap* B, int np, int M, int N, int kps,
-                        int S, float* o, int ak, int bk) -> int {
-    GemmMaps m{};
-    GemmArgs g = gemm_args_default(L.st);
-    for (int i = 0; i < np; ++i) {
-      m.a[i] = A[i];
-      m.b[i] = B[i];
-      g.a_k_off[i] = ak;
-      g.b_k_off[i] = bk;
-    }
-    g.npairs = np; g.M = M; g.N = N; g.batch = BH; g.k_steps = kps; g.splits = S;
-    g.o32 = o; g.ld32 = N; g.o32_ss = (long long)M * N; g.o32_bs = (long long)S * M * N;
-    return gemm_launch(GEMM_AMN_BMN, m, g, stream, K_GEMM_GRAD);
-  };
 
   CUtensorMap mq_k{}, mq_mn{}, mk_k{}, mk_mn{}, mv_k{}, mv_mn{}, mdo_k{}, mdo_mn{};
   if (f.N_in > 0) {
@@ -708,7 +708,11 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     BwdFwdArgs ba{};
     ba.BH = BH; ba.C = C; ba.cmax = w.cmax; ba.dh = dh; ba.t0 = t0; ba.lr_len = f.N_in;
     ba.n_mt = w.cmax / bf::BM; ba.key = key ? 1 : 0; ba.lr = f.lr; ba.st = L.st;
-    for (int i = 0; i < 7; ++i) ba.out[i] = key ? Hb(w.b16[i]) : (i < 3 ? rb16[i] : nullptr);
+    ba.v8 = 1;
+    for (int i = 0; i < 7; ++i) {
+      ba.out[i] = key ? Hb(w.b16[i]) : (i < 3 ? rb16[i] : nullptr);
+      if (reinterpret_cast<uintptr_t>(ba.out[i]) % 32 != 0) ba.v8 = 0;
+    }
     prof_before(K_BWD_FWD, stream);
     bwd_fwd_fused_kernel<<<dim3((unsigned)std::min(ba.n_mt * (dh / bf::HB) * BH, num_sms_bwd())),
                            dim3(bf::THREADS), key ? bf::SMEM_KEY : bf::SMEM_READ, stream>>>(m, ba);
@@ -754,6 +758,82 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     return read_dq(t0, C);
   };
 
+  // The products of a chunk on the fused path, in one grouped launch:
+  //   dk rows  = d_h1 W1 + d_h3 W3 + e1 R1 + e3 R3       (M = C, N = d, K = 4 dh)
+  //   d_dy     = d_dg W2^T + g R2^T                        (M = C, N = d, K = 2 dh)
+  //   dq rows  = dhq1 W1 + dhq3 W3                         (with the read; M = C, N = d)
+  //   dW1, dW3 partials = d_h1^T K (+ dhq1^T Q), d_h3^T K (+ dhq3^T Q)   (M = dh, N = d)
+  //   dW2 partial       = V^T (-lr d_dg) (+ dout^T gq)     (M = d, N = dh)
+  // the weight-gradient products split over the chunk's tokens into the
+  // (free) fp32 intermediates, then one pass adds the splits to dW (16 output
+  // tiles per matrix would leave most SMs idle); steps past the chunk read
+  // zero rows of the bf16 intermediates.  Each split's partial is d x dh per
+  // head, so S splits fit the region while S d <= cmax.
+  static std::atomic<uint64_t> group_attr{0};
+  if (fused_fwd && allow_dynamic_smem(gemm_group_kernel, (int)gg::SMEM, group_attr)) return -1;
+  auto chunk_products = [&](int t0, int C, bool with_read) -> int {
+    const int ks = (C + 63) / 64;
+    const int S = std::max(1, std::min(std::min(8, ks), w.cmax / d)), kps = (ks + S - 1) / S;
+    GroupMaps m{};
+    GroupArgs g{};
+    g.st = L.st;
+    int units = 0;
+    auto add = [&](int M, int N, int splits, int k_steps, int np, bool a_mn, bool b_mn,
+                   const CUtensorMap* A, const CUtensorMap* B, int a_k_off, int b_k_off, float* o,
+                   long long o_bs, long long o_ss, int ld, int row_off) {
+      GroupProblem& q = g.p[g.nprob];
+      q.M = M; q.N = N;
+      q.tiles_m = (M + 127) / 128; q.tiles_n = N / gg::BN; q.splits = splits;
+      q.k_steps = k_steps; q.npairs = np; q.a_mn = a_mn ? 1 : 0; q.b_mn = b_mn ? 1 : 0;
+      q.unit0 = units;
+      for (int i = 0; i < np; ++i) {
+        m.a[g.nprob][i] = A[i];
+        m.b[g.nprob][i] = B[i];
+        q.a_k_off[i] = a_k_off;
+        q.b_k_off[i] = b_k_off;
+      }
+      q.o = o; q.o_bs = o_bs; q.o_ss = o_ss; q.ld = ld; q.out_row_off = row_off;
+      q.v8 = (reinterpret_cast<uintptr_t>(o) % 32 == 0 && ld % 8 == 0 && o_bs % 8 == 0 &&
+              o_ss % 8 == 0) ? 1 : 0;
+      units += q.tiles_m * q.tiles_n * splits * BH;
+      ++g.nprob;
+    };
+    const int kd = dh / 64;
+    {
+      const CUtensorMap A[4] = {mb_k[0], mb_k[1], mb_k[4], mb_k[5]}, B[4] = {mW1mn, mW3mn, mR1mn, mR3mn};
+      add(C, d, 1, kd, 4, false, true, A, B, 0, 0, L.dk, (long long)f.N_in * d, 0, d, t0);
+    }
+    {
+      const CUtensorMap A[2] = {mb_k[2], mb_k[6]}, B[2] = {mW2k, mR2k};
+      add(C, d, 1, kd, 2, false, false, A, B, 0, 0, F(w.ddy), (long long)w.cmax * d, 0, d, 0);
+    }
+    if (with_read) {
+      const CUtensorMap A[2] = {mrb_k[0], mrb_k[1]}, B[2] = {mW1mn, mW3mn};
+      add(C, d, 1, kd, 2, false, true, A, B, 0, 0, L.dq, (long long)q_rows * d, 0, d, t0);
+    }
+    const int np = with_read ? 2 : 1;
+    const long long wsz = (long long)d * dh;
+    {
+      const CUtensorMap A1[2] = {mb_mn[0], mrb_mn[0]}, A3[2] = {mb_mn[1], mrb_mn[1]}, B13[2] = {mk_mn, mq_mn};
+      add(dh, d, S, kps, np, true, true, A1, B13, 0, t0, f32[3], S * wsz, wsz, d, 0);
+      add(dh, d, S, kps, np, true, true, A3, B13, 0, t0, f32[4], S * wsz, wsz, d, 0);
+    }
+    {
+      const CUtensorMap A2[2] = {mv_mn, mdo_mn}, B2[2] = {mb_mn[3], mrb_mn[2]};
+      add(d, dh, S, kps, np, true, true, A2, B2, t0, 0, f32[5], S * wsz, wsz, dh, 0);
+    }
+    g.units = units;
+    prof_before(K_BWD_GROUP, stream);
+    const cudaError_t e = launch_pdl(gemm_group_kernel, dim3((unsigned)std::min(units, num_sms_bwd())),
+                                     dim3(192), gg::SMEM, stream, m, g);
+    prof_after(K_BWD_GROUP, stream);
+    if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return -1;
+    WgradSumArgs sa{BH, S, wsz, {f32[3], f32[4], f32[5]}, {dW1, dW3, dW2}};
+    const long long n4 = 3LL * BH * d * dh / 4;
+    bwd_wgrad_sum_kernel<<<(unsigned)std::min<long long>((n4 + 255) / 256, 4096), 256, 0, stream>>>(sa);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  };
+
   // ---------------------------------------------------------------- 2. reverse
   if (L.dW_end)
     BWD_TRY(cudaMemcpyAsync(dW, L.dW_end, 3 * mat * 4, cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1);
@@ -797,47 +877,26 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
       bwd_key_ew_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 8192), 256, 0, stream>>>(ka);
       BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     }
-    // dk rows = d_h1 W1 + d_h3 W3 + e1 R1, then + e3 R3   (M = C, N = d, K = dh)
-    {
+    if (fused_fwd) {
+      BWD_TRY(chunk_products(t0, C, both));
+    } else {
+      // dk rows = d_h1 W1 + d_h3 W3 + e1 R1, then + e3 R3   (M = C, N = d, K = dh)
       const CUtensorMap A[3] = {mb_k[0], mb_k[1], mb_k[4]}, B[3] = {mW1mn, mW3mn, mR1mn};
       BWD_TRY(gemm(GEMM_AK_BMN, A, B, 3, C, d, dh / 64, F(w.ddy), d, (long long)w.cmax * d, false, 0,
                    0, 0, 0));
       BWD_TRY(gemm(GEMM_AK_BMN, &mb_k[5], &mR3mn, 1, C, d, dh / 64, F(w.ddy), d, (long long)w.cmax * d,
                    true, 0, 0, 0, 0));
-    }
-    // the chunk's dk rows: copy out of the temporary (rows t0.. of dk)
-    BWD_TRY(cudaMemcpy2DAsync(L.dk + (size_t)t0 * d, (size_t)f.N_in * d * 4, F(w.ddy),
-                              (size_t)w.cmax * d * 4, (size_t)C * d * 4, BH, cudaMemcpyDeviceToDevice,
-                              stream) == cudaSuccess ? 0 : -1);
-    // weight gradients: dW1 += d_h1^T K, dW3 += d_h3^T K, dW2 += V^T (-lr d_dg);
-    // with `both`, plus the read's dhq1^T Q, dhq3^T Q, dout^T gq as second pairs
-    {
-      const int np = both ? 2 : 1;
-      const CUtensorMap A1[2] = {mb_mn[0], mrb_mn[0]}, A3[2] = {mb_mn[1], mrb_mn[1]}, B13[2] = {mk_mn, mq_mn};
-      const CUtensorMap A2[2] = {mv_mn, mdo_mn}, B2m[2] = {mb_mn[3], mrb_mn[2]};
-      if (fused_fwd) {
-        // split-K over the chunk's tokens into the (free) fp32 intermediates,
-        // then one pass adds the splits to dW: 16 output tiles per matrix
-        // would leave most SMs idle.  Steps past the chunk read zero rows.
-        // (each split's partial is d x dh per head: S splits fit the region while S d <= cmax)
-        const int S = std::max(1, std::min(std::min(8, ks), w.cmax / d)), kps = (ks + S - 1) / S;
-        BWD_TRY(gemm_split(A1, B13, np, dh, d, kps, S, f32[3], 0, t0));
-        BWD_TRY(gemm_split(A3, B13, np, dh, d, kps, S, f32[4], 0, t0));
-        BWD_TRY(gemm_split(A2, B2m, np, d, dh, kps, S, f32[5], t0, 0));
-        WgradSumArgs sa{BH, S, (long long)d * dh, {f32[3], f32[4], f32[5]}, {dW1, dW3, dW2}};
-        const long long n4 = 3LL * BH * d * dh / 4;
-        bwd_wgrad_sum_kernel<<<(unsigned)std::min<long long>((n4 + 255) / 256, 4096), 256, 0, stream>>>(sa);
-        BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
-      } else {
-        BWD_TRY(gemm(GEMM_AMN_BMN, A1, B13, np, dh, d, ks, dW1, d, w13bs, true, 0, 0, 0, t0));
-        BWD_TRY(gemm(GEMM_AMN_BMN, A3, B13, np, dh, d, ks, dW3, d, w13bs, true, 0, 0, 0, t0));
-        BWD_TRY(gemm(GEMM_AMN_BMN, A2, B2m, np, d, dh, ks, dW2, dh, w2bs, true, 0, 0, t0, 0));
-      }
-    }
-    // d_dy = d_dg W2^T + g R2^T   (M = C, N = d, K = dh)
-    {
-      const CUtensorMap A[2] = {mb_k[2], mb_k[6]}, B[2] = {mW2k, mR2k};
-      BWD_TRY(gemm(GEMM_AK_BK, A, B, 2, C, d, dh / 64, F(w.ddy), d, (long long)w.cmax * d, false, 0,
+      // the chunk's dk rows: copy out of the temporary (rows t0.. of dk)
+      BWD_TRY(cudaMemcpy2DAsync(L.dk + (size_t)t0 * d, (size_t)f.N_in * d * 4, F(w.ddy),
+                                (size_t)w.cmax * d * 4, (size_t)C * d * 4, BH, cudaMemcpyDeviceToDevice,
+                                stream) == cudaSuccess ? 0 : -1);
+      // weight gradients: dW1 += d_h1^T K, dW3 += d_h3^T K, dW2 += V^T (-lr d_dg)
+      BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[0], &mk_mn, 1, dh, d, ks, dW1, d, w13bs, true, 0, 0, 0, t0));
+      BWD_TRY(gemm(GEMM_AMN_BMN, &mb_mn[1], &mk_mn, 1, dh, d, ks, dW3, d, w13bs, true, 0, 0, 0, t0));
+      BWD_TRY(gemm(GEMM_AMN_BMN, &mv_mn, &mb_mn[3], 1, d, dh, ks, dW2, dh, w2bs, true, 0, 0, t0, 0));
+      // d_dy = d_dg W2^T + g R2^T   (M = C, N = d, K = dh)
+      const CUtensorMap A2[2] = {mb_k[2], mb_k[6]}, B2[2] = {mW2k, mR2k};
+      BWD_TRY(gemm(GEMM_AK_BK, A2, B2, 2, C, d, dh / 64, F(w.ddy), d, (long long)w.cmax * d, false, 0,
                    0, 0, 0));
     }
     {
@@ -847,8 +906,7 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
           L.dv, L.dlr);
       BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     }
-    if (both) BWD_TRY(read_dq(t0, C));
-    else if (f.causal) BWD_TRY(read_vjp(t0, C));
+    if (!both && f.causal) BWD_TRY(read_vjp(t0, C));
   }
   return cudaMemcpyAsync(L.dW0, dW, 3 * mat * 4, cudaMemcpyDeviceToDevice, stream) == cudaSuccess
              ? 0 : -1;

@@ -12,7 +12,8 @@ static const char* kKindNames[K_NUM] = {
     "ttt_linear_simt", "ttt_linear_umma", "lact_cast",     "lact_keypass",
     "gemm_read",       "gemm_grad",       "lact_update",   "muon_momentum",
     "ns_prep",         "gemm_ns",         "muon_apply",    "lact_keygrad",
-    "ttt_linear_segstate", "ttt_linear_bwd_ew", "window_attention", "lact_loop", "lact_bwd_fwd"};
+    "ttt_linear_segstate", "ttt_linear_bwd_ew", "window_attention", "lact_loop", "lact_bwd_fwd",
+    "lact_bwd_gemm"};
 
 struct ProfRec {
   int kind;

@@ -16,7 +16,18 @@ TOL = 2e-2
 NAMES = ("q", "k", "v", "lr", "W1", "W3", "W2")
 
 
-def _run(x, g, opt="gd", with_dw=True, **kw):
+def _nan_at16(shape):
+    """A NaN-filled float32 tensor whose data starts 16 bytes past a 32-byte
+    boundary (the API asks for 16-byte alignment only)."""
+    n = int(np.prod(shape))
+    base = torch.full((n + 8,), float("nan"), device="cuda")
+    off = (4 - (base.data_ptr() % 32) // 4) % 8
+    t = base[off:off + n]
+    assert t.data_ptr() % 32 == 16
+    return t.view(shape)
+
+
+def _run(x, g, opt="gd", with_dw=True, offset16=False, **kw):
     B, H, N, d = x.k.values.shape
     dh = x.W1.shape[-2]
     R = x.q.values.shape[2]
@@ -28,12 +39,17 @@ def _run(x, g, opt="gd", with_dw=True, **kw):
     dW_end = None
     if with_dw:
         dW_end = torch.from_numpy(np.concatenate([w.ravel() for w in g.dW_end])).cuda()
-    grads = [torch.full((B, H, R, d), float("nan"), device="cuda"),
-             torch.full((B, H, N, d), float("nan"), device="cuda"),
-             torch.full((B, H, N, d), float("nan"), device="cuda"),
-             torch.full((B, H, N), float("nan"), device="cuda"),
-             torch.full((3 * mat,), float("nan"), device="cuda")]
-    ws = T.alloc_workspace(T.lact_bwd_workspace_bytes(desc))
+    shapes = [(B, H, R, d), (B, H, N, d), (B, H, N, d), (B, H, N), (3 * mat,)]
+    if offset16:
+        grads = [_nan_at16(sh) for sh in shapes]
+        nb = T.lact_bwd_workspace_bytes(desc)
+        raw = T.alloc_workspace(nb + 64)
+        skip = (16 - raw.data_ptr() % 32) % 32
+        ws = raw[skip:skip + nb]
+        assert ws.data_ptr() % 32 == 16
+    else:
+        grads = [torch.full(sh, float("nan"), device="cuda") for sh in shapes]
+        ws = T.alloc_workspace(T.lact_bwd_workspace_bytes(desc))
     T.lact_chunk_bwd(desc, to_dev(x.q), to_dev(x.k), to_dev(x.v), torch.from_numpy(x.lr).cuda(),
                      state0, to_dev(g.dout), dW_end, *grads, ws)
     assert T.ttt_check_device_status(ws) == T.TTT_OK
@@ -53,8 +69,8 @@ def _oracle(x, g, opt="gd", with_dw=True, **kw):
                                   opt=opt, **okw)
 
 
-def _check(x, g, opt="gd", with_dw=True, **kw):
-    got = _run(x, g, opt, with_dw, **kw)
+def _check(x, g, opt="gd", with_dw=True, offset16=False, **kw):
+    got = _run(x, g, opt, with_dw, offset16, **kw)
     ref = _oracle(x, g, opt, with_dw, **kw)
     for name, a, r in zip(NAMES, got, ref):
         assert not np.isnan(a).any(), name
@@ -66,6 +82,13 @@ def test_causal_chunks(cuda_device, opt):
     """Three chunks (128, 128, 72 tokens: the last ragged), d = 128, dh = 256."""
     x = make_lact_inputs(1, 2, 328, 128, 256, chunk=128, order="causal", cfg=81)
     _check(x, make_lact_grads(x, cfg=81), opt, beta=0.9)
+
+
+def test_buffers_only_16_byte_aligned(cuda_device):
+    """Gradient outputs and workspace 16 bytes past a 32-byte boundary: the
+    kernels' 256-bit stores give way to 128-bit ones."""
+    x = make_lact_inputs(1, 2, 300, 128, 256, chunk=128, order="causal", cfg=86)
+    _check(x, make_lact_grads(x, cfg=86), "momentum", beta=0.9, offset16=True)
 
 
 def test_causal_without_end_gradient(cuda_device):
