@@ -190,6 +190,15 @@ TTT_DEVICE_INLINE void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* ba
       : "memory");
 }
 
+TTT_DEVICE_INLINE void tma_load_4d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y,
+                                   int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
 // Make generic-proxy shared-memory writes visible to the async proxy
 // (tcgen05.mma operand reads, TMA stores).
 TTT_DEVICE_INLINE void fence_async_smem() {

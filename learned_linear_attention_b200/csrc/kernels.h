@@ -67,6 +67,15 @@ inline int allow_dynamic_smem(void (*kernel)(KArgs...), int bytes, std::atomic<u
 int make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                       uint64_t batch, uint64_t row_stride, uint64_t batch_stride,
                       uint32_t box_inner, uint32_t box_rows);
+// The same bf16 matrices [batch][rows][inner] seen as 4-D {64, rows,
+// inner / 64, batch}: the third dimension steps 128 bytes, one 64-element
+// block of a row.  A box {64, box_rows, box_blocks, 1} lands in shared
+// memory as box_blocks blocks of box_rows 128-byte rows (8 KB apart for 64
+// rows), the MN-major operand layout of the tensor cores with 128-byte
+// swizzle, so one copy brings a whole MN-major operand block.
+int make_tmap_bf16_blocked(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                           uint64_t batch, uint64_t row_stride, uint64_t batch_stride,
+                           uint32_t box_rows, uint32_t box_blocks);
 
 // ----------------------------------------------------------------- TTT-linear
 // Sequence split of the tensor-core linear kernel (see ttt_linear.cu).
@@ -212,7 +221,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream);
 
 // Backward pass of the LaCT layer (lact_bwd.cu).
 struct LactBwdWorkspace {
-  size_t status, fws, fws_bytes, state, wsave, rn, G, dW, dM, R, Rb, Wb, ddy, total;
+  size_t status, fws, fws_bytes, state, wsave, rn, G, dW, dM, R, Rb, Wb, ddy, gctr, total;
   size_t f32[6], b16[7];   // per-chunk intermediates [BH][cmax][dh]
   int cmax, nch;
 };

@@ -565,6 +565,7 @@ LactBwdWorkspace lact_bwd_layout(const LactLaunch& f) {
   for (int i = 0; i < 6; ++i) { w.f32[i] = o; o = al(o + inter * 4); }
   for (int i = 0; i < 7; ++i) { w.b16[i] = o; o = al(o + inter * 2); }
   w.ddy = o; o = al(o + BH * w.cmax * f.d * 4);
+  w.gctr = o; o = al(o + (size_t)std::max(nch, 1) * 4);   // unit counters of the grouped launches
   w.total = o;
   return w;
 }
@@ -758,17 +759,45 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     return read_dq(t0, C);
   };
 
-  // The products of a chunk on the fused path, in one grouped launch:
-  //   dk rows  = d_h1 W1 + d_h3 W3 + e1 R1 + e3 R3       (M = C, N = d, K = 4 dh)
-  //   d_dy     = d_dg W2^T + g R2^T                        (M = C, N = d, K = 2 dh)
-  //   dq rows  = dhq1 W1 + dhq3 W3                         (with the read; M = C, N = d)
-  //   dW1, dW3 partials = d_h1^T K (+ dhq1^T Q), d_h3^T K (+ dhq3^T Q)   (M = dh, N = d)
-  //   dW2 partial       = V^T (-lr d_dg) (+ dout^T gq)     (M = d, N = dh)
+  // maps of the grouped launch: K-major token-row operands in boxes of 256
+  // rows, MN-major operands through blocked views (one copy per block)
+  CUtensorMap gk_b16[7], gk_rb16[3], gm_b16[7], gm_rb16[3], gm_w[4], gm_tok[4];
+  if (fused_fwd) {
+    for (int i = 0; i < 7; ++i)
+      BWD_TRY(make_tmap_bf16_3d(&gk_b16[i], b16[i], dh, w.cmax, BHu, (uint64_t)dh * 2,
+                                (uint64_t)dh * 2 * w.cmax, 64, 256) |
+              make_tmap_bf16_blocked(&gm_b16[i], b16[i], dh, w.cmax, BHu, (uint64_t)dh * 2,
+                                     (uint64_t)dh * 2 * w.cmax, 64, 4));
+    for (int i = 0; i < 3; ++i)
+      BWD_TRY(make_tmap_bf16_3d(&gk_rb16[i], rb16[i], dh, w.cmax, BHu, (uint64_t)dh * 2,
+                                (uint64_t)dh * 2 * w.cmax, 64, 256) |
+              make_tmap_bf16_blocked(&gm_rb16[i], rb16[i], dh, w.cmax, BHu, (uint64_t)dh * 2,
+                                     (uint64_t)dh * 2 * w.cmax, 64, 4));
+    // W1, W3, R1, R3 as [m = d][k = hidden] (MN-major A)
+    const __nv_bfloat16* wsrc[4] = {Wb, Wb + mat, Rb, Rb + mat};
+    for (int i = 0; i < 4; ++i)
+      BWD_TRY(make_tmap_bf16_blocked(&gm_w[i], wsrc[i], d, dh, BHu, (uint64_t)d * 2,
+                                     (uint64_t)d * dh * 2, 64, 2));
+    // K, V (N_in rows), Q, dout (q_rows rows) as [m = d][k = token] (MN-major A)
+    const void* tsrc[4] = {f.k, f.v, f.q, L.dout};
+    const int trows[4] = {f.N_in, f.N_in, q_rows, q_rows};
+    for (int i = 0; i < 4; ++i)
+      if (tsrc[i] != nullptr && trows[i] > 0)
+        BWD_TRY(make_tmap_bf16_blocked(&gm_tok[i], tsrc[i], d, trows[i], BHu, (uint64_t)d * 2,
+                                       (uint64_t)d * 2 * trows[i], 64, 2));
+  }
+  // The products of a chunk on the fused path, in one grouped launch, each
+  // posed with M = d and N the long side (tokens or hidden units):
+  //   dk rows^T  = W1^T d_h1^T + W3^T d_h3^T + R1^T e1^T + R3^T e3^T   (N = C, K = 4 dh)
+  //   d_dy^T     = W2 d_dg^T + R2 g^T                                   (N = C, K = 2 dh)
+  //   dq rows^T  = W1^T dhq1^T + W3^T dhq3^T                            (with the read)
+  //   dW1^T, dW3^T partials = K^T d_h1 (+ Q^T dhq1), K^T d_h3 (+ Q^T dhq3)   (N = dh)
+  //   dW2 partial           = V^T (-lr d_dg) (+ dout^T gq)                   (N = dh)
   // the weight-gradient products split over the chunk's tokens into the
-  // (free) fp32 intermediates, then one pass adds the splits to dW (16 output
-  // tiles per matrix would leave most SMs idle); steps past the chunk read
-  // zero rows of the bf16 intermediates.  Each split's partial is d x dh per
-  // head, so S splits fit the region while S d <= cmax.
+  // (free) fp32 intermediates, then one pass adds the splits to dW (a few
+  // output tiles per matrix would leave most SMs idle); steps past the chunk
+  // read zero rows of the bf16 intermediates.  Each split's partial is
+  // d x dh per head, so S splits fit the region while S d <= cmax.
   static std::atomic<uint64_t> group_attr{0};
   if (fused_fwd && allow_dynamic_smem(gemm_group_kernel, (int)gg::SMEM, group_attr)) return -1;
   auto chunk_products = [&](int t0, int C, bool with_read) -> int {
@@ -777,13 +806,14 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     GroupMaps m{};
     GroupArgs g{};
     g.st = L.st;
+    g.ctr = reinterpret_cast<unsigned int*>(ws + w.gctr) + t0 / f.chunk;
     int units = 0;
-    auto add = [&](int M, int N, int splits, int k_steps, int np, bool a_mn, bool b_mn,
+    auto add = [&](int N, int splits, int k_steps, int np, bool a_mn, bool b_mn,
                    const CUtensorMap* A, const CUtensorMap* B, int a_k_off, int b_k_off, float* o,
-                   long long o_bs, long long o_ss, int ld, int row_off) {
+                   long long o_bs, long long o_ss, int ld, bool out_t, int row_off) {
       GroupProblem& q = g.p[g.nprob];
-      q.M = M; q.N = N;
-      q.tiles_m = (M + 127) / 128; q.tiles_n = N / gg::BN; q.splits = splits;
+      q.M = d; q.N = N;
+      q.tiles_m = d / 128; q.tiles_n = (N + gg::BN - 1) / gg::BN; q.splits = splits;
       q.k_steps = k_steps; q.npairs = np; q.a_mn = a_mn ? 1 : 0; q.b_mn = b_mn ? 1 : 0;
       q.unit0 = units;
       for (int i = 0; i < np; ++i) {
@@ -792,7 +822,7 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
         q.a_k_off[i] = a_k_off;
         q.b_k_off[i] = b_k_off;
       }
-      q.o = o; q.o_bs = o_bs; q.o_ss = o_ss; q.ld = ld; q.out_row_off = row_off;
+      q.o = o; q.o_bs = o_bs; q.o_ss = o_ss; q.ld = ld; q.out_t = out_t ? 1 : 0; q.row_off = row_off;
       q.v8 = (reinterpret_cast<uintptr_t>(o) % 32 == 0 && ld % 8 == 0 && o_bs % 8 == 0 &&
               o_ss % 8 == 0) ? 1 : 0;
       units += q.tiles_m * q.tiles_n * splits * BH;
@@ -800,32 +830,34 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     };
     const int kd = dh / 64;
     {
-      const CUtensorMap A[4] = {mb_k[0], mb_k[1], mb_k[4], mb_k[5]}, B[4] = {mW1mn, mW3mn, mR1mn, mR3mn};
-      add(C, d, 1, kd, 4, false, true, A, B, 0, 0, L.dk, (long long)f.N_in * d, 0, d, t0);
+      const CUtensorMap A[4] = {gm_w[0], gm_w[1], gm_w[2], gm_w[3]};
+      const CUtensorMap B[4] = {gk_b16[0], gk_b16[1], gk_b16[4], gk_b16[5]};
+      add(C, 1, kd, 4, true, false, A, B, 0, 0, L.dk, (long long)f.N_in * d, 0, d, true, t0);
     }
     {
-      const CUtensorMap A[2] = {mb_k[2], mb_k[6]}, B[2] = {mW2k, mR2k};
-      add(C, d, 1, kd, 2, false, false, A, B, 0, 0, F(w.ddy), (long long)w.cmax * d, 0, d, 0);
+      const CUtensorMap A[2] = {mW2k, mR2k}, B[2] = {gk_b16[2], gk_b16[6]};
+      add(C, 1, kd, 2, false, false, A, B, 0, 0, F(w.ddy), (long long)w.cmax * d, 0, d, true, 0);
     }
     if (with_read) {
-      const CUtensorMap A[2] = {mrb_k[0], mrb_k[1]}, B[2] = {mW1mn, mW3mn};
-      add(C, d, 1, kd, 2, false, true, A, B, 0, 0, L.dq, (long long)q_rows * d, 0, d, t0);
+      const CUtensorMap A[2] = {gm_w[0], gm_w[1]}, B[2] = {gk_rb16[0], gk_rb16[1]};
+      add(C, 1, kd, 2, true, false, A, B, 0, 0, L.dq, (long long)q_rows * d, 0, d, true, t0);
     }
     const int np = with_read ? 2 : 1;
     const long long wsz = (long long)d * dh;
     {
-      const CUtensorMap A1[2] = {mb_mn[0], mrb_mn[0]}, A3[2] = {mb_mn[1], mrb_mn[1]}, B13[2] = {mk_mn, mq_mn};
-      add(dh, d, S, kps, np, true, true, A1, B13, 0, t0, f32[3], S * wsz, wsz, d, 0);
-      add(dh, d, S, kps, np, true, true, A3, B13, 0, t0, f32[4], S * wsz, wsz, d, 0);
+      const CUtensorMap A13[2] = {gm_tok[0], gm_tok[2]};
+      const CUtensorMap B1[2] = {gm_b16[0], gm_rb16[0]}, B3[2] = {gm_b16[1], gm_rb16[1]};
+      add(dh, S, kps, np, true, true, A13, B1, t0, 0, f32[3], S * wsz, wsz, d, true, 0);
+      add(dh, S, kps, np, true, true, A13, B3, t0, 0, f32[4], S * wsz, wsz, d, true, 0);
     }
     {
-      const CUtensorMap A2[2] = {mv_mn, mdo_mn}, B2[2] = {mb_mn[3], mrb_mn[2]};
-      add(d, dh, S, kps, np, true, true, A2, B2, t0, 0, f32[5], S * wsz, wsz, dh, 0);
+      const CUtensorMap A2[2] = {gm_tok[1], gm_tok[3]}, B2[2] = {gm_b16[3], gm_rb16[2]};
+      add(dh, S, kps, np, true, true, A2, B2, t0, 0, f32[5], S * wsz, wsz, dh, false, 0);
     }
     g.units = units;
     prof_before(K_BWD_GROUP, stream);
     const cudaError_t e = launch_pdl(gemm_group_kernel, dim3((unsigned)std::min(units, num_sms_bwd())),
-                                     dim3(192), gg::SMEM, stream, m, g);
+                                     dim3(gg::THREADS), gg::SMEM, stream, m, g);
     prof_after(K_BWD_GROUP, stream);
     if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return -1;
     WgradSumArgs sa{BH, S, wsz, {f32[3], f32[4], f32[5]}, {dW1, dW3, dW2}};
@@ -840,6 +872,8 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
   else
     BWD_TRY(cudaMemsetAsync(dW, 0, 3 * mat * 4, stream) == cudaSuccess ? 0 : -1);
   BWD_TRY(cudaMemsetAsync(dM, 0, 3 * mat * 4, stream) == cudaSuccess ? 0 : -1);
+  if (fused_fwd && nch > 0)
+    BWD_TRY(cudaMemsetAsync(ws + w.gctr, 0, (size_t)nch * 4, stream) == cudaSuccess ? 0 : -1);
   if (!f.causal && f.N_q > 0) {   // the queries read the final weights
     BWD_TRY(cast(wsave + (size_t)nch * 3 * mat, Wb, 3 * mat));
     BWD_TRY(read_vjp(0, f.N_q));
