@@ -70,8 +70,14 @@ struct RowStepArgs {
   const float* rn;       // row norms of U_c, [BH][2 dh + d]
   float* R;              // out: dL/dG_c (fp32)
   __nv_bfloat16* Rb;     // out: bf16 copy
+  const float* Wc;       // W_c (the chunk's start weights), cast to Wb alongside
+  __nv_bfloat16* Wb;
 };
-// One warp per row of one matrix of one head (rows of up to 1024 columns).
+// One warp per row of one matrix of one head (rows of 128 to 1024 columns,
+// a multiple of 128): each lane holds four-column slices of the row in
+// registers across the two passes (projection onto W_{c+1}, then the step).
+// The same warp writes the bf16 copy of the row of W_c the chunk's products
+// read.
 __global__ void bwd_row_step_kernel(RowStepArgs a) {
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int per = 2 * a.dh + a.d;
@@ -82,39 +88,74 @@ __global__ void bwd_row_step_kernel(RowStepArgs a) {
   const int rows = mat < 2 ? a.dh : a.d, cols = mat < 2 ? a.d : a.dh;
   const size_t mat_elems = (size_t)a.BH * a.d * a.dh;
   const size_t off = mat * mat_elems + ((size_t)bh * rows + row) * cols;
+  const int nv = cols / 128;   // float4 slices per lane (<= 8)
+  {
+    const float4* wc = reinterpret_cast<const float4*>(a.Wc + off);
+    uint2* wb = reinterpret_cast<uint2*>(a.Wb + off);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k < nv) {
+        const float4 x = wc[k * 32 + lane];
+        wb[k * 32 + lane] = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+      }
+  }
+  float4* R4 = reinterpret_cast<float4*>(a.R + off);
+  uint2* Rb2 = reinterpret_cast<uint2*>(a.Rb + off);
   if (!(a.mask & (1 << mat))) {   // not updated: no dependence on G, dW passes through
-    for (int c = lane; c < cols; c += 32) {
-      a.R[off + c] = 0.f;
-      a.Rb[off + c] = __float2bfloat16_rn(0.f);
-    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k < nv) {
+        R4[k * 32 + lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        Rb2[k * 32 + lane] = make_uint2(0u, 0u);
+      }
     return;
   }
-  float* dW = a.dW + off;
+  float4* dW4 = reinterpret_cast<float4*>(a.dW + off);
+  const float4* Wn4 = reinterpret_cast<const float4*>(a.Wn + off);
+  float4 du[8], wn[8];
   float proj = 0.f, inv = 1.f;
   bool big = true;
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    if (k < nv) {
+      du[k] = dW4[k * 32 + lane];
+      if (a.normalize) {
+        wn[k] = Wn4[k * 32 + lane];
+        proj += wn[k].x * du[k].x + wn[k].y * du[k].y + wn[k].z * du[k].z + wn[k].w * du[k].w;
+      }
+    }
   if (a.normalize) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) proj += __shfl_xor_sync(0xffffffffu, proj, o);
     const float n = a.rn[gw];
     big = n > a.norm_eps;
     inv = 1.f / (big ? n : a.norm_eps);
-    for (int c = lane; c < cols; c += 32) proj += a.Wn[off + c] * dW[c];
+  }
+  float4* dM4 = reinterpret_cast<float4*>(a.dM + off);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) proj += __shfl_xor_sync(0xffffffffu, proj, o);
-  }
-  for (int c = lane; c < cols; c += 32) {
-    float du = dW[c];
-    if (a.normalize) du = big ? (du - a.Wn[off + c] * proj) * inv : du * inv;
-    float r;
-    if (a.momentum) {
-      const float m = a.dM[off + c] - du;
-      r = m;
-      a.dM[off + c] = a.beta * m;
-    } else {
-      r = -du;
+  for (int k = 0; k < 8; ++k)
+    if (k < nv) {
+      float4 u = du[k];
+      if (a.normalize) {
+        if (big) {
+          u.x = (u.x - wn[k].x * proj) * inv; u.y = (u.y - wn[k].y * proj) * inv;
+          u.z = (u.z - wn[k].z * proj) * inv; u.w = (u.w - wn[k].w * proj) * inv;
+        } else {
+          u.x *= inv; u.y *= inv; u.z *= inv; u.w *= inv;
+        }
+      }
+      float4 r;
+      if (a.momentum) {
+        const float4 m0 = dM4[k * 32 + lane];
+        r = make_float4(m0.x - u.x, m0.y - u.y, m0.z - u.z, m0.w - u.w);
+        dM4[k * 32 + lane] = make_float4(a.beta * r.x, a.beta * r.y, a.beta * r.z, a.beta * r.w);
+      } else {
+        r = make_float4(-u.x, -u.y, -u.z, -u.w);
+      }
+      dW4[k * 32 + lane] = u;
+      R4[k * 32 + lane] = r;
+      Rb2[k * 32 + lane] = make_uint2(pack_bf16x2(r.x, r.y), pack_bf16x2(r.z, r.w));
     }
-    dW[c] = du;
-    a.R[off + c] = r;
-    a.Rb[off + c] = __float2bfloat16_rn(r);
-  }
 }
 
 struct KeyEwArgs {
@@ -188,17 +229,21 @@ __global__ void bwd_read_ew_kernel(ReadEwArgs a) {
 // dv = -lr d_dy, dlr = -v . d_dy for the chunk's tokens (one warp per token).
 __global__ void bwd_dv_kernel(int BH, int C, int cmax, int d, int N, int t0, const float* lr,
                               const __nv_bfloat16* v, const float* ddy, float* dv, float* dlr) {
+  // one warp per token row, four consecutive columns per lane (d % 128 == 0)
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (gw >= BH * C) return;
   const int bh = gw / C, t = gw % C;
   const size_t tok = (size_t)bh * N + t0 + t;
   const float eta = lr[tok];
-  const float* src = ddy + ((size_t)bh * cmax + t) * d;
+  const float4* src = reinterpret_cast<const float4*>(ddy + ((size_t)bh * cmax + t) * d);
+  const uint2* vr = reinterpret_cast<const uint2*>(v + tok * d);
+  float4* dst = reinterpret_cast<float4*>(dv + tok * d);
   float acc = 0.f;
-  for (int c = lane; c < d; c += 32) {
-    const float x = src[c];
-    dv[tok * d + c] = -eta * x;
-    acc += __bfloat162float(v[tok * d + c]) * x;
+  for (int c = lane; c < d / 4; c += 32) {
+    const float4 x = src[c];
+    const uint2 vv = vr[c];
+    dst[c] = make_float4(-eta * x.x, -eta * x.y, -eta * x.z, -eta * x.w);
+    acc += bf16lo(vv.x) * x.x + bf16hi(vv.x) * x.y + bf16lo(vv.y) * x.z + bf16hi(vv.y) * x.w;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -881,16 +926,16 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
   RowStepArgs rs{};
   rs.BH = BH; rs.d = d; rs.dh = dh; rs.mask = f.update_mask; rs.normalize = f.normalize_rows;
   rs.momentum = f.opt == 1; rs.beta = f.beta; rs.norm_eps = f.norm_eps;
-  rs.dW = dW; rs.dM = dM; rs.R = F(w.R); rs.Rb = Rb;
+  rs.dW = dW; rs.dM = dM; rs.R = F(w.R); rs.Rb = Rb; rs.Wb = Wb;
   const int row_warps = BH * (2 * dh + d);
   for (int c = nch - 1; c >= 0; --c) {
     const int t0 = c * f.chunk, C = std::min(f.chunk, f.N_in - t0);
     const int ks = (C + 63) / 64;
     rs.Wn = wsave + (size_t)(c + 1) * 3 * mat;
     rs.rn = rn + (size_t)c * BH * (2 * dh + d);
+    rs.Wc = wsave + (size_t)c * 3 * mat;   // its bf16 copy is the chunk's product operand
     bwd_row_step_kernel<<<(row_warps * 32 + 255) / 256, 256, 0, stream>>>(rs);
     BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
-    BWD_TRY(cast(wsave + (size_t)c * 3 * mat, Wb, 3 * mat));
     // a causal chunk on the fused path: the read's elementwise step too, so
     // both feed the weight-gradient products below
     const bool both = fused_fwd && f.causal;
