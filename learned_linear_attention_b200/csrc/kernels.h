@@ -171,8 +171,14 @@ struct LactLaunch {
   float* G;                // [G1 | G3 | G2] fp32, laid out like the weights of the state
   float* rownorm_out;      // APPLY, nullable: each updated row's norm before the
                            // normalisation, [BH][2 dh + d] (W1 rows, W3 rows, W2 rows)
+  // LACT_REPLAY (the backward pass's forward replay): the chunk sequence
+  // without the read, keeping the fp32 weights at the start of every chunk
+  // and after the last ([chunks + 1][W1 | W3 | W2]) and the row norms of
+  // every update ([chunks][BH][2 dh + d]).
+  float* wsave;
+  float* rownorm_all;
 };
-enum LactMode { LACT_FULL = 0, LACT_GRAD = 1, LACT_APPLY = 2, LACT_READ = 3 };
+enum LactMode { LACT_FULL = 0, LACT_GRAD = 1, LACT_APPLY = 2, LACT_READ = 3, LACT_REPLAY = 4 };
 // The batched tcgen05 GEMM of gemm.cuh (operand majorness by variant).
 struct GemmMaps;
 struct GemmArgs;

@@ -1137,6 +1137,15 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   }
   ra.nbuf = 1;
   TTT_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
+  // replay: the chunk's start weights are kept, and its update records the
+  // row norms
+  auto replay_save = [&](int chunk) -> int {
+    if (L.mode != LACT_REPLAY) return 0;
+    ra.rownorm = L.rownorm_all ? L.rownorm_all + (size_t)chunk * BH * (2 * dh + d) : nullptr;
+    if (L.wsave == nullptr) return 0;
+    return cudaMemcpyAsync(L.wsave + (size_t)chunk * 3 * mat_elems, L.state, 3 * mat_elems * sizeof(float),
+                           cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1;
+  };
 
   // ---- tensor maps.  Token tensors {d, rows, BH}; K-major boxes {64, 128},
   // MN-major boxes {64, 64}.  Weights (bf16 copies): W1, W3 [BH][dh][d],
@@ -1161,7 +1170,8 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   };
   // which token tensors this call reads (the context-parallel pieces read a
   // subset and may leave the others null)
-  const bool uses_kv = L.N_in > 0 && (L.mode == LACT_FULL || L.mode == LACT_GRAD);
+  const bool uses_kv =
+      L.N_in > 0 && (L.mode == LACT_FULL || L.mode == LACT_GRAD || L.mode == LACT_REPLAY);
   const bool uses_q = q_rows > 0 && (L.mode == LACT_FULL || L.mode == LACT_READ);
   KeyPassMaps km{};
   if (uses_kv) {
@@ -1200,6 +1210,8 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   if (allow_dynamic_smem(lact_keypass_kernel, (int)kp::SMEM, kp_attr)) return -1;
 
   auto key_pass_on = [&](int t0, int C, int nkt, int nqt, cudaStream_t kstream) -> int {
+    // never launch on a token map this call did not encode
+    if ((nkt > 0 && !uses_kv) || (nqt > 0 && !uses_q)) return -1;
     KeyPassArgs a{};
     a.C = C; a.t0 = t0; a.n_key_tiles = nkt; a.n_q_tiles = nqt; a.n_hb = dh / 64; a.BH = BH;
     a.d_steps = d / 64; a.dh = dh; a.lr_len = L.N_in; a.lr = L.lr;
@@ -1256,12 +1268,13 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // partial sums go to the row update kernels.
   const int cmax_chunk = std::min(L.chunk, std::max(L.N_in, 1));
   const bool fused_update = L.opt != 2 && (d == 128 || d == 256) && (dh == 128 || dh == 256) &&
-                            cmax_chunk <= 8192;
+                            cmax_chunk <= 8192 && L.mode != LACT_REPLAY;
   auto d13_map = [&](CUtensorMap* m, const void* p, int rows) {
     return make_tmap_bf16_3d(m, p, 2 * dh, rows, BH, (uint64_t)dh * 4, (uint64_t)w.cmax * dh * 4,
                              64, 64);
   };
   auto gradients = [&](int t0, int C, cudaStream_t* mstream, bool partials_only) -> int {
+    if (!uses_kv) return -1;   // the K / V maps were not encoded for this call
     CUtensorMap md, mdl, mg, mgl;
     TTT_TRY(d13_map(&md, D13, C));
     TTT_TRY(inter_map(&mg, Gm, C, 64));
@@ -1618,17 +1631,18 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     kgl.BH = BH; kgl.N_in = L.N_in; kgl.C = C; kgl.t0 = t0; kgl.dh = dh;
     kgl.groups = keygrad_groups(BH, dh, C, w.splits);
     kgl.k = L.k; kgl.v = L.v; kgl.lr = L.lr;
-    kgl.q = L.causal ? L.q : nullptr;
+    const bool reads = L.causal && L.mode != LACT_REPLAY;
+    kgl.q = reads ? L.q : nullptr;
     kgl.Aq = aq; kgl.aq_bs = (long long)w.cmax * dh;
     kgl.w1b = wbuf[cur][0]; kgl.w3b = wbuf[cur][1]; kgl.w2b = wbuf[cur][2];
     kgl.part[0] = const_cast<float*>(ra.part[0]);
     kgl.part[1] = const_cast<float*>(ra.part[1]);
     kgl.part[2] = const_cast<float*>(ra.part[2]);
     kgl.st = L.st;
-    if (L.causal && ss && ci >= w.naq)
+    if (reads && ss && ci >= w.naq)
       TTT_TRY(cudaStreamWaitEvent(stream, ss->read_done[ci & 1], 0) == cudaSuccess ? 0 : -1);
     TTT_TRY(launch_lact_keygrad(kgl, stream));
-    if (L.causal) {   // the read of this chunk runs beside the update and the next chunk
+    if (reads) {   // the read of this chunk runs beside the update and the next chunk
       if (ss) {
         TTT_TRY(cudaEventRecord(ss->fork, stream) == cudaSuccess ? 0 : -1);
         TTT_TRY(cudaStreamWaitEvent(rstream, ss->fork, 0) == cudaSuccess ? 0 : -1);
@@ -1639,17 +1653,19 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     }
     ra.splits = kgl.groups;
     set_out_buf(nxt(cur));
+    TTT_TRY(replay_save(ci));
     TTT_TRY(row_update(stream));
     cur = nxt(cur);
   }
-  if (keygrad && L.causal && ss && ci >= 1)   // the reads join the caller's stream
+  if (keygrad && L.causal && L.mode != LACT_REPLAY && ss && ci >= 1)   // the reads join the caller's stream
     TTT_TRY(cudaStreamWaitEvent(stream, ss->read_done[(ci - 1) & 1], 0) == cudaSuccess ? 0 : -1);
-  for (int t0 = 0; !keygrad && t0 < L.N_in; t0 += L.chunk) {
+  for (int t0 = 0; !keygrad && t0 < L.N_in; t0 += L.chunk, ++ci) {
     const int C = std::min(L.chunk, L.N_in - t0);
     const int nt = (C + 127) / 128;
-    TTT_TRY(key_pass(t0, C, nt, L.causal ? nt : 0));
+    const bool reads = L.causal && L.mode != LACT_REPLAY;
+    TTT_TRY(key_pass(t0, C, nt, reads ? nt : 0));
     TTT_TRY(fork());
-    if (L.causal) TTT_TRY(read_out(t0, C, rstream, Aq));
+    if (reads) TTT_TRY(read_out(t0, C, rstream, Aq));
     const int splits = gradients(t0, C, gstream, false);
     if (splits < 0) return -1;
     TTT_TRY(join());
@@ -1659,6 +1675,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     }
     ra.splits = splits;
     set_out_buf(nxt(cur));
+    TTT_TRY(replay_save(ci));
     if (L.opt == 2) {
       TTT_TRY(muon());
     } else {
@@ -1666,7 +1683,10 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     }
     cur = nxt(cur);
   }
-  if (!L.causal && L.N_q > 0) {
+  if (L.mode == LACT_REPLAY && L.wsave != nullptr)   // the weights after the last chunk
+    TTT_TRY(cudaMemcpyAsync(L.wsave + (size_t)ci * 3 * mat_elems, L.state, 3 * mat_elems * sizeof(float),
+                            cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1);
+  if (!L.causal && L.N_q > 0 && L.mode != LACT_REPLAY) {
     if (d == 128 && !split) {   // the fused read: Q -> out in one kernel
       ReadFusedLaunch rl{};
       rl.BH = BH; rl.rows = L.N_q; rl.t0 = 0; rl.C = L.N_q; rl.dh = dh; rl.out_bf16 = L.out_bf16;

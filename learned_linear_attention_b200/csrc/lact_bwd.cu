@@ -644,18 +644,11 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
   p.ws_bytes = w.fws_bytes;
   p.split = 0;
   p.rownorm_out = nullptr;
-  for (int c = 0; c < nch; ++c) {
-    const int t0 = c * f.chunk, C = std::min(f.chunk, f.N_in - t0);
-    BWD_TRY(cudaMemcpyAsync(wsave + (size_t)c * 3 * mat, state, 3 * mat * 4,
-                            cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1);
-    p.mode = LACT_GRAD; p.t0 = t0; p.n = C; p.G = F(w.G);
-    BWD_TRY(launch_lact(p, stream));
-    p.mode = LACT_APPLY; p.rownorm_out = rn + (size_t)c * BH * (2 * dh + d);
-    BWD_TRY(launch_lact(p, stream));
-    p.rownorm_out = nullptr;
-  }
-  BWD_TRY(cudaMemcpyAsync(wsave + (size_t)nch * 3 * mat, state, 3 * mat * 4,
-                          cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1);
+  p.out = nullptr;
+  p.mode = LACT_REPLAY;
+  p.wsave = wsave;
+  p.rownorm_all = rn;
+  BWD_TRY(launch_lact(p, stream));
 
   // ---------------------------------------------------------------- maps and helpers
   const uint64_t BHu = (uint64_t)BH;
