@@ -199,6 +199,38 @@ TTT_DEVICE_INLINE void tma_load_4d(void* dst, const CUtensorMap* m, uint64_t* ba
       : "memory");
 }
 
+// Barrier `id` (1..15) over `n` threads (a multiple of 32): every thread of
+// the participating warps must reach it on every path.
+TTT_DEVICE_INLINE void named_bar_sync(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Barrier `id` over `n` threads that also ANDs a per-thread flag: every
+// participant gets the same answer, so a loop can leave on it uniformly.
+TTT_DEVICE_INLINE bool named_bar_all(uint32_t id, uint32_t n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// Tensor store shared -> global (bulk async group of the issuing thread).
+// The shared source must not be rewritten before bulk_wait_read() returns;
+// every group is waited for (bulk_wait_all) before the CTA exits.
+TTT_DEVICE_INLINE void tma_store_3d(const CUtensorMap* m, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+TTT_DEVICE_INLINE void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+TTT_DEVICE_INLINE void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+TTT_DEVICE_INLINE void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Make generic-proxy shared-memory writes visible to the async proxy
 // (tcgen05.mma operand reads, TMA stores).
 TTT_DEVICE_INLINE void fence_async_smem() {

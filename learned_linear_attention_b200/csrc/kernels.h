@@ -73,6 +73,10 @@ int make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t
 // memory as box_blocks blocks of box_rows 128-byte rows (8 KB apart for 64
 // rows), the MN-major operand layout of the tensor cores with 128-byte
 // swizzle, so one copy brings a whole MN-major operand block.
+// As make_tmap_bf16_3d with the swizzle given in bytes (0, 32, 64 or 128).
+int make_tmap_bf16_3d_sw(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                         uint64_t batch, uint64_t row_stride, uint64_t batch_stride,
+                         uint32_t box_inner, uint32_t box_rows, int swizzle_bytes);
 int make_tmap_bf16_blocked(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                            uint64_t batch, uint64_t row_stride, uint64_t batch_stride,
                            uint32_t box_rows, uint32_t box_blocks);

@@ -291,12 +291,26 @@ constexpr int BM = 128, HB = 64, D = 128;
 constexpr uint32_t ATILE = BM * D * 2;      // 32 KB: 128 token rows x 128 d, two 64-column boxes
 constexpr uint32_t ASTAGE = 2 * ATILE;      // K | V (key) or Q | dout (read)
 constexpr uint32_t B2 = 2 * HB * D * 2;     // 32 KB: two weight blocks of 64 hidden x 128 d
-constexpr uint32_t OFF_A = 0;                               // two A stages
-constexpr uint32_t OFF_B13 = 2 * ASTAGE, OFF_R13 = OFF_B13 + B2, OFF_B2 = OFF_R13 + B2;
-constexpr uint32_t OFF_BAR_KEY = OFF_B2 + B2, OFF_BAR_READ = OFF_R13 + B2 / 2;   // read: [W1|W3], then W2 alone
+constexpr uint32_t STG_OUT = BM * 32 * 2;   // 8 KB: one output's 128 rows x 32 columns (staging)
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
-constexpr uint32_t SMEM_KEY = OFF_BAR_KEY + 256 + 1024, SMEM_READ = OFF_BAR_READ + 256 + 1024;
+// Shared memory.  Key: one token stage (the next tile's loads only have to
+// beat the elementwise step), [W1|W3], [R1|R3], [W2|R2], staging for seven
+// outputs.  Read: two token stages, [W1|W3], W2, staging for three.
+struct Layout {
+  uint32_t nst, b13, r13, b2, stg, bar, bytes;
+};
+__host__ __device__ inline Layout layout(bool key) {
+  Layout l;
+  l.nst = key ? 1u : 2u;
+  l.b13 = l.nst * ASTAGE;
+  l.r13 = l.b13 + B2;
+  l.b2 = key ? l.r13 + B2 : l.r13;          // read: W2 alone where [R1|R3] would go
+  l.stg = key ? l.b2 + B2 : l.r13 + B2 / 2;
+  l.bar = l.stg + (key ? 7u : 3u) * STG_OUT;
+  l.bytes = l.bar + 256 + 1024;
+  return l;
+}
 constexpr uint32_t TM_COLS = 512;
 }  // namespace bf
 
@@ -304,32 +318,28 @@ struct BwdFwdMaps {
   CUtensorMap a0, a1;        // K / V (key) or Q / dout (read): token maps, box {64, 128}
   CUtensorMap w1, w3, w2;    // bf16 weights: W1, W3 box {64 d, 64 rows}; W2 box {64 hidden, 64 d rows}
   CUtensorMap r1, r3, r2;    // key: bf16 R (same shapes)
+  CUtensorMap o[7];          // outputs [BH][cmax][dh] bf16, box {32, 128}, 64-byte swizzle
 };
 struct BwdFwdArgs {
   int BH, C, cmax, dh, t0, lr_len, n_mt, key;
   const float* lr;           // key: [BH][lr_len]
-  __nv_bfloat16* out[7];     // [BH][cmax][dh]: key d_h1, d_h3, d_dg, d_dgn, e1, e3, g; read dhq1, dhq3, gq
-  int v8;                    // every output starts on a 32-byte boundary: 256-bit stores
   DevStatus st;
 };
 
-// 16 bf16 pairs' worth (32 bytes) of one output row
-TTT_DEVICE_INLINE void store_row32(__nv_bfloat16* dst, const uint32_t* o, bool v8) {
-  if (v8) {
-    st_global_v8(dst, o);
-  } else {
-    uint4* d4 = reinterpret_cast<uint4*>(dst);
-    d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
-  }
+// Byte offset of 16-byte chunk `c` (0..3) of row `r` in a 64-byte-row tile
+// under the 64-byte swizzle of the tensor store (chunk ^= bits 1-2 of the row)
+TTT_DEVICE_INLINE uint32_t sw64_offset(int r, int c) {
+  return (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
 }
 
 // Persistent: CTA c takes a contiguous range of the (head, hidden block,
 // token tile) tiles, token tile fastest, so consecutive tiles share their
-// weight blocks (reloaded only when the block changes).  Token tiles are
-// double-buffered, so the next tile's loads and products overlap this
-// tile's elementwise step and stores; one set of accumulators in TMEM (the
-// next tile's products wait until the epilogue has read them out).
+// weight blocks (reloaded only when the block changes).  The next tile's
+// loads and products overlap this tile's elementwise step; one set of
+// accumulators in TMEM (the next tile's products wait until the epilogue has
+// read them out).  The epilogue stages each half tile (32 hidden columns) of
+// every output in shared memory and one lane per output writes it with a
+// tensor store, so the rows leave as whole 64-byte segments.
 __global__ void __launch_bounds__(bf::THREADS, 1)
     bwd_fwd_fused_kernel(const __grid_constant__ BwdFwdMaps maps, const BwdFwdArgs a) {
   using namespace bf;
@@ -337,7 +347,10 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const bool key = a.key != 0;
-  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + (key ? OFF_BAR_KEY : OFF_BAR_READ));   // [2]
+  const Layout lay = layout(key);
+  const uint32_t nst = lay.nst;
+  const int nout = key ? 7 : 3;
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + lay.bar);   // [2]
   uint64_t* a_empty = a_full + 2;     // [2]
   uint64_t* w_full = a_empty + 2;
   uint64_t* w_empty = w_full + 1;
@@ -394,26 +407,26 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
           mbar_arrive_expect_tx(w_full, wbytes);
           // K-major weight blocks: atom h (d 64h .. 64h + 63) = [first 64 rows | second 64 rows]
           for (int h = 0; h < 2; ++h) {
-            tma_load_3d(smem + OFF_B13 + h * (B2 / 2), &maps.w1, w_full, h * 64, j0, bh);
-            tma_load_3d(smem + OFF_B13 + h * (B2 / 2) + B2 / 4, &maps.w3, w_full, h * 64, j0, bh);
+            tma_load_3d(smem + lay.b13 + h * (B2 / 2), &maps.w1, w_full, h * 64, j0, bh);
+            tma_load_3d(smem + lay.b13 + h * (B2 / 2) + B2 / 4, &maps.w3, w_full, h * 64, j0, bh);
           }
           // MN-major W2[:, J] (and R2[:, J]): 128 d rows of 64 hidden units, two 64-row boxes
-          uint8_t* b2 = smem + (key ? OFF_B2 : OFF_R13);
+          uint8_t* b2 = smem + lay.b2;
           for (int h = 0; h < 2; ++h) tma_load_3d(b2 + h * (B2 / 4), &maps.w2, w_full, j0, h * 64, bh);
           if (key) {
             for (int h = 0; h < 2; ++h) {
-              tma_load_3d(smem + OFF_R13 + h * (B2 / 2), &maps.r1, w_full, h * 64, j0, bh);
-              tma_load_3d(smem + OFF_R13 + h * (B2 / 2) + B2 / 4, &maps.r3, w_full, h * 64, j0, bh);
+              tma_load_3d(smem + lay.r13 + h * (B2 / 2), &maps.r1, w_full, h * 64, j0, bh);
+              tma_load_3d(smem + lay.r13 + h * (B2 / 2) + B2 / 4, &maps.r3, w_full, h * 64, j0, bh);
               tma_load_3d(b2 + B2 / 2 + h * (B2 / 4), &maps.r2, w_full, j0, h * 64, bh);
             }
           }
           ++wl;
           cur = grpw;
         }
-        const uint32_t s = at & 1;
-        if (at >= 2 && !W.wait(&a_empty[s], ((at >> 1) - 1) & 1, 2)) { ok = false; break; }
+        const uint32_t s = at % nst, u = at / nst;
+        if (at >= nst && !W.wait(&a_empty[s], (u - 1) & 1, 2)) { ok = false; break; }
         const int row = a.t0 + mt * BM;
-        uint8_t* st = smem + OFF_A + s * ASTAGE;
+        uint8_t* st = smem + s * ASTAGE;
         mbar_arrive_expect_tx(&a_full[s], ASTAGE);
         for (int h = 0; h < 2; ++h) {
           tma_load_3d(st + h * (ATILE / 2), &maps.a0, &a_full[s], h * 64, row, bh);
@@ -427,11 +440,11 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
     if (lane == 0) {
       const uint32_t id_k = make_idesc(128, 128, false, false);          // K-major B, N = 128
       const uint32_t id_mn = make_idesc(128, key ? 128 : 64, false, true);   // MN-major B
-      const uint64_t da = make_sdesc(smem_u32(smem + OFF_A), 16, 1024);
-      const uint64_t db13 = make_sdesc(smem_u32(smem + OFF_B13), 16, 1024);
-      const uint64_t dr13 = make_sdesc(smem_u32(smem + OFF_R13), 16, 1024);
+      const uint64_t da = make_sdesc(smem_u32(smem), 16, 1024);
+      const uint64_t db13 = make_sdesc(smem_u32(smem + lay.b13), 16, 1024);
+      const uint64_t dr13 = make_sdesc(smem_u32(smem + lay.r13), 16, 1024);
       // [W2_J | R2_J]: two 64-wide N blocks 16 KB apart
-      const uint64_t db2 = make_sdesc(smem_u32(smem + (key ? OFF_B2 : OFF_R13)), B2 / 2, 1024);
+      const uint64_t db2 = make_sdesc(smem_u32(smem + lay.b2), B2 / 2, 1024);
       uint32_t am = 0, wu = 0;
       int cur = -1;
       bool ok = true;
@@ -445,8 +458,8 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
           ++wu;
           cur = grpw;
         }
-        const uint32_t s = am & 1;
-        if (!W.wait(&a_full[s], (am >> 1) & 1, 4)) { ok = false; break; }
+        const uint32_t s = am % nst, u = am / nst;
+        if (!W.wait(&a_full[s], u & 1, 4)) { ok = false; break; }
         if (am >= 1 && !W.wait(acc_empty, (am - 1) & 1, 5)) { ok = false; break; }
         tc_fence_after();
         const uint64_t da0 = sdesc_add(da, s * ASTAGE), da1 = sdesc_add(da0, ATILE);
@@ -468,9 +481,12 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
     __syncwarp();
   } else {
     const int q4 = warp & 3;
-    const int cg = (warp - 2) >> 2;                 // 32 hidden columns of the 64
+    const int cg = (warp - 2) >> 2;                 // 16 columns of each 32-column half
     const int r = q4 * 32 + lane;
     const uint32_t lb = (uint32_t)(q4 * 32) << 16;
+    const int ew = warp - 2;                        // epilogue warp 0..7: output ew's store lane
+    const bool issuer = lane == 0 && ew < nout;
+    uint8_t* stg = smem + lay.stg;
     uint32_t ae = 0;
     for (int t = lo; t < hi; ++t, ++ae) {
       int bh, hb, mt;
@@ -479,11 +495,12 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
       const int tok = mt * BM + r;                  // row of the chunk
       const bool valid = tok < a.C;
       const float eta = (key && valid) ? a.lr[(size_t)bh * a.lr_len + a.t0 + tok] : 0.f;
-      if (!W.wait(acc_full, ae & 1, 6)) break;
+      // the epilogue warps meet at named barriers below: they leave together
+      if (!named_bar_all(1, EPI_WARPS * 32, W.wait(acc_full, ae & 1, 6))) break;
       tc_fence_after();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint32_t c0 = (uint32_t)(cg * 32 + h * 16);
+        const uint32_t c0 = (uint32_t)(h * 32 + cg * 16);
         uint32_t x1[16], x3[16], x5[16], y1[16], y3[16], y5[16];
         // every lane takes part in the warp-collective loads
         tmem_ld16_issue(tmem + lb + c0, x1);            // h1 / hq1
@@ -499,14 +516,13 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
           tc_fence_before();
           mbar_arrive(acc_empty);
         }
-        const size_t base = ((size_t)bh * a.cmax + tok) * a.dh + j0 + c0;
-        auto f2 = [](const uint32_t* r, int j) {
-          return make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+        auto f2 = [](const uint32_t* rr, int j) {
+          return make_float2(__uint_as_float(rr[j]), __uint_as_float(rr[j + 1]));
         };
         const float2 one = x2_splat(1.f);
+        uint32_t o[7][8];
         if (key) {
           // pairs of adjacent hidden columns on the packed fp32 instructions
-          uint32_t o[7][8];
           const float2 ne = x2_splat(-eta);
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
@@ -535,16 +551,7 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
             o[5][j >> 1] = pack_bf16x2(ve3.x, ve3.y);
             o[6][j >> 1] = pack_bf16x2(vg.x, vg.y);
           }
-          if (!valid) {   // rows past the chunk hold zeros
-#pragma unroll
-            for (int q = 0; q < 7; ++q)
-#pragma unroll
-              for (int u = 0; u < 8; ++u) o[q][u] = 0u;
-          }
-#pragma unroll
-          for (int q = 0; q < 7; ++q) store_row32(a.out[q] + base, o[q], a.v8 != 0);
         } else {
-          uint32_t o[3][8];
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
             const float2 x = f2(x1, j), y = f2(x3, j), dg = f2(x5, j);
@@ -558,22 +565,38 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
             o[1][j >> 1] = pack_bf16x2(v3.x, v3.y);
             o[2][j >> 1] = pack_bf16x2(vg.x, vg.y);
           }
-          if (!valid) {
+        }
+        if (!valid) {   // rows past the chunk hold zeros
 #pragma unroll
-            for (int q = 0; q < 3; ++q)
+          for (int q = 0; q < 7; ++q)
 #pragma unroll
-              for (int u = 0; u < 8; ++u) o[q][u] = 0u;
+            for (int u = 0; u < 8; ++u) o[q][u] = 0u;
+        }
+        // the staging buffer is free once the previous half's stores have read it
+        if (issuer) bulk_wait_read();
+        named_bar_sync(1, EPI_WARPS * 32);
+        const uint32_t sb = smem_u32(stg);
+#pragma unroll
+        for (int q = 0; q < 7; ++q) {
+          if (q < nout) {
+            st_shared_v4(sb + q * STG_OUT + sw64_offset(r, 2 * cg), o[q][0], o[q][1], o[q][2], o[q][3]);
+            st_shared_v4(sb + q * STG_OUT + sw64_offset(r, 2 * cg + 1), o[q][4], o[q][5], o[q][6], o[q][7]);
           }
-#pragma unroll
-          for (int q = 0; q < 3; ++q) store_row32(a.out[q] + base, o[q], a.v8 != 0);
+        }
+        fence_async_smem();   // the tensor store (async proxy) reads what these threads wrote
+        named_bar_sync(1, EPI_WARPS * 32);
+        if (issuer) {
+          tma_store_3d(&maps.o[ew], stg + ew * STG_OUT, j0 + h * 32, mt * BM, bh);
+          bulk_commit();
         }
       }
     }
+    if (issuer) bulk_wait_all();   // every tensor store is complete before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0 && lane == 0 && W.aborted()) {   // an aborted CTA: its copies land before it leaves
-    for (uint32_t i = at > 2 ? at - 2 : 0; i < at; ++i) W.drain(&a_full[i & 1], (i >> 1) & 1);
+    for (uint32_t i = at > nst ? at - nst : 0; i < at; ++i) W.drain(&a_full[i % nst], (i / nst) & 1);
     if (wl >= 1) W.drain(w_full, (wl - 1) & 1);
   }
   if (warp == 1) {
@@ -738,23 +761,31 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     BWD_TRY(inter(&mrb_k[i], rb16[i], 128) | inter(&mrb_mn[i], rb16[i], 64));
   }
   static std::atomic<uint64_t> fused_attr{0};
-  if (fused_fwd && allow_dynamic_smem(bwd_fwd_fused_kernel, (int)bf::SMEM_KEY, fused_attr)) return -1;
+  const int fused_smem = (int)std::max(bf::layout(true).bytes, bf::layout(false).bytes);
+  if (fused_fwd && allow_dynamic_smem(bwd_fwd_fused_kernel, fused_smem, fused_attr)) return -1;
+  // the fused kernel's outputs as tensor-store targets: boxes of 32 hidden
+  // columns x 128 token rows, 64-byte swizzle (its staging layout)
+  CUtensorMap mo_key[7], mo_read[3];
+  if (fused_fwd) {
+    for (int i = 0; i < 7; ++i)
+      BWD_TRY(make_tmap_bf16_3d_sw(&mo_key[i], b16[i], dh, w.cmax, BHu, (uint64_t)dh * 2,
+                                   (uint64_t)dh * 2 * w.cmax, 32, 128, 64));
+    for (int i = 0; i < 3; ++i)
+      BWD_TRY(make_tmap_bf16_3d_sw(&mo_read[i], rb16[i], dh, w.cmax, BHu, (uint64_t)dh * 2,
+                                   (uint64_t)dh * 2 * w.cmax, 32, 128, 64));
+  }
   auto fused = [&](bool key, const CUtensorMap& a0, const CUtensorMap& a1, int t0, int C) -> int {
     BwdFwdMaps m{};
     m.a0 = a0; m.a1 = a1;
     m.w1 = mW1mn; m.w3 = mW3mn; m.w2 = mW2mn;
     m.r1 = mR1mn; m.r3 = mR3mn; m.r2 = mR2mn;
+    for (int i = 0; i < (key ? 7 : 3); ++i) m.o[i] = key ? mo_key[i] : mo_read[i];
     BwdFwdArgs ba{};
     ba.BH = BH; ba.C = C; ba.cmax = w.cmax; ba.dh = dh; ba.t0 = t0; ba.lr_len = f.N_in;
     ba.n_mt = w.cmax / bf::BM; ba.key = key ? 1 : 0; ba.lr = f.lr; ba.st = L.st;
-    ba.v8 = 1;
-    for (int i = 0; i < 7; ++i) {
-      ba.out[i] = key ? Hb(w.b16[i]) : (i < 3 ? rb16[i] : nullptr);
-      if (reinterpret_cast<uintptr_t>(ba.out[i]) % 32 != 0) ba.v8 = 0;
-    }
     prof_before(K_BWD_FWD, stream);
     bwd_fwd_fused_kernel<<<dim3((unsigned)std::min(ba.n_mt * (dh / bf::HB) * BH, num_sms_bwd())),
-                           dim3(bf::THREADS), key ? bf::SMEM_KEY : bf::SMEM_READ, stream>>>(m, ba);
+                           dim3(bf::THREADS), bf::layout(key).bytes, stream>>>(m, ba);
     prof_after(K_BWD_FWD, stream);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   };

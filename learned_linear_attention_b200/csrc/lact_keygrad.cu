@@ -160,9 +160,6 @@ TTT_DEVICE_INLINE uint32_t query_ops_x2(uint32_t x0, uint32_t x1, uint32_t y0, u
 TTT_DEVICE_INLINE void mbar_arrive_n(uint64_t* bar, uint32_t n) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
 }
-TTT_DEVICE_INLINE void named_bar_sync(uint32_t id, uint32_t n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 // The row update of chunk c inside the chunk loop.  The worker of item
 // (head bh, hidden block hb, token group grp) owns an even share (by token
 // group) of the 64 rows of W1 and of W3 in block hb, and an even share (by
