@@ -208,7 +208,9 @@ TTT_DEVICE_INLINE void epilogue_update(const GemmArgs& g, uint32_t tacc, int b, 
   }
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES>
+// BLK: the MN-major operands come through blocked 4-D maps (make_tmap_bf16_blocked,
+// boxes of 2 blocks for A and BN / 64 for B), one copy per operand per stage.
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool BLK = false>
 __global__ void __launch_bounds__(192, 1)
     gemm_bf16_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs g) {
   using L = GemmSmem<BN, STAGES>;
@@ -296,12 +298,16 @@ __global__ void __launch_bounds__(192, 1)
           const int bn = g.b_n_off[p] + tn * BN, bk = g.b_k_off[p] + ks * 64;
           if (!A_MN) {
             tma_load_3d(sa, &maps.a[p], &full[s], ak, am, b + g.a_b_off);
+          } else if (BLK) {
+            tma_load_4d(sa, &maps.a[p], &full[s], 0, ak, am >> 6, b + g.a_b_off);
           } else {
             tma_load_3d(sa, &maps.a[p], &full[s], am, ak, b + g.a_b_off);
             tma_load_3d(sa + 8192, &maps.a[p], &full[s], am + 64, ak, b + g.a_b_off);
           }
           if (!B_MN) {
             tma_load_3d(sb, &maps.b[p], &full[s], bk, bn, b + g.b_b_off);
+          } else if (BLK) {
+            tma_load_4d(sb, &maps.b[p], &full[s], 0, bk, bn >> 6, b + g.b_b_off);
           } else {
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j)

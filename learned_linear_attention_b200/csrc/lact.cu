@@ -946,10 +946,10 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
   return w;
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES>
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool BLK = false>
 static int run_gemm(const GemmMaps& maps, const GemmArgs& g, cudaStream_t stream, int kind,
                     int max_grid = 0) {
-  auto kfn = gemm_bf16_kernel<BN, A_MN, B_MN, STAGES>;
+  auto kfn = gemm_bf16_kernel<BN, A_MN, B_MN, STAGES, BLK>;
   const int smem = (int)GemmSmem<BN, STAGES>::BYTES;
   static std::atomic<uint64_t> attr_done{0};
   if (allow_dynamic_smem(kfn, smem, attr_done)) return -1;
@@ -1322,6 +1322,22 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     }
     const int splits = std::min(w.splits, ksteps_total);
     const int kps = (ksteps_total + splits - 1) / splits;
+    // the same operands through blocked views: one copy per operand per stage
+    // (A blocks of 128 rows, B blocks of the tile width)
+    const int bn13 = d % 192 == 0 ? 192 : 128, bn2 = dh % 256 == 0 ? 256 : 128;
+    CUtensorMap bd13[2], bk13, bv, bg[2];
+    TTT_TRY(make_tmap_bf16_blocked(&bd13[0], D13, 2 * dh, C, BH, (uint64_t)dh * 4,
+                                   (uint64_t)w.cmax * dh * 4, 64, 2));
+    TTT_TRY(make_tmap_bf16_blocked(&bg[0], Gm, dh, C, BH, (uint64_t)dh * 2,
+                                   (uint64_t)w.cmax * dh * 2, 64, bn2 / 64));
+    if (split) {
+      TTT_TRY(make_tmap_bf16_blocked(&bd13[1], D13lo, 2 * dh, C, BH, (uint64_t)dh * 4,
+                                     (uint64_t)w.cmax * dh * 4, 64, 2));
+      TTT_TRY(make_tmap_bf16_blocked(&bg[1], Gmlo, dh, C, BH, (uint64_t)dh * 2,
+                                     (uint64_t)w.cmax * dh * 2, 64, bn2 / 64));
+    }
+    TTT_TRY(make_tmap_bf16_blocked(&bk13, L.k, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, bn13 / 64));
+    TTT_TRY(make_tmap_bf16_blocked(&bv, L.v, d, L.N_in, BH, tok_row, tok_row * L.N_in, 64, 2));
     GemmArgs g = gemm_defaults(L.st);
     g.batch = BH; g.splits = splits; g.k_steps = kps; g.npairs = np;
     g.o32_ss = (long long)BH * d * dh;
@@ -1331,27 +1347,27 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       if (mat < 2) {
         g.M = dh; g.N = d; g.ld32 = d;
         for (int p = 0; p < np; ++p) {
-          m.a[p] = p == 0 ? md : mdl;
-          m.b[p] = mk_mn;
+          m.a[p] = bd13[p];
+          m.b[p] = bk13;
           g.a_m_off[p] = mat * dh; g.a_k_off[p] = 0; g.b_k_off[p] = t0;
         }
       } else {
         g.M = d; g.N = dh; g.ld32 = dh;
         for (int p = 0; p < np; ++p) {
-          m.a[p] = mv_mn;
-          m.b[p] = p == 0 ? mg : mgl;
+          m.a[p] = bv;
+          m.b[p] = bg[p];
           g.a_m_off[p] = 0; g.a_k_off[p] = t0; g.b_k_off[p] = 0;
         }
       }
       g.o32 = const_cast<float*>(ra.part[mat]);
       // wide N tiles read the long token-major operands fewer times: 192 for
       // [G1; G3] (N = d), 256 for G2 (N = dh)
-      if (mat < 2 && d % 192 == 0)
-        TTT_TRY(run_gemm<192, true, true, 5>(m, g, mstream[mat], K_GEMM_GRAD));
-      else if (mat == 2 && dh % 256 == 0)
-        TTT_TRY(run_gemm<256, true, true, 4>(m, g, mstream[mat], K_GEMM_GRAD));
+      if (mat < 2 && bn13 == 192)
+        TTT_TRY((run_gemm<192, true, true, 5, true>(m, g, mstream[mat], K_GEMM_GRAD)));
+      else if (mat == 2 && bn2 == 256)
+        TTT_TRY((run_gemm<256, true, true, 4, true>(m, g, mstream[mat], K_GEMM_GRAD)));
       else
-        TTT_TRY(run_gemm<128, true, true, 4>(m, g, mstream[mat], K_GEMM_GRAD));
+        TTT_TRY((run_gemm<128, true, true, 4, true>(m, g, mstream[mat], K_GEMM_GRAD)));
     }
     return splits;
   };
