@@ -91,6 +91,14 @@ def test_buffers_only_16_byte_aligned(cuda_device):
     _check(x, make_lact_grads(x, cfg=86), "momentum", beta=0.9, offset16=True)
 
 
+@pytest.mark.parametrize("dh", [128, 384])
+def test_hidden_widths_on_the_fused_route(cuda_device, dh):
+    """d = 128 with dh = 128 (a hidden width below one 256-wide product tile)
+    and dh = 384 (one and a half tiles), causal, a ragged last chunk."""
+    x = make_lact_inputs(1, 2, 200, 128, dh, chunk=128, order="causal", cfg=87)
+    _check(x, make_lact_grads(x, cfg=87), "momentum", beta=0.9)
+
+
 def test_causal_without_end_gradient(cuda_device):
     x = make_lact_inputs(2, 1, 256, 128, 256, chunk=128, order="causal", cfg=82)
     _check(x, make_lact_grads(x, cfg=82), with_dw=False)
