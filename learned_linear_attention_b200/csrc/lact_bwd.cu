@@ -326,6 +326,11 @@ struct BwdFwdArgs {
   DevStatus st;
 };
 
+// TMEM column of product j (0: [h1|h3], 1: [r1|r3], 2: [vw2|vr2]) of the
+// CTA's tile t in the key step: three 128-column products rotate over four
+// slots, so product 0 of tile t + 1 lands in the slot tile t left free
+TTT_DEVICE_INLINE uint32_t key_slot(uint32_t t, int j) { return ((3u * t + (uint32_t)j) & 3u) * 128u; }
+
 // Byte offset of 16-byte chunk `c` (0..3) of row `r` in a 64-byte-row tile
 // under the 64-byte swizzle of the tensor store (chunk ^= bits 1-2 of the row)
 TTT_DEVICE_INLINE uint32_t sw64_offset(int r, int c) {
@@ -354,9 +359,9 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
   uint64_t* a_empty = a_full + 2;     // [2]
   uint64_t* w_full = a_empty + 2;
   uint64_t* w_empty = w_full + 1;
-  uint64_t* acc_full = w_empty + 1;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* fin = acc_empty + 1;
+  uint64_t* acc_full = w_empty + 1;   // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* fin = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   uint32_t* abort_flag = tmem_slot + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -376,8 +381,10 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
     }
     mbar_init(w_full, 1);
     mbar_init(w_empty, 1);
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, EPI_WARPS * 32);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], EPI_WARPS * 32);
+    }
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -460,19 +467,41 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
         }
         const uint32_t s = am % nst, u = am / nst;
         if (!W.wait(&a_full[s], u & 1, 4)) { ok = false; break; }
-        if (am >= 1 && !W.wait(acc_empty, (am - 1) & 1, 5)) { ok = false; break; }
         tc_fence_after();
         const uint64_t da0 = sdesc_add(da, s * ASTAGE), da1 = sdesc_add(da0, ATILE);
+        auto off_a = [](int kk) -> uint32_t { return (kk >> 2) * (ATILE / 2) + (kk & 3) * 32; };
+        auto off_b = [](int kk) -> uint32_t { return (kk >> 2) * (B2 / 2) + (kk & 3) * 32; };
+        if (key) {
+          // three 128-column products in four TMEM slots, rotating: the
+          // first goes to the slot the previous tile left free and starts
+          // before the epilogue has read that tile out
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * (ATILE / 2) + (kk & 3) * 32;
-          const uint32_t offb = (kk >> 2) * (B2 / 2) + (kk & 3) * 32;
-          mma_bf16(tmem, sdesc_add(da0, off), sdesc_add(db13, offb), id_k, kk > 0);
-          if (key) mma_bf16(tmem + 128, sdesc_add(da0, off), sdesc_add(dr13, offb), id_k, kk > 0);
-          mma_bf16(tmem + 256, sdesc_add(da1, off), sdesc_add(db2, kk * 2048), id_mn, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16(tmem + key_slot(am, 0), sdesc_add(da0, off_a(kk)), sdesc_add(db13, off_b(kk)), id_k, kk > 0);
+          if (am >= 1 && !W.wait(&acc_empty[0], (am - 1) & 1, 5)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            mma_bf16(tmem + key_slot(am, 1), sdesc_add(da0, off_a(kk)), sdesc_add(dr13, off_b(kk)), id_k, kk > 0);
+            mma_bf16(tmem + key_slot(am, 2), sdesc_add(da1, off_a(kk)), sdesc_add(db2, kk * 2048), id_mn, kk > 0);
+          }
+          mma_commit(&a_empty[s]);
+          mma_commit(&acc_full[0]);
+        } else {
+          // two accumulator sets of 256 columns: a tile's products only wait
+          // for the epilogue of the tile two back
+          const uint32_t ab = am & 1;
+          if (am >= 2 && !W.wait(&acc_empty[ab], ((am >> 1) - 1) & 1, 5)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t tb = tmem + ab * 256;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            mma_bf16(tb, sdesc_add(da0, off_a(kk)), sdesc_add(db13, off_b(kk)), id_k, kk > 0);
+            mma_bf16(tb + 128, sdesc_add(da1, off_a(kk)), sdesc_add(db2, kk * 2048), id_mn, kk > 0);
+          }
+          mma_commit(&a_empty[s]);
+          mma_commit(&acc_full[ab]);
         }
-        mma_commit(&a_empty[s]);
-        mma_commit(acc_full);
         ++am;
       }
       mma_commit(fin);
@@ -495,26 +524,33 @@ __global__ void __launch_bounds__(bf::THREADS, 1)
       const int tok = mt * BM + r;                  // row of the chunk
       const bool valid = tok < a.C;
       const float eta = (key && valid) ? a.lr[(size_t)bh * a.lr_len + a.t0 + tok] : 0.f;
+      // accumulators of this tile: key, slots rotating over four; read, the
+      // set of the tile's parity
+      const uint32_t eb = key ? 0u : (ae & 1u);
+      const uint32_t e_par = key ? (ae & 1u) : ((ae >> 1) & 1u);
+      const uint32_t p13 = key ? key_slot(ae, 0) : eb * 256;
+      const uint32_t pr13 = key ? key_slot(ae, 1) : 0;
+      const uint32_t p2 = key ? key_slot(ae, 2) : eb * 256 + 128;
       // the epilogue warps meet at named barriers below: they leave together
-      if (!named_bar_all(1, EPI_WARPS * 32, W.wait(acc_full, ae & 1, 6))) break;
+      if (!named_bar_all(1, EPI_WARPS * 32, W.wait(&acc_full[eb], e_par, 6))) break;
       tc_fence_after();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t c0 = (uint32_t)(h * 32 + cg * 16);
         uint32_t x1[16], x3[16], x5[16], y1[16], y3[16], y5[16];
         // every lane takes part in the warp-collective loads
-        tmem_ld16_issue(tmem + lb + c0, x1);            // h1 / hq1
-        tmem_ld16_issue(tmem + lb + 64 + c0, x3);       // h3 / hq3
-        tmem_ld16_issue(tmem + lb + 256 + c0, x5);      // vw2 / dgq
+        tmem_ld16_issue(tmem + lb + p13 + c0, x1);          // h1 / hq1
+        tmem_ld16_issue(tmem + lb + p13 + 64 + c0, x3);     // h3 / hq3
+        tmem_ld16_issue(tmem + lb + p2 + c0, x5);           // vw2 / dgq
         if (key) {
-          tmem_ld16_issue(tmem + lb + 128 + c0, y1);    // r1
-          tmem_ld16_issue(tmem + lb + 192 + c0, y3);    // r3
-          tmem_ld16_issue(tmem + lb + 320 + c0, y5);    // vr2
+          tmem_ld16_issue(tmem + lb + pr13 + c0, y1);       // r1
+          tmem_ld16_issue(tmem + lb + pr13 + 64 + c0, y3);  // r3
+          tmem_ld16_issue(tmem + lb + p2 + 64 + c0, y5);    // vr2
         }
         tmem_wait_ld();
-        if (h == 1) {   // the accumulators are read out: the next tile's products may start
+        if (h == 1) {   // the accumulators are read out: later products may reuse them
           tc_fence_before();
-          mbar_arrive(acc_empty);
+          mbar_arrive(&acc_empty[eb]);
         }
         auto f2 = [](const uint32_t* rr, int j) {
           return make_float2(__uint_as_float(rr[j]), __uint_as_float(rr[j + 1]));
