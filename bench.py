@@ -415,9 +415,11 @@ class LaCTBwdBench(LaCTBench):
         key step ([h1|h3], [r1|r3], [vw2|vr2]: 12 d dh) and of the read step
         ([hq1|hq3], dgq: 6 d dh); the grouped chunk products (dk 8 d dh, d_dy
         4, dq 4, the three weight gradients 12).  The forward replay's
-        key/gradient kernel: 12 d dh per key token."""
+        key/gradient work: 12 d dh per key token."""
         BH, d, dh, N, Nq = self.B * self.H, self.d, self.dh, self.N, self.Nq
-        f = {"lact_keygrad": 12 * d * dh * N * BH}
+        # the forward replay: per-chunk key/gradient kernels, or the chunk
+        # loop without queries (12 d dh per key token either way)
+        f = {"lact_keygrad": 12 * d * dh * N * BH, "lact_loop": 12 * d * dh * N * BH}
         if self.causal:
             f.update({"lact_bwd_fwd": 18 * d * dh * N * BH, "lact_bwd_gemm": 28 * d * dh * N * BH})
         else:

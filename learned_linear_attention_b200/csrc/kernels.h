@@ -280,6 +280,8 @@ struct KeyGradLoopLaunch {
   int groups, workers, readers;   // from lact_loop_plan (0: the launch plans itself)
   int cast_first;             // the kernel writes the start weights' bf16 copies (every buffer
                               // for a matrix the update leaves alone) before the first chunk
+  float* wsave;               // nullable: the weights after every chunk (slots 1 .. chunks)
+  float* rownorm;             // nullable: every update's row norms (normalising layers)
   DevStatus st;
 };
 // 0 when the chunk loop can run this shape on the current device (groups,

@@ -1125,8 +1125,12 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // SMs; it also makes the start weights' bf16 copies itself.
   // TTT_LACT_CHUNK_LOOP=0 in the environment keeps the per-chunk launches.
   int loop_g = 0, loop_nw = 0, loop_nr = 0;
-  const bool use_loop = w.keygrad && L.causal && L.mode == LACT_FULL && !split && L.opt != 2 &&
-                        L.N_in > 0 && L.out != nullptr && w.nbuf == 3 && w.naq == 2 &&
+  // the backward's replay runs the loop too (no queries, no read), when every
+  // matrix is updated (a matrix the update leaves alone is not snapshotted)
+  const bool loop_mode = (L.mode == LACT_FULL && L.out != nullptr) ||
+                         (L.mode == LACT_REPLAY && (L.update_mask & 7) == 7);
+  const bool use_loop = w.keygrad && L.causal && loop_mode && !split && L.opt != 2 &&
+                        L.N_in > 0 && w.nbuf == 3 && w.naq == 2 &&
                         lact_chunk_loop_enabled() &&
                         lact_loop_plan(BH, L.N_in, L.chunk, dh, w.splits, &loop_g, &loop_nw, &loop_nr) == 0;
   if (L.mode != LACT_APPLY && !use_loop) {   // the update of an APPLY call writes its own copies
@@ -1636,6 +1640,16 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
       ll.cast_first = 1;
       ll.groups = loop_g; ll.workers = loop_nw; ll.readers = loop_nr;
       ll.st = L.st;
+      if (L.mode == LACT_REPLAY) {   // keys only; the updates keep every chunk's weights and norms
+        ll.q = nullptr;
+        ll.out = nullptr;
+        ll.readers = 0;
+        ll.wsave = L.wsave;
+        ll.rownorm = L.normalize_rows ? L.rownorm_all : nullptr;
+        if (L.wsave != nullptr)
+          TTT_TRY(cudaMemcpyAsync(L.wsave, L.state, 3 * mat_elems * sizeof(float), cudaMemcpyDeviceToDevice,
+                                  stream) == cudaSuccess ? 0 : -1);
+      }
       TTT_TRY(launch_lact_loop(ll, stream));
       looped = true;
     }
@@ -1699,7 +1713,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     }
     cur = nxt(cur);
   }
-  if (L.mode == LACT_REPLAY && L.wsave != nullptr)   // the weights after the last chunk
+  if (L.mode == LACT_REPLAY && L.wsave != nullptr && !looped)   // the weights after the last chunk
     TTT_TRY(cudaMemcpyAsync(L.wsave + (size_t)ci * 3 * mat_elems, L.state, 3 * mat_elems * sizeof(float),
                             cudaMemcpyDeviceToDevice, stream) == cudaSuccess ? 0 : -1);
   if (!L.causal && L.N_q > 0 && L.mode != LACT_REPLAY) {

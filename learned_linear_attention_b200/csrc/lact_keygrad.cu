@@ -72,6 +72,11 @@ struct KeyGradLoopArgs {
   long long out_bs;      // N * 128
   int cast_first;        // workers write the start weights' bf16 copies first (counted
                          // on the heads' update counters like an update)
+  // the backward pass's replay (nullable): the weights after chunk c go to
+  // wsave + (c + 1) [W1 | W3 | W2], and each updated row's norm before the
+  // normalisation to rownorm + c [BH][2 dh + 128]
+  float* wsave;
+  float* rownorm;
 };
 struct KeyGradMaps {
   CUtensorMap k, v, q;
@@ -186,13 +191,20 @@ TTT_DEVICE_INLINE float4 row_step(const KeyGradArgs& a, const KeyGradLoopArgs& l
   ss += w.x * w.x + w.y * w.y + w.z * w.z + w.w * w.w;
   return w;
 }
-TTT_DEVICE_INLINE float row_scale(const KeyGradArgs& a, const KeyGradLoopArgs& la, float ss) {
-  return la.normalize ? 1.f / fmaxf(sqrtf(kg_warp_sum(ss)), la.norm_eps) : 1.f;
+// the scale of an updated row (1 without the row norm); with `norm`, the
+// row's norm before the normalisation is recorded by lane 0
+TTT_DEVICE_INLINE float row_scale(const KeyGradArgs& a, const KeyGradLoopArgs& la, float ss, float* norm) {
+  if (!la.normalize) return 1.f;
+  const float n = sqrtf(kg_warp_sum(ss));
+  if (norm != nullptr && (threadIdx.x & 31) == 0) *norm = n;
+  return 1.f / fmaxf(n, la.norm_eps);
 }
-TTT_DEVICE_INLINE void row_store(const KeyGradArgs& a, const KeyGradLoopArgs& la, int m, int nb, size_t c, float4 w, float scale) {
+TTT_DEVICE_INLINE void row_store(const KeyGradArgs& a, const KeyGradLoopArgs& la, int m, int nb, size_t c, float4 w, float scale,
+                                 float* snap) {
   const float4 x = make_float4(w.x * scale, w.y * scale, w.z * scale, w.w * scale);
   *reinterpret_cast<float4*>(la.W[m] + c) = x;
   *reinterpret_cast<uint2*>(la.Wb[nb][m] + c) = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+  if (snap != nullptr) *reinterpret_cast<float4*>(snap + c) = x;
 }
 TTT_DEVICE_INLINE void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -259,8 +271,21 @@ TTT_DEVICE_INLINE void loop_cast_rows(const KeyGradArgs& a, const KeyGradLoopArg
       }
   }
 }
+template <bool SNAP>
 TTT_DEVICE_INLINE void loop_row_update(const KeyGradArgs& a, const KeyGradLoopArgs& la, int bh, const OwnRows& o, int e, int lane,
-                                       int nb, const uint8_t* sp0) {
+                                       int nb, const uint8_t* sp0, int c) {
+  // SNAP (the backward's replay): the chunk's updated weights and row norms
+  // are also kept; the forward's build of the kernel carries none of it
+  const size_t mat_elems = (size_t)a.BH * a.dh * kg::D;
+  auto snap = [&](int m) -> float* {
+    if constexpr (SNAP)
+      return la.wsave != nullptr ? la.wsave + (size_t)(c + 1) * 3 * mat_elems + (size_t)m * mat_elems : nullptr;
+    return nullptr;
+  };
+  // row norms of chunk c: [BH][W1 rows | W3 rows | W2 rows]
+  float* rn = nullptr;
+  if constexpr (SNAP)
+    if (la.rownorm != nullptr) rn = la.rownorm + ((size_t)c * a.BH + bh) * (2 * a.dh + kg::D);
   const uint32_t gb = own_group_bytes(a, la, o);
   auto psum = [&](uint32_t byte_off) {   // byte offset within one group's block
     float4 u = *reinterpret_cast<const float4*>(sp0 + byte_off);
@@ -279,7 +304,7 @@ TTT_DEVICE_INLINE void loop_row_update(const KeyGradArgs& a, const KeyGradLoopAr
       const float4 u = psum(base + (uint32_t)(i * kg::D + 4 * lane) * 4u);
       float ss = 0.f;
       const float4 x = row_step(a, la, m, c, u, w, ss);
-      row_store(a, la, m, nb, c, x, row_scale(a, la, ss));
+      row_store(a, la, m, nb, c, x, row_scale(a, la, ss, rn ? rn + m * a.dh + o.lo13 + i : nullptr), snap(m));
     }
     base += (uint32_t)o.n13 * kg::D * 4u;
   }
@@ -295,9 +320,9 @@ TTT_DEVICE_INLINE void loop_row_update(const KeyGradArgs& a, const KeyGradLoopAr
       float ss = 0.f;
       w0 = row_step(a, la, 2, c0, u0, w0, ss);
       if (two) w1 = row_step(a, la, 2, c1, u1, w1, ss);
-      const float sc = row_scale(a, la, ss);
-      row_store(a, la, 2, nb, c0, w0, sc);
-      if (two) row_store(a, la, 2, nb, c1, w1, sc);
+      const float sc = row_scale(a, la, ss, rn ? rn + 2 * a.dh + o.lo2 + i : nullptr);
+      row_store(a, la, 2, nb, c0, w0, sc, snap(2));
+      if (two) row_store(a, la, 2, nb, c1, w1, sc, snap(2));
     }
   }
 }
@@ -314,7 +339,7 @@ TTT_DEVICE_INLINE void loop_row_update(const KeyGradArgs& a, const KeyGradLoopAr
 // and count themselves done on the readers' counter; a worker starts chunk
 // c once the readers are done with chunk c - 2, whose Aq and W2 buffers
 // chunk c reuses.
-template <bool LOOP>
+template <bool LOOP, bool SNAP = false>
 __global__ void __launch_bounds__(kg::THREADS, 1)
     lact_keygrad_kernel(const __grid_constant__ KeyGradMaps maps, const KeyGradArgs a,
                         const __grid_constant__ KeyGradLoopArgs la) {
@@ -937,7 +962,7 @@ __global__ void __launch_bounds__(kg::THREADS, 1)
         named_bar_sync(1, EPI_WARPS * 32);
         if (W.aborted()) break;
         if (!W.wait(upd_full, c & 1, 14)) break;
-        loop_row_update(a, la, bh, own, warp - 2, lane, (c + 1) % 3, smem + OFF_W13);
+        loop_row_update<SNAP>(a, la, bh, own, warp - 2, lane, (c + 1) % 3, smem + OFF_W13, c);
         // the next chunk's weights: read by TMA in the head's workers
         fence_proxy_async_global();
         named_bar_sync(1, EPI_WARPS * 32);
@@ -1062,6 +1087,8 @@ int lact_loop_plan(int BH, int N_in, int C, int dh, int max_groups, int* groups,
   }
   static std::atomic<uint64_t> attr{0};
   if (allow_dynamic_smem(lact_keygrad_kernel<true>, (int)kg::SMEM, attr)) return -1;
+  static std::atomic<uint64_t> attr_snap{0};
+  if (allow_dynamic_smem(lact_keygrad_kernel<true, true>, (int)kg::SMEM, attr_snap)) return -1;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lact_keygrad_kernel<true>, kg::THREADS,
                                                     kg::SMEM) != cudaSuccess ||
@@ -1076,8 +1103,11 @@ int lact_loop_plan(int BH, int N_in, int C, int dh, int max_groups, int* groups,
 int launch_lact_loop(const KeyGradLoopLaunch& L, cudaStream_t stream) {
   // the caller's plan (lact_loop_plan), else this call's
   int g = L.groups, nw = L.workers, nr = L.readers;
-  if ((g <= 0 || nw <= 0 || nr <= 0) && lact_loop_plan(L.BH, L.N_in, L.C, L.dh, L.max_groups, &g, &nw, &nr))
+  const bool reads = L.q != nullptr;   // without queries there is nothing to read out
+  if ((g <= 0 || nw <= 0 || (reads && nr <= 0)) &&
+      lact_loop_plan(L.BH, L.N_in, L.C, L.dh, L.max_groups, &g, &nw, &nr))
     return -1;
+  if (!reads) nr = 0;
   KeyGradMaps m{};
   if (keygrad_maps(m, L.BH, L.N_in, L.dh, L.k, L.v, L.q)) return -1;
   const uint64_t BH = (uint64_t)L.BH;
@@ -1104,7 +1134,7 @@ int launch_lact_loop(const KeyGradLoopLaunch& L, cudaStream_t stream) {
     la.M[i] = L.M[i];
     for (int b = 0; b < 3; ++b) la.Wb[b][i] = L.Wb[b][i];
   }
-  a.queries = 1;
+  a.queries = reads ? 1 : 0;
   a.Aq = L.Aq;
   a.aq_bs = (long long)L.cmax * L.dh;
   la.aq_buf = L.aq_buf;
@@ -1117,6 +1147,8 @@ int launch_lact_loop(const KeyGradLoopLaunch& L, cudaStream_t stream) {
   la.beta = L.beta; la.norm_eps = L.norm_eps;
   la.out = L.out; la.out_bf16 = L.out_bf16; la.out_bs = (long long)L.N_in * kg::D;
   la.cast_first = L.cast_first;
+  la.wsave = L.wsave;
+  la.rownorm = L.rownorm;
   if (cudaMemsetAsync(L.ctr, 0, (3 * (size_t)L.BH + 2) * sizeof(unsigned), stream) != cudaSuccess) return -1;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(nw + nr);
@@ -1129,7 +1161,9 @@ int launch_lact_loop(const KeyGradLoopLaunch& L, cudaStream_t stream) {
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
   prof_before(K_LOOP, stream);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, lact_keygrad_kernel<true>, m, a, la);
+  const bool snap = L.wsave != nullptr || L.rownorm != nullptr;
+  const cudaError_t e = snap ? cudaLaunchKernelEx(&cfg, lact_keygrad_kernel<true, true>, m, a, la)
+                             : cudaLaunchKernelEx(&cfg, lact_keygrad_kernel<true>, m, a, la);
   prof_after(K_LOOP, stream);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
