@@ -72,6 +72,10 @@ struct RowStepArgs {
   __nv_bfloat16* Rb;     // out: bf16 copy
   const float* Wc;       // W_c (the chunk's start weights), cast to Wb alongside
   __nv_bfloat16* Wb;
+  // nullable: the later chunk's split weight-gradient partials, added to dW
+  // first ([BH][splits][rows][cols] per matrix, in split order)
+  const float* part[3];
+  int splits;
 };
 // One warp per row of one matrix of one head (rows of 128 to 1024 columns,
 // a multiple of 128): each lane holds four-column slices of the row in
@@ -101,16 +105,32 @@ __global__ void bwd_row_step_kernel(RowStepArgs a) {
   }
   float4* R4 = reinterpret_cast<float4*>(a.R + off);
   uint2* Rb2 = reinterpret_cast<uint2*>(a.Rb + off);
+  float4* dW4 = reinterpret_cast<float4*>(a.dW + off);
+  // dW of this chunk's end weights: the later chunk's partial products
+  // still to be added (in split order, as a separate summing pass would)
+  const float4* P4 = a.part[mat] != nullptr
+                         ? reinterpret_cast<const float4*>(a.part[mat] + ((size_t)bh * a.splits * rows + row) * cols)
+                         : nullptr;
+  const size_t pstride4 = (size_t)rows * cols / 4;
+  auto dw_in = [&](int k) {
+    float4 u = dW4[k * 32 + lane];
+    if (P4 != nullptr)
+      for (int sp = 0; sp < a.splits; ++sp) {
+        const float4 x = P4[sp * pstride4 + k * 32 + lane];
+        u.x += x.x; u.y += x.y; u.z += x.z; u.w += x.w;
+      }
+    return u;
+  };
   if (!(a.mask & (1 << mat))) {   // not updated: no dependence on G, dW passes through
 #pragma unroll
     for (int k = 0; k < 8; ++k)
       if (k < nv) {
+        if (P4 != nullptr) dW4[k * 32 + lane] = dw_in(k);
         R4[k * 32 + lane] = make_float4(0.f, 0.f, 0.f, 0.f);
         Rb2[k * 32 + lane] = make_uint2(0u, 0u);
       }
     return;
   }
-  float4* dW4 = reinterpret_cast<float4*>(a.dW + off);
   const float4* Wn4 = reinterpret_cast<const float4*>(a.Wn + off);
   float4 du[8], wn[8];
   float proj = 0.f, inv = 1.f;
@@ -118,7 +138,7 @@ __global__ void bwd_row_step_kernel(RowStepArgs a) {
 #pragma unroll
   for (int k = 0; k < 8; ++k)
     if (k < nv) {
-      du[k] = dW4[k * 32 + lane];
+      du[k] = dw_in(k);
       if (a.normalize) {
         wn[k] = Wn4[k * 32 + lane];
         proj += wn[k].x * du[k].x + wn[k].y * du[k].y + wn[k].z * du[k].z + wn[k].w * du[k].w;
@@ -905,6 +925,7 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
   // d x dh per head, so S splits fit the region while S d <= cmax.
   static std::atomic<uint64_t> group_attr{0};
   if (fused_fwd && allow_dynamic_smem(gemm_group_kernel, (int)gg::SMEM, group_attr)) return -1;
+  int pending_splits = 0;   // partials of the last grouped launch not yet in dW
   auto chunk_products = [&](int t0, int C, bool with_read) -> int {
     const int ks = (C + 63) / 64;
     const int S = std::max(1, std::min(std::min(8, ks), w.cmax / d)), kps = (ks + S - 1) / S;
@@ -965,10 +986,10 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
                                      dim3(gg::THREADS), gg::SMEM, stream, m, g);
     prof_after(K_BWD_GROUP, stream);
     if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return -1;
-    WgradSumArgs sa{BH, S, wsz, {f32[3], f32[4], f32[5]}, {dW1, dW3, dW2}};
-    const long long n4 = 3LL * BH * d * dh / 4;
-    bwd_wgrad_sum_kernel<<<(unsigned)std::min<long long>((n4 + 255) / 256, 4096), 256, 0, stream>>>(sa);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    // the splits are added to dW by the next chunk's row step (or the final
+    // sum after the last chunk)
+    pending_splits = S;
+    return 0;
   };
 
   // ---------------------------------------------------------------- 2. reverse
@@ -994,6 +1015,9 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
     rs.Wn = wsave + (size_t)(c + 1) * 3 * mat;
     rs.rn = rn + (size_t)c * BH * (2 * dh + d);
     rs.Wc = wsave + (size_t)c * 3 * mat;   // its bf16 copy is the chunk's product operand
+    for (int m = 0; m < 3; ++m) rs.part[m] = pending_splits > 0 ? f32[3 + m] : nullptr;
+    rs.splits = pending_splits;
+    pending_splits = 0;
     bwd_row_step_kernel<<<(row_warps * 32 + 255) / 256, 256, 0, stream>>>(rs);
     BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     // a causal chunk on the fused path: the read's elementwise step too, so
@@ -1046,6 +1070,12 @@ int launch_lact_bwd(const LactBwdLaunch& L, cudaStream_t stream) {
       BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
     }
     if (!both && f.causal) BWD_TRY(read_vjp(t0, C));
+  }
+  if (pending_splits > 0) {   // the first chunk's partial products
+    WgradSumArgs sa{BH, pending_splits, (long long)d * dh, {f32[3], f32[4], f32[5]}, {dW1, dW3, dW2}};
+    const long long n4 = 3LL * BH * d * dh / 4;
+    bwd_wgrad_sum_kernel<<<(unsigned)std::min<long long>((n4 + 255) / 256, 4096), 256, 0, stream>>>(sa);
+    BWD_TRY(cudaGetLastError() == cudaSuccess ? 0 : -1);
   }
   return cudaMemcpyAsync(L.dW0, dW, 3 * mat * 4, cudaMemcpyDeviceToDevice, stream) == cudaSuccess
              ? 0 : -1;
