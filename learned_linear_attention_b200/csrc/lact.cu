@@ -18,6 +18,8 @@
 // queries run step 1 (queries only) and step 2 with the final weights.
 #include <algorithm>
 #include <cstdlib>
+#include <functional>
+#include <vector>
 
 #include "gemm.cuh"
 #include "kernels.h"
@@ -829,6 +831,45 @@ static int grad_splits(int BH, int d, int dh, int cmax) {
   return s;
 }
 
+// Tile widths of the split-K gradient products: [G1; G3] (N = d) and G2 (N = dh).
+static int grad_bn13(int d) { return d % 192 == 0 ? 192 : 128; }
+static int grad_bn2(int dh) { return dh % 256 == 0 ? 256 : 128; }
+
+// Split count of the unfused path's three gradient products.  They run side
+// by side on three streams, one CTA per SM, G2 launched first (its tiles are
+// the wider ones where dh > d).  The count taken is the one whose greedy
+// schedule of those CTAs, in launch order on the SMs, ends first (a CTA's time
+// taken as its tile width times its k-steps plus a few for the prologue and
+// the epilogue); at most UPB_MAX_SPLITS, so the slab update still sums the
+// partials, and at least eight k-steps per split.
+static int grad_splits_sched(int BH, int d, int dh, int cmax) {
+  const int ksteps = (cmax + 63) / 64;
+  const int bn13 = grad_bn13(d), bn2 = grad_bn2(dh);
+  const long long t13 = (long long)BH * ((dh + 127) / 128) * (d / bn13);
+  const long long t2 = (long long)BH * ((d + 127) / 128) * (dh / bn2);
+  const int sms = num_sms();
+  const int smax = std::max(1, std::min(UPB_MAX_SPLITS, ksteps / 8));
+  int best = 1;
+  double best_t = 0.0;
+  std::vector<double> free_at;
+  for (int s = 1; s <= smax; ++s) {
+    const int kps = (ksteps + s - 1) / s;
+    free_at.assign(sms, 0.0);   // min-heap of the times the SMs come free
+    auto place = [&](long long n, int bn) {
+      for (long long i = 0; i < n; ++i) {
+        std::pop_heap(free_at.begin(), free_at.end(), std::greater<double>());
+        free_at.back() += (double)bn * (kps + 4);
+        std::push_heap(free_at.begin(), free_at.end(), std::greater<double>());
+      }
+    };
+    place(t2 * s, bn2);
+    place(2 * t13 * s, bn13);
+    const double t = *std::max_element(free_at.begin(), free_at.end());
+    if (s == 1 || t < best_t) { best = s; best_t = t; }
+  }
+  return best;
+}
+
 // head dim 128 (dh a multiple of 64), no split operands, GD or momentum: the
 // key pass and the chunk gradient run as one fused kernel (lact_keygrad.cu)
 // The chunk-loop launch is on unless TTT_LACT_CHUNK_LOOP=0 (read once).
@@ -893,9 +934,9 @@ LactWorkspace lact_workspace_layout(int B, int H, int N_in, int N_q, int d, int 
     w.total = o;
     return w;
   }
-  w.splits = grad_splits((int)BH, d, dh, cin);
   w.keygrad = lact_uses_keygrad(d, dh, opt, split) ? 1 : 0;
-  if (w.keygrad) w.splits = std::max(w.splits, keygrad_groups((int)BH, dh, cin, 0));
+  w.splits = w.keygrad ? std::max(grad_splits((int)BH, d, dh, cin), keygrad_groups((int)BH, dh, cin, 0))
+                       : grad_splits_sched((int)BH, d, dh, cin);
   // bf16 operand copies: chunk c reads buffer c mod nbuf while its update
   // writes the next one.  On the fused causal path the read of chunk c runs
   // beside the next chunk, so a third buffer (and a second Aq) keeps what it
@@ -1328,7 +1369,7 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     const int kps = (ksteps_total + splits - 1) / splits;
     // the same operands through blocked views: one copy per operand per stage
     // (A blocks of 128 rows, B blocks of the tile width)
-    const int bn13 = d % 192 == 0 ? 192 : 128, bn2 = dh % 256 == 0 ? 256 : 128;
+    const int bn13 = grad_bn13(d), bn2 = grad_bn2(dh);
     CUtensorMap bd13[2], bk13, bv, bg[2];
     TTT_TRY(make_tmap_bf16_blocked(&bd13[0], D13, 2 * dh, C, BH, (uint64_t)dh * 4,
                                    (uint64_t)w.cmax * dh * 4, 64, 2));
@@ -1346,7 +1387,10 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     g.batch = BH; g.splits = splits; g.k_steps = kps; g.npairs = np;
     g.o32_ss = (long long)BH * d * dh;
     g.o32_bs = (long long)d * dh;
-    for (int mat = 0; mat < 3; ++mat) {
+    // G2 first (grad_splits_sched models this order): where dh > d its CTAs
+    // are the longest, and the shorter ones fill in behind them
+    for (int mi = 0; mi < 3; ++mi) {
+      const int mat = (mi + 2) % 3;
       GemmMaps m{};
       if (mat < 2) {
         g.M = dh; g.N = d; g.ld32 = d;
