@@ -37,7 +37,9 @@ constexpr uint32_t W13_BYTES = 2 * HB * 64 * 2;      // 16 KB (W1 rows | W3 rows
 constexpr uint32_t W2_BYTES = 64 * HB * 2;           // 8 KB  (W2 block, MN-major)
 constexpr uint32_t STAGE = X_BYTES + V_BYTES + W13_BYTES + W2_BYTES;
 constexpr int STAGES = 3;
-constexpr uint32_t BAR_OFF = STAGES * STAGE;
+constexpr uint32_t STG_OUT = BM * HB * 2;            // 16 KB: one output tile, 128-byte swizzle
+constexpr uint32_t STG_OFF = STAGES * STAGE;         // [dH1 | dH3 | Gm'] or [Aq] staging
+constexpr uint32_t BAR_OFF = STG_OFF + 3 * STG_OUT;
 constexpr uint32_t SMEM = BAR_OFF + 256 + 1024;
 constexpr uint32_t ACC_COLS = 256;                   // [H1 64 | H3 64 | dG 64 | pad]
 constexpr int EPI_WARPS = 8;                         // two per TMEM lane quadrant
@@ -69,7 +71,16 @@ struct KeyPassArgs {
 
 struct KeyPassMaps {
   CUtensorMap k, v, q, w1, w3, w2, w1lo, w3lo, w2lo;
+  // tensor-store views of the intermediates (box 64 hidden x 128 rows,
+  // 128-byte swizzle): D13 {2 dh, cmax, BH}, Gm' and Aq {dh, cmax, BH}
+  CUtensorMap od13, ogm, oaq;
 };
+
+// Byte offset of 16-byte chunk c (0..7) of row r in a tile of 128-byte rows
+// laid out with the 128-byte swizzle (chunk index XOR row mod 8).
+TTT_DEVICE_INLINE uint32_t sw128_offset(int r, int c) {
+  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
 
 // bf16 residual of x given its bf16 rounding h: the "lo" part of x = hi + lo.
 TTT_DEVICE_INLINE __nv_bfloat16 bf16_residual(float x, __nv_bfloat16 h) {
@@ -227,22 +238,34 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
     }
   } else {
     // epilogue: warps 2..9; quadrant q4 = TMEM lanes, column group cg = 32
-    // of the tile's 64 hidden units, processed as two 16-column halves
+    // of the tile's 64 hidden units, processed as two 16-column halves.
+    // Without split operands every output tile is staged in shared memory
+    // (128-byte swizzle) and leaves by one tensor store, issued by lane 0 of
+    // epilogue warp ew for output ew, so the rows go out as whole 128-byte
+    // lines; rows past the pass are staged as zeros (the intermediates hold
+    // cmax rows and their readers stop at the pass length).  Split operands
+    // (six outputs) store each row's 32 bytes directly.
     const int q4 = warp & 3;
     const int cg = (warp - 2) >> 2;
+    const int ew = warp - 2;
     const int r = q4 * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const bool staged = !a.split;
+    const uint32_t stg = smem_u32(smem + STG_OFF);
     uint32_t lt = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
       int bh, tt, hb;
       decode(t, bh, tt, hb);
       const bool is_key = tt < a.n_key_tiles;
-      const int tc = (is_key ? tt : tt - a.n_key_tiles) * BM + r;   // row within the pass
+      const bool full_key = is_key && !a.feat_only;
+      const int nout = full_key ? 3 : 1;
+      const int prow = (is_key ? tt : tt - a.n_key_tiles) * BM;   // first row within the pass
+      const int tc = prow + r;
       const bool valid = tc < a.C;
       const uint32_t ab = lt & 1;
       // the learning rate is fetched before waiting for the accumulator
       const float eta = (is_key && valid) ? a.lr[(size_t)bh * a.lr_len + a.t0 + tc] : 0.f;
-      if (!W.wait(&afull[ab], (lt >> 1) & 1, 4)) break;
+      if (!named_bar_all(1, EPI_WARPS * 32, W.wait(&afull[ab], (lt >> 1) & 1, 4))) break;
       tc_fence_after();
       const uint32_t base = tmem + lane_base + ab * ACC_COLS;
       const size_t obase = (size_t)bh * a.inter_bs + (size_t)tc * a.dh + hb * HB;
@@ -253,71 +276,70 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
         uint32_t rh1[16], rh3[16], rg[16];
         tmem_ld16_issue(base + jc, rh1);
         tmem_ld16_issue(base + 64 + jc, rh3);
-        if (is_key && !a.feat_only) tmem_ld16_issue(base + 128 + jc, rg);
+        if (full_key) tmem_ld16_issue(base + 128 + jc, rg);
         tmem_wait_ld();
+        if (half == 1) {   // this thread's last read of the accumulators
+          tc_fence_before();
+          mbar_arrive(&aempty[ab]);
+        }
         float h1[16], h3[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           h1[j] = __uint_as_float(rh1[j]);
           h3[j] = __uint_as_float(rh3[j]);
         }
+        uint32_t o[3][8];   // output q of this row's 16 columns, bf16 pairs
         if (is_key && a.feat_only) {
-          if (valid) {
-            uint32_t om[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float x0 = h1[2 * j], x1 = h1[2 * j + 1];
-              om[j] = pack_bf16x2(-eta * x0 * sigmoidf_tanh(x0) * h3[2 * j],
+          for (int j = 0; j < 8; ++j) {
+            const float x0 = h1[2 * j], x1 = h1[2 * j + 1];
+            o[0][j] = pack_bf16x2(-eta * x0 * sigmoidf_tanh(x0) * h3[2 * j],
                                   -eta * x1 * sigmoidf_tanh(x1) * h3[2 * j + 1]);
-            }
+          }
+          if (!staged && valid) {
             uint4* dm = reinterpret_cast<uint4*>(a.Gm + obase + jc);
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
-              dm[j] = make_uint4(om[4 * j], om[4 * j + 1], om[4 * j + 2], om[4 * j + 3]);
+            for (int j = 0; j < 2; ++j) dm[j] = make_uint4(o[0][4 * j], o[0][4 * j + 1], o[0][4 * j + 2], o[0][4 * j + 3]);
           }
         } else if (is_key) {
-          float g[16];
+          float r1[16], r3[16], rm[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) g[j] = __uint_as_float(rg[j]);
-          if (valid) {
-            uint32_t o1[8], o3[8], om[8];
-            float r1[16], r3[16], rm[16];
+          for (int j = 0; j < 16; ++j) {
+            const float x = h1[j], y = h3[j];
+            const float sg = a.split ? sigmoidf_fast(x) : sigmoidf_tanh(x);
+            const float act = x * sg;
+            const float dg = -eta * __uint_as_float(rg[j]);
+            r3[j] = dg * act;
+            r1[j] = dg * y * (sg * (1.f + x * (1.f - sg)));
+            rm[j] = -eta * act * y;
+          }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float x = h1[j], y = h3[j];
-              const float sg = a.split ? sigmoidf_fast(x) : sigmoidf_tanh(x);
-              const float act = x * sg;
-              const float dg = -eta * g[j];
-              r3[j] = dg * act;
-              r1[j] = dg * y * (sg * (1.f + x * (1.f - sg)));
-              rm[j] = -eta * act * y;
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              o1[j] = pack_bf16x2(r1[2 * j], r1[2 * j + 1]);
-              o3[j] = pack_bf16x2(r3[2 * j], r3[2 * j + 1]);
-              om[j] = pack_bf16x2(rm[2 * j], rm[2 * j + 1]);
-            }
+          for (int j = 0; j < 8; ++j) {
+            o[0][j] = pack_bf16x2(r1[2 * j], r1[2 * j + 1]);
+            o[1][j] = pack_bf16x2(r3[2 * j], r3[2 * j + 1]);
+            o[2][j] = pack_bf16x2(rm[2 * j], rm[2 * j + 1]);
+          }
+          if (!staged && valid) {
             uint4* dm = reinterpret_cast<uint4*>(a.Gm + obase + jc);
             if (a.D13 != nullptr) {   // dH1, dH3 (absent when only W2 is updated)
               uint4* d1 = reinterpret_cast<uint4*>(a.D13 + dbase + jc);
               uint4* d3 = reinterpret_cast<uint4*>(a.D13 + dbase + a.dh + jc);
 #pragma unroll
               for (int j = 0; j < 2; ++j) {
-                d1[j] = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
-                d3[j] = make_uint4(o3[4 * j], o3[4 * j + 1], o3[4 * j + 2], o3[4 * j + 3]);
+                d1[j] = make_uint4(o[0][4 * j], o[0][4 * j + 1], o[0][4 * j + 2], o[0][4 * j + 3]);
+                d3[j] = make_uint4(o[1][4 * j], o[1][4 * j + 1], o[1][4 * j + 2], o[1][4 * j + 3]);
               }
             }
 #pragma unroll
             for (int j = 0; j < 2; ++j)
-              dm[j] = make_uint4(om[4 * j], om[4 * j + 1], om[4 * j + 2], om[4 * j + 3]);
+              dm[j] = make_uint4(o[2][4 * j], o[2][4 * j + 1], o[2][4 * j + 2], o[2][4 * j + 3]);
             if (a.split) {
               uint32_t l1[8], l3[8], lm[8];
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                l1[j] = pack_bf16x2(r1[2 * j] - bf16lo(o1[j]), r1[2 * j + 1] - bf16hi(o1[j]));
-                l3[j] = pack_bf16x2(r3[2 * j] - bf16lo(o3[j]), r3[2 * j + 1] - bf16hi(o3[j]));
-                lm[j] = pack_bf16x2(rm[2 * j] - bf16lo(om[j]), rm[2 * j + 1] - bf16hi(om[j]));
+                l1[j] = pack_bf16x2(r1[2 * j] - bf16lo(o[0][j]), r1[2 * j + 1] - bf16hi(o[0][j]));
+                l3[j] = pack_bf16x2(r3[2 * j] - bf16lo(o[1][j]), r3[2 * j + 1] - bf16hi(o[1][j]));
+                lm[j] = pack_bf16x2(rm[2 * j] - bf16lo(o[2][j]), rm[2 * j + 1] - bf16hi(o[2][j]));
               }
               uint4* e1 = reinterpret_cast<uint4*>(a.D13lo + dbase + jc);
               uint4* e3 = reinterpret_cast<uint4*>(a.D13lo + dbase + a.dh + jc);
@@ -330,33 +352,63 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
               }
             }
           }
-        } else if (valid) {
+        } else {
           float aq[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             aq[j] = h1[j] * (a.split ? sigmoidf_fast(h1[j]) : sigmoidf_tanh(h1[j])) * h3[j];
-          uint32_t oq[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) oq[j] = pack_bf16x2(aq[2 * j], aq[2 * j + 1]);
-          uint4* dq = reinterpret_cast<uint4*>(a.Aq + obase + jc);
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-            dq[j] = make_uint4(oq[4 * j], oq[4 * j + 1], oq[4 * j + 2], oq[4 * j + 3]);
-          if (a.split) {
-            uint32_t lq[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              lq[j] = pack_bf16x2(aq[2 * j] - bf16lo(oq[j]), aq[2 * j + 1] - bf16hi(oq[j]));
-            uint4* eq = reinterpret_cast<uint4*>(a.Aqlo + obase + jc);
+          for (int j = 0; j < 8; ++j) o[0][j] = pack_bf16x2(aq[2 * j], aq[2 * j + 1]);
+          if (!staged && valid) {
+            uint4* dq = reinterpret_cast<uint4*>(a.Aq + obase + jc);
 #pragma unroll
             for (int j = 0; j < 2; ++j)
-              eq[j] = make_uint4(lq[4 * j], lq[4 * j + 1], lq[4 * j + 2], lq[4 * j + 3]);
+              dq[j] = make_uint4(o[0][4 * j], o[0][4 * j + 1], o[0][4 * j + 2], o[0][4 * j + 3]);
+            if (a.split) {
+              uint32_t lq[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                lq[j] = pack_bf16x2(aq[2 * j] - bf16lo(o[0][j]), aq[2 * j + 1] - bf16hi(o[0][j]));
+              uint4* eq = reinterpret_cast<uint4*>(a.Aqlo + obase + jc);
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                eq[j] = make_uint4(lq[4 * j], lq[4 * j + 1], lq[4 * j + 2], lq[4 * j + 3]);
+            }
+          }
+        }
+        if (staged) {
+          if (!valid) {
+#pragma unroll
+            for (int q = 0; q < 3; ++q)
+#pragma unroll
+              for (int j = 0; j < 8; ++j) o[q][j] = 0u;
+          }
+          if (half == 0) {   // the staging tiles are free once the previous tile's stores have read them
+            if (lane == 0 && ew < 3) bulk_wait_read();
+            named_bar_sync(1, EPI_WARPS * 32);
+          }
+#pragma unroll
+          for (int q = 0; q < 3; ++q) {
+            if (q < nout) {
+              st_shared_v4(stg + q * STG_OUT + sw128_offset(r, jc >> 3), o[q][0], o[q][1], o[q][2], o[q][3]);
+              st_shared_v4(stg + q * STG_OUT + sw128_offset(r, (jc >> 3) + 1), o[q][4], o[q][5], o[q][6],
+                           o[q][7]);
+            }
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&aempty[ab]);
+      if (staged) {
+        fence_async_smem();   // the tensor stores (async proxy) read what these threads wrote
+        named_bar_sync(1, EPI_WARPS * 32);
+        if (lane == 0 && ew < nout) {
+          const CUtensorMap* m = !is_key ? &maps.oaq : (full_key && ew < 2) ? &maps.od13 : &maps.ogm;
+          const int x = hb * HB + ((full_key && ew == 1) ? a.dh : 0);
+          tma_store_3d(m, smem + STG_OFF + ew * STG_OUT, x, prow, bh);
+          bulk_commit();
+        }
+      }
     }
+    if (lane == 0 && ew < 3) bulk_wait_all();   // every tensor store is complete before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -1226,6 +1278,17 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   if (uses_q) TTT_TRY(tok_map(&km.q, L.q, q_rows, 128));
   else km.q = km.k;
   if (!uses_kv) { km.k = km.q; km.v = km.q; }
+  // the key pass's tensor-store views (its staged epilogue: no split
+  // operands); a workspace laid out for the fused key-gradient kernel has no
+  // key-pass intermediates and gets none
+  const bool kp_staged = !split && !w.keygrad;
+  if (kp_staged) {
+    const uint64_t ibs = (uint64_t)w.cmax * dh * 2;   // bytes per head of Gm' / Aq
+    if (D13 != nullptr)
+      TTT_TRY(make_tmap_bf16_3d_sw(&km.od13, D13, 2 * dh, w.cmax, BH, (uint64_t)dh * 4, 2 * ibs, 64, 128, 128));
+    TTT_TRY(make_tmap_bf16_3d_sw(&km.ogm, Gm, dh, w.cmax, BH, (uint64_t)dh * 2, ibs, 64, 128, 128));
+    TTT_TRY(make_tmap_bf16_3d_sw(&km.oaq, Aq, dh, w.cmax, BH, (uint64_t)dh * 2, ibs, 64, 128, 128));
+  }
   KeyPassMaps kmb[3] = {km, km, km};
   CUtensorMap mw2k[3], mw2klo[3];
   for (int b = 0; b < nbuf; ++b) {
@@ -1255,8 +1318,8 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   if (allow_dynamic_smem(lact_keypass_kernel, (int)kp::SMEM, kp_attr)) return -1;
 
   auto key_pass_on = [&](int t0, int C, int nkt, int nqt, cudaStream_t kstream) -> int {
-    // never launch on a token map this call did not encode
-    if ((nkt > 0 && !uses_kv) || (nqt > 0 && !uses_q)) return -1;
+    // never launch on a token or store map this call did not encode
+    if ((nkt > 0 && !uses_kv) || (nqt > 0 && !uses_q) || (!split && !kp_staged)) return -1;
     KeyPassArgs a{};
     a.C = C; a.t0 = t0; a.n_key_tiles = nkt; a.n_q_tiles = nqt; a.n_hb = dh / 64; a.BH = BH;
     a.d_steps = d / 64; a.dh = dh; a.lr_len = L.N_in; a.lr = L.lr;
