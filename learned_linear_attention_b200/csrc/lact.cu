@@ -38,6 +38,7 @@ constexpr uint32_t W2_BYTES = 64 * HB * 2;           // 8 KB  (W2 block, MN-majo
 constexpr uint32_t STAGE = X_BYTES + V_BYTES + W13_BYTES + W2_BYTES;
 constexpr int STAGES = 3;
 constexpr uint32_t STG_OUT = BM * HB * 2;            // 16 KB: one output tile, 128-byte swizzle
+constexpr uint32_t STG_HALF = BM * 32 * 2;           // 8 KB: half an output tile (split operands)
 constexpr uint32_t STG_OFF = STAGES * STAGE;         // [dH1 | dH3 | Gm'] or [Aq] staging
 constexpr uint32_t BAR_OFF = STG_OFF + 3 * STG_OUT;
 constexpr uint32_t SMEM = BAR_OFF + 256 + 1024;
@@ -71,15 +72,21 @@ struct KeyPassArgs {
 
 struct KeyPassMaps {
   CUtensorMap k, v, q, w1, w3, w2, w1lo, w3lo, w2lo;
-  // tensor-store views of the intermediates (box 64 hidden x 128 rows,
-  // 128-byte swizzle): D13 {2 dh, cmax, BH}, Gm' and Aq {dh, cmax, BH}
+  // tensor-store views of the intermediates: D13 {2 dh, cmax, BH}, Gm' and
+  // Aq {dh, cmax, BH}.  Box 64 hidden x 128 rows, 128-byte swizzle; with split
+  // operands [hi, lo] pairs with box 32 x 128, 64-byte swizzle.
   CUtensorMap od13, ogm, oaq;
+  CUtensorMap sd13[2], sgm[2], saq[2];
 };
 
 // Byte offset of 16-byte chunk c (0..7) of row r in a tile of 128-byte rows
 // laid out with the 128-byte swizzle (chunk index XOR row mod 8).
 TTT_DEVICE_INLINE uint32_t sw128_offset(int r, int c) {
   return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+// The same for 64-byte rows and the 64-byte swizzle (chunk c = 0..3).
+TTT_DEVICE_INLINE uint32_t kp_sw64_offset(int r, int c) {
+  return (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
 }
 
 // bf16 residual of x given its bf16 rounding h: the "lo" part of x = hi + lo.
@@ -97,6 +104,9 @@ TTT_DEVICE_INLINE float sigmoidf_tanh(float x) {
   return fmaf(0.5f, t, 0.5f);
 }
 
+// SP: split operands (a.split != 0); one instance per mode, so each keeps
+// only its own epilogue's registers
+template <bool SP>
 __global__ void __launch_bounds__(kp::THREADS, 1)
     lact_keypass_kernel(const __grid_constant__ KeyPassMaps maps, const KeyPassArgs a) {
   using namespace kp;
@@ -237,20 +247,24 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
       W.drain(fin, 0);
     }
   } else {
-    // epilogue: warps 2..9; quadrant q4 = TMEM lanes, column group cg = 32
-    // of the tile's 64 hidden units, processed as two 16-column halves.
-    // Without split operands every output tile is staged in shared memory
-    // (128-byte swizzle) and leaves by one tensor store, issued by lane 0 of
-    // epilogue warp ew for output ew, so the rows go out as whole 128-byte
-    // lines; rows past the pass are staged as zeros (the intermediates hold
-    // cmax rows and their readers stop at the pass length).  Split operands
-    // (six outputs) store each row's 32 bytes directly.
+    // epilogue: warps 2..9; quadrant q4 = TMEM lanes, column group cg, two
+    // halves of 16 columns per thread.  Every output tile is staged in shared
+    // memory and leaves by tensor stores, issued by lane 0 of epilogue warp ew
+    // for staged output ew, so the rows go out as whole lines; rows past the
+    // pass are staged as zeros (the intermediates hold cmax rows and their
+    // readers stop at the pass length).
+    //  - bf16 operands: cg takes 32 of the 64 hidden units, the halves 16 each;
+    //    each output (dH1, dH3, Gm' or Aq) is one 128 x 64 tile with the
+    //    128-byte swizzle, stored once per tile;
+    //  - split operands: half h is hidden units [32h, 32h + 32), cg 16 of
+    //    them; the hi and lo parts of each output are 128 x 32 tiles with the
+    //    64-byte swizzle, stored once per half.
     const int q4 = warp & 3;
     const int cg = (warp - 2) >> 2;
     const int ew = warp - 2;
     const int r = q4 * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const bool staged = !a.split;
+    constexpr bool sp = SP;
     const uint32_t stg = smem_u32(smem + STG_OFF);
     uint32_t lt = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
@@ -259,6 +273,9 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
       const bool is_key = tt < a.n_key_tiles;
       const bool full_key = is_key && !a.feat_only;
       const int nout = full_key ? 3 : 1;
+      // staged outputs: the hi parts, then (split operands) the lo parts;
+      // only W2 updated (no split operands) writes Gm' alone
+      const int nst = sp && (full_key || !is_key) ? 2 * nout : nout;
       const int prow = (is_key ? tt : tt - a.n_key_tiles) * BM;   // first row within the pass
       const int tc = prow + r;
       const bool valid = tc < a.C;
@@ -268,11 +285,9 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
       if (!named_bar_all(1, EPI_WARPS * 32, W.wait(&afull[ab], (lt >> 1) & 1, 4))) break;
       tc_fence_after();
       const uint32_t base = tmem + lane_base + ab * ACC_COLS;
-      const size_t obase = (size_t)bh * a.inter_bs + (size_t)tc * a.dh + hb * HB;
-      const size_t dbase = 2 * ((size_t)bh * a.inter_bs + (size_t)tc * a.dh) + hb * HB;
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
-        const int jc = cg * 32 + half * 16;
+        const int jc = sp ? half * 32 + cg * 16 : cg * 32 + half * 16;
         uint32_t rh1[16], rh3[16], rg[16];
         tmem_ld16_issue(base + jc, rh1);
         tmem_ld16_issue(base + 64 + jc, rh3);
@@ -288,7 +303,8 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
           h1[j] = __uint_as_float(rh1[j]);
           h3[j] = __uint_as_float(rh3[j]);
         }
-        uint32_t o[3][8];   // output q of this row's 16 columns, bf16 pairs
+        uint32_t o[3][8];   // hi part of output q for this row's 16 columns, bf16 pairs
+        uint32_t l[3][8];   // lo part (split operands)
         if (is_key && a.feat_only) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -296,17 +312,12 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
             o[0][j] = pack_bf16x2(-eta * x0 * sigmoidf_tanh(x0) * h3[2 * j],
                                   -eta * x1 * sigmoidf_tanh(x1) * h3[2 * j + 1]);
           }
-          if (!staged && valid) {
-            uint4* dm = reinterpret_cast<uint4*>(a.Gm + obase + jc);
-#pragma unroll
-            for (int j = 0; j < 2; ++j) dm[j] = make_uint4(o[0][4 * j], o[0][4 * j + 1], o[0][4 * j + 2], o[0][4 * j + 3]);
-          }
         } else if (is_key) {
           float r1[16], r3[16], rm[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const float x = h1[j], y = h3[j];
-            const float sg = a.split ? sigmoidf_fast(x) : sigmoidf_tanh(x);
+            const float sg = sp ? sigmoidf_fast(x) : sigmoidf_tanh(x);
             const float act = x * sg;
             const float dg = -eta * __uint_as_float(rg[j]);
             r3[j] = dg * act;
@@ -319,70 +330,34 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
             o[1][j] = pack_bf16x2(r3[2 * j], r3[2 * j + 1]);
             o[2][j] = pack_bf16x2(rm[2 * j], rm[2 * j + 1]);
           }
-          if (!staged && valid) {
-            uint4* dm = reinterpret_cast<uint4*>(a.Gm + obase + jc);
-            if (a.D13 != nullptr) {   // dH1, dH3 (absent when only W2 is updated)
-              uint4* d1 = reinterpret_cast<uint4*>(a.D13 + dbase + jc);
-              uint4* d3 = reinterpret_cast<uint4*>(a.D13 + dbase + a.dh + jc);
+          if (sp) {
 #pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                d1[j] = make_uint4(o[0][4 * j], o[0][4 * j + 1], o[0][4 * j + 2], o[0][4 * j + 3]);
-                d3[j] = make_uint4(o[1][4 * j], o[1][4 * j + 1], o[1][4 * j + 2], o[1][4 * j + 3]);
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-              dm[j] = make_uint4(o[2][4 * j], o[2][4 * j + 1], o[2][4 * j + 2], o[2][4 * j + 3]);
-            if (a.split) {
-              uint32_t l1[8], l3[8], lm[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                l1[j] = pack_bf16x2(r1[2 * j] - bf16lo(o[0][j]), r1[2 * j + 1] - bf16hi(o[0][j]));
-                l3[j] = pack_bf16x2(r3[2 * j] - bf16lo(o[1][j]), r3[2 * j + 1] - bf16hi(o[1][j]));
-                lm[j] = pack_bf16x2(rm[2 * j] - bf16lo(o[2][j]), rm[2 * j + 1] - bf16hi(o[2][j]));
-              }
-              uint4* e1 = reinterpret_cast<uint4*>(a.D13lo + dbase + jc);
-              uint4* e3 = reinterpret_cast<uint4*>(a.D13lo + dbase + a.dh + jc);
-              uint4* em = reinterpret_cast<uint4*>(a.Gmlo + obase + jc);
-#pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                e1[j] = make_uint4(l1[4 * j], l1[4 * j + 1], l1[4 * j + 2], l1[4 * j + 3]);
-                e3[j] = make_uint4(l3[4 * j], l3[4 * j + 1], l3[4 * j + 2], l3[4 * j + 3]);
-                em[j] = make_uint4(lm[4 * j], lm[4 * j + 1], lm[4 * j + 2], lm[4 * j + 3]);
-              }
+            for (int j = 0; j < 8; ++j) {
+              l[0][j] = pack_bf16x2(r1[2 * j] - bf16lo(o[0][j]), r1[2 * j + 1] - bf16hi(o[0][j]));
+              l[1][j] = pack_bf16x2(r3[2 * j] - bf16lo(o[1][j]), r3[2 * j + 1] - bf16hi(o[1][j]));
+              l[2][j] = pack_bf16x2(rm[2 * j] - bf16lo(o[2][j]), rm[2 * j + 1] - bf16hi(o[2][j]));
             }
           }
         } else {
           float aq[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            aq[j] = h1[j] * (a.split ? sigmoidf_fast(h1[j]) : sigmoidf_tanh(h1[j])) * h3[j];
+            aq[j] = h1[j] * (sp ? sigmoidf_fast(h1[j]) : sigmoidf_tanh(h1[j])) * h3[j];
 #pragma unroll
           for (int j = 0; j < 8; ++j) o[0][j] = pack_bf16x2(aq[2 * j], aq[2 * j + 1]);
-          if (!staged && valid) {
-            uint4* dq = reinterpret_cast<uint4*>(a.Aq + obase + jc);
+          if (sp) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
-              dq[j] = make_uint4(o[0][4 * j], o[0][4 * j + 1], o[0][4 * j + 2], o[0][4 * j + 3]);
-            if (a.split) {
-              uint32_t lq[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                lq[j] = pack_bf16x2(aq[2 * j] - bf16lo(o[0][j]), aq[2 * j + 1] - bf16hi(o[0][j]));
-              uint4* eq = reinterpret_cast<uint4*>(a.Aqlo + obase + jc);
-#pragma unroll
-              for (int j = 0; j < 2; ++j)
-                eq[j] = make_uint4(lq[4 * j], lq[4 * j + 1], lq[4 * j + 2], lq[4 * j + 3]);
-            }
+            for (int j = 0; j < 8; ++j)
+              l[0][j] = pack_bf16x2(aq[2 * j] - bf16lo(o[0][j]), aq[2 * j + 1] - bf16hi(o[0][j]));
           }
         }
-        if (staged) {
-          if (!valid) {
+        if (!valid) {
 #pragma unroll
-            for (int q = 0; q < 3; ++q)
+          for (int q = 0; q < 3; ++q)
 #pragma unroll
-              for (int j = 0; j < 8; ++j) o[q][j] = 0u;
-          }
+            for (int j = 0; j < 8; ++j) o[q][j] = l[q][j] = 0u;
+        }
+        if (!sp) {
           if (half == 0) {   // the staging tiles are free once the previous tile's stores have read them
             if (lane == 0 && ew < 3) bulk_wait_read();
             named_bar_sync(1, EPI_WARPS * 32);
@@ -395,9 +370,37 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
                            o[q][7]);
             }
           }
+        } else {
+          // the staging tiles are free once the previous half's stores have read them
+          if (lane == 0 && ew < 6) bulk_wait_read();
+          named_bar_sync(1, EPI_WARPS * 32);
+#pragma unroll
+          for (int q = 0; q < 3; ++q) {
+            if (q < nout) {
+              st_shared_v4(stg + q * STG_HALF + kp_sw64_offset(r, 2 * cg), o[q][0], o[q][1], o[q][2], o[q][3]);
+              st_shared_v4(stg + q * STG_HALF + kp_sw64_offset(r, 2 * cg + 1), o[q][4], o[q][5], o[q][6],
+                           o[q][7]);
+              if (nst > nout) {
+                const uint32_t sl = stg + (nout + q) * STG_HALF;
+                st_shared_v4(sl + kp_sw64_offset(r, 2 * cg), l[q][0], l[q][1], l[q][2], l[q][3]);
+                st_shared_v4(sl + kp_sw64_offset(r, 2 * cg + 1), l[q][4], l[q][5], l[q][6], l[q][7]);
+              }
+            }
+          }
+          fence_async_smem();   // the tensor stores (async proxy) read what these threads wrote
+          named_bar_sync(1, EPI_WARPS * 32);
+          if (lane == 0 && ew < nst) {
+            // staged output ew: kind 0 dH1, 1 dH3, 2 Gm', 3 Aq; part 0 hi, 1 lo
+            const int kind = full_key ? ew % 3 : is_key ? 2 : 3;
+            const int part = full_key ? ew / 3 : is_key ? 0 : ew;
+            const CUtensorMap* m = kind == 3 ? &maps.saq[part] : kind == 2 ? &maps.sgm[part] : &maps.sd13[part];
+            const int x = hb * HB + half * 32 + (kind == 1 ? a.dh : 0);
+            tma_store_3d(m, smem + STG_OFF + ew * STG_HALF, x, prow, bh);
+            bulk_commit();
+          }
         }
       }
-      if (staged) {
+      if (!sp) {
         fence_async_smem();   // the tensor stores (async proxy) read what these threads wrote
         named_bar_sync(1, EPI_WARPS * 32);
         if (lane == 0 && ew < nout) {
@@ -408,7 +411,7 @@ __global__ void __launch_bounds__(kp::THREADS, 1)
         }
       }
     }
-    if (lane == 0 && ew < 3) bulk_wait_all();   // every tensor store is complete before the CTA exits
+    if (lane == 0 && ew < 6) bulk_wait_all();   // every tensor store is complete before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -1281,13 +1284,25 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
   // the key pass's tensor-store views (its staged epilogue: no split
   // operands); a workspace laid out for the fused key-gradient kernel has no
   // key-pass intermediates and gets none
-  const bool kp_staged = !split && !w.keygrad;
+  const bool kp_staged = !w.keygrad;
   if (kp_staged) {
     const uint64_t ibs = (uint64_t)w.cmax * dh * 2;   // bytes per head of Gm' / Aq
-    if (D13 != nullptr)
-      TTT_TRY(make_tmap_bf16_3d_sw(&km.od13, D13, 2 * dh, w.cmax, BH, (uint64_t)dh * 4, 2 * ibs, 64, 128, 128));
-    TTT_TRY(make_tmap_bf16_3d_sw(&km.ogm, Gm, dh, w.cmax, BH, (uint64_t)dh * 2, ibs, 64, 128, 128));
-    TTT_TRY(make_tmap_bf16_3d_sw(&km.oaq, Aq, dh, w.cmax, BH, (uint64_t)dh * 2, ibs, 64, 128, 128));
+    if (!split) {
+      if (D13 != nullptr)
+        TTT_TRY(make_tmap_bf16_3d_sw(&km.od13, D13, 2 * dh, w.cmax, BH, (uint64_t)dh * 4, 2 * ibs, 64, 128, 128));
+      TTT_TRY(make_tmap_bf16_3d_sw(&km.ogm, Gm, dh, w.cmax, BH, (uint64_t)dh * 2, ibs, 64, 128, 128));
+      TTT_TRY(make_tmap_bf16_3d_sw(&km.oaq, Aq, dh, w.cmax, BH, (uint64_t)dh * 2, ibs, 64, 128, 128));
+    } else {
+      __nv_bfloat16* d13p[2] = {D13, D13lo};
+      __nv_bfloat16* gmp[2] = {Gm, Gmlo};
+      __nv_bfloat16* aqp[2] = {Aq, Aqlo};
+      for (int p = 0; p < 2; ++p) {
+        if (d13p[p] != nullptr)
+          TTT_TRY(make_tmap_bf16_3d_sw(&km.sd13[p], d13p[p], 2 * dh, w.cmax, BH, (uint64_t)dh * 4, 2 * ibs, 32, 128, 64));
+        TTT_TRY(make_tmap_bf16_3d_sw(&km.sgm[p], gmp[p], dh, w.cmax, BH, (uint64_t)dh * 2, ibs, 32, 128, 64));
+        TTT_TRY(make_tmap_bf16_3d_sw(&km.saq[p], aqp[p], dh, w.cmax, BH, (uint64_t)dh * 2, ibs, 32, 128, 64));
+      }
+    }
   }
   KeyPassMaps kmb[3] = {km, km, km};
   CUtensorMap mw2k[3], mw2klo[3];
@@ -1314,12 +1329,14 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     TTT_TRY(tok_map(&mv_mn, L.v, L.N_in, 64));
   }
 
-  static std::atomic<uint64_t> kp_attr{0};
-  if (allow_dynamic_smem(lact_keypass_kernel, (int)kp::SMEM, kp_attr)) return -1;
+  static std::atomic<uint64_t> kp_attr[2];
+  if (split ? allow_dynamic_smem(lact_keypass_kernel<true>, (int)kp::SMEM, kp_attr[1])
+            : allow_dynamic_smem(lact_keypass_kernel<false>, (int)kp::SMEM, kp_attr[0]))
+    return -1;
 
   auto key_pass_on = [&](int t0, int C, int nkt, int nqt, cudaStream_t kstream) -> int {
     // never launch on a token or store map this call did not encode
-    if ((nkt > 0 && !uses_kv) || (nqt > 0 && !uses_q) || (!split && !kp_staged)) return -1;
+    if ((nkt > 0 && !uses_kv) || (nqt > 0 && !uses_q) || !kp_staged) return -1;
     KeyPassArgs a{};
     a.C = C; a.t0 = t0; a.n_key_tiles = nkt; a.n_q_tiles = nqt; a.n_hb = dh / 64; a.BH = BH;
     a.d_steps = d / 64; a.dh = dh; a.lr_len = L.N_in; a.lr = L.lr;
@@ -1330,9 +1347,12 @@ int launch_lact(const LactLaunch& L, cudaStream_t stream) {
     const int tiles = (nkt + nqt) * a.n_hb * BH;
     if (tiles <= 0) return 0;
     prof_before(K_KEYPASS, kstream);
-    if (launch_pdl(lact_keypass_kernel, dim3(std::min(tiles, num_sms())), dim3(kp::THREADS),
-                   kp::SMEM, kstream, kmb[cur], a) != cudaSuccess)
-      return -1;
+    const cudaError_t e =
+        split ? launch_pdl(lact_keypass_kernel<true>, dim3(std::min(tiles, num_sms())), dim3(kp::THREADS),
+                           kp::SMEM, kstream, kmb[cur], a)
+              : launch_pdl(lact_keypass_kernel<false>, dim3(std::min(tiles, num_sms())), dim3(kp::THREADS),
+                           kp::SMEM, kstream, kmb[cur], a);
+    if (e != cudaSuccess) return -1;
     prof_after(K_KEYPASS, kstream);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   };
